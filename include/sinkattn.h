@@ -1,0 +1,238 @@
+/*
+ * libsinkattn -- gpt-oss-style sink-augmented grouped-query attention for
+ * NVIDIA B200 (sm_100a). Plain C ABI: pointers, sizes and status codes only.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - bf16 tensors are passed as void pointers to 16-bit bfloat16 storage.
+ * - "Device" pointers must be CUDA device memory of the current device;
+ *   "host" pointers are ordinary host memory.
+ * - Strides are in ELEMENTS. A q/k/v/out operand of logical shape
+ *   [B][T][H][d] is addressed as base + b*s[0] + t*s[1] + h*s[2] + c, i.e.
+ *   the last (head-width) dimension must be contiguous. This admits views
+ *   into a fused qkv tensor [B][T][d*(n_q+2*n_kv)] (GQA Attention study note,
+ *   "How it works": the fused qkv width 5120 split into Q, K, V).
+ *   Every base pointer and stride must keep 16-byte alignment of each row
+ *   (d*2 bytes rows, strides multiples of 8 elements).
+ * - All device work is enqueued asynchronously on the given stream (NULL =
+ *   the legacy default stream). Argument checks run on the host BEFORE any
+ *   launch: a call that returns an error other than SA_ERR_CUDA has enqueued
+ *   nothing and changed no state.
+ * - The library never allocates device memory. The caller owns every buffer,
+ *   including the KV cache and the decode workspace.
+ * - Kernels never trap and never wait without bound: a device-side wait that
+ *   exceeds its limit records SA_ERR_TIMEOUT in a device status word and the
+ *   kernel returns; read it with sa_get_device_status().
+ *
+ * Position / mask contract (MoE-Xtend README, "DESIGN CONTRACTS" and
+ * "ATTENTION STACK"): a call that starts at cache offset `off` handles query
+ * rows i = 0..T-1 at global positions p = off + i. RoPE uses p (never reset
+ * per window, no wrap). Row i may attend cache row j iff j <= p and, on
+ * windowed calls (window > 0), j > p - window (the band i-W<j<=i of the GQA
+ * Attention study note). The layer schedule (window on even layers, full on
+ * odd ones) is the caller's choice of `window`.
+ */
+#ifndef SINKATTN_H
+#define SINKATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sa_stream_t; /* == cudaStream_t */
+
+typedef enum sa_status {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,      /* null pointer, bad stride/alignment, T or B < 0 ... */
+  SA_ERR_SHAPE = 2,            /* n_q % n_kv != 0, d not in {64, 96, 128}, q_mult > 16 */
+  SA_ERR_CAPACITY = 3,         /* offset + T > cache capacity, or position >= max_pos */
+  SA_ERR_OFFSET_MISMATCH = 4,  /* the call's offset differs from cache->offset */
+  SA_ERR_STALE_SNAPSHOT = 5,   /* restore after rows below the snapshot were rewritten */
+  SA_ERR_CUDA = 6,             /* a CUDA runtime/driver call failed (launch, tensor map) */
+  SA_ERR_TIMEOUT = 7,          /* a bounded device wait ran out (read via sa_get_device_status) */
+  SA_ERR_WORKSPACE = 8         /* decode workspace missing or too small */
+} sa_status;
+
+/* Capacity of the cache's overwrite log (see sa_kv_restore). */
+#define SA_KV_LOG_CAP 32
+
+/*
+ * One layer's KV cache (MoE-Xtend README, "NOTATION": K,V [B, T_cache, H_kv, d];
+ * "KV CACHE": preallocated, Cache.extend writes rows [offset, offset+t) then
+ * advances offset; Cache.snapshot / Cache.restore).
+ *
+ * k, v : device, bf16, dense [B][cap][n_kv][d], caller-owned. K rows hold
+ *        ROTATED keys, V rows unrotated values (GPT-OSS-Lite visual guide,
+ *        "Overview": decode stores rotated K and unchanged V).
+ * offset: rows [0, offset) are valid. Host-authoritative: the library updates
+ *        it when an append is enqueued.
+ * The remaining fields are bookkeeping for snapshot/restore; initialise the
+ * whole struct with sa_kv_cache_init and do not edit them.
+ */
+typedef struct sa_kv_cache {
+  void* k;
+  void* v;
+  int32_t B, cap, n_kv, d;
+  int64_t offset;
+  int64_t seq;          /* +1 per append and per restore */
+  int64_t high_water;   /* largest offset ever reached */
+  int64_t log_seq[SA_KV_LOG_CAP];  /* appends that started below high_water */
+  int64_t log_row[SA_KV_LOG_CAP];
+  int32_t log_len;
+  int64_t log_floor_seq; /* summary of entries dropped from the full log: */
+  int64_t log_floor_row; /* latest dropped seq, lowest dropped row        */
+} sa_kv_cache;
+
+typedef struct sa_snapshot {
+  uint64_t cache_id;    /* identity of the cache (its K base address) */
+  int64_t offset;
+  int64_t seq;
+  int32_t cap;
+} sa_snapshot;
+
+/*
+ * Arguments of one attention call (prefill: T >= 0 rows; decode: T == 1).
+ *
+ * q      : device bf16 [B][T][n_q][d] via q_strides.
+ * k, v   : device bf16 [B][T][n_kv][d] via k_strides / v_strides: the call's
+ *          NEW rows, appended to the cache at rows [offset, offset+T).
+ * sinks  : device fp32 [n_q], one logit per query head (a raw logit compared
+ *          with sm_scale*<q,k>, not itself scaled), or NULL for no sink
+ *          (sink = -inf, plain softmax attention). Query head h = g*q_mult+m
+ *          uses KV head g = h / q_mult and sink sinks[h].
+ * offset : must equal cache->offset (the offset used for RoPE and masks).
+ * window : <= 0 full causal; > 0 band of `window` keys.
+ * sm_scale: score scale, e.g. 1/sqrt(d).
+ * rope_fused: 1 = q and k are UNrotated and the library rotates them with
+ *          cos/sin at p = offset + i; 0 = they are already rotated.
+ * cos, sin: device fp32 [max_pos][d/2] tables from sa_yarn_rope_tables
+ *          (concentration folded in); required when rope_fused = 1 (needs
+ *          offset + T <= max_pos), ignored otherwise.
+ * out    : device bf16 [B][T][n_q][d] via out_strides.
+ * lse    : device fp32 [B][n_q][T] or NULL: ln(sum_j e^{s_j} + e^{sink}).
+ */
+typedef struct sa_attn_args {
+  const void* q;   int64_t q_strides[3];
+  const void* k;   int64_t k_strides[3];
+  const void* v;   int64_t v_strides[3];
+  const float* sinks;
+  int32_t B, T, n_q;
+  int64_t offset;
+  int32_t window;
+  float sm_scale;
+  int32_t rope_fused;
+  const float* cos; const float* sin; int32_t max_pos;
+  void* out;       int64_t out_strides[3];
+  float* lse;
+} sa_attn_args;
+
+/* Human-readable name of a status code (static string). */
+const char* sa_status_string(sa_status s);
+
+/*
+ * YaRN / NTK-by-parts rotary tables (MoE-Xtend README, "ROPE + SCALING").
+ * For pair i < d/2 and position t < max_pos:
+ *   freq_i = theta^(i/(d/2)); extrap = 1/freq_i; interp = 1/(scaling*freq_i);
+ *   i_beta  = (d/2) ln(orig_ctx/(beta*2pi)) / ln(theta);
+ *   i_alpha = (d/2) ln(orig_ctx/(alpha*2pi)) / ln(theta);
+ *   mask = 1 - clamp((i - i_beta)/(i_alpha - i_beta), 0, 1);
+ *   inv_freq = interp*(1-mask) + extrap*mask;  conc = 0.1 ln(scaling) + 1;
+ *   cos[t][i] = conc*cos(t*inv_freq), sin[t][i] = conc*sin(t*inv_freq).
+ * Angles are formed in fp64 and the results rounded to fp32.
+ * cos_out, sin_out: device fp32 [max_pos][d/2], caller-owned.
+ * Errors: SA_ERR_INVALID_ARG (null, max_pos < 1, d odd or < 2, theta <= 1,
+ * scaling <= 0, orig_ctx < 1, alpha/beta <= 0, alpha >= beta).
+ */
+sa_status sa_yarn_rope_tables(float* cos_out, float* sin_out, int32_t max_pos, int32_t d,
+                              double theta, double scaling, int32_t orig_ctx,
+                              double alpha, double beta, sa_stream_t stream);
+
+/*
+ * In-place RoPE of Q and K (MoE-Xtend README, "DESIGN CONTRACTS": positions
+ * t = offset + local_t). Half-split pairs (x[c], x[c+d/2]):
+ *   x1' = x1*cos - x2*sin, x2' = x2*cos + x1*sin  (fp32, rounded to bf16).
+ * q: device bf16 [B][T][n_q][d] (q_strides), k: [B][T][n_kv][d] (k_strides);
+ * either may be NULL to skip it. Requires offset + T <= max_pos.
+ */
+sa_status sa_rope_apply_qk(void* q, const int64_t q_strides[3], void* k, const int64_t k_strides[3],
+                           int32_t B, int32_t T, int32_t n_q, int32_t n_kv, int32_t d, int64_t offset,
+                           const float* cos, const float* sin, int32_t max_pos, sa_stream_t stream);
+
+/* Initialise a cache descriptor over caller-owned K/V buffers (offset 0). */
+sa_status sa_kv_cache_init(sa_kv_cache* cache, void* k, void* v, int32_t B, int32_t cap,
+                           int32_t n_kv, int32_t d);
+
+/*
+ * Append T already-rotated K rows and V rows at [offset, offset+T), then
+ * offset += T (MoE-Xtend README, "KV CACHE": Cache.extend). k_rot/v: device
+ * bf16 [B][T][n_kv][d] via strides. Bit copy. SA_ERR_CAPACITY if
+ * offset + T > cap.
+ */
+sa_status sa_kv_append(sa_kv_cache* cache, const void* k_rot, const int64_t k_strides[3],
+                       const void* v, const int64_t v_strides[3], int32_t T, sa_stream_t stream);
+
+/* Capture the cache state (offset; rows below it are immutable under
+ * append-only use). Host only, no device work. */
+sa_status sa_kv_snapshot(const sa_kv_cache* cache, sa_snapshot* out);
+
+/*
+ * Reinstate a snapshot ("prefill once, decode many"): rolls the offset back
+ * to snap->offset. Host only. SA_ERR_STALE_SNAPSHOT when some row below
+ * snap->offset was rewritten after the snapshot (a restore to a lower
+ * offset followed by an append). The log keeps the last SA_KV_LOG_CAP such
+ * rewrites exactly and summarises older ones conservatively (a snapshot
+ * older than a dropped rewrite, with rows above that rewrite's first row, is
+ * reported stale). SA_ERR_INVALID_ARG for another cache's snapshot.
+ */
+sa_status sa_kv_restore(sa_kv_cache* cache, const sa_snapshot* snap);
+
+/*
+ * Prefill: rotate (if rope_fused) and append the call's K/V rows to the
+ * cache, then attend the T query rows to cache rows [0, offset+T) with the
+ * per-head sink column (MoE-Xtend README, "ATTENTION STACK": softmax over
+ * [QK + B, S], sink column dropped after normalisation; GQA Attention study
+ * note, "How it works"). cache->offset += T on success. T == 0 is a no-op.
+ * The attention runs on tcgen05 tensor cores with fp32 accumulation; the
+ * softmax weights enter the PV product as bf16.
+ */
+sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* args, sa_stream_t stream);
+
+/*
+ * Decode: one new row per sequence (args->T must be 1). Rotates q and k,
+ * appends the new K/V row at cache row `offset`, and attends to cache rows
+ * [max(0, offset+1-window), offset] (all rows when window <= 0), split
+ * across SMs. cache->offset += 1 on success (MoE-Xtend README, "DESIGN
+ * CONTRACTS": exactly one row per layer per step).
+ * workspace: device memory of at least sa_attn_decode_workspace_size()
+ *   bytes, caller-owned, ZERO-FILLED before its first use; the kernel leaves
+ *   it zeroed again on completion. Calls that share a workspace must not
+ *   overlap on the device (order them on one stream).
+ */
+sa_status sa_attn_decode(sa_kv_cache* cache, const sa_attn_args* args, void* workspace,
+                         size_t workspace_bytes, sa_stream_t stream);
+
+/* Workspace bytes sa_attn_decode needs for B sequences of n_q/n_kv heads of
+ * width d on any device with at most 256 SMs. */
+size_t sa_attn_decode_workspace_size(int32_t B, int32_t n_q, int32_t n_kv, int32_t d);
+
+/*
+ * Reads and clears the device status word of the current device (waits for
+ * the device to be idle). *code receives SA_OK or SA_ERR_TIMEOUT.
+ */
+sa_status sa_get_device_status(int32_t* code);
+
+/*
+ * Upper bound, in SM clock cycles, of every device-side wait of later
+ * launches on the current device (default about one second). For tests of
+ * the timeout path only.
+ */
+sa_status sa_set_wait_limit(int64_t cycles);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SINKATTN_H */

@@ -1,0 +1,475 @@
+// libsinkattn: C ABI, argument validation, cache bookkeeping, tensor-map
+// construction and kernel launches. Every declaration lives in
+// include/sinkattn.h; this file is the single translation unit of the
+// library, so the device status word in ptx.cuh exists once per device.
+
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/sinkattn.h"
+#include "decode.cuh"
+#include "prefill.cuh"
+#include "ptx.cuh"
+#include "rope.cuh"
+
+namespace {
+
+using sa::DecodeCfg;
+using sa::DecodeParams;
+using sa::PrefillCfg;
+using sa::PrefillParams;
+
+// ---------------------------------------------------------------------------
+// Small host helpers
+// ---------------------------------------------------------------------------
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool strides_ok(const int64_t s[3]) {
+  return s != nullptr && s[0] >= 0 && s[1] >= 0 && s[2] >= 0 && s[0] % 8 == 0 && s[1] % 8 == 0 &&
+         s[2] % 8 == 0;
+}
+
+bool head_dim_ok(int d) { return d == 64 || d == 96 || d == 128; }
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 256 ? 256 : (n < 1 ? 1 : n);
+}
+
+int grid_for(long long n) {
+  long long blocks = (n + 255) / 256;
+  const long long cap = (long long)num_sms() * 8;
+  if (blocks > cap) blocks = cap;
+  return blocks < 1 ? 1 : (int)blocks;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Tensor map over one cache buffer [B][cap][n_kv][d] bf16 that exposes only
+// rows [0, rows_valid) (later rows read back as zeros), box {CB, 1, box_rows, 1}.
+bool make_cache_map(CUtensorMap* map, void* base, int d, int n_kv, long long rows_valid, int cap,
+                    int B, int box_rows, int cb) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || rows_valid < 1) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)n_kv, (cuuint64_t)rows_valid, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)n_kv * d * 2,
+                                 (cuuint64_t)cap * n_kv * d * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)cb, 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         cb == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+sa_status last_launch_status() {
+  return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
+}
+
+// Cache bookkeeping after an append of T rows at `start`.
+void note_append(sa_kv_cache* c, int64_t start, int T) {
+  c->seq += 1;
+  if (start < c->high_water) {
+    if (c->log_len == SA_KV_LOG_CAP) {
+      if (c->log_seq[0] > c->log_floor_seq) c->log_floor_seq = c->log_seq[0];
+      if (c->log_row[0] < c->log_floor_row) c->log_floor_row = c->log_row[0];
+      memmove(c->log_seq, c->log_seq + 1, sizeof(int64_t) * (SA_KV_LOG_CAP - 1));
+      memmove(c->log_row, c->log_row + 1, sizeof(int64_t) * (SA_KV_LOG_CAP - 1));
+      c->log_len -= 1;
+    }
+    c->log_seq[c->log_len] = c->seq;
+    c->log_row[c->log_len] = start;
+    c->log_len += 1;
+  }
+  c->offset = start + T;
+  if (c->offset > c->high_water) c->high_water = c->offset;
+}
+
+sa_status check_cache(const sa_kv_cache* c) {
+  if (c == nullptr || c->k == nullptr || c->v == nullptr) return SA_ERR_INVALID_ARG;
+  if (c->B < 1 || c->cap < 1 || c->n_kv < 1) return SA_ERR_INVALID_ARG;
+  if (!head_dim_ok(c->d)) return SA_ERR_SHAPE;
+  if (!aligned16(c->k) || !aligned16(c->v)) return SA_ERR_INVALID_ARG;
+  if (c->offset < 0 || c->offset > c->cap) return SA_ERR_INVALID_ARG;
+  return SA_OK;
+}
+
+// Checks shared by prefill and decode.
+sa_status check_attn(const sa_kv_cache* c, const sa_attn_args* a) {
+  sa_status st = check_cache(c);
+  if (st != SA_OK) return st;
+  if (a == nullptr) return SA_ERR_INVALID_ARG;
+  if (a->B != c->B || a->T < 0 || a->n_q < 1) return SA_ERR_INVALID_ARG;
+  if (a->n_q % c->n_kv != 0) return SA_ERR_SHAPE;
+  if (a->offset != c->offset) return SA_ERR_OFFSET_MISMATCH;
+  if (a->T == 0) return SA_OK;
+  if (a->q == nullptr || a->k == nullptr || a->v == nullptr || a->out == nullptr)
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->out))
+    return SA_ERR_INVALID_ARG;
+  if (!strides_ok(a->q_strides) || !strides_ok(a->k_strides) || !strides_ok(a->v_strides) ||
+      !strides_ok(a->out_strides))
+    return SA_ERR_INVALID_ARG;
+  if (!(a->sm_scale > 0.f) || !isfinite(a->sm_scale)) return SA_ERR_INVALID_ARG;
+  if (a->offset + (int64_t)a->T > (int64_t)c->cap) return SA_ERR_CAPACITY;
+  if (a->rope_fused) {
+    if (a->cos == nullptr || a->sin == nullptr || !aligned16(a->cos) || !aligned16(a->sin))
+      return SA_ERR_INVALID_ARG;
+    if (a->offset + (int64_t)a->T > (int64_t)a->max_pos) return SA_ERR_CAPACITY;
+  }
+  return SA_OK;
+}
+
+template <typename K>
+void set_smem(K kernel, uint32_t bytes) {
+  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int D>
+sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream_t stream) {
+  using Cfg = PrefillCfg<D>;
+  CUtensorMap tmK, tmV;
+  const long long rows = a->offset + a->T;
+  if (!make_cache_map(&tmK, c->k, D, c->n_kv, rows, c->cap, c->B, 128, Cfg::CB) ||
+      !make_cache_map(&tmV, c->v, D, c->n_kv, rows, c->cap, c->B, 128, Cfg::CB))
+    return SA_ERR_CUDA;
+  PrefillParams p;
+  p.q = static_cast<const __nv_bfloat16*>(a->q);
+  p.qs0 = a->q_strides[0];
+  p.qs1 = a->q_strides[1];
+  p.qs2 = a->q_strides[2];
+  p.out = static_cast<__nv_bfloat16*>(a->out);
+  p.os0 = a->out_strides[0];
+  p.os1 = a->out_strides[1];
+  p.os2 = a->out_strides[2];
+  p.lse = a->lse;
+  p.sinks = a->sinks;
+  p.cos_t = a->cos;
+  p.sin_t = a->sin;
+  p.B = a->B;
+  p.T = a->T;
+  p.n_q = a->n_q;
+  p.n_kv = c->n_kv;
+  p.q_mult = a->n_q / c->n_kv;
+  p.off = a->offset;
+  p.window = a->window > 0 ? a->window : 0;
+  p.scale_log2 = a->sm_scale * 1.4426950408889634f;
+  p.rope = a->rope_fused ? 1 : 0;
+  p.n_pairs = (a->T + 255) / 256;
+  static bool configured = false;
+  if (!configured) {
+    set_smem(sa::prefill_kernel<D>, Cfg::SMEM_BYTES);
+    configured = true;
+  }
+  dim3 grid(p.n_pairs, a->n_q, a->B);
+  sa::prefill_kernel<D><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmK, tmV, p);
+  return last_launch_status();
+}
+
+struct DecodeSplit {
+  int S;
+  long long chunk;
+};
+
+DecodeSplit decode_split(int B, int n_kv, long long n_cache) {
+  DecodeSplit r{1, 64};
+  if (n_cache <= 0) return r;
+  const long long target = 2LL * num_sms();
+  long long S = (target + (long long)B * n_kv - 1) / ((long long)B * n_kv);
+  if (S < 1) S = 1;
+  long long chunk = (n_cache + S - 1) / S;
+  chunk = ((chunk + 63) / 64) * 64;
+  r.chunk = chunk;
+  r.S = (int)((n_cache + chunk - 1) / chunk);
+  return r;
+}
+
+// Workspace layout: counters [B*n_kv] int32 (256-byte padded), then
+// m [B*n_kv*S*q_mult], l [same], O [B*n_kv*S*q_mult*d] fp32.
+size_t decode_ws_bytes(int B, int n_kv, int q_mult, int d, int S) {
+  const size_t cnt = (((size_t)B * n_kv * 4) + 255) / 256 * 256;
+  const size_t rows = (size_t)B * n_kv * S * q_mult;
+  return cnt + rows * 4 * 2 + rows * d * 4;
+}
+
+template <int D>
+sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, size_t ws_bytes,
+                        cudaStream_t stream) {
+  using Cfg = DecodeCfg<D>;
+  const int q_mult = a->n_q / c->n_kv;
+  DecodeParams p;
+  p.off = a->offset;
+  p.lo = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
+  const long long n_cache = p.off - p.lo;
+  const DecodeSplit sp = decode_split(a->B, c->n_kv, n_cache);
+  p.S = sp.S;
+  p.chunk = sp.chunk;
+  if (p.S > 1) {
+    if (ws == nullptr || !aligned16(ws) || ws_bytes < decode_ws_bytes(a->B, c->n_kv, q_mult, D, p.S))
+      return SA_ERR_WORKSPACE;
+  }
+  CUtensorMap tmK, tmV;
+  memset(&tmK, 0, sizeof(tmK));
+  memset(&tmV, 0, sizeof(tmV));
+  if (n_cache > 0) {
+    if (!make_cache_map(&tmK, c->k, D, c->n_kv, p.off, c->cap, c->B, Cfg::R, Cfg::CB) ||
+        !make_cache_map(&tmV, c->v, D, c->n_kv, p.off, c->cap, c->B, Cfg::R, Cfg::CB))
+      return SA_ERR_CUDA;
+  }
+  p.q = static_cast<const __nv_bfloat16*>(a->q);
+  p.qs0 = a->q_strides[0];
+  p.qs2 = a->q_strides[2];
+  p.k = static_cast<const __nv_bfloat16*>(a->k);
+  p.ks0 = a->k_strides[0];
+  p.ks2 = a->k_strides[2];
+  p.v = static_cast<const __nv_bfloat16*>(a->v);
+  p.vs0 = a->v_strides[0];
+  p.vs2 = a->v_strides[2];
+  p.ck = static_cast<__nv_bfloat16*>(c->k);
+  p.cv = static_cast<__nv_bfloat16*>(c->v);
+  p.cap = c->cap;
+  p.out = static_cast<__nv_bfloat16*>(a->out);
+  p.os0 = a->out_strides[0];
+  p.os2 = a->out_strides[2];
+  p.lse = a->lse;
+  p.sinks = a->sinks;
+  p.cos_t = a->cos;
+  p.sin_t = a->sin;
+  p.B = a->B;
+  p.n_q = a->n_q;
+  p.n_kv = c->n_kv;
+  p.q_mult = q_mult;
+  p.scale_log2 = a->sm_scale * 1.4426950408889634f;
+  p.rope = a->rope_fused ? 1 : 0;
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  const size_t cnt = (((size_t)a->B * c->n_kv * 4) + 255) / 256 * 256;
+  const size_t rows = (size_t)a->B * c->n_kv * p.S * q_mult;
+  p.ws_cnt = reinterpret_cast<int*>(w);
+  p.ws_m = reinterpret_cast<float*>(w + cnt);
+  p.ws_l = reinterpret_cast<float*>(w + cnt + rows * 4);
+  p.ws_o = reinterpret_cast<float*>(w + cnt + rows * 8);
+  static bool configured = false;
+  if (!configured) {
+    set_smem(sa::decode_kernel<D>, Cfg::SMEM_BYTES);
+    configured = true;
+  }
+  dim3 grid(p.S, c->n_kv, a->B);
+  sa::decode_kernel<D><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmK, tmV, p);
+  return last_launch_status();
+}
+
+sa_status launch_append(sa_kv_cache* c, const void* k, const int64_t ks[3], const void* v,
+                        const int64_t vs[3], int T, int rope, const float* cos_t,
+                        const float* sin_t, cudaStream_t stream) {
+  const long long n = (long long)c->B * T * c->n_kv * (c->d / 16);
+  sa::kv_append_kernel<<<grid_for(n), 256, 0, stream>>>(
+      static_cast<__nv_bfloat16*>(c->k), static_cast<__nv_bfloat16*>(c->v), c->cap,
+      static_cast<const __nv_bfloat16*>(k), ks[0], ks[1], ks[2],
+      static_cast<const __nv_bfloat16*>(v), vs[0], vs[1], vs[2], c->B, T, c->n_kv, c->d, c->offset,
+      rope, cos_t, sin_t);
+  return last_launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sa_status_string(sa_status s) {
+  switch (s) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG";
+    case SA_ERR_SHAPE: return "SA_ERR_SHAPE";
+    case SA_ERR_CAPACITY: return "SA_ERR_CAPACITY";
+    case SA_ERR_OFFSET_MISMATCH: return "SA_ERR_OFFSET_MISMATCH";
+    case SA_ERR_STALE_SNAPSHOT: return "SA_ERR_STALE_SNAPSHOT";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA";
+    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT";
+    case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE";
+  }
+  return "SA_UNKNOWN";
+}
+
+sa_status sa_yarn_rope_tables(float* cos_out, float* sin_out, int32_t max_pos, int32_t d,
+                              double theta, double scaling, int32_t orig_ctx, double alpha,
+                              double beta, sa_stream_t stream) {
+  if (cos_out == nullptr || sin_out == nullptr || max_pos < 1 || d < 2 || d % 2 != 0)
+    return SA_ERR_INVALID_ARG;
+  if (!(theta > 1.0) || !(scaling > 0.0) || orig_ctx < 1 || !(alpha > 0.0) || !(beta > 0.0) ||
+      !(alpha < beta))
+    return SA_ERR_INVALID_ARG;
+  const int half = d / 2;
+  sa::yarn_tables_kernel<<<grid_for((long long)max_pos * half), 256, 0, (cudaStream_t)stream>>>(
+      cos_out, sin_out, max_pos, half, theta, scaling, (double)orig_ctx, alpha, beta);
+  return last_launch_status();
+}
+
+sa_status sa_rope_apply_qk(void* q, const int64_t q_strides[3], void* k, const int64_t k_strides[3],
+                           int32_t B, int32_t T, int32_t n_q, int32_t n_kv, int32_t d,
+                           int64_t offset, const float* cos, const float* sin, int32_t max_pos,
+                           sa_stream_t stream) {
+  if (B < 0 || T < 0 || n_q < 0 || n_kv < 0 || offset < 0) return SA_ERR_INVALID_ARG;
+  if (!head_dim_ok(d)) return SA_ERR_SHAPE;
+  if (cos == nullptr || sin == nullptr || !aligned16(cos) || !aligned16(sin)) return SA_ERR_INVALID_ARG;
+  if (q != nullptr && (!aligned16(q) || !strides_ok(q_strides))) return SA_ERR_INVALID_ARG;
+  if (k != nullptr && (!aligned16(k) || !strides_ok(k_strides))) return SA_ERR_INVALID_ARG;
+  if (offset + (int64_t)T > (int64_t)max_pos) return SA_ERR_CAPACITY;
+  if (B == 0 || T == 0) return SA_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (q != nullptr && n_q > 0) {
+    const long long n = (long long)B * T * n_q * (d / 16);
+    sa::rope_inplace_kernel<<<grid_for(n), 256, 0, s>>>(static_cast<__nv_bfloat16*>(q), q_strides[0],
+                                                        q_strides[1], q_strides[2], B, T, n_q, d,
+                                                        offset, cos, sin);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  }
+  if (k != nullptr && n_kv > 0) {
+    const long long n = (long long)B * T * n_kv * (d / 16);
+    sa::rope_inplace_kernel<<<grid_for(n), 256, 0, s>>>(static_cast<__nv_bfloat16*>(k), k_strides[0],
+                                                        k_strides[1], k_strides[2], B, T, n_kv, d,
+                                                        offset, cos, sin);
+    if (cudaGetLastError() != cudaSuccess) return SA_ERR_CUDA;
+  }
+  return SA_OK;
+}
+
+sa_status sa_kv_cache_init(sa_kv_cache* cache, void* k, void* v, int32_t B, int32_t cap,
+                           int32_t n_kv, int32_t d) {
+  if (cache == nullptr) return SA_ERR_INVALID_ARG;
+  memset(cache, 0, sizeof(*cache));
+  cache->k = k;
+  cache->v = v;
+  cache->B = B;
+  cache->cap = cap;
+  cache->n_kv = n_kv;
+  cache->d = d;
+  cache->log_floor_seq = -1;
+  cache->log_floor_row = INT64_MAX;
+  return check_cache(cache);
+}
+
+sa_status sa_kv_append(sa_kv_cache* cache, const void* k_rot, const int64_t k_strides[3],
+                       const void* v, const int64_t v_strides[3], int32_t T, sa_stream_t stream) {
+  sa_status st = check_cache(cache);
+  if (st != SA_OK) return st;
+  if (T < 0) return SA_ERR_INVALID_ARG;
+  if (T == 0) return SA_OK;
+  if (k_rot == nullptr || v == nullptr || !aligned16(k_rot) || !aligned16(v) ||
+      !strides_ok(k_strides) || !strides_ok(v_strides))
+    return SA_ERR_INVALID_ARG;
+  if (cache->offset + (int64_t)T > (int64_t)cache->cap) return SA_ERR_CAPACITY;
+  st = launch_append(cache, k_rot, k_strides, v, v_strides, T, 0, nullptr, nullptr,
+                     (cudaStream_t)stream);
+  if (st != SA_OK) return st;
+  note_append(cache, cache->offset, T);
+  return SA_OK;
+}
+
+sa_status sa_kv_snapshot(const sa_kv_cache* cache, sa_snapshot* out) {
+  sa_status st = check_cache(cache);
+  if (st != SA_OK) return st;
+  if (out == nullptr) return SA_ERR_INVALID_ARG;
+  out->cache_id = (uint64_t)reinterpret_cast<uintptr_t>(cache->k);
+  out->offset = cache->offset;
+  out->seq = cache->seq;
+  out->cap = cache->cap;
+  return SA_OK;
+}
+
+sa_status sa_kv_restore(sa_kv_cache* cache, const sa_snapshot* snap) {
+  sa_status st = check_cache(cache);
+  if (st != SA_OK) return st;
+  if (snap == nullptr) return SA_ERR_INVALID_ARG;
+  if (snap->cache_id != (uint64_t)reinterpret_cast<uintptr_t>(cache->k) || snap->cap != cache->cap ||
+      snap->offset < 0 || snap->offset > cache->high_water || snap->seq > cache->seq)
+    return SA_ERR_INVALID_ARG;
+  if (snap->seq < cache->log_floor_seq && cache->log_floor_row < snap->offset) return SA_ERR_STALE_SNAPSHOT;
+  for (int i = 0; i < cache->log_len; ++i)
+    if (cache->log_seq[i] > snap->seq && cache->log_row[i] < snap->offset) return SA_ERR_STALE_SNAPSHOT;
+  cache->offset = snap->offset;
+  cache->seq += 1;
+  return SA_OK;
+}
+
+sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* a, sa_stream_t stream) {
+  sa_status st = check_attn(cache, a);
+  if (st != SA_OK) return st;
+  if (a->T == 0) return SA_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  st = launch_append(cache, a->k, a->k_strides, a->v, a->v_strides, a->T, a->rope_fused ? 1 : 0,
+                     a->cos, a->sin, s);
+  if (st != SA_OK) return st;
+  switch (cache->d) {
+    case 64: st = launch_prefill<64>(cache, a, s); break;
+    case 96: st = launch_prefill<96>(cache, a, s); break;
+    case 128: st = launch_prefill<128>(cache, a, s); break;
+    default: return SA_ERR_SHAPE;
+  }
+  // The append is enqueued either way; the offset follows it.
+  note_append(cache, cache->offset, a->T);
+  return st;
+}
+
+sa_status sa_attn_decode(sa_kv_cache* cache, const sa_attn_args* a, void* workspace,
+                         size_t workspace_bytes, sa_stream_t stream) {
+  sa_status st = check_attn(cache, a);
+  if (st != SA_OK) return st;
+  if (a->T != 1) return SA_ERR_INVALID_ARG;
+  if (a->n_q / cache->n_kv > 8) return SA_ERR_SHAPE;
+  cudaStream_t s = (cudaStream_t)stream;
+  switch (cache->d) {
+    case 64: st = launch_decode<64>(cache, a, workspace, workspace_bytes, s); break;
+    case 96: st = launch_decode<96>(cache, a, workspace, workspace_bytes, s); break;
+    case 128: st = launch_decode<128>(cache, a, workspace, workspace_bytes, s); break;
+    default: return SA_ERR_SHAPE;
+  }
+  if (st == SA_OK) note_append(cache, cache->offset, 1);
+  return st;
+}
+
+size_t sa_attn_decode_workspace_size(int32_t B, int32_t n_q, int32_t n_kv, int32_t d) {
+  if (B < 1 || n_kv < 1 || n_q < n_kv || d < 1) return 0;
+  const int q_mult = n_q / n_kv;
+  // B*n_kv*S <= 2*256 + B*n_kv for any device of at most 256 SMs.
+  const long long units = 512 + (long long)B * n_kv;
+  const size_t cnt = (((size_t)B * n_kv * 4) + 255) / 256 * 256;
+  return cnt + (size_t)units * q_mult * (2 + d) * 4;
+}
+
+sa_status sa_get_device_status(int32_t* code) {
+  if (code == nullptr) return SA_ERR_INVALID_ARG;
+  int v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, sa::g_status, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(sa::g_status, &zero, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
+  *code = (v & sa::STATUS_TIMEOUT) ? SA_ERR_TIMEOUT : SA_OK;
+  return SA_OK;
+}
+
+sa_status sa_set_wait_limit(int64_t cycles) {
+  if (cycles < 0) return SA_ERR_INVALID_ARG;
+  long long v = cycles;
+  if (cudaMemcpyToSymbol(sa::g_wait_limit, &v, sizeof(v)) != cudaSuccess) return SA_ERR_CUDA;
+  return SA_OK;
+}
+
+}  // extern "C"

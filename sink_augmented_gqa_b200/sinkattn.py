@@ -1,0 +1,279 @@
+"""Thin Python binding of libsinkattn (ctypes).
+
+Argument marshalling only: every computation runs in the CUDA library
+(``libsinkattn.so``, built in-tree by ``sink_augmented_gqa_b200.build``).
+PyTorch supplies device memory and the current stream. There is no CPU or
+PyTorch fallback: if the library is missing, every call raises.
+
+Names mirror the C ABI in ``include/sinkattn.h`` without the ``sa_`` prefix:
+``yarn_rope_tables``, ``rope_apply_qk``, ``KVCache`` (``kv_append``,
+``kv_snapshot``, ``kv_restore``), ``attn_prefill``, ``attn_decode``.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsinkattn.so")
+KV_LOG_CAP = 32
+
+STATUS = {
+    0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_SHAPE", 3: "SA_ERR_CAPACITY",
+    4: "SA_ERR_OFFSET_MISMATCH", 5: "SA_ERR_STALE_SNAPSHOT", 6: "SA_ERR_CUDA",
+    7: "SA_ERR_TIMEOUT", 8: "SA_ERR_WORKSPACE",
+}
+
+
+class SinkAttnError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        self.name = STATUS.get(code, f"status {code}")
+        super().__init__(f"{where}: {self.name}")
+
+
+class _KVCache(ctypes.Structure):
+    _fields_ = [
+        ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("B", ctypes.c_int32), ("cap", ctypes.c_int32), ("n_kv", ctypes.c_int32), ("d", ctypes.c_int32),
+        ("offset", ctypes.c_int64), ("seq", ctypes.c_int64), ("high_water", ctypes.c_int64),
+        ("log_seq", ctypes.c_int64 * KV_LOG_CAP), ("log_row", ctypes.c_int64 * KV_LOG_CAP),
+        ("log_len", ctypes.c_int32), ("log_floor_seq", ctypes.c_int64), ("log_floor_row", ctypes.c_int64),
+    ]
+
+
+class _Snapshot(ctypes.Structure):
+    _fields_ = [("cache_id", ctypes.c_uint64), ("offset", ctypes.c_int64),
+                ("seq", ctypes.c_int64), ("cap", ctypes.c_int32)]
+
+
+_I64x3 = ctypes.c_int64 * 3
+
+
+class _AttnArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("q_strides", _I64x3),
+        ("k", ctypes.c_void_p), ("k_strides", _I64x3),
+        ("v", ctypes.c_void_p), ("v_strides", _I64x3),
+        ("sinks", ctypes.c_void_p),
+        ("B", ctypes.c_int32), ("T", ctypes.c_int32), ("n_q", ctypes.c_int32),
+        ("offset", ctypes.c_int64), ("window", ctypes.c_int32), ("sm_scale", ctypes.c_float),
+        ("rope_fused", ctypes.c_int32),
+        ("cos", ctypes.c_void_p), ("sin", ctypes.c_void_p), ("max_pos", ctypes.c_int32),
+        ("out", ctypes.c_void_p), ("out_strides", _I64x3),
+        ("lse", ctypes.c_void_p),
+    ]
+
+
+# Every symbol include/sinkattn.h declares.
+EXPORTS = (
+    "sa_status_string", "sa_yarn_rope_tables", "sa_rope_apply_qk", "sa_kv_cache_init",
+    "sa_kv_append", "sa_kv_snapshot", "sa_kv_restore", "sa_attn_prefill", "sa_attn_decode",
+    "sa_attn_decode_workspace_size", "sa_get_device_status", "sa_set_wait_limit",
+)
+
+_lib = None
+
+
+def lib():
+    """The loaded library (loads it on first use; raises if it is not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libsinkattn.so not found at {LIB_PATH}; build it with "
+                "`python -m sink_augmented_gqa_b200.build` (there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, f64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+        P = ctypes.POINTER
+        L.sa_status_string.restype = ctypes.c_char_p
+        L.sa_status_string.argtypes = [ctypes.c_int]
+        L.sa_yarn_rope_tables.argtypes = [vp, vp, i32, i32, f64, f64, i32, f64, f64, vp]
+        L.sa_rope_apply_qk.argtypes = [vp, P(i64), vp, P(i64), i32, i32, i32, i32, i32, i64, vp, vp, i32, vp]
+        L.sa_kv_cache_init.argtypes = [P(_KVCache), vp, vp, i32, i32, i32, i32]
+        L.sa_kv_append.argtypes = [P(_KVCache), vp, P(i64), vp, P(i64), i32, vp]
+        L.sa_kv_snapshot.argtypes = [P(_KVCache), P(_Snapshot)]
+        L.sa_kv_restore.argtypes = [P(_KVCache), P(_Snapshot)]
+        L.sa_attn_prefill.argtypes = [P(_KVCache), P(_AttnArgs), vp]
+        L.sa_attn_decode.argtypes = [P(_KVCache), P(_AttnArgs), vp, ctypes.c_size_t, vp]
+        L.sa_attn_decode_workspace_size.restype = ctypes.c_size_t
+        L.sa_attn_decode_workspace_size.argtypes = [i32, i32, i32, i32]
+        L.sa_get_device_status.argtypes = [P(i32)]
+        L.sa_set_wait_limit.argtypes = [i64]
+        for name in EXPORTS:
+            if name not in ("sa_status_string", "sa_attn_decode_workspace_size"):
+                getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(code, where):
+    if code != 0:
+        raise SinkAttnError(code, where)
+
+
+def _stream(t=None):
+    dev = t.device if t is not None else torch.device("cuda")
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _strides(t):
+    """Element strides [batch, token, head] of a [B, T, H, d] view (d contiguous)."""
+    if t.dim() != 4 or t.stride(3) != 1:
+        raise ValueError("expected a [B, T, H, d] tensor with a contiguous last dimension")
+    return _I64x3(t.stride(0), t.stride(1), t.stride(2))
+
+
+def _require_bf16_cuda(name, t):
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA bf16 tensor")
+
+
+# ---------------------------------------------------------------------------
+# Public API
+# ---------------------------------------------------------------------------
+
+def yarn_rope_tables(max_pos, d, theta=150000.0, scaling=32.0, orig_ctx=4096, alpha=1.0, beta=32.0,
+                     device="cuda"):
+    """fp32 cos/sin tables [max_pos, d/2] (concentration folded in)."""
+    cos = torch.empty((max_pos, d // 2), dtype=torch.float32, device=device)
+    sin = torch.empty_like(cos)
+    _check(lib().sa_yarn_rope_tables(_ptr(cos), _ptr(sin), max_pos, d, float(theta), float(scaling),
+                                     int(orig_ctx), float(alpha), float(beta), _stream(cos)),
+           "sa_yarn_rope_tables")
+    return cos, sin
+
+
+def rope_apply_qk(q, k, offset, cos, sin):
+    """Rotate q [B,T,n_q,d] and k [B,T,n_kv,d] in place at positions offset + t."""
+    ref = q if q is not None else k
+    B, T, _, d = ref.shape
+    n_q = q.shape[2] if q is not None else 0
+    n_kv = k.shape[2] if k is not None else 0
+    qs = _strides(q) if q is not None else _I64x3(0, 0, 0)
+    ks = _strides(k) if k is not None else _I64x3(0, 0, 0)
+    _check(lib().sa_rope_apply_qk(_ptr(q), qs, _ptr(k), ks, B, T, n_q, n_kv, d, int(offset),
+                                  _ptr(cos), _ptr(sin), cos.shape[0], _stream(ref)),
+           "sa_rope_apply_qk")
+
+
+class Snapshot:
+    def __init__(self, raw):
+        self.raw = raw
+
+    @property
+    def offset(self):
+        return self.raw.offset
+
+
+class KVCache:
+    """One layer's bf16 KV cache [B, cap, n_kv, d] (torch-owned device memory)."""
+
+    def __init__(self, B, cap, n_kv, d, device="cuda", k=None, v=None):
+        shape = (B, cap, n_kv, d)
+        self.k = k if k is not None else torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        self.v = v if v is not None else torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        assert tuple(self.k.shape) == shape and self.k.is_contiguous() and self.v.is_contiguous()
+        self.raw = _KVCache()
+        _check(lib().sa_kv_cache_init(ctypes.byref(self.raw), _ptr(self.k), _ptr(self.v), B, cap, n_kv, d),
+               "sa_kv_cache_init")
+
+    @property
+    def offset(self):
+        return self.raw.offset
+
+    @property
+    def B(self):
+        return self.raw.B
+
+    def append(self, k_rot, v):
+        """kv_append: copy already-rotated k and v rows at [offset, offset + T)."""
+        _check(lib().sa_kv_append(ctypes.byref(self.raw), _ptr(k_rot), _strides(k_rot), _ptr(v),
+                                  _strides(v), k_rot.shape[1], _stream(self.k)), "sa_kv_append")
+
+    def snapshot(self):
+        s = _Snapshot()
+        _check(lib().sa_kv_snapshot(ctypes.byref(self.raw), ctypes.byref(s)), "sa_kv_snapshot")
+        return Snapshot(s)
+
+    def restore(self, snap):
+        _check(lib().sa_kv_restore(ctypes.byref(self.raw), ctypes.byref(snap.raw)), "sa_kv_restore")
+
+
+def _args(cache, q, k, v, sinks, window, sm_scale, cos, sin, rope_fused, out, lse):
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        _require_bf16_cuda(n, t)
+    if sinks is not None and (sinks.dtype != torch.float32 or not sinks.is_contiguous()):
+        raise TypeError("sinks must be a contiguous fp32 CUDA tensor")
+    a = _AttnArgs()
+    a.q, a.q_strides = q.data_ptr(), _strides(q)
+    a.k, a.k_strides = k.data_ptr(), _strides(k)
+    a.v, a.v_strides = v.data_ptr(), _strides(v)
+    a.sinks = 0 if sinks is None else sinks.data_ptr()
+    a.B, a.T, a.n_q = q.shape[0], q.shape[1], q.shape[2]
+    a.offset = cache.offset
+    a.window = int(window)
+    a.sm_scale = float(sm_scale)
+    a.rope_fused = 1 if rope_fused else 0
+    a.cos = 0 if cos is None else cos.data_ptr()
+    a.sin = 0 if sin is None else sin.data_ptr()
+    a.max_pos = 0 if cos is None else cos.shape[0]
+    a.out, a.out_strides = out.data_ptr(), _strides(out)
+    a.lse = 0 if lse is None else lse.data_ptr()
+    return a
+
+
+def attn_prefill(cache, q, k, v, sinks, window, sm_scale, cos=None, sin=None, rope_fused=True,
+                 out=None, return_lse=False, lse=None):
+    """Prefill T rows: append (rotated) k/v to the cache, attend q to rows
+    [0, offset + T). Returns out [B,T,n_q,d] bf16 (and lse [B,n_q,T] fp32)."""
+    B, T, n_q, d = q.shape
+    if out is None:
+        out = torch.empty((B, T, n_q, d), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, n_q, T), dtype=torch.float32, device=q.device)
+    a = _args(cache, q, k, v, sinks, window, sm_scale, cos, sin, rope_fused, out, lse)
+    _check(lib().sa_attn_prefill(ctypes.byref(cache.raw), ctypes.byref(a), _stream(q)), "sa_attn_prefill")
+    return (out, lse) if return_lse else out
+
+
+def decode_workspace_bytes(B, n_q, n_kv, d):
+    return int(lib().sa_attn_decode_workspace_size(B, n_q, n_kv, d))
+
+
+def decode_workspace(B, n_q, n_kv, d, device="cuda"):
+    """A zero-filled workspace for attn_decode (reusable across calls)."""
+    return torch.zeros(decode_workspace_bytes(B, n_q, n_kv, d), dtype=torch.uint8, device=device)
+
+
+def attn_decode(cache, q, k, v, sinks, window, sm_scale, cos=None, sin=None, rope_fused=True,
+                workspace=None, out=None, return_lse=False, lse=None):
+    """One decode step (T == 1): append the new row, attend to the cache."""
+    B, T, n_q, d = q.shape
+    if workspace is None:
+        workspace = decode_workspace(B, n_q, cache.raw.n_kv, d, q.device)
+    if out is None:
+        out = torch.empty((B, T, n_q, d), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, n_q, T), dtype=torch.float32, device=q.device)
+    a = _args(cache, q, k, v, sinks, window, sm_scale, cos, sin, rope_fused, out, lse)
+    _check(lib().sa_attn_decode(ctypes.byref(cache.raw), ctypes.byref(a), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(q)),
+           "sa_attn_decode")
+    return (out, lse) if return_lse else out
+
+
+def device_status():
+    """Reads and clears the device status word: 'SA_OK' or 'SA_ERR_TIMEOUT'."""
+    code = ctypes.c_int32(0)
+    _check(lib().sa_get_device_status(ctypes.byref(code)), "sa_get_device_status")
+    return STATUS.get(code.value, str(code.value))
+
+
+def set_wait_limit(cycles):
+    _check(lib().sa_set_wait_limit(int(cycles)), "sa_set_wait_limit")

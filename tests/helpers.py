@@ -1,0 +1,100 @@
+"""Shared test helpers: tolerance checks and oracle runs on seeded inputs.
+
+Tolerance (the stated bar for bf16 outputs with fp32 accumulation): compared
+with the oracle's exact output rounded to bf16 (the stored precision), every
+element is within max-abs 1e-2 -- or exactly one bf16 step away, which is a
+rounding-boundary flip that max-abs cannot exclude once |out| >= 2, where one
+bf16 step is already 0.0156 -- and the mean absolute error is <= 1e-3.
+"""
+
+import numpy as np
+import torch
+
+from oracle import attention as oatt
+from oracle import bf16 as obf16
+from oracle import kvcache as okv
+from oracle import rope as orope
+from oracle import yarn as oyarn
+
+MAX_ABS = 1e-2
+MEAN_ABS = 1e-3
+
+
+def to64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def check_bf16_output(gpu, ref, what=""):
+    """gpu: torch bf16 tensor; ref: fp64 numpy array of the same shape."""
+    g = to64(gpu)
+    r = obf16.round_bf16(ref)
+    assert g.shape == r.shape, (g.shape, r.shape)
+    assert np.all(np.isfinite(g)), f"{what}: non-finite output"
+    err = np.abs(g - r)
+    ok = (err <= MAX_ABS) | (err <= obf16.bf16_ulp(r) * 1.0000001)
+    bad = np.argwhere(~ok)
+    assert bad.size == 0, (f"{what}: {len(bad)} elements beyond tolerance; first {bad[:5].tolist()} "
+                           f"gpu={g[tuple(bad[0])]} ref={r[tuple(bad[0])]}")
+    mean = float(err.mean()) if err.size else 0.0
+    assert mean <= MEAN_ABS, f"{what}: mean abs err {mean}"
+    return float(err.max()) if err.size else 0.0, mean
+
+
+LSE_LOG = []
+
+
+def check_lse(gpu, ref, what="", rtol=2e-5, atol=2e-4):
+    """lse in fp32 (log-sum-exp of fp32 scores of bf16 operands, with the sink)."""
+    g = to64(gpu)
+    err = float(np.abs(g - ref).max()) if np.size(g) else 0.0
+    LSE_LOG.append((what, err))
+    assert np.allclose(g, ref, rtol=rtol, atol=atol), f"{what}: lse max err {err}"
+
+
+def yarn_cfg(cfg):
+    y = cfg.yarn
+    return dict(theta=y["theta"], s=y["scaling"], orig_ctx=y["orig_ctx"], alpha=y["alpha"], beta=y["beta"])
+
+
+def oracle_tables(cfg, max_pos):
+    y = yarn_cfg(cfg)
+    return oyarn.stored_tables(max_pos, cfg.d, y["theta"], y["s"], y["orig_ctx"], y["alpha"], y["beta"])
+
+
+def oracle_cache(B, cap, n_kv, d, k_prefix=None, v_prefix=None):
+    c = okv.KVCache(B, cap, n_kv, d)
+    if k_prefix is not None:
+        c.append(to64(k_prefix), to64(v_prefix))
+    return c
+
+
+def oracle_step(cache, q, k, v, sinks, window, sm_scale, cos, sin, rope_fused=True):
+    """fp64 oracle of one prefill/decode call on torch inputs."""
+    return oatt.attend_step(cache, to64(q), to64(k), to64(v),
+                            None if sinks is None else to64(sinks), window, sm_scale, cos, sin,
+                            rope_fused=rope_fused)
+
+
+def oracle_rows(q_raw, k_prefix_rot, k_new_raw, v_prefix, v_new, sinks, off, rows, heads, b,
+                window, sm_scale, cos, sin, q_mult):
+    """Oracle output of selected query rows i (positions off+i) and heads h of
+    sequence b, computed one row at a time from raw inputs.
+
+    k_prefix_rot/v_prefix: [rows_before, n_kv, d] cache rows before the call
+    (already rotated), k_new_raw/v_new: [T, n_kv, d] the call's new rows.
+    Returns {(i, h): (out [d], lse)}.
+    """
+    res = {}
+    n_new = k_new_raw.shape[0]
+    k_new_rot = orope.rotate_bsh(k_new_raw[None], off, cos, sin)[0]
+    K = np.concatenate([k_prefix_rot, k_new_rot], axis=0) if k_prefix_rot is not None else k_new_rot
+    V = np.concatenate([v_prefix, v_new], axis=0) if v_prefix is not None else v_new
+    assert K.shape[0] == off + n_new
+    for i in rows:
+        for h in heads:
+            g = h // q_mult
+            qr = orope.rotate_bsh(q_raw[None, i:i + 1, h:h + 1], off + i, cos, sin)
+            out, lse = oatt.sink_attention(qr, K[None, :off + i + 1, g:g + 1], V[None, :off + i + 1, g:g + 1],
+                                           None if sinks is None else sinks[h:h + 1], off + i, window, sm_scale)
+            res[(i, h)] = (out[0, 0, 0], lse[0, 0, 0])
+    return res

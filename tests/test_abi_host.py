@@ -1,0 +1,131 @@
+"""CPU-only checks of the C ABI: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any launch."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from sink_augmented_gqa_b200 import build as sbuild
+from sink_augmented_gqa_b200 import sinkattn as S
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "sinkattn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    sbuild.build()
+    return S.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(S.EXPORTS) == names
+
+
+def test_status_strings(L):
+    for code, name in S.STATUS.items():
+        assert L.sa_status_string(code).decode() == name
+
+
+def _fake_cache(B=1, cap=100, n_kv=2, d=64):
+    c = S._KVCache()
+    # Host-only bookkeeping never dereferences these (16-byte aligned) addresses.
+    st = L_.sa_kv_cache_init(ctypes.byref(c), ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000), B, cap, n_kv, d)
+    return c, st
+
+
+L_ = None
+
+
+@pytest.fixture(autouse=True)
+def _bind(L):
+    global L_
+    L_ = L
+
+
+def test_cache_init_validation(L):
+    c, st = _fake_cache()
+    assert st == 0 and c.offset == 0 and c.cap == 100
+    c2 = S._KVCache()
+    assert L.sa_kv_cache_init(ctypes.byref(c2), ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000), 1, 10, 2, 80) == 2
+    assert L.sa_kv_cache_init(ctypes.byref(c2), None, ctypes.c_void_p(0x20000), 1, 10, 2, 64) == 1
+    assert L.sa_kv_cache_init(ctypes.byref(c2), ctypes.c_void_p(0x10008), ctypes.c_void_p(0x20000), 1, 10, 2, 64) == 1
+
+
+def test_snapshot_restore_host_logic(L):
+    c, _ = _fake_cache()
+    # Simulate the bookkeeping the library does after appends: appends are
+    # device work, so drive the fields the way an append would (offset moves,
+    # high-water mark, overwrite log) via restore/snapshot only.
+    c.offset, c.high_water, c.seq = 40, 40, 1
+    s40 = S._Snapshot()
+    assert L.sa_kv_snapshot(ctypes.byref(c), ctypes.byref(s40)) == 0
+    assert (s40.offset, s40.seq, s40.cap) == (40, 1, 100)
+    c.offset, c.high_water, c.seq = 60, 60, 2
+    s60 = S._Snapshot()
+    L.sa_kv_snapshot(ctypes.byref(c), ctypes.byref(s60))
+    assert L.sa_kv_restore(ctypes.byref(c), ctypes.byref(s40)) == 0 and c.offset == 40 and c.seq == 3
+    assert L.sa_kv_restore(ctypes.byref(c), ctypes.byref(s60)) == 0 and c.offset == 60   # nothing rewritten
+    # record an overwrite at row 45 after s60 (what an append from offset 45 logs)
+    c.seq = 5
+    c.log_seq[0], c.log_row[0], c.log_len = 5, 45, 1
+    assert L.sa_kv_restore(ctypes.byref(c), ctypes.byref(s60)) == 5      # stale
+    assert L.sa_kv_restore(ctypes.byref(c), ctypes.byref(s40)) == 0      # rows < 40 untouched
+    other = S._Snapshot()
+    other.cache_id, other.offset, other.seq, other.cap = 0x999, 10, 1, 100
+    assert L.sa_kv_restore(ctypes.byref(c), ctypes.byref(other)) == 1
+
+
+def _args(offset=0, T=4, n_q=4, B=1, window=0):
+    a = S._AttnArgs()
+    for f in ("q", "k", "v", "out"):
+        setattr(a, f, 0x30000)
+    for f in ("q_strides", "k_strides", "v_strides", "out_strides"):
+        setattr(a, f, S._I64x3(4096, 256, 64))
+    a.B, a.T, a.n_q, a.offset, a.window, a.sm_scale = B, T, n_q, offset, window, 0.125
+    a.rope_fused = 0
+    return a
+
+
+def test_attention_argument_errors_return_before_launch(L):
+    c, _ = _fake_cache(cap=100)
+    stream = ctypes.c_void_p(0)
+    assert L.sa_attn_prefill(ctypes.byref(c), ctypes.byref(_args(offset=3)), stream) == 4     # offset mismatch
+    assert L.sa_attn_prefill(ctypes.byref(c), ctypes.byref(_args(T=101)), stream) == 3        # capacity
+    assert L.sa_attn_prefill(ctypes.byref(c), ctypes.byref(_args(n_q=5)), stream) == 2        # n_q % n_kv
+    assert L.sa_attn_prefill(ctypes.byref(c), ctypes.byref(_args(B=2)), stream) == 1          # batch mismatch
+    a = _args()
+    a.q_strides = S._I64x3(4096, 256, 60)                                                       # misaligned head stride
+    assert L.sa_attn_prefill(ctypes.byref(c), ctypes.byref(a), stream) == 1
+    a = _args()
+    a.rope_fused = 1                                                                            # no tables
+    assert L.sa_attn_prefill(ctypes.byref(c), ctypes.byref(a), stream) == 1
+    assert L.sa_attn_prefill(ctypes.byref(c), ctypes.byref(_args(T=0)), stream) == 0          # empty: no-op
+    assert c.offset == 0
+    assert L.sa_attn_decode(ctypes.byref(c), ctypes.byref(_args(T=2)), None, 0, stream) == 1  # decode is T == 1
+    assert L.sa_attn_decode(ctypes.byref(c), ctypes.byref(_args(n_q=20, T=1)), None, 0, stream) == 2  # q_mult > 8
+    assert c.offset == 0
+
+
+def test_workspace_size_bound(L):
+    n = L.sa_attn_decode_workspace_size(1, 64, 8, 64)
+    assert n >= (512 + 8) * 8 * 66 * 4
+    assert L.sa_attn_decode_workspace_size(0, 64, 8, 64) == 0
+
+
+def test_table_argument_errors(L):
+    p = ctypes.c_void_p(0x40000)
+    assert L.sa_yarn_rope_tables(p, p, 0, 64, 150000.0, 32.0, 4096, 1.0, 32.0, None) == 1
+    assert L.sa_yarn_rope_tables(p, p, 10, 63, 150000.0, 32.0, 4096, 1.0, 32.0, None) == 1
+    assert L.sa_yarn_rope_tables(p, p, 10, 64, 150000.0, 32.0, 4096, 32.0, 1.0, None) == 1   # alpha >= beta
