@@ -2,7 +2,7 @@
 //
 // The work is reading the KV cache once: for each (sequence b, KV head g)
 // the rows [lo, off) are cut into S contiguous splits, one CTA each
-// (grid S x n_kv x B). Inside a CTA one producer warp streams 64-row K and V
+// (grid n_kv x S x B). Inside a CTA one producer warp streams 64-row K and V
 // tiles of head g from the cache with TMA (128-byte swizzled smem, rows past
 // `off` read as zeros) through a deep ring, and four consumer warps each take
 // 16 rows of every tile. A consumer computes S^T = K Q^T for the q_mult <= 8
@@ -148,8 +148,8 @@ __global__ void __launch_bounds__(160)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int split = blockIdx.x;
-  const int g = blockIdx.y;
+  const int g = blockIdx.x;      // KV heads of one split run side by side (same cache rows)
+  const int split = blockIdx.y;
   const int b = blockIdx.z;
   const int QM = p.q_mult;
   constexpr int HALF = D / 2;
@@ -363,23 +363,63 @@ __global__ void __launch_bounds__(160)
   if (!flag[1]) return;
   __threadfence();
 
+  // Merge the S partials of (b, g). The K/V ring is idle now; reuse it for
+  // the per-split weights so every global load below is independent.
   const long long slot0 = ((long long)b * p.n_kv + g) * p.S;
+  float* wsm = reinterpret_cast<float*>(smem);                 // [S][QM] e^{m_s - M}
+  float* Msm = wsm + (size_t)p.S * QM;                          // [QM] M (log2 units)
+  float* Lsm = Msm + 8;                                         // [QM] total l
+  for (int idx = tid; idx < p.S * QM; idx += 128) wsm[idx] = __ldcg(p.ws_m + slot0 * QM + idx);
+  named_bar_sync(1, 128);
+  if (tid < 32 * ((QM + 3) / 4)) {
+    // one warp per group of heads: lanes stride over the splits
+    const int w = tid >> 5;
+    for (int n = w; n < QM; n += (QM + 3) / 4) {
+      const int h = g * QM + n;
+      const float sink2 = p.sinks ? p.sinks[h] * LOG2E : -INFINITY;
+      float M = sink2;
+      for (int s = lane; s < p.S; s += 32) M = fmaxf(M, wsm[s * QM + n]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+      float L = 0.f;
+      for (int s = lane; s < p.S; s += 32) {
+        const float ms = wsm[s * QM + n];
+        const float f = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+        L += __ldcg(p.ws_l + (slot0 + s) * QM + n) * f;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+      __syncwarp();
+      for (int s = lane; s < p.S; s += 32) {
+        const float ms = wsm[s * QM + n];
+        wsm[s * QM + n] = (ms == -INFINITY) ? 0.f : ex2(ms - M);
+      }
+      if (lane == 0) {
+        L += ex2(sink2 - M);
+        Msm[n] = M;
+        Lsm[n] = L;
+      }
+    }
+  }
+  named_bar_sync(1, 128);
   for (int idx = tid; idx < QM * D; idx += 128) {
     const int n = idx / D, d = idx % D;
-    const int h = g * QM + n;
-    const float sink2 = p.sinks ? p.sinks[h] * LOG2E : -INFINITY;
-    float M = sink2;
-    for (int s = 0; s < p.S; ++s) M = fmaxf(M, __ldcg(p.ws_m + (slot0 + s) * QM + n));
-    float L = ex2(sink2 - M), O = 0.f;
-    for (int s = 0; s < p.S; ++s) {
-      const float ms = __ldcg(p.ws_m + (slot0 + s) * QM + n);
-      if (ms == -INFINITY) continue;
-      const float f = ex2(ms - M);
-      L += __ldcg(p.ws_l + (slot0 + s) * QM + n) * f;
-      O += __ldcg(p.ws_o + ((slot0 + s) * QM + n) * D + d) * f;
+    const float* src = p.ws_o + (slot0 * QM + n) * D + d;
+    float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
+    int s = 0;
+    for (; s + 4 <= p.S; s += 4) {
+      const float v0 = __ldcg(src + (size_t)(s + 0) * QM * D), v1 = __ldcg(src + (size_t)(s + 1) * QM * D);
+      const float v2 = __ldcg(src + (size_t)(s + 2) * QM * D), v3 = __ldcg(src + (size_t)(s + 3) * QM * D);
+      O0 = fmaf(v0, wsm[(s + 0) * QM + n], O0);
+      O1 = fmaf(v1, wsm[(s + 1) * QM + n], O1);
+      O2 = fmaf(v2, wsm[(s + 2) * QM + n], O2);
+      O3 = fmaf(v3, wsm[(s + 3) * QM + n], O3);
     }
-    p.out[b * p.os0 + (long long)h * p.os2 + d] = __float2bfloat16_rn(O / L);
-    if (d == 0 && p.lse) p.lse[(long long)b * p.n_q + h] = (M + __log2f(L)) * LN2;
+    for (; s < p.S; ++s) O0 = fmaf(__ldcg(src + (size_t)s * QM * D), wsm[s * QM + n], O0);
+    const int h = g * QM + n;
+    const float L = Lsm[n];
+    p.out[b * p.os0 + (long long)h * p.os2 + d] = __float2bfloat16_rn(((O0 + O1) + (O2 + O3)) / L);
+    if (d == 0 && p.lse) p.lse[(long long)b * p.n_q + h] = (Msm[n] + __log2f(L)) * LN2;
   }
   if (tid == 0) p.ws_cnt[b * p.n_kv + g] = 0;
 }

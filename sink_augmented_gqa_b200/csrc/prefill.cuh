@@ -9,7 +9,7 @@
 //   warp 1      allocates TMEM and issues every tcgen05.mma from one thread:
 //               S_X = Q_X K^T (smem x smem, fp32 in TMEM), then O_X += P_X V
 //               with P_X read from TMEM (bf16, aliased over S_X).
-//   warps 2-5   softmax for tile A, warps 6-9 for tile B, one query row per
+//   warps 4-7   softmax for tile A, warps 8-11 for tile B, one query row per
 //               thread (TMEM lane = row): load + RoPE the Q row into swizzled
 //               smem, then per key tile: mask, running max in log2 units,
 //               exp2, P -> TMEM, and at the end O / l -> bf16 out.
@@ -65,7 +65,7 @@ struct PrefillCfg {
   static constexpr int TMEM_COLS = 512;
   static constexpr int S_COL0 = 0, S_COL1 = 128;       // S_A, S_B (P aliased in cols [0,64))
   static constexpr int O_COL0 = 256, O_COL1 = 256 + D;
-  static constexpr int NUM_THREADS = 320;
+  static constexpr int NUM_THREADS = 384;
   // smem: Q[2] | K[NS] | V[NS] | barriers
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_K = 2 * TILE_BYTES;
@@ -136,8 +136,32 @@ __device__ __forceinline__ TileGeom make_geom(const PrefillParams& p, int pair) 
   return g;
 }
 
+// MMA issue helpers (one thread). S_X = Q_X K_t^T over d/16 K-steps.
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t qbase, uint32_t kbase) {
+  using C = PrefillCfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t coff = (kk * 16 / C::CB) * C::BLOCK_BYTES + (kk * 16 % C::CB) * 2;
+    const uint64_t adesc = smem_desc(qbase + coff, 16, C::SBO, C::LAYOUT);
+    const uint64_t bdesc = smem_desc(kbase + coff, 16, C::SBO, C::LAYOUT);
+    mma_ss(s_tmem, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
+  }
+}
+// O_X (+)= P_X V_t over 128/16 K-steps; P_X is bf16 in TMEM (cols [0,64) of S_X).
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t vbase,
+                                         bool accumulate) {
+  using C = PrefillCfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < 128 / 16; ++kk) {
+    const uint64_t bdesc = smem_desc(vbase + kk * 16 * C::SWZ, C::BLOCK_BYTES, C::SBO, C::LAYOUT);
+    mma_ts(o_tmem, p_tmem + kk * 8, bdesc, C::IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const PrefillParams p) {
   using C = PrefillCfg<D>;
@@ -189,9 +213,13 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp < 4) {
+    // Warpgroup 0: producer (warp 0) and MMA issuer (warp 1); warps 2-3 idle.
+    // It gives registers to the two softmax warpgroups: 128*56 + 256*224 =
+    // 384*168, the launch allocation.
+    regs_dec<56>();
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------ producer
       int issued = 0;
       for (int t = 0; t < geo.ntiles && !*abort_flag; ++t) {
         const int s = t % C::NS;
@@ -203,7 +231,8 @@ __global__ void __launch_bounds__(320, 1)
         for (int cb = 0; cb < C::NCB; ++cb)
           tma_load_4d(sbase + C::OFF_K + s * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmK,
                       bar(BAR_KFULL + s), cb * C::CB, g, krow, b);
-        if (!mbar_wait(bar(BAR_VEMPTY + s), ph ^ 1)) { *abort_flag = 1; issued = t * 2 + 1; break; }
+        issued = t * 2 + 1;
+        if (!mbar_wait(bar(BAR_VEMPTY + s), ph ^ 1)) { *abort_flag = 1; break; }
         mbar_arrive_expect_tx(bar(BAR_VFULL + s), C::TILE_BYTES);
 #pragma unroll
         for (int cb = 0; cb < C::NCB; ++cb)
@@ -219,62 +248,52 @@ __global__ void __launch_bounds__(320, 1)
         for (int t = (nv > C::NS ? nv - C::NS : 0); t < nv; ++t)
           mbar_wait(bar(BAR_VFULL + t % C::NS), (uint32_t)((t / C::NS) & 1));
       }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    } else if (warp == 1 && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
       bool ok = true;
-      for (int X = 0; X < 2; ++X)
-        if (geo.valid(X) && !mbar_wait(bar(BAR_QREADY + X), 0)) ok = false;
+      if (geo.valid(0) && !mbar_wait(bar(BAR_QREADY + 0), 0)) ok = false;
+      if (ok && geo.valid(1) && !mbar_wait(bar(BAR_QREADY + 1), 0)) ok = false;
       tc_fence_after();
-      int nS[2] = {0, 0};   // S tiles issued per query tile
-      int nPV[2] = {0, 0};  // PV products issued per query tile
-      const uint32_t s_col[2] = {(uint32_t)C::S_COL0, (uint32_t)C::S_COL1};
-      const uint32_t o_col[2] = {(uint32_t)C::O_COL0, (uint32_t)C::O_COL1};
-
-      auto issue_pv = [&](int X, int t) -> bool {
-        if (!mbar_wait(bar(BAR_PFULL + X), (uint32_t)((nS[X] - 1) & 1))) return false;
-        tc_fence_after();
-        const uint32_t vbase = sbase + C::OFF_V + (t % C::NS) * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk) {
-          const uint64_t bdesc = smem_desc(vbase + kk * 16 * C::SWZ, C::BLOCK_BYTES, C::SBO, C::LAYOUT);
-          mma_ts(tmem + o_col[X], tmem + s_col[X] + kk * 8, bdesc, C::IDESC_PV,
-                 (nPV[X] > 0 || kk > 0) ? 1u : 0u);
-        }
-        ++nPV[X];
-        return true;
-      };
-      auto issue_qk = [&](int X, int t) {
-        const uint32_t qbase = sbase + C::OFF_Q + X * C::TILE_BYTES;
-        const uint32_t kbase = sbase + C::OFF_K + (t % C::NS) * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t coff = (kk * 16 / C::CB) * C::BLOCK_BYTES + (kk * 16 % C::CB) * 2;
-          const uint64_t adesc = smem_desc(qbase + coff, 16, C::SBO, C::LAYOUT);
-          const uint64_t bdesc = smem_desc(kbase + coff, 16, C::SBO, C::LAYOUT);
-          mma_ss(tmem + s_col[X], adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar(BAR_SFULL + X));
-        ++nS[X];
-      };
-
+      const uint32_t qA = sbase + C::OFF_Q, qB = sbase + C::OFF_Q + C::TILE_BYTES;
+      const uint32_t sA = tmem + C::S_COL0, sB = tmem + C::S_COL1;
+      const uint32_t oA = tmem + C::O_COL0, oB = tmem + C::O_COL1;
+      int nA = 0, nB = 0;  // S tiles issued for A / B (P barrier phases)
       for (int t = 0; t <= geo.ntiles && ok; ++t) {
+        const int ks = t % C::NS, vs = (t + C::NS - 1) % C::NS;
         if (t < geo.ntiles) {
-          if (!mbar_wait(bar(BAR_KFULL + t % C::NS), (uint32_t)((t / C::NS) & 1))) { ok = false; break; }
+          if (!mbar_wait(bar(BAR_KFULL + ks), (uint32_t)((t / C::NS) & 1))) { ok = false; break; }
           tc_fence_after();
         }
         if (t > 0) {
-          if (!mbar_wait(bar(BAR_VFULL + (t - 1) % C::NS), (uint32_t)(((t - 1) / C::NS) & 1))) { ok = false; break; }
+          if (!mbar_wait(bar(BAR_VFULL + vs), (uint32_t)(((t - 1) / C::NS) & 1))) { ok = false; break; }
           tc_fence_after();
         }
-        for (int X = 0; X < 2 && ok; ++X) {
-          if (geo.active(X, t - 1) && !issue_pv(X, t - 1)) { ok = false; break; }
-          if (t < geo.ntiles && geo.active(X, t)) issue_qk(X, t);
+        const uint32_t kb = sbase + C::OFF_K + ks * C::TILE_BYTES;
+        const uint32_t vb = sbase + C::OFF_V + vs * C::TILE_BYTES;
+        // tile A: O_A += P_A(t-1) V(t-1), then S_A = Q_A K(t)^T
+        if (geo.active(0, t - 1)) {
+          if (!mbar_wait(bar(BAR_PFULL + 0), (uint32_t)((nA - 1) & 1))) { ok = false; break; }
+          tc_fence_after();
+          issue_pv<D>(oA, sA, vb, nA > 1);
         }
-        if (!ok) break;
-        if (t < geo.ntiles) mma_commit(bar(BAR_KEMPTY + t % C::NS));
-        if (t > 0) mma_commit(bar(BAR_VEMPTY + (t - 1) % C::NS));
+        if (t < geo.ntiles && geo.active(0, t)) {
+          issue_qk<D>(sA, qA, kb);
+          mma_commit(bar(BAR_SFULL + 0));
+          ++nA;
+        }
+        // tile B
+        if (geo.active(1, t - 1)) {
+          if (!mbar_wait(bar(BAR_PFULL + 1), (uint32_t)((nB - 1) & 1))) { ok = false; break; }
+          tc_fence_after();
+          issue_pv<D>(oB, sB, vb, nB > 1);
+        }
+        if (t < geo.ntiles && geo.active(1, t)) {
+          issue_qk<D>(sB, qB, kb);
+          mma_commit(bar(BAR_SFULL + 1));
+          ++nB;
+        }
+        if (t < geo.ntiles) mma_commit(bar(BAR_KEMPTY + ks));
+        if (t > 0) mma_commit(bar(BAR_VEMPTY + vs));
         if (*abort_flag) { ok = false; break; }
       }
       if (ok) {
@@ -289,7 +308,8 @@ __global__ void __launch_bounds__(320, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int X = (warp - 2) >> 2;
+    regs_inc<224>();
+    const int X = (warp - 4) >> 2;
     const int quarter = warp & 3;               // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;          // row within the query tile
     const int i = geo.i0 + 128 * X + r;         // query row within the call
@@ -310,13 +330,14 @@ __global__ void __launch_bounds__(320, 1)
           uint4 a = *reinterpret_cast<const uint4*>(qrow + ch * 8);
           uint4 c = *reinterpret_cast<const uint4*>(qrow + HALF + ch * 8);
           if (p.rope) {
-            const float* cs = p.cos_t + pos * HALF + ch * 8;
-            const float* sn = p.sin_t + pos * HALF + ch * 8;
-            uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
-            uint32_t* pc = reinterpret_cast<uint32_t*>(&c);
-#pragma unroll
-            for (int w = 0; w < 4; ++w)
-              rope_pair2(pa[w], pc[w], cs[2 * w], cs[2 * w + 1], sn[2 * w], sn[2 * w + 1]);
+            const float4 c0 = *reinterpret_cast<const float4*>(p.cos_t + pos * HALF + ch * 8);
+            const float4 c1 = *reinterpret_cast<const float4*>(p.cos_t + pos * HALF + ch * 8 + 4);
+            const float4 s0 = *reinterpret_cast<const float4*>(p.sin_t + pos * HALF + ch * 8);
+            const float4 s1 = *reinterpret_cast<const float4*>(p.sin_t + pos * HALF + ch * 8 + 4);
+            rope_pair2(a.x, c.x, c0.x, c0.y, s0.x, s0.y);
+            rope_pair2(a.y, c.y, c0.z, c0.w, s0.z, s0.w);
+            rope_pair2(a.z, c.z, c1.x, c1.y, s1.x, s1.y);
+            rope_pair2(a.w, c.w, c1.z, c1.w, s1.z, s1.w);
           }
           *reinterpret_cast<uint4*>(qtile + swz_off<C::CB>(r, ch * 8, C::BLOCK_BYTES)) = a;
           *reinterpret_cast<uint4*>(qtile + swz_off<C::CB>(r, HALF + ch * 8, C::BLOCK_BYTES)) = c;
@@ -331,6 +352,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(bar(BAR_QREADY + X));
 
       const float LOG2E = 1.4426950408889634f;
+      const float scale = p.scale_log2;
       const float sink2 = p.sinks ? p.sinks[h] * LOG2E : -INFINITY;
       float m = sink2;                              // running max (log2 units)
       float l = (sink2 == -INFINITY) ? 0.f : 1.f;   // running sum, sink included
@@ -340,40 +362,52 @@ __global__ void __launch_bounds__(320, 1)
         if (!geo.active(X, t)) continue;
         if (!mbar_wait(bar(BAR_SFULL + X), (uint32_t)(n & 1))) { ok = false; *abort_flag = 1; break; }
         tc_fence_after();
-        float s[128];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t rr[32];
-          tmem_ld32(s_tm + q4 * 32, rr);
-          tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) s[q4 * 32 + c] = __uint_as_float(rr[c]) * p.scale_log2;
-        }
+        uint32_t sr[128];
+        tmem_ld32(s_tm + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+        tmem_ld32(s_tm + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+        tmem_ld32(s_tm + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
+        tmem_ld32(s_tm + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        tmem_wait_ld();
         if (!geo.full(X, t)) {
+          // admitted columns c (key klo + c): c >= cmin and c <= cmax
           const long long klo = geo.base + 128LL * t;
-          // admitted columns: c >= c_min and c <= c_max (relative to klo)
-          long long cmin = -klo;
-          if (p.window > 0 && pos - p.window + 1 - klo > cmin) cmin = pos - p.window + 1 - klo;
-          const long long cmax = pos - klo;
+          long long lo_k = 0;
+          if (p.window > 0 && pos - p.window + 1 > lo_k) lo_k = pos - p.window + 1;
+          long long cmin = lo_k - klo, cmax = pos - klo;
+          const int cmin_i = (int)(cmin < -1 ? -1 : (cmin > 128 ? 128 : cmin));
+          const int cmax_i = (int)(cmax < -1 ? -1 : (cmax > 128 ? 128 : cmax));
 #pragma unroll
           for (int c = 0; c < 128; ++c)
-            if (c < cmin || c > cmax) s[c] = -INFINITY;
+            if (c < cmin_i || c > cmax_i) sr[c] = __float_as_uint(-INFINITY);
         }
-        float mx = s[0];
+        // raw row max (scale > 0, so max(s * scale) = scale * max(s))
+        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < 128; c += 8) {
+          m0 = max3f(m0, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
+          m1 = max3f(m1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+          m2 = max3f(m2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+          m3 = max3f(m3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+        }
+        const float mx = fmaxf(max3f(m0, m1, m2), m3) * scale;
         const float m_new = fmaxf(m, mx);
         const bool need = m_new > m + 8.0f;
         if (__any_sync(0xffffffffu, need)) {
           const float f = need ? ex2(m - m_new) : 1.0f;
           if (n > 0) {
+            // O rows stay in TMEM; S_X(t) complete implies PV_X(t-1) complete.
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
               uint32_t rr[32];
               tmem_ld32(o_tm + c0, rr);
               tmem_wait_ld();
 #pragma unroll
-              for (int c = 0; c < 32; ++c) rr[c] = __float_as_uint(__uint_as_float(rr[c]) * f);
+              for (int c = 0; c < 32; c += 2) {
+                float a0 = __uint_as_float(rr[c]), a1 = __uint_as_float(rr[c + 1]);
+                mul2(a0, a1, f, f);
+                rr[c] = __float_as_uint(a0);
+                rr[c + 1] = __float_as_uint(a1);
+              }
               tmem_st32(o_tm + c0, rr);
             }
             tmem_wait_st();
@@ -383,19 +417,26 @@ __global__ void __launch_bounds__(320, 1)
             m = m_new;
           }
         }
-        const float m_use = (m == -INFINITY) ? 0.f : m;
+        const float neg = (m == -INFINITY) ? 0.f : -m;
+        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
 #pragma unroll
         for (int q2 = 0; q2 < 2; ++q2) {
           uint32_t pk[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float p0 = ex2(s[q2 * 64 + 2 * c] - m_use);
-            const float p1 = ex2(s[q2 * 64 + 2 * c + 1] - m_use);
-            l += p0 + p1;
+          for (int c = 0; c < 32; c += 2) {
+            const int j = q2 * 64 + 2 * c;
+            float x0, x1, x2, x3;
+            fma2(x0, x1, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]), scale, scale, neg, neg);
+            fma2(x2, x3, __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]), scale, scale, neg, neg);
+            const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+            add2(l0, l1, p0, p1);
+            add2(l2, l3, p2, p3);
             pk[c] = pack_bf16(p0, p1);
+            pk[c + 1] = pack_bf16(p2, p3);
           }
           tmem_st32(s_tm + q2 * 32, pk);
         }
+        l += (l0 + l1) + (l2 + l3);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(BAR_PFULL + X));

@@ -272,7 +272,7 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
     set_smem(sa::decode_kernel<D>, Cfg::SMEM_BYTES);
     configured = true;
   }
-  dim3 grid(p.S, c->n_kv, a->B);
+  dim3 grid(c->n_kv, p.S, a->B);
   sa::decode_kernel<D><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmK, tmV, p);
   return last_launch_status();
 }
