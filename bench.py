@@ -271,7 +271,7 @@ def long_decode(dev, peaks, steps=8, layers=24):
         c.v.normal_(generator=g)
         # rows [0, off) stand for an already-filled, rotated prefix: append them
         # in place (a self-copy) so the cache's offset and bookkeeping follow.
-        c.append(c.k[:, :off], c.v[:, :off])
+        c.append(c.k_rows(0, off), c.v_rows(0, off))
         caches.append(c)
         ins.append(dict(window=cfg.layer_window(layer), sinks=wl.sinks(cfg, layer, device=dev),
                         ws=sa.decode_workspace(cfg.B, cfg.n_q, cfg.n_kv, cfg.d, device=dev),
@@ -322,7 +322,8 @@ def long_decode(dev, peaks, steps=8, layers=24):
             "KV_GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm"], 4),
             "full_layer_kernel": {"ms": round(ms_full, 4), "KV_GB/s": round(gbs_full, 1),
                                   "frac_of_hbm": round(gbs_full / peaks["hbm"], 4)},
-            "kv_cache_GiB": round(layers * 2 * cfg.B * cap * cfg.n_kv * cfg.d * 2 / 2 ** 30, 3)}
+            "kv_cache_GiB": round(layers * 2 * cfg.B * cap * cfg.n_kv * cfg.d * 2 / 2 ** 30, 3),
+            "cache_layout": "head-major [B][n_kv][cap][d]"}
 
 
 def e2e_lite(step, steps, warmup):
@@ -453,7 +454,7 @@ def profile_case(name, dev, steps, warmup):
         g.manual_seed(cfg.seed * 1000 + 50_001)
         cache.k.normal_(generator=g)
         cache.v.normal_(generator=g)
-        cache.append(cache.k[:, :off], cache.v[:, :off])
+        cache.append(cache.k_rows(0, off), cache.v_rows(0, off))
         snap = cache.snapshot()
         q, k, v = wl.qkv(cfg, 1, device=dev)
         sinks = wl.sinks(cfg, 1, device=dev)

@@ -64,9 +64,13 @@ typedef enum sa_status {
  * "KV CACHE": preallocated, Cache.extend writes rows [offset, offset+t) then
  * advances offset; Cache.snapshot / Cache.restore).
  *
- * k, v : device, bf16, dense [B][cap][n_kv][d], caller-owned. K rows hold
- *        ROTATED keys, V rows unrotated values (GPT-OSS-Lite visual guide,
- *        "Overview": decode stores rotated K and unchanged V).
+ * k, v : device, bf16, dense [B][n_kv][cap][d] (head-major), caller-owned.
+ *        Row j of KV head g of sequence b is k + ((b*n_kv + g)*cap + j)*d.
+ *        The pages write the cache as [B, T_cache, H_kv, d]; this library
+ *        keeps each (sequence, KV head) as one contiguous run of rows so that
+ *        decode streams it at full HBM bandwidth. K rows hold ROTATED keys,
+ *        V rows unrotated values (GPT-OSS-Lite visual guide, "Overview":
+ *        decode stores rotated K and unchanged V).
  * offset: rows [0, offset) are valid. Host-authoritative: the library updates
  *        it when an append is enqueued.
  * The remaining fields are bookkeeping for snapshot/restore; initialise the

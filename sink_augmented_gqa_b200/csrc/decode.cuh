@@ -49,7 +49,7 @@ struct DecodeParams {
   int S;
   float scale_log2;
   int rope;
-  float* ws_o;  // [B][n_kv][S][q_mult][D]
+  float* ws_o;  // [B][n_kv][S][q_mult][D] (16-byte aligned rows)
   float* ws_m;  // [B][n_kv][S][q_mult]
   float* ws_l;  // [B][n_kv][S][q_mult]
   int* ws_cnt;  // [B][n_kv]
@@ -185,9 +185,9 @@ __global__ void __launch_bounds__(160)
 #pragma unroll
         for (int cb = 0; cb < C::NCB; ++cb) {
           tma_load_4d(sbase + C::OFF_K + s * C::STAGE_BYTES + cb * C::BLOCK_BYTES, &tmK, full_bar(s),
-                      cb * C::CB, g, row, b);
+                      cb * C::CB, row, g, b);
           tma_load_4d(sbase + C::OFF_V + s * C::STAGE_BYTES + cb * C::BLOCK_BYTES, &tmV, full_bar(s),
-                      cb * C::CB, g, row, b);
+                      cb * C::CB, row, g, b);
         }
         issued = it + 1;
         if (flag[0]) break;
@@ -244,8 +244,8 @@ __global__ void __launch_bounds__(160)
     uint8_t* xv = smem + C::OFF_XV;
     const __nv_bfloat16* krow = p.k + b * p.ks0 + (long long)g * p.ks2;
     const __nv_bfloat16* vrow = p.v + b * p.vs0 + (long long)g * p.vs2;
-    __nv_bfloat16* ckrow = p.ck + (((long long)b * p.cap + p.off) * p.n_kv + g) * D;
-    __nv_bfloat16* cvrow = p.cv + (((long long)b * p.cap + p.off) * p.n_kv + g) * D;
+    __nv_bfloat16* ckrow = p.ck + (((long long)b * p.n_kv + g) * p.cap + p.off) * D;
+    __nv_bfloat16* cvrow = p.cv + (((long long)b * p.n_kv + g) * p.cap + p.off) * D;
     // zero rows 1..15 (and row 0, overwritten below)
     for (int idx = lane; idx < (int)(C::XTILE / 16); idx += 32) {
       reinterpret_cast<uint4*>(xk)[idx] = make_uint4(0, 0, 0, 0);
@@ -364,36 +364,58 @@ __global__ void __launch_bounds__(160)
   __threadfence();
 
   // Merge the S partials of (b, g). The K/V ring is idle now; reuse it for
-  // the per-split weights so every global load below is independent.
+  // the per-split weights. Every global read below is batched (independent
+  // loads in flight) because this tail runs on one CTA per (b, g) while the
+  // rest of the GPU has finished.
   const long long slot0 = ((long long)b * p.n_kv + g) * p.S;
-  float* wsm = reinterpret_cast<float*>(smem);                 // [S][QM] e^{m_s - M}
-  float* Msm = wsm + (size_t)p.S * QM;                          // [QM] M (log2 units)
+  const int S = p.S;
+  float* wsm = reinterpret_cast<float*>(smem);                 // [S][QM] m_s, then e^{m_s - M}
+  float* lsm = wsm + (size_t)S * QM;                            // [S][QM] l_s
+  float* Msm = lsm + (size_t)S * QM;                            // [QM] M (log2 units)
   float* Lsm = Msm + 8;                                         // [QM] total l
-  for (int idx = tid; idx < p.S * QM; idx += 128) wsm[idx] = __ldcg(p.ws_m + slot0 * QM + idx);
+  {
+    const float* gm = p.ws_m + slot0 * QM;
+    const float* gl = p.ws_l + slot0 * QM;
+    const int nml = S * QM;
+    int idx = tid;
+    for (; idx + 3 * 128 < nml; idx += 4 * 128) {
+      float a[4], c[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        a[j] = __ldcg(gm + idx + j * 128);
+        c[j] = __ldcg(gl + idx + j * 128);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        wsm[idx + j * 128] = a[j];
+        lsm[idx + j * 128] = c[j];
+      }
+    }
+    for (; idx < nml; idx += 128) {
+      wsm[idx] = __ldcg(gm + idx);
+      lsm[idx] = __ldcg(gl + idx);
+    }
+  }
   named_bar_sync(1, 128);
-  if (tid < 32 * ((QM + 3) / 4)) {
-    // one warp per group of heads: lanes stride over the splits
+  {
+    // warp w reduces heads n = w, w + 4, ...: lanes stride over the splits
     const int w = tid >> 5;
-    for (int n = w; n < QM; n += (QM + 3) / 4) {
+    for (int n = w; n < QM; n += 4) {
       const int h = g * QM + n;
       const float sink2 = p.sinks ? p.sinks[h] * LOG2E : -INFINITY;
       float M = sink2;
-      for (int s = lane; s < p.S; s += 32) M = fmaxf(M, wsm[s * QM + n]);
+      for (int s2 = lane; s2 < S; s2 += 32) M = fmaxf(M, wsm[s2 * QM + n]);
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
       float L = 0.f;
-      for (int s = lane; s < p.S; s += 32) {
-        const float ms = wsm[s * QM + n];
+      for (int s2 = lane; s2 < S; s2 += 32) {
+        const float ms = wsm[s2 * QM + n];
         const float f = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-        L += __ldcg(p.ws_l + (slot0 + s) * QM + n) * f;
+        wsm[s2 * QM + n] = f;
+        L += lsm[s2 * QM + n] * f;
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-      __syncwarp();
-      for (int s = lane; s < p.S; s += 32) {
-        const float ms = wsm[s * QM + n];
-        wsm[s * QM + n] = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-      }
       if (lane == 0) {
         L += ex2(sink2 - M);
         Msm[n] = M;
@@ -402,24 +424,44 @@ __global__ void __launch_bounds__(160)
     }
   }
   named_bar_sync(1, 128);
-  for (int idx = tid; idx < QM * D; idx += 128) {
-    const int n = idx / D, d = idx % D;
-    const float* src = p.ws_o + (slot0 * QM + n) * D + d;
-    float O0 = 0.f, O1 = 0.f, O2 = 0.f, O3 = 0.f;
-    int s = 0;
-    for (; s + 4 <= p.S; s += 4) {
-      const float v0 = __ldcg(src + (size_t)(s + 0) * QM * D), v1 = __ldcg(src + (size_t)(s + 1) * QM * D);
-      const float v2 = __ldcg(src + (size_t)(s + 2) * QM * D), v3 = __ldcg(src + (size_t)(s + 3) * QM * D);
-      O0 = fmaf(v0, wsm[(s + 0) * QM + n], O0);
-      O1 = fmaf(v1, wsm[(s + 1) * QM + n], O1);
-      O2 = fmaf(v2, wsm[(s + 2) * QM + n], O2);
-      O3 = fmaf(v3, wsm[(s + 3) * QM + n], O3);
+  {
+    // O = sum_s w_s O_s, four consecutive d per thread, eight splits in flight.
+    const int nf4 = QM * D / 4;
+    const float4* src0 = reinterpret_cast<const float4*>(p.ws_o + slot0 * QM * D);
+    for (int idx = tid; idx < nf4; idx += 128) {
+      const int n = (idx * 4) / D, d = (idx * 4) % D;
+      const float4* src = src0 + idx;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      int s2 = 0;
+      for (; s2 + 8 <= S; s2 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = __ldcg(src + (size_t)(s2 + j) * nf4);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float w = wsm[(s2 + j) * QM + n];
+          acc.x = fmaf(v[j].x, w, acc.x);
+          acc.y = fmaf(v[j].y, w, acc.y);
+          acc.z = fmaf(v[j].z, w, acc.z);
+          acc.w = fmaf(v[j].w, w, acc.w);
+        }
+      }
+      for (; s2 < S; ++s2) {
+        const float4 v = __ldcg(src + (size_t)s2 * nf4);
+        const float w = wsm[s2 * QM + n];
+        acc.x = fmaf(v.x, w, acc.x);
+        acc.y = fmaf(v.y, w, acc.y);
+        acc.z = fmaf(v.z, w, acc.z);
+        acc.w = fmaf(v.w, w, acc.w);
+      }
+      const int h = g * QM + n;
+      const float inv = 1.0f / Lsm[n];
+      uint2 packed;
+      packed.x = pack_bf16(acc.x * inv, acc.y * inv);
+      packed.y = pack_bf16(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(p.out + b * p.os0 + (long long)h * p.os2 + d) = packed;
+      if (d == 0 && p.lse) p.lse[(long long)b * p.n_q + h] = (Msm[n] + __log2f(Lsm[n])) * LN2;
     }
-    for (; s < p.S; ++s) O0 = fmaf(__ldcg(src + (size_t)s * QM * D), wsm[s * QM + n], O0);
-    const int h = g * QM + n;
-    const float L = Lsm[n];
-    p.out[b * p.os0 + (long long)h * p.os2 + d] = __float2bfloat16_rn(((O0 + O1) + (O2 + O3)) / L);
-    if (d == 0 && p.lse) p.lse[(long long)b * p.n_q + h] = (Msm[n] + __log2f(L)) * LN2;
   }
   if (tid == 0) p.ws_cnt[b * p.n_kv + g] = 0;
 }

@@ -1,32 +1,37 @@
 // Flash-style sink-augmented GQA prefill on tcgen05 tensor cores.
 //
 // One CTA owns two 128-row query tiles (A, B) of one (batch, query head) and
-// walks the 128-key tiles of the cache the mask admits for them:
+// walks the BN-key tiles of the cache the mask admits for them:
 //
 //   warp 0      TMA producer: K and V tiles of the head's KV group, straight
-//               from the cache [B][cap][n_kv][d] (rows past offset+T read as
-//               zeros through the tensor map's bounds), NS-deep ring each.
+//               from the head-major cache [B][n_kv][cap][d] (rows past
+//               offset+T read as zeros through the tensor map's bounds),
+//               NS-deep ring each.
 //   warp 1      allocates TMEM and issues every tcgen05.mma from one thread:
-//               S_X = Q_X K^T (smem x smem, fp32 in TMEM), then O_X += P_X V
-//               with P_X read from TMEM (bf16, aliased over S_X).
+//               S_X = Q_X K^T (smem x smem, fp32 in TMEM), then
+//               O_X += P_X V with P_X read from its own TMEM columns (bf16).
 //   warps 4-7   softmax for tile A, warps 8-11 for tile B, one query row per
 //               thread (TMEM lane = row): load + RoPE the Q row into swizzled
-//               smem, then per key tile: mask, running max in log2 units,
-//               exp2, P -> TMEM, and at the end O / l -> bf16 out.
+//               smem, then per key tile: read S, release it at once (so the
+//               tensor core computes the next S while this one is
+//               exponentiated), mask, running max in log2 units, exp2, P ->
+//               TMEM, and at the end O / l -> bf16 out.
+//
+// TMEM (512 columns): S_A, S_B (BN each), P_A, P_B (BN/2 bf16 pairs each),
+// O_A, O_B (d each); BN = 128 for d = 64, 96 for d = 96, 64 for d = 128.
 //
 // The softmax is seeded with the sink logit (m = sink, l = 1), so the extra
 // sink column of the MoE-Xtend README ("ATTENTION STACK", sink bias) is
 // folded in without ever materialising it, and dropped by construction (it
 // adds to l, never to O). The O rescale is lazy: the running max only moves
 // when it grows by more than 2^8, which keeps every P <= 256 and the result
-// exact up to rounding. Issue order S_A(t) after PV_A(t-1) makes the
-// completion of S_A(t) imply that of PV_A(t-1), so a softmax thread may
-// rescale O in TMEM as soon as its S is ready.
+// exact up to rounding. A softmax thread touches O (rescale) or P_X (next
+// store) only after the previous PV_X has completed (O_DONE barrier).
 //
-// Key tiles are aligned to tile A's diagonal (key off+i0), so each query
-// tile needs a mask only on its diagonal tile, its band edge and the first
-// (possibly partial, negative-start) tile; the band layers visit only the
-// tiles that intersect [p-W+1, p] -- O(T*W) work.
+// Key tiles are aligned to tile A's diagonal (key off+i0), so a query tile
+// needs a mask only on the tiles its diagonal or band edge crosses and on a
+// leading partial (negative-start) tile; band layers visit only the tiles that
+// intersect [p-W+1, p] -- O(T*W) work.
 #pragma once
 
 #include "ptx.cuh"
@@ -50,53 +55,73 @@ struct PrefillParams {
   int n_pairs;
 };
 
+__host__ __device__ constexpr int align32(int x) { return (x + 31) / 32 * 32; }
+
 template <int D>
 struct PrefillCfg {
-  static constexpr int BM = 128;                       // query rows per tile
-  static constexpr int BN = 128;                       // keys per tile
-  static constexpr int CB = (D % 64 == 0) ? 64 : 32;   // column-block width (elements)
-  static constexpr int SWZ = CB * 2;                   // bytes per block row (128 / 64)
+  static constexpr int BM = 128;                              // query rows per tile
+  static constexpr int BN = (D == 64) ? 128 : (D == 96 ? 96 : 64);  // keys per tile
+  static constexpr int CB = (D % 64 == 0) ? 64 : 32;          // column-block width (elements)
+  static constexpr int SWZ = CB * 2;                          // bytes per block row (128 / 64)
   static constexpr int NCB = D / CB;
-  static constexpr uint32_t BLOCK_BYTES = 128u * SWZ;  // one column block of a 128-row tile
-  static constexpr uint32_t TILE_BYTES = 128u * D * 2;
-  static constexpr int NS = (D == 64) ? 4 : (D == 96 ? 3 : 2);  // K and V ring depth
+  static constexpr uint32_t QBLOCK = 128u * SWZ;              // column block of a Q tile
+  static constexpr uint32_t Q_BYTES = 128u * D * 2;
+  static constexpr uint32_t KBLOCK = (uint32_t)BN * SWZ;      // column block of a K/V tile
+  static constexpr uint32_t KV_BYTES = (uint32_t)BN * D * 2;
+  static constexpr int NS = 4;                                // K and V ring depth
   static constexpr uint32_t LAYOUT = (SWZ == 128) ? 2u : 4u;
-  static constexpr uint32_t SBO = 8u * SWZ;            // 8-row core-matrix group stride
+  static constexpr uint32_t SBO = 8u * SWZ;                   // 8-row core-matrix group stride
   static constexpr int TMEM_COLS = 512;
-  static constexpr int S_COL0 = 0, S_COL1 = 128;       // S_A, S_B (P aliased in cols [0,64))
-  static constexpr int O_COL0 = 256, O_COL1 = 256 + D;
+  static constexpr int S_COL0 = 0, S_COL1 = BN;
+  static constexpr int P_COL0 = 2 * BN, P_COL1 = 2 * BN + align32(BN / 2);
+  static constexpr int O_COL0 = align32(P_COL1 + BN / 2), O_COL1 = O_COL0 + D;
+  static_assert(O_COL1 + D <= TMEM_COLS, "TMEM plan exceeds 512 columns");
+  static_assert(KBLOCK % 1024 == 0 && QBLOCK % 1024 == 0, "swizzle atoms need 1 KB alignment");
   static constexpr int NUM_THREADS = 384;
   // smem: Q[2] | K[NS] | V[NS] | barriers
   static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = 2 * TILE_BYTES;
-  static constexpr uint32_t OFF_V = OFF_K + NS * TILE_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_V + NS * TILE_BYTES;
+  static constexpr uint32_t OFF_K = 2 * Q_BYTES;
+  static constexpr uint32_t OFF_V = OFF_K + NS * KV_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_V + NS * KV_BYTES;
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
-  static constexpr uint32_t IDESC_QK = idesc_bf16(128, 128, 0, 0);
+  static constexpr uint32_t IDESC_QK = idesc_bf16(128, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, 0, 1);
 };
 
 // Barrier slots (8 bytes each) at OFF_BAR.
 enum : int {
-  BAR_QREADY = 0,  // [2]
-  BAR_SFULL = 2,   // [2]
-  BAR_PFULL = 4,   // [2]
-  BAR_OFINAL = 6,
-  BAR_DRAIN = 7,
-  BAR_KFULL = 8,   // [NS]
-  BAR_KEMPTY = 12, // [NS]
-  BAR_VFULL = 16,  // [NS]
-  BAR_VEMPTY = 20, // [NS]
-  BAR_TMEM_SLOT = 24,
-  BAR_ABORT_SLOT = 25,
+  BAR_QREADY = 0,  // [2] softmax threads -> MMA: Q tile in smem
+  BAR_SFULL = 2,   // [2] MMA -> softmax: S_X computed
+  BAR_SFREE = 4,   // [2] softmax -> MMA: S_X read into registers
+  BAR_PFULL = 6,   // [2] softmax -> MMA: P_X stored (and O_X rescaled)
+  BAR_ODONE = 8,   // [2] MMA -> softmax: PV_X completed
+  BAR_DRAIN = 10,
+  BAR_KFULL = 11,  // [NS]
+  BAR_KEMPTY = 15, // [NS]
+  BAR_VFULL = 19,  // [NS]
+  BAR_VEMPTY = 23, // [NS]
+  BAR_TMEM_SLOT = 28,
+  BAR_ABORT_SLOT = 29,
 };
 
+__device__ __forceinline__ long long floordiv(long long a, long long b) {  // b > 0
+  return a >= 0 ? a / b : -((-a + b - 1) / b);
+}
+
+// Key-tile geometry of one CTA: tile t covers keys [base + BN t, base + BN t + BN).
+// For query tile X (rows i0 + 128 X .. + 127, positions p = off + row):
+//   active tiles  [a_lo[X], a_hi[X]): the tile meets the admitted keys of some row;
+//   full tiles    [f_lo[X], f_hi[X]): every key of the tile is admitted for all
+//                 128 rows (0 <= key <= p, and key > p - W on band layers), so
+//                 no mask is applied there.
+template <int BN>
 struct TileGeom {
   long long off;
   int T, window;
   int i0;          // first query row of tile A
   long long base;  // first key of key tile 0
   int ntiles;
+  int a_lo[2], a_hi[2], f_lo[2], f_hi[2];
   __device__ __forceinline__ bool valid(int X) const { return i0 + 128 * X < T; }
   __device__ __forceinline__ long long lo(int X) const {
     const long long p0 = off + i0 + 128 * X;
@@ -106,58 +131,72 @@ struct TileGeom {
     const int last = min(T, i0 + 128 * X + 128);
     return off + last;
   }
-  __device__ __forceinline__ bool active(int X, int t) const {
-    if (t < 0 || t >= ntiles || !valid(X)) return false;
-    const long long klo = base + 128LL * t;
-    return klo < hi(X) && klo + 128 > lo(X);
-  }
-  // True when every (row, key) pair of the tile is admitted for all 128 rows.
-  __device__ __forceinline__ bool full(int X, int t) const {
-    const long long klo = base + 128LL * t;
-    const long long p0 = off + i0 + 128 * X;
-    if (klo < 0 || klo + 127 > p0) return false;
-    if (window > 0 && klo <= p0 + 127 - window) return false;
-    return true;
-  }
+  __device__ __forceinline__ bool active(int X, int t) const { return t >= a_lo[X] && t < a_hi[X]; }
+  __device__ __forceinline__ bool full(int X, int t) const { return t >= f_lo[X] && t < f_hi[X]; }
 };
 
-__device__ __forceinline__ TileGeom make_geom(const PrefillParams& p, int pair) {
-  TileGeom g;
+template <int BN>
+__device__ __forceinline__ TileGeom<BN> make_geom(const PrefillParams& p, int pair) {
+  TileGeom<BN> g;
   g.off = p.off;
   g.T = p.T;
   g.window = p.window;
   g.i0 = pair * 256;
   const long long diag = p.off + g.i0;
   const long long loA = g.lo(0);
-  const long long nb = (diag - loA + 127) / 128;
-  g.base = diag - 128 * nb;
+  const long long nb = (diag - loA + BN - 1) / BN;
+  g.base = diag - (long long)BN * nb;
   const long long hi = p.off + min(p.T, g.i0 + 256);
-  g.ntiles = (int)((hi - g.base + 127) / 128);
+  g.ntiles = (int)((hi - g.base + BN - 1) / BN);
+#pragma unroll
+  for (int X = 0; X < 2; ++X) {
+    if (!g.valid(X)) {
+      g.a_lo[X] = g.a_hi[X] = g.f_lo[X] = g.f_hi[X] = 0;
+      continue;
+    }
+    // active: klo < hi(X) and klo + BN > lo(X)
+    const long long alo = floordiv(g.lo(X) - g.base, BN);
+    const long long ahi = floordiv(g.hi(X) - g.base + BN - 1, BN);
+    g.a_lo[X] = (int)(alo < 0 ? 0 : alo);
+    g.a_hi[X] = (int)(ahi > g.ntiles ? g.ntiles : ahi);
+    // full: klo >= 0, klo + BN - 1 <= p0, and (band) klo > p0 + 127 - W
+    const long long p0 = p.off + g.i0 + 128 * X;
+    long long flo = floordiv(-g.base + BN - 1, BN);
+    if (p.window > 0) {
+      const long long w = floordiv(p0 + 127 - p.window - g.base, BN) + 1;
+      if (w > flo) flo = w;
+    }
+    const long long fhi = floordiv(p0 - BN + 1 - g.base, BN) + 1;
+    g.f_lo[X] = (int)(flo < g.a_lo[X] ? g.a_lo[X] : (flo > g.a_hi[X] ? g.a_hi[X] : flo));
+    g.f_hi[X] = (int)(fhi > g.a_hi[X] ? g.a_hi[X] : (fhi < g.f_lo[X] ? g.f_lo[X] : fhi));
+  }
   return g;
 }
 
-// MMA issue helpers (one thread). S_X = Q_X K_t^T over d/16 K-steps.
+// MMA issue helpers (one thread). Descriptors are built once per CTA and
+// advanced by compile-time offsets of their start-address field (16-byte
+// units; every operand stays below 256 KB of shared memory, so the 14-bit
+// field never carries).
+// S_X = Q_X K_t^T over d/16 K-steps.
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t qbase, uint32_t kbase) {
+__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint64_t qdesc, uint64_t kdesc) {
   using C = PrefillCfg<D>;
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t coff = (kk * 16 / C::CB) * C::BLOCK_BYTES + (kk * 16 % C::CB) * 2;
-    const uint64_t adesc = smem_desc(qbase + coff, 16, C::SBO, C::LAYOUT);
-    const uint64_t bdesc = smem_desc(kbase + coff, 16, C::SBO, C::LAYOUT);
-    mma_ss(s_tmem, adesc, bdesc, C::IDESC_QK, kk > 0 ? 1u : 0u);
+    const uint32_t cb = kk * 16 / C::CB, cin = (kk * 16 % C::CB) * 2;
+    mma_ss(s_tmem, qdesc + ((cb * C::QBLOCK + cin) >> 4), kdesc + ((cb * C::KBLOCK + cin) >> 4),
+           C::IDESC_QK, kk > 0 ? 1u : 0u);
   }
 }
-// O_X (+)= P_X V_t over 128/16 K-steps; P_X is bf16 in TMEM (cols [0,64) of S_X).
+// O_X (+)= P_X V_t over BN/16 K-steps; P_X is bf16 in TMEM.
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t vbase,
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t vdesc,
                                          bool accumulate) {
   using C = PrefillCfg<D>;
 #pragma unroll
-  for (int kk = 0; kk < 128 / 16; ++kk) {
-    const uint64_t bdesc = smem_desc(vbase + kk * 16 * C::SWZ, C::BLOCK_BYTES, C::SBO, C::LAYOUT);
-    mma_ts(o_tmem, p_tmem + kk * 8, bdesc, C::IDESC_PV, (accumulate || kk > 0) ? 1u : 0u);
-  }
+  for (int kk = 0; kk < C::BN / 16; ++kk)
+    mma_ts(o_tmem, p_tmem + kk * 8, vdesc + ((kk * 16 * C::SWZ) >> 4), C::IDESC_PV,
+           (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D>
@@ -165,6 +204,7 @@ __global__ void __launch_bounds__(384, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const PrefillParams p) {
   using C = PrefillCfg<D>;
+  constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -180,16 +220,16 @@ __global__ void __launch_bounds__(384, 1)
   const int h = blockIdx.y;
   const int b = blockIdx.z;
   const int g = h / p.q_mult;
-  const TileGeom geo = make_geom(p, pair);
+  const TileGeom<BN> geo = make_geom<BN>(p, pair);
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(BAR_QREADY + 0), 128);
-    mbar_init(bar(BAR_QREADY + 1), 128);
-    mbar_init(bar(BAR_SFULL + 0), 1);
-    mbar_init(bar(BAR_SFULL + 1), 1);
-    mbar_init(bar(BAR_PFULL + 0), 128);
-    mbar_init(bar(BAR_PFULL + 1), 128);
-    mbar_init(bar(BAR_OFINAL), 1);
+    for (int X = 0; X < 2; ++X) {
+      mbar_init(bar(BAR_QREADY + X), 128);
+      mbar_init(bar(BAR_SFULL + X), 1);
+      mbar_init(bar(BAR_SFREE + X), 128);
+      mbar_init(bar(BAR_PFULL + X), 128);
+      mbar_init(bar(BAR_ODONE + X), 1);
+    }
     mbar_init(bar(BAR_DRAIN), 1);
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar(BAR_KFULL + s), 1);
@@ -224,20 +264,20 @@ __global__ void __launch_bounds__(384, 1)
       for (int t = 0; t < geo.ntiles && !*abort_flag; ++t) {
         const int s = t % C::NS;
         const uint32_t ph = (uint32_t)((t / C::NS) & 1);
-        const int krow = (int)(geo.base + 128LL * t);
+        const int krow = (int)(geo.base + (long long)BN * t);
         if (!mbar_wait(bar(BAR_KEMPTY + s), ph ^ 1)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(bar(BAR_KFULL + s), C::TILE_BYTES);
+        mbar_arrive_expect_tx(bar(BAR_KFULL + s), C::KV_BYTES);
 #pragma unroll
         for (int cb = 0; cb < C::NCB; ++cb)
-          tma_load_4d(sbase + C::OFF_K + s * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmK,
-                      bar(BAR_KFULL + s), cb * C::CB, g, krow, b);
+          tma_load_4d(sbase + C::OFF_K + s * C::KV_BYTES + cb * C::KBLOCK, &tmK, bar(BAR_KFULL + s),
+                      cb * C::CB, krow, g, b);
         issued = t * 2 + 1;
         if (!mbar_wait(bar(BAR_VEMPTY + s), ph ^ 1)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(bar(BAR_VFULL + s), C::TILE_BYTES);
+        mbar_arrive_expect_tx(bar(BAR_VFULL + s), C::KV_BYTES);
 #pragma unroll
         for (int cb = 0; cb < C::NCB; ++cb)
-          tma_load_4d(sbase + C::OFF_V + s * C::TILE_BYTES + cb * C::BLOCK_BYTES, &tmV,
-                      bar(BAR_VFULL + s), cb * C::CB, g, krow, b);
+          tma_load_4d(sbase + C::OFF_V + s * C::KV_BYTES + cb * C::KBLOCK, &tmV, bar(BAR_VFULL + s),
+                      cb * C::CB, krow, g, b);
         issued = t * 2 + 2;
       }
       if (*abort_flag) {
@@ -250,60 +290,72 @@ __global__ void __launch_bounds__(384, 1)
       }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------ MMA issuer
+      // Per key tile t: S_A(t), S_B(t) as soon as the softmax released the
+      // previous S; then O_A += P_A(t-1) V(t-1), O_B += P_B(t-1) V(t-1).
       bool ok = true;
       if (geo.valid(0) && !mbar_wait(bar(BAR_QREADY + 0), 0)) ok = false;
       if (ok && geo.valid(1) && !mbar_wait(bar(BAR_QREADY + 1), 0)) ok = false;
       tc_fence_after();
-      const uint32_t qA = sbase + C::OFF_Q, qB = sbase + C::OFF_Q + C::TILE_BYTES;
-      const uint32_t sA = tmem + C::S_COL0, sB = tmem + C::S_COL1;
-      const uint32_t oA = tmem + C::O_COL0, oB = tmem + C::O_COL1;
-      int nA = 0, nB = 0;  // S tiles issued for A / B (P barrier phases)
+      const uint64_t qdA = smem_desc(sbase + C::OFF_Q, 16, C::SBO, C::LAYOUT);
+      const uint64_t qdB = smem_desc(sbase + C::OFF_Q + C::Q_BYTES, 16, C::SBO, C::LAYOUT);
+      const uint64_t kd0 = smem_desc(sbase + C::OFF_K, 16, C::SBO, C::LAYOUT);
+      const uint64_t vd0 = smem_desc(sbase + C::OFF_V, C::KBLOCK, C::SBO, C::LAYOUT);
+      const int a0lo = geo.a_lo[0], a0hi = geo.a_hi[0], a1lo = geo.a_lo[1], a1hi = geo.a_hi[1];
+      int nS0 = 0, nS1 = 0, nP0 = 0, nP1 = 0;
+      int ks = 0, kph = 0;                  // ring slot / phase of K(t)
+      int vs = C::NS - 1, vph = 1;          // ring slot / phase of V(t-1)
       for (int t = 0; t <= geo.ntiles && ok; ++t) {
-        const int ks = t % C::NS, vs = (t + C::NS - 1) % C::NS;
         if (t < geo.ntiles) {
-          if (!mbar_wait(bar(BAR_KFULL + ks), (uint32_t)((t / C::NS) & 1))) { ok = false; break; }
+          if (!mbar_wait(bar(BAR_KFULL + ks), (uint32_t)kph)) { ok = false; break; }
           tc_fence_after();
+          const uint64_t kd = kd0 + ((uint32_t)(ks * C::KV_BYTES) >> 4);
+          if (t >= a0lo && t < a0hi) {
+            if (nS0 > 0 && !mbar_wait(bar(BAR_SFREE + 0), (uint32_t)((nS0 - 1) & 1))) { ok = false; break; }
+            tc_fence_after();
+            issue_qk<D>(tmem + C::S_COL0, qdA, kd);
+            mma_commit(bar(BAR_SFULL + 0));
+            ++nS0;
+          }
+          if (t >= a1lo && t < a1hi) {
+            if (nS1 > 0 && !mbar_wait(bar(BAR_SFREE + 1), (uint32_t)((nS1 - 1) & 1))) { ok = false; break; }
+            tc_fence_after();
+            issue_qk<D>(tmem + C::S_COL1, qdB, kd);
+            mma_commit(bar(BAR_SFULL + 1));
+            ++nS1;
+          }
+          mma_commit(bar(BAR_KEMPTY + ks));
         }
         if (t > 0) {
-          if (!mbar_wait(bar(BAR_VFULL + vs), (uint32_t)(((t - 1) / C::NS) & 1))) { ok = false; break; }
+          if (!mbar_wait(bar(BAR_VFULL + vs), (uint32_t)vph)) { ok = false; break; }
           tc_fence_after();
+          const uint64_t vd = vd0 + ((uint32_t)(vs * C::KV_BYTES) >> 4);
+          if (t - 1 >= a0lo && t - 1 < a0hi) {
+            if (!mbar_wait(bar(BAR_PFULL + 0), (uint32_t)(nP0 & 1))) { ok = false; break; }
+            tc_fence_after();
+            issue_pv<D>(tmem + C::O_COL0, tmem + C::P_COL0, vd, nP0 > 0);
+            mma_commit(bar(BAR_ODONE + 0));
+            ++nP0;
+          }
+          if (t - 1 >= a1lo && t - 1 < a1hi) {
+            if (!mbar_wait(bar(BAR_PFULL + 1), (uint32_t)(nP1 & 1))) { ok = false; break; }
+            tc_fence_after();
+            issue_pv<D>(tmem + C::O_COL1, tmem + C::P_COL1, vd, nP1 > 0);
+            mma_commit(bar(BAR_ODONE + 1));
+            ++nP1;
+          }
+          mma_commit(bar(BAR_VEMPTY + vs));
         }
-        const uint32_t kb = sbase + C::OFF_K + ks * C::TILE_BYTES;
-        const uint32_t vb = sbase + C::OFF_V + vs * C::TILE_BYTES;
-        // tile A: O_A += P_A(t-1) V(t-1), then S_A = Q_A K(t)^T
-        if (geo.active(0, t - 1)) {
-          if (!mbar_wait(bar(BAR_PFULL + 0), (uint32_t)((nA - 1) & 1))) { ok = false; break; }
-          tc_fence_after();
-          issue_pv<D>(oA, sA, vb, nA > 1);
-        }
-        if (t < geo.ntiles && geo.active(0, t)) {
-          issue_qk<D>(sA, qA, kb);
-          mma_commit(bar(BAR_SFULL + 0));
-          ++nA;
-        }
-        // tile B
-        if (geo.active(1, t - 1)) {
-          if (!mbar_wait(bar(BAR_PFULL + 1), (uint32_t)((nB - 1) & 1))) { ok = false; break; }
-          tc_fence_after();
-          issue_pv<D>(oB, sB, vb, nB > 1);
-        }
-        if (t < geo.ntiles && geo.active(1, t)) {
-          issue_qk<D>(sB, qB, kb);
-          mma_commit(bar(BAR_SFULL + 1));
-          ++nB;
-        }
-        if (t < geo.ntiles) mma_commit(bar(BAR_KEMPTY + ks));
-        if (t > 0) mma_commit(bar(BAR_VEMPTY + vs));
+        // advance the ring positions: K(t+1), V(t)
+        vs = ks;
+        vph = kph;
+        if (++ks == C::NS) { ks = 0; kph ^= 1; }
         if (*abort_flag) { ok = false; break; }
       }
-      if (ok) {
-        mma_commit(bar(BAR_OFINAL));
-      } else {
+      if (!ok) {
         *abort_flag = 1;
         // Drain the tensor pipe before anything is released.
         mma_commit(bar(BAR_DRAIN));
         mbar_wait(bar(BAR_DRAIN), 0);
-        mma_commit(bar(BAR_OFINAL));  // wake the epilogue (its data is discarded)
       }
     }
   } else {
@@ -317,11 +369,12 @@ __global__ void __launch_bounds__(384, 1)
     const long long pos = p.off + i;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_tm = tmem + lane_base + (X ? C::S_COL1 : C::S_COL0);
+    const uint32_t p_tm = tmem + lane_base + (X ? C::P_COL1 : C::P_COL0);
     const uint32_t o_tm = tmem + lane_base + (X ? C::O_COL1 : C::O_COL0);
 
     if (geo.valid(X)) {
       // Q row -> (RoPE) -> bf16 -> swizzled smem, K-major for the MMA.
-      uint8_t* qtile = smem + C::OFF_Q + X * C::TILE_BYTES;
+      uint8_t* qtile = smem + C::OFF_Q + X * C::Q_BYTES;
       if (row_ok) {
         const __nv_bfloat16* qrow = p.q + b * p.qs0 + (long long)i * p.qs1 + (long long)h * p.qs2;
         constexpr int HALF = D / 2;
@@ -339,14 +392,14 @@ __global__ void __launch_bounds__(384, 1)
             rope_pair2(a.z, c.z, c1.x, c1.y, s1.x, s1.y);
             rope_pair2(a.w, c.w, c1.z, c1.w, s1.z, s1.w);
           }
-          *reinterpret_cast<uint4*>(qtile + swz_off<C::CB>(r, ch * 8, C::BLOCK_BYTES)) = a;
-          *reinterpret_cast<uint4*>(qtile + swz_off<C::CB>(r, HALF + ch * 8, C::BLOCK_BYTES)) = c;
+          *reinterpret_cast<uint4*>(qtile + swz_off<C::CB>(r, ch * 8, C::QBLOCK)) = a;
+          *reinterpret_cast<uint4*>(qtile + swz_off<C::CB>(r, HALF + ch * 8, C::QBLOCK)) = c;
         }
       } else {
         const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
         for (int ch = 0; ch < D / 8; ++ch)
-          *reinterpret_cast<uint4*>(qtile + swz_off<C::CB>(r, ch * 8, C::BLOCK_BYTES)) = z;
+          *reinterpret_cast<uint4*>(qtile + swz_off<C::CB>(r, ch * 8, C::QBLOCK)) = z;
       }
       fence_proxy_async_smem();
       mbar_arrive(bar(BAR_QREADY + X));
@@ -358,32 +411,34 @@ __global__ void __launch_bounds__(384, 1)
       float l = (sink2 == -INFINITY) ? 0.f : 1.f;   // running sum, sink included
       int n = 0;
       bool ok = true;
-      for (int t = 0; t < geo.ntiles; ++t) {
-        if (!geo.active(X, t)) continue;
+      const int t_lo = X ? geo.a_lo[1] : geo.a_lo[0], t_hi = X ? geo.a_hi[1] : geo.a_hi[0];
+      const int full_lo = X ? geo.f_lo[1] : geo.f_lo[0], full_hi = X ? geo.f_hi[1] : geo.f_hi[0];
+      for (int t = t_lo; t < t_hi; ++t) {
         if (!mbar_wait(bar(BAR_SFULL + X), (uint32_t)(n & 1))) { ok = false; *abort_flag = 1; break; }
         tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld32(s_tm + 0, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-        tmem_ld32(s_tm + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-        tmem_ld32(s_tm + 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[64]));
-        tmem_ld32(s_tm + 96, *reinterpret_cast<uint32_t(*)[32]>(&sr[96]));
+        uint32_t sr[BN];
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += 32)
+          tmem_ld32(s_tm + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[c0]));
         tmem_wait_ld();
-        if (!geo.full(X, t)) {
+        tc_fence_before();
+        mbar_arrive(bar(BAR_SFREE + X));   // the tensor core may overwrite S_X now
+        if (t < full_lo || t >= full_hi) {
           // admitted columns c (key klo + c): c >= cmin and c <= cmax
-          const long long klo = geo.base + 128LL * t;
+          const long long klo = geo.base + (long long)BN * t;
           long long lo_k = 0;
           if (p.window > 0 && pos - p.window + 1 > lo_k) lo_k = pos - p.window + 1;
-          long long cmin = lo_k - klo, cmax = pos - klo;
-          const int cmin_i = (int)(cmin < -1 ? -1 : (cmin > 128 ? 128 : cmin));
-          const int cmax_i = (int)(cmax < -1 ? -1 : (cmax > 128 ? 128 : cmax));
+          const long long cmin = lo_k - klo, cmax = pos - klo;
+          const int cmin_i = (int)(cmin < -1 ? -1 : (cmin > BN ? BN : cmin));
+          const int cmax_i = (int)(cmax < -1 ? -1 : (cmax > BN ? BN : cmax));
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
+          for (int c = 0; c < BN; ++c)
             if (c < cmin_i || c > cmax_i) sr[c] = __float_as_uint(-INFINITY);
         }
         // raw row max (scale > 0, so max(s * scale) = scale * max(s))
         float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 128; c += 8) {
+        for (int c = 0; c < BN; c += 8) {
           m0 = max3f(m0, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
           m1 = max3f(m1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
           m2 = max3f(m2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
@@ -392,25 +447,28 @@ __global__ void __launch_bounds__(384, 1)
         const float mx = fmaxf(max3f(m0, m1, m2), m3) * scale;
         const float m_new = fmaxf(m, mx);
         const bool need = m_new > m + 8.0f;
+        bool pv_done = (n == 0);
         if (__any_sync(0xffffffffu, need)) {
           const float f = need ? ex2(m - m_new) : 1.0f;
           if (n > 0) {
-            // O rows stay in TMEM; S_X(t) complete implies PV_X(t-1) complete.
-#pragma unroll
-            for (int c0 = 0; c0 < D; c0 += 32) {
-              uint32_t rr[32];
-              tmem_ld32(o_tm + c0, rr);
+            // O_X may only be touched once the previous PV_X has landed.
+            if (!mbar_wait(bar(BAR_ODONE + X), (uint32_t)((n - 1) & 1))) { ok = false; *abort_flag = 1; break; }
+            tc_fence_after();
+            pv_done = true;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 16) {
+              uint32_t rr[16];
+              tmem_ld16(o_tm + c0, rr);
               tmem_wait_ld();
 #pragma unroll
-              for (int c = 0; c < 32; c += 2) {
+              for (int c = 0; c < 16; c += 2) {
                 float a0 = __uint_as_float(rr[c]), a1 = __uint_as_float(rr[c + 1]);
                 mul2(a0, a1, f, f);
                 rr[c] = __float_as_uint(a0);
                 rr[c + 1] = __float_as_uint(a1);
               }
-              tmem_st32(o_tm + c0, rr);
+              tmem_st16(o_tm + c0, rr);
             }
-            tmem_wait_st();
           }
           if (need) {
             l *= f;
@@ -418,33 +476,40 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         const float neg = (m == -INFINITY) ? 0.f : -m;
+        uint32_t pk[BN / 2];
         float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
 #pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const int j = q2 * 64 + 2 * c;
-            float x0, x1, x2, x3;
-            fma2(x0, x1, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]), scale, scale, neg, neg);
-            fma2(x2, x3, __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]), scale, scale, neg, neg);
-            const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
-            add2(l0, l1, p0, p1);
-            add2(l2, l3, p2, p3);
-            pk[c] = pack_bf16(p0, p1);
-            pk[c + 1] = pack_bf16(p2, p3);
-          }
-          tmem_st32(s_tm + q2 * 32, pk);
+        for (int c = 0; c < BN / 2; c += 2) {
+          float x0, x1, x2, x3;
+          fma2(x0, x1, __uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]), scale, scale, neg, neg);
+          fma2(x2, x3, __uint_as_float(sr[2 * c + 2]), __uint_as_float(sr[2 * c + 3]), scale, scale, neg, neg);
+          x0 = ex2(x0);
+          x1 = ex2(x1);
+          x2 = ex2(x2);
+          x3 = ex2(x3);
+          add2(l0, l1, x0, x1);
+          add2(l2, l3, x2, x3);
+          pk[c] = pack_bf16(x0, x1);
+          pk[c + 1] = pack_bf16(x2, x3);
         }
         l += (l0 + l1) + (l2 + l3);
+        // P_X is read by the previous PV_X until it completes.
+        if (!pv_done) {
+          if (!mbar_wait(bar(BAR_ODONE + X), (uint32_t)((n - 1) & 1))) { ok = false; *abort_flag = 1; break; }
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int c0 = 0; c0 + 32 <= BN / 2; c0 += 32)
+          tmem_st32(p_tm + c0, *reinterpret_cast<uint32_t(*)[32]>(&pk[c0]));
+        if constexpr ((BN / 2) % 32 == 16) tmem_st16(p_tm + (BN / 2 - 16), &pk[BN / 2 - 16]);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(BAR_PFULL + X));
         ++n;
         if (*abort_flag) { ok = false; break; }
       }
-      // Epilogue: O / l -> bf16.
-      if (n > 0 && mbar_wait(bar(BAR_OFINAL), 0) && ok && !*abort_flag) {
+      // Epilogue: O / l -> bf16, once the last PV_X has landed.
+      if (n > 0 && mbar_wait(bar(BAR_ODONE + X), (uint32_t)((n - 1) & 1)) && ok && !*abort_flag) {
         tc_fence_after();
         const float inv_l = 1.0f / l;
         __nv_bfloat16* orow = p.out + b * p.os0 + (long long)i * p.os1 + (long long)h * p.os2;

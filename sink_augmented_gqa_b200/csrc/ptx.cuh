@@ -164,6 +164,23 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -255,6 +272,42 @@ __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, f
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
+// (d0, d1) = (a0 + b0, a1 + b1), one packed instruction.
+__device__ __forceinline__ void addto2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
+// Two values of 2^x on the FMA pipe instead of the MUFU unit, for
+// x in [-120, 8] (smaller x is clamped to -120: 2^-120 stands in for the
+// vanishing weight). Range reduction: t = x + 1.5*2^23 rounds x to the
+// nearest integer j (held in t's low mantissa bits), f = x - j in
+// [-1/2, 1/2] exactly; then 2^x = 2^j * p(f), the 2^j applied as an integer
+// add of j << 23 to p's bit pattern. p is the degree-4 fit of 2^f on
+// [-1/2, 1/2] produced by fit_exp2_poly.py (relative error < 3e-6 in fp32
+// Horner form).
+constexpr float EXP2_C0 = 0.999999285f, EXP2_C1 = 0.693121791f, EXP2_C2 = 0.240247443f,
+                EXP2_C3 = 0.0559178591f, EXP2_C4 = 0.00957009662f;
+__device__ __forceinline__ void exp2_fma2(float& a, float& b) {
+  constexpr float MAGIC = 12582912.0f;  // 1.5 * 2^23
+  a = fmaxf(a, -120.0f);
+  b = fmaxf(b, -120.0f);
+  float ta, tb, ja, jb, fa, fb;
+  addto2(ta, tb, a, b, MAGIC, MAGIC);
+  addto2(ja, jb, ta, tb, -MAGIC, -MAGIC);
+  addto2(fa, fb, a, b, -ja, -jb);
+  float pa = EXP2_C4, pb = EXP2_C4;
+  fma2(pa, pb, pa, pb, fa, fb, EXP2_C3, EXP2_C3);
+  fma2(pa, pb, pa, pb, fa, fb, EXP2_C2, EXP2_C2);
+  fma2(pa, pb, pa, pb, fa, fb, EXP2_C1, EXP2_C1);
+  fma2(pa, pb, pa, pb, fa, fb, EXP2_C0, EXP2_C0);
+  a = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
+  b = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
+}
+
 // (a0, a1) += (b0, b1), one packed instruction.
 __device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
   asm("{\n\t.reg .b64 ra, rb, rd;\n\t"

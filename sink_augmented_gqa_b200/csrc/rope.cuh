@@ -105,7 +105,7 @@ __global__ void kv_append_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat16* 
     uint4 c = *reinterpret_cast<const uint4*>(krow + half + ch * 8);
     const long long p = off + t;
     if (rope) rotate8(a, c, cos_t + p * half + ch * 8, sin_t + p * half + ch * 8);
-    const long long dst = (((long long)b * cap + p) * n_kv + g) * d;
+    const long long dst = (((long long)b * n_kv + g) * cap + p) * d;
     *reinterpret_cast<uint4*>(ck + dst + ch * 8) = a;
     *reinterpret_cast<uint4*>(ck + dst + half + ch * 8) = c;
     *reinterpret_cast<uint4*>(cv + dst + ch * 8) = *reinterpret_cast<const uint4*>(vrow + ch * 8);

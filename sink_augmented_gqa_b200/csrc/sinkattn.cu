@@ -63,16 +63,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Tensor map over one cache buffer [B][cap][n_kv][d] bf16 that exposes only
-// rows [0, rows_valid) (later rows read back as zeros), box {CB, 1, box_rows, 1}.
+// Tensor map over one cache buffer [B][n_kv][cap][d] bf16 that exposes only
+// rows [0, rows_valid) (later rows read back as zeros): dims {d, rows, n_kv,
+// B}, box {CB, box_rows, 1, 1}.
 bool make_cache_map(CUtensorMap* map, void* base, int d, int n_kv, long long rows_valid, int cap,
                     int B, int box_rows, int cb) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr || rows_valid < 1) return false;
-  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)n_kv, (cuuint64_t)rows_valid, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)n_kv * d * 2,
-                                 (cuuint64_t)cap * n_kv * d * 2};
-  const cuuint32_t box[4] = {(cuuint32_t)cb, 1, (cuuint32_t)box_rows, 1};
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)rows_valid, (cuuint64_t)n_kv, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)cap * d * 2,
+                                 (cuuint64_t)n_kv * cap * d * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)cb, (cuuint32_t)box_rows, 1, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -149,8 +150,11 @@ sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream
   using Cfg = PrefillCfg<D>;
   CUtensorMap tmK, tmV;
   const long long rows = a->offset + a->T;
-  if (!make_cache_map(&tmK, c->k, D, c->n_kv, rows, c->cap, c->B, 128, Cfg::CB) ||
-      !make_cache_map(&tmV, c->v, D, c->n_kv, rows, c->cap, c->B, 128, Cfg::CB))
+  // The box is one BN-row K/V tile: the kernel's expect-tx byte count and
+  // ring-slot size are both Cfg::KV_BYTES = BN * D * 2.
+  static_assert(Cfg::KV_BYTES == (uint32_t)Cfg::BN * D * 2, "tile size");
+  if (!make_cache_map(&tmK, c->k, D, c->n_kv, rows, c->cap, c->B, Cfg::BN, Cfg::CB) ||
+      !make_cache_map(&tmV, c->v, D, c->n_kv, rows, c->cap, c->B, Cfg::BN, Cfg::CB))
     return SA_ERR_CUDA;
   PrefillParams p;
   p.q = static_cast<const __nv_bfloat16*>(a->q);
@@ -204,7 +208,7 @@ DecodeSplit decode_split(int B, int n_kv, long long n_cache) {
 }
 
 // Workspace layout: counters [B*n_kv] int32 (256-byte padded), then
-// m [B*n_kv*S*q_mult], l [same], O [B*n_kv*S*q_mult*d] fp32.
+// O [B*n_kv*S*q_mult*d], m [B*n_kv*S*q_mult], l [same] fp32.
 size_t decode_ws_bytes(int B, int n_kv, int q_mult, int d, int S) {
   const size_t cnt = (((size_t)B * n_kv * 4) + 255) / 256 * 256;
   const size_t rows = (size_t)B * n_kv * S * q_mult;
@@ -264,9 +268,9 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   const size_t cnt = (((size_t)a->B * c->n_kv * 4) + 255) / 256 * 256;
   const size_t rows = (size_t)a->B * c->n_kv * p.S * q_mult;
   p.ws_cnt = reinterpret_cast<int*>(w);
-  p.ws_m = reinterpret_cast<float*>(w + cnt);
-  p.ws_l = reinterpret_cast<float*>(w + cnt + rows * 4);
-  p.ws_o = reinterpret_cast<float*>(w + cnt + rows * 8);
+  p.ws_o = reinterpret_cast<float*>(w + cnt);
+  p.ws_m = reinterpret_cast<float*>(w + cnt + rows * D * 4);
+  p.ws_l = reinterpret_cast<float*>(w + cnt + rows * D * 4 + rows * 4);
   static bool configured = false;
   if (!configured) {
     set_smem(sa::decode_kernel<D>, Cfg::SMEM_BYTES);

@@ -172,10 +172,11 @@ class Snapshot:
 
 
 class KVCache:
-    """One layer's bf16 KV cache [B, cap, n_kv, d] (torch-owned device memory)."""
+    """One layer's bf16 KV cache, head-major [B, n_kv, cap, d] (torch-owned
+    device memory). ``rows(b_slice, start, stop)`` views rows as [B, T, n_kv, d]."""
 
     def __init__(self, B, cap, n_kv, d, device="cuda", k=None, v=None):
-        shape = (B, cap, n_kv, d)
+        shape = (B, n_kv, cap, d)
         self.k = k if k is not None else torch.zeros(shape, dtype=torch.bfloat16, device=device)
         self.v = v if v is not None else torch.zeros(shape, dtype=torch.bfloat16, device=device)
         assert tuple(self.k.shape) == shape and self.k.is_contiguous() and self.v.is_contiguous()
@@ -186,6 +187,13 @@ class KVCache:
     @property
     def offset(self):
         return self.raw.offset
+
+    def k_rows(self, start=0, stop=None):
+        """K rows [start, stop) as a [B, T, n_kv, d] view."""
+        return self.k[:, :, start:stop].transpose(1, 2)
+
+    def v_rows(self, start=0, stop=None):
+        return self.v[:, :, start:stop].transpose(1, 2)
 
     @property
     def B(self):

@@ -78,9 +78,9 @@ def test_kv_append_snapshot_restore_bit_exact(cuda_device):
     v2 = wl.randn_bf16((B, 50, n_kv, d), 9, 4).to(DEV)
     cache.append(k2, v2)
     torch.cuda.synchronize()
-    assert torch.equal(cache.k[:, :100], k1) and torch.equal(cache.v[:, :100], v1)
-    assert torch.equal(cache.k[:, 100:150], k2) and torch.equal(cache.v[:, 100:150], v2)
-    assert torch.count_nonzero(cache.k[:, 150:]) == 0
+    assert torch.equal(cache.k_rows(0, 100), k1) and torch.equal(cache.v_rows(0, 100), v1)
+    assert torch.equal(cache.k_rows(100, 150), k2) and torch.equal(cache.v_rows(100, 150), v2)
+    assert torch.count_nonzero(cache.k_rows(150)) == 0
     snap150 = cache.snapshot()
     cache.restore(snap)
     assert cache.offset == 100
@@ -97,7 +97,7 @@ def test_kv_append_snapshot_restore_bit_exact(cuda_device):
     big = wl.randn_bf16((B, 5, 2 * n_kv, d), 9, 7).to(DEV)
     cache.append(big[:, :, ::2], big[:, :, 1::2])
     torch.cuda.synchronize()
-    assert torch.equal(cache.k[:, 100:105], big[:, :, ::2]) and torch.equal(cache.v[:, 100:105], big[:, :, 1::2])
+    assert torch.equal(cache.k_rows(100, 105), big[:, :, ::2]) and torch.equal(cache.v_rows(100, 105), big[:, :, 1::2])
 
 
 # ---------------------------------------------------------------------------
@@ -157,9 +157,9 @@ def test_prefill_matches_oracle(cuda_device, name, over, off, T, layer):
     check_lse(lse, ref_lse, f"{name}/{layer}")
     # the cache now holds the oracle's rotated K (within one bf16 step) and V bit for bit
     n = off + T
-    kdiff = np.abs(to64(cache.k[:, :n]) - ocache.K[:, :n])
+    kdiff = np.abs(to64(cache.k_rows(0, n)) - ocache.K[:, :n])
     assert np.all(kdiff <= obf16.bf16_ulp(ocache.K[:, :n]) * 1.0000001)
-    assert np.array_equal(to64(cache.v[:, :n]), ocache.V[:, :n])
+    assert np.array_equal(to64(cache.v_rows(0, n)), ocache.V[:, :n])
     assert cache.offset == ocache.offset == n
 
 
@@ -302,7 +302,7 @@ def test_handoff_prefill_equals_prefix_plus_decode(cuda_device, layer):
                                cfg.sm_scale, cos, sin, workspace=ws)
             check_bf16_output(o, oref[:, t:t + 1], f"handoff decode {t}")
         torch.cuda.synchronize()
-        assert torch.equal(cache.k[:, :cap], full.k[:, :cap]) and torch.equal(cache.v[:, :cap], full.v[:, :cap])
+        assert torch.equal(cache.k, full.k) and torch.equal(cache.v, full.v)
         cache.restore(snap)
         assert cache.offset == cfg.offset + cfg.T
 
