@@ -223,6 +223,29 @@ sa_status sa_attn_decode(sa_kv_cache* cache, const sa_attn_args* args, void* wor
 size_t sa_attn_decode_workspace_size(int32_t B, int32_t n_q, int32_t n_kv, int32_t d);
 
 /*
+ * Decode for callers that cannot allocate device memory: an embedded runtime
+ * without its own allocator, code that must not call cudaMalloc in its
+ * serving loop, or a host process that only ever receives device pointers
+ * from someone else. The pages have no counterpart to this entry point.
+ *
+ * Same operation, arguments and results as sa_attn_decode, but the split
+ * scratch lives in a fixed array inside the library (a file-scope
+ * __device__ array of SA_DECODE_STATIC_SCRATCH_BYTES bytes, which every GPU
+ * that loads the library holds until the process exits). No call allocates:
+ * no cudaMalloc, cudaFree or allocating library routine.
+ * - The first call on a device (with that device current) looks up the
+ *   array's device address and zeroes it once; make that first call before
+ *   any stream capture.
+ * - SA_ERR_WORKSPACE when this call's split scratch would exceed
+ *   SA_DECODE_STATIC_SCRATCH_BYTES (large B * n_kv * q_mult * d); use
+ *   sa_attn_decode with a workspace then.
+ * - Every call shares the one array: calls that overlap on the GPU (other
+ *   streams, other threads) race. Order them on one stream.
+ */
+#define SA_DECODE_STATIC_SCRATCH_BYTES (1u << 20)
+sa_status sa_attn_decode_static(sa_kv_cache* cache, const sa_attn_args* args, sa_stream_t stream);
+
+/*
  * Reads and clears the device status word of the current device (waits for
  * the device to be idle). *code receives SA_OK or SA_ERR_TIMEOUT.
  */

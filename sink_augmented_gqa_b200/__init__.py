@@ -11,6 +11,7 @@ from .sinkattn import (  # noqa: F401
     KVCache,
     SinkAttnError,
     attn_decode,
+    attn_decode_static,
     attn_prefill,
     decode_workspace,
     decode_workspace_bytes,

@@ -7,6 +7,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/sinkattn.h"
 #include "decode.cuh"
 #include "prefill.cuh"
@@ -293,6 +295,31 @@ sa_status launch_append(sa_kv_cache* c, const void* k, const int64_t ks[3], cons
   return last_launch_status();
 }
 
+// Scratch of sa_attn_decode_static: one fixed array per device, its device
+// address looked up once per device (host code may not use the symbol itself
+// as an address).
+static __device__ __align__(256) uint8_t g_decode_scratch[SA_DECODE_STATIC_SCRATCH_BYTES];
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+sa_status static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || ptr == nullptr) return SA_ERR_CUDA;
+    // the split counters must start at zero (each call leaves them at zero)
+    if (cudaMemset(ptr, 0, SA_DECODE_STATIC_SCRATCH_BYTES) != cudaSuccess) return SA_ERR_CUDA;
+    if (cudaDeviceSynchronize() != cudaSuccess) return SA_ERR_CUDA;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return SA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -447,6 +474,22 @@ sa_status sa_attn_decode(sa_kv_cache* cache, const sa_attn_args* a, void* worksp
   }
   if (st == SA_OK) note_append(cache, cache->offset, 1);
   return st;
+}
+
+sa_status sa_attn_decode_static(sa_kv_cache* cache, const sa_attn_args* a, sa_stream_t stream) {
+  sa_status st = check_attn(cache, a);
+  if (st != SA_OK) return st;
+  if (a->T != 1) return SA_ERR_INVALID_ARG;
+  const int q_mult = a->n_q / cache->n_kv;
+  if (q_mult > 8) return SA_ERR_SHAPE;
+  const long long lo = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
+  const DecodeSplit sp = decode_split(a->B, cache->n_kv, a->offset - lo);
+  if (sp.S > 1 && decode_ws_bytes(a->B, cache->n_kv, q_mult, cache->d, sp.S) > SA_DECODE_STATIC_SCRATCH_BYTES)
+    return SA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  st = static_scratch(&scratch);
+  if (st != SA_OK) return st;
+  return sa_attn_decode(cache, a, scratch, SA_DECODE_STATIC_SCRATCH_BYTES, stream);
 }
 
 size_t sa_attn_decode_workspace_size(int32_t B, int32_t n_q, int32_t n_kv, int32_t d) {

@@ -71,6 +71,7 @@ EXPORTS = (
     "sa_status_string", "sa_yarn_rope_tables", "sa_rope_apply_qk", "sa_kv_cache_init",
     "sa_kv_append", "sa_kv_snapshot", "sa_kv_restore", "sa_attn_prefill", "sa_attn_decode",
     "sa_attn_decode_workspace_size", "sa_get_device_status", "sa_set_wait_limit",
+    "sa_attn_decode_static",
 )
 
 _lib = None
@@ -97,6 +98,7 @@ def lib():
         L.sa_kv_restore.argtypes = [P(_KVCache), P(_Snapshot)]
         L.sa_attn_prefill.argtypes = [P(_KVCache), P(_AttnArgs), vp]
         L.sa_attn_decode.argtypes = [P(_KVCache), P(_AttnArgs), vp, ctypes.c_size_t, vp]
+        L.sa_attn_decode_static.argtypes = [P(_KVCache), P(_AttnArgs), vp]
         L.sa_attn_decode_workspace_size.restype = ctypes.c_size_t
         L.sa_attn_decode_workspace_size.argtypes = [i32, i32, i32, i32]
         L.sa_get_device_status.argtypes = [P(i32)]
@@ -273,6 +275,22 @@ def attn_decode(cache, q, k, v, sinks, window, sm_scale, cos=None, sin=None, rop
     _check(lib().sa_attn_decode(ctypes.byref(cache.raw), ctypes.byref(a), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(q)),
            "sa_attn_decode")
+    return (out, lse) if return_lse else out
+
+
+def attn_decode_static(cache, q, k, v, sinks, window, sm_scale, cos=None, sin=None, rope_fused=True,
+                       out=None, return_lse=False, lse=None):
+    """attn_decode for callers that cannot allocate: the split scratch is a
+    fixed array inside the library (SA_DECODE_STATIC_SCRATCH_BYTES per device),
+    shared by every call -- do not overlap calls on the GPU."""
+    B, T, n_q, d = q.shape
+    if out is None:
+        out = torch.empty((B, T, n_q, d), dtype=torch.bfloat16, device=q.device)
+    if return_lse and lse is None:
+        lse = torch.empty((B, n_q, T), dtype=torch.float32, device=q.device)
+    a = _args(cache, q, k, v, sinks, window, sm_scale, cos, sin, rope_fused, out, lse)
+    _check(lib().sa_attn_decode_static(ctypes.byref(cache.raw), ctypes.byref(a), _stream(q)),
+           "sa_attn_decode_static")
     return (out, lse) if return_lse else out
 
 
