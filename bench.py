@@ -62,6 +62,30 @@ def pairs(off, T, window):
     return n
 
 
+def profiled_traffic(summary, sources):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel sources changed since that capture (their sha256 no longer matches)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", summary)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line:
+            k, _, v = line.partition(":")
+            fields[k.strip()] = v.strip()
+    h = hashlib.sha256()
+    for src in sources:
+        with open(os.path.join(ROOT, "sink_augmented_gqa_b200", "csrc", src), "rb") as f:
+            h.update(f.read())
+    if fields.get("kernel_sources_sha256") != h.hexdigest():
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def flops(cfg, off, T, window):
     return 4 * cfg.d * cfg.B * cfg.n_q * pairs(off, T, window)
 
@@ -194,11 +218,22 @@ def _time_loop(fn, steps, warmup, dist=None):
     if dist is not None:
         dist.barrier()
     ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return max_over_ranks(ms, dist, "cuda")
+
+
+def max_over_ranks(x, dist, device):
+    """The largest of every rank's x (the job's time is its slowest rank's)."""
+    if dist is None:
+        return x
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_rank_step, ms_per_step):
+    """Whole-job rate: every rank processes its own batch (weak scaling), and
+    the step takes as long as the slowest rank."""
+    return world * units_per_rank_step / (ms_per_step * 1e-3)
 
 
 def full_prefill_roofline(step, steps, peaks):
@@ -519,10 +554,11 @@ def main():
         full_ms, full_tf = full_prefill_roofline(step, max(3, min(args.steps, 10)), peaks)
     clocks = clk.summary()
     ms_step = ms / args.steps
-    value = world * step.flops / (ms_step * 1e-3) / 1e12
+    value = job_throughput(world, step.flops, ms_step) / 1e12
 
-    e2e_ms, h2d, d2h = e2e_lite(step, max(3, args.steps // 2), 2)
-    e2e_val = world * step.flops / (e2e_ms * 1e-3) / 1e12
+    e2e_ms, h2d, d2h = e2e_lite(step, max(3, args.steps // 2), 3)
+    e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
+    e2e_val = job_throughput(world, step.flops, e2e_ms) / 1e12
 
     extras = {}
     if not args.no_extras and rank == 0:
@@ -537,13 +573,7 @@ def main():
     if dist is not None:
         dist.barrier()
     if rank == 0:
-        prof = os.path.join(ROOT, "profiles", "prefill_full_lite_traffic.json")
-        traffic = None
-        if os.path.exists(prof):
-            try:
-                traffic = json.load(open(prof)).get("traffic_bytes_per_launch")
-            except Exception:
-                traffic = None
+        traffic = profiled_traffic("prefill_lite_full.md", ("prefill.cuh", "ptx.cuh"))
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),

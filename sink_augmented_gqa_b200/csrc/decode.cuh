@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(160)
       }
       if (flag[0]) {
         for (int it = (issued > C::NS ? issued - C::NS : 0); it < issued; ++it)
-          mbar_wait(full_bar(it % C::NS), (uint32_t)((it / C::NS) & 1));
+          mbar_wait_drain(full_bar(it % C::NS), (uint32_t)((it / C::NS) & 1));
       }
     }
     return;  // the producer takes no part in the merge (named barriers below count 128)

@@ -284,9 +284,9 @@ __global__ void __launch_bounds__(384, 1)
         // Let every copy still in flight land before the CTA can exit.
         const int nk = (issued + 1) / 2, nv = issued / 2;
         for (int t = (nk > C::NS ? nk - C::NS : 0); t < nk; ++t)
-          mbar_wait(bar(BAR_KFULL + t % C::NS), (uint32_t)((t / C::NS) & 1));
+          mbar_wait_drain(bar(BAR_KFULL + t % C::NS), (uint32_t)((t / C::NS) & 1));
         for (int t = (nv > C::NS ? nv - C::NS : 0); t < nv; ++t)
-          mbar_wait(bar(BAR_VFULL + t % C::NS), (uint32_t)((t / C::NS) & 1));
+          mbar_wait_drain(bar(BAR_VFULL + t % C::NS), (uint32_t)((t / C::NS) & 1));
       }
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------ MMA issuer
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(384, 1)
         *abort_flag = 1;
         // Drain the tensor pipe before anything is released.
         mma_commit(bar(BAR_DRAIN));
-        mbar_wait(bar(BAR_DRAIN), 0);
+        mbar_wait_drain(bar(BAR_DRAIN), 0);
       }
     }
   } else {

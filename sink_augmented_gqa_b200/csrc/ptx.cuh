@@ -66,6 +66,22 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
+// Bounded wait with a fixed limit (~1 s) that ignores the tunable one: used
+// only to drain work already in flight (TMA copies, queued MMAs) before a CTA
+// that aborted releases its shared or tensor memory. Such work always
+// completes on its own, so this wait never runs out in practice.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try(bar, parity)) return true;
+    if (clock64() - t0 > 2000000000LL) {
+      atomicOr(&g_status, STATUS_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

@@ -1,0 +1,63 @@
+"""Failure detection without faulting the GPU.
+
+Every device-side wait of the library is bounded. With the bound set to zero
+cycles, the waits that are not already satisfied give up at once: the
+kernels record SA_ERR_TIMEOUT in the device status word, drain the copies and
+MMAs they already started, release their memory and return. The host reads
+the status, restores the bound, and the same context keeps computing
+correct results.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import sink_augmented_gqa_b200 as sa
+from sink_augmented_gqa_b200 import workloads as wl
+
+from helpers import check_bf16_output, oracle_cache, oracle_step, oracle_tables
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+DEFAULT_LIMIT = 2_000_000_000
+
+
+def _tables(cfg, max_pos):
+    y = cfg.yarn
+    return sa.yarn_rope_tables(max_pos, cfg.d, y["theta"], y["scaling"], y["orig_ctx"], y["alpha"],
+                               y["beta"], device=DEV)
+
+
+def test_zero_wait_limit_reports_timeout_and_context_survives(cuda_device):
+    cfg = wl.scaled(wl.CONFIGS["tiny"], B=2)
+    off = 3000
+    cap = off + 300
+    cos, sin = _tables(cfg, cap)
+    sinks = wl.sinks(cfg).to(DEV)
+    assert sa.device_status() == "SA_OK"
+    sa.set_wait_limit(0)
+    try:
+        cache = sa.KVCache(cfg.B, cap, cfg.n_kv, cfg.d, device=DEV)
+        kp, vp = wl.prefilled_cache_rows(cfg, rows=off, device=DEV)
+        cache.append(kp, vp)
+        q, k, v = wl.qkv(cfg, 256, device=DEV)
+        sa.attn_prefill(cache, q, k, v, sinks, 0, cfg.sm_scale, cos, sin)
+        qd, kd, vd = wl.qkv(cfg, 1, step=1, device=DEV)
+        sa.attn_decode(cache, qd, kd, vd, sinks, 0, cfg.sm_scale, cos, sin)
+        torch.cuda.synchronize()
+        status = sa.device_status()
+    finally:
+        sa.set_wait_limit(DEFAULT_LIMIT)
+    assert status == "SA_ERR_TIMEOUT"
+    assert sa.device_status() == "SA_OK"          # reading the word clears it
+
+    # The context is intact: a fresh call computes the right answer.
+    rc, rs = oracle_tables(cfg, cap)
+    cache = sa.KVCache(cfg.B, cap, cfg.n_kv, cfg.d, device=DEV)
+    ocache = oracle_cache(cfg.B, cap, cfg.n_kv, cfg.d)
+    q, k, v = wl.qkv(cfg, 200, step=5)
+    out = sa.attn_prefill(cache, q.to(DEV), k.to(DEV), v.to(DEV), sinks, 16, cfg.sm_scale, cos, sin)
+    torch.cuda.synchronize()
+    ref, _ = oracle_step(ocache, q, k, v, sinks.cpu(), 16, cfg.sm_scale, rc, rs)
+    check_bf16_output(out, ref, "after timeout")
+    assert sa.device_status() == "SA_OK"
