@@ -2,9 +2,9 @@
 //
 // The work is reading the KV cache once: for each (sequence b, KV head g)
 // the rows [lo, off) are cut into S contiguous splits, one CTA each
-// (grid n_kv x S x B). Inside a CTA one producer warp streams 64-row K and V
+// (grid n_kv x S x B). Inside a CTA one producer warp streams 128-row K and V
 // tiles of head g from the cache with TMA (128-byte swizzled smem, rows past
-// `off` read as zeros) through a deep ring, and four consumer warps each take
+// `off` read as zeros) through a ring, and eight consumer warps each take
 // 16 rows of every tile. A consumer computes S^T = K Q^T for the q_mult <= 8
 // query heads of the group with mma.sync m16n8k16 (keys are the M side, the
 // heads the N side, so every KV row is read from smem exactly once for the
@@ -15,7 +15,7 @@
 // attended from registers by the CTA of the last split, so no CTA ever reads
 // a cache row written in the same launch.
 //
-// Partials (m, l, O) of the four warps are merged in smem; with S > 1 each
+// Partials (m, l, O) of the eight warps are merged in smem; with S > 1 each
 // CTA writes its partial to the workspace and the last CTA of (b, g) to
 // finish (atomic ticket, no spinning) merges all S of them and folds in the
 // sink: M = max(max_s m_s, sink), l = sum_s e^{m_s-M} l_s + e^{sink-M},
@@ -57,23 +57,27 @@ struct DecodeParams {
 
 template <int D>
 struct DecodeCfg {
-  static constexpr int R = 64;                          // rows per stage
+  static constexpr int NCW = 8;                         // consumer warps
+  static constexpr int R = 16 * NCW;                    // rows per stage (16 per consumer warp)
   static constexpr int CB = (D % 64 == 0) ? 64 : 32;
   static constexpr int SWZ = CB * 2;
   static constexpr int NCB = D / CB;
   static constexpr uint32_t BLOCK_BYTES = R * SWZ;       // one column block of a stage
   static constexpr uint32_t STAGE_BYTES = R * D * 2;     // K (or V) of one stage
-  static constexpr int NS = (D == 64) ? 6 : (D == 96 ? 4 : 3);
+  static constexpr int NS = (D == 64) ? 3 : 2;
   static constexpr uint32_t XBLOCK = 16 * SWZ;           // column block of the new-row tile
   static constexpr uint32_t XTILE = 16 * D * 2;
-  static constexpr int NUM_THREADS = 160;
+  static constexpr int NUM_THREADS = 32 * (NCW + 1);
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_V = NS * STAGE_BYTES;
   static constexpr uint32_t OFF_XK = 2 * NS * STAGE_BYTES;
   static constexpr uint32_t OFF_XV = OFF_XK + XTILE;
-  static constexpr uint32_t OFF_RED = OFF_XV + XTILE;    // [4 warps][8 m | 8 l | 8*D O] fp32
+  // [NCW warps][8 m | 8 l | 8*D O] fp32, aliased over the K ring: written only
+  // after every consumer warp has finished with the ring
+  static constexpr uint32_t OFF_RED = OFF_K;
   static constexpr uint32_t RED_WARP = (16 + 8 * D) * 4;
-  static constexpr uint32_t OFF_BAR = OFF_RED + 4 * RED_WARP;
+  static_assert(NCW * RED_WARP <= 2 * NS * STAGE_BYTES, "warp partials must fit in the ring");
+  static constexpr uint32_t OFF_BAR = OFF_XV + XTILE;
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + 8 * (2 * NS) + 16 + 1024;
 };
 
@@ -132,7 +136,7 @@ __device__ __forceinline__ void decode_subtile(uint32_t kbase, uint32_t vbase, u
 }
 
 template <int D>
-__global__ void __launch_bounds__(160)
+__global__ void __launch_bounds__(288)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecodeParams p) {
   using C = DecodeCfg<D>;
@@ -163,7 +167,7 @@ __global__ void __launch_bounds__(160)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 4);
+      mbar_init(empty_bar(s), C::NCW);
     }
     flag[0] = 0;
     flag[1] = 0;
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(160)
   }
   __syncthreads();
 
-  if (warp == 4) {
+  if (warp == C::NCW) {
     // ------------------------------------------------------------ producer
     if (lane == 0 && n_stages > 0) {
       tma_prefetch_desc(&tmK);
@@ -197,7 +201,7 @@ __global__ void __launch_bounds__(160)
           mbar_wait_drain(full_bar(it % C::NS), (uint32_t)((it / C::NS) & 1));
       }
     }
-    return;  // the producer takes no part in the merge (named barriers below count 128)
+    return;  // the producer takes no part in the merge (named barriers below count 32*NCW)
   }
 
   // ---------------------------------------------------------------- consumers
@@ -290,7 +294,8 @@ __global__ void __launch_bounds__(160)
     decode_subtile<D>(sbase + C::OFF_XK, sbase + C::OFF_XV, C::XBLOCK, 0, 1, qf, p.scale_log2, m, l,
                       o, lane);
 
-  // ---------------------------------------------------------------- merge the 4 warps
+  // ---------------------------------------------------------------- merge the consumer warps
+  named_bar_sync(1, 32 * C::NCW);   // every warp is done reading the K/V ring
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     l[e] += __shfl_xor_sync(0xffffffffu, l[e], 4);
@@ -316,20 +321,21 @@ __global__ void __launch_bounds__(160)
       rw[16 + (2 * t + 1) * D + d0 + 8] = o[md][3];
     }
   }
-  named_bar_sync(1, 128);
+  named_bar_sync(1, 32 * C::NCW);
 
   const float LOG2E = 1.4426950408889634f, LN2 = 0.6931471805599453f;
-  const int tid = threadIdx.x;  // 0..127
+  const int tid = threadIdx.x;  // 0 .. 32*NCW-1
+  constexpr int NT = 32 * C::NCW;
   const long long slot = ((long long)b * p.n_kv + g) * p.S + split;
-  for (int idx = tid; idx < QM * D; idx += 128) {
+  for (int idx = tid; idx < QM * D; idx += NT) {
     const int n = idx / D, d = idx % D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, red[w * (C::RED_WARP / 4) + n]);
+    for (int w = 0; w < C::NCW; ++w) M = fmaxf(M, red[w * (C::RED_WARP / 4) + n]);
     const float Mu = (M == -INFINITY) ? 0.f : M;
     float L = 0.f, O = 0.f;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
+    for (int w = 0; w < C::NCW; ++w) {
       const float* rw = red + w * (C::RED_WARP / 4);
       const float f = ex2(rw[n] - Mu);
       L += rw[8 + n] * f;
@@ -354,12 +360,12 @@ __global__ void __launch_bounds__(160)
   if (p.S == 1) return;
 
   __threadfence();
-  named_bar_sync(1, 128);
+  named_bar_sync(1, NT);
   if (tid == 0) {
     const int ticket = atomicAdd(p.ws_cnt + (b * p.n_kv + g), 1);
     flag[1] = (ticket == p.S - 1) ? 1 : 0;
   }
-  named_bar_sync(1, 128);
+  named_bar_sync(1, NT);
   if (!flag[1]) return;
   __threadfence();
 
@@ -378,29 +384,29 @@ __global__ void __launch_bounds__(160)
     const float* gl = p.ws_l + slot0 * QM;
     const int nml = S * QM;
     int idx = tid;
-    for (; idx + 3 * 128 < nml; idx += 4 * 128) {
+    for (; idx + 3 * NT < nml; idx += 4 * NT) {
       float a[4], c[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        a[j] = __ldcg(gm + idx + j * 128);
-        c[j] = __ldcg(gl + idx + j * 128);
+        a[j] = __ldcg(gm + idx + j * NT);
+        c[j] = __ldcg(gl + idx + j * NT);
       }
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        wsm[idx + j * 128] = a[j];
-        lsm[idx + j * 128] = c[j];
+        wsm[idx + j * NT] = a[j];
+        lsm[idx + j * NT] = c[j];
       }
     }
-    for (; idx < nml; idx += 128) {
+    for (; idx < nml; idx += NT) {
       wsm[idx] = __ldcg(gm + idx);
       lsm[idx] = __ldcg(gl + idx);
     }
   }
-  named_bar_sync(1, 128);
+  named_bar_sync(1, NT);
   {
-    // warp w reduces heads n = w, w + 4, ...: lanes stride over the splits
+    // warp w reduces head n = w (QM <= 8 <= NCW): lanes stride over the splits
     const int w = tid >> 5;
-    for (int n = w; n < QM; n += 4) {
+    for (int n = w; n < QM; n += C::NCW) {
       const int h = g * QM + n;
       const float sink2 = p.sinks ? p.sinks[h] * LOG2E : -INFINITY;
       float M = sink2;
@@ -423,12 +429,12 @@ __global__ void __launch_bounds__(160)
       }
     }
   }
-  named_bar_sync(1, 128);
+  named_bar_sync(1, NT);
   {
     // O = sum_s w_s O_s, four consecutive d per thread, eight splits in flight.
     const int nf4 = QM * D / 4;
     const float4* src0 = reinterpret_cast<const float4*>(p.ws_o + slot0 * QM * D);
-    for (int idx = tid; idx < nf4; idx += 128) {
+    for (int idx = tid; idx < nf4; idx += NT) {
       const int n = (idx * 4) / D, d = (idx * 4) % D;
       const float4* src = src0 + idx;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -203,7 +203,8 @@ DecodeSplit decode_split(int B, int n_kv, long long n_cache) {
   long long S = (target + (long long)B * n_kv - 1) / ((long long)B * n_kv);
   if (S < 1) S = 1;
   long long chunk = (n_cache + S - 1) / S;
-  chunk = ((chunk + 63) / 64) * 64;
+  constexpr long long kStage = 128;   // decode rows per ring stage (DecodeCfg<D>::R)
+  chunk = ((chunk + kStage - 1) / kStage) * kStage;
   r.chunk = chunk;
   r.S = (int)((n_cache + chunk - 1) / chunk);
   return r;
