@@ -1,18 +1,24 @@
 // Flash-style sink-augmented GQA prefill on tcgen05 tensor cores.
 //
-// One CTA owns two 128-row query tiles (A, B) of one (batch, query head) and
-// walks the BN-key tiles of the cache the mask admits for them:
+// A persistent CTA per SM walks work items; an item is two 128-row query
+// tiles (A, B) of one (batch, query head), and the CTA walks the BN-key tiles
+// of the cache the mask admits for them:
 //
-//   warp 0      TMA producer: K and V tiles of the head's KV group, straight
-//               from the head-major cache [B][n_kv][cap][d] (rows past
-//               offset+T read as zeros through the tensor map's bounds),
-//               NS-deep ring each.
-//   warp 1      allocates TMEM and issues every tcgen05.mma from one thread:
+//   warp 0      TMA producer: the item's two Q tiles (already rotated, rows
+//               past T read as zeros) into one of two Q buffers, then the K
+//               and V tiles of the head's KV group, straight from the
+//               head-major cache [B][n_kv][cap][d] (rows past offset+T read as
+//               zeros through the tensor map's bounds), NS-deep ring each.
+//   warps 1, 2  one thread each issues the tcgen05.mma of query tile A (warp
+//               1, which also owns the TMEM allocation) or B (warp 2):
 //               S_X = Q_X K^T (smem x smem, fp32 in TMEM), then
 //               O_X += P_X V with P_X read from its own TMEM columns (bf16).
+//               The two streams are independent: each walks every K/V tile of
+//               the item, multiplies the ones its tile admits and releases the
+//               others at once (the ring slots count one release from each).
+//   warp 3      idle.
 //   warps 4-7   softmax for tile A, warps 8-11 for tile B, one query row per
-//               thread (TMEM lane = row): load + RoPE the Q row into swizzled
-//               smem, then per key tile: read S, release it at once (so the
+//               thread (TMEM lane = row): per key tile: read S, release it at once (so the
 //               tensor core computes the next S while this one is
 //               exponentiated), mask, running max in log2 units, exp2, P ->
 //               TMEM, and at the end O / l -> bf16 out.
@@ -68,7 +74,7 @@ struct PrefillCfg {
   static constexpr uint32_t Q_BYTES = 128u * D * 2;
   static constexpr uint32_t KBLOCK = (uint32_t)BN * SWZ;      // column block of a K/V tile
   static constexpr uint32_t KV_BYTES = (uint32_t)BN * D * 2;
-  static constexpr int NS = 4;                                // K and V ring depth
+  static constexpr int NS = (D == 64) ? 4 : (D == 96 ? 3 : 2);  // K and V ring depth
   static constexpr uint32_t LAYOUT = (SWZ == 128) ? 2u : 4u;
   static constexpr uint32_t SBO = 8u * SWZ;                   // 8-row core-matrix group stride
   static constexpr int TMEM_COLS = 512;
@@ -78,30 +84,51 @@ struct PrefillCfg {
   static_assert(O_COL1 + D <= TMEM_COLS, "TMEM plan exceeds 512 columns");
   static_assert(KBLOCK % 1024 == 0 && QBLOCK % 1024 == 0, "swizzle atoms need 1 KB alignment");
   static constexpr int NUM_THREADS = 384;
-  // smem: Q[2] | K[NS] | V[NS] | barriers
+  // smem: Q[2 buffers][2 tiles] | K[NS] | V[NS] | barriers
   static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = 2 * Q_BYTES;
+  static constexpr uint32_t OFF_K = 4 * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + NS * KV_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_V + NS * KV_BYTES;
-  static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
+  static constexpr uint32_t SMEM_BYTES = OFF_BAR + 512 + 1024;  // + alignment slack
   static constexpr uint32_t IDESC_QK = idesc_bf16(128, BN, 0, 0);
   static constexpr uint32_t IDESC_PV = idesc_bf16(128, D, 0, 1);
 };
 
-// Barrier slots (8 bytes each) at OFF_BAR.
+// Barrier slots (8 bytes each) at OFF_BAR. [2] = one per Q buffer or per
+// query tile X; [NS] = one per K/V ring slot.
 enum : int {
-  BAR_QREADY = 0,  // [2] softmax threads -> MMA: Q tile in smem
-  BAR_SFULL = 2,   // [2] MMA -> softmax: S_X computed
-  BAR_SFREE = 4,   // [2] softmax -> MMA: S_X read into registers
-  BAR_PFULL = 6,   // [2] softmax -> MMA: P_X stored (and O_X rescaled)
-  BAR_ODONE = 8,   // [2] MMA -> softmax: PV_X completed
-  BAR_DRAIN = 10,
-  BAR_KFULL = 11,  // [NS]
-  BAR_KEMPTY = 15, // [NS]
-  BAR_VFULL = 19,  // [NS]
-  BAR_VEMPTY = 23, // [NS]
-  BAR_TMEM_SLOT = 28,
-  BAR_ABORT_SLOT = 29,
+  BAR_QFULL = 0,    // [2 buffers] producer (TMA) -> MMA: an item's Q tiles landed
+  BAR_QEMPTY = 2,   // [2 buffers] MMA A and B -> producer: last S product read them
+  BAR_SFULL = 4,    // [2 tiles] MMA -> softmax: S_X computed
+  BAR_SFREE = 6,    // [2] softmax -> MMA: S_X read into registers
+  BAR_PFULL = 8,    // [2] softmax -> MMA: P_X stored (and O_X rescaled)
+  BAR_ODONE = 10,   // [2] MMA -> softmax: PV_X completed
+  BAR_OFREE = 12,   // [2] softmax -> MMA: the item's epilogue has read O_X
+  BAR_DRAIN = 14,   // [2] per MMA issuer, on abort
+  BAR_KFULL = 16,   // [NS <= 4]
+  BAR_KEMPTY = 20,  // [NS] count 2: MMA A and MMA B
+  BAR_VFULL = 24,   // [NS]
+  BAR_VEMPTY = 28,  // [NS] count 2
+  BAR_TMEM_SLOT = 32,
+  BAR_ABORT_SLOT = 33,
+};
+
+// Work items are (query-tile pair, query head, sequence), heaviest pairs
+// first; CTA c of G takes item r*G + c in even rounds r and r*G + G-1-c in
+// odd ones (a snake, so the heavy and light ends of each round balance).
+struct ItemSchedule {
+  int G, n_items, per_pair, n_pairs, n_q;
+  __device__ __forceinline__ int at(int r) const {
+    const int idx = r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+    return idx < n_items ? idx : -1;
+  }
+  __device__ __forceinline__ int rounds() const { return (n_items + G - 1) / G; }
+  __device__ __forceinline__ void coords(int item, int& pair, int& h, int& b) const {
+    const int rank = item / per_pair, rem = item % per_pair;
+    pair = n_pairs - 1 - rank;
+    h = rem % n_q;
+    b = rem / n_q;
+  }
 };
 
 __device__ __forceinline__ long long floordiv(long long a, long long b) {  // b > 0
@@ -201,8 +228,8 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint6
 
 template <int D>
 __global__ void __launch_bounds__(384, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                   const PrefillParams p) {
+    prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
   using C = PrefillCfg<D>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -216,26 +243,30 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int pair = p.n_pairs - 1 - (int)blockIdx.x;  // heaviest query tiles first
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int g = h / p.q_mult;
-  const TileGeom<BN> geo = make_geom<BN>(p, pair);
+  ItemSchedule sched;
+  sched.G = gridDim.x;
+  sched.per_pair = p.n_q * p.B;
+  sched.n_pairs = p.n_pairs;
+  sched.n_items = p.n_pairs * sched.per_pair;
+  sched.n_q = p.n_q;
+  const int rounds = sched.rounds();
 
   if (threadIdx.x == 0) {
     for (int X = 0; X < 2; ++X) {
-      mbar_init(bar(BAR_QREADY + X), 128);
+      mbar_init(bar(BAR_QFULL + X), 1);
+      mbar_init(bar(BAR_QEMPTY + X), 2);
       mbar_init(bar(BAR_SFULL + X), 1);
       mbar_init(bar(BAR_SFREE + X), 128);
       mbar_init(bar(BAR_PFULL + X), 128);
       mbar_init(bar(BAR_ODONE + X), 1);
+      mbar_init(bar(BAR_OFREE + X), 128);
+      mbar_init(bar(BAR_DRAIN + X), 1);
     }
-    mbar_init(bar(BAR_DRAIN), 1);
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar(BAR_KFULL + s), 1);
-      mbar_init(bar(BAR_KEMPTY + s), 1);
+      mbar_init(bar(BAR_KEMPTY + s), 2);
       mbar_init(bar(BAR_VFULL + s), 1);
-      mbar_init(bar(BAR_VEMPTY + s), 1);
+      mbar_init(bar(BAR_VEMPTY + s), 2);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -245,6 +276,7 @@ __global__ void __launch_bounds__(384, 1)
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
@@ -254,289 +286,304 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp < 4) {
-    // Warpgroup 0: producer (warp 0) and MMA issuer (warp 1); warps 2-3 idle.
-    // It gives registers to the two softmax warpgroups: 128*56 + 256*224 =
-    // 384*168, the launch allocation.
-    regs_dec<56>();
+    // Warpgroup 0: producer (warp 0), MMA issuers (warps 1, 2). It gives
+    // registers to the two softmax warpgroups: 128*72 + 256*216 = 384*168,
+    // the launch allocation.
+    regs_dec<72>();
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------ producer
-      int issued = 0;
-      for (int t = 0; t < geo.ntiles && !*abort_flag; ++t) {
-        const int s = t % C::NS;
-        const uint32_t ph = (uint32_t)((t / C::NS) & 1);
-        const int krow = (int)(geo.base + (long long)BN * t);
-        if (!mbar_wait(bar(BAR_KEMPTY + s), ph ^ 1)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(bar(BAR_KFULL + s), C::KV_BYTES);
+      int gt = 0;  // K/V tiles issued so far (ring position)
+      int j = 0;   // Q loads issued so far
+      for (int rr = 0; rr < rounds && !*abort_flag; ++rr) {
+        const int item = sched.at(rr);
+        if (item < 0) continue;
+        int pair, h, b;
+        sched.coords(item, pair, h, b);
+        const int g = h / p.q_mult;
+        const TileGeom<BN> geo = make_geom<BN>(p, pair);
+        const int qb = j & 1;
+        if (j >= 2 && !mbar_wait(bar(BAR_QEMPTY + qb), (uint32_t)(((j >> 1) - 1) & 1))) {
+          *abort_flag = 1;
+          break;
+        }
+        const int nq = geo.valid(1) ? 2 : 1;
+        mbar_arrive_expect_tx(bar(BAR_QFULL + qb), (uint32_t)nq * C::Q_BYTES);
+        for (int X = 0; X < nq; ++X) {
 #pragma unroll
-        for (int cb = 0; cb < C::NCB; ++cb)
-          tma_load_4d(sbase + C::OFF_K + s * C::KV_BYTES + cb * C::KBLOCK, &tmK, bar(BAR_KFULL + s),
-                      cb * C::CB, krow, g, b);
-        issued = t * 2 + 1;
-        if (!mbar_wait(bar(BAR_VEMPTY + s), ph ^ 1)) { *abort_flag = 1; break; }
-        mbar_arrive_expect_tx(bar(BAR_VFULL + s), C::KV_BYTES);
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_load_4d(sbase + C::OFF_Q + (2 * qb + X) * C::Q_BYTES + cb * C::QBLOCK, &tmQ,
+                        bar(BAR_QFULL + qb), cb * C::CB, geo.i0 + 128 * X, h, b);
+        }
+        ++j;
+        for (int t = 0; t < geo.ntiles; ++t, ++gt) {
+          const int s = gt % C::NS;
+          const uint32_t ph = (uint32_t)((gt / C::NS) & 1);
+          const int krow = (int)(geo.base + (long long)BN * t);
+          if (!mbar_wait(bar(BAR_KEMPTY + s), ph ^ 1)) { *abort_flag = 1; break; }
+          mbar_arrive_expect_tx(bar(BAR_KFULL + s), C::KV_BYTES);
 #pragma unroll
-        for (int cb = 0; cb < C::NCB; ++cb)
-          tma_load_4d(sbase + C::OFF_V + s * C::KV_BYTES + cb * C::KBLOCK, &tmV, bar(BAR_VFULL + s),
-                      cb * C::CB, krow, g, b);
-        issued = t * 2 + 2;
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_load_4d(sbase + C::OFF_K + s * C::KV_BYTES + cb * C::KBLOCK, &tmK, bar(BAR_KFULL + s),
+                        cb * C::CB, krow, g, b);
+          if (!mbar_wait(bar(BAR_VEMPTY + s), ph ^ 1)) {
+            *abort_flag = 1;
+            // K(gt) is in flight, V(gt) is not
+            mbar_wait_drain(bar(BAR_KFULL + s), ph);
+            break;
+          }
+          mbar_arrive_expect_tx(bar(BAR_VFULL + s), C::KV_BYTES);
+#pragma unroll
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_load_4d(sbase + C::OFF_V + s * C::KV_BYTES + cb * C::KBLOCK, &tmV, bar(BAR_VFULL + s),
+                        cb * C::CB, krow, g, b);
+        }
       }
       if (*abort_flag) {
         // Let every copy still in flight land before the CTA can exit.
-        const int nk = (issued + 1) / 2, nv = issued / 2;
-        for (int t = (nk > C::NS ? nk - C::NS : 0); t < nk; ++t)
-          mbar_wait_drain(bar(BAR_KFULL + t % C::NS), (uint32_t)((t / C::NS) & 1));
-        for (int t = (nv > C::NS ? nv - C::NS : 0); t < nv; ++t)
-          mbar_wait_drain(bar(BAR_VFULL + t % C::NS), (uint32_t)((t / C::NS) & 1));
+        for (int u = (gt > C::NS ? gt - C::NS : 0); u < gt; ++u) {
+          mbar_wait_drain(bar(BAR_KFULL + u % C::NS), (uint32_t)((u / C::NS) & 1));
+          mbar_wait_drain(bar(BAR_VFULL + u % C::NS), (uint32_t)((u / C::NS) & 1));
+        }
+        for (int u = (j > 2 ? j - 2 : 0); u < j; ++u)
+          mbar_wait_drain(bar(BAR_QFULL + (u & 1)), (uint32_t)((u >> 1) & 1));
       }
-    } else if (warp == 1 && lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      // Per key tile t: S_A(t), S_B(t) as soon as the softmax released the
-      // previous S; then O_A += P_A(t-1) V(t-1), O_B += P_B(t-1) V(t-1).
+    } else if ((warp == 1 || warp == 2) && lane == 0) {
+      // ------------------------------------------------------------ MMA issuer of tile X
+      // Per key tile t: S_X(t) as soon as the softmax released the previous
+      // S_X; then O_X += P_X(t-1) V(t-1). Tiles outside X's range are only
+      // released. Every wait is bounded; a failed one aborts the CTA.
+      const int X = warp - 1;
+      const uint32_t s_col = tmem + (X ? C::S_COL1 : C::S_COL0);
+      const uint32_t p_col = tmem + (X ? C::P_COL1 : C::P_COL0);
+      const uint32_t o_col = tmem + (X ? C::O_COL1 : C::O_COL0);
+      const uint32_t b_sfull = bar(BAR_SFULL + X), b_sfree = bar(BAR_SFREE + X);
+      const uint32_t b_pfull = bar(BAR_PFULL + X), b_odone = bar(BAR_ODONE + X);
+      const uint32_t b_ofree = bar(BAR_OFREE + X);
       bool ok = true;
-      if (geo.valid(0) && !mbar_wait(bar(BAR_QREADY + 0), 0)) ok = false;
-      if (ok && geo.valid(1) && !mbar_wait(bar(BAR_QREADY + 1), 0)) ok = false;
-      tc_fence_after();
-      const uint64_t qdA = smem_desc(sbase + C::OFF_Q, 16, C::SBO, C::LAYOUT);
-      const uint64_t qdB = smem_desc(sbase + C::OFF_Q + C::Q_BYTES, 16, C::SBO, C::LAYOUT);
       const uint64_t kd0 = smem_desc(sbase + C::OFF_K, 16, C::SBO, C::LAYOUT);
       const uint64_t vd0 = smem_desc(sbase + C::OFF_V, C::KBLOCK, C::SBO, C::LAYOUT);
-      const int a0lo = geo.a_lo[0], a0hi = geo.a_hi[0], a1lo = geo.a_lo[1], a1hi = geo.a_hi[1];
-      int nS0 = 0, nS1 = 0, nP0 = 0, nP1 = 0;
-      int ks = 0, kph = 0;                  // ring slot / phase of K(t)
-      int vs = C::NS - 1, vph = 1;          // ring slot / phase of V(t-1)
-      for (int t = 0; t <= geo.ntiles && ok; ++t) {
-        if (t < geo.ntiles) {
-          if (!mbar_wait(bar(BAR_KFULL + ks), (uint32_t)kph)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t kd = kd0 + ((uint32_t)(ks * C::KV_BYTES) >> 4);
-          if (t >= a0lo && t < a0hi) {
-            if (nS0 > 0 && !mbar_wait(bar(BAR_SFREE + 0), (uint32_t)((nS0 - 1) & 1))) { ok = false; break; }
-            tc_fence_after();
-            issue_qk<D>(tmem + C::S_COL0, qdA, kd);
-            mma_commit(bar(BAR_SFULL + 0));
-            ++nS0;
+      int nS = 0, nP = 0;  // cumulative S products / PV products of this tile
+      int gt = 0;          // ring position of K(0) of the current item
+      int j = 0;           // items done by this CTA
+      for (int rr = 0; rr < rounds && ok; ++rr) {
+        const int item = sched.at(rr);
+        if (item < 0) continue;
+        int pair, h, b;
+        sched.coords(item, pair, h, b);
+        const TileGeom<BN> geo = make_geom<BN>(p, pair);
+        const int qb = j & 1;
+        if (!mbar_wait(bar(BAR_QFULL + qb), (uint32_t)((j >> 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t qd = smem_desc(sbase + C::OFF_Q + (2 * qb + X) * C::Q_BYTES, 16, C::SBO, C::LAYOUT);
+        const int lo = X ? geo.a_lo[1] : geo.a_lo[0], hi = X ? geo.a_hi[1] : geo.a_hi[0];
+        if (hi <= lo) mbar_arrive(bar(BAR_QEMPTY + qb));   // this tile reads no Q
+        bool first = true;                                  // no PV of this item issued yet
+        for (int t = 0; t <= geo.ntiles; ++t) {
+          if (t < geo.ntiles) {
+            const int u = gt + t;
+            const int ks = u % C::NS;
+            if (!mbar_wait(bar(BAR_KFULL + ks), (uint32_t)((u / C::NS) & 1))) { ok = false; break; }
+            if (t >= lo && t < hi) {
+              if (nS > 0 && !mbar_wait(b_sfree, (uint32_t)((nS - 1) & 1))) { ok = false; break; }
+              tc_fence_after();
+              issue_qk<D>(s_col, qd, kd0 + ((uint32_t)(ks * C::KV_BYTES) >> 4));
+              mma_commit(b_sfull);
+              ++nS;
+              if (t == hi - 1) mma_commit(bar(BAR_QEMPTY + qb));   // last read of this Q tile
+              mma_commit(bar(BAR_KEMPTY + ks));
+            } else {
+              mbar_arrive(bar(BAR_KEMPTY + ks));
+            }
           }
-          if (t >= a1lo && t < a1hi) {
-            if (nS1 > 0 && !mbar_wait(bar(BAR_SFREE + 1), (uint32_t)((nS1 - 1) & 1))) { ok = false; break; }
-            tc_fence_after();
-            issue_qk<D>(tmem + C::S_COL1, qdB, kd);
-            mma_commit(bar(BAR_SFULL + 1));
-            ++nS1;
+          if (t > 0) {
+            const int u = gt + t - 1;
+            const int vs = u % C::NS;
+            if (!mbar_wait(bar(BAR_VFULL + vs), (uint32_t)((u / C::NS) & 1))) { ok = false; break; }
+            if (t - 1 >= lo && t - 1 < hi) {
+              if (first && j > 0 && !mbar_wait(b_ofree, (uint32_t)((j - 1) & 1))) { ok = false; break; }
+              if (!mbar_wait(b_pfull, (uint32_t)(nP & 1))) { ok = false; break; }
+              tc_fence_after();
+              issue_pv<D>(o_col, p_col, vd0 + ((uint32_t)(vs * C::KV_BYTES) >> 4), !first);
+              mma_commit(b_odone);
+              ++nP;
+              first = false;
+              mma_commit(bar(BAR_VEMPTY + vs));
+            } else {
+              mbar_arrive(bar(BAR_VEMPTY + vs));
+            }
           }
-          mma_commit(bar(BAR_KEMPTY + ks));
+          if (*abort_flag) { ok = false; break; }
         }
-        if (t > 0) {
-          if (!mbar_wait(bar(BAR_VFULL + vs), (uint32_t)vph)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t vd = vd0 + ((uint32_t)(vs * C::KV_BYTES) >> 4);
-          if (t - 1 >= a0lo && t - 1 < a0hi) {
-            if (!mbar_wait(bar(BAR_PFULL + 0), (uint32_t)(nP0 & 1))) { ok = false; break; }
-            tc_fence_after();
-            issue_pv<D>(tmem + C::O_COL0, tmem + C::P_COL0, vd, nP0 > 0);
-            mma_commit(bar(BAR_ODONE + 0));
-            ++nP0;
-          }
-          if (t - 1 >= a1lo && t - 1 < a1hi) {
-            if (!mbar_wait(bar(BAR_PFULL + 1), (uint32_t)(nP1 & 1))) { ok = false; break; }
-            tc_fence_after();
-            issue_pv<D>(tmem + C::O_COL1, tmem + C::P_COL1, vd, nP1 > 0);
-            mma_commit(bar(BAR_ODONE + 1));
-            ++nP1;
-          }
-          mma_commit(bar(BAR_VEMPTY + vs));
-        }
-        // advance the ring positions: K(t+1), V(t)
-        vs = ks;
-        vph = kph;
-        if (++ks == C::NS) { ks = 0; kph ^= 1; }
-        if (*abort_flag) { ok = false; break; }
+        gt += geo.ntiles;
+        ++j;
       }
       if (!ok) {
         *abort_flag = 1;
-        // Drain the tensor pipe before anything is released.
-        mma_commit(bar(BAR_DRAIN));
-        mbar_wait_drain(bar(BAR_DRAIN), 0);
+        // Drain this issuer's tensor-core work before anything is released.
+        mma_commit(bar(BAR_DRAIN + X));
+        mbar_wait_drain(bar(BAR_DRAIN + X), 0);
       }
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    regs_inc<224>();
+    regs_inc<216>();
     const int X = (warp - 4) >> 2;
     const int quarter = warp & 3;               // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;          // row within the query tile
-    const int i = geo.i0 + 128 * X + r;         // query row within the call
-    const bool row_ok = i < p.T;
-    const long long pos = p.off + i;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_tm = tmem + lane_base + (X ? C::S_COL1 : C::S_COL0);
     const uint32_t p_tm = tmem + lane_base + (X ? C::P_COL1 : C::P_COL0);
     const uint32_t o_tm = tmem + lane_base + (X ? C::O_COL1 : C::O_COL0);
-
-    if (geo.valid(X)) {
-      // Q row -> (RoPE) -> bf16 -> swizzled smem, K-major for the MMA.
-      uint8_t* qtile = smem + C::OFF_Q + X * C::Q_BYTES;
-      if (row_ok) {
-        const __nv_bfloat16* qrow = p.q + b * p.qs0 + (long long)i * p.qs1 + (long long)h * p.qs2;
-        constexpr int HALF = D / 2;
-#pragma unroll
-        for (int ch = 0; ch < HALF / 8; ++ch) {
-          uint4 a = *reinterpret_cast<const uint4*>(qrow + ch * 8);
-          uint4 c = *reinterpret_cast<const uint4*>(qrow + HALF + ch * 8);
-          if (p.rope) {
-            const float4 c0 = *reinterpret_cast<const float4*>(p.cos_t + pos * HALF + ch * 8);
-            const float4 c1 = *reinterpret_cast<const float4*>(p.cos_t + pos * HALF + ch * 8 + 4);
-            const float4 s0 = *reinterpret_cast<const float4*>(p.sin_t + pos * HALF + ch * 8);
-            const float4 s1 = *reinterpret_cast<const float4*>(p.sin_t + pos * HALF + ch * 8 + 4);
-            rope_pair2(a.x, c.x, c0.x, c0.y, s0.x, s0.y);
-            rope_pair2(a.y, c.y, c0.z, c0.w, s0.z, s0.w);
-            rope_pair2(a.z, c.z, c1.x, c1.y, s1.x, s1.y);
-            rope_pair2(a.w, c.w, c1.z, c1.w, s1.z, s1.w);
-          }
-          *reinterpret_cast<uint4*>(qtile + swz_off<C::CB>(r, ch * 8, C::QBLOCK)) = a;
-          *reinterpret_cast<uint4*>(qtile + swz_off<C::CB>(r, HALF + ch * 8, C::QBLOCK)) = c;
-        }
-      } else {
-        const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int ch = 0; ch < D / 8; ++ch)
-          *reinterpret_cast<uint4*>(qtile + swz_off<C::CB>(r, ch * 8, C::QBLOCK)) = z;
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar(BAR_QREADY + X));
-
-      const float LOG2E = 1.4426950408889634f;
-      const float scale = p.scale_log2;
-      const float sink2 = p.sinks ? p.sinks[h] * LOG2E : -INFINITY;
-      float m = sink2;                              // running max (log2 units)
-      float l = (sink2 == -INFINITY) ? 0.f : 1.f;   // running sum, sink included
-      int n = 0;
-      bool ok = true;
-      const int t_lo = X ? geo.a_lo[1] : geo.a_lo[0], t_hi = X ? geo.a_hi[1] : geo.a_hi[0];
-      const int full_lo = X ? geo.f_lo[1] : geo.f_lo[0], full_hi = X ? geo.f_hi[1] : geo.f_hi[0];
-      for (int t = t_lo; t < t_hi; ++t) {
-        if (!mbar_wait(bar(BAR_SFULL + X), (uint32_t)(n & 1))) { ok = false; *abort_flag = 1; break; }
-        tc_fence_after();
-        uint32_t sr[BN];
-#pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += 32)
-          tmem_ld32(s_tm + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[c0]));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(BAR_SFREE + X));   // the tensor core may overwrite S_X now
-        if (t < full_lo || t >= full_hi) {
-          // admitted columns c (key klo + c): c >= cmin and c <= cmax
-          const long long klo = geo.base + (long long)BN * t;
-          long long lo_k = 0;
-          if (p.window > 0 && pos - p.window + 1 > lo_k) lo_k = pos - p.window + 1;
-          const long long cmin = lo_k - klo, cmax = pos - klo;
-          const int cmin_i = (int)(cmin < -1 ? -1 : (cmin > BN ? BN : cmin));
-          const int cmax_i = (int)(cmax < -1 ? -1 : (cmax > BN ? BN : cmax));
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c < cmin_i || c > cmax_i) sr[c] = __float_as_uint(-INFINITY);
-        }
-        // raw row max (scale > 0, so max(s * scale) = scale * max(s))
-        float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < BN; c += 8) {
-          m0 = max3f(m0, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
-          m1 = max3f(m1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
-          m2 = max3f(m2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
-          m3 = max3f(m3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
-        }
-        const float mx = fmaxf(max3f(m0, m1, m2), m3) * scale;
-        const float m_new = fmaxf(m, mx);
-        const bool need = m_new > m + 8.0f;
-        bool pv_done = (n == 0);
-        if (__any_sync(0xffffffffu, need)) {
-          const float f = need ? ex2(m - m_new) : 1.0f;
-          if (n > 0) {
-            // O_X may only be touched once the previous PV_X has landed.
-            if (!mbar_wait(bar(BAR_ODONE + X), (uint32_t)((n - 1) & 1))) { ok = false; *abort_flag = 1; break; }
-            tc_fence_after();
-            pv_done = true;
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16) {
-              uint32_t rr[16];
-              tmem_ld16(o_tm + c0, rr);
-              tmem_wait_ld();
-#pragma unroll
-              for (int c = 0; c < 16; c += 2) {
-                float a0 = __uint_as_float(rr[c]), a1 = __uint_as_float(rr[c + 1]);
-                mul2(a0, a1, f, f);
-                rr[c] = __float_as_uint(a0);
-                rr[c + 1] = __float_as_uint(a1);
-              }
-              tmem_st16(o_tm + c0, rr);
-            }
-          }
-          if (need) {
-            l *= f;
-            m = m_new;
-          }
-        }
-        const float neg = (m == -INFINITY) ? 0.f : -m;
-        uint32_t pk[BN / 2];
-        float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-#pragma unroll
-        for (int c = 0; c < BN / 2; c += 2) {
-          float x0, x1, x2, x3;
-          fma2(x0, x1, __uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]), scale, scale, neg, neg);
-          fma2(x2, x3, __uint_as_float(sr[2 * c + 2]), __uint_as_float(sr[2 * c + 3]), scale, scale, neg, neg);
-          x0 = ex2(x0);
-          x1 = ex2(x1);
-          x2 = ex2(x2);
-          x3 = ex2(x3);
-          add2(l0, l1, x0, x1);
-          add2(l2, l3, x2, x3);
-          pk[c] = pack_bf16(x0, x1);
-          pk[c + 1] = pack_bf16(x2, x3);
-        }
-        l += (l0 + l1) + (l2 + l3);
-        // P_X is read by the previous PV_X until it completes.
-        if (!pv_done) {
-          if (!mbar_wait(bar(BAR_ODONE + X), (uint32_t)((n - 1) & 1))) { ok = false; *abort_flag = 1; break; }
+    const float LOG2E = 1.4426950408889634f;
+    const float scale = p.scale_log2;
+    int ntot = 0;   // cumulative key tiles of this query tile slot (S / P / O-done phases)
+    bool ok = true;
+    for (int rr = 0; rr < rounds && ok; ++rr) {
+      const int item = sched.at(rr);
+      if (item < 0) continue;
+      int pair, h, b;
+      sched.coords(item, pair, h, b);
+      const TileGeom<BN> geo = make_geom<BN>(p, pair);
+      const int i = geo.i0 + 128 * X + r;       // query row within the call
+      const bool row_ok = i < p.T;
+      const long long pos = p.off + i;
+      if (geo.valid(X)) {
+        const float sink2 = p.sinks ? p.sinks[h] * LOG2E : -INFINITY;
+        float m = sink2;                              // running max (log2 units)
+        float l = (sink2 == -INFINITY) ? 0.f : 1.f;   // running sum, sink included
+        int n = 0;                                    // key tiles of this item
+        const int t_lo = X ? geo.a_lo[1] : geo.a_lo[0], t_hi = X ? geo.a_hi[1] : geo.a_hi[0];
+        const int full_lo = X ? geo.f_lo[1] : geo.f_lo[0], full_hi = X ? geo.f_hi[1] : geo.f_hi[0];
+        for (int t = t_lo; t < t_hi; ++t) {
+          if (!mbar_wait(bar(BAR_SFULL + X), (uint32_t)(ntot & 1))) { ok = false; *abort_flag = 1; break; }
           tc_fence_after();
-        }
+          uint32_t sr[BN];
 #pragma unroll
-        for (int c0 = 0; c0 + 32 <= BN / 2; c0 += 32)
-          tmem_st32(p_tm + c0, *reinterpret_cast<uint32_t(*)[32]>(&pk[c0]));
-        if constexpr ((BN / 2) % 32 == 16) tmem_st16(p_tm + (BN / 2 - 16), &pk[BN / 2 - 16]);
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(BAR_PFULL + X));
-        ++n;
-        if (*abort_flag) { ok = false; break; }
-      }
-      // Epilogue: O / l -> bf16, once the last PV_X has landed.
-      if (n > 0 && mbar_wait(bar(BAR_ODONE + X), (uint32_t)((n - 1) & 1)) && ok && !*abort_flag) {
-        tc_fence_after();
-        const float inv_l = 1.0f / l;
-        __nv_bfloat16* orow = p.out + b * p.os0 + (long long)i * p.os1 + (long long)h * p.os2;
-#pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t rr[32];
-          tmem_ld32(o_tm + c0, rr);
+          for (int c0 = 0; c0 < BN; c0 += 32)
+            tmem_ld32(s_tm + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[c0]));
           tmem_wait_ld();
-          if (row_ok) {
+          tc_fence_before();
+          mbar_arrive(bar(BAR_SFREE + X));   // the tensor core may overwrite S_X now
+          if (t < full_lo || t >= full_hi) {
+            // admitted columns c (key klo + c): c >= cmin and c <= cmax
+            const long long klo = geo.base + (long long)BN * t;
+            long long lo_k = 0;
+            if (p.window > 0 && pos - p.window + 1 > lo_k) lo_k = pos - p.window + 1;
+            const long long cmin = lo_k - klo, cmax = pos - klo;
+            const int cmin_i = (int)(cmin < -1 ? -1 : (cmin > BN ? BN : cmin));
+            const int cmax_i = (int)(cmax < -1 ? -1 : (cmax > BN ? BN : cmax));
 #pragma unroll
-            for (int c = 0; c < 32; c += 8) {
-              uint4 v;
-              v.x = pack_bf16(__uint_as_float(rr[c + 0]) * inv_l, __uint_as_float(rr[c + 1]) * inv_l);
-              v.y = pack_bf16(__uint_as_float(rr[c + 2]) * inv_l, __uint_as_float(rr[c + 3]) * inv_l);
-              v.z = pack_bf16(__uint_as_float(rr[c + 4]) * inv_l, __uint_as_float(rr[c + 5]) * inv_l);
-              v.w = pack_bf16(__uint_as_float(rr[c + 6]) * inv_l, __uint_as_float(rr[c + 7]) * inv_l);
-              *reinterpret_cast<uint4*>(orow + c0 + c) = v;
+            for (int c = 0; c < BN; ++c)
+              if (c < cmin_i || c > cmax_i) sr[c] = __float_as_uint(-INFINITY);
+          }
+          // raw row max (scale > 0, so max(s * scale) = scale * max(s))
+          float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < BN; c += 8) {
+            m0 = max3f(m0, __uint_as_float(sr[c + 0]), __uint_as_float(sr[c + 1]));
+            m1 = max3f(m1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+            m2 = max3f(m2, __uint_as_float(sr[c + 4]), __uint_as_float(sr[c + 5]));
+            m3 = max3f(m3, __uint_as_float(sr[c + 6]), __uint_as_float(sr[c + 7]));
+          }
+          const float mx = fmaxf(max3f(m0, m1, m2), m3) * scale;
+          const float m_new = fmaxf(m, mx);
+          const bool need = m_new > m + 8.0f;
+          bool pv_done = (ntot == 0);
+          if (__any_sync(0xffffffffu, need)) {
+            const float f = need ? ex2(m - m_new) : 1.0f;
+            if (n > 0) {
+              // O_X may only be touched once the previous PV_X has landed.
+              if (!mbar_wait(bar(BAR_ODONE + X), (uint32_t)((ntot - 1) & 1))) { ok = false; *abort_flag = 1; break; }
+              tc_fence_after();
+              pv_done = true;
+#pragma unroll 1
+              for (int c0 = 0; c0 < D; c0 += 16) {
+                uint32_t rr16[16];
+                tmem_ld16(o_tm + c0, rr16);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 16; c += 2) {
+                  float a0 = __uint_as_float(rr16[c]), a1 = __uint_as_float(rr16[c + 1]);
+                  mul2(a0, a1, f, f);
+                  rr16[c] = __float_as_uint(a0);
+                  rr16[c + 1] = __float_as_uint(a1);
+                }
+                tmem_st16(o_tm + c0, rr16);
+              }
+            }
+            if (need) {
+              l *= f;
+              m = m_new;
             }
           }
+          const float neg = (m == -INFINITY) ? 0.f : -m;
+          uint32_t pk[BN / 2];
+          float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
+#pragma unroll
+          for (int c = 0; c < BN / 2; c += 2) {
+            float x0, x1, x2, x3;
+            fma2(x0, x1, __uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]), scale, scale, neg, neg);
+            fma2(x2, x3, __uint_as_float(sr[2 * c + 2]), __uint_as_float(sr[2 * c + 3]), scale, scale, neg, neg);
+            x0 = ex2(x0);
+            x1 = ex2(x1);
+            x2 = ex2(x2);
+            x3 = ex2(x3);
+            add2(l0, l1, x0, x1);
+            add2(l2, l3, x2, x3);
+            pk[c] = pack_bf16(x0, x1);
+            pk[c + 1] = pack_bf16(x2, x3);
+          }
+          l += (l0 + l1) + (l2 + l3);
+          // P_X is read by the previous PV_X until it completes.
+          if (!pv_done) {
+            if (!mbar_wait(bar(BAR_ODONE + X), (uint32_t)((ntot - 1) & 1))) { ok = false; *abort_flag = 1; break; }
+            tc_fence_after();
+          }
+#pragma unroll
+          for (int c0 = 0; c0 + 32 <= BN / 2; c0 += 32)
+            tmem_st32(p_tm + c0, *reinterpret_cast<uint32_t(*)[32]>(&pk[c0]));
+          if constexpr ((BN / 2) % 32 == 16) tmem_st16(p_tm + (BN / 2 - 16), &pk[BN / 2 - 16]);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(BAR_PFULL + X));
+          ++n;
+          ++ntot;
+          if (*abort_flag) { ok = false; break; }
         }
-        if (row_ok && p.lse) {
-          const float LN2 = 0.6931471805599453f;
-          p.lse[((long long)b * p.n_q + h) * p.T + i] = (m + __log2f(l)) * LN2;
+        // Epilogue: O / l -> bf16, once the item's last PV_X has landed.
+        if (ok && n > 0 && mbar_wait(bar(BAR_ODONE + X), (uint32_t)((ntot - 1) & 1)) && !*abort_flag) {
+          tc_fence_after();
+          const float inv_l = 1.0f / l;
+          __nv_bfloat16* orow = p.out + b * p.os0 + (long long)i * p.os1 + (long long)h * p.os2;
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o32[32];
+            tmem_ld32(o_tm + c0, o32);
+            tmem_wait_ld();
+            if (row_ok) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 8) {
+                uint4 v;
+                v.x = pack_bf16(__uint_as_float(o32[c + 0]) * inv_l, __uint_as_float(o32[c + 1]) * inv_l);
+                v.y = pack_bf16(__uint_as_float(o32[c + 2]) * inv_l, __uint_as_float(o32[c + 3]) * inv_l);
+                v.z = pack_bf16(__uint_as_float(o32[c + 4]) * inv_l, __uint_as_float(o32[c + 5]) * inv_l);
+                v.w = pack_bf16(__uint_as_float(o32[c + 6]) * inv_l, __uint_as_float(o32[c + 7]) * inv_l);
+                *reinterpret_cast<uint4*>(orow + c0 + c) = v;
+              }
+            }
+          }
+          if (row_ok && p.lse) {
+            const float LN2 = 0.6931471805599453f;
+            p.lse[((long long)b * p.n_q + h) * p.T + i] = (m + __log2f(l)) * LN2;
+          }
+        } else if (!ok || *abort_flag) {
+          ok = false;
+          *abort_flag = 1;
         }
-      } else if (!ok) {
-        *abort_flag = 1;
       }
+      // O_X is free for the next item's first PV.
+      tc_fence_before();
+      mbar_arrive(bar(BAR_OFREE + X));
     }
   }
 

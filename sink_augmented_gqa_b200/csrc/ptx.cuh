@@ -368,24 +368,66 @@ __device__ __forceinline__ uint32_t bf16_bits_from_f64(double x) {
   return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
-// One RoPE pair: (x1, x2) -> (x1 c - x2 s, x2 c + x1 s). The bf16 x fp32
-// products are exact in fp64, so each result carries one fp64 rounding and
-// is then rounded once more to bf16 -- the same value an fp64 evaluation of
-// the formula rounds to.
-__device__ __forceinline__ void rope_pair(float x1, float x2, float c, float s, uint32_t& y1,
-                                          uint32_t& y2) {
+// One RoPE pair: (x1, x2) -> (x1 c - x2 s, x2 c + x1 s), each result the
+// bf16 round-to-nearest-even of the exact value. The bf16 x fp32 products are
+// exact in fp64, so an fp64 evaluation carries one fp64 rounding and is then
+// rounded once more to bf16 (rope_pair_f64). The fast path evaluates in fp32
+// and keeps the result only where the fp32 error bound proves that the exact
+// value lies in the same bf16 rounding cell (rope_fast_ok); elsewhere (about
+// one element in 2^14, and zeros) it falls back to fp64.
+__device__ __forceinline__ void rope_pair_f64(float x1, float x2, float c, float s, uint32_t& y1,
+                                              uint32_t& y2) {
   const double a = (double)x1, b = (double)x2, cd = (double)c, sd = (double)s;
   y1 = bf16_bits_from_f64(a * cd - b * sd);
   y2 = bf16_bits_from_f64(b * cd + a * sd);
 }
+
+// v = RN32(x c -+ t) with t = RN32(y s) differs from the exact x c -+ y s by at
+// most 2^-24 (|v| + |t|)(1 + 2^-22) (one relative rounding in each of the two
+// operations; |v| >= 2^-100 keeps both away from the subnormal range, where
+// the bound is absolute and below 2^-149). e below is twice that bound. The
+// bf16 rounding of a value changes only at the midpoints between adjacent
+// bf16 numbers; the midpoint inside v's bf16 interval is v's bit pattern with
+// the low 16 bits set to 0x8000 (same sign and binade, so v - mid is exact),
+// and every other midpoint is at least |v| 2^-10 away. With both distances
+// above e, v and the exact value round to the same bf16.
+__device__ __forceinline__ bool rope_fast_ok(float v, float t) {
+  const float av = fabsf(v);
+  const float e = (av + fabsf(t)) * 0x1p-23f;
+  const float mid = __uint_as_float((__float_as_uint(v) & 0xFFFF0000u) | 0x8000u);
+  return (fabsf(v - mid) > e) & (av * 0x1p-10f > e) & (av >= 0x1p-100f);
+}
+
+__device__ __forceinline__ void rope_pair(float x1, float x2, float c, float s, uint32_t& y1,
+                                          uint32_t& y2) {
+  const float t1 = __fmul_rn(x2, s), t2 = __fmul_rn(x1, s);
+  const float v1 = __fmaf_rn(x1, c, -t1), v2 = __fmaf_rn(x2, c, t2);
+  if (rope_fast_ok(v1, t1) & rope_fast_ok(v2, t2)) {
+    y1 = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v1));
+    y2 = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v2));
+  } else {
+    rope_pair_f64(x1, x2, c, s, y1, y2);
+  }
+}
+
 // Two adjacent pairs packed as bf16x2 words (low half = lower index).
 __device__ __forceinline__ void rope_pair2(uint32_t& w1, uint32_t& w2, float c0, float c1, float s0,
                                            float s1) {
-  uint32_t a0, a1, b0, b1;
-  rope_pair(bf16_lo(w1), bf16_lo(w2), c0, s0, a0, b0);
-  rope_pair(bf16_hi(w1), bf16_hi(w2), c1, s1, a1, b1);
-  w1 = a0 | (a1 << 16);
-  w2 = b0 | (b1 << 16);
+  const float a0 = bf16_lo(w1), a1 = bf16_hi(w1), b0 = bf16_lo(w2), b1 = bf16_hi(w2);
+  const float t0 = __fmul_rn(b0, s0), t1 = __fmul_rn(b1, s1);
+  const float u0 = __fmul_rn(a0, s0), u1 = __fmul_rn(a1, s1);
+  const float v0 = __fmaf_rn(a0, c0, -t0), v1 = __fmaf_rn(a1, c1, -t1);
+  const float z0 = __fmaf_rn(b0, c0, u0), z1 = __fmaf_rn(b1, c1, u1);
+  if (rope_fast_ok(v0, t0) & rope_fast_ok(v1, t1) & rope_fast_ok(z0, u0) & rope_fast_ok(z1, u1)) {
+    w1 = pack_bf16(v0, v1);
+    w2 = pack_bf16(z0, z1);
+  } else {
+    uint32_t p0, p1, q0, q1;
+    rope_pair_f64(a0, b0, c0, s0, p0, q0);
+    rope_pair_f64(a1, b1, c1, s1, p1, q1);
+    w1 = p0 | (p1 << 16);
+    w2 = q0 | (q1 << 16);
+  }
 }
 
 // Byte offset of element (row, col) in a tile stored as column blocks of

@@ -39,7 +39,7 @@ __global__ void yarn_tables_kernel(float* __restrict__ cos_out, float* __restric
 }
 
 // Rotate 8 consecutive pairs (x1[c..c+7], x2[c..c+7]) with fp32 tables
-// (arithmetic in fp64, one rounding to bf16; see rope_pair).
+// (each result the correctly rounded bf16 of the exact rotation; see rope_pair).
 __device__ __forceinline__ void rotate8(uint4& a, uint4& b, const float* __restrict__ cs,
                                        const float* __restrict__ sn) {
   uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
@@ -111,6 +111,63 @@ __global__ void kv_append_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat16* 
     *reinterpret_cast<uint4*>(cv + dst + ch * 8) = *reinterpret_cast<const uint4*>(vrow + ch * 8);
     *reinterpret_cast<uint4*>(cv + dst + half + ch * 8) =
         *reinterpret_cast<const uint4*>(vrow + half + ch * 8);
+  }
+}
+
+// Prefill staging, one launch: the kv_append_kernel work for the call's K/V
+// rows, then (stage_q) each query row rotated at its position off + t into
+// qo [B][T][n_q][d] (strides os*), from which the attention kernel reads its
+// query tiles. One thread per (row, 8-pair chunk); K/V units first.
+__global__ void prefill_stage_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat16* __restrict__ cv,
+                                     int cap, const __nv_bfloat16* __restrict__ k, long long ks0,
+                                     long long ks1, long long ks2, const __nv_bfloat16* __restrict__ v,
+                                     long long vs0, long long vs1, long long vs2, int B, int T,
+                                     int n_kv, int d, long long off, int rope,
+                                     const float* __restrict__ cos_t, const float* __restrict__ sin_t,
+                                     const __nv_bfloat16* q, long long qs0, long long qs1,
+                                     long long qs2, int n_q, __nv_bfloat16* qo, long long os0,
+                                     long long os1, long long os2, int stage_q) {
+  const int half = d / 2, chunks = half / 8;
+  const long long n_kv_units = (long long)B * T * n_kv * chunks;
+  const long long n = n_kv_units + (stage_q ? (long long)B * T * n_q * chunks : 0);
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+       idx += (long long)gridDim.x * blockDim.x) {
+    if (idx < n_kv_units) {
+      const int ch = (int)(idx % chunks);
+      long long r = idx / chunks;
+      const int g = (int)(r % n_kv);
+      r /= n_kv;
+      const int t = (int)(r % T);
+      const int b = (int)(r / T);
+      const __nv_bfloat16* krow = k + b * ks0 + t * ks1 + g * ks2;
+      const __nv_bfloat16* vrow = v + b * vs0 + t * vs1 + g * vs2;
+      uint4 a = *reinterpret_cast<const uint4*>(krow + ch * 8);
+      uint4 c = *reinterpret_cast<const uint4*>(krow + half + ch * 8);
+      const long long p = off + t;
+      if (rope) rotate8(a, c, cos_t + p * half + ch * 8, sin_t + p * half + ch * 8);
+      const long long dst = (((long long)b * n_kv + g) * cap + p) * d;
+      *reinterpret_cast<uint4*>(ck + dst + ch * 8) = a;
+      *reinterpret_cast<uint4*>(ck + dst + half + ch * 8) = c;
+      *reinterpret_cast<uint4*>(cv + dst + ch * 8) = *reinterpret_cast<const uint4*>(vrow + ch * 8);
+      *reinterpret_cast<uint4*>(cv + dst + half + ch * 8) =
+          *reinterpret_cast<const uint4*>(vrow + half + ch * 8);
+    } else {
+      const long long iq = idx - n_kv_units;
+      const int ch = (int)(iq % chunks);
+      long long r = iq / chunks;
+      const int h = (int)(r % n_q);
+      r /= n_q;
+      const int t = (int)(r % T);
+      const int b = (int)(r / T);
+      const __nv_bfloat16* qrow = q + b * qs0 + t * qs1 + h * qs2;
+      __nv_bfloat16* orow = qo + b * os0 + t * os1 + h * os2;
+      uint4 a = *reinterpret_cast<const uint4*>(qrow + ch * 8);
+      uint4 c = *reinterpret_cast<const uint4*>(qrow + half + ch * 8);
+      const long long p = off + t;
+      if (rope) rotate8(a, c, cos_t + p * half + ch * 8, sin_t + p * half + ch * 8);
+      *reinterpret_cast<uint4*>(orow + ch * 8) = a;
+      *reinterpret_cast<uint4*>(orow + half + ch * 8) = c;
+    }
   }
 }
 

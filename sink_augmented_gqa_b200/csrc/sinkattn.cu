@@ -84,6 +84,25 @@ bool make_cache_map(CUtensorMap* map, void* base, int d, int n_kv, long long row
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over a strided [B][T][H][d] bf16 activation (inner dim
+// contiguous, other strides in elements, multiples of 8): dims {d, T, H, B},
+// box {CB, 128, 1, 1} -- one 128-row query tile of one head per CB-wide
+// column block; rows past T read as zeros.
+bool make_rows_map(CUtensorMap* map, const void* base, int d, int T, int H, int B,
+                   const int64_t st[3], int cb) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || T < 1) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)H, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)st[1] * 2, (cuuint64_t)st[2] * 2, (cuuint64_t)st[0] * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)cb, 128, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         cb == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 sa_status last_launch_status() {
   return cudaGetLastError() == cudaSuccess ? SA_OK : SA_ERR_CUDA;
 }
@@ -150,8 +169,14 @@ void set_smem(K kernel, uint32_t bytes) {
 template <int D>
 sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream_t stream) {
   using Cfg = PrefillCfg<D>;
-  CUtensorMap tmK, tmV;
+  CUtensorMap tmQ, tmK, tmV;
   const long long rows = a->offset + a->T;
+  // Query tiles come from the staged (rotated) copy in `out` when RoPE is
+  // fused, else straight from q; the kernel overwrites each staged tile with
+  // its output rows only after it has read it.
+  const void* qsrc = a->rope_fused ? a->out : a->q;
+  const int64_t* qst = a->rope_fused ? a->out_strides : a->q_strides;
+  if (!make_rows_map(&tmQ, qsrc, D, a->T, a->n_q, a->B, qst, Cfg::CB)) return SA_ERR_CUDA;
   // The box is one BN-row K/V tile: the kernel's expect-tx byte count and
   // ring-slot size are both Cfg::KV_BYTES = BN * D * 2.
   static_assert(Cfg::KV_BYTES == (uint32_t)Cfg::BN * D * 2, "tile size");
@@ -186,8 +211,10 @@ sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream
     set_smem(sa::prefill_kernel<D>, Cfg::SMEM_BYTES);
     configured = true;
   }
-  dim3 grid(p.n_pairs, a->n_q, a->B);
-  sa::prefill_kernel<D><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmK, tmV, p);
+  // persistent: one CTA per SM (or per item when there are fewer)
+  const long long n_items = (long long)p.n_pairs * a->n_q * a->B;
+  const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
+  sa::prefill_kernel<D><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
   return last_launch_status();
 }
 
@@ -293,6 +320,22 @@ sa_status launch_append(sa_kv_cache* c, const void* k, const int64_t ks[3], cons
       static_cast<const __nv_bfloat16*>(k), ks[0], ks[1], ks[2],
       static_cast<const __nv_bfloat16*>(v), vs[0], vs[1], vs[2], c->B, T, c->n_kv, c->d, c->offset,
       rope, cos_t, sin_t);
+  return last_launch_status();
+}
+
+// Prefill staging: append K/V (rotating k) and, when RoPE is fused, write the
+// rotated queries into `out` for the attention kernel to load by TMA.
+sa_status launch_stage(sa_kv_cache* c, const sa_attn_args* a, cudaStream_t stream) {
+  const int stage_q = a->rope_fused ? 1 : 0;
+  const long long n = (long long)c->B * a->T * (c->n_kv + (stage_q ? a->n_q : 0)) * (c->d / 16);
+  sa::prefill_stage_kernel<<<grid_for(n), 256, 0, stream>>>(
+      static_cast<__nv_bfloat16*>(c->k), static_cast<__nv_bfloat16*>(c->v), c->cap,
+      static_cast<const __nv_bfloat16*>(a->k), a->k_strides[0], a->k_strides[1], a->k_strides[2],
+      static_cast<const __nv_bfloat16*>(a->v), a->v_strides[0], a->v_strides[1], a->v_strides[2],
+      c->B, a->T, c->n_kv, c->d, c->offset, a->rope_fused ? 1 : 0, a->cos, a->sin,
+      static_cast<const __nv_bfloat16*>(a->q), a->q_strides[0], a->q_strides[1], a->q_strides[2],
+      a->n_q, static_cast<__nv_bfloat16*>(a->out), a->out_strides[0], a->out_strides[1],
+      a->out_strides[2], stage_q);
   return last_launch_status();
 }
 
@@ -446,8 +489,7 @@ sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* a, sa_stream_t
   if (st != SA_OK) return st;
   if (a->T == 0) return SA_OK;
   cudaStream_t s = (cudaStream_t)stream;
-  st = launch_append(cache, a->k, a->k_strides, a->v, a->v_strides, a->T, a->rope_fused ? 1 : 0,
-                     a->cos, a->sin, s);
+  st = launch_stage(cache, a, s);
   if (st != SA_OK) return st;
   switch (cache->d) {
     case 64: st = launch_prefill<64>(cache, a, s); break;
