@@ -465,16 +465,31 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_before();
           mbar_arrive(bar(BAR_SFREE + X));   // the tensor core may overwrite S_X now
           if (t < full_lo || t >= full_hi) {
-            // admitted columns c (key klo + c): c >= cmin and c <= cmax
+            // Admitted columns c (key klo + c) satisfy cmin <= c <= cmax. A
+            // tile needs the upper bound where it crosses the diagonal of
+            // some row and the lower one where it reaches below the band (or
+            // below key 0) of some row; each side is one compare + select
+            // per column, skipped when no row of the tile needs it.
             const long long klo = geo.base + (long long)BN * t;
+            const long long p0 = p.off + geo.i0 + 128 * X;   // position of row 0
+            long long lo_last = 0;                            // lowest key of row 127
+            if (p.window > 0 && p0 + 128 - p.window > 0) lo_last = p0 + 128 - p.window;
             long long lo_k = 0;
             if (p.window > 0 && pos - p.window + 1 > lo_k) lo_k = pos - p.window + 1;
-            const long long cmin = lo_k - klo, cmax = pos - klo;
-            const int cmin_i = (int)(cmin < -1 ? -1 : (cmin > BN ? BN : cmin));
-            const int cmax_i = (int)(cmax < -1 ? -1 : (cmax > BN ? BN : cmax));
+            if (klo + BN - 1 > p0) {
+              const long long cmax = pos - klo;
+              const int cmax_i = (int)(cmax < -1 ? -1 : (cmax > BN ? BN : cmax));
 #pragma unroll
-            for (int c = 0; c < BN; ++c)
-              if (c < cmin_i || c > cmax_i) sr[c] = __float_as_uint(-INFINITY);
+              for (int c = 0; c < BN; ++c)
+                if (c > cmax_i) sr[c] = __float_as_uint(-INFINITY);
+            }
+            if (klo < lo_last) {
+              const long long cmin = lo_k - klo;
+              const int cmin_i = (int)(cmin < -1 ? -1 : (cmin > BN ? BN : cmin));
+#pragma unroll
+              for (int c = 0; c < BN; ++c)
+                if (c < cmin_i) sr[c] = __float_as_uint(-INFINITY);
+            }
           }
           // raw row max (scale > 0, so max(s * scale) = scale * max(s))
           float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
@@ -488,33 +503,13 @@ __global__ void __launch_bounds__(384, 1)
           const float mx = fmaxf(max3f(m0, m1, m2), m3) * scale;
           const float m_new = fmaxf(m, mx);
           const bool need = m_new > m + 8.0f;
-          bool pv_done = (ntot == 0);
-          if (__any_sync(0xffffffffu, need)) {
-            const float f = need ? ex2(m - m_new) : 1.0f;
-            if (n > 0) {
-              // O_X may only be touched once the previous PV_X has landed.
-              if (!mbar_wait(bar(BAR_ODONE + X), (uint32_t)((ntot - 1) & 1))) { ok = false; *abort_flag = 1; break; }
-              tc_fence_after();
-              pv_done = true;
-#pragma unroll 1
-              for (int c0 = 0; c0 < D; c0 += 16) {
-                uint32_t rr16[16];
-                tmem_ld16(o_tm + c0, rr16);
-                tmem_wait_ld();
-#pragma unroll
-                for (int c = 0; c < 16; c += 2) {
-                  float a0 = __uint_as_float(rr16[c]), a1 = __uint_as_float(rr16[c + 1]);
-                  mul2(a0, a1, f, f);
-                  rr16[c] = __float_as_uint(a0);
-                  rr16[c + 1] = __float_as_uint(a1);
-                }
-                tmem_st16(o_tm + c0, rr16);
-              }
-            }
-            if (need) {
-              l *= f;
-              m = m_new;
-            }
+          // O_X is rescaled by f later, once the previous PV_X has landed.
+          const bool rescale = __any_sync(0xffffffffu, need) && n > 0;
+          float f = 1.0f;
+          if (need) {
+            f = ex2(m - m_new);
+            l *= f;
+            m = m_new;
           }
           const float neg = (m == -INFINITY) ? 0.f : -m;
           uint32_t pk[BN / 2];
@@ -524,8 +519,14 @@ __global__ void __launch_bounds__(384, 1)
             float x0, x1, x2, x3;
             fma2(x0, x1, __uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1]), scale, scale, neg, neg);
             fma2(x2, x3, __uint_as_float(sr[2 * c + 2]), __uint_as_float(sr[2 * c + 3]), scale, scale, neg, neg);
-            x0 = ex2(x0);
-            x1 = ex2(x1);
+            // One pair in four goes to the FMA pipe (polynomial exp2), the
+            // rest to the MUFU unit: the two run side by side.
+            if ((c / 2) % 2 == 0) {
+              exp2_fma2(x0, x1);
+            } else {
+              x0 = ex2(x0);
+              x1 = ex2(x1);
+            }
             x2 = ex2(x2);
             x3 = ex2(x3);
             add2(l0, l1, x0, x1);
@@ -534,10 +535,26 @@ __global__ void __launch_bounds__(384, 1)
             pk[c + 1] = pack_bf16(x2, x3);
           }
           l += (l0 + l1) + (l2 + l3);
-          // P_X is read by the previous PV_X until it completes.
-          if (!pv_done) {
+          // O_X and P_X are read by the previous PV_X until it completes.
+          if (ntot > 0) {
             if (!mbar_wait(bar(BAR_ODONE + X), (uint32_t)((ntot - 1) & 1))) { ok = false; *abort_flag = 1; break; }
             tc_fence_after();
+          }
+          if (rescale) {
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o32[32];
+              tmem_ld32(o_tm + c0, o32);
+              tmem_wait_ld();
+#pragma unroll
+              for (int c = 0; c < 32; c += 2) {
+                float a0 = __uint_as_float(o32[c]), a1 = __uint_as_float(o32[c + 1]);
+                mul2(a0, a1, f, f);
+                o32[c] = __float_as_uint(a0);
+                o32[c + 1] = __float_as_uint(a1);
+              }
+              tmem_st32(o_tm + c0, o32);
+            }
           }
 #pragma unroll
           for (int c0 = 0; c0 + 32 <= BN / 2; c0 += 32)
