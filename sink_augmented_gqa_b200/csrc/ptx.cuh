@@ -308,11 +308,12 @@ __device__ __forceinline__ void addto2(float& d0, float& d1, float a0, float a1,
 // vanishing weight). Range reduction: t = x + 1.5*2^23 rounds x to the
 // nearest integer j (held in t's low mantissa bits), f = x - j in
 // [-1/2, 1/2] exactly; then 2^x = 2^j * p(f), the 2^j applied as an integer
-// add of j << 23 to p's bit pattern. p is the degree-4 fit of 2^f on
-// [-1/2, 1/2] produced by fit_exp2_poly.py (relative error < 3e-6 in fp32
-// Horner form).
-constexpr float EXP2_C0 = 0.999999285f, EXP2_C1 = 0.693121791f, EXP2_C2 = 0.240247443f,
-                EXP2_C3 = 0.0559178591f, EXP2_C4 = 0.00957009662f;
+// add of j << 23 to p's bit pattern. p is the degree-3 fit of 2^f on
+// [-1/2, 1/2] with constant term 1 (so integer x give exact powers of two)
+// produced by fit_exp2_poly.py: relative error < 1.1e-4 in fp32 Horner form,
+// well below the 2^-9 of the bf16 P it feeds.
+constexpr float EXP2_C0 = 1.0f, EXP2_C1 = 0.693282962f, EXP2_C2 = 0.242210969f,
+                EXP2_C3 = 0.0550089031f;
 __device__ __forceinline__ void exp2_fma2(float& a, float& b) {
   constexpr float MAGIC = 12582912.0f;  // 1.5 * 2^23
   a = fmaxf(a, -120.0f);
@@ -321,8 +322,7 @@ __device__ __forceinline__ void exp2_fma2(float& a, float& b) {
   addto2(ta, tb, a, b, MAGIC, MAGIC);
   addto2(ja, jb, ta, tb, -MAGIC, -MAGIC);
   addto2(fa, fb, a, b, -ja, -jb);
-  float pa = EXP2_C4, pb = EXP2_C4;
-  fma2(pa, pb, pa, pb, fa, fb, EXP2_C3, EXP2_C3);
+  float pa = EXP2_C3, pb = EXP2_C3;
   fma2(pa, pb, pa, pb, fa, fb, EXP2_C2, EXP2_C2);
   fma2(pa, pb, pa, pb, fa, fb, EXP2_C1, EXP2_C1);
   fma2(pa, pb, pa, pb, fa, fb, EXP2_C0, EXP2_C0);
