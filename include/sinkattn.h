@@ -201,6 +201,11 @@ sa_status sa_kv_restore(sa_kv_cache* cache, const sa_snapshot* snap);
  * note, "How it works"). cache->offset += T on success. T == 0 is a no-op.
  * The attention runs on tcgen05 tensor cores with fp32 accumulation; the
  * softmax weights enter the PV product as bf16.
+ * When rope_fused, the rotated queries are first staged in args->out (same
+ * [B][T][n_q][d] view) and each output tile overwrites its own staged query
+ * rows, so `out` may be `q` itself but must not overlap k, v, the cache, the
+ * sinks, the tables or lse otherwise. Two launches on `stream` (staging,
+ * attention).
  */
 sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* args, sa_stream_t stream);
 
@@ -257,6 +262,18 @@ sa_status sa_get_device_status(int32_t* code);
  * the timeout path only.
  */
 sa_status sa_set_wait_limit(int64_t cycles);
+
+/*
+ * Timing hook for the attention kernel of sa_attn_prefill (no counterpart in
+ * the method; measurement support). While set, every sa_attn_prefill call
+ * records `before` on its stream after the staging launch (RoPE + append)
+ * and just before the attention kernel, and `after` just after it, so the
+ * caller can time the attention kernel alone with cudaEventElapsedTime.
+ * before/after: cudaEvent_t handles owned by the caller, both NULL to clear
+ * (one NULL and one not: SA_ERR_INVALID_ARG). Process-wide; not for
+ * concurrent use from several threads.
+ */
+sa_status sa_set_prefill_events(void* before, void* after);
 
 #ifdef __cplusplus
 }

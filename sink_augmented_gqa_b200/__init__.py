@@ -17,6 +17,7 @@ from .sinkattn import (  # noqa: F401
     decode_workspace_bytes,
     device_status,
     rope_apply_qk,
+    set_prefill_events,
     set_wait_limit,
     yarn_rope_tables,
 )

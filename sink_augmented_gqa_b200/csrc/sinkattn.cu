@@ -323,6 +323,10 @@ sa_status launch_append(sa_kv_cache* c, const void* k, const int64_t ks[3], cons
   return last_launch_status();
 }
 
+// Events of sa_set_prefill_events (null: not recording).
+cudaEvent_t g_prefill_ev_before = nullptr;
+cudaEvent_t g_prefill_ev_after = nullptr;
+
 // Prefill staging: append K/V (rotating k) and, when RoPE is fused, write the
 // rotated queries into `out` for the attention kernel to load by TMA.
 sa_status launch_stage(sa_kv_cache* c, const sa_attn_args* a, cudaStream_t stream) {
@@ -491,12 +495,15 @@ sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* a, sa_stream_t
   cudaStream_t s = (cudaStream_t)stream;
   st = launch_stage(cache, a, s);
   if (st != SA_OK) return st;
+  cudaEvent_t ev0 = g_prefill_ev_before, ev1 = g_prefill_ev_after;
+  if (ev0 != nullptr && cudaEventRecord(ev0, s) != cudaSuccess) return SA_ERR_CUDA;
   switch (cache->d) {
     case 64: st = launch_prefill<64>(cache, a, s); break;
     case 96: st = launch_prefill<96>(cache, a, s); break;
     case 128: st = launch_prefill<128>(cache, a, s); break;
     default: return SA_ERR_SHAPE;
   }
+  if (ev1 != nullptr && cudaEventRecord(ev1, s) != cudaSuccess) return SA_ERR_CUDA;
   // The append is enqueued either way; the offset follows it.
   note_append(cache, cache->offset, a->T);
   return st;
@@ -552,6 +559,13 @@ sa_status sa_get_device_status(int32_t* code) {
   const int zero = 0;
   if (cudaMemcpyToSymbol(sa::g_status, &zero, sizeof(int)) != cudaSuccess) return SA_ERR_CUDA;
   *code = (v & sa::STATUS_TIMEOUT) ? SA_ERR_TIMEOUT : SA_OK;
+  return SA_OK;
+}
+
+sa_status sa_set_prefill_events(void* before, void* after) {
+  if ((before == nullptr) != (after == nullptr)) return SA_ERR_INVALID_ARG;
+  g_prefill_ev_before = static_cast<cudaEvent_t>(before);
+  g_prefill_ev_after = static_cast<cudaEvent_t>(after);
   return SA_OK;
 }
 

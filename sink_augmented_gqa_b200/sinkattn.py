@@ -71,7 +71,7 @@ EXPORTS = (
     "sa_status_string", "sa_yarn_rope_tables", "sa_rope_apply_qk", "sa_kv_cache_init",
     "sa_kv_append", "sa_kv_snapshot", "sa_kv_restore", "sa_attn_prefill", "sa_attn_decode",
     "sa_attn_decode_workspace_size", "sa_get_device_status", "sa_set_wait_limit",
-    "sa_attn_decode_static",
+    "sa_attn_decode_static", "sa_set_prefill_events",
 )
 
 _lib = None
@@ -103,6 +103,7 @@ def lib():
         L.sa_attn_decode_workspace_size.argtypes = [i32, i32, i32, i32]
         L.sa_get_device_status.argtypes = [P(i32)]
         L.sa_set_wait_limit.argtypes = [i64]
+        L.sa_set_prefill_events.argtypes = [vp, vp]
         for name in EXPORTS:
             if name not in ("sa_status_string", "sa_attn_decode_workspace_size"):
                 getattr(L, name).restype = ctypes.c_int
@@ -303,3 +304,11 @@ def device_status():
 
 def set_wait_limit(cycles):
     _check(lib().sa_set_wait_limit(int(cycles)), "sa_set_wait_limit")
+
+
+def set_prefill_events(before=None, after=None):
+    """Record torch.cuda.Event `before`/`after` around the attention kernel of
+    every later attn_prefill (None, None: stop recording)."""
+    h0 = None if before is None else ctypes.c_void_p(before.cuda_event)
+    h1 = None if after is None else ctypes.c_void_p(after.cuda_event)
+    _check(lib().sa_set_prefill_events(h0, h1), "sa_set_prefill_events")

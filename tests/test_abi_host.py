@@ -129,3 +129,10 @@ def test_table_argument_errors(L):
     assert L.sa_yarn_rope_tables(p, p, 0, 64, 150000.0, 32.0, 4096, 1.0, 32.0, None) == 1
     assert L.sa_yarn_rope_tables(p, p, 10, 63, 150000.0, 32.0, 4096, 1.0, 32.0, None) == 1
     assert L.sa_yarn_rope_tables(p, p, 10, 64, 150000.0, 32.0, 4096, 32.0, 1.0, None) == 1   # alpha >= beta
+
+
+def test_prefill_event_hook_arguments(L):
+    inv = [k for k, v in S.STATUS.items() if v == "SA_ERR_INVALID_ARG"][0]
+    assert L.sa_set_prefill_events(ctypes.c_void_p(0x10), None) == inv
+    assert L.sa_set_prefill_events(None, ctypes.c_void_p(0x10)) == inv
+    assert L.sa_set_prefill_events(None, None) == 0
