@@ -98,7 +98,8 @@ struct PrefillCfg {
 // query tile X; [NS] = one per K/V ring slot.
 enum : int {
   BAR_QFULL = 0,    // [2 buffers] producer (TMA) -> MMA: an item's Q tiles landed
-  BAR_QEMPTY = 2,   // [2 buffers] MMA A and B -> producer: last S product read them
+  BAR_QEMPTY = 2,   // [2 buffers] count 4: MMA A and B (last S product read the
+                    // tiles) and the two output stores (which stage O in them)
   BAR_SFULL = 4,    // [2 tiles] MMA -> softmax: S_X computed
   BAR_SFREE = 6,    // [2] softmax -> MMA: S_X read into registers
   BAR_PFULL = 8,    // [2] softmax -> MMA: P_X stored (and O_X rescaled)
@@ -111,6 +112,7 @@ enum : int {
   BAR_VEMPTY = 28,  // [NS] count 2
   BAR_TMEM_SLOT = 32,
   BAR_ABORT_SLOT = 33,
+  BAR_EPI = 34,     // [2] softmax X threads -> its store thread: O rows staged in smem
 };
 
 // Work items are (query-tile pair, query head, sequence), heaviest pairs
@@ -123,6 +125,10 @@ struct ItemSchedule {
     return idx < n_items ? idx : -1;
   }
   __device__ __forceinline__ int rounds() const { return (n_items + G - 1) / G; }
+  // In odd rounds the two pipelines trade row tiles (pipeline X takes row
+  // tile X ^ 1): the upper tile of a causal pair has one key tile more, and
+  // alternating it keeps both pipelines equally loaded.
+  __device__ __forceinline__ static int swap(int r) { return r & 1; }
   __device__ __forceinline__ void coords(int item, int& pair, int& h, int& b) const {
     const int rank = item / per_pair, rem = item % per_pair;
     pair = n_pairs - 1 - rank;
@@ -229,7 +235,8 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint6
 template <int D>
 __global__ void __launch_bounds__(384, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const PrefillParams p) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const PrefillParams p) {
   using C = PrefillCfg<D>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -254,7 +261,8 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     for (int X = 0; X < 2; ++X) {
       mbar_init(bar(BAR_QFULL + X), 1);
-      mbar_init(bar(BAR_QEMPTY + X), 2);
+      mbar_init(bar(BAR_QEMPTY + X), 4);
+      mbar_init(bar(BAR_EPI + X), 128);
       mbar_init(bar(BAR_SFULL + X), 1);
       mbar_init(bar(BAR_SFREE + X), 128);
       mbar_init(bar(BAR_PFULL + X), 128);
@@ -279,6 +287,7 @@ __global__ void __launch_bounds__(384, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
   }
   tc_fence_before();
   __syncthreads();
@@ -306,13 +315,17 @@ __global__ void __launch_bounds__(384, 1)
           *abort_flag = 1;
           break;
         }
+        // pipeline X takes row tile X ^ sw (see ItemSchedule::swap)
+        const int sw = ItemSchedule::swap(rr);
         const int nq = geo.valid(1) ? 2 : 1;
         mbar_arrive_expect_tx(bar(BAR_QFULL + qb), (uint32_t)nq * C::Q_BYTES);
-        for (int X = 0; X < nq; ++X) {
+        for (int X = 0; X < 2; ++X) {
+          const int rt = X ^ sw;
+          if (!geo.valid(rt)) continue;
 #pragma unroll
           for (int cb = 0; cb < C::NCB; ++cb)
             tma_load_4d(sbase + C::OFF_Q + (2 * qb + X) * C::Q_BYTES + cb * C::QBLOCK, &tmQ,
-                        bar(BAR_QFULL + qb), cb * C::CB, geo.i0 + 128 * X, h, b);
+                        bar(BAR_QFULL + qb), cb * C::CB, geo.i0 + 128 * rt, h, b);
         }
         ++j;
         for (int t = 0; t < geo.ntiles; ++t, ++gt) {
@@ -375,7 +388,8 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(bar(BAR_QFULL + qb), (uint32_t)((j >> 1) & 1))) { ok = false; break; }
         tc_fence_after();
         const uint64_t qd = smem_desc(sbase + C::OFF_Q + (2 * qb + X) * C::Q_BYTES, 16, C::SBO, C::LAYOUT);
-        const int lo = X ? geo.a_lo[1] : geo.a_lo[0], hi = X ? geo.a_hi[1] : geo.a_hi[0];
+        const int rt = X ^ ItemSchedule::swap(rr);   // row tile of this pipeline
+        const int lo = rt ? geo.a_lo[1] : geo.a_lo[0], hi = rt ? geo.a_hi[1] : geo.a_hi[0];
         if (hi <= lo) mbar_arrive(bar(BAR_QEMPTY + qb));   // this tile reads no Q
         bool first = true;                                  // no PV of this item issued yet
         for (int t = 0; t <= geo.ntiles; ++t) {
@@ -437,6 +451,9 @@ __global__ void __launch_bounds__(384, 1)
     const float LOG2E = 1.4426950408889634f;
     const float scale = p.scale_log2;
     int ntot = 0;   // cumulative key tiles of this query tile slot (S / P / O-done phases)
+    int j = 0;      // items of this CTA so far (Q buffer j & 1 stages this item's output)
+    int nepi = 0;   // output tiles staged by this pipeline (BAR_EPI phases)
+    const bool store_thread = (threadIdx.x & 127) == 0;
     bool ok = true;
     for (int rr = 0; rr < rounds && ok; ++rr) {
       const int item = sched.at(rr);
@@ -444,16 +461,17 @@ __global__ void __launch_bounds__(384, 1)
       int pair, h, b;
       sched.coords(item, pair, h, b);
       const TileGeom<BN> geo = make_geom<BN>(p, pair);
-      const int i = geo.i0 + 128 * X + r;       // query row within the call
+      const int rt = X ^ ItemSchedule::swap(rr);   // row tile of this pipeline
+      const int i = geo.i0 + 128 * rt + r;      // query row within the call
       const bool row_ok = i < p.T;
       const long long pos = p.off + i;
-      if (geo.valid(X)) {
+      if (geo.valid(rt)) {
         const float sink2 = p.sinks ? p.sinks[h] * LOG2E : -INFINITY;
         float m = sink2;                              // running max (log2 units)
         float l = (sink2 == -INFINITY) ? 0.f : 1.f;   // running sum, sink included
         int n = 0;                                    // key tiles of this item
-        const int t_lo = X ? geo.a_lo[1] : geo.a_lo[0], t_hi = X ? geo.a_hi[1] : geo.a_hi[0];
-        const int full_lo = X ? geo.f_lo[1] : geo.f_lo[0], full_hi = X ? geo.f_hi[1] : geo.f_hi[0];
+        const int t_lo = rt ? geo.a_lo[1] : geo.a_lo[0], t_hi = rt ? geo.a_hi[1] : geo.a_hi[0];
+        const int full_lo = rt ? geo.f_lo[1] : geo.f_lo[0], full_hi = rt ? geo.f_hi[1] : geo.f_hi[0];
         for (int t = t_lo; t < t_hi; ++t) {
           if (!mbar_wait(bar(BAR_SFULL + X), (uint32_t)(ntot & 1))) { ok = false; *abort_flag = 1; break; }
           tc_fence_after();
@@ -471,7 +489,7 @@ __global__ void __launch_bounds__(384, 1)
             // below key 0) of some row; each side is one compare + select
             // per column, skipped when no row of the tile needs it.
             const long long klo = geo.base + (long long)BN * t;
-            const long long p0 = p.off + geo.i0 + 128 * X;   // position of row 0
+            const long long p0 = p.off + geo.i0 + 128 * rt;   // position of row 0
             long long lo_last = 0;                            // lowest key of row 127
             if (p.window > 0 && p0 + 128 - p.window > 0) lo_last = p0 + 128 - p.window;
             long long lo_k = 0;
@@ -567,26 +585,27 @@ __global__ void __launch_bounds__(384, 1)
           ++ntot;
           if (*abort_flag) { ok = false; break; }
         }
-        // Epilogue: O / l -> bf16, once the item's last PV_X has landed.
+        // Epilogue, once the item's last PV_X has landed: O / l -> bf16 into
+        // this pipeline's Q tile of the item (its last S product has been
+        // read, so the tile is free), then one TMA store of the 128 x d tile
+        // (rows past T are dropped by the tensor map's bounds).
+        uint8_t* stage = smem + C::OFF_Q + (2 * (j & 1) + X) * C::Q_BYTES;
         if (ok && n > 0 && mbar_wait(bar(BAR_ODONE + X), (uint32_t)((ntot - 1) & 1)) && !*abort_flag) {
           tc_fence_after();
           const float inv_l = 1.0f / l;
-          __nv_bfloat16* orow = p.out + b * p.os0 + (long long)i * p.os1 + (long long)h * p.os2;
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o32[32];
             tmem_ld32(o_tm + c0, o32);
             tmem_wait_ld();
-            if (row_ok) {
 #pragma unroll
-              for (int c = 0; c < 32; c += 8) {
-                uint4 v;
-                v.x = pack_bf16(__uint_as_float(o32[c + 0]) * inv_l, __uint_as_float(o32[c + 1]) * inv_l);
-                v.y = pack_bf16(__uint_as_float(o32[c + 2]) * inv_l, __uint_as_float(o32[c + 3]) * inv_l);
-                v.z = pack_bf16(__uint_as_float(o32[c + 4]) * inv_l, __uint_as_float(o32[c + 5]) * inv_l);
-                v.w = pack_bf16(__uint_as_float(o32[c + 6]) * inv_l, __uint_as_float(o32[c + 7]) * inv_l);
-                *reinterpret_cast<uint4*>(orow + c0 + c) = v;
-              }
+            for (int c = 0; c < 32; c += 8) {
+              uint4 v;
+              v.x = pack_bf16(__uint_as_float(o32[c + 0]) * inv_l, __uint_as_float(o32[c + 1]) * inv_l);
+              v.y = pack_bf16(__uint_as_float(o32[c + 2]) * inv_l, __uint_as_float(o32[c + 3]) * inv_l);
+              v.z = pack_bf16(__uint_as_float(o32[c + 4]) * inv_l, __uint_as_float(o32[c + 5]) * inv_l);
+              v.w = pack_bf16(__uint_as_float(o32[c + 6]) * inv_l, __uint_as_float(o32[c + 7]) * inv_l);
+              *reinterpret_cast<uint4*>(stage + swz_off<C::CB>(r, c0 + c, C::QBLOCK)) = v;
             }
           }
           if (row_ok && p.lse) {
@@ -597,13 +616,28 @@ __global__ void __launch_bounds__(384, 1)
           ok = false;
           *abort_flag = 1;
         }
+        fence_proxy_async_smem();
+        mbar_arrive(bar(BAR_EPI + X));
+        if (store_thread) {
+          if (mbar_wait(bar(BAR_EPI + X), (uint32_t)(nepi & 1)) && ok && !*abort_flag) {
+#pragma unroll
+            for (int cb = 0; cb < C::NCB; ++cb)
+              tma_store_4d(&tmO, smem_u32(stage) + cb * C::QBLOCK, cb * C::CB, geo.i0 + 128 * rt, h, b);
+            bulk_commit();
+            bulk_wait_read_all();
+          }
+        }
+        ++nepi;
       }
+      if (store_thread) mbar_arrive(bar(BAR_QEMPTY + (j & 1)));   // the staged tile has been read
+      ++j;
       // O_X is free for the next item's first PV.
       tc_fence_before();
       mbar_arrive(bar(BAR_OFREE + X));
     }
   }
 
+  if (warp >= 4 && (threadIdx.x & 127) == 0) bulk_wait_all();   // output stores complete
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

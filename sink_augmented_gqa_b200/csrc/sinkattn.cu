@@ -177,6 +177,8 @@ sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream
   const void* qsrc = a->rope_fused ? a->out : a->q;
   const int64_t* qst = a->rope_fused ? a->out_strides : a->q_strides;
   if (!make_rows_map(&tmQ, qsrc, D, a->T, a->n_q, a->B, qst, Cfg::CB)) return SA_ERR_CUDA;
+  CUtensorMap tmO;   // the output tiles are stored through the same box shape
+  if (!make_rows_map(&tmO, a->out, D, a->T, a->n_q, a->B, a->out_strides, Cfg::CB)) return SA_ERR_CUDA;
   // The box is one BN-row K/V tile: the kernel's expect-tx byte count and
   // ring-slot size are both Cfg::KV_BYTES = BN * D * 2.
   static_assert(Cfg::KV_BYTES == (uint32_t)Cfg::BN * D * 2, "tile size");
@@ -214,7 +216,7 @@ sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream
   // persistent: one CTA per SM (or per item when there are fewer)
   const long long n_items = (long long)p.n_pairs * a->n_q * a->B;
   const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
-  sa::prefill_kernel<D><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+  sa::prefill_kernel<D><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmO, p);
   return last_launch_status();
 }
 
