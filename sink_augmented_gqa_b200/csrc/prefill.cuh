@@ -262,12 +262,12 @@ __global__ void __launch_bounds__(384, 1)
     for (int X = 0; X < 2; ++X) {
       mbar_init(bar(BAR_QFULL + X), 1);
       mbar_init(bar(BAR_QEMPTY + X), 4);
-      mbar_init(bar(BAR_EPI + X), 128);
+      mbar_init(bar(BAR_EPI + X), 4);   // one arrival per warp
       mbar_init(bar(BAR_SFULL + X), 1);
-      mbar_init(bar(BAR_SFREE + X), 128);
-      mbar_init(bar(BAR_PFULL + X), 128);
+      mbar_init(bar(BAR_SFREE + X), 4);   // one arrival per warp
+      mbar_init(bar(BAR_PFULL + X), 4);   // one arrival per warp
       mbar_init(bar(BAR_ODONE + X), 1);
-      mbar_init(bar(BAR_OFREE + X), 128);
+      mbar_init(bar(BAR_OFREE + X), 4);   // one arrival per warp
       mbar_init(bar(BAR_DRAIN + X), 1);
     }
     for (int s = 0; s < C::NS; ++s) {
@@ -481,7 +481,8 @@ __global__ void __launch_bounds__(384, 1)
             tmem_ld32(s_tm + c0, *reinterpret_cast<uint32_t(*)[32]>(&sr[c0]));
           tmem_wait_ld();
           tc_fence_before();
-          mbar_arrive(bar(BAR_SFREE + X));   // the tensor core may overwrite S_X now
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_SFREE + X));   // the tensor core may overwrite S_X now
           if (t < full_lo || t >= full_hi) {
             // Admitted columns c (key klo + c) satisfy cmin <= c <= cmax. A
             // tile needs the upper bound where it crosses the diagonal of
@@ -580,7 +581,8 @@ __global__ void __launch_bounds__(384, 1)
           if constexpr ((BN / 2) % 32 == 16) tmem_st16(p_tm + (BN / 2 - 16), &pk[BN / 2 - 16]);
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(bar(BAR_PFULL + X));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_PFULL + X));
           ++n;
           ++ntot;
           if (*abort_flag) { ok = false; break; }
@@ -617,7 +619,8 @@ __global__ void __launch_bounds__(384, 1)
           *abort_flag = 1;
         }
         fence_proxy_async_smem();
-        mbar_arrive(bar(BAR_EPI + X));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_EPI + X));
         if (store_thread) {
           if (mbar_wait(bar(BAR_EPI + X), (uint32_t)(nepi & 1)) && ok && !*abort_flag) {
 #pragma unroll
@@ -633,7 +636,8 @@ __global__ void __launch_bounds__(384, 1)
       ++j;
       // O_X is free for the next item's first PV.
       tc_fence_before();
-      mbar_arrive(bar(BAR_OFREE + X));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_OFREE + X));
     }
   }
 
