@@ -114,6 +114,12 @@ PREFILL_CASES = [
     ("chunk_at_offset", dict(B=2, n_q=8, n_kv=2, d=64), 200, 150),
     ("chunk_unaligned_offset", dict(B=1, n_q=4, n_kv=2, d=64), 77, 300),
     ("single_row", dict(B=3, n_q=8, n_kv=2, d=64), 5, 1),
+    # more work items than SMs: every persistent CTA walks several items, so
+    # both Q buffers, the cumulative ring and barrier phases and the
+    # alternating row-tile assignment are exercised, with ragged last pairs
+    ("persistent_d64", dict(B=4, n_q=16, n_kv=4, d=64), 0, 1500),
+    ("persistent_d96_offset", dict(B=4, n_q=8, n_kv=4, d=96, sm_scale=1 / math.sqrt(96), sink_std=0.5), 100, 1900),
+    ("persistent_d128", dict(B=4, n_q=16, n_kv=2, d=128, sm_scale=1 / math.sqrt(128)), 0, 1100),
 ]
 
 
