@@ -489,25 +489,23 @@ __global__ void __launch_bounds__(384, 1)
             // some row and the lower one where it reaches below the band (or
             // below key 0) of some row; each side is one compare + select
             // per column, skipped when no row of the tile needs it.
-            const long long klo = geo.base + (long long)BN * t;
-            const long long p0 = p.off + geo.i0 + 128 * rt;   // position of row 0
-            long long lo_last = 0;                            // lowest key of row 127
-            if (p.window > 0 && p0 + 128 - p.window > 0) lo_last = p0 + 128 - p.window;
-            long long lo_k = 0;
-            if (p.window > 0 && pos - p.window + 1 > lo_k) lo_k = pos - p.window + 1;
+            // Positions fit in 32 bits (cap < 2^31).
+            const int klo = (int)geo.base + BN * t;
+            const int p0 = (int)p.off + geo.i0 + 128 * rt;   // position of row 0
+            const int ipos = (int)pos;
             if (klo + BN - 1 > p0) {
-              const long long cmax = pos - klo;
-              const int cmax_i = (int)(cmax < -1 ? -1 : (cmax > BN ? BN : cmax));
+              const int cmax = min(max(ipos - klo, -1), BN);
 #pragma unroll
               for (int c = 0; c < BN; ++c)
-                if (c > cmax_i) sr[c] = __float_as_uint(-INFINITY);
+                if (c > cmax) sr[c] = __float_as_uint(-INFINITY);
             }
+            const int lo_last = p.window > 0 ? max(p0 + 128 - p.window, 0) : 0;   // lowest key of row 127
             if (klo < lo_last) {
-              const long long cmin = lo_k - klo;
-              const int cmin_i = (int)(cmin < -1 ? -1 : (cmin > BN ? BN : cmin));
+              const int lo_k = p.window > 0 ? max(ipos - p.window + 1, 0) : 0;
+              const int cmin = min(max(lo_k - klo, 0), BN);
 #pragma unroll
               for (int c = 0; c < BN; ++c)
-                if (c < cmin_i) sr[c] = __float_as_uint(-INFINITY);
+                if (c < cmin) sr[c] = __float_as_uint(-INFINITY);
             }
           }
           // raw row max (scale > 0, so max(s * scale) = scale * max(s))
