@@ -16,7 +16,9 @@
 //               The two streams are independent: each walks every K/V tile of
 //               the item, multiplies the ones its tile admits and releases the
 //               others at once (the ring slots count one release from each).
-//   warp 3      idle.
+//   warp 3      one thread stores each normalised output tile with a TMA
+//               tile store from the item's Q buffer, where the softmax
+//               warps staged it.
 //   warps 4-7   softmax for tile A, warps 8-11 for tile B, one query row per
 //               thread (TMEM lane = row): per key tile: read S, release it at once (so the
 //               tensor core computes the next S while this one is
@@ -112,7 +114,9 @@ enum : int {
   BAR_VEMPTY = 28,  // [NS] count 2
   BAR_TMEM_SLOT = 32,
   BAR_ABORT_SLOT = 33,
-  BAR_EPI = 34,     // [2] softmax X threads -> its store thread: O rows staged in smem
+  BAR_EPI = 34,     // [2 X][2 Q buffers] softmax X warps -> the store thread: O rows
+                    // staged in Q buffer b (one barrier per buffer, so a pipeline
+                    // running an item ahead cannot complete a phase twice)
 };
 
 // Work items are (query-tile pair, query head, sequence), heaviest pairs
@@ -262,7 +266,8 @@ __global__ void __launch_bounds__(384, 1)
     for (int X = 0; X < 2; ++X) {
       mbar_init(bar(BAR_QFULL + X), 1);
       mbar_init(bar(BAR_QEMPTY + X), 4);
-      mbar_init(bar(BAR_EPI + X), 4);   // one arrival per warp
+      mbar_init(bar(BAR_EPI + 2 * X), 4);   // one arrival per warp
+      mbar_init(bar(BAR_EPI + 2 * X + 1), 4);
       mbar_init(bar(BAR_SFULL + X), 1);
       mbar_init(bar(BAR_SFREE + X), 4);   // one arrival per warp
       mbar_init(bar(BAR_PFULL + X), 4);   // one arrival per warp
@@ -360,6 +365,43 @@ __global__ void __launch_bounds__(384, 1)
         for (int u = (j > 2 ? j - 2 : 0); u < j; ++u)
           mbar_wait_drain(bar(BAR_QFULL + (u & 1)), (uint32_t)((u >> 1) & 1));
       }
+    } else if (warp == 3 && lane == 0) {
+      // ------------------------------------------------------------ output stores
+      // Per item and query tile: once the softmax warps have staged the
+      // normalised output tile in the item's Q buffer (BAR_EPI), one TMA
+      // tile store; the Q buffer is released to the producer once the stores
+      // have read it.
+      int j = 0;
+      int nepi[2][2] = {{0, 0}, {0, 0}};   // phases of BAR_EPI [X][buffer]
+      bool ok = true;
+      for (int rr = 0; rr < rounds && ok; ++rr) {
+        const int item = sched.at(rr);
+        if (item < 0) continue;
+        int pair, h, b;
+        sched.coords(item, pair, h, b);
+        const TileGeom<BN> geo = make_geom<BN>(p, pair);
+        const int sw = ItemSchedule::swap(rr);
+#pragma unroll
+        for (int X = 0; X < 2; ++X) {
+          const int rt = X ^ sw;
+          if (!geo.valid(rt)) continue;
+          const int qb = j & 1;
+          if (!mbar_wait(bar(BAR_EPI + 2 * X + qb), (uint32_t)(nepi[X][qb] & 1))) { ok = false; *abort_flag = 1; break; }
+          ++nepi[X][qb];
+          if (*abort_flag) { ok = false; break; }
+          const uint32_t stage = sbase + C::OFF_Q + (2 * (j & 1) + X) * C::Q_BYTES;
+#pragma unroll
+          for (int cb = 0; cb < C::NCB; ++cb)
+            tma_store_4d(&tmO, stage + cb * C::QBLOCK, cb * C::CB, geo.i0 + 128 * rt, h, b);
+          bulk_commit();
+        }
+        if (!ok) break;
+        bulk_wait_read_all();
+        mbar_arrive(bar(BAR_QEMPTY + (j & 1)));   // both staged tiles have been read
+        mbar_arrive(bar(BAR_QEMPTY + (j & 1)));
+        ++j;
+      }
+      bulk_wait_all();   // output stores complete before the CTA exits
     } else if ((warp == 1 || warp == 2) && lane == 0) {
       // ------------------------------------------------------------ MMA issuer of tile X
       // Per key tile t: S_X(t) as soon as the softmax released the previous
@@ -452,10 +494,19 @@ __global__ void __launch_bounds__(384, 1)
     const float scale = p.scale_log2;
     int ntot = 0;   // cumulative key tiles of this query tile slot (S / P / O-done phases)
     int j = 0;      // items of this CTA so far (Q buffer j & 1 stages this item's output)
-    int nepi = 0;   // output tiles staged by this pipeline (BAR_EPI phases)
-    const bool store_thread = (threadIdx.x & 127) == 0;
     bool ok = true;
+    // The sink of the next item is loaded one item ahead, off the critical path.
+    auto sink_of = [&](int rr_) -> float {
+      const int it_ = rr_ < rounds ? sched.at(rr_) : -1;
+      if (it_ < 0 || p.sinks == nullptr) return -INFINITY;
+      int pr_, h_, b_;
+      sched.coords(it_, pr_, h_, b_);
+      return p.sinks[h_];
+    };
+    float sink_next = sink_of(0);
     for (int rr = 0; rr < rounds && ok; ++rr) {
+      const float sink_raw = sink_next;
+      sink_next = sink_of(rr + 1);
       const int item = sched.at(rr);
       if (item < 0) continue;
       int pair, h, b;
@@ -466,7 +517,7 @@ __global__ void __launch_bounds__(384, 1)
       const bool row_ok = i < p.T;
       const long long pos = p.off + i;
       if (geo.valid(rt)) {
-        const float sink2 = p.sinks ? p.sinks[h] * LOG2E : -INFINITY;
+        const float sink2 = sink_raw * LOG2E;   // -inf without sinks
         float m = sink2;                              // running max (log2 units)
         float l = (sink2 == -INFINITY) ? 0.f : 1.f;   // running sum, sink included
         int n = 0;                                    // key tiles of this item
@@ -618,19 +669,8 @@ __global__ void __launch_bounds__(384, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_EPI + X));
-        if (store_thread) {
-          if (mbar_wait(bar(BAR_EPI + X), (uint32_t)(nepi & 1)) && ok && !*abort_flag) {
-#pragma unroll
-            for (int cb = 0; cb < C::NCB; ++cb)
-              tma_store_4d(&tmO, smem_u32(stage) + cb * C::QBLOCK, cb * C::CB, geo.i0 + 128 * rt, h, b);
-            bulk_commit();
-            bulk_wait_read_all();
-          }
-        }
-        ++nepi;
+        if (lane == 0) mbar_arrive(bar(BAR_EPI + 2 * X + (j & 1)));   // warp 3 stores the tile
       }
-      if (store_thread) mbar_arrive(bar(BAR_QEMPTY + (j & 1)));   // the staged tile has been read
       ++j;
       // O_X is free for the next item's first PV.
       tc_fence_before();
@@ -639,7 +679,6 @@ __global__ void __launch_bounds__(384, 1)
     }
   }
 
-  if (warp >= 4 && (threadIdx.x & 127) == 0) bulk_wait_all();   // output stores complete
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
