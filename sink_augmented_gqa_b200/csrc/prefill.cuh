@@ -61,7 +61,14 @@ struct PrefillParams {
   float scale_log2;
   int rope;
   int n_pairs;
+  int sched_slot;   // which counter pair of g_prefill_sched this launch uses
 };
+
+// Work counters of the dynamic item schedule, one pair per launch slot (the
+// host hands out slots round robin): [0] items handed out beyond the first
+// gridDim.x, [1] CTAs finished. The last CTA to finish resets both.
+constexpr int kPrefillSchedSlots = 64;
+__device__ int g_prefill_sched[kPrefillSchedSlots][2];
 
 __host__ __device__ constexpr int align32(int x) { return (x + 31) / 32 * 32; }
 
@@ -114,25 +121,26 @@ enum : int {
   BAR_VEMPTY = 28,  // [NS] count 2
   BAR_TMEM_SLOT = 32,
   BAR_ABORT_SLOT = 33,
+  BAR_IFULL = 38,   // [4] producer -> every role: item descriptor k published in ring slot k & 3
+  BAR_IEMPTY = 42,  // [4] count 11 (MMA A, MMA B, store thread, 8 softmax warps): read
+  BAR_IRING = 46,   // int item[4] then float sink[4] (slots 46-49)
   BAR_EPI = 34,     // [2 X][2 Q buffers] softmax X warps -> the store thread: O rows
                     // staged in Q buffer b (one barrier per buffer, so a pipeline
                     // running an item ahead cannot complete a phase twice)
 };
 
-// Work items are (query-tile pair, query head, sequence), heaviest pairs
-// first; CTA c of G takes item r*G + c in even rounds r and r*G + G-1-c in
-// odd ones (a snake, so the heavy and light ends of each round balance).
+// Work items are (query-tile pair, query head, sequence), numbered heaviest
+// pair first. CTA c starts with item c; every further item comes from an
+// atomic counter (dynamic schedule: an SM that finishes early takes more, so
+// neither the uneven item sizes nor uneven SM speeds leave a tail). The
+// producer thread fetches the ids and publishes each, with its sink logit, in
+// a 4-slot shared-memory ring that every role reads in the same order.
 struct ItemSchedule {
   int G, n_items, per_pair, n_pairs, n_q;
-  __device__ __forceinline__ int at(int r) const {
-    const int idx = r * G + ((r & 1) ? (G - 1 - (int)blockIdx.x) : (int)blockIdx.x);
-    return idx < n_items ? idx : -1;
-  }
-  __device__ __forceinline__ int rounds() const { return (n_items + G - 1) / G; }
-  // In odd rounds the two pipelines trade row tiles (pipeline X takes row
-  // tile X ^ 1): the upper tile of a causal pair has one key tile more, and
-  // alternating it keeps both pipelines equally loaded.
-  __device__ __forceinline__ static int swap(int r) { return r & 1; }
+  // The two pipelines trade row tiles on every other item of a CTA
+  // (pipeline X takes row tile X ^ 1): the upper tile of a causal pair has one
+  // key tile more, and alternating it keeps both pipelines equally loaded.
+  __device__ __forceinline__ static int swap(int k) { return k & 1; }
   __device__ __forceinline__ void coords(int item, int& pair, int& h, int& b) const {
     const int rank = item / per_pair, rem = item % per_pair;
     pair = n_pairs - 1 - rank;
@@ -260,7 +268,23 @@ __global__ void __launch_bounds__(384, 1)
   sched.n_pairs = p.n_pairs;
   sched.n_items = p.n_pairs * sched.per_pair;
   sched.n_q = p.n_q;
-  const int rounds = sched.rounds();
+  volatile int* ring_item = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * BAR_IRING);
+  volatile float* ring_sink = reinterpret_cast<volatile float*>(smem + C::OFF_BAR + 8 * BAR_IRING + 16);
+  // Read item k of this CTA from the ring (all roles, in order); `elected`:
+  // whether this thread arrives on the slot's release barrier for its group.
+  // Returns n_items (no more work) on a timed-out wait.
+  auto fetch = [&](int k, bool elected, float& sink) -> int {
+    const int sl = k & 3;
+    if (!mbar_wait(bar(BAR_IFULL + sl), (uint32_t)((k >> 2) & 1))) {
+      *abort_flag = 1;
+      return sched.n_items;
+    }
+    const int it = ring_item[sl];
+    sink = ring_sink[sl];
+    __syncwarp(__activemask());
+    if (elected) mbar_arrive(bar(BAR_IEMPTY + sl));
+    return it;
+  };
 
   if (threadIdx.x == 0) {
     for (int X = 0; X < 2; ++X) {
@@ -274,6 +298,10 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar(BAR_ODONE + X), 1);
       mbar_init(bar(BAR_OFREE + X), 4);   // one arrival per warp
       mbar_init(bar(BAR_DRAIN + X), 1);
+    }
+    for (int sl = 0; sl < 4; ++sl) {
+      mbar_init(bar(BAR_IFULL + sl), 1);
+      mbar_init(bar(BAR_IEMPTY + sl), 11);
     }
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar(BAR_KFULL + s), 1);
@@ -308,11 +336,27 @@ __global__ void __launch_bounds__(384, 1)
       // ------------------------------------------------------------ producer
       int gt = 0;  // K/V tiles issued so far (ring position)
       int j = 0;   // Q loads issued so far
-      for (int rr = 0; rr < rounds && !*abort_flag; ++rr) {
-        const int item = sched.at(rr);
-        if (item < 0) continue;
-        int pair, h, b;
-        sched.coords(item, pair, h, b);
+      int* ctr = &g_prefill_sched[p.sched_slot][0];
+      int next = blockIdx.x;   // the first item; later ones from the counter
+      for (int k = 0; !*abort_flag; ++k) {
+        const int sl = k & 3;
+        if (k >= 4 && !mbar_wait(bar(BAR_IEMPTY + sl), (uint32_t)(((k >> 2) - 1) & 1))) {
+          *abort_flag = 1;
+          break;
+        }
+        const int item = next < sched.n_items ? next : sched.n_items;
+        int pair = 0, h = 0, b = 0;
+        float sink = -INFINITY;
+        if (item < sched.n_items) {
+          next = sched.G + atomicAdd(ctr, 1);   // the following item, fetched one ahead
+          sched.coords(item, pair, h, b);
+          if (p.sinks) sink = p.sinks[h];
+        }
+        ring_item[sl] = item;
+        ring_sink[sl] = sink;
+        mbar_arrive(bar(BAR_IFULL + sl));   // release: the ring entry is visible to acquirers
+        if (item >= sched.n_items) break;
+        const int rr = k;
         const int g = h / p.q_mult;
         const TileGeom<BN> geo = make_geom<BN>(p, pair);
         const int qb = j & 1;
@@ -374,9 +418,10 @@ __global__ void __launch_bounds__(384, 1)
       int j = 0;
       int nepi[2][2] = {{0, 0}, {0, 0}};   // phases of BAR_EPI [X][buffer]
       bool ok = true;
-      for (int rr = 0; rr < rounds && ok; ++rr) {
-        const int item = sched.at(rr);
-        if (item < 0) continue;
+      for (int rr = 0; ok; ++rr) {
+        float sink_unused;
+        const int item = fetch(rr, true, sink_unused);
+        if (item >= sched.n_items) break;
         int pair, h, b;
         sched.coords(item, pair, h, b);
         const TileGeom<BN> geo = make_geom<BN>(p, pair);
@@ -420,9 +465,10 @@ __global__ void __launch_bounds__(384, 1)
       int nS = 0, nP = 0;  // cumulative S products / PV products of this tile
       int gt = 0;          // ring position of K(0) of the current item
       int j = 0;           // items done by this CTA
-      for (int rr = 0; rr < rounds && ok; ++rr) {
-        const int item = sched.at(rr);
-        if (item < 0) continue;
+      for (int rr = 0; ok; ++rr) {
+        float sink_unused;
+        const int item = fetch(rr, true, sink_unused);
+        if (item >= sched.n_items) break;
         int pair, h, b;
         sched.coords(item, pair, h, b);
         const TileGeom<BN> geo = make_geom<BN>(p, pair);
@@ -495,20 +541,10 @@ __global__ void __launch_bounds__(384, 1)
     int ntot = 0;   // cumulative key tiles of this query tile slot (S / P / O-done phases)
     int j = 0;      // items of this CTA so far (Q buffer j & 1 stages this item's output)
     bool ok = true;
-    // The sink of the next item is loaded one item ahead, off the critical path.
-    auto sink_of = [&](int rr_) -> float {
-      const int it_ = rr_ < rounds ? sched.at(rr_) : -1;
-      if (it_ < 0 || p.sinks == nullptr) return -INFINITY;
-      int pr_, h_, b_;
-      sched.coords(it_, pr_, h_, b_);
-      return p.sinks[h_];
-    };
-    float sink_next = sink_of(0);
-    for (int rr = 0; rr < rounds && ok; ++rr) {
-      const float sink_raw = sink_next;
-      sink_next = sink_of(rr + 1);
-      const int item = sched.at(rr);
-      if (item < 0) continue;
+    for (int rr = 0; ok; ++rr) {
+      float sink_raw;
+      const int item = fetch(rr, lane == 0, sink_raw);
+      if (item >= sched.n_items) break;
       int pair, h, b;
       sched.coords(item, pair, h, b);
       const TileGeom<BN> geo = make_geom<BN>(p, pair);
@@ -685,6 +721,16 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (threadIdx.x == 0) {
+    // Every producer of the grid has fetched its last id once all CTAs got
+    // here, so the last one can reset the counters for the next launch.
+    __threadfence();
+    if (atomicAdd(&g_prefill_sched[p.sched_slot][1], 1) == (int)gridDim.x - 1) {
+      g_prefill_sched[p.sched_slot][0] = 0;
+      g_prefill_sched[p.sched_slot][1] = 0;
+      __threadfence();
+    }
   }
 }
 

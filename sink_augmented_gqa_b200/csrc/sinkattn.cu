@@ -7,6 +7,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/sinkattn.h"
@@ -208,6 +209,11 @@ sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream
   p.scale_log2 = a->sm_scale * 1.4426950408889634f;
   p.rope = a->rope_fused ? 1 : 0;
   p.n_pairs = (a->T + 255) / 256;
+  // Launches take the dynamic-schedule counter pairs round robin; a pair is
+  // reset by the last CTA of its launch, so up to kPrefillSchedSlots
+  // launches may be in flight at once on one device.
+  static std::atomic<unsigned> sched_seq{0};
+  p.sched_slot = (int)(sched_seq.fetch_add(1, std::memory_order_relaxed) % sa::kPrefillSchedSlots);
   static bool configured = false;
   if (!configured) {
     set_smem(sa::prefill_kernel<D>, Cfg::SMEM_BYTES);
