@@ -123,7 +123,7 @@ enum : int {
   BAR_ABORT_SLOT = 33,
   BAR_IFULL = 38,   // [4] producer -> every role: item descriptor k published in ring slot k & 3
   BAR_IEMPTY = 42,  // [4] count 11 (MMA A, MMA B, store thread, 8 softmax warps): read
-  BAR_IRING = 46,   // int item[4] then float sink[4] (slots 46-49)
+  BAR_IRING = 46,   // int {item, pair, h, b}[4] then float sink[4] (slots 46-55)
   BAR_EPI = 34,     // [2 X][2 Q buffers] softmax X warps -> the store thread: O rows
                     // staged in Q buffer b (one barrier per buffer, so a pipeline
                     // running an item ahead cannot complete a phase twice)
@@ -268,18 +268,22 @@ __global__ void __launch_bounds__(384, 1)
   sched.n_pairs = p.n_pairs;
   sched.n_items = p.n_pairs * sched.per_pair;
   sched.n_q = p.n_q;
-  volatile int* ring_item = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * BAR_IRING);
-  volatile float* ring_sink = reinterpret_cast<volatile float*>(smem + C::OFF_BAR + 8 * BAR_IRING + 16);
-  // Read item k of this CTA from the ring (all roles, in order); `elected`:
-  // whether this thread arrives on the slot's release barrier for its group.
-  // Returns n_items (no more work) on a timed-out wait.
-  auto fetch = [&](int k, bool elected, float& sink) -> int {
+  volatile int4* ring_item = reinterpret_cast<volatile int4*>(smem + C::OFF_BAR + 8 * BAR_IRING);
+  volatile float* ring_sink = reinterpret_cast<volatile float*>(smem + C::OFF_BAR + 8 * BAR_IRING + 64);
+  // Read item k of this CTA from the ring (all roles, in order): its id,
+  // coordinates and sink; `elected`: whether this thread arrives on the
+  // slot's release barrier for its group. Returns n_items (no more work) on a
+  // timed-out wait.
+  auto fetch = [&](int k, bool elected, int& pair, int& h, int& b, float& sink) -> int {
     const int sl = k & 3;
     if (!mbar_wait(bar(BAR_IFULL + sl), (uint32_t)((k >> 2) & 1))) {
       *abort_flag = 1;
       return sched.n_items;
     }
-    const int it = ring_item[sl];
+    const int it = ring_item[sl].x;
+    pair = ring_item[sl].y;
+    h = ring_item[sl].z;
+    b = ring_item[sl].w;
     sink = ring_sink[sl];
     __syncwarp(__activemask());
     if (elected) mbar_arrive(bar(BAR_IEMPTY + sl));
@@ -352,7 +356,10 @@ __global__ void __launch_bounds__(384, 1)
           sched.coords(item, pair, h, b);
           if (p.sinks) sink = p.sinks[h];
         }
-        ring_item[sl] = item;
+        ring_item[sl].x = item;
+        ring_item[sl].y = pair;
+        ring_item[sl].z = h;
+        ring_item[sl].w = b;
         ring_sink[sl] = sink;
         mbar_arrive(bar(BAR_IFULL + sl));   // release: the ring entry is visible to acquirers
         if (item >= sched.n_items) break;
@@ -380,7 +387,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int t = 0; t < geo.ntiles; ++t, ++gt) {
           const int s = gt % C::NS;
           const uint32_t ph = (uint32_t)((gt / C::NS) & 1);
-          const int krow = (int)(geo.base + (long long)BN * t);
+          const int krow = geo.base + BN * t;
           if (!mbar_wait(bar(BAR_KEMPTY + s), ph ^ 1)) { *abort_flag = 1; break; }
           mbar_arrive_expect_tx(bar(BAR_KFULL + s), C::KV_BYTES);
 #pragma unroll
@@ -420,10 +427,9 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = true;
       for (int rr = 0; ok; ++rr) {
         float sink_unused;
-        const int item = fetch(rr, true, sink_unused);
-        if (item >= sched.n_items) break;
         int pair, h, b;
-        sched.coords(item, pair, h, b);
+        const int item = fetch(rr, true, pair, h, b, sink_unused);
+        if (item >= sched.n_items) break;
         const TileGeom<BN> geo = make_geom<BN>(p, pair);
         const int sw = ItemSchedule::swap(rr);
 #pragma unroll
@@ -467,10 +473,9 @@ __global__ void __launch_bounds__(384, 1)
       int j = 0;           // items done by this CTA
       for (int rr = 0; ok; ++rr) {
         float sink_unused;
-        const int item = fetch(rr, true, sink_unused);
-        if (item >= sched.n_items) break;
         int pair, h, b;
-        sched.coords(item, pair, h, b);
+        const int item = fetch(rr, true, pair, h, b, sink_unused);
+        if (item >= sched.n_items) break;
         const TileGeom<BN> geo = make_geom<BN>(p, pair);
         const int qb = j & 1;
         if (!mbar_wait(bar(BAR_QFULL + qb), (uint32_t)((j >> 1) & 1))) { ok = false; break; }
@@ -543,10 +548,9 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int rr = 0; ok; ++rr) {
       float sink_raw;
-      const int item = fetch(rr, lane == 0, sink_raw);
-      if (item >= sched.n_items) break;
       int pair, h, b;
-      sched.coords(item, pair, h, b);
+      const int item = fetch(rr, lane == 0, pair, h, b, sink_raw);
+      if (item >= sched.n_items) break;
       const TileGeom<BN> geo = make_geom<BN>(p, pair);
       const int rt = X ^ ItemSchedule::swap(rr);   // row tile of this pipeline
       const int i = geo.i0 + 128 * rt + r;      // query row within the call
@@ -577,7 +581,7 @@ __global__ void __launch_bounds__(384, 1)
             // below key 0) of some row; each side is one compare + select
             // per column, skipped when no row of the tile needs it.
             // Positions fit in 32 bits (cap < 2^31).
-            const int klo = (int)geo.base + BN * t;
+            const int klo = geo.base + BN * t;
             const int p0 = (int)p.off + geo.i0 + 128 * rt;   // position of row 0
             const int ipos = (int)pos;
             if (klo + BN - 1 > p0) {
