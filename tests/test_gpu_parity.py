@@ -265,6 +265,20 @@ def test_decode_multi_split(cuda_device, over, layer):
     _decode_steps(cfg, cache, ocache, 3, window, cos, sin, rc, rs, sinks)
 
 
+@pytest.mark.parametrize("window", [1, 2, 127, 129], ids=["w1", "w2", "w127", "w129"])
+def test_prefill_and_decode_window_edges_mha(cuda_device, window):
+    # q_mult = 1 (plain multi-head) with band widths around the degenerate
+    # W = 1 (each row sees only itself and the sink) and the 128-key tile edge
+    cfg = wl.scaled(wl.CONFIGS["tiny"], B=2, n_q=4, n_kv=4, d=64)
+    out, lse, ref, ref_lse, cache, ocache = _run_prefill_case(cfg, 60, 420, window)
+    check_bf16_output(out, ref, f"mha W={window}")
+    check_lse(lse, ref_lse, f"mha W={window}")
+    cap = cache.raw.cap
+    cos, sin = _tables(cfg, cap)
+    rc, rs = oracle_tables(cfg, cap)
+    _decode_steps(cfg, cache, ocache, 3, window, cos, sin, rc, rs, wl.sinks(cfg).to(DEV))
+
+
 def test_decode_from_empty_cache_and_no_sink(cuda_device):
     cfg = wl.scaled(wl.CONFIGS["tiny"], B=2)
     cos, sin = _tables(cfg, 8)
