@@ -104,7 +104,7 @@ class Clocks:
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={q}",
-                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                       "--format=csv,noheader,nounits", "-lms", "20"],
                                       stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.p = None
@@ -434,19 +434,25 @@ def e2e_lite(step, steps, warmup):
 # ---------------------------------------------------------------------------
 
 def oracle_sample(budget_s=12.0, min_units=1):
-    """Times the fp64 oracle on a bounded sample of the Lite workload: whole
-    (sequence, query head) units of the full layer, T = 4096 rows each, until
-    the time budget is spent. Returns (TFLOP/s, cores, description)."""
-    import numpy as np
+    """Times the fp64 oracle on a bounded sample of the bench step: whole
+    (sequence, query head) units, each the step's work for that unit -- both
+    layers (band and full causal), prefill of T rows and the decode row, i.e.
+    T + 1 rows per layer (the decode row attends exactly like a prefill row
+    at position T) -- until the time budget is spent. Returns (TFLOP/s,
+    cores, description)."""
     from oracle import attention as oatt
     from oracle import rope as orope
     from oracle import yarn as oyarn
     cfg = wl.CONFIGS[WORKLOAD]
     y = cfg.yarn
-    cos, sin = oyarn.stored_tables(cfg.T, cfg.d, y["theta"], y["scaling"], y["orig_ctx"], y["alpha"], y["beta"])
-    q, k, v = wl.qkv(cfg, cfg.T, layer=1)
-    sinks = wl.sinks(cfg, 1).double().numpy()
-    qn, kn, vn = (t.to(torch.float64).numpy() for t in (q, k, v))
+    n = cfg.T + 1
+    cos, sin = oyarn.stored_tables(n, cfg.d, y["theta"], y["scaling"], y["orig_ctx"], y["alpha"], y["beta"])
+    layers = []
+    for layer in range(2):
+        q, k, v = wl.qkv(cfg, n, layer=layer)
+        layers.append(dict(window=cfg.layer_window(layer), sinks=wl.sinks(cfg, layer).double().numpy(),
+                           q=q.to(torch.float64).numpy(), k=k.to(torch.float64).numpy(),
+                           v=v.to(torch.float64).numpy()))
     done = 0
     t0 = time.perf_counter()
     units = 0
@@ -454,18 +460,30 @@ def oracle_sample(budget_s=12.0, min_units=1):
         b, h = divmod(units, cfg.n_q)
         b %= cfg.B
         g = h // cfg.q_mult
-        qr = orope.rotate_bsh(qn[b:b + 1, :, h:h + 1], 0, cos, sin)
-        kr = orope.rotate_bsh(kn[b:b + 1, :, g:g + 1], 0, cos, sin)
-        oatt.sink_attention(qr, kr, vn[b:b + 1, :, g:g + 1], sinks[h:h + 1], 0, 0, cfg.sm_scale)
+        for L in layers:
+            qr = orope.rotate_bsh(L["q"][b:b + 1, :, h:h + 1], 0, cos, sin)
+            kr = orope.rotate_bsh(L["k"][b:b + 1, :, g:g + 1], 0, cos, sin)
+            oatt.sink_attention(qr, kr, L["v"][b:b + 1, :, g:g + 1], L["sinks"][h:h + 1], 0, L["window"],
+                                cfg.sm_scale)
+            done += 4 * cfg.d * pairs(0, n, L["window"])
         units += 1
-        done += 4 * cfg.d * pairs(0, cfg.T, 0)
         if units >= min_units and time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
     threads = int(os.environ.get("OMP_NUM_THREADS", "0")) or os.cpu_count()
-    desc = (f"fp64 numpy oracle, full-causal layer of the Lite workload: {units} (sequence, head) "
-            f"units x {cfg.T} rows x up to {cfg.T} keys (RoPE included), {dt:.1f} s")
+    desc = (f"fp64 numpy oracle on {units} of the step's {cfg.B * cfg.n_q} (sequence, head) units: both layers "
+            f"(W={cfg.window} band, full causal), {cfg.T} prefill rows + the decode row each, RoPE included, "
+            f"{dt:.1f} s")
     return done / dt / 1e12, threads, desc
+
+
+def step_config(cfg, world, parallelism):
+    """The bench step's workload, the same for both arms."""
+    return {"workload": "GPT-OSS-Lite attention: B=8, T=4096 prefill + 1 decode row, "
+                        "n_q=8, n_kv=4, d=96, W=128 band layer + full causal layer, "
+                        "YaRN theta=150000 s=32 from 4096",
+            "global_batch": cfg.B * world, "seq_len": cfg.T, "parallelism": parallelism,
+            "l2": "inputs larger than L2 (step working set ~300 MB > 126 MB)"}
 
 
 def run_reference(args, rank, world):
@@ -485,8 +503,7 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": (time.perf_counter() - t_all) * 1e3 / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": "GPT-OSS-Lite attention prefill (B=8, T=4096, 8/4 heads, d=96), full layer",
-                       "global_batch": cfg.B, "seq_len": cfg.T, "parallelism": "none (host oracle)"},
+            "config": step_config(cfg, 1, "none (host oracle)"),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -619,11 +636,7 @@ def main():
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) bf16 q/k/v, N(0,0.25) fp32 sinks)",
-            "config": {"workload": "GPT-OSS-Lite attention: B=8, T=4096 prefill + 1 decode row, "
-                                   "n_q=8, n_kv=4, d=96, W=128 band layer + full causal layer, "
-                                   "YaRN theta=150000 s=32 from 4096",
-                       "global_batch": cfg.B * world, "seq_len": cfg.T, "parallelism": f"dp{world}",
-                       "l2": "inputs larger than L2 (step working set ~300 MB > 126 MB)"},
+            "config": step_config(cfg, world, f"dp{world}"),
             "roofline": {"bound": "tensor", "kernel": "prefill_kernel (full-causal layer attention; the staging launch before it is not included)",
                          "achieved": round(full_tf, 2), "peak": peaks["tf"], "unit": "TFLOP/s",
                          "frac": round(full_tf / peaks["tf"], 4), "traffic": traffic,
