@@ -185,21 +185,22 @@ class LiteStep:
                                              float(self.yarn[3]), float(self.yarn[4]), S._stream(self.cos)),
                  "sa_yarn_rope_tables")
 
-    def run(self, ev_full=None, q_in=None):
+    def run(self, ev_full=None, q_in=None, outs=None):
         sa, cfg, T = self.sa, self.cfg, self.cfg.T
         self.tables()
         for li, L in enumerate(self.layers):
             c = L["cache"]
             c.restore(L["snap"])
             q, k, v = (L["q"], L["k"], L["v"]) if q_in is None else q_in[li]
+            out, dec = (L["out"], L["dec"]) if outs is None else outs[li]
             if ev_full is not None and L["window"] == 0:
                 sa.set_prefill_events(*ev_full)   # around the attention kernel alone
             sa.attn_prefill(c, q[:, :T], k[:, :T], v[:, :T], L["sinks"], L["window"], cfg.sm_scale,
-                            self.cos, self.sin, out=L["out"])
+                            self.cos, self.sin, out=out)
             if ev_full is not None and L["window"] == 0:
                 sa.set_prefill_events()
             sa.attn_decode(c, q[:, T:], k[:, T:], v[:, T:], L["sinks"], L["window"], cfg.sm_scale,
-                           self.cos, self.sin, workspace=L["ws"], out=L["dec"])
+                           self.cos, self.sin, workspace=L["ws"], out=dec)
 
 
 def _time_loop(fn, steps, warmup, dist=None):
@@ -402,31 +403,66 @@ def long_decode(dev, peaks, steps=8, layers=24):
 
 
 def e2e_lite(step, steps, warmup):
-    """Same step through host buffers: pinned host -> device copies of the
-    step's q/k/v every step, and the outputs read back to host."""
+    """Same step through host buffers: every step copies its q/k/v from pinned
+    host memory to the device and reads both layers' outputs back to pinned
+    host memory. Steps are pipelined over three streams (host-to-device copies,
+    compute, device-to-host copies) with two buffer sets, so one step's copies
+    overlap its neighbours' work, as a serving loop would run; the timed
+    region spans the first step's first copy to the last step's last copy."""
     cfg = step.cfg
-    host_in, dev_in = [], []
+    host_in, dev_in, dev_out, host_out = [], [], [], []
     h2d = d2h = 0
     for L in step.layers:
         hq, hk, hv = (L[n].cpu().pin_memory() for n in ("q", "k", "v"))
         host_in.append((hq, hk, hv))
-        dev_in.append(tuple(torch.empty_like(L[n]) for n in ("q", "k", "v")))
         h2d += sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-    host_out = [(torch.empty(L["out"].shape, dtype=torch.bfloat16).pin_memory(),
-                 torch.empty(L["dec"].shape, dtype=torch.bfloat16).pin_memory()) for L in step.layers]
-    d2h = sum(a.numel() * 2 + b.numel() * 2 for a, b in host_out)
+    for _ in range(2):
+        dev_in.append([tuple(torch.empty_like(L[n]) for n in ("q", "k", "v")) for L in step.layers])
+        dev_out.append([(torch.empty_like(L["out"]), torch.empty_like(L["dec"])) for L in step.layers])
+        host_out.append([(torch.empty(L["out"].shape, dtype=torch.bfloat16).pin_memory(),
+                          torch.empty(L["dec"].shape, dtype=torch.bfloat16).pin_memory()) for L in step.layers])
+    d2h = sum(a.numel() * 2 + b.numel() * 2 for a, b in host_out[0])
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    computed = [ev(), ev()]   # set s: its inputs are consumed
+    landed = [ev(), ev()]     # set s: its inputs are on the device
+    read = [ev(), ev()]       # set s: its outputs are on the host
+    used = [False, False]
 
-    def fn():
-        for (hq, hk, hv), (dq, dk, dv) in zip(host_in, dev_in):
-            dq.copy_(hq, non_blocking=True)
-            dk.copy_(hk, non_blocking=True)
-            dv.copy_(hv, non_blocking=True)
-        step.run(q_in=dev_in)
-        for L, (ho, hd) in zip(step.layers, host_out):
-            ho.copy_(L["out"], non_blocking=True)
-            hd.copy_(L["dec"], non_blocking=True)
-    ms = _time_loop(fn, steps, warmup)
-    return ms / steps, h2d, d2h
+    def run(n, first=None, last=None):
+        for i in range(n):
+            st = i % 2
+            with torch.cuda.stream(s_in):
+                if used[st]:
+                    s_in.wait_event(computed[st])
+                if i == 0 and first is not None:
+                    first.record(s_in)
+                for (hq, hk, hv), (dq, dk, dv) in zip(host_in, dev_in[st]):
+                    dq.copy_(hq, non_blocking=True)
+                    dk.copy_(hk, non_blocking=True)
+                    dv.copy_(hv, non_blocking=True)
+                landed[st].record(s_in)
+            with torch.cuda.stream(s_comp):
+                s_comp.wait_event(landed[st])
+                if used[st]:
+                    s_comp.wait_event(read[st])
+                step.run(q_in=dev_in[st], outs=dev_out[st])
+                computed[st].record(s_comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(computed[st])
+                for (ho, hd), (do, dd) in zip(host_out[st], dev_out[st]):
+                    ho.copy_(do, non_blocking=True)
+                    hd.copy_(dd, non_blocking=True)
+                read[st].record(s_out)
+                if i == n - 1 and last is not None:
+                    last.record(s_out)
+            used[st] = True
+        torch.cuda.synchronize()
+
+    run(warmup)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    run(steps, e0, e1)
+    return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
 # ---------------------------------------------------------------------------
