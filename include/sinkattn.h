@@ -205,7 +205,10 @@ sa_status sa_kv_restore(sa_kv_cache* cache, const sa_snapshot* snap);
  * [B][T][n_q][d] view) and each output tile overwrites its own staged query
  * rows, so `out` may be `q` itself but must not overlap k, v, the cache, the
  * sinks, the tables or lse otherwise. Two launches on `stream` (staging,
- * attention).
+ * attention). The attention kernel schedules its work items from a device
+ * counter; the library keeps 64 such counters per device and hands them out
+ * round robin, so at most 64 prefill calls may be in flight on one device at
+ * a time (across all streams).
  */
 sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* args, sa_stream_t stream);
 
