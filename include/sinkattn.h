@@ -73,8 +73,15 @@ typedef enum sa_status {
  *        decode stores rotated K and unchanged V).
  * offset: rows [0, offset) are valid. Host-authoritative: the library updates
  *        it when an append is enqueued.
+ * ring  : 0 for the linear cache above (position j in row j, offset <= cap).
+ *        > 0 for a ring cache serving band layers of exactly `ring` keys
+ *        (the pages' sliding-window KV reduction; MoE-Xtend README, "KV
+ *        CACHE" sizing): position p lives in row p mod cap, positions are
+ *        unbounded, and the cache holds the last cap positions (cap a
+ *        multiple of 384, cap >= ring). Calls on a ring cache must use
+ *        window == ring. Initialise with sa_kv_cache_init_ring.
  * The remaining fields are bookkeeping for snapshot/restore; initialise the
- * whole struct with sa_kv_cache_init and do not edit them.
+ * whole struct with sa_kv_cache_init (or _ring) and do not edit them.
  */
 typedef struct sa_kv_cache {
   void* k;
@@ -88,6 +95,7 @@ typedef struct sa_kv_cache {
   int32_t log_len;
   int64_t log_floor_seq; /* summary of entries dropped from the full log: */
   int64_t log_floor_row; /* latest dropped seq, lowest dropped row        */
+  int32_t ring;          /* 0: linear; > 0: ring cache for `ring`-key bands */
 } sa_kv_cache;
 
 typedef struct sa_snapshot {
@@ -168,6 +176,20 @@ sa_status sa_rope_apply_qk(void* q, const int64_t q_strides[3], void* k, const i
 /* Initialise a cache descriptor over caller-owned K/V buffers (offset 0). */
 sa_status sa_kv_cache_init(sa_kv_cache* cache, void* k, void* v, int32_t B, int32_t cap,
                            int32_t n_kv, int32_t d);
+
+/*
+ * Ring cache for band layers of `window` keys (see `ring` above): k, v as
+ * for sa_kv_cache_init with cap rows per (sequence, KV head), cap a multiple
+ * of 384 and >= window (SA_ERR_SHAPE otherwise). The buffers must be zeroed
+ * before first use (rows never written are read, masked, by the kernels).
+ * Appends of T rows need T <= cap; a prefill of T rows needs
+ * T + window - 1 <= cap (the keys of the call's first row must survive the
+ * call's own appends); otherwise SA_ERR_CAPACITY. A snapshot can be restored
+ * while the rows its band needs, positions [offset - window + 1, offset),
+ * have not been overwritten (else SA_ERR_STALE_SNAPSHOT).
+ */
+sa_status sa_kv_cache_init_ring(sa_kv_cache* cache, void* k, void* v, int32_t B, int32_t cap,
+                                int32_t n_kv, int32_t d, int32_t window);
 
 /*
  * Append T already-rotated K rows and V rows at [offset, offset+T), then

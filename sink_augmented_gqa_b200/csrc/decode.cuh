@@ -44,7 +44,9 @@ struct DecodeParams {
   const float* sin_t;
   int B, n_q, n_kv, q_mult;
   long long off;    // position of the new row == cache rows before it
-  long long lo;     // first cache row attended
+  long long lo;     // first cache position of split 0's first stage
+  long long lo_mask;  // first cache position attended (keys before it masked)
+  int ring_cap;     // 0: row = position; > 0: ring cache, row = position mod ring_cap
   long long chunk;  // cache rows per split (multiple of 64)
   int S;
   float scale_log2;
@@ -82,10 +84,12 @@ struct DecodeCfg {
 };
 
 // Warp-level processing of one 16-key sub-tile (rows row0..row0+15 of a tile
-// stored as swizzled column blocks of `block_bytes`), keys >= n_valid masked.
+// stored as swizzled column blocks of `block_bytes`), keys < n_first and
+// keys >= n_valid masked.
 template <int D>
 __device__ __forceinline__ void decode_subtile(uint32_t kbase, uint32_t vbase, uint32_t block_bytes,
-                                               int row0, int n_valid, const uint32_t (&qf)[D / 16][2],
+                                               int row0, int n_first, int n_valid,
+                                               const uint32_t (&qf)[D / 16][2],
                                                float scale_log2, float (&m)[2], float (&l)[2],
                                                float (&o)[D / 16][4], int lane) {
   using C = DecodeCfg<D>;
@@ -99,10 +103,11 @@ __device__ __forceinline__ void decode_subtile(uint32_t kbase, uint32_t vbase, u
   }
   const int key_a = lane >> 2, key_b = key_a + 8;
   float s[4];
-  s[0] = key_a < n_valid ? c[0] * scale_log2 : -INFINITY;
-  s[1] = key_a < n_valid ? c[1] * scale_log2 : -INFINITY;
-  s[2] = key_b < n_valid ? c[2] * scale_log2 : -INFINITY;
-  s[3] = key_b < n_valid ? c[3] * scale_log2 : -INFINITY;
+  const bool va = key_a >= n_first && key_a < n_valid, vb = key_b >= n_first && key_b < n_valid;
+  s[0] = va ? c[0] * scale_log2 : -INFINITY;
+  s[1] = va ? c[1] * scale_log2 : -INFINITY;
+  s[2] = vb ? c[2] * scale_log2 : -INFINITY;
+  s[3] = vb ? c[3] * scale_log2 : -INFINITY;
   float pr[4];
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
@@ -136,7 +141,7 @@ __device__ __forceinline__ void decode_subtile(uint32_t kbase, uint32_t vbase, u
 }
 
 template <int D>
-__global__ void __launch_bounds__(288)
+__global__ void __launch_bounds__(288, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const DecodeParams p) {
   using C = DecodeCfg<D>;
@@ -185,7 +190,8 @@ __global__ void __launch_bounds__(288)
         const int s = it % C::NS;
         if (!mbar_wait(empty_bar(s), (uint32_t)(((it / C::NS) & 1) ^ 1))) { flag[0] = 1; break; }
         mbar_arrive_expect_tx(full_bar(s), 2 * C::STAGE_BYTES);
-        const int row = (int)(r_begin + (long long)it * C::R);
+        const long long pos = r_begin + (long long)it * C::R;   // stages never wrap a ring
+        const int row = (int)(p.ring_cap > 0 ? pos % p.ring_cap : pos);
 #pragma unroll
         for (int cb = 0; cb < C::NCB; ++cb) {
           tma_load_4d(sbase + C::OFF_K + s * C::STAGE_BYTES + cb * C::BLOCK_BYTES, &tmK, full_bar(s),
@@ -248,8 +254,9 @@ __global__ void __launch_bounds__(288)
     uint8_t* xv = smem + C::OFF_XV;
     const __nv_bfloat16* krow = p.k + b * p.ks0 + (long long)g * p.ks2;
     const __nv_bfloat16* vrow = p.v + b * p.vs0 + (long long)g * p.vs2;
-    __nv_bfloat16* ckrow = p.ck + (((long long)b * p.n_kv + g) * p.cap + p.off) * D;
-    __nv_bfloat16* cvrow = p.cv + (((long long)b * p.n_kv + g) * p.cap + p.off) * D;
+    const long long slot = p.ring_cap > 0 ? p.off % p.ring_cap : p.off;
+    __nv_bfloat16* ckrow = p.ck + (((long long)b * p.n_kv + g) * p.cap + slot) * D;
+    __nv_bfloat16* cvrow = p.cv + (((long long)b * p.n_kv + g) * p.cap + slot) * D;
     // zero rows 1..15 (and row 0, overwritten below)
     for (int idx = lane; idx < (int)(C::XTILE / 16); idx += 32) {
       reinterpret_cast<uint4*>(xk)[idx] = make_uint4(0, 0, 0, 0);
@@ -283,15 +290,16 @@ __global__ void __launch_bounds__(288)
     if (!mbar_wait(full_bar(s), (uint32_t)((it / C::NS) & 1))) { flag[0] = 1; break; }
     const long long row0 = r_begin + (long long)it * C::R + 16 * warp;
     const long long nv = r_end - row0;
-    if (nv > 0 && !flag[0])
+    const long long nf = p.lo_mask - row0;
+    if (nv > 0 && nf < 16 && !flag[0])
       decode_subtile<D>(sbase + C::OFF_K + s * C::STAGE_BYTES, sbase + C::OFF_V + s * C::STAGE_BYTES,
-                        C::BLOCK_BYTES, 16 * warp, nv > 16 ? 16 : (int)nv, qf, p.scale_log2, m, l, o,
-                        lane);
+                        C::BLOCK_BYTES, 16 * warp, nf > 0 ? (int)nf : 0, nv > 16 ? 16 : (int)nv, qf,
+                        p.scale_log2, m, l, o, lane);
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));
   }
   if (last_split && warp == 0)
-    decode_subtile<D>(sbase + C::OFF_XK, sbase + C::OFF_XV, C::XBLOCK, 0, 1, qf, p.scale_log2, m, l,
+    decode_subtile<D>(sbase + C::OFF_XK, sbase + C::OFF_XV, C::XBLOCK, 0, 0, 1, qf, p.scale_log2, m, l,
                       o, lane);
 
   // ---------------------------------------------------------------- merge the consumer warps

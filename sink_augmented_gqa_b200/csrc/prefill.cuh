@@ -62,6 +62,7 @@ struct PrefillParams {
   int rope;
   int n_pairs;
   int sched_slot;   // which counter pair of g_prefill_sched this launch uses
+  int ring_cap;     // 0: cache row = position; > 0: ring cache, row = position mod ring_cap
 };
 
 // Work counters of the dynamic item schedule, one pair per launch slot (the
@@ -149,7 +150,9 @@ struct ItemSchedule {
   }
 };
 
-__device__ __forceinline__ long long floordiv(long long a, long long b) {  // b > 0
+// Positions (offset + row) fit in 32 bits: the cache capacity and every
+// offset are below 2^31.
+__device__ __forceinline__ int floordiv(int a, int b) {  // b > 0
   return a >= 0 ? a / b : -((-a + b - 1) / b);
 }
 
@@ -161,18 +164,18 @@ __device__ __forceinline__ long long floordiv(long long a, long long b) {  // b 
 //                 no mask is applied there.
 template <int BN>
 struct TileGeom {
-  long long off;
+  int off;
   int T, window;
   int i0;          // first query row of tile A
-  long long base;  // first key of key tile 0
+  int base;        // first key of key tile 0
   int ntiles;
   int a_lo[2], a_hi[2], f_lo[2], f_hi[2];
   __device__ __forceinline__ bool valid(int X) const { return i0 + 128 * X < T; }
-  __device__ __forceinline__ long long lo(int X) const {
-    const long long p0 = off + i0 + 128 * X;
+  __device__ __forceinline__ int lo(int X) const {
+    const int p0 = off + i0 + 128 * X;
     return window > 0 ? (p0 - window + 1 > 0 ? p0 - window + 1 : 0) : 0;
   }
-  __device__ __forceinline__ long long hi(int X) const {  // exclusive
+  __device__ __forceinline__ int hi(int X) const {  // exclusive
     const int last = min(T, i0 + 128 * X + 128);
     return off + last;
   }
@@ -183,16 +186,22 @@ struct TileGeom {
 template <int BN>
 __device__ __forceinline__ TileGeom<BN> make_geom(const PrefillParams& p, int pair) {
   TileGeom<BN> g;
-  g.off = p.off;
+  g.off = (int)p.off;
   g.T = p.T;
   g.window = p.window;
   g.i0 = pair * 256;
-  const long long diag = p.off + g.i0;
-  const long long loA = g.lo(0);
-  const long long nb = (diag - loA + BN - 1) / BN;
-  g.base = diag - (long long)BN * nb;
-  const long long hi = p.off + min(p.T, g.i0 + 256);
-  g.ntiles = (int)((hi - g.base + BN - 1) / BN);
+  const int diag = g.off + g.i0;
+  const int loA = g.lo(0);
+  if (p.ring_cap > 0) {
+    // ring cache: key tiles start at multiples of BN, so none wraps around
+    g.base = floordiv(loA, BN) * BN;
+  } else {
+    // key tiles aligned to tile A's diagonal: one masked tile per query tile
+    const int nb = (diag - loA + BN - 1) / BN;
+    g.base = diag - BN * nb;
+  }
+  const int hi = g.off + min(p.T, g.i0 + 256);
+  g.ntiles = (hi - g.base + BN - 1) / BN;
 #pragma unroll
   for (int X = 0; X < 2; ++X) {
     if (!g.valid(X)) {
@@ -200,20 +209,20 @@ __device__ __forceinline__ TileGeom<BN> make_geom(const PrefillParams& p, int pa
       continue;
     }
     // active: klo < hi(X) and klo + BN > lo(X)
-    const long long alo = floordiv(g.lo(X) - g.base, BN);
-    const long long ahi = floordiv(g.hi(X) - g.base + BN - 1, BN);
-    g.a_lo[X] = (int)(alo < 0 ? 0 : alo);
-    g.a_hi[X] = (int)(ahi > g.ntiles ? g.ntiles : ahi);
+    const int alo = floordiv(g.lo(X) - g.base, BN);
+    const int ahi = floordiv(g.hi(X) - g.base + BN - 1, BN);
+    g.a_lo[X] = alo < 0 ? 0 : alo;
+    g.a_hi[X] = ahi > g.ntiles ? g.ntiles : ahi;
     // full: klo >= 0, klo + BN - 1 <= p0, and (band) klo > p0 + 127 - W
-    const long long p0 = p.off + g.i0 + 128 * X;
-    long long flo = floordiv(-g.base + BN - 1, BN);
+    const int p0 = g.off + g.i0 + 128 * X;
+    int flo = floordiv(-g.base + BN - 1, BN);
     if (p.window > 0) {
-      const long long w = floordiv(p0 + 127 - p.window - g.base, BN) + 1;
+      const int w = floordiv(p0 + 127 - p.window - g.base, BN) + 1;
       if (w > flo) flo = w;
     }
-    const long long fhi = floordiv(p0 - BN + 1 - g.base, BN) + 1;
-    g.f_lo[X] = (int)(flo < g.a_lo[X] ? g.a_lo[X] : (flo > g.a_hi[X] ? g.a_hi[X] : flo));
-    g.f_hi[X] = (int)(fhi > g.a_hi[X] ? g.a_hi[X] : (fhi < g.f_lo[X] ? g.f_lo[X] : fhi));
+    const int fhi = floordiv(p0 - BN + 1 - g.base, BN) + 1;
+    g.f_lo[X] = flo < g.a_lo[X] ? g.a_lo[X] : (flo > g.a_hi[X] ? g.a_hi[X] : flo);
+    g.f_hi[X] = fhi > g.a_hi[X] ? g.a_hi[X] : (fhi < g.f_lo[X] ? g.f_lo[X] : fhi);
   }
   return g;
 }
@@ -387,7 +396,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int t = 0; t < geo.ntiles; ++t, ++gt) {
           const int s = gt % C::NS;
           const uint32_t ph = (uint32_t)((gt / C::NS) & 1);
-          const int krow = geo.base + BN * t;
+          const int kpos = geo.base + BN * t;
+          const int krow = p.ring_cap > 0 ? kpos % p.ring_cap : kpos;
           if (!mbar_wait(bar(BAR_KEMPTY + s), ph ^ 1)) { *abort_flag = 1; break; }
           mbar_arrive_expect_tx(bar(BAR_KFULL + s), C::KV_BYTES);
 #pragma unroll

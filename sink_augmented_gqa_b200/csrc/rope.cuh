@@ -88,7 +88,7 @@ __global__ void kv_append_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat16* 
                                  long long vs0, long long vs1, long long vs2, int B, int T,
                                  int n_kv, int d, long long off, int rope,
                                  const float* __restrict__ cos_t,
-                                 const float* __restrict__ sin_t) {
+                                 const float* __restrict__ sin_t, int ring) {
   const int half = d / 2, chunks = half / 8;
   const long long n = (long long)B * T * n_kv * chunks;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
@@ -105,7 +105,7 @@ __global__ void kv_append_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat16* 
     uint4 c = *reinterpret_cast<const uint4*>(krow + half + ch * 8);
     const long long p = off + t;
     if (rope) rotate8(a, c, cos_t + p * half + ch * 8, sin_t + p * half + ch * 8);
-    const long long dst = (((long long)b * n_kv + g) * cap + p) * d;
+    const long long dst = (((long long)b * n_kv + g) * cap + (ring ? p % cap : p)) * d;
     *reinterpret_cast<uint4*>(ck + dst + ch * 8) = a;
     *reinterpret_cast<uint4*>(ck + dst + half + ch * 8) = c;
     *reinterpret_cast<uint4*>(cv + dst + ch * 8) = *reinterpret_cast<const uint4*>(vrow + ch * 8);
@@ -114,6 +114,8 @@ __global__ void kv_append_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat16* 
   }
 }
 
+// Both this kernel and kv_append_kernel write position p of a ring cache
+// (ring != 0) to row p mod cap, else to row p.
 // Prefill staging, one launch: the kv_append_kernel work for the call's K/V
 // rows, then (stage_q) each query row rotated at its position off + t into
 // qo [B][T][n_q][d] (strides os*), from which the attention kernel reads its
@@ -126,7 +128,7 @@ __global__ void prefill_stage_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat
                                      const float* __restrict__ cos_t, const float* __restrict__ sin_t,
                                      const __nv_bfloat16* q, long long qs0, long long qs1,
                                      long long qs2, int n_q, __nv_bfloat16* qo, long long os0,
-                                     long long os1, long long os2, int stage_q) {
+                                     long long os1, long long os2, int stage_q, int ring) {
   const int half = d / 2, chunks = half / 8;
   const long long n_kv_units = (long long)B * T * n_kv * chunks;
   const long long n = n_kv_units + (stage_q ? (long long)B * T * n_q * chunks : 0);
@@ -145,7 +147,7 @@ __global__ void prefill_stage_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat
       uint4 c = *reinterpret_cast<const uint4*>(krow + half + ch * 8);
       const long long p = off + t;
       if (rope) rotate8(a, c, cos_t + p * half + ch * 8, sin_t + p * half + ch * 8);
-      const long long dst = (((long long)b * n_kv + g) * cap + p) * d;
+      const long long dst = (((long long)b * n_kv + g) * cap + (ring ? p % cap : p)) * d;
       *reinterpret_cast<uint4*>(ck + dst + ch * 8) = a;
       *reinterpret_cast<uint4*>(ck + dst + half + ch * 8) = c;
       *reinterpret_cast<uint4*>(cv + dst + ch * 8) = *reinterpret_cast<const uint4*>(vrow + ch * 8);

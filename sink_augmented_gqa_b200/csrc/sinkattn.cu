@@ -35,6 +35,10 @@ bool strides_ok(const int64_t s[3]) {
 
 bool head_dim_ok(int d) { return d == 64 || d == 96 || d == 128; }
 
+// Ring capacity granule: a multiple of every key-tile height the kernels use
+// (128 decode rows; 128, 96, 64 prefill keys), so no tile wraps around.
+constexpr int kRingQuantum = 384;
+
 int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -132,6 +136,12 @@ sa_status check_cache(const sa_kv_cache* c) {
   if (c->B < 1 || c->cap < 1 || c->n_kv < 1) return SA_ERR_INVALID_ARG;
   if (!head_dim_ok(c->d)) return SA_ERR_SHAPE;
   if (!aligned16(c->k) || !aligned16(c->v)) return SA_ERR_INVALID_ARG;
+  if (c->ring < 0) return SA_ERR_INVALID_ARG;
+  if (c->ring > 0) {
+    if (c->cap % kRingQuantum != 0 || c->ring > c->cap) return SA_ERR_SHAPE;
+    if (c->offset < 0 || c->offset > INT32_MAX - 1) return SA_ERR_INVALID_ARG;
+    return SA_OK;
+  }
   if (c->offset < 0 || c->offset > c->cap) return SA_ERR_INVALID_ARG;
   return SA_OK;
 }
@@ -153,7 +163,13 @@ sa_status check_attn(const sa_kv_cache* c, const sa_attn_args* a) {
       !strides_ok(a->out_strides))
     return SA_ERR_INVALID_ARG;
   if (!(a->sm_scale > 0.f) || !isfinite(a->sm_scale)) return SA_ERR_INVALID_ARG;
-  if (a->offset + (int64_t)a->T > (int64_t)c->cap) return SA_ERR_CAPACITY;
+  if (c->ring > 0) {
+    if (a->window != c->ring) return SA_ERR_INVALID_ARG;
+    if ((int64_t)a->T + c->ring - 1 > (int64_t)c->cap) return SA_ERR_CAPACITY;
+    if (a->offset + (int64_t)a->T > (int64_t)INT32_MAX) return SA_ERR_CAPACITY;
+  } else if (a->offset + (int64_t)a->T > (int64_t)c->cap) {
+    return SA_ERR_CAPACITY;
+  }
   if (a->rope_fused) {
     if (a->cos == nullptr || a->sin == nullptr || !aligned16(a->cos) || !aligned16(a->sin))
       return SA_ERR_INVALID_ARG;
@@ -171,7 +187,8 @@ template <int D>
 sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream_t stream) {
   using Cfg = PrefillCfg<D>;
   CUtensorMap tmQ, tmK, tmV;
-  const long long rows = a->offset + a->T;
+  // a ring exposes all of its rows (positions outside the band are masked)
+  const long long rows = c->ring > 0 ? (long long)c->cap : a->offset + a->T;
   // Query tiles come from the staged (rotated) copy in `out` when RoPE is
   // fused, else straight from q; the kernel overwrites each staged tile with
   // its output rows only after it has read it.
@@ -209,6 +226,7 @@ sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream
   p.scale_log2 = a->sm_scale * 1.4426950408889634f;
   p.rope = a->rope_fused ? 1 : 0;
   p.n_pairs = (a->T + 255) / 256;
+  p.ring_cap = c->ring > 0 ? c->cap : 0;
   // Launches take the dynamic-schedule counter pairs round robin; a pair is
   // reset by the last CTA of its launch, so up to kPrefillSchedSlots
   // launches may be in flight at once on one device.
@@ -260,7 +278,10 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   const int q_mult = a->n_q / c->n_kv;
   DecodeParams p;
   p.off = a->offset;
-  p.lo = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
+  p.lo_mask = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
+  // a ring's stages start at multiples of the stage height so that none wraps
+  p.ring_cap = c->ring > 0 ? c->cap : 0;
+  p.lo = p.ring_cap > 0 ? p.lo_mask / Cfg::R * Cfg::R : p.lo_mask;
   const long long n_cache = p.off - p.lo;
   const DecodeSplit sp = decode_split(a->B, c->n_kv, n_cache);
   p.S = sp.S;
@@ -273,8 +294,9 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   memset(&tmK, 0, sizeof(tmK));
   memset(&tmV, 0, sizeof(tmV));
   if (n_cache > 0) {
-    if (!make_cache_map(&tmK, c->k, D, c->n_kv, p.off, c->cap, c->B, Cfg::R, Cfg::CB) ||
-        !make_cache_map(&tmV, c->v, D, c->n_kv, p.off, c->cap, c->B, Cfg::R, Cfg::CB))
+    const long long rows = p.ring_cap > 0 ? (long long)c->cap : p.off;
+    if (!make_cache_map(&tmK, c->k, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::CB) ||
+        !make_cache_map(&tmV, c->v, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::CB))
       return SA_ERR_CUDA;
   }
   p.q = static_cast<const __nv_bfloat16*>(a->q);
@@ -327,7 +349,7 @@ sa_status launch_append(sa_kv_cache* c, const void* k, const int64_t ks[3], cons
       static_cast<__nv_bfloat16*>(c->k), static_cast<__nv_bfloat16*>(c->v), c->cap,
       static_cast<const __nv_bfloat16*>(k), ks[0], ks[1], ks[2],
       static_cast<const __nv_bfloat16*>(v), vs[0], vs[1], vs[2], c->B, T, c->n_kv, c->d, c->offset,
-      rope, cos_t, sin_t);
+      rope, cos_t, sin_t, c->ring > 0 ? 1 : 0);
   return last_launch_status();
 }
 
@@ -347,7 +369,7 @@ sa_status launch_stage(sa_kv_cache* c, const sa_attn_args* a, cudaStream_t strea
       c->B, a->T, c->n_kv, c->d, c->offset, a->rope_fused ? 1 : 0, a->cos, a->sin,
       static_cast<const __nv_bfloat16*>(a->q), a->q_strides[0], a->q_strides[1], a->q_strides[2],
       a->n_q, static_cast<__nv_bfloat16*>(a->out), a->out_strides[0], a->out_strides[1],
-      a->out_strides[2], stage_q);
+      a->out_strides[2], stage_q, c->ring > 0 ? 1 : 0);
   return last_launch_status();
 }
 
@@ -453,6 +475,15 @@ sa_status sa_kv_cache_init(sa_kv_cache* cache, void* k, void* v, int32_t B, int3
   return check_cache(cache);
 }
 
+sa_status sa_kv_cache_init_ring(sa_kv_cache* cache, void* k, void* v, int32_t B, int32_t cap,
+                                int32_t n_kv, int32_t d, int32_t window) {
+  if (cache == nullptr || window < 1) return SA_ERR_INVALID_ARG;
+  sa_status st = sa_kv_cache_init(cache, k, v, B, cap, n_kv, d);
+  if (st != SA_OK) return st;
+  cache->ring = window;
+  return check_cache(cache);
+}
+
 sa_status sa_kv_append(sa_kv_cache* cache, const void* k_rot, const int64_t k_strides[3],
                        const void* v, const int64_t v_strides[3], int32_t T, sa_stream_t stream) {
   sa_status st = check_cache(cache);
@@ -462,7 +493,9 @@ sa_status sa_kv_append(sa_kv_cache* cache, const void* k_rot, const int64_t k_st
   if (k_rot == nullptr || v == nullptr || !aligned16(k_rot) || !aligned16(v) ||
       !strides_ok(k_strides) || !strides_ok(v_strides))
     return SA_ERR_INVALID_ARG;
-  if (cache->offset + (int64_t)T > (int64_t)cache->cap) return SA_ERR_CAPACITY;
+  if (cache->ring > 0 ? (T > cache->cap || cache->offset + (int64_t)T > (int64_t)INT32_MAX)
+                      : cache->offset + (int64_t)T > (int64_t)cache->cap)
+    return SA_ERR_CAPACITY;
   st = launch_append(cache, k_rot, k_strides, v, v_strides, T, 0, nullptr, nullptr,
                      (cudaStream_t)stream);
   if (st != SA_OK) return st;
@@ -489,6 +522,10 @@ sa_status sa_kv_restore(sa_kv_cache* cache, const sa_snapshot* snap) {
       snap->offset < 0 || snap->offset > cache->high_water || snap->seq > cache->seq)
     return SA_ERR_INVALID_ARG;
   if (snap->seq < cache->log_floor_seq && cache->log_floor_row < snap->offset) return SA_ERR_STALE_SNAPSHOT;
+  // a ring keeps the last cap positions: the band rows the snapshot needs,
+  // [offset - ring + 1, offset), must not have been overwritten since
+  if (cache->ring > 0 && cache->high_water > snap->offset + cache->cap - (cache->ring - 1))
+    return SA_ERR_STALE_SNAPSHOT;
   for (int i = 0; i < cache->log_len; ++i)
     if (cache->log_seq[i] > snap->seq && cache->log_row[i] < snap->offset) return SA_ERR_STALE_SNAPSHOT;
   cache->offset = snap->offset;
@@ -540,7 +577,8 @@ sa_status sa_attn_decode_static(sa_kv_cache* cache, const sa_attn_args* a, sa_st
   if (a->T != 1) return SA_ERR_INVALID_ARG;
   const int q_mult = a->n_q / cache->n_kv;
   if (q_mult > 8) return SA_ERR_SHAPE;
-  const long long lo = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
+  long long lo = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
+  if (cache->ring > 0) lo = lo / 128 * 128;   // the decode's ring stages start aligned (see launch_decode)
   const DecodeSplit sp = decode_split(a->B, cache->n_kv, a->offset - lo);
   if (sp.S > 1 && decode_ws_bytes(a->B, cache->n_kv, q_mult, cache->d, sp.S) > SA_DECODE_STATIC_SCRATCH_BYTES)
     return SA_ERR_WORKSPACE;

@@ -40,6 +40,7 @@ class _KVCache(ctypes.Structure):
         ("offset", ctypes.c_int64), ("seq", ctypes.c_int64), ("high_water", ctypes.c_int64),
         ("log_seq", ctypes.c_int64 * KV_LOG_CAP), ("log_row", ctypes.c_int64 * KV_LOG_CAP),
         ("log_len", ctypes.c_int32), ("log_floor_seq", ctypes.c_int64), ("log_floor_row", ctypes.c_int64),
+        ("ring", ctypes.c_int32),
     ]
 
 
@@ -71,7 +72,7 @@ EXPORTS = (
     "sa_status_string", "sa_yarn_rope_tables", "sa_rope_apply_qk", "sa_kv_cache_init",
     "sa_kv_append", "sa_kv_snapshot", "sa_kv_restore", "sa_attn_prefill", "sa_attn_decode",
     "sa_attn_decode_workspace_size", "sa_get_device_status", "sa_set_wait_limit",
-    "sa_attn_decode_static", "sa_set_prefill_events",
+    "sa_attn_decode_static", "sa_set_prefill_events", "sa_kv_cache_init_ring",
 )
 
 _lib = None
@@ -93,6 +94,7 @@ def lib():
         L.sa_yarn_rope_tables.argtypes = [vp, vp, i32, i32, f64, f64, i32, f64, f64, vp]
         L.sa_rope_apply_qk.argtypes = [vp, P(i64), vp, P(i64), i32, i32, i32, i32, i32, i64, vp, vp, i32, vp]
         L.sa_kv_cache_init.argtypes = [P(_KVCache), vp, vp, i32, i32, i32, i32]
+        L.sa_kv_cache_init_ring.argtypes = [P(_KVCache), vp, vp, i32, i32, i32, i32, i32]
         L.sa_kv_append.argtypes = [P(_KVCache), vp, P(i64), vp, P(i64), i32, vp]
         L.sa_kv_snapshot.argtypes = [P(_KVCache), P(_Snapshot)]
         L.sa_kv_restore.argtypes = [P(_KVCache), P(_Snapshot)]
@@ -178,25 +180,37 @@ class KVCache:
     """One layer's bf16 KV cache, head-major [B, n_kv, cap, d] (torch-owned
     device memory). ``rows(b_slice, start, stop)`` views rows as [B, T, n_kv, d]."""
 
-    def __init__(self, B, cap, n_kv, d, device="cuda", k=None, v=None):
+    def __init__(self, B, cap, n_kv, d, device="cuda", k=None, v=None, ring=0):
         shape = (B, n_kv, cap, d)
         self.k = k if k is not None else torch.zeros(shape, dtype=torch.bfloat16, device=device)
         self.v = v if v is not None else torch.zeros(shape, dtype=torch.bfloat16, device=device)
         assert tuple(self.k.shape) == shape and self.k.is_contiguous() and self.v.is_contiguous()
         self.raw = _KVCache()
-        _check(lib().sa_kv_cache_init(ctypes.byref(self.raw), _ptr(self.k), _ptr(self.v), B, cap, n_kv, d),
-               "sa_kv_cache_init")
+        if ring:
+            _check(lib().sa_kv_cache_init_ring(ctypes.byref(self.raw), _ptr(self.k), _ptr(self.v), B, cap,
+                                               n_kv, d, int(ring)), "sa_kv_cache_init_ring")
+        else:
+            _check(lib().sa_kv_cache_init(ctypes.byref(self.raw), _ptr(self.k), _ptr(self.v), B, cap, n_kv,
+                                          d), "sa_kv_cache_init")
 
     @property
     def offset(self):
         return self.raw.offset
 
     def k_rows(self, start=0, stop=None):
-        """K rows [start, stop) as a [B, T, n_kv, d] view."""
-        return self.k[:, :, start:stop].transpose(1, 2)
+        """K rows [start, stop) as a [B, T, n_kv, d] view (a gathered copy
+        of positions [start, stop) for a ring cache)."""
+        return self._rows(self.k, start, stop)
 
     def v_rows(self, start=0, stop=None):
-        return self.v[:, :, start:stop].transpose(1, 2)
+        return self._rows(self.v, start, stop)
+
+    def _rows(self, t, start, stop):
+        if not self.raw.ring:
+            return t[:, :, start:stop].transpose(1, 2)
+        stop = self.raw.offset if stop is None else stop
+        idx = torch.arange(start, stop, device=t.device) % self.raw.cap
+        return t[:, :, idx].transpose(1, 2)
 
     @property
     def B(self):

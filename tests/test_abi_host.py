@@ -136,3 +136,30 @@ def test_prefill_event_hook_arguments(L):
     assert L.sa_set_prefill_events(ctypes.c_void_p(0x10), None) == inv
     assert L.sa_set_prefill_events(None, ctypes.c_void_p(0x10)) == inv
     assert L.sa_set_prefill_events(None, None) == 0
+
+
+def test_ring_cache_host_rules(L):
+    ring = lambda cap, window: (lambda c: (c, L.sa_kv_cache_init_ring(ctypes.byref(c), ctypes.c_void_p(0x10000),
+                                                                      ctypes.c_void_p(0x20000), 1, cap, 2, 64,
+                                                                      window)))(S._KVCache())
+    assert ring(768, 128)[1] == 0
+    assert ring(700, 128)[1] == 2           # capacity not a multiple of 384
+    assert ring(384, 500)[1] == 2           # band wider than the ring
+    assert ring(768, 0)[1] == 1
+    c, _ = ring(768, 128)
+    assert c.ring == 128
+    stream = ctypes.c_void_p(0)
+    # calls on a ring must use its band; a prefill must fit T + W - 1 rows
+    assert L.sa_attn_prefill(ctypes.byref(c), ctypes.byref(_args(T=4, window=0)), stream) == 1
+    assert L.sa_attn_prefill(ctypes.byref(c), ctypes.byref(_args(T=4, window=64)), stream) == 1
+    assert L.sa_attn_prefill(ctypes.byref(c), ctypes.byref(_args(T=642, window=128)), stream) == 3
+    # positions are unbounded: an offset beyond cap is valid
+    c.offset, c.high_water, c.seq = 5000, 5000, 3
+    s = S._Snapshot()
+    assert L.sa_kv_snapshot(ctypes.byref(c), ctypes.byref(s)) == 0 and s.offset == 5000
+    # rows [offset - 127, offset) of the snapshot survive while the ring has
+    # not advanced past offset + cap - 127
+    c.offset = c.high_water = 5000 + 768 - 127
+    assert L.sa_kv_restore(ctypes.byref(c), ctypes.byref(s)) == 0 and c.offset == 5000
+    c.offset = c.high_water = 5000 + 768 - 126
+    assert L.sa_kv_restore(ctypes.byref(c), ctypes.byref(s)) == 5       # stale

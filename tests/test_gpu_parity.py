@@ -279,6 +279,54 @@ def test_prefill_and_decode_window_edges_mha(cuda_device, window):
     _decode_steps(cfg, cache, ocache, 3, window, cos, sin, rc, rs, wl.sinks(cfg).to(DEV))
 
 
+@pytest.mark.parametrize("over", [dict(B=2, n_q=8, n_kv=2, d=64),
+                                  dict(B=2, n_q=8, n_kv=4, d=96, sm_scale=1 / math.sqrt(96)),
+                                  dict(B=1, n_q=4, n_kv=1, d=128, sm_scale=1 / math.sqrt(128))],
+                         ids=["d64", "d96", "d128"])
+def test_ring_cache_matches_oracle(cuda_device, over):
+    # A band layer on a 384-row ring: prefill, decode, a second prefill chunk
+    # that wraps the ring, decode again, then snapshot / restore. Every output
+    # against the oracle on a plain (unbounded) cache; the ring's live rows
+    # against the oracle's rows of the same positions.
+    cfg = wl.scaled(wl.CONFIGS["tiny"], **over)
+    W, cap = 128, 384
+    n_total = 200 + 3 + 250 + 6
+    cos, sin = _tables(cfg, n_total + 8)
+    rc, rs = oracle_tables(cfg, n_total + 8)
+    sinks = wl.sinks(cfg).to(DEV)
+    cache = sa.KVCache(cfg.B, cap, cfg.n_kv, cfg.d, device=DEV, ring=W)
+    ocache = oracle_cache(cfg.B, n_total + 8, cfg.n_kv, cfg.d)
+
+    def prefill(T, seed):
+        q, k, v = wl.qkv(cfg, T, step=seed)
+        out, lse = sa.attn_prefill(cache, q.to(DEV), k.to(DEV), v.to(DEV), sinks, W, cfg.sm_scale, cos, sin,
+                                   return_lse=True)
+        torch.cuda.synchronize()
+        ref, ref_lse = oracle_step(ocache, q, k, v, sinks.cpu(), W, cfg.sm_scale, rc, rs)
+        check_bf16_output(out, ref, f"ring prefill {T}")
+        check_lse(lse, ref_lse, f"ring prefill {T}")
+
+    def live_rows_match():
+        off = cache.offset
+        lo = max(0, off - W + 1)
+        k_ring, v_ring = to64(cache.k_rows(lo, off)), to64(cache.v_rows(lo, off))
+        assert np.array_equal(v_ring, ocache.V[:, lo:off])
+        assert np.all(np.abs(k_ring - ocache.K[:, lo:off]) <= obf16.bf16_ulp(ocache.K[:, lo:off]) * 1.0000001)
+
+    prefill(200, 100)
+    _decode_steps(cfg, cache, ocache, 3, W, cos, sin, rc, rs, sinks, first_step=200)
+    prefill(250, 300)                       # positions 203..452: wraps rows 383 -> 0
+    live_rows_match()
+    snap, osnap = cache.snapshot(), ocache.snapshot()
+    _decode_steps(cfg, cache, ocache, 3, W, cos, sin, rc, rs, sinks, first_step=400)
+    live_rows_match()
+    cache.restore(snap)                     # the band rows of the snapshot are still held
+    ocache.restore(osnap)
+    assert cache.offset == ocache.offset == 453
+    _decode_steps(cfg, cache, ocache, 3, W, cos, sin, rc, rs, sinks, first_step=500)
+    live_rows_match()
+
+
 def test_decode_from_empty_cache_and_no_sink(cuda_device):
     cfg = wl.scaled(wl.CONFIGS["tiny"], B=2)
     cos, sin = _tables(cfg, 8)
