@@ -293,26 +293,40 @@ def gptoss_prefill(dev, peaks, reps=10):
     return res
 
 
-def long_decode(dev, peaks, steps=8, layers=24):
+def long_decode(dev, peaks, steps=8, layers=24, ring=False):
     """131,072-context decode: 24 layers alternating band / full, one row per
-    layer per step, KV bytes actually read / time."""
+    layer per step, KV bytes actually read / time. ring=True keeps the band
+    layers in 384-row ring caches instead of full-length ones."""
     import sink_augmented_gqa_b200 as sa
     cfg = wl.CONFIGS["long_decode"]
     off = cfg.offset
     cap = off + steps + 4
+    ring_cap = 384
     y = cfg.yarn
     cos, sin = sa.yarn_rope_tables(cap, cfg.d, y["theta"], y["scaling"], y["orig_ctx"], y["alpha"],
                                    y["beta"], device=dev)
     caches, ins = [], []
     for layer in range(layers):
-        c = sa.KVCache(cfg.B, cap, cfg.n_kv, cfg.d, device=dev)
+        w = cfg.layer_window(layer)
         g = torch.Generator(device=dev)
         g.manual_seed(cfg.seed * 1000 + 50_000 + layer)
-        c.k.normal_(generator=g)
-        c.v.normal_(generator=g)
-        # rows [0, off) stand for an already-filled, rotated prefix: append them
-        # in place (a self-copy) so the cache's offset and bookkeeping follow.
-        c.append(c.k_rows(0, off), c.v_rows(0, off))
+        if ring and w:
+            # a band layer's ring: the last ring_cap positions, up to `off`
+            c = sa.KVCache(cfg.B, ring_cap, cfg.n_kv, cfg.d, device=dev, ring=w)
+            pre_k = torch.empty((cfg.B, ring_cap, cfg.n_kv, cfg.d), dtype=torch.bfloat16, device=dev)
+            pre_v = torch.empty_like(pre_k)
+            pre_k.normal_(generator=g)
+            pre_v.normal_(generator=g)
+            while c.offset < off:   # the prefix streamed through the ring, one ring-full at a time
+                n = min(ring_cap, off - c.offset)
+                c.append(pre_k[:, :n], pre_v[:, :n])
+        else:
+            c = sa.KVCache(cfg.B, cap, cfg.n_kv, cfg.d, device=dev)
+            c.k.normal_(generator=g)
+            c.v.normal_(generator=g)
+            # rows [0, off) stand for an already-filled, rotated prefix: append them
+            # in place (a self-copy) so the cache's offset and bookkeeping follow.
+            c.append(c.k_rows(0, off), c.v_rows(0, off))
         caches.append(c)
         ins.append(dict(window=cfg.layer_window(layer), sinks=wl.sinks(cfg, layer, device=dev),
                         ws=sa.decode_workspace(cfg.B, cfg.n_q, cfg.n_kv, cfg.d, device=dev),
@@ -390,6 +404,7 @@ def long_decode(dev, peaks, steps=8, layers=24):
         gbytes += (min(off + 1, w) if w else off + 1) * row_bytes
     gbs_graph = gbytes / (ms_graph * 1e-3) / 1e9
     del graph
+    kv_gib = sum(2 * c.k.numel() * 2 for c in caches) / 2 ** 30
     del caches
     torch.cuda.empty_cache()
     return {"steps": steps, "layers": layers, "ms_per_token_step": round(ms / steps, 4),
@@ -398,8 +413,8 @@ def long_decode(dev, peaks, steps=8, layers=24):
                                   "frac_of_hbm": round(gbs_full / peaks["hbm"], 4)},
             "cuda_graph_token_step": {"ms": round(ms_graph, 4), "KV_GB/s": round(gbs_graph, 1),
                                       "frac_of_hbm": round(gbs_graph / peaks["hbm"], 4)},
-            "kv_cache_GiB": round(layers * 2 * cfg.B * cap * cfg.n_kv * cfg.d * 2 / 2 ** 30, 3),
-            "cache_layout": "head-major [B][n_kv][cap][d]"}
+            "kv_cache_GiB": round(kv_gib, 3),
+            "cache_layout": "head-major [B][n_kv][cap][d]" + (", band layers in 384-row rings" if ring else "")}
 
 
 def e2e_lite(step, steps, warmup):
@@ -657,6 +672,7 @@ def main():
     if not args.no_extras and rank == 0:
         extras["gptoss_prefill_T8192"] = gptoss_prefill(dev, peaks)
         extras["long_context_decode_131072"] = long_decode(dev, peaks)
+        extras["long_context_decode_131072_ring"] = long_decode(dev, peaks, ring=True)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
