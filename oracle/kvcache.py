@@ -77,3 +77,11 @@ class KVCache:
 def kv_bytes(L, B, T, H_kv, d, dtype_bytes):
     """Back-of-the-envelope KV-cache size in bytes (K and V, all layers)."""
     return 2 * L * B * T * H_kv * d * dtype_bytes
+
+
+def kv_bytes_windowed(L, L_windowed, window, B, T, H_kv, d, dtype_bytes):
+    """The same when L_windowed of the L layers keep only their last `window`
+    tokens (MoE-Xtend project page, "Results": windowed layers cache 128
+    tokens regardless of sequence length)."""
+    rows = (L - L_windowed) * T + L_windowed * min(T, window)
+    return 2 * B * rows * H_kv * d * dtype_bytes

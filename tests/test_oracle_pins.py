@@ -356,6 +356,18 @@ def test_kv_bytes_matches_printed_example():
     assert n == 6 * 2 ** 30   # the printed figure is exact here
 
 
+def test_windowed_kv_reduction_matches_printed_ratios():
+    g = json.load(open(os.path.join(GOLDEN, "kv_window_reduction.json")))
+    L = 24
+    Lw = int(L * g["windowed_fraction"])
+    for pt in g["points"]:
+        full = kvcache.kv_bytes(L, 1, pt["T"], 8, 96, 2)
+        ring = kvcache.kv_bytes_windowed(L, Lw, g["window"], 1, pt["T"], 8, 96, 2)
+        ratio = full / ring
+        assert abs(ratio - pt["printed_ratio"]) < pt["resolution"], (pt, ratio)
+        assert ratio == 2 * pt["T"] / (pt["T"] + g["window"])   # the closed form for half the layers windowed
+
+
 def test_gqa_shapes_match_printed_values():
     g = json.load(open(os.path.join(GOLDEN, "gqa_shapes.json")))
     assert g["d_h"] * (g["n_q"] + 2 * g["n_kv"]) == g["qkv_width"]
