@@ -327,6 +327,61 @@ def test_ring_cache_matches_oracle(cuda_device, over):
     live_rows_match()
 
 
+def _random_cases(n, seed=2026):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for idx in range(n):
+        d = int(rng.choice([64, 96, 128]))
+        n_kv = int(rng.choice([1, 2, 4]))
+        q_mult = int(rng.choice([1, 2, 4, 8]))
+        B = int(rng.integers(1, 4))
+        T = int(rng.integers(1, 700))
+        off = int(rng.choice([0, 0, int(rng.integers(1, 900))]))
+        window = int(rng.choice([0, 0, 1, 7, 64, 128, 200, 1000]))
+        ring = bool(window > 0 and rng.random() < 0.3)
+        cases.append((idx, d, n_kv, q_mult, B, T, off, window, ring))
+    return cases
+
+
+@pytest.mark.parametrize("idx,d,n_kv,q_mult,B,T,off,window,ring", _random_cases(24),
+                         ids=[f"r{c[0]}" for c in _random_cases(24)])
+def test_random_shapes_prefill_then_decode(cuda_device, idx, d, n_kv, q_mult, B, T, off, window, ring):
+    # Seeded random shapes: head dims, GQA ratios (1..8), ragged T, prefixes,
+    # band widths (including 1 and wider than a tile) and ring caches; every
+    # output row and lse against the oracle, then two decode steps.
+    cfg = wl.scaled(wl.CONFIGS["tiny"], B=B, n_q=n_kv * q_mult, n_kv=n_kv, d=d, sm_scale=1 / math.sqrt(d),
+                    seed=100 + idx)
+    n_total = off + T + 2
+    cos, sin = _tables(cfg, n_total + 8)
+    rc, rs = oracle_tables(cfg, n_total + 8)
+    sinks = wl.sinks(cfg).to(DEV)
+    if ring:
+        cap = ((max(T, 1) + window - 1 + 383) // 384) * 384
+        cache = sa.KVCache(cfg.B, cap, cfg.n_kv, cfg.d, device=DEV, ring=window)
+    else:
+        cache = sa.KVCache(cfg.B, n_total + 8, cfg.n_kv, cfg.d, device=DEV)
+    ocache = oracle_cache(cfg.B, n_total + 8, cfg.n_kv, cfg.d)
+    if off:
+        kp, vp = wl.prefilled_cache_rows(cfg, rows=off)
+        if ring:   # stream the prefix through the ring in chunks that fit
+            done = 0
+            while done < off:
+                n = min(cache.raw.cap, off - done)
+                cache.append(kp[:, done:done + n].to(DEV), vp[:, done:done + n].to(DEV))
+                done += n
+        else:
+            cache.append(kp.to(DEV), vp.to(DEV))
+        ocache.append(to64(kp), to64(vp))
+    q, k, v = wl.qkv(cfg, T, step=7)
+    out, lse = sa.attn_prefill(cache, q.to(DEV), k.to(DEV), v.to(DEV), sinks, window, cfg.sm_scale, cos, sin,
+                               return_lse=True)
+    torch.cuda.synchronize()
+    ref, ref_lse = oracle_step(ocache, q, k, v, sinks.cpu(), window, cfg.sm_scale, rc, rs)
+    check_bf16_output(out, ref, f"random case {idx}")
+    check_lse(lse, ref_lse, f"random case {idx}")
+    _decode_steps(cfg, cache, ocache, 2, window, cos, sin, rc, rs, sinks, first_step=50)
+
+
 def test_decode_from_empty_cache_and_no_sink(cuda_device):
     cfg = wl.scaled(wl.CONFIGS["tiny"], B=2)
     cos, sin = _tables(cfg, 8)
