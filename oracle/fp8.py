@@ -28,6 +28,10 @@ the oracle takes that decision in the same precision as the kernel.
 
 import numpy as np
 
+from .attention import sink_attention
+from .bf16 import round_bf16
+from .rope import rotate_bsh
+
 E4M3_MAX = 448.0
 # Smallest normal binade exponent and the subnormal quantum (2**-9).
 _E4M3_MIN_NORMAL_EXP = -6
@@ -97,6 +101,27 @@ def quantize_rows(x):
 def dequantize_rows(codes, scales):
     """fp64 values a reader of the quantised cache sees: code value * scale."""
     return e4m3_value(codes) * np.asarray(scales, dtype=np.float64)[..., None]
+
+
+def attend_step_fp8(cache, q, k, v, sinks, window, sm_scale, cos_tab, sin_tab, rope_fused=True):
+    """One call of the hot path on a quantised cache.
+
+    As ``attention.attend_step``, except that the rows stored are the
+    quantised bf16 rows (K after rotation) and every key and value read --
+    the call's own new rows included -- is the dequantised row. ``cache`` is
+    an fp64 ``kvcache.KVCache`` holding dequantised rows.
+    """
+    off = cache.offset
+    if rope_fused:
+        q_rot = rotate_bsh(q, off, cos_tab, sin_tab)
+        k_rot = rotate_bsh(k, off, cos_tab, sin_tab)
+    else:
+        q_rot = round_bf16(q)
+        k_rot = round_bf16(k)
+    kc, ks = quantize_rows(k_rot)
+    vc, vs = quantize_rows(round_bf16(v))
+    cache.append(dequantize_rows(kc, ks), dequantize_rows(vc, vs))
+    return sink_attention(q_rot, cache.K, cache.V, sinks, off, window, sm_scale)
 
 
 def kv_bytes_fp8(L, B, T, H_kv, d):

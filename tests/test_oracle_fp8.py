@@ -134,3 +134,38 @@ def test_fp8_kv_bytes_halve_the_printed_bf16_example():
     f8 = fp8.kv_bytes_fp8(24, 1, 131072, 8, 64)
     assert f8 - 2 * 24 * 131072 * 8 * 4 == bf16 // 2
     assert f8 / 2 ** 30 == pytest.approx(3.1875)
+
+
+def test_quantised_step_is_lossless_on_representable_rows():
+    """Rows whose values are E4M3 values times a power of two whose row
+    maximum is 448 times that power quantise without loss, so the quantised
+    step reduces to the bf16 step (pre-rotated inputs, no RoPE)."""
+    from oracle import attention as oatt
+    rng = np.random.default_rng(5)
+    B, T, n_kv, q_mult, d = 1, 9, 2, 2, 64
+    table = fp8.e4m3_value(np.arange(256, dtype=np.uint8))
+    table = table[np.isfinite(table)]
+
+    def rows(shape):
+        x = rng.choice(table, size=shape)
+        x[..., 0] = 448.0                      # row maximum: scale = 2**e exactly
+        e = rng.integers(-8, 8, size=shape[:-1])[..., None]
+        return np.ldexp(x, e)
+
+    k, v = rows((B, T, n_kv, d)), rows((B, T, n_kv, d))
+    q = round_bf16(rng.standard_normal((B, T, n_kv * q_mult, d)))
+    sinks = rng.standard_normal(n_kv * q_mult)
+    c1 = kvcache.KVCache(B, T, n_kv, d)
+    c2 = kvcache.KVCache(B, T, n_kv, d)
+    o1, l1 = oatt.attend_step(c1, q, k, v, sinks, 0, 0.125, None, None, rope_fused=False)
+    o2, l2 = fp8.attend_step_fp8(c2, q, k, v, sinks, 0, 0.125, None, None, rope_fused=False)
+    assert np.array_equal(c1.K, c2.K) and np.array_equal(c1.V, c2.V)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+    # ... while a value between two E4M3 steps is rounded: 0.3 * 448 = 134.4
+    # lies between the steps 128 and 144 of its binade
+    k2 = k.copy()
+    k2[0, 0, 0, 1] = round_bf16(0.3 * k[0, 0, 0, 0])
+    c3 = kvcache.KVCache(B, T, n_kv, d)
+    fp8.attend_step_fp8(c3, q, k2, v, sinks, 0, 0.125, None, None, rope_fused=False)
+    assert c3.K[0, 0, 0, 1] != k2[0, 0, 0, 1]
+    assert c3.K[0, 0, 0, 1] / k[0, 0, 0, 0] * 448 in (128.0, 144.0)
