@@ -53,8 +53,15 @@ typedef enum sa_status {
   SA_ERR_STALE_SNAPSHOT = 5,   /* restore after rows below the snapshot were rewritten */
   SA_ERR_CUDA = 6,             /* a CUDA runtime/driver call failed (launch, tensor map) */
   SA_ERR_TIMEOUT = 7,          /* a bounded device wait ran out (read via sa_get_device_status) */
-  SA_ERR_WORKSPACE = 8         /* decode workspace missing or too small */
+  SA_ERR_WORKSPACE = 8,        /* decode workspace missing or too small */
+  SA_ERR_UNSUPPORTED = 9       /* operation not provided for this cache format (prefill on FP8) */
 } sa_status;
+
+/* Element format of a cache (sa_kv_cache.kv_dtype). */
+typedef enum sa_kv_dtype {
+  SA_KV_BF16 = 0,      /* bf16 rows */
+  SA_KV_FP8_E4M3 = 1   /* e4m3 codes + one fp32 scale per row (sa_kv_cache_init_fp8) */
+} sa_kv_dtype;
 
 /* Capacity of the cache's overwrite log (see sa_kv_restore). */
 #define SA_KV_LOG_CAP 32
@@ -80,8 +87,12 @@ typedef enum sa_status {
  *        unbounded, and the cache holds the last cap positions (cap a
  *        multiple of 384, cap >= ring). Calls on a ring cache must use
  *        window == ring. Initialise with sa_kv_cache_init_ring.
+ * kv_dtype, k_scale, v_scale: SA_KV_BF16 with NULL scales, or
+ *        SA_KV_FP8_E4M3: k and v then hold e4m3 codes (one byte per element,
+ *        same [B][n_kv][cap][d] layout) and k_scale / v_scale fp32
+ *        [B][n_kv][cap] row scales (see sa_kv_cache_init_fp8).
  * The remaining fields are bookkeeping for snapshot/restore; initialise the
- * whole struct with sa_kv_cache_init (or _ring) and do not edit them.
+ * whole struct with sa_kv_cache_init (or _ring, _fp8) and do not edit them.
  */
 typedef struct sa_kv_cache {
   void* k;
@@ -96,6 +107,9 @@ typedef struct sa_kv_cache {
   int64_t log_floor_seq; /* summary of entries dropped from the full log: */
   int64_t log_floor_row; /* latest dropped seq, lowest dropped row        */
   int32_t ring;          /* 0: linear; > 0: ring cache for `ring`-key bands */
+  int32_t kv_dtype;      /* sa_kv_dtype */
+  void* k_scale;         /* FP8 only: fp32 [B][n_kv][cap] */
+  void* v_scale;
 } sa_kv_cache;
 
 typedef struct sa_snapshot {
@@ -192,9 +206,33 @@ sa_status sa_kv_cache_init_ring(sa_kv_cache* cache, void* k, void* v, int32_t B,
                                 int32_t n_kv, int32_t d, int32_t window);
 
 /*
+ * FP8 cache: quantised K/V rows with the dequantisation fused into decode
+ * (MoE-Xtend README, "ROADMAP": quantisation-aware long-context runs,
+ * bandwidth first -- KV plus its dequantisation). Decode reads 1 byte per
+ * element plus 8 bytes of scales per (position, KV head) instead of 2 bytes.
+ * k, v    : device e4m3 codes [B][n_kv][cap][d], 16-byte aligned.
+ * k_scale, v_scale: device fp32 [B][n_kv][cap], 16-byte aligned.
+ * window  : 0 for a linear cache, > 0 for a ring cache of `window`-key
+ *           bands (same rules as sa_kv_cache_init_ring).
+ * cap must be a multiple of 16 (SA_ERR_SHAPE). Every stored row x (K after
+ * rotation, V as given, each the bf16 row a bf16 cache would hold) is kept
+ * as scale = fl32(amax|x| / 448) and codes e4m3(fl32(x_d / scale)) rounded
+ * to nearest even with saturation (a zero row: scale 0, codes 0); readers
+ * see code * scale. Appends (sa_kv_append, and the new row of
+ * sa_attn_decode, which also attends its quantised value) quantise;
+ * sa_attn_prefill returns SA_ERR_UNSUPPORTED on an FP8 cache: run prefill
+ * on a bf16 cache and move its rows over with sa_kv_append (strides
+ * {n_kv*cap*d, d, cap*d} describe a bf16 cache as [B][T][n_kv][d]).
+ * Buffers of a ring cache, scales included, must be zeroed before first use.
+ */
+sa_status sa_kv_cache_init_fp8(sa_kv_cache* cache, void* k, void* v, void* k_scale, void* v_scale,
+                               int32_t B, int32_t cap, int32_t n_kv, int32_t d, int32_t window);
+
+/*
  * Append T already-rotated K rows and V rows at [offset, offset+T), then
  * offset += T (MoE-Xtend README, "KV CACHE": Cache.extend). k_rot/v: device
- * bf16 [B][T][n_kv][d] via strides. Bit copy. SA_ERR_CAPACITY if
+ * bf16 [B][T][n_kv][d] via strides. Bit copy into a bf16 cache; into an FP8
+ * cache each row is quantised (sa_kv_cache_init_fp8). SA_ERR_CAPACITY if
  * offset + T > cap.
  */
 sa_status sa_kv_append(sa_kv_cache* cache, const void* k_rot, const int64_t k_strides[3],
@@ -230,7 +268,7 @@ sa_status sa_kv_restore(sa_kv_cache* cache, const sa_snapshot* snap);
  * attention). The attention kernel schedules its work items from a device
  * counter; the library keeps 64 such counters per device and hands them out
  * round robin, so at most 64 prefill calls may be in flight on one device at
- * a time (across all streams).
+ * a time (across all streams). SA_ERR_UNSUPPORTED on an FP8 cache.
  */
 sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* args, sa_stream_t stream);
 
@@ -239,7 +277,11 @@ sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* args, sa_strea
  * appends the new K/V row at cache row `offset`, and attends to cache rows
  * [max(0, offset+1-window), offset] (all rows when window <= 0), split
  * across SMs. cache->offset += 1 on success (MoE-Xtend README, "DESIGN
- * CONTRACTS": exactly one row per layer per step).
+ * CONTRACTS": exactly one row per layer per step). On an FP8 cache the
+ * kernel dequantises K/V as it reads them and stores and attends the new
+ * row quantised; queries enter the QK product as f16 after an exact
+ * per-head power-of-two scaling, and the scaled softmax weights enter the PV
+ * product as f16.
  * workspace: device memory of at least sa_attn_decode_workspace_size()
  *   bytes, caller-owned, ZERO-FILLED before its first use; the kernel leaves
  *   it zeroed again on completion. Calls that share a workspace must not

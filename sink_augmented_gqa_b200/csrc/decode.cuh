@@ -20,8 +20,23 @@
 // finish (atomic ticket, no spinning) merges all S of them and folds in the
 // sink: M = max(max_s m_s, sink), l = sum_s e^{m_s-M} l_s + e^{sink-M},
 // out = sum_s e^{m_s-M} O_s / l.
+//
+// FP8 caches (decode_kernel<D, true>) store e4m3 codes plus one fp32 scale
+// per row (fp8.cuh). Their stages carry R codes rows of K and of V and the
+// 2R row scales; a consumer converts codes to f16 in registers (exact), so
+// K enters S^T = K Q^T unscaled and each score is multiplied by its row's K
+// scale afterwards, while each probability is multiplied by its row's V
+// scale before it becomes the f16 operand of O^T = V^T P^T. To keep those
+// f16 operands in range, Q is taken in f16 after a per-head power-of-two
+// scaling (undone in the score scale), and P*scale_v is taken relative to a
+// per-warp power of two that only grows (undone when the warp's partial is
+// written). Rows of a sub-tile are visited in a permuted order chosen so
+// that the byte-granular shared-memory reads of V hit distinct banks.
 #pragma once
 
+#include <type_traits>
+
+#include "fp8.cuh"
 #include "ptx.cuh"
 
 namespace sa {
@@ -47,7 +62,9 @@ struct DecodeParams {
   long long lo;     // first cache position of split 0's first stage
   long long lo_mask;  // first cache position attended (keys before it masked)
   int ring_cap;     // 0: row = position; > 0: ring cache, row = position mod ring_cap
-  long long chunk;  // cache rows per split (multiple of 64)
+  long long chunk;  // cache rows per split (multiple of 128)
+  float* cks;       // FP8 caches: row scales [B][n_kv][cap] of K and of V
+  float* cvs;
   int S;
   float scale_log2;
   int rope;
@@ -81,7 +98,55 @@ struct DecodeCfg {
   static_assert(NCW * RED_WARP <= 2 * NS * STAGE_BYTES, "warp partials must fit in the ring");
   static constexpr uint32_t OFF_BAR = OFF_XV + XTILE;
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + 8 * (2 * NS) + 16 + 1024;
+  static constexpr int BLKCOLS = CB;                    // tensor-map columns per column block
+  static constexpr uint32_t STAGE_TX = 2 * STAGE_BYTES;  // bytes one stage's TMA loads bring
 };
+
+// FP8 caches: codes rows of D bytes, stored as column blocks of ROWB bytes
+// (one swizzle span: 64 B for d = 64, 128 B for d = 128, 3 x 32 B for d = 96),
+// with the stage's 128 K and 128 V row scales beside them.
+template <int D>
+struct DecodeF8Cfg {
+  static constexpr int NCW = 8;
+  static constexpr int R = 16 * NCW;
+  static constexpr int ROWB = (D == 96) ? 32 : D;
+  static constexpr int NCB = D / ROWB;
+  static constexpr int BLKCOLS = ROWB;
+  static constexpr uint32_t BLOCK_BYTES = R * ROWB;
+  static constexpr uint32_t STAGE_BYTES = R * D;        // K (or V) codes of one stage
+  // as many bytes in flight per CTA as the bf16 kernel keeps
+  static constexpr int NS = (D == 64) ? 6 : (D == 96 ? 4 : 3);
+  static constexpr uint32_t STAGE_TX = 2 * STAGE_BYTES + 2 * R * 4;
+  static constexpr uint32_t XBLOCK = 16 * ROWB;
+  static constexpr uint32_t XTILE = 16 * D;
+  static constexpr int NUM_THREADS = 32 * (NCW + 1);
+  static constexpr uint32_t OFF_K = 0;
+  static constexpr uint32_t OFF_V = NS * STAGE_BYTES;
+  static constexpr uint32_t OFF_KS = 2 * NS * STAGE_BYTES;   // [NS][R] fp32
+  static constexpr uint32_t OFF_VS = OFF_KS + NS * R * 4;
+  static constexpr uint32_t OFF_XK = OFF_VS + NS * R * 4;
+  static constexpr uint32_t OFF_XV = OFF_XK + XTILE;
+  static constexpr uint32_t OFF_XS = OFF_XV + XTILE;         // [2][16] fp32: new-row scales
+  static constexpr uint32_t OFF_RED = OFF_K;
+  static constexpr uint32_t RED_WARP = (16 + 8 * D) * 4;
+  static_assert(NCW * RED_WARP <= 2 * NS * STAGE_BYTES, "warp partials must fit in the ring");
+  static_assert(OFF_XK % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static constexpr uint32_t OFF_BAR = OFF_XS + 128;
+  static constexpr uint32_t SMEM_BYTES = OFF_BAR + 8 * (2 * NS) + 16 + 1024;
+};
+
+template <int D, bool F8>
+using DecodeCfgT = typename std::conditional<F8, DecodeF8Cfg<D>, DecodeCfg<D>>::type;
+
+// Physical row (within a 16-row sub-tile) of logical key L of the FP8
+// consumer: logical keys {2c, 2c+1, 2c+8, 2c+9} of lane group c must sit in
+// rows whose swizzled V words fall in distinct banks.
+template <int D>
+__device__ __forceinline__ int f8_row(int L) {
+  const int l = L & 7;
+  const int r = (D == 64) ? (2 * (l & 3) + (l >> 2)) : (D == 96 ? ((l >> 1) + 4 * (l & 1)) : l);
+  return (L & 8) | r;
+}
 
 // Warp-level processing of one 16-key sub-tile (rows row0..row0+15 of a tile
 // stored as swizzled column blocks of `block_bytes`), keys < n_first and
@@ -140,11 +205,130 @@ __device__ __forceinline__ void decode_subtile(uint32_t kbase, uint32_t vbase, u
   }
 }
 
+// FP8 counterpart of decode_subtile: codes tiles in swizzled ROWB-byte column
+// blocks, row scales ksc/vsc (indexed by tile row), Q fragments in f16 laid
+// out for the byte order ldmatrix delivers (see the kernel), per-head score
+// scales hs (scale_log2 * 2^e of heads 2(lane%4), +1), and ev[e] the running
+// power of two of head column e's accumulator: O is kept in units of 2^ev,
+// ev the largest exponent of any weight p * scale_v seen so far, so that the
+// f16 weights p * scale_v * 2^-ev stay below 2 and lose only terms under
+// 2^-24 of the largest one.
 template <int D>
+__device__ __forceinline__ void decode_subtile_f8(uint32_t kbase, uint32_t vbase, uint32_t block_bytes,
+                                                  const float* ksc, const float* vsc, int row0,
+                                                  int n_first, int n_valid,
+                                                  const uint32_t (&qf)[D / 16][2],
+                                                  const float (&hs)[2], float (&m)[2], float (&l)[2],
+                                                  float (&o)[D / 16][4], int (&ev)[2], int lane) {
+  using C = DecodeF8Cfg<D>;
+  const int r = lane >> 2, cq = lane & 3;
+  // ---- S^T = K Q^T: ldmatrix over bytes gives lane (r, cq) key rows r, r+8 and
+  // code bytes 4cq..4cq+3 (+16) of each 32-byte group; its two 16-bit halves
+  // are the two K-steps of the group (the Q fragments follow the same order).
+  float c[4] = {0.f, 0.f, 0.f, 0.f};
+  {
+    const int prow = row0 + f8_row<D>((lane & 7) + 8 * ((lane >> 3) & 1));
+#pragma unroll
+    for (int grp = 0; grp < D / 32; ++grp) {
+      uint32_t r0, r1, r2, r3;
+      ldmatrix_x4(kbase + swz8<C::ROWB>(prow, 32 * grp + 16 * (lane >> 4), block_bytes), r0, r1, r2, r3);
+#pragma unroll
+      for (int st = 0; st < 2; ++st) {
+        const int sh = 16 * st;
+        mma_16816_f16(c, f16x2_from_e4m3x2((uint16_t)(r0 >> sh)), f16x2_from_e4m3x2((uint16_t)(r1 >> sh)),
+                      f16x2_from_e4m3x2((uint16_t)(r2 >> sh)), f16x2_from_e4m3x2((uint16_t)(r3 >> sh)),
+                      qf[2 * grp + st][0], qf[2 * grp + st][1]);
+      }
+    }
+  }
+  const int ka = f8_row<D>(r), kb = ka + 8;   // tile rows of logical keys r, r + 8
+  const bool va = ka >= n_first && ka < n_valid, vb = kb >= n_first && kb < n_valid;
+  const float ksa = ksc[row0 + ka], ksb = ksc[row0 + kb];
+  float s[4];
+  s[0] = va ? c[0] * (ksa * hs[0]) : -INFINITY;
+  s[1] = va ? c[1] * (ksa * hs[1]) : -INFINITY;
+  s[2] = vb ? c[2] * (ksb * hs[0]) : -INFINITY;
+  s[3] = vb ? c[3] * (ksb * hs[1]) : -INFINITY;
+  // Masked rows weigh 0 (their scales may be anything a never-written row holds).
+  const float vsa = va ? vsc[row0 + ka] : 0.f, vsb = vb ? vsc[row0 + kb] : 0.f;
+  float pr[4], alpha[2];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    float mx = fmaxf(s[e], s[2 + e]);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    const float m_new = fmaxf(m[e], mx);
+    const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+    alpha[e] = ex2(m[e] - m_use);
+    pr[e] = ex2(s[e] - m_use);
+    pr[2 + e] = ex2(s[2 + e] - m_use);
+    l[e] = l[e] * alpha[e] + pr[e] + pr[2 + e];
+    m[e] = m_new;
+  }
+  // ---- weights p * scale_v relative to the head's power of two 2^ev (ev
+  // never shrinks, so the rescale of O is at most 1)
+  float pw[4] = {pr[0] * vsa, pr[1] * vsa, pr[2] * vsb, pr[3] * vsb};
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    float mx = fmaxf(pw[e], pw[2 + e]);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    int ev_new = ev[e];
+    if (mx > 0.f) {
+      const int x = (int)((__float_as_uint(mx) >> 23) & 0xFFu) - 127;   // -127 for subnormals
+      ev_new = x > ev_new ? x : ev_new;
+    }
+    const int dv = ev[e] - ev_new;                                       // <= 0
+    const float fo = dv < -126 ? 0.f : __uint_as_float((uint32_t)(127 + dv) << 23);
+    const float inv = __uint_as_float((uint32_t)(127 - ev_new) << 23);   // 2^-ev_new
+    ev[e] = ev_new;
+    pw[e] *= inv;
+    pw[2 + e] *= inv;
+    const float ao = alpha[e] * fo;
+#pragma unroll
+    for (int md = 0; md < D / 16; ++md) {
+      o[md][e] *= ao;
+      o[md][2 + e] *= ao;
+    }
+  }
+  const uint32_t b01 = movmatrix_trans(pack_f16(pw[0], pw[1]));
+  const uint32_t b23 = movmatrix_trans(pack_f16(pw[2], pw[3]));
+  // ---- O^T += V^T P'^T: lane (r, cq) reads one 32-bit word (code bytes
+  // 4r..4r+3 of a 32-byte group) from each of the rows of logical keys 2cq,
+  // 2cq+1, 2cq+8, 2cq+9 and regroups the bytes into the A fragments of two
+  // 16-row blocks of d: block A holds d = 32 grp + 4r + {0, 1}, block B
+  // d = 32 grp + 4r + {2, 3} (rows r and r + 8 of the fragment).
+  const int k0 = f8_row<D>(2 * cq), k1 = f8_row<D>(2 * cq + 1), k2 = k0 + 8, k3 = k1 + 8;
+  const bool u0 = k0 >= n_first && k0 < n_valid, u1 = k1 >= n_first && k1 < n_valid;
+  const bool u2 = k2 >= n_first && k2 < n_valid, u3 = k3 >= n_first && k3 < n_valid;
+#pragma unroll
+  for (int grp = 0; grp < D / 32; ++grp) {
+    const int bc = 32 * grp + 4 * r;
+    uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;   // rows never written may hold NaN codes
+    if (u0) w0 = ld_shared_u32(vbase + swz8<C::ROWB>(row0 + k0, bc, block_bytes));
+    if (u1) w1 = ld_shared_u32(vbase + swz8<C::ROWB>(row0 + k1, bc, block_bytes));
+    if (u2) w2 = ld_shared_u32(vbase + swz8<C::ROWB>(row0 + k2, bc, block_bytes));
+    if (u3) w3 = ld_shared_u32(vbase + swz8<C::ROWB>(row0 + k3, bc, block_bytes));
+    const uint32_t x01a = __byte_perm(w0, w1, 0x5140), x23a = __byte_perm(w2, w3, 0x5140);
+    const uint32_t x01b = __byte_perm(w0, w1, 0x7362), x23b = __byte_perm(w2, w3, 0x7362);
+    mma_16816_f16(o[2 * grp], f16x2_from_e4m3x2((uint16_t)x01a), f16x2_from_e4m3x2((uint16_t)(x01a >> 16)),
+                  f16x2_from_e4m3x2((uint16_t)x23a), f16x2_from_e4m3x2((uint16_t)(x23a >> 16)), b01, b23);
+    mma_16816_f16(o[2 * grp + 1], f16x2_from_e4m3x2((uint16_t)x01b),
+                  f16x2_from_e4m3x2((uint16_t)(x01b >> 16)), f16x2_from_e4m3x2((uint16_t)x23b),
+                  f16x2_from_e4m3x2((uint16_t)(x23b >> 16)), b01, b23);
+  }
+}
+
+// tmK/tmV: the cache's K/V (bf16 elements, or FP8 code bytes); tmKS/tmVS
+// (FP8 only): the row scales, dims {rows, n_kv, B, 1}, box {R, 1, 1, 1}.
+template <int D, bool F8>
 __global__ void __launch_bounds__(288, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmKS, const __grid_constant__ CUtensorMap tmVS,
                   const DecodeParams p) {
-  using C = DecodeCfg<D>;
+  using C = DecodeCfgT<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -185,19 +369,29 @@ __global__ void __launch_bounds__(288, 2)
     if (lane == 0 && n_stages > 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
+      if constexpr (F8) {
+        tma_prefetch_desc(&tmKS);
+        tma_prefetch_desc(&tmVS);
+      }
       int issued = 0;
       for (int it = 0; it < n_stages; ++it) {
         const int s = it % C::NS;
         if (!mbar_wait(empty_bar(s), (uint32_t)(((it / C::NS) & 1) ^ 1))) { flag[0] = 1; break; }
-        mbar_arrive_expect_tx(full_bar(s), 2 * C::STAGE_BYTES);
+        mbar_arrive_expect_tx(full_bar(s), C::STAGE_TX);
         const long long pos = r_begin + (long long)it * C::R;   // stages never wrap a ring
         const int row = (int)(p.ring_cap > 0 ? pos % p.ring_cap : pos);
 #pragma unroll
         for (int cb = 0; cb < C::NCB; ++cb) {
           tma_load_4d(sbase + C::OFF_K + s * C::STAGE_BYTES + cb * C::BLOCK_BYTES, &tmK, full_bar(s),
-                      cb * C::CB, row, g, b);
+                      cb * C::BLKCOLS, row, g, b);
           tma_load_4d(sbase + C::OFF_V + s * C::STAGE_BYTES + cb * C::BLOCK_BYTES, &tmV, full_bar(s),
-                      cb * C::CB, row, g, b);
+                      cb * C::BLKCOLS, row, g, b);
+        }
+        if constexpr (F8) {
+          // row is a multiple of R (the FP8 launch aligns every stage), so the
+          // innermost coordinate of these fp32 boxes is 16-byte aligned
+          tma_load_4d(sbase + C::OFF_KS + s * C::R * 4, &tmKS, full_bar(s), row, g, b, 0);
+          tma_load_4d(sbase + C::OFF_VS + s * C::R * 4, &tmVS, full_bar(s), row, g, b, 0);
         }
         issued = it + 1;
         if (flag[0]) break;
@@ -214,7 +408,56 @@ __global__ void __launch_bounds__(288, 2)
   // Q fragments (B operand, col-major [d][head]): head n = lane/4 of the group,
   // dims kk*16 + 2*(lane%4) + {0,1} and +8, rotated at position off.
   uint32_t qf[D / 16][2];
-  {
+  float hs[2] = {0.f, 0.f};   // FP8: score scale of heads 2(lane%4), 2(lane%4)+1
+  if constexpr (F8) {
+    // FP8 layout: fragment (grp, st) holds dims 32 grp + 4(lane%4) + 2 st + {0,1}
+    // (register 0) and the same + 16 (register 1), matching the code bytes
+    // ldmatrix hands each lane. Head n is scaled by 2^-e_n so that its
+    // largest |q| lies in [2^14, 2^15): every bf16 q is then exact in f16
+    // down to 2^-29 of that maximum.
+    const int n = lane >> 2;
+    const bool hv = n < QM;
+    const __nv_bfloat16* qrow = p.q + b * p.qs0 + (long long)(g * QM + (hv ? n : 0)) * p.qs2;
+    const float* cs = p.cos_t + p.off * HALF;
+    const float* sn = p.sin_t + p.off * HALF;
+    float qv[D / 16][2][2];
+    float amax = 0.f;
+#pragma unroll
+    for (int f = 0; f < D / 16; ++f) {
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = 32 * (f >> 1) + 16 * hlf + 4 * (lane & 3) + 2 * (f & 1) + e;
+          float x = __bfloat162float(qrow[c]);
+          if (p.rope) {
+            const int i = c < HALF ? c : c - HALF;
+            uint32_t y1, y2;
+            rope_pair(__bfloat162float(qrow[i]), __bfloat162float(qrow[i + HALF]), cs[i], sn[i], y1, y2);
+            x = __uint_as_float((c < HALF ? y1 : y2) << 16);
+          }
+          x = hv ? x : 0.f;
+          qv[f][hlf][e] = x;
+          amax = fmaxf(amax, fabsf(x));
+        }
+      }
+    }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    int eq = 0;
+    if (amax > 0.f) {
+      eq = (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127 - 14;
+      eq = eq < -110 ? -110 : (eq > 110 ? 110 : eq);
+    }
+    const float down = __uint_as_float((uint32_t)(127 - eq) << 23);
+#pragma unroll
+    for (int f = 0; f < D / 16; ++f)
+#pragma unroll
+      for (int hlf = 0; hlf < 2; ++hlf) qf[f][hlf] = pack_f16(qv[f][hlf][0] * down, qv[f][hlf][1] * down);
+    const float hs_mine = p.scale_log2 * __uint_as_float((uint32_t)(127 + eq) << 23);
+    hs[0] = __shfl_sync(0xffffffffu, hs_mine, 8 * (lane & 3));
+    hs[1] = __shfl_sync(0xffffffffu, hs_mine, 8 * (lane & 3) + 4);
+  } else {
     const int n = lane >> 2;
     const bool hv = n < QM;
     const __nv_bfloat16* qrow = p.q + b * p.qs0 + (long long)(g * QM + (hv ? n : 0)) * p.qs2;
@@ -242,6 +485,7 @@ __global__ void __launch_bounds__(288, 2)
       }
     }
   }
+  int ev[2] = {-127, -127};   // FP8: powers of two of the two head columns' accumulators
 
   float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
   float o[D / 16][4];
@@ -249,7 +493,64 @@ __global__ void __launch_bounds__(288, 2)
   for (int md = 0; md < D / 16; ++md) o[md][0] = o[md][1] = o[md][2] = o[md][3] = 0.f;
 
   // The new row: rotate k, write K/V row `off` of the cache, stage it in smem.
-  if (last_split && warp == 0) {
+  // An FP8 cache stores (and this call attends) the row quantised.
+  if constexpr (F8) {
+    if (last_split && warp == 0) {
+      uint8_t* xk = smem + C::OFF_XK;
+      uint8_t* xv = smem + C::OFF_XV;
+      float* xs = reinterpret_cast<float*>(smem + C::OFF_XS);
+      const __nv_bfloat16* krow = p.k + b * p.ks0 + (long long)g * p.ks2;
+      const __nv_bfloat16* vrow = p.v + b * p.vs0 + (long long)g * p.vs2;
+      const long long slot = p.ring_cap > 0 ? p.off % p.ring_cap : p.off;
+      const long long crow = ((long long)b * p.n_kv + g) * p.cap + slot;
+      for (int idx = lane; idx < (int)(C::XTILE / 16); idx += 32) {
+        reinterpret_cast<uint4*>(xk)[idx] = make_uint4(0, 0, 0, 0);
+        reinterpret_cast<uint4*>(xv)[idx] = make_uint4(0, 0, 0, 0);
+      }
+      xs[lane] = 0.f;
+      __syncwarp();
+      float xkv[2][2], xvv[2][2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = 2 * lane + 64 * i + e;
+          float kx = 0.f, vx = 0.f;
+          if (c < D) {
+            kx = __bfloat162float(krow[c]);
+            if (p.rope) {
+              const int i0 = c < HALF ? c : c - HALF;
+              uint32_t y1, y2;
+              rope_pair(__bfloat162float(krow[i0]), __bfloat162float(krow[i0 + HALF]),
+                        p.cos_t[p.off * HALF + i0], p.sin_t[p.off * HALF + i0], y1, y2);
+              kx = __uint_as_float((c < HALF ? y1 : y2) << 16);
+            }
+            vx = __bfloat162float(vrow[c]);
+          }
+          xkv[i][e] = kx;
+          xvv[i][e] = vx;
+        }
+      }
+      uint16_t kc[2], vc[2];
+      const float sk = quantize_row_warp<2>(xkv, D, reinterpret_cast<uint8_t*>(p.ck) + crow * D, lane, kc);
+      const float sv = quantize_row_warp<2>(xvv, D, reinterpret_cast<uint8_t*>(p.cv) + crow * D, lane, vc);
+      if (lane == 0) {
+        p.cks[crow] = sk;
+        p.cvs[crow] = sv;
+        xs[0] = sk;
+        xs[16] = sv;
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int c = 2 * lane + 64 * i;
+        if (c < D) {
+          *reinterpret_cast<uint16_t*>(xk + swz8<C::ROWB>(0, c, C::XBLOCK)) = kc[i];
+          *reinterpret_cast<uint16_t*>(xv + swz8<C::ROWB>(0, c, C::XBLOCK)) = vc[i];
+        }
+      }
+      __syncwarp();
+    }
+  } else if (last_split && warp == 0) {
     uint8_t* xk = smem + C::OFF_XK;
     uint8_t* xv = smem + C::OFF_XV;
     const __nv_bfloat16* krow = p.k + b * p.ks0 + (long long)g * p.ks2;
@@ -291,16 +592,30 @@ __global__ void __launch_bounds__(288, 2)
     const long long row0 = r_begin + (long long)it * C::R + 16 * warp;
     const long long nv = r_end - row0;
     const long long nf = p.lo_mask - row0;
-    if (nv > 0 && nf < 16 && !flag[0])
-      decode_subtile<D>(sbase + C::OFF_K + s * C::STAGE_BYTES, sbase + C::OFF_V + s * C::STAGE_BYTES,
-                        C::BLOCK_BYTES, 16 * warp, nf > 0 ? (int)nf : 0, nv > 16 ? 16 : (int)nv, qf,
-                        p.scale_log2, m, l, o, lane);
+    if (nv > 0 && nf < 16 && !flag[0]) {
+      if constexpr (F8)
+        decode_subtile_f8<D>(sbase + C::OFF_K + s * C::STAGE_BYTES, sbase + C::OFF_V + s * C::STAGE_BYTES,
+                             C::BLOCK_BYTES, reinterpret_cast<const float*>(smem + C::OFF_KS) + s * C::R,
+                             reinterpret_cast<const float*>(smem + C::OFF_VS) + s * C::R, 16 * warp,
+                             nf > 0 ? (int)nf : 0, nv > 16 ? 16 : (int)nv, qf, hs, m, l, o, ev, lane);
+      else
+        decode_subtile<D>(sbase + C::OFF_K + s * C::STAGE_BYTES, sbase + C::OFF_V + s * C::STAGE_BYTES,
+                          C::BLOCK_BYTES, 16 * warp, nf > 0 ? (int)nf : 0, nv > 16 ? 16 : (int)nv, qf,
+                          p.scale_log2, m, l, o, lane);
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(empty_bar(s));
   }
-  if (last_split && warp == 0)
-    decode_subtile<D>(sbase + C::OFF_XK, sbase + C::OFF_XV, C::XBLOCK, 0, 0, 1, qf, p.scale_log2, m, l,
-                      o, lane);
+  if (last_split && warp == 0) {
+    if constexpr (F8) {
+      const float* xs = reinterpret_cast<const float*>(smem + C::OFF_XS);
+      decode_subtile_f8<D>(sbase + C::OFF_XK, sbase + C::OFF_XV, C::XBLOCK, xs, xs + 16, 0, 0, 1, qf, hs,
+                           m, l, o, ev, lane);
+    } else {
+      decode_subtile<D>(sbase + C::OFF_XK, sbase + C::OFF_XV, C::XBLOCK, 0, 0, 1, qf, p.scale_log2, m, l,
+                        o, lane);
+    }
+  }
 
   // ---------------------------------------------------------------- merge the consumer warps
   named_bar_sync(1, 32 * C::NCW);   // every warp is done reading the K/V ring
@@ -320,13 +635,27 @@ __global__ void __launch_bounds__(288, 2)
       rw[8 + 2 * t] = l[0];
       rw[8 + 2 * t + 1] = l[1];
     }
+    if constexpr (F8) {
+      // fragment rows r, r + 8 of block md are d = 32(md/2) + 4r + 2(md%2) + {0, 1};
+      // head column e's accumulators are in units of 2^ev[e]
+      const float f0 = ldexpf(1.0f, ev[0]), f1 = ldexpf(1.0f, ev[1]);
 #pragma unroll
-    for (int md = 0; md < D / 16; ++md) {
-      const int d0 = md * 16 + (lane >> 2);
-      rw[16 + (2 * t) * D + d0] = o[md][0];
-      rw[16 + (2 * t + 1) * D + d0] = o[md][1];
-      rw[16 + (2 * t) * D + d0 + 8] = o[md][2];
-      rw[16 + (2 * t + 1) * D + d0 + 8] = o[md][3];
+      for (int md = 0; md < D / 16; ++md) {
+        const int d0 = 32 * (md >> 1) + 4 * (lane >> 2) + 2 * (md & 1);
+        rw[16 + (2 * t) * D + d0] = o[md][0] * f0;
+        rw[16 + (2 * t + 1) * D + d0] = o[md][1] * f1;
+        rw[16 + (2 * t) * D + d0 + 1] = o[md][2] * f0;
+        rw[16 + (2 * t + 1) * D + d0 + 1] = o[md][3] * f1;
+      }
+    } else {
+#pragma unroll
+      for (int md = 0; md < D / 16; ++md) {
+        const int d0 = md * 16 + (lane >> 2);
+        rw[16 + (2 * t) * D + d0] = o[md][0];
+        rw[16 + (2 * t + 1) * D + d0] = o[md][1];
+        rw[16 + (2 * t) * D + d0 + 8] = o[md][2];
+        rw[16 + (2 * t + 1) * D + d0 + 8] = o[md][3];
+      }
     }
   }
   named_bar_sync(1, 32 * C::NCW);

@@ -12,6 +12,7 @@
 
 #include "../../include/sinkattn.h"
 #include "decode.cuh"
+#include "fp8.cuh"
 #include "prefill.cuh"
 #include "ptx.cuh"
 #include "rope.cuh"
@@ -89,6 +90,41 @@ bool make_cache_map(CUtensorMap* map, void* base, int d, int n_kv, long long row
   return r == CUDA_SUCCESS;
 }
 
+// FP8 caches: tensor map over the codes [B][n_kv][cap][d] bytes exposing rows
+// [0, rows_valid), box {rowb, box_rows, 1, 1} swizzled over rowb bytes.
+bool make_codes_map(CUtensorMap* map, void* base, int d, int n_kv, long long rows_valid, int cap,
+                    int B, int box_rows, int rowb) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || rows_valid < 1) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)rows_valid, (cuuint64_t)n_kv, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d, (cuuint64_t)cap * d, (cuuint64_t)n_kv * cap * d};
+  const cuuint32_t box[4] = {(cuuint32_t)rowb, (cuuint32_t)box_rows, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUtensorMapSwizzle sw = rowb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : (rowb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// FP8 caches: tensor map over the row scales [B][n_kv][cap] fp32 exposing
+// rows [0, rows_valid): dims {rows_valid, n_kv, B, 1}, box {box_rows, 1, 1, 1}.
+bool make_scales_map(CUtensorMap* map, void* base, int n_kv, long long rows_valid, int cap, int B,
+                     int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || rows_valid < 1) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)rows_valid, (cuuint64_t)n_kv, (cuuint64_t)B, 1};
+  const cuuint64_t strides[3] = {(cuuint64_t)cap * 4, (cuuint64_t)n_kv * cap * 4,
+                                 (cuuint64_t)B * n_kv * cap * 4};
+  const cuuint32_t box[4] = {(cuuint32_t)box_rows, 1, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Tensor map over a strided [B][T][H][d] bf16 activation (inner dim
 // contiguous, other strides in elements, multiples of 8): dims {d, T, H, B},
 // box {CB, 128, 1, 1} -- one 128-row query tile of one head per CB-wide
@@ -137,6 +173,13 @@ sa_status check_cache(const sa_kv_cache* c) {
   if (!head_dim_ok(c->d)) return SA_ERR_SHAPE;
   if (!aligned16(c->k) || !aligned16(c->v)) return SA_ERR_INVALID_ARG;
   if (c->ring < 0) return SA_ERR_INVALID_ARG;
+  if (c->kv_dtype == SA_KV_FP8_E4M3) {
+    if (c->k_scale == nullptr || c->v_scale == nullptr || !aligned16(c->k_scale) || !aligned16(c->v_scale))
+      return SA_ERR_INVALID_ARG;
+    if (c->cap % 16 != 0) return SA_ERR_SHAPE;
+  } else if (c->kv_dtype != SA_KV_BF16) {
+    return SA_ERR_INVALID_ARG;
+  }
   if (c->ring > 0) {
     if (c->cap % kRingQuantum != 0 || c->ring > c->cap) return SA_ERR_SHAPE;
     if (c->offset < 0 || c->offset > INT32_MAX - 1) return SA_ERR_INVALID_ARG;
@@ -271,17 +314,19 @@ size_t decode_ws_bytes(int B, int n_kv, int q_mult, int d, int S) {
   return cnt + rows * 4 * 2 + rows * d * 4;
 }
 
-template <int D>
+template <int D, bool F8>
 sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, size_t ws_bytes,
                         cudaStream_t stream) {
-  using Cfg = DecodeCfg<D>;
+  using Cfg = sa::DecodeCfgT<D, F8>;
   const int q_mult = a->n_q / c->n_kv;
   DecodeParams p;
   p.off = a->offset;
   p.lo_mask = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
   // a ring's stages start at multiples of the stage height so that none wraps
   p.ring_cap = c->ring > 0 ? c->cap : 0;
-  p.lo = p.ring_cap > 0 ? p.lo_mask / Cfg::R * Cfg::R : p.lo_mask;
+  // FP8 stages start aligned too: the scales' TMA boxes begin at the stage's
+  // first row, their innermost coordinate
+  p.lo = (p.ring_cap > 0 || F8) ? p.lo_mask / Cfg::R * Cfg::R : p.lo_mask;
   const long long n_cache = p.off - p.lo;
   const DecodeSplit sp = decode_split(a->B, c->n_kv, n_cache);
   p.S = sp.S;
@@ -290,14 +335,24 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
     if (ws == nullptr || !aligned16(ws) || ws_bytes < decode_ws_bytes(a->B, c->n_kv, q_mult, D, p.S))
       return SA_ERR_WORKSPACE;
   }
-  CUtensorMap tmK, tmV;
+  CUtensorMap tmK, tmV, tmKS, tmVS;
   memset(&tmK, 0, sizeof(tmK));
   memset(&tmV, 0, sizeof(tmV));
+  memset(&tmKS, 0, sizeof(tmKS));
+  memset(&tmVS, 0, sizeof(tmVS));
   if (n_cache > 0) {
     const long long rows = p.ring_cap > 0 ? (long long)c->cap : p.off;
-    if (!make_cache_map(&tmK, c->k, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::CB) ||
-        !make_cache_map(&tmV, c->v, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::CB))
-      return SA_ERR_CUDA;
+    if constexpr (F8) {
+      if (!make_codes_map(&tmK, c->k, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::ROWB) ||
+          !make_codes_map(&tmV, c->v, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::ROWB) ||
+          !make_scales_map(&tmKS, c->k_scale, c->n_kv, rows, c->cap, c->B, Cfg::R) ||
+          !make_scales_map(&tmVS, c->v_scale, c->n_kv, rows, c->cap, c->B, Cfg::R))
+        return SA_ERR_CUDA;
+    } else {
+      if (!make_cache_map(&tmK, c->k, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::CB) ||
+          !make_cache_map(&tmV, c->v, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::CB))
+        return SA_ERR_CUDA;
+    }
   }
   p.q = static_cast<const __nv_bfloat16*>(a->q);
   p.qs0 = a->q_strides[0];
@@ -311,6 +366,8 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   p.ck = static_cast<__nv_bfloat16*>(c->k);
   p.cv = static_cast<__nv_bfloat16*>(c->v);
   p.cap = c->cap;
+  p.cks = static_cast<float*>(c->k_scale);
+  p.cvs = static_cast<float*>(c->v_scale);
   p.out = static_cast<__nv_bfloat16*>(a->out);
   p.os0 = a->out_strides[0];
   p.os2 = a->out_strides[2];
@@ -333,17 +390,27 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   p.ws_l = reinterpret_cast<float*>(w + cnt + rows * D * 4 + rows * 4);
   static bool configured = false;
   if (!configured) {
-    set_smem(sa::decode_kernel<D>, Cfg::SMEM_BYTES);
+    set_smem(sa::decode_kernel<D, F8>, Cfg::SMEM_BYTES);
     configured = true;
   }
   dim3 grid(c->n_kv, p.S, a->B);
-  sa::decode_kernel<D><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmK, tmV, p);
+  sa::decode_kernel<D, F8><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmK, tmV, tmKS, tmVS, p);
   return last_launch_status();
 }
 
 sa_status launch_append(sa_kv_cache* c, const void* k, const int64_t ks[3], const void* v,
                         const int64_t vs[3], int T, int rope, const float* cos_t,
                         const float* sin_t, cudaStream_t stream) {
+  if (c->kv_dtype == SA_KV_FP8_E4M3) {
+    if (rope) return SA_ERR_UNSUPPORTED;
+    const long long rows = (long long)c->B * T * c->n_kv;   // one warp per row
+    sa::kv_append_fp8_kernel<<<grid_for(rows * 32), 256, 0, stream>>>(
+        static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v), static_cast<float*>(c->k_scale),
+        static_cast<float*>(c->v_scale), c->cap, static_cast<const __nv_bfloat16*>(k), ks[0], ks[1],
+        ks[2], static_cast<const __nv_bfloat16*>(v), vs[0], vs[1], vs[2], c->B, T, c->n_kv, c->d,
+        c->offset, c->ring > 0 ? 1 : 0);
+    return last_launch_status();
+  }
   const long long n = (long long)c->B * T * c->n_kv * (c->d / 16);
   sa::kv_append_kernel<<<grid_for(n), 256, 0, stream>>>(
       static_cast<__nv_bfloat16*>(c->k), static_cast<__nv_bfloat16*>(c->v), c->cap,
@@ -413,6 +480,7 @@ const char* sa_status_string(sa_status s) {
     case SA_ERR_CUDA: return "SA_ERR_CUDA";
     case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT";
     case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
   }
   return "SA_UNKNOWN";
 }
@@ -484,6 +552,18 @@ sa_status sa_kv_cache_init_ring(sa_kv_cache* cache, void* k, void* v, int32_t B,
   return check_cache(cache);
 }
 
+sa_status sa_kv_cache_init_fp8(sa_kv_cache* cache, void* k, void* v, void* k_scale, void* v_scale,
+                               int32_t B, int32_t cap, int32_t n_kv, int32_t d, int32_t window) {
+  if (cache == nullptr || window < 0) return SA_ERR_INVALID_ARG;
+  sa_status st = sa_kv_cache_init(cache, k, v, B, cap, n_kv, d);
+  if (st != SA_OK) return st;
+  cache->ring = window;
+  cache->kv_dtype = SA_KV_FP8_E4M3;
+  cache->k_scale = k_scale;
+  cache->v_scale = v_scale;
+  return check_cache(cache);
+}
+
 sa_status sa_kv_append(sa_kv_cache* cache, const void* k_rot, const int64_t k_strides[3],
                        const void* v, const int64_t v_strides[3], int32_t T, sa_stream_t stream) {
   sa_status st = check_cache(cache);
@@ -536,6 +616,7 @@ sa_status sa_kv_restore(sa_kv_cache* cache, const sa_snapshot* snap) {
 sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* a, sa_stream_t stream) {
   sa_status st = check_attn(cache, a);
   if (st != SA_OK) return st;
+  if (cache->kv_dtype != SA_KV_BF16) return SA_ERR_UNSUPPORTED;
   if (a->T == 0) return SA_OK;
   cudaStream_t s = (cudaStream_t)stream;
   st = launch_stage(cache, a, s);
@@ -561,10 +642,20 @@ sa_status sa_attn_decode(sa_kv_cache* cache, const sa_attn_args* a, void* worksp
   if (a->T != 1) return SA_ERR_INVALID_ARG;
   if (a->n_q / cache->n_kv > 8) return SA_ERR_SHAPE;
   cudaStream_t s = (cudaStream_t)stream;
+  const bool f8 = cache->kv_dtype == SA_KV_FP8_E4M3;
   switch (cache->d) {
-    case 64: st = launch_decode<64>(cache, a, workspace, workspace_bytes, s); break;
-    case 96: st = launch_decode<96>(cache, a, workspace, workspace_bytes, s); break;
-    case 128: st = launch_decode<128>(cache, a, workspace, workspace_bytes, s); break;
+    case 64:
+      st = f8 ? launch_decode<64, true>(cache, a, workspace, workspace_bytes, s)
+              : launch_decode<64, false>(cache, a, workspace, workspace_bytes, s);
+      break;
+    case 96:
+      st = f8 ? launch_decode<96, true>(cache, a, workspace, workspace_bytes, s)
+              : launch_decode<96, false>(cache, a, workspace, workspace_bytes, s);
+      break;
+    case 128:
+      st = f8 ? launch_decode<128, true>(cache, a, workspace, workspace_bytes, s)
+              : launch_decode<128, false>(cache, a, workspace, workspace_bytes, s);
+      break;
     default: return SA_ERR_SHAPE;
   }
   if (st == SA_OK) note_append(cache, cache->offset, 1);
@@ -578,7 +669,8 @@ sa_status sa_attn_decode_static(sa_kv_cache* cache, const sa_attn_args* a, sa_st
   const int q_mult = a->n_q / cache->n_kv;
   if (q_mult > 8) return SA_ERR_SHAPE;
   long long lo = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
-  if (cache->ring > 0) lo = lo / 128 * 128;   // the decode's ring stages start aligned (see launch_decode)
+  if (cache->ring > 0 || cache->kv_dtype == SA_KV_FP8_E4M3)
+    lo = lo / 128 * 128;   // ring and FP8 stages start aligned (see launch_decode)
   const DecodeSplit sp = decode_split(a->B, cache->n_kv, a->offset - lo);
   if (sp.S > 1 && decode_ws_bytes(a->B, cache->n_kv, q_mult, cache->d, sp.S) > SA_DECODE_STATIC_SCRATCH_BYTES)
     return SA_ERR_WORKSPACE;

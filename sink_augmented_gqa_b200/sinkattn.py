@@ -22,8 +22,10 @@ KV_LOG_CAP = 32
 STATUS = {
     0: "SA_OK", 1: "SA_ERR_INVALID_ARG", 2: "SA_ERR_SHAPE", 3: "SA_ERR_CAPACITY",
     4: "SA_ERR_OFFSET_MISMATCH", 5: "SA_ERR_STALE_SNAPSHOT", 6: "SA_ERR_CUDA",
-    7: "SA_ERR_TIMEOUT", 8: "SA_ERR_WORKSPACE",
+    7: "SA_ERR_TIMEOUT", 8: "SA_ERR_WORKSPACE", 9: "SA_ERR_UNSUPPORTED",
 }
+
+KV_BF16, KV_FP8_E4M3 = 0, 1
 
 
 class SinkAttnError(RuntimeError):
@@ -40,7 +42,8 @@ class _KVCache(ctypes.Structure):
         ("offset", ctypes.c_int64), ("seq", ctypes.c_int64), ("high_water", ctypes.c_int64),
         ("log_seq", ctypes.c_int64 * KV_LOG_CAP), ("log_row", ctypes.c_int64 * KV_LOG_CAP),
         ("log_len", ctypes.c_int32), ("log_floor_seq", ctypes.c_int64), ("log_floor_row", ctypes.c_int64),
-        ("ring", ctypes.c_int32),
+        ("ring", ctypes.c_int32), ("kv_dtype", ctypes.c_int32),
+        ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
     ]
 
 
@@ -73,6 +76,7 @@ EXPORTS = (
     "sa_kv_append", "sa_kv_snapshot", "sa_kv_restore", "sa_attn_prefill", "sa_attn_decode",
     "sa_attn_decode_workspace_size", "sa_get_device_status", "sa_set_wait_limit",
     "sa_attn_decode_static", "sa_set_prefill_events", "sa_kv_cache_init_ring",
+    "sa_kv_cache_init_fp8",
 )
 
 _lib = None
@@ -177,16 +181,28 @@ class Snapshot:
 
 
 class KVCache:
-    """One layer's bf16 KV cache, head-major [B, n_kv, cap, d] (torch-owned
-    device memory). ``rows(b_slice, start, stop)`` views rows as [B, T, n_kv, d]."""
+    """One layer's KV cache, head-major [B, n_kv, cap, d] (torch-owned device
+    memory): bf16 rows, or with ``fp8=True`` e4m3 codes (uint8) plus fp32
+    row scales ``k_scale``/``v_scale`` [B, n_kv, cap]. ``k_rows(start,
+    stop)`` views rows as [B, T, n_kv, d]; ``k_scales(start, stop)`` the
+    scales as [B, T, n_kv]."""
 
-    def __init__(self, B, cap, n_kv, d, device="cuda", k=None, v=None, ring=0):
+    def __init__(self, B, cap, n_kv, d, device="cuda", k=None, v=None, ring=0, fp8=False):
         shape = (B, n_kv, cap, d)
-        self.k = k if k is not None else torch.zeros(shape, dtype=torch.bfloat16, device=device)
-        self.v = v if v is not None else torch.zeros(shape, dtype=torch.bfloat16, device=device)
+        dt = torch.uint8 if fp8 else torch.bfloat16
+        self.k = k if k is not None else torch.zeros(shape, dtype=dt, device=device)
+        self.v = v if v is not None else torch.zeros(shape, dtype=dt, device=device)
         assert tuple(self.k.shape) == shape and self.k.is_contiguous() and self.v.is_contiguous()
+        assert self.k.dtype == dt and self.v.dtype == dt
         self.raw = _KVCache()
-        if ring:
+        self.fp8 = bool(fp8)
+        if fp8:
+            self.k_scale = torch.zeros((B, n_kv, cap), dtype=torch.float32, device=self.k.device)
+            self.v_scale = torch.zeros((B, n_kv, cap), dtype=torch.float32, device=self.k.device)
+            _check(lib().sa_kv_cache_init_fp8(ctypes.byref(self.raw), _ptr(self.k), _ptr(self.v),
+                                              _ptr(self.k_scale), _ptr(self.v_scale), B, cap, n_kv, d,
+                                              int(ring)), "sa_kv_cache_init_fp8")
+        elif ring:
             _check(lib().sa_kv_cache_init_ring(ctypes.byref(self.raw), _ptr(self.k), _ptr(self.v), B, cap,
                                                n_kv, d, int(ring)), "sa_kv_cache_init_ring")
         else:
@@ -204,6 +220,13 @@ class KVCache:
 
     def v_rows(self, start=0, stop=None):
         return self._rows(self.v, start, stop)
+
+    def k_scales(self, start=0, stop=None):
+        """FP8 caches: K row scales of positions [start, stop) as [B, T, n_kv]."""
+        return self._rows(self.k_scale, start, stop)
+
+    def v_scales(self, start=0, stop=None):
+        return self._rows(self.v_scale, start, stop)
 
     def _rows(self, t, start, stop):
         if not self.raw.ring:

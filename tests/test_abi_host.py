@@ -163,3 +163,28 @@ def test_ring_cache_host_rules(L):
     assert L.sa_kv_restore(ctypes.byref(c), ctypes.byref(s)) == 0 and c.offset == 5000
     c.offset = c.high_water = 5000 + 768 - 126
     assert L.sa_kv_restore(ctypes.byref(c), ctypes.byref(s)) == 5       # stale
+
+
+def test_fp8_cache_host_rules(L):
+    def init(cap=96, ks=0x30000, vs=0x40000, window=0):
+        c = S._KVCache()
+        st = L.sa_kv_cache_init_fp8(ctypes.byref(c), ctypes.c_void_p(0x10000), ctypes.c_void_p(0x20000),
+                                    ctypes.c_void_p(ks), ctypes.c_void_p(vs), 1, cap, 2, 64, window)
+        return c, st
+    c, st = init()
+    # the struct layout agrees with the header: the library wrote these fields
+    assert st == 0 and c.kv_dtype == S.KV_FP8_E4M3 and c.k_scale == 0x30000 and c.v_scale == 0x40000
+    assert c.ring == 0
+    assert init(ks=0)[1] == 1                  # scales required
+    assert init(vs=0x40008)[1] == 1            # 16-byte aligned scales
+    assert init(cap=100)[1] == 2               # capacity a multiple of 16
+    assert init(cap=768, window=128)[1] == 0   # ring FP8 cache
+    assert init(cap=400, window=128)[1] == 2   # ring rule: multiple of 384
+    assert init(window=-1)[1] == 1
+    stream = ctypes.c_void_p(0)
+    # prefill is not provided on an FP8 cache; the check comes before any launch
+    assert L.sa_attn_prefill(ctypes.byref(c), ctypes.byref(_args(T=4, window=0)), stream) == 9
+    # a bf16 descriptor with an unknown format is rejected
+    b, _ = _fake_cache()
+    b.kv_dtype = 7
+    assert L.sa_kv_snapshot(ctypes.byref(b), ctypes.byref(S._Snapshot())) == 1
