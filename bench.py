@@ -293,10 +293,12 @@ def gptoss_prefill(dev, peaks, reps=10):
     return res
 
 
-def long_decode(dev, peaks, steps=8, layers=24, ring=False):
+def long_decode(dev, peaks, steps=8, layers=24, ring=False, fp8=False):
     """131,072-context decode: 24 layers alternating band / full, one row per
     layer per step, KV bytes actually read / time. ring=True keeps the band
-    layers in 384-row ring caches instead of full-length ones."""
+    layers in 384-row ring caches instead of full-length ones; fp8=True keeps
+    every layer's cache as e4m3 codes with fp32 row scales (the bytes counted
+    are then codes plus scales)."""
     import sink_augmented_gqa_b200 as sa
     cfg = wl.CONFIGS["long_decode"]
     off = cfg.offset
@@ -312,7 +314,7 @@ def long_decode(dev, peaks, steps=8, layers=24, ring=False):
         g.manual_seed(cfg.seed * 1000 + 50_000 + layer)
         if ring and w:
             # a band layer's ring: the last ring_cap positions, up to `off`
-            c = sa.KVCache(cfg.B, ring_cap, cfg.n_kv, cfg.d, device=dev, ring=w)
+            c = sa.KVCache(cfg.B, ring_cap, cfg.n_kv, cfg.d, device=dev, ring=w, fp8=fp8)
             pre_k = torch.empty((cfg.B, ring_cap, cfg.n_kv, cfg.d), dtype=torch.bfloat16, device=dev)
             pre_v = torch.empty_like(pre_k)
             pre_k.normal_(generator=g)
@@ -320,6 +322,15 @@ def long_decode(dev, peaks, steps=8, layers=24, ring=False):
             while c.offset < off:   # the prefix streamed through the ring, one ring-full at a time
                 n = min(ring_cap, off - c.offset)
                 c.append(pre_k[:, :n], pre_v[:, :n])
+        elif fp8:
+            # the prefix generated in bf16, appended (quantised) into the FP8 cache
+            c = sa.KVCache(cfg.B, (cap + 15) // 16 * 16, cfg.n_kv, cfg.d, device=dev, fp8=True)
+            pre_k = torch.empty((cfg.B, off, cfg.n_kv, cfg.d), dtype=torch.bfloat16, device=dev)
+            pre_v = torch.empty_like(pre_k)
+            pre_k.normal_(generator=g)
+            pre_v.normal_(generator=g)
+            c.append(pre_k, pre_v)
+            del pre_k, pre_v
         else:
             c = sa.KVCache(cfg.B, cap, cfg.n_kv, cfg.d, device=dev)
             c.k.normal_(generator=g)
@@ -344,18 +355,47 @@ def long_decode(dev, peaks, steps=8, layers=24, ring=False):
                                cfg.sm_scale, cos, sin, workspace=I["ws"], out=I["out"])
     run_steps()
     torch.cuda.synchronize()
-    # full-layer kernel alone: one layer, one step
-    full = [i for i in range(layers) if ins[i]["window"] == 0][0]
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(10)]
-    for a, b in evs:
-        caches[full].restore(snaps[full])
-        a.record()
-        sa.attn_decode(caches[full], q[:, :1], k[:, :1], v[:, :1], ins[full]["sinks"], 0, cfg.sm_scale, cos, sin,
-                       workspace=ins[full]["ws"], out=ins[full]["out"])
-        b.record()
-    torch.cuda.synchronize()
-    ms_full = statistics.median(a.elapsed_time(b) for a, b in evs)
-    row_bytes = cfg.n_kv * cfg.d * 2 * 2 * cfg.B
+    # K and V of one position of every KV head (FP8: codes plus one fp32 scale each)
+    row_bytes = cfg.n_kv * (cfg.d + 4 if fp8 else cfg.d * 2) * 2 * cfg.B
+
+    def graph_of(layer_ids):
+        """A CUDA graph of one decode call per listed layer (each on its own
+        cache, all at offset `off`): replaying it runs the kernels back to back
+        with no host work between them."""
+        for li in layer_ids:
+            caches[li].restore(snaps[li])
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(gr, stream=side):
+                for li in layer_ids:
+                    I = ins[li]
+                    sa.attn_decode(caches[li], q[:, :1], k[:, :1], v[:, :1], I["sinks"], I["window"], cfg.sm_scale,
+                                   cos, sin, workspace=I["ws"], out=I["out"])
+        torch.cuda.current_stream().wait_stream(side)
+        for li in layer_ids:
+            caches[li].restore(snaps[li])
+        return gr
+
+    def replay_ms(gr, reps):
+        for _ in range(3):
+            gr.replay()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record()
+        for _ in range(reps):
+            gr.replay()
+        g1.record()
+        torch.cuda.synchronize()
+        return g0.elapsed_time(g1) / reps
+
+    # the full-layer kernel: the full layers' calls back to back from a graph,
+    # each on its own cache, so the data streamed (~1.7-3.2 GB) is far beyond L2
+    full_ids = [i for i in range(layers) if ins[i]["window"] == 0]
+    gfull = graph_of(full_ids)
+    ms_full = replay_ms(gfull, 10) / len(full_ids)
+    del gfull
     gbs_full = (off + 1) * row_bytes / (ms_full * 1e-3) / 1e9
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -373,48 +413,31 @@ def long_decode(dev, peaks, steps=8, layers=24, ring=False):
     gbs = nbytes / (ms * 1e-3) / 1e9
     # the same token step (24 layers at offset off) replayed from a CUDA graph:
     # no host launch overhead between the layers
-    for c, sn in zip(caches, snaps):
-        c.restore(sn)
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(side):
-        with torch.cuda.graph(graph, stream=side):
-            for li, c in enumerate(caches):
-                I = ins[li]
-                sa.attn_decode(c, q[:, :1], k[:, :1], v[:, :1], I["sinks"], I["window"], cfg.sm_scale, cos, sin,
-                               workspace=I["ws"], out=I["out"])
-    torch.cuda.current_stream().wait_stream(side)
-    for c, sn in zip(caches, snaps):
-        c.restore(sn)
-    reps = 20
-    for _ in range(3):
-        graph.replay()
-    torch.cuda.synchronize()
-    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    g0.record()
-    for _ in range(reps):
-        graph.replay()
-    g1.record()
-    torch.cuda.synchronize()
-    ms_graph = g0.elapsed_time(g1) / reps
+    graph = graph_of(list(range(layers)))
+    ms_graph = replay_ms(graph, 20)
     gbytes = 0
     for li in range(layers):
         w = ins[li]["window"]
         gbytes += (min(off + 1, w) if w else off + 1) * row_bytes
     gbs_graph = gbytes / (ms_graph * 1e-3) / 1e9
     del graph
-    kv_gib = sum(2 * c.k.numel() * 2 for c in caches) / 2 ** 30
+    kv_gib = sum(2 * (c.k.numel() * c.k.element_size() + (c.k_scale.numel() * 4 if fp8 else 0))
+                 for c in caches) / 2 ** 30
     del caches
     torch.cuda.empty_cache()
     return {"steps": steps, "layers": layers, "ms_per_token_step": round(ms / steps, 4),
             "KV_GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm"], 4),
             "full_layer_kernel": {"ms": round(ms_full, 4), "KV_GB/s": round(gbs_full, 1),
-                                  "frac_of_hbm": round(gbs_full / peaks["hbm"], 4)},
+                                  "frac_of_hbm": round(gbs_full / peaks["hbm"], 4),
+                                  "timing": "device time per launch, full layers back to back from a CUDA graph",
+                                  "traffic": profiled_traffic(
+                                      "decode_long_context_fp8.md" if fp8 else "decode_long_context_full.md",
+                                      ("decode.cuh", "fp8.cuh", "ptx.cuh"))},
             "cuda_graph_token_step": {"ms": round(ms_graph, 4), "KV_GB/s": round(gbs_graph, 1),
                                       "frac_of_hbm": round(gbs_graph / peaks["hbm"], 4)},
             "kv_cache_GiB": round(kv_gib, 3),
-            "cache_layout": "head-major [B][n_kv][cap][d]" + (", band layers in 384-row rings" if ring else "")}
+            "cache_layout": ("head-major [B][n_kv][cap][d]" + (", band layers in 384-row rings" if ring else "")
+                             + (", e4m3 codes + fp32 row scales [B][n_kv][cap]" if fp8 else ", bf16"))}
 
 
 def e2e_lite(step, steps, warmup):
@@ -565,7 +588,8 @@ def run_reference(args, rank, world):
 # Single-call loops for profilers (ncu): no timing, no output but a summary
 # ---------------------------------------------------------------------------
 
-PROFILE_CASES = ("gptoss_prefill_full", "gptoss_prefill_band", "lite_prefill_full", "long_decode_full")
+PROFILE_CASES = ("gptoss_prefill_full", "gptoss_prefill_band", "lite_prefill_full", "long_decode_full",
+                 "long_decode_fp8")
 
 
 def profile_case(name, dev, steps, warmup):
@@ -592,12 +616,20 @@ def profile_case(name, dev, steps, warmup):
         y = cfg.yarn
         cos, sin = sa.yarn_rope_tables(off + 2, cfg.d, y["theta"], y["scaling"], y["orig_ctx"], y["alpha"],
                                        y["beta"], device=dev)
-        cache = sa.KVCache(cfg.B, off + 2, cfg.n_kv, cfg.d, device=dev)
+        fp8 = name.endswith("fp8")
         g = torch.Generator(device=dev)
         g.manual_seed(cfg.seed * 1000 + 50_001)
-        cache.k.normal_(generator=g)
-        cache.v.normal_(generator=g)
-        cache.append(cache.k_rows(0, off), cache.v_rows(0, off))
+        if fp8:
+            cache = sa.KVCache(cfg.B, (off + 2 + 15) // 16 * 16, cfg.n_kv, cfg.d, device=dev, fp8=True)
+            pre = torch.empty((2, cfg.B, off, cfg.n_kv, cfg.d), dtype=torch.bfloat16, device=dev)
+            pre.normal_(generator=g)
+            cache.append(pre[0], pre[1])
+            del pre
+        else:
+            cache = sa.KVCache(cfg.B, off + 2, cfg.n_kv, cfg.d, device=dev)
+            cache.k.normal_(generator=g)
+            cache.v.normal_(generator=g)
+            cache.append(cache.k_rows(0, off), cache.v_rows(0, off))
         snap = cache.snapshot()
         q, k, v = wl.qkv(cfg, 1, device=dev)
         sinks = wl.sinks(cfg, 1, device=dev)
@@ -607,7 +639,7 @@ def profile_case(name, dev, steps, warmup):
         def once():
             cache.restore(snap)
             sa.attn_decode(cache, q, k, v, sinks, 0, cfg.sm_scale, cos, sin, workspace=ws, out=out)
-        units = (off + 1) * cfg.n_kv * cfg.d * 2 * 2 * cfg.B
+        units = (off + 1) * cfg.n_kv * (cfg.d + 4 if fp8 else cfg.d * 2) * 2 * cfg.B
     for _ in range(warmup + steps):
         once()
     torch.cuda.synchronize()
@@ -673,6 +705,8 @@ def main():
         extras["gptoss_prefill_T8192"] = gptoss_prefill(dev, peaks)
         extras["long_context_decode_131072"] = long_decode(dev, peaks)
         extras["long_context_decode_131072_ring"] = long_decode(dev, peaks, ring=True)
+        extras["long_context_decode_131072_fp8"] = long_decode(dev, peaks, fp8=True)
+        extras["long_context_decode_131072_fp8_ring"] = long_decode(dev, peaks, ring=True, fp8=True)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:

@@ -100,6 +100,8 @@ struct DecodeCfg {
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + 8 * (2 * NS) + 16 + 1024;
   static constexpr int BLKCOLS = CB;                    // tensor-map columns per column block
   static constexpr uint32_t STAGE_TX = 2 * STAGE_BYTES;  // bytes one stage's TMA loads bring
+  static constexpr int RW = 16;                         // rows per consumer warp per stage
+  static constexpr int NBOX = 1;                        // 128-row TMA boxes per stage
 };
 
 // FP8 caches: codes rows of D bytes, stored as column blocks of ROWB bytes
@@ -108,14 +110,20 @@ struct DecodeCfg {
 template <int D>
 struct DecodeF8Cfg {
   static constexpr int NCW = 8;
-  static constexpr int R = 16 * NCW;
+  // rows per consumer warp and stage: two 16-row sub-tiles (their dependent
+  // chains interleave) where shared memory allows; a stage is loaded as
+  // 128-row TMA boxes, each starting on a multiple of 128 positions, so no
+  // box wraps a ring
+  static constexpr int RW = (D == 128) ? 16 : 32;
+  static constexpr int R = RW * NCW;
+  static constexpr int NBOX = R / 128;
   static constexpr int ROWB = (D == 96) ? 32 : D;
   static constexpr int NCB = D / ROWB;
   static constexpr int BLKCOLS = ROWB;
   static constexpr uint32_t BLOCK_BYTES = R * ROWB;
   static constexpr uint32_t STAGE_BYTES = R * D;        // K (or V) codes of one stage
-  // as many bytes in flight per CTA as the bf16 kernel keeps
-  static constexpr int NS = (D == 64) ? 6 : (D == 96 ? 4 : 3);
+  // about as many bytes in flight per CTA as the bf16 kernel keeps
+  static constexpr int NS = (D == 96) ? 2 : 3;
   static constexpr uint32_t STAGE_TX = 2 * STAGE_BYTES + 2 * R * 4;
   static constexpr uint32_t XBLOCK = 16 * ROWB;
   static constexpr uint32_t XTILE = 16 * D;
@@ -127,6 +135,7 @@ struct DecodeF8Cfg {
   static constexpr uint32_t OFF_XK = OFF_VS + NS * R * 4;
   static constexpr uint32_t OFF_XV = OFF_XK + XTILE;
   static constexpr uint32_t OFF_XS = OFF_XV + XTILE;         // [2][16] fp32: new-row scales
+  static_assert(RW % 16 == 0 && R % 128 == 0, "stages are whole 128-row boxes of 16-row sub-tiles");
   static constexpr uint32_t OFF_RED = OFF_K;
   static constexpr uint32_t RED_WARP = (16 + 8 * D) * 4;
   static_assert(NCW * RED_WARP <= 2 * NS * STAGE_BYTES, "warp partials must fit in the ring");
@@ -205,18 +214,43 @@ __device__ __forceinline__ void decode_subtile(uint32_t kbase, uint32_t vbase, u
   }
 }
 
-// FP8 counterpart of decode_subtile: codes tiles in swizzled ROWB-byte column
-// blocks, row scales ksc/vsc (indexed by tile row), Q fragments in f16 laid
-// out for the byte order ldmatrix delivers (see the kernel), per-head score
-// scales hs (scale_log2 * 2^e of heads 2(lane%4), +1), and ev[e] the running
-// power of two of head column e's accumulator: O is kept in units of 2^ev,
-// ev the largest exponent of any weight p * scale_v seen so far, so that the
-// f16 weights p * scale_v * 2^-ev stay below 2 and lose only terms under
-// 2^-24 of the largest one.
-template <int D>
-__device__ __forceinline__ void decode_subtile_f8(uint32_t kbase, uint32_t vbase, uint32_t block_bytes,
-                                                  const float* ksc, const float* vsc, int row0,
-                                                  int n_first, int n_valid,
+// Shared-memory offsets (from a stage's K or V base) that the FP8 consumer
+// lane reads for a warp whose sub-tiles start at tile row row0, in 32-byte
+// column group 0 (grp_addr gives the others): ko[u] its ldmatrix row of
+// sub-tile u, vo[u][i] the V rows of logical keys 2cq, 2cq+1, 2cq+8, 2cq+9.
+template <int D, int NSUB>
+__device__ __forceinline__ void f8_offsets(int row0, int lane, uint32_t block_bytes, uint32_t (&ko)[NSUB],
+                                           uint32_t (&vo)[NSUB][4]) {
+  using C = DecodeF8Cfg<D>;
+  const int r = lane >> 2, cq = lane & 3;
+  const int k0 = f8_row<D>(2 * cq), k1 = f8_row<D>(2 * cq + 1);
+#pragma unroll
+  for (int u = 0; u < NSUB; ++u) {
+    const int base = row0 + 16 * u;
+    ko[u] = swz8<C::ROWB>(base + f8_row<D>((lane & 7) + 8 * ((lane >> 3) & 1)), 16 * (lane >> 4), block_bytes);
+    vo[u][0] = swz8<C::ROWB>(base + k0, 4 * r, block_bytes);
+    vo[u][1] = swz8<C::ROWB>(base + k1, 4 * r, block_bytes);
+    vo[u][2] = swz8<C::ROWB>(base + k0 + 8, 4 * r, block_bytes);
+    vo[u][3] = swz8<C::ROWB>(base + k1 + 8, 4 * r, block_bytes);
+  }
+}
+
+// FP8 counterpart of decode_subtile for NSUB consecutive 16-row sub-tiles
+// of a tile stored as swizzled ROWB-byte column blocks (stage bases kst/vst,
+// this lane's offsets ko/vo from f8_offsets; with MASK, keys k < n_first and
+// k >= n_valid, counted from the first row, are masked, without it all
+// 16 NSUB keys are valid), with row scales ksc/vsc from the first row on, Q fragments in f16
+// laid out for the byte order ldmatrix delivers (see the kernel), per-head
+// score scales hs (scale_log2 * 2^e of heads 2(lane%4), +1), and ev[e] the
+// running power of two of head column e's accumulator: O is kept in units of
+// 2^ev, ev the largest exponent of any weight p * scale_v seen so far, so
+// that the f16 weights p * scale_v * 2^-ev stay below 2 and lose only terms
+// under 2^-24 of the largest one. The sub-tiles share one max reduction and
+// one exponent reduction, and their independent chains interleave.
+template <int D, int NSUB, bool MASK>
+__device__ __forceinline__ void decode_subtile_f8(uint32_t kst, uint32_t vst, uint32_t block_bytes,
+                                                  const uint32_t (&ko)[NSUB], const uint32_t (&vo)[NSUB][4],
+                                                  const float* ksc, const float* vsc, int n_first, int n_valid,
                                                   const uint32_t (&qf)[D / 16][2],
                                                   const float (&hs)[2], float (&m)[2], float (&l)[2],
                                                   float (&o)[D / 16][4], int (&ev)[2], int lane) {
@@ -225,53 +259,69 @@ __device__ __forceinline__ void decode_subtile_f8(uint32_t kbase, uint32_t vbase
   // ---- S^T = K Q^T: ldmatrix over bytes gives lane (r, cq) key rows r, r+8 and
   // code bytes 4cq..4cq+3 (+16) of each 32-byte group; its two 16-bit halves
   // are the two K-steps of the group (the Q fragments follow the same order).
-  float c[4] = {0.f, 0.f, 0.f, 0.f};
-  {
-    const int prow = row0 + f8_row<D>((lane & 7) + 8 * ((lane >> 3) & 1));
+  float c[NSUB][4];
+#pragma unroll
+  for (int u = 0; u < NSUB; ++u) {
+    c[u][0] = c[u][1] = c[u][2] = c[u][3] = 0.f;
 #pragma unroll
     for (int grp = 0; grp < D / 32; ++grp) {
       uint32_t r0, r1, r2, r3;
-      ldmatrix_x4(kbase + swz8<C::ROWB>(prow, 32 * grp + 16 * (lane >> 4), block_bytes), r0, r1, r2, r3);
+      ldmatrix_x4(grp_addr<C::ROWB>(kst + ko[u], grp, block_bytes), r0, r1, r2, r3);
 #pragma unroll
       for (int st = 0; st < 2; ++st) {
         const int sh = 16 * st;
-        mma_16816_f16(c, f16x2_from_e4m3x2((uint16_t)(r0 >> sh)), f16x2_from_e4m3x2((uint16_t)(r1 >> sh)),
+        mma_16816_f16(c[u], f16x2_from_e4m3x2((uint16_t)(r0 >> sh)), f16x2_from_e4m3x2((uint16_t)(r1 >> sh)),
                       f16x2_from_e4m3x2((uint16_t)(r2 >> sh)), f16x2_from_e4m3x2((uint16_t)(r3 >> sh)),
                       qf[2 * grp + st][0], qf[2 * grp + st][1]);
       }
     }
   }
-  const int ka = f8_row<D>(r), kb = ka + 8;   // tile rows of logical keys r, r + 8
-  const bool va = ka >= n_first && ka < n_valid, vb = kb >= n_first && kb < n_valid;
-  const float ksa = ksc[row0 + ka], ksb = ksc[row0 + kb];
-  float s[4];
-  s[0] = va ? c[0] * (ksa * hs[0]) : -INFINITY;
-  s[1] = va ? c[1] * (ksa * hs[1]) : -INFINITY;
-  s[2] = vb ? c[2] * (ksb * hs[0]) : -INFINITY;
-  s[3] = vb ? c[3] * (ksb * hs[1]) : -INFINITY;
-  // Masked rows weigh 0 (their scales may be anything a never-written row holds).
-  const float vsa = va ? vsc[row0 + ka] : 0.f, vsb = vb ? vsc[row0 + kb] : 0.f;
-  float pr[4], alpha[2];
+  const int ka = f8_row<D>(r), kb = ka + 8;   // rows (within a sub-tile) of logical keys r, r + 8
+  float s[NSUB][4], vsa[NSUB], vsb[NSUB];
+#pragma unroll
+  for (int u = 0; u < NSUB; ++u) {
+    const int a = 16 * u + ka, bq = 16 * u + kb;
+    const bool va = !MASK || (a >= n_first && a < n_valid);
+    const bool vb = !MASK || (bq >= n_first && bq < n_valid);
+    const float ksa = ksc[a], ksb = ksc[bq];
+    s[u][0] = va ? c[u][0] * (ksa * hs[0]) : -INFINITY;
+    s[u][1] = va ? c[u][1] * (ksa * hs[1]) : -INFINITY;
+    s[u][2] = vb ? c[u][2] * (ksb * hs[0]) : -INFINITY;
+    s[u][3] = vb ? c[u][3] * (ksb * hs[1]) : -INFINITY;
+    // masked rows weigh 0 (their scales may be anything a never-written row holds)
+    vsa[u] = va ? vsc[a] : 0.f;
+    vsb[u] = vb ? vsc[bq] : 0.f;
+  }
+  float pw[NSUB][4], alpha[2];
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
-    float mx = fmaxf(s[e], s[2 + e]);
+    float mx = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < NSUB; ++u) mx = fmaxf(mx, fmaxf(s[u][e], s[u][2 + e]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
     const float m_new = fmaxf(m[e], mx);
     const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
     alpha[e] = ex2(m[e] - m_use);
-    pr[e] = ex2(s[e] - m_use);
-    pr[2 + e] = ex2(s[2 + e] - m_use);
-    l[e] = l[e] * alpha[e] + pr[e] + pr[2 + e];
+    float add = 0.f;
+#pragma unroll
+    for (int u = 0; u < NSUB; ++u) {
+      const float pa = ex2(s[u][e] - m_use), pb = ex2(s[u][2 + e] - m_use);
+      add += pa + pb;
+      pw[u][e] = pa * vsa[u];
+      pw[u][2 + e] = pb * vsb[u];
+    }
+    l[e] = l[e] * alpha[e] + add;
     m[e] = m_new;
   }
   // ---- weights p * scale_v relative to the head's power of two 2^ev (ev
   // never shrinks, so the rescale of O is at most 1)
-  float pw[4] = {pr[0] * vsa, pr[1] * vsa, pr[2] * vsb, pr[3] * vsb};
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
-    float mx = fmaxf(pw[e], pw[2 + e]);
+    float mx = 0.f;
+#pragma unroll
+    for (int u = 0; u < NSUB; ++u) mx = fmaxf(mx, fmaxf(pw[u][e], pw[u][2 + e]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
@@ -284,8 +334,11 @@ __device__ __forceinline__ void decode_subtile_f8(uint32_t kbase, uint32_t vbase
     const float fo = dv < -126 ? 0.f : __uint_as_float((uint32_t)(127 + dv) << 23);
     const float inv = __uint_as_float((uint32_t)(127 - ev_new) << 23);   // 2^-ev_new
     ev[e] = ev_new;
-    pw[e] *= inv;
-    pw[2 + e] *= inv;
+#pragma unroll
+    for (int u = 0; u < NSUB; ++u) {
+      pw[u][e] *= inv;
+      pw[u][2 + e] *= inv;
+    }
     const float ao = alpha[e] * fo;
 #pragma unroll
     for (int md = 0; md < D / 16; ++md) {
@@ -293,31 +346,34 @@ __device__ __forceinline__ void decode_subtile_f8(uint32_t kbase, uint32_t vbase
       o[md][2 + e] *= ao;
     }
   }
-  const uint32_t b01 = movmatrix_trans(pack_f16(pw[0], pw[1]));
-  const uint32_t b23 = movmatrix_trans(pack_f16(pw[2], pw[3]));
   // ---- O^T += V^T P'^T: lane (r, cq) reads one 32-bit word (code bytes
   // 4r..4r+3 of a 32-byte group) from each of the rows of logical keys 2cq,
   // 2cq+1, 2cq+8, 2cq+9 and regroups the bytes into the A fragments of two
   // 16-row blocks of d: block A holds d = 32 grp + 4r + {0, 1}, block B
   // d = 32 grp + 4r + {2, 3} (rows r and r + 8 of the fragment).
   const int k0 = f8_row<D>(2 * cq), k1 = f8_row<D>(2 * cq + 1), k2 = k0 + 8, k3 = k1 + 8;
-  const bool u0 = k0 >= n_first && k0 < n_valid, u1 = k1 >= n_first && k1 < n_valid;
-  const bool u2 = k2 >= n_first && k2 < n_valid, u3 = k3 >= n_first && k3 < n_valid;
 #pragma unroll
-  for (int grp = 0; grp < D / 32; ++grp) {
-    const int bc = 32 * grp + 4 * r;
-    uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;   // rows never written may hold NaN codes
-    if (u0) w0 = ld_shared_u32(vbase + swz8<C::ROWB>(row0 + k0, bc, block_bytes));
-    if (u1) w1 = ld_shared_u32(vbase + swz8<C::ROWB>(row0 + k1, bc, block_bytes));
-    if (u2) w2 = ld_shared_u32(vbase + swz8<C::ROWB>(row0 + k2, bc, block_bytes));
-    if (u3) w3 = ld_shared_u32(vbase + swz8<C::ROWB>(row0 + k3, bc, block_bytes));
-    const uint32_t x01a = __byte_perm(w0, w1, 0x5140), x23a = __byte_perm(w2, w3, 0x5140);
-    const uint32_t x01b = __byte_perm(w0, w1, 0x7362), x23b = __byte_perm(w2, w3, 0x7362);
-    mma_16816_f16(o[2 * grp], f16x2_from_e4m3x2((uint16_t)x01a), f16x2_from_e4m3x2((uint16_t)(x01a >> 16)),
-                  f16x2_from_e4m3x2((uint16_t)x23a), f16x2_from_e4m3x2((uint16_t)(x23a >> 16)), b01, b23);
-    mma_16816_f16(o[2 * grp + 1], f16x2_from_e4m3x2((uint16_t)x01b),
-                  f16x2_from_e4m3x2((uint16_t)(x01b >> 16)), f16x2_from_e4m3x2((uint16_t)x23b),
-                  f16x2_from_e4m3x2((uint16_t)(x23b >> 16)), b01, b23);
+  for (int u = 0; u < NSUB; ++u) {
+    const uint32_t b01 = movmatrix_trans(pack_f16(pw[u][0], pw[u][1]));
+    const uint32_t b23 = movmatrix_trans(pack_f16(pw[u][2], pw[u][3]));
+    const int t0 = 16 * u + k0, t1 = 16 * u + k1, t2 = 16 * u + k2, t3 = 16 * u + k3;
+    const bool u0 = !MASK || (t0 >= n_first && t0 < n_valid), u1 = !MASK || (t1 >= n_first && t1 < n_valid);
+    const bool u2 = !MASK || (t2 >= n_first && t2 < n_valid), u3 = !MASK || (t3 >= n_first && t3 < n_valid);
+#pragma unroll
+    for (int grp = 0; grp < D / 32; ++grp) {
+      uint32_t w0 = 0, w1 = 0, w2 = 0, w3 = 0;   // rows never written may hold NaN codes
+      if (u0) w0 = ld_shared_u32(grp_addr<C::ROWB>(vst + vo[u][0], grp, block_bytes));
+      if (u1) w1 = ld_shared_u32(grp_addr<C::ROWB>(vst + vo[u][1], grp, block_bytes));
+      if (u2) w2 = ld_shared_u32(grp_addr<C::ROWB>(vst + vo[u][2], grp, block_bytes));
+      if (u3) w3 = ld_shared_u32(grp_addr<C::ROWB>(vst + vo[u][3], grp, block_bytes));
+      const uint32_t x01a = __byte_perm(w0, w1, 0x5140), x23a = __byte_perm(w2, w3, 0x5140);
+      const uint32_t x01b = __byte_perm(w0, w1, 0x7362), x23b = __byte_perm(w2, w3, 0x7362);
+      mma_16816_f16(o[2 * grp], f16x2_from_e4m3x2((uint16_t)x01a), f16x2_from_e4m3x2((uint16_t)(x01a >> 16)),
+                    f16x2_from_e4m3x2((uint16_t)x23a), f16x2_from_e4m3x2((uint16_t)(x23a >> 16)), b01, b23);
+      mma_16816_f16(o[2 * grp + 1], f16x2_from_e4m3x2((uint16_t)x01b),
+                    f16x2_from_e4m3x2((uint16_t)(x01b >> 16)), f16x2_from_e4m3x2((uint16_t)x23b),
+                    f16x2_from_e4m3x2((uint16_t)(x23b >> 16)), b01, b23);
+    }
   }
 }
 
@@ -378,20 +434,25 @@ __global__ void __launch_bounds__(288, 2)
         const int s = it % C::NS;
         if (!mbar_wait(empty_bar(s), (uint32_t)(((it / C::NS) & 1) ^ 1))) { flag[0] = 1; break; }
         mbar_arrive_expect_tx(full_bar(s), C::STAGE_TX);
-        const long long pos = r_begin + (long long)it * C::R;   // stages never wrap a ring
-        const int row = (int)(p.ring_cap > 0 ? pos % p.ring_cap : pos);
 #pragma unroll
-        for (int cb = 0; cb < C::NCB; ++cb) {
-          tma_load_4d(sbase + C::OFF_K + s * C::STAGE_BYTES + cb * C::BLOCK_BYTES, &tmK, full_bar(s),
-                      cb * C::BLKCOLS, row, g, b);
-          tma_load_4d(sbase + C::OFF_V + s * C::STAGE_BYTES + cb * C::BLOCK_BYTES, &tmV, full_bar(s),
-                      cb * C::BLKCOLS, row, g, b);
-        }
-        if constexpr (F8) {
-          // row is a multiple of R (the FP8 launch aligns every stage), so the
-          // innermost coordinate of these fp32 boxes is 16-byte aligned
-          tma_load_4d(sbase + C::OFF_KS + s * C::R * 4, &tmKS, full_bar(s), row, g, b, 0);
-          tma_load_4d(sbase + C::OFF_VS + s * C::R * 4, &tmVS, full_bar(s), row, g, b, 0);
+        for (int bx = 0; bx < C::NBOX; ++bx) {
+          // boxes of 128 rows: none wraps a ring (ring stages start on multiples of 128)
+          const long long pos = r_begin + (long long)it * C::R + 128 * bx;
+          const int row = (int)(p.ring_cap > 0 ? pos % p.ring_cap : pos);
+          const uint32_t boff = (uint32_t)bx * 128u * (C::BLOCK_BYTES / C::R);
+#pragma unroll
+          for (int cb = 0; cb < C::NCB; ++cb) {
+            tma_load_4d(sbase + C::OFF_K + s * C::STAGE_BYTES + cb * C::BLOCK_BYTES + boff, &tmK, full_bar(s),
+                        cb * C::BLKCOLS, row, g, b);
+            tma_load_4d(sbase + C::OFF_V + s * C::STAGE_BYTES + cb * C::BLOCK_BYTES + boff, &tmV, full_bar(s),
+                        cb * C::BLKCOLS, row, g, b);
+          }
+          if constexpr (F8) {
+            // row is a multiple of 128 (the FP8 launch aligns every stage), so
+            // the innermost coordinate of these fp32 boxes is 16-byte aligned
+            tma_load_4d(sbase + C::OFF_KS + s * C::R * 4 + bx * 512, &tmKS, full_bar(s), row, g, b, 0);
+            tma_load_4d(sbase + C::OFF_VS + s * C::R * 4 + bx * 512, &tmVS, full_bar(s), row, g, b, 0);
+          }
         }
         issued = it + 1;
         if (flag[0]) break;
@@ -486,6 +547,9 @@ __global__ void __launch_bounds__(288, 2)
     }
   }
   int ev[2] = {-127, -127};   // FP8: powers of two of the two head columns' accumulators
+  // FP8: this lane's shared-memory offsets within a stage (the same for every stage)
+  uint32_t f8ko[C::RW / 16], f8vo[C::RW / 16][4];
+  if constexpr (F8) f8_offsets<D, C::RW / 16>(C::RW * warp, lane, C::BLOCK_BYTES, f8ko, f8vo);
 
   float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
   float o[D / 16][4];
@@ -589,16 +653,22 @@ __global__ void __launch_bounds__(288, 2)
   for (int it = 0; it < n_stages; ++it) {
     const int s = it % C::NS;
     if (!mbar_wait(full_bar(s), (uint32_t)((it / C::NS) & 1))) { flag[0] = 1; break; }
-    const long long row0 = r_begin + (long long)it * C::R + 16 * warp;
+    const long long row0 = r_begin + (long long)it * C::R + C::RW * warp;
     const long long nv = r_end - row0;
     const long long nf = p.lo_mask - row0;
-    if (nv > 0 && nf < 16 && !flag[0]) {
-      if constexpr (F8)
-        decode_subtile_f8<D>(sbase + C::OFF_K + s * C::STAGE_BYTES, sbase + C::OFF_V + s * C::STAGE_BYTES,
-                             C::BLOCK_BYTES, reinterpret_cast<const float*>(smem + C::OFF_KS) + s * C::R,
-                             reinterpret_cast<const float*>(smem + C::OFF_VS) + s * C::R, 16 * warp,
-                             nf > 0 ? (int)nf : 0, nv > 16 ? 16 : (int)nv, qf, hs, m, l, o, ev, lane);
-      else
+    if (nv > 0 && nf < C::RW && !flag[0]) {
+      if constexpr (F8) {
+        const uint32_t kst = sbase + C::OFF_K + s * C::STAGE_BYTES, vst = sbase + C::OFF_V + s * C::STAGE_BYTES;
+        const float* ks = reinterpret_cast<const float*>(smem + C::OFF_KS) + s * C::R + C::RW * warp;
+        const float* vs = reinterpret_cast<const float*>(smem + C::OFF_VS) + s * C::R + C::RW * warp;
+        if (nf <= 0 && nv >= C::RW)
+          decode_subtile_f8<D, C::RW / 16, false>(kst, vst, C::BLOCK_BYTES, f8ko, f8vo, ks, vs, 0, C::RW, qf, hs,
+                                                  m, l, o, ev, lane);
+        else
+          decode_subtile_f8<D, C::RW / 16, true>(kst, vst, C::BLOCK_BYTES, f8ko, f8vo, ks, vs,
+                                                 nf > 0 ? (int)nf : 0, nv > C::RW ? C::RW : (int)nv, qf, hs, m,
+                                                 l, o, ev, lane);
+      } else
         decode_subtile<D>(sbase + C::OFF_K + s * C::STAGE_BYTES, sbase + C::OFF_V + s * C::STAGE_BYTES,
                           C::BLOCK_BYTES, 16 * warp, nf > 0 ? (int)nf : 0, nv > 16 ? 16 : (int)nv, qf,
                           p.scale_log2, m, l, o, lane);
@@ -609,8 +679,10 @@ __global__ void __launch_bounds__(288, 2)
   if (last_split && warp == 0) {
     if constexpr (F8) {
       const float* xs = reinterpret_cast<const float*>(smem + C::OFF_XS);
-      decode_subtile_f8<D>(sbase + C::OFF_XK, sbase + C::OFF_XV, C::XBLOCK, xs, xs + 16, 0, 0, 1, qf, hs,
-                           m, l, o, ev, lane);
+      uint32_t xko[1], xvo[1][4];
+      f8_offsets<D, 1>(0, lane, C::XBLOCK, xko, xvo);
+      decode_subtile_f8<D, 1, true>(sbase + C::OFF_XK, sbase + C::OFF_XV, C::XBLOCK, xko, xvo, xs, xs + 16, 0, 1,
+                                    qf, hs, m, l, o, ev, lane);
     } else {
       decode_subtile<D>(sbase + C::OFF_XK, sbase + C::OFF_XV, C::XBLOCK, 0, 0, 1, qf, p.scale_log2, m, l,
                         o, lane);

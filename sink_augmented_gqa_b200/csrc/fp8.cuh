@@ -64,6 +64,16 @@ __device__ __forceinline__ uint32_t swz8(int row, int bcol, uint32_t block_bytes
   return off ^ (((off >> 7) & MASK) << 4);
 }
 
+// Address of 32-byte column group grp given the address of group 0 (same row,
+// same byte within the group) in a swizzled tile: with ROWB >= 64 the group
+// sits in address bits 5.. below the swizzle's source bits, so it is an XOR;
+// with 32-byte blocks each group is its own block, block_bytes apart (a
+// multiple of 256, which leaves the swizzle unchanged).
+template <int ROWB>
+__device__ __forceinline__ uint32_t grp_addr(uint32_t a0, int grp, uint32_t block_bytes) {
+  return ROWB == 32 ? a0 + (uint32_t)grp * block_bytes : a0 ^ (uint32_t)(32 * grp);
+}
+
 // Quantise one row held by a warp, two elements per lane per pass
 // (x[i] = elements 2*lane + 64*i, +1; passes with 2*lane + 64*i >= d hold
 // zeros and are not stored). Writes codes to dst (device bytes) and returns

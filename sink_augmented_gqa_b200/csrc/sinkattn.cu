@@ -292,15 +292,16 @@ struct DecodeSplit {
   long long chunk;
 };
 
-DecodeSplit decode_split(int B, int n_kv, long long n_cache) {
-  DecodeSplit r{1, 64};
+// stage: cache rows per ring stage of the decode kernel (its Cfg::R); every
+// split but the last covers whole stages.
+DecodeSplit decode_split(int B, int n_kv, long long n_cache, long long stage) {
+  DecodeSplit r{1, stage};
   if (n_cache <= 0) return r;
   const long long target = 2LL * num_sms();
   long long S = (target + (long long)B * n_kv - 1) / ((long long)B * n_kv);
   if (S < 1) S = 1;
   long long chunk = (n_cache + S - 1) / S;
-  constexpr long long kStage = 128;   // decode rows per ring stage (DecodeCfg<D>::R)
-  chunk = ((chunk + kStage - 1) / kStage) * kStage;
+  chunk = ((chunk + stage - 1) / stage) * stage;
   r.chunk = chunk;
   r.S = (int)((n_cache + chunk - 1) / chunk);
   return r;
@@ -328,7 +329,7 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   // first row, their innermost coordinate
   p.lo = (p.ring_cap > 0 || F8) ? p.lo_mask / Cfg::R * Cfg::R : p.lo_mask;
   const long long n_cache = p.off - p.lo;
-  const DecodeSplit sp = decode_split(a->B, c->n_kv, n_cache);
+  const DecodeSplit sp = decode_split(a->B, c->n_kv, n_cache, Cfg::R);
   p.S = sp.S;
   p.chunk = sp.chunk;
   if (p.S > 1) {
@@ -342,15 +343,17 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   memset(&tmVS, 0, sizeof(tmVS));
   if (n_cache > 0) {
     const long long rows = p.ring_cap > 0 ? (long long)c->cap : p.off;
+    constexpr int kBoxRows = Cfg::R / Cfg::NBOX;   // a stage is NBOX boxes of 128 rows
+    static_assert(kBoxRows == 128, "decode TMA boxes are 128 rows");
     if constexpr (F8) {
-      if (!make_codes_map(&tmK, c->k, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::ROWB) ||
-          !make_codes_map(&tmV, c->v, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::ROWB) ||
-          !make_scales_map(&tmKS, c->k_scale, c->n_kv, rows, c->cap, c->B, Cfg::R) ||
-          !make_scales_map(&tmVS, c->v_scale, c->n_kv, rows, c->cap, c->B, Cfg::R))
+      if (!make_codes_map(&tmK, c->k, D, c->n_kv, rows, c->cap, c->B, kBoxRows, Cfg::ROWB) ||
+          !make_codes_map(&tmV, c->v, D, c->n_kv, rows, c->cap, c->B, kBoxRows, Cfg::ROWB) ||
+          !make_scales_map(&tmKS, c->k_scale, c->n_kv, rows, c->cap, c->B, kBoxRows) ||
+          !make_scales_map(&tmVS, c->v_scale, c->n_kv, rows, c->cap, c->B, kBoxRows))
         return SA_ERR_CUDA;
     } else {
-      if (!make_cache_map(&tmK, c->k, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::CB) ||
-          !make_cache_map(&tmV, c->v, D, c->n_kv, rows, c->cap, c->B, Cfg::R, Cfg::CB))
+      if (!make_cache_map(&tmK, c->k, D, c->n_kv, rows, c->cap, c->B, kBoxRows, Cfg::CB) ||
+          !make_cache_map(&tmV, c->v, D, c->n_kv, rows, c->cap, c->B, kBoxRows, Cfg::CB))
         return SA_ERR_CUDA;
     }
   }
@@ -669,9 +672,13 @@ sa_status sa_attn_decode_static(sa_kv_cache* cache, const sa_attn_args* a, sa_st
   const int q_mult = a->n_q / cache->n_kv;
   if (q_mult > 8) return SA_ERR_SHAPE;
   long long lo = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
-  if (cache->ring > 0 || cache->kv_dtype == SA_KV_FP8_E4M3)
-    lo = lo / 128 * 128;   // ring and FP8 stages start aligned (see launch_decode)
-  const DecodeSplit sp = decode_split(a->B, cache->n_kv, a->offset - lo);
+  // the split of launch_decode: ring and FP8 stages start on multiples of the stage height
+  const bool f8 = cache->kv_dtype == SA_KV_FP8_E4M3;
+  const long long stage = f8 ? (cache->d == 128 ? sa::DecodeF8Cfg<128>::R : sa::DecodeF8Cfg<64>::R) : 128;
+  static_assert(sa::DecodeF8Cfg<64>::R == sa::DecodeF8Cfg<96>::R, "one FP8 stage height for d = 64, 96");
+  static_assert(sa::DecodeCfg<64>::R == 128 && sa::DecodeCfg<128>::R == 128, "bf16 stage height");
+  if (cache->ring > 0 || f8) lo = lo / stage * stage;
+  const DecodeSplit sp = decode_split(a->B, cache->n_kv, a->offset - lo, stage);
   if (sp.S > 1 && decode_ws_bytes(a->B, cache->n_kv, q_mult, cache->d, sp.S) > SA_DECODE_STATIC_SCRATCH_BYTES)
     return SA_ERR_WORKSPACE;
   void* scratch = nullptr;
