@@ -19,6 +19,10 @@ Modules, each citing the passage it restates:
                    STACK"; GQA Attention study note, "How it works").
 * ``kvcache``   -- the append-only KV cache with snapshot / restore and the
                    KV-byte estimator (MoE-Xtend README, "KV CACHE").
+* ``linear``    -- pre-norm RMSNorm, the fused qkv linear and the out
+                   projection with the residual add (GQA Attention study
+                   note, "How it works"; pinned by
+                   ``tests/test_oracle_linear.py``).
 * ``fp8``       -- E4M3 rows with one fp32 scale per row: quantise and
                    dequantise (MoE-Xtend README, "ROADMAP": KV quantisation
                    with dequantisation; the format is a reading, pinned by
@@ -29,4 +33,4 @@ except the two readings listed there as "parity unpinned" (the RoPE pair
 convention against a real checkpoint, and the GPT-OSS-Lite rotary base).
 """
 
-from . import bf16, yarn, rope, attention, kvcache, fp8  # noqa: F401
+from . import bf16, yarn, rope, attention, kvcache, fp8, linear  # noqa: F401
