@@ -318,6 +318,51 @@ size_t sa_attn_decode_workspace_size(int32_t B, int32_t n_q, int32_t n_kv, int32
 sa_status sa_attn_decode_static(sa_kv_cache* cache, const sa_attn_args* args, sa_stream_t stream);
 
 /*
+ * The dense projections around the attention (GQA Attention study note, "How
+ * it works": the residual stream x [T, 2880] goes through pre-norm RMSNorm
+ * and one fused linear qkv of width d_h (n_q + 2 n_kv) = 5120 whose columns
+ * are q, then k, then v; after attention the heads, flattened to [T, 4096],
+ * go through the linear out back to [T, 2880], added to the residual; both
+ * linears are bf16 with bias). Matrices are row-major bf16 with leading
+ * dimensions (ld*, in elements, multiples of 8, >= the row width); bases
+ * 16-byte aligned. Weights follow nn.Linear: W [N][K], y = x W^T + b. The
+ * product runs on tcgen05 tensor cores with fp32 accumulation, one rounding
+ * to bf16 at the end. Errors: SA_ERR_INVALID_ARG for a null or misaligned
+ * pointer, a bad leading dimension, M < 0, N or K < 1; SA_ERR_CUDA if a
+ * launch fails. M == 0 is a no-op.
+ */
+
+/*
+ * Fold RMSNorm's gain into the qkv weight, once per model: w_folded[n][k] =
+ * bf16(w[n][k] * gamma[k]) (the product formed exactly, rounded once).
+ * w, w_folded: [N][K] bf16 (ld ldw / ldf); gamma: fp32 [K]. May be in place.
+ */
+sa_status sa_rmsnorm_fold_weight(const void* w, int64_t ldw, const float* gamma, void* w_folded,
+                                 int64_t ldf, int32_t N, int32_t K, sa_stream_t stream);
+
+/*
+ * Pre-norm RMSNorm + fused qkv projection:
+ *   y[m][n] = (sum_k x[m][k] w_folded[n][k]) / sqrt(mean_k x[m][k]^2 + eps) + bias[n]
+ * which is RMSNorm(x; gamma, eps) W^T + b with w_folded from
+ * sa_rmsnorm_fold_weight. x [M][K], y [M][N] (e.g. the fused q|k|v rows
+ * that sa_attn_prefill / sa_attn_decode take as strided views), bias bf16
+ * [N] or NULL, eps >= 0. The row statistics come from the same x tiles the
+ * product reads; the normalised x is never written. y must not overlap x.
+ */
+sa_status sa_qkv_proj(const void* x, int64_t ldx, const void* w_folded, int64_t ldw, const void* bias,
+                      float eps, void* y, int64_t ldy, int32_t M, int32_t N, int32_t K, sa_stream_t stream);
+
+/*
+ * Out projection with the residual add, in place: x[m][n] += sum_k
+ * o[m][k] w[n][k] + bias[n] (the sum, the bias and the old x added in fp32,
+ * rounded once). o [M][K] (the attention output flattened over heads),
+ * w [N][K], bias bf16 [N] or NULL, x [M][N] the residual stream. o must not
+ * overlap x.
+ */
+sa_status sa_out_proj(const void* o, int64_t ldo, const void* w, int64_t ldw, const void* bias, void* x,
+                      int64_t ldx, int32_t M, int32_t N, int32_t K, sa_stream_t stream);
+
+/*
  * Reads and clears the device status word of the current device (waits for
  * the device to be idle). *code receives SA_OK or SA_ERR_TIMEOUT.
  */

@@ -16,6 +16,9 @@ from .sinkattn import (  # noqa: F401
     decode_workspace,
     decode_workspace_bytes,
     device_status,
+    out_proj,
+    qkv_proj,
+    rmsnorm_fold_weight,
     rope_apply_qk,
     set_prefill_events,
     set_wait_limit,

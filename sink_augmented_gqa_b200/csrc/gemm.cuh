@@ -1,0 +1,352 @@
+// The dense projections around the attention, as one persistent tcgen05 GEMM
+// with fused prologue / epilogue work (GQA Attention study note, "How it
+// works": pre-norm RMSNorm, the fused linear qkv of width d_h (n_q + 2 n_kv),
+// and after attention the linear out back to the residual width with the
+// residual add; both linears bf16 with bias):
+//
+//   y[m][n] = s_m * sum_k a[m][k] w[n][k] + bias[n] (+ residual[m][n])
+//
+// with s_m = 1 / sqrt(mean_k a[m][k]^2 + eps) for the qkv projection (the
+// RMSNorm gain gamma is folded into w once, w[n][k] * gamma[k], so the
+// normalised activations are never materialised) and s_m = 1 for the out
+// projection, whose epilogue adds the residual (x <- x + out(o), in place).
+//
+// One CTA per SM walks 128 x 256 output tiles (tile t, t + grid, ...):
+//
+//   warp 0      TMA producer: per 64-wide K step, the A tile (128 x 64) and
+//               the W tile (256 x 64), 128-byte swizzled, into a 4-deep ring.
+//   warp 1      one thread issues tcgen05.mma (kind::f16, M 128, N 256, K 16
+//               per instruction, fp32 accumulation in TMEM); the tile's
+//               accumulator alternates between two 256-column TMEM buffers so
+//               the epilogue of one tile overlaps the main loop of the next.
+//   warps 2, 3  (RMSNorm only) sum the squares of each A row from the same
+//               shared-memory tiles the tensor core reads, and publish s_m.
+//   warps 4-7   epilogue, one output row per thread (TMEM lane = row): per
+//               32-column chunk, tcgen05.ld, scale, bias, residual, bf16,
+//               staged in shared memory (64-byte swizzle) and written by a
+//               TMA tile store (which clips the ragged edges of M and N).
+#pragma once
+
+#include "ptx.cuh"
+
+namespace sa {
+
+struct GemmParams {
+  int M, N, K;
+  const __nv_bfloat16* bias;      // [N] or null
+  const __nv_bfloat16* residual;  // [M] rows of ldr elements, or null; may alias the output
+  long long ldr;
+  int rms;                        // 1: scale row m by 1 / sqrt(mean_k a^2 + eps)
+  float eps;
+  int tiles_m, tiles_n;
+};
+
+struct GemmCfg {
+  static constexpr int BM = 128, BN = 256, BK = 64;
+  static constexpr int NS = 4;                               // ring depth
+  static constexpr uint32_t A_BYTES = BM * BK * 2;           // 16 KB
+  static constexpr uint32_t B_BYTES = BN * BK * 2;           // 32 KB
+  static constexpr uint32_t OFF_A = 0;
+  static constexpr uint32_t OFF_B = NS * A_BYTES;
+  static constexpr uint32_t OFF_ST = OFF_B + NS * B_BYTES;   // [4 warps][2] 32 rows x 64 B
+  static constexpr uint32_t ST_BYTES = 32 * 64;
+  static constexpr uint32_t OFF_RMS = OFF_ST + 8 * ST_BYTES;  // [2][128] fp32 row scales
+  static constexpr uint32_t OFF_BAR = OFF_RMS + 2 * 128 * 4;
+  static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;   // + alignment slack
+  static constexpr int TMEM_COLS = 512;
+  static constexpr uint32_t IDESC = idesc_bf16(128, 256, 0, 0);
+  static constexpr uint32_t SBO = 1024;                      // 8 rows x 128 B
+  static constexpr int NUM_THREADS = 256;
+  static_assert(OFF_B % 1024 == 0 && OFF_ST % 1024 == 0, "swizzled buffers need 1 KB alignment");
+};
+
+enum : int {
+  GB_FULL = 0,        // [NS] producer -> MMA, RMS warps: A and W tiles landed
+  GB_EMPTY = 4,       // [NS] MMA (commit) + RMS warps -> producer
+  GB_ACC_FULL = 8,    // [2] MMA -> epilogue: the tile's accumulator is complete
+  GB_ACC_EMPTY = 10,  // [2] epilogue warps -> MMA: accumulator read
+  GB_RMS_FULL = 12,   // [2] RMS warps -> epilogue: row scales of the tile
+  GB_RMS_EMPTY = 14,  // [2] epilogue warps -> RMS warps
+  GB_DRAIN = 16,      // MMA issuer, on abort
+  GB_TMEM_SLOT = 17,
+  GB_ABORT_SLOT = 18,
+};
+
+__device__ __forceinline__ void bulk_wait_read_1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(256, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
+  using C = GemmCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * GB_TMEM_SLOT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * GB_ABORT_SLOT);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_tiles = p.tiles_m * p.tiles_n;
+  const int n_kb = (p.K + C::BK - 1) / C::BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(bar(GB_FULL + s), 1);
+      mbar_init(bar(GB_EMPTY + s), p.rms ? 3 : 1);   // MMA commit (+ one arrival per RMS warp)
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(GB_ACC_FULL + b), 1);
+      mbar_init(bar(GB_ACC_EMPTY + b), 4);
+      mbar_init(bar(GB_RMS_FULL + b), 2);
+      mbar_init(bar(GB_RMS_EMPTY + b), 4);
+    }
+    mbar_init(bar(GB_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmC);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // output tiles walk M fastest, so CTAs running side by side share W tiles
+  auto tile_origin = [&](int t, int& m0, int& n0) {
+    m0 = (t % p.tiles_m) * C::BM;
+    n0 = (t / p.tiles_m) * C::BN;
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        int m0, n0;
+        tile_origin(t, m0, n0);
+        for (int kb = 0; kb < n_kb; ++kb) {
+          const int s = it % C::NS;
+          const uint32_t ph = (uint32_t)((it / C::NS) & 1);
+          if (it >= C::NS && !mbar_wait(bar(GB_EMPTY + s), ph ^ 1)) { ok = false; break; }
+          if (*abort_flag) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(GB_FULL + s), C::A_BYTES + C::B_BYTES);
+          tma_load_4d(sbase + C::OFF_A + s * C::A_BYTES, &tmA, bar(GB_FULL + s), kb * C::BK, m0, 0, 0);
+          tma_load_4d(sbase + C::OFF_B + s * C::B_BYTES, &tmB, bar(GB_FULL + s), kb * C::BK, n0, 0, 0);
+          ++it;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        // let every copy still in flight land before the CTA can exit
+        for (int u = (it > C::NS ? it - C::NS : 0); u < it; ++u)
+          mbar_wait_drain(bar(GB_FULL + u % C::NS), (uint32_t)((u / C::NS) & 1));
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      const uint64_t ad0 = smem_desc(sbase + C::OFF_A, 16, C::SBO, 2u);
+      const uint64_t bd0 = smem_desc(sbase + C::OFF_B, 16, C::SBO, 2u);
+      int it = 0, tl = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+        const int buf = tl & 1;
+        if (tl >= 2 && !mbar_wait(bar(GB_ACC_EMPTY + buf), (uint32_t)(((tl >> 1) - 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(buf * C::BN);
+        for (int kb = 0; kb < n_kb; ++kb, ++it) {
+          const int s = it % C::NS;
+          if (!mbar_wait(bar(GB_FULL + s), (uint32_t)((it / C::NS) & 1))) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = ad0 + ((uint32_t)(s * C::A_BYTES) >> 4);
+          const uint64_t bd = bd0 + ((uint32_t)(s * C::B_BYTES) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < C::BK / 16; ++kk)   // 32 bytes further along the swizzled rows
+            mma_ss(d, ad + 2 * kk, bd + 2 * kk, C::IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar(GB_EMPTY + s));
+        }
+        if (!ok) break;
+        mma_commit(bar(GB_ACC_FULL + buf));
+        if (*abort_flag) { ok = false; break; }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        mma_commit(bar(GB_DRAIN));
+        mbar_wait_drain(bar(GB_DRAIN), 0);
+      }
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ RMSNorm row scales
+    if (p.rms) {
+      const int r0 = 32 * (warp - 2) + lane, r1 = r0 + 64;   // rows of the A tile
+      const float inv_k = 1.0f / (float)p.K;
+      int it = 0, tl = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+        float s0 = 0.f, s1 = 0.f;
+        for (int kb = 0; kb < n_kb; ++kb, ++it) {
+          const int s = it % C::NS;
+          if (!mbar_wait(bar(GB_FULL + s), (uint32_t)((it / C::NS) & 1))) { ok = false; break; }
+          const uint8_t* a = smem + C::OFF_A + s * C::A_BYTES;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {   // 16-byte chunk j of a row sits at chunk j ^ (row % 8)
+            const uint4 u0 = *reinterpret_cast<const uint4*>(a + r0 * 128 + ((j ^ (r0 & 7)) << 4));
+            const uint4 u1 = *reinterpret_cast<const uint4*>(a + r1 * 128 + ((j ^ (r1 & 7)) << 4));
+            const uint32_t w0[4] = {u0.x, u0.y, u0.z, u0.w}, w1[4] = {u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float a0 = bf16_lo(w0[e]), a1 = bf16_hi(w0[e]);
+              const float b0 = bf16_lo(w1[e]), b1 = bf16_hi(w1[e]);
+              s0 = fmaf(a0, a0, fmaf(a1, a1, s0));
+              s1 = fmaf(b0, b0, fmaf(b1, b1, s1));
+            }
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(GB_EMPTY + s));
+        }
+        if (!ok) break;
+        const int buf = tl & 1;
+        if (tl >= 2 && !mbar_wait(bar(GB_RMS_EMPTY + buf), (uint32_t)(((tl >> 1) - 1) & 1))) { ok = false; break; }
+        float* rb = reinterpret_cast<float*>(smem + C::OFF_RMS) + buf * 128;
+        rb[r0] = 1.0f / sqrtf(s0 * inv_k + p.eps);
+        rb[r1] = 1.0f / sqrtf(s1 * inv_k + p.eps);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(GB_RMS_FULL + buf));
+        if (*abort_flag) { ok = false; break; }
+      }
+      if (!ok) *abort_flag = 1;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                  // TMEM lane quarter of this warp
+    const int r = 32 * q + lane;             // row within the tile
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    int tl = 0, cnt = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+      int m0, n0;
+      tile_origin(t, m0, n0);
+      const int buf = tl & 1;
+      if (!mbar_wait(bar(GB_ACC_FULL + buf), (uint32_t)((tl >> 1) & 1))) { ok = false; break; }
+      tc_fence_after();
+      float sc = 1.f;
+      if (p.rms) {
+        if (!mbar_wait(bar(GB_RMS_FULL + buf), (uint32_t)((tl >> 1) & 1))) { ok = false; break; }
+        sc = reinterpret_cast<const float*>(smem + C::OFF_RMS)[buf * 128 + r];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(GB_RMS_EMPTY + buf));
+      }
+      const int m = m0 + r;
+      const bool row_ok = m < p.M;
+      const int nch = min(C::BN / 32, (p.N - n0 + 31) / 32);
+      for (int c = 0; c < nch; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem + lane_base + (uint32_t)(buf * C::BN + 32 * c), v);
+        tmem_wait_ld();
+        const int nb = n0 + 32 * c;
+        const bool full = nb + 32 <= p.N;
+        float y[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) y[j] = __uint_as_float(v[j]) * sc;
+        if (p.bias) {
+          if (full) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              const uint4 bv = __ldg(reinterpret_cast<const uint4*>(p.bias + nb + j));
+              y[j + 0] += bf16_lo(bv.x); y[j + 1] += bf16_hi(bv.x);
+              y[j + 2] += bf16_lo(bv.y); y[j + 3] += bf16_hi(bv.y);
+              y[j + 4] += bf16_lo(bv.z); y[j + 5] += bf16_hi(bv.z);
+              y[j + 6] += bf16_lo(bv.w); y[j + 7] += bf16_hi(bv.w);
+            }
+          } else {
+            for (int j = 0; j < 32; ++j)
+              if (nb + j < p.N) y[j] += __bfloat162float(p.bias[nb + j]);
+          }
+        }
+        if (p.residual && row_ok) {
+          const __nv_bfloat16* rr = p.residual + (long long)m * p.ldr + nb;
+          if (full) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 8) {
+              const uint4 rv = *reinterpret_cast<const uint4*>(rr + j);
+              y[j + 0] += bf16_lo(rv.x); y[j + 1] += bf16_hi(rv.x);
+              y[j + 2] += bf16_lo(rv.y); y[j + 3] += bf16_hi(rv.y);
+              y[j + 4] += bf16_lo(rv.z); y[j + 5] += bf16_hi(rv.z);
+              y[j + 6] += bf16_lo(rv.w); y[j + 7] += bf16_hi(rv.w);
+            }
+          } else {
+            for (int j = 0; j < 32; ++j)
+              if (nb + j < p.N) y[j] += __bfloat162float(rr[j]);
+          }
+        }
+        // stage the 32 x 32 chunk of this warp (64-byte rows, 64-byte swizzle:
+        // 16-byte chunk j of row r at j ^ ((r / 2) % 4)) and store it by TMA
+        const int sb = cnt & 1;
+        uint8_t* st = smem + C::OFF_ST + (uint32_t)(q * 2 + sb) * C::ST_BYTES;
+        if (cnt >= 2) {
+          if (lane == 0) bulk_wait_read_1();   // the store that last used this buffer has read it
+          __syncwarp();
+        }
+#pragma unroll
+        for (int j4 = 0; j4 < 4; ++j4) {
+          uint4 w;
+          w.x = pack_bf16(y[8 * j4 + 0], y[8 * j4 + 1]);
+          w.y = pack_bf16(y[8 * j4 + 2], y[8 * j4 + 3]);
+          w.z = pack_bf16(y[8 * j4 + 4], y[8 * j4 + 5]);
+          w.w = pack_bf16(y[8 * j4 + 6], y[8 * j4 + 7]);
+          *reinterpret_cast<uint4*>(st + lane * 64 + ((j4 ^ ((lane >> 1) & 3)) << 4)) = w;
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (m0 + 32 * q < p.M)   // rows past M are clipped; a wholly outside chunk is not stored
+            tma_store_4d(&tmC, smem_u32(st), nb, m0 + 32 * q, 0, 0);
+          bulk_commit();
+        }
+        ++cnt;
+      }
+      // the accumulator buffer is free for the tile after next
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(GB_ACC_EMPTY + buf));
+      if (*abort_flag) { ok = false; break; }
+    }
+    if (lane == 0) bulk_wait_all();   // output stores complete before the CTA exits
+    if (!ok) *abort_flag = 1;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// w_folded[n][k] = bf16(w[n][k] * gamma[k]), the product formed exactly in
+// fp64 and rounded once (RMSNorm's gain folded into the qkv weight).
+__global__ void fold_gamma_kernel(const __nv_bfloat16* __restrict__ w, long long ldw,
+                                  const float* __restrict__ gamma, __nv_bfloat16* __restrict__ out,
+                                  long long ldo, int N, int K) {
+  const long long n_el = (long long)N * K;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n_el;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int n = (int)(idx / K), k = (int)(idx % K);
+    const double prod = (double)__bfloat162float(w[n * ldw + k]) * (double)gamma[k];
+    out[n * ldo + k] = __ushort_as_bfloat16((unsigned short)bf16_bits_from_f64(prod));
+  }
+}
+
+}  // namespace sa

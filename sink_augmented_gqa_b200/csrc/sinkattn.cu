@@ -13,6 +13,7 @@
 #include "../../include/sinkattn.h"
 #include "decode.cuh"
 #include "fp8.cuh"
+#include "gemm.cuh"
 #include "prefill.cuh"
 #include "ptx.cuh"
 #include "rope.cuh"
@@ -122,6 +123,22 @@ bool make_scales_map(CUtensorMap* map, void* base, int n_kv, long long rows_vali
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Tensor map over a row-major bf16 matrix [rows][ld] exposing columns
+// [0, cols): dims {cols, rows, 1, 1}, box {box_cols, box_rows, 1, 1}.
+bool make_matrix_map(CUtensorMap* map, const void* base, long long cols, long long rows, long long ld,
+                     int box_cols, int box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || rows < 1 || cols < 1) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)cols, (cuuint64_t)rows, 1, 1};
+  const cuuint64_t strides[3] = {(cuuint64_t)ld * 2, (cuuint64_t)ld * 2 * rows, (cuuint64_t)ld * 2 * rows};
+  const cuuint32_t box[4] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -468,6 +485,43 @@ sa_status static_scratch(void** out) {
   return SA_OK;
 }
 
+// Projections around the attention: one GEMM launch (csrc/gemm.cuh).
+
+bool matrix_ok(const void* p, int64_t ld, int64_t cols) {
+  return p != nullptr && aligned16(p) && ld >= cols && ld % 8 == 0;
+}
+
+sa_status launch_gemm(const void* a, int64_t lda, const void* w, int64_t ldw, const void* bias,
+                      const void* residual, int64_t ldr, void* y, int64_t ldy, int32_t M, int32_t N,
+                      int32_t K, int rms, float eps, cudaStream_t stream) {
+  using C = sa::GemmCfg;
+  CUtensorMap tmA, tmB, tmC;
+  if (!make_matrix_map(&tmA, a, K, M, lda, C::BK, C::BM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_matrix_map(&tmB, w, K, N, ldw, C::BK, C::BN, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_matrix_map(&tmC, y, N, M, ldy, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return SA_ERR_CUDA;
+  sa::GemmParams p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.bias = static_cast<const __nv_bfloat16*>(bias);
+  p.residual = static_cast<const __nv_bfloat16*>(residual);
+  p.ldr = ldr;
+  p.rms = rms;
+  p.eps = eps;
+  p.tiles_m = (M + C::BM - 1) / C::BM;
+  p.tiles_n = (N + C::BN - 1) / C::BN;
+  const long long tiles = (long long)p.tiles_m * p.tiles_n;
+  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  static bool configured = false;
+  if (!configured) {
+    set_smem(sa::gemm_kernel, C::SMEM_BYTES);
+    configured = true;
+  }
+  sa::gemm_kernel<<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tmA, tmB, tmC, p);
+  return last_launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -694,6 +748,35 @@ size_t sa_attn_decode_workspace_size(int32_t B, int32_t n_q, int32_t n_kv, int32
   const long long units = 512 + (long long)B * n_kv;
   const size_t cnt = (((size_t)B * n_kv * 4) + 255) / 256 * 256;
   return cnt + (size_t)units * q_mult * (2 + d) * 4;
+}
+
+sa_status sa_rmsnorm_fold_weight(const void* w, int64_t ldw, const float* gamma, void* w_folded,
+                                 int64_t ldf, int32_t N, int32_t K, sa_stream_t stream) {
+  if (N < 1 || K < 1 || gamma == nullptr || !matrix_ok(w, ldw, K) || !matrix_ok(w_folded, ldf, K))
+    return SA_ERR_INVALID_ARG;
+  sa::fold_gamma_kernel<<<grid_for((long long)N * K), 256, 0, (cudaStream_t)stream>>>(
+      static_cast<const __nv_bfloat16*>(w), ldw, gamma, static_cast<__nv_bfloat16*>(w_folded), ldf, N, K);
+  return last_launch_status();
+}
+
+sa_status sa_qkv_proj(const void* x, int64_t ldx, const void* w_folded, int64_t ldw, const void* bias,
+                      float eps, void* y, int64_t ldy, int32_t M, int32_t N, int32_t K, sa_stream_t stream) {
+  if (M < 0 || N < 1 || K < 1 || !(eps >= 0.f) || !isfinite(eps)) return SA_ERR_INVALID_ARG;
+  if (M == 0) return SA_OK;
+  if (!matrix_ok(x, ldx, K) || !matrix_ok(w_folded, ldw, K) || !matrix_ok(y, ldy, N) ||
+      (bias != nullptr && !aligned16(bias)))
+    return SA_ERR_INVALID_ARG;
+  return launch_gemm(x, ldx, w_folded, ldw, bias, nullptr, 0, y, ldy, M, N, K, 1, eps, (cudaStream_t)stream);
+}
+
+sa_status sa_out_proj(const void* o, int64_t ldo, const void* w, int64_t ldw, const void* bias, void* x,
+                      int64_t ldx, int32_t M, int32_t N, int32_t K, sa_stream_t stream) {
+  if (M < 0 || N < 1 || K < 1) return SA_ERR_INVALID_ARG;
+  if (M == 0) return SA_OK;
+  if (!matrix_ok(o, ldo, K) || !matrix_ok(w, ldw, K) || !matrix_ok(x, ldx, N) ||
+      (bias != nullptr && !aligned16(bias)))
+    return SA_ERR_INVALID_ARG;
+  return launch_gemm(o, ldo, w, ldw, bias, x, ldx, x, ldx, M, N, K, 0, 0.f, (cudaStream_t)stream);
 }
 
 sa_status sa_get_device_status(int32_t* code) {

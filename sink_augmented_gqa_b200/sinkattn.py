@@ -76,7 +76,7 @@ EXPORTS = (
     "sa_kv_append", "sa_kv_snapshot", "sa_kv_restore", "sa_attn_prefill", "sa_attn_decode",
     "sa_attn_decode_workspace_size", "sa_get_device_status", "sa_set_wait_limit",
     "sa_attn_decode_static", "sa_set_prefill_events", "sa_kv_cache_init_ring",
-    "sa_kv_cache_init_fp8",
+    "sa_kv_cache_init_fp8", "sa_rmsnorm_fold_weight", "sa_qkv_proj", "sa_out_proj",
 )
 
 _lib = None
@@ -110,6 +110,11 @@ def lib():
         L.sa_get_device_status.argtypes = [P(i32)]
         L.sa_set_wait_limit.argtypes = [i64]
         L.sa_set_prefill_events.argtypes = [vp, vp]
+        L.sa_kv_cache_init_fp8.argtypes = [P(_KVCache), vp, vp, vp, vp, i32, i32, i32, i32, i32]
+        f32 = ctypes.c_float
+        L.sa_rmsnorm_fold_weight.argtypes = [vp, i64, vp, vp, i64, i32, i32, vp]
+        L.sa_qkv_proj.argtypes = [vp, i64, vp, i64, vp, f32, vp, i64, i32, i32, i32, vp]
+        L.sa_out_proj.argtypes = [vp, i64, vp, i64, vp, vp, i64, i32, i32, i32, vp]
         for name in EXPORTS:
             if name not in ("sa_status_string", "sa_attn_decode_workspace_size"):
                 getattr(L, name).restype = ctypes.c_int
@@ -314,6 +319,45 @@ def attn_decode(cache, q, k, v, sinks, window, sm_scale, cos=None, sin=None, rop
                                 workspace.numel() * workspace.element_size(), _stream(q)),
            "sa_attn_decode")
     return (out, lse) if return_lse else out
+
+
+def _require_matrix(name, t):
+    if not (t.is_cuda and t.dtype == torch.bfloat16 and t.dim() == 2 and t.stride(1) == 1):
+        raise TypeError(f"{name} must be a 2-D bf16 CUDA tensor with contiguous rows")
+
+
+def rmsnorm_fold_weight(w, gamma, out=None):
+    """w [N, K] bf16, gamma fp32 [K] -> bf16(w * gamma) (RMSNorm gain folded in)."""
+    _require_matrix("w", w)
+    if out is None:
+        out = torch.empty_like(w)
+    _check(lib().sa_rmsnorm_fold_weight(_ptr(w), w.stride(0), _ptr(gamma), _ptr(out), out.stride(0),
+                                        w.shape[0], w.shape[1], _stream(w)), "sa_rmsnorm_fold_weight")
+    return out
+
+
+def qkv_proj(x, w_folded, bias, eps, out=None):
+    """RMSNorm(x) W^T + b with the gain folded into w_folded: x [M, K] -> [M, N]."""
+    _require_matrix("x", x)
+    _require_matrix("w_folded", w_folded)
+    M, K = x.shape
+    N = w_folded.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().sa_qkv_proj(_ptr(x), x.stride(0), _ptr(w_folded), w_folded.stride(0), _ptr(bias),
+                             float(eps), _ptr(out), out.stride(0), M, N, K, _stream(x)), "sa_qkv_proj")
+    return out
+
+
+def out_proj(o, w, bias, x):
+    """x += o W^T + b in place (o [M, K], w [N, K], x [M, N]); returns x."""
+    for n, t in (("o", o), ("w", w), ("x", x)):
+        _require_matrix(n, t)
+    M, K = o.shape
+    N = w.shape[0]
+    _check(lib().sa_out_proj(_ptr(o), o.stride(0), _ptr(w), w.stride(0), _ptr(bias), _ptr(x), x.stride(0),
+                             M, N, K, _stream(o)), "sa_out_proj")
+    return x
 
 
 def attn_decode_static(cache, q, k, v, sinks, window, sm_scale, cos=None, sin=None, rope_fused=True,
