@@ -23,6 +23,10 @@ Modules, each citing the passage it restates:
                    projection with the residual add (GQA Attention study
                    note, "How it works"; pinned by
                    ``tests/test_oracle_linear.py``).
+* ``backward``  -- gradients of the attention with respect to q, k, v and
+                   the sinks (GPT-OSS-Lite README: learned sinks, trained
+                   end to end); pinned to finite differences by
+                   ``tests/test_oracle_backward.py``.
 * ``fp8``       -- E4M3 rows with one fp32 scale per row: quantise and
                    dequantise (MoE-Xtend README, "ROADMAP": KV quantisation
                    with dequantisation; the format is a reading, pinned by
@@ -33,4 +37,4 @@ except the two readings listed there as "parity unpinned" (the RoPE pair
 convention against a real checkpoint, and the GPT-OSS-Lite rotary base).
 """
 
-from . import bf16, yarn, rope, attention, kvcache, fp8, linear  # noqa: F401
+from . import bf16, yarn, rope, attention, kvcache, fp8, linear, backward  # noqa: F401
