@@ -318,6 +318,56 @@ size_t sa_attn_decode_workspace_size(int32_t B, int32_t n_q, int32_t n_kv, int32
 sa_status sa_attn_decode_static(sa_kv_cache* cache, const sa_attn_args* args, sa_stream_t stream);
 
 /*
+ * Backward pass of sink-augmented GQA attention, for a sequence attending to
+ * itself (a training step: no cache prefix, positions 0..T-1), on the
+ * ROTATED q and k the forward used (GPT-OSS-Lite README, "Architecture":
+ * learned attention sinks, trained end to end). With P the forward's softmax
+ * weights (sink column included in the normalisation), D_i = <dO_i, o_i>
+ * and dS = P (dO V^T - D):
+ *   dq = sm_scale dS K,  dk = sm_scale dS^T Q,  dv = P^T dO
+ *   (dk, dv summed over the q_mult heads of each KV group),
+ *   dsinks[h] = -sum_{b,i} exp(sinks[h] - lse[b][h][i]) D_i.
+ * Gradients with respect to unrotated q, k: apply sa_rope_apply_qk with the
+ * sin table negated (the rotation's transpose).
+ *
+ * q, k, v, out (the forward's output), d_out: device bf16 [B][T][H][d] via
+ *   strides (inner dimension contiguous, strides multiples of 8), 16-byte
+ *   aligned.
+ * lse    : the forward's fp32 [B][n_q][T] log-sum-exp (sa_attn_prefill's lse).
+ * sinks  : fp32 [n_q] or NULL (no sink; dsinks is then not written).
+ * window : <= 0 full causal, > 0 band of `window` keys.
+ * dq     : fp32 [B][T][n_q][d] dense; dk, dv: fp32 [B][T][n_kv][d] dense;
+ *   dsinks: fp32 [n_q] (overwritten) or NULL. All outputs are written, not
+ *   accumulated into.
+ * workspace: device memory of sa_attn_backward_workspace_size() bytes
+ *   (16-byte aligned, contents irrelevant).
+ * Products run on the tensor cores (bf16 operands, fp32 accumulation); P and
+ * dS enter their products as bf16. Errors: SA_ERR_INVALID_ARG (null,
+ * misaligned, bad stride, B/T/n_q < 1), SA_ERR_SHAPE (d not in {64, 96,
+ * 128}, n_q % n_kv != 0), SA_ERR_WORKSPACE (too small), SA_ERR_CUDA.
+ */
+typedef struct sa_attn_bwd_args {
+  const void* q;     int64_t q_strides[3];
+  const void* k;     int64_t k_strides[3];
+  const void* v;     int64_t v_strides[3];
+  const void* out;   int64_t out_strides[3];
+  const void* d_out; int64_t d_out_strides[3];
+  const float* lse;
+  const float* sinks;
+  int32_t B, T, n_q, n_kv, d;
+  int32_t window;
+  float sm_scale;
+  float* dq;
+  float* dk;
+  float* dv;
+  float* dsinks;
+} sa_attn_bwd_args;
+
+sa_status sa_attn_backward(const sa_attn_bwd_args* args, void* workspace, size_t workspace_bytes,
+                           sa_stream_t stream);
+size_t sa_attn_backward_workspace_size(int32_t B, int32_t T, int32_t n_q);
+
+/*
  * The dense projections around the attention (GQA Attention study note, "How
  * it works": the residual stream x [T, 2880] goes through pre-norm RMSNorm
  * and one fused linear qkv of width d_h (n_q + 2 n_kv) = 5120 whose columns

@@ -10,6 +10,7 @@ built.
 from .sinkattn import (  # noqa: F401
     KVCache,
     SinkAttnError,
+    attn_backward,
     attn_decode,
     attn_decode_static,
     attn_prefill,

@@ -121,10 +121,12 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  // output tiles walk M fastest, so CTAs running side by side share W tiles
+  // output tiles walk N fastest: the ~grid tiles in flight at a time cover all
+  // of W and a band of grid / tiles_n row tiles of A, which together stay in L2
+  // (every A row is read from DRAM once; W once per pass over it)
   auto tile_origin = [&](int t, int& m0, int& n0) {
-    m0 = (t % p.tiles_m) * C::BM;
-    n0 = (t / p.tiles_m) * C::BN;
+    n0 = (t % p.tiles_n) * C::BN;
+    m0 = (t / p.tiles_n) * C::BM;
   };
 
   if (warp == 0) {

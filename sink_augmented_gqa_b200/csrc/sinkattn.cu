@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/sinkattn.h"
+#include "backward.cuh"
 #include "decode.cuh"
 #include "fp8.cuh"
 #include "gemm.cuh"
@@ -522,6 +523,51 @@ sa_status launch_gemm(const void* a, int64_t lda, const void* w, int64_t ldw, co
   return last_launch_status();
 }
 
+// Backward pass (csrc/backward.cuh): row pass, key-tile pass, query-tile pass.
+template <int D>
+sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t stream) {
+  using Cfg = sa::BwdCfg<D>;
+  sa::BwdParams p;
+  p.q = static_cast<const __nv_bfloat16*>(a->q);
+  p.k = static_cast<const __nv_bfloat16*>(a->k);
+  p.v = static_cast<const __nv_bfloat16*>(a->v);
+  p.o = static_cast<const __nv_bfloat16*>(a->out);
+  p.dout = static_cast<const __nv_bfloat16*>(a->d_out);
+  p.qs0 = a->q_strides[0]; p.qs1 = a->q_strides[1]; p.qs2 = a->q_strides[2];
+  p.ks0 = a->k_strides[0]; p.ks1 = a->k_strides[1]; p.ks2 = a->k_strides[2];
+  p.vs0 = a->v_strides[0]; p.vs1 = a->v_strides[1]; p.vs2 = a->v_strides[2];
+  p.os0 = a->out_strides[0]; p.os1 = a->out_strides[1]; p.os2 = a->out_strides[2];
+  p.ds0 = a->d_out_strides[0]; p.ds1 = a->d_out_strides[1]; p.ds2 = a->d_out_strides[2];
+  p.lse = a->lse;
+  p.sinks = a->sinks;
+  p.dvec = dvec;
+  p.dq = a->dq;
+  p.dk = a->dk;
+  p.dv = a->dv;
+  p.dsinks = a->sinks ? a->dsinks : nullptr;
+  p.B = a->B;
+  p.T = a->T;
+  p.n_q = a->n_q;
+  p.n_kv = a->n_kv;
+  p.q_mult = a->n_q / a->n_kv;
+  p.window = a->window;
+  p.scale = a->sm_scale;
+  p.scale_log2 = a->sm_scale * 1.4426950408889634f;
+  if (p.dsinks && cudaMemsetAsync(p.dsinks, 0, sizeof(float) * a->n_q, stream) != cudaSuccess) return SA_ERR_CUDA;
+  const long long rows = (long long)a->B * a->T * a->n_q;
+  sa::bwd_rows_kernel<D><<<grid_for(rows * 32), 256, 0, stream>>>(p);
+  static bool configured = false;
+  if (!configured) {
+    set_smem(sa::bwd_dkdv_kernel<D>, Cfg::SMEM_BYTES);
+    set_smem(sa::bwd_dq_kernel<D>, Cfg::SMEM_BYTES);
+    configured = true;
+  }
+  const int tiles = (a->T + Cfg::TILE - 1) / Cfg::TILE;
+  sa::bwd_dkdv_kernel<D><<<dim3(tiles, a->n_kv, a->B), 128, Cfg::SMEM_BYTES, stream>>>(p);
+  sa::bwd_dq_kernel<D><<<dim3(tiles, a->n_q, a->B), 128, Cfg::SMEM_BYTES, stream>>>(p);
+  return last_launch_status();
+}
+
 }  // namespace
 
 extern "C" {
@@ -777,6 +823,36 @@ sa_status sa_out_proj(const void* o, int64_t ldo, const void* w, int64_t ldw, co
       (bias != nullptr && !aligned16(bias)))
     return SA_ERR_INVALID_ARG;
   return launch_gemm(o, ldo, w, ldw, bias, x, ldx, x, ldx, M, N, K, 0, 0.f, (cudaStream_t)stream);
+}
+
+size_t sa_attn_backward_workspace_size(int32_t B, int32_t T, int32_t n_q) {
+  if (B < 1 || T < 1 || n_q < 1) return 0;
+  return ((size_t)B * n_q * T * 4 + 255) / 256 * 256;
+}
+
+sa_status sa_attn_backward(const sa_attn_bwd_args* a, void* workspace, size_t workspace_bytes,
+                           sa_stream_t stream) {
+  if (a == nullptr || a->B < 1 || a->T < 1 || a->n_q < 1 || a->n_kv < 1) return SA_ERR_INVALID_ARG;
+  if (!head_dim_ok(a->d)) return SA_ERR_SHAPE;
+  if (a->n_q % a->n_kv != 0) return SA_ERR_SHAPE;
+  const void* ins[5] = {a->q, a->k, a->v, a->out, a->d_out};
+  const int64_t* st[5] = {a->q_strides, a->k_strides, a->v_strides, a->out_strides, a->d_out_strides};
+  for (int i = 0; i < 5; ++i)
+    if (ins[i] == nullptr || !aligned16(ins[i]) || !strides_ok(st[i])) return SA_ERR_INVALID_ARG;
+  if (a->lse == nullptr || a->dq == nullptr || a->dk == nullptr || a->dv == nullptr) return SA_ERR_INVALID_ARG;
+  if (!aligned16(a->dq) || !aligned16(a->dk) || !aligned16(a->dv)) return SA_ERR_INVALID_ARG;
+  if (!(a->sm_scale > 0.f) || !isfinite(a->sm_scale)) return SA_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned16(workspace) ||
+      workspace_bytes < sa_attn_backward_workspace_size(a->B, a->T, a->n_q))
+    return SA_ERR_WORKSPACE;
+  float* dvec = static_cast<float*>(workspace);
+  cudaStream_t s = (cudaStream_t)stream;
+  switch (a->d) {
+    case 64: return launch_backward<64>(a, dvec, s);
+    case 96: return launch_backward<96>(a, dvec, s);
+    case 128: return launch_backward<128>(a, dvec, s);
+  }
+  return SA_ERR_SHAPE;
 }
 
 sa_status sa_get_device_status(int32_t* code) {

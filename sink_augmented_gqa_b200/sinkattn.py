@@ -47,6 +47,20 @@ class _KVCache(ctypes.Structure):
     ]
 
 
+class _BwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("q_strides", ctypes.c_int64 * 3),
+        ("k", ctypes.c_void_p), ("k_strides", ctypes.c_int64 * 3),
+        ("v", ctypes.c_void_p), ("v_strides", ctypes.c_int64 * 3),
+        ("out", ctypes.c_void_p), ("out_strides", ctypes.c_int64 * 3),
+        ("d_out", ctypes.c_void_p), ("d_out_strides", ctypes.c_int64 * 3),
+        ("lse", ctypes.c_void_p), ("sinks", ctypes.c_void_p),
+        ("B", ctypes.c_int32), ("T", ctypes.c_int32), ("n_q", ctypes.c_int32), ("n_kv", ctypes.c_int32),
+        ("d", ctypes.c_int32), ("window", ctypes.c_int32), ("sm_scale", ctypes.c_float),
+        ("dq", ctypes.c_void_p), ("dk", ctypes.c_void_p), ("dv", ctypes.c_void_p), ("dsinks", ctypes.c_void_p),
+    ]
+
+
 class _Snapshot(ctypes.Structure):
     _fields_ = [("cache_id", ctypes.c_uint64), ("offset", ctypes.c_int64),
                 ("seq", ctypes.c_int64), ("cap", ctypes.c_int32)]
@@ -77,6 +91,7 @@ EXPORTS = (
     "sa_attn_decode_workspace_size", "sa_get_device_status", "sa_set_wait_limit",
     "sa_attn_decode_static", "sa_set_prefill_events", "sa_kv_cache_init_ring",
     "sa_kv_cache_init_fp8", "sa_rmsnorm_fold_weight", "sa_qkv_proj", "sa_out_proj",
+    "sa_attn_backward", "sa_attn_backward_workspace_size",
 )
 
 _lib = None
@@ -115,8 +130,12 @@ def lib():
         L.sa_rmsnorm_fold_weight.argtypes = [vp, i64, vp, vp, i64, i32, i32, vp]
         L.sa_qkv_proj.argtypes = [vp, i64, vp, i64, vp, f32, vp, i64, i32, i32, i32, vp]
         L.sa_out_proj.argtypes = [vp, i64, vp, i64, vp, vp, i64, i32, i32, i32, vp]
+        L.sa_attn_backward.argtypes = [P(_BwdArgs), vp, ctypes.c_size_t, vp]
+        L.sa_attn_backward_workspace_size.restype = ctypes.c_size_t
+        L.sa_attn_backward_workspace_size.argtypes = [i32, i32, i32]
         for name in EXPORTS:
-            if name not in ("sa_status_string", "sa_attn_decode_workspace_size"):
+            if name not in ("sa_status_string", "sa_attn_decode_workspace_size",
+                            "sa_attn_backward_workspace_size"):
                 getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -358,6 +377,41 @@ def out_proj(o, w, bias, x):
     _check(lib().sa_out_proj(_ptr(o), o.stride(0), _ptr(w), w.stride(0), _ptr(bias), _ptr(x), x.stride(0),
                              M, N, K, _stream(o)), "sa_out_proj")
     return x
+
+
+def attn_backward(q, k, v, out, d_out, lse, sinks, window, sm_scale, workspace=None):
+    """Gradients of a self-attention call (offset 0) with respect to the
+    rotated q, k, v and the sinks. q/k/v/out/d_out [B, T, H, d] bf16 (strided
+    views allowed), lse [B, n_q, T] fp32 from the forward. Returns (dq, dk,
+    dv, dsinks) fp32 (dsinks None without sinks)."""
+    B, T, n_q, d = q.shape
+    n_kv = k.shape[2]
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("d_out", d_out)):
+        _require_bf16_cuda(n, t)
+    dev = q.device
+    dq = torch.empty((B, T, n_q, d), dtype=torch.float32, device=dev)
+    dk = torch.empty((B, T, n_kv, d), dtype=torch.float32, device=dev)
+    dv = torch.empty((B, T, n_kv, d), dtype=torch.float32, device=dev)
+    dsinks = None if sinks is None else torch.empty(n_q, dtype=torch.float32, device=dev)
+    if workspace is None:
+        nb = lib().sa_attn_backward_workspace_size(B, T, n_q)
+        workspace = torch.empty(nb, dtype=torch.uint8, device=dev)
+    a = _BwdArgs()
+    a.q, a.q_strides = q.data_ptr(), _strides(q)
+    a.k, a.k_strides = k.data_ptr(), _strides(k)
+    a.v, a.v_strides = v.data_ptr(), _strides(v)
+    a.out, a.out_strides = out.data_ptr(), _strides(out)
+    a.d_out, a.d_out_strides = d_out.data_ptr(), _strides(d_out)
+    a.lse = lse.data_ptr()
+    a.sinks = 0 if sinks is None else sinks.data_ptr()
+    a.B, a.T, a.n_q, a.n_kv, a.d = B, T, n_q, n_kv, d
+    a.window = int(window)
+    a.sm_scale = float(sm_scale)
+    a.dq, a.dk, a.dv = dq.data_ptr(), dk.data_ptr(), dv.data_ptr()
+    a.dsinks = 0 if dsinks is None else dsinks.data_ptr()
+    _check(lib().sa_attn_backward(ctypes.byref(a), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(q)), "sa_attn_backward")
+    return dq, dk, dv, dsinks
 
 
 def attn_decode_static(cache, q, k, v, sinks, window, sm_scale, cos=None, sin=None, rope_fused=True,
