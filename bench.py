@@ -293,6 +293,95 @@ def gptoss_prefill(dev, peaks, reps=10):
     return res
 
 
+def projection_inputs(dev, which, T=8192):
+    """Seeded inputs of the gpt-oss projections at T rows: ("qkv") x [T, 2880],
+    RMSNorm gain, qkv weight [5120, 2880] with bias; ("out") attention output
+    [T, 4096], out weight [2880, 4096] with bias, residual x [T, 2880]."""
+    seed = wl.CONFIGS["gptoss_prefill"].seed
+    N, K = (5120, 2880) if which == "qkv" else (2880, 4096)
+    a = wl.randn_bf16((T, K), seed, 70_000, dev)
+    w = (wl.randn_bf16((N, K), seed, 70_001, dev).float() / math.sqrt(K)).to(torch.bfloat16)
+    b = wl.randn_bf16((N,), seed, 70_002, dev)
+    extra = (wl.randn_bf16((K,), seed, 70_003, dev).float().abs() + 0.5 if which == "qkv"
+             else wl.randn_bf16((T, N), seed, 70_004, dev))
+    return a, w, b, extra
+
+
+def projections(dev, peaks, reps=20):
+    """The dense projections around a gpt-oss attention layer at T = 8192:
+    RMSNorm + fused qkv (2880 -> 5120) and the out projection with the
+    residual add (4096 -> 2880), on the tensor cores; 2 T N K flops each.
+    Back-to-back launches between CUDA events; each call's operands and
+    output (138-160 MB) exceed L2."""
+    import sink_augmented_gqa_b200 as sa
+    T = 8192
+    res = {}
+    for which in ("qkv", "out"):
+        a, w, b, extra = projection_inputs(dev, which, T)
+        N, K = w.shape
+        if which == "qkv":
+            wf = sa.rmsnorm_fold_weight(w, extra)
+            y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+            fn = lambda: sa.qkv_proj(a, wf, b, 1e-5, out=y)
+        else:
+            fn = lambda: sa.out_proj(a, w, b, extra)
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        tf = 2 * T * N * K / (ms * 1e-3) / 1e12
+        res[f"{which}_proj_T8192"] = {"M_N_K": [T, N, K], "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                                      "frac_of_bf16_peak": round(tf / peaks["tf"], 4),
+                                      "traffic": profiled_traffic(f"gemm_gptoss_{which}_proj.md",
+                                                                  ("gemm.cuh", "ptx.cuh"))}
+    return res
+
+
+def lite_backward(dev, peaks, reps=10):
+    """Backward pass of a Lite training layer (B = 8, T = 4096, 8/4 heads,
+    d = 96), full causal and band, after the library's own forward. Work is
+    counted as the algorithmic 5 products of the backward (S, dP, dV, dK,
+    dQ: 10 d flops per admitted pair and head); the kernels recompute S and
+    dP for dQ, which is not counted."""
+    import sink_augmented_gqa_b200 as sa
+    cfg = wl.CONFIGS["lite"]
+    res = {}
+    for layer in (1, 0):
+        window = cfg.layer_window(layer)
+        q, k, v = wl.qkv(cfg, cfg.T, layer=layer, device=dev)
+        dout = wl.randn_bf16((cfg.B, cfg.T, cfg.n_q, cfg.d), cfg.seed, 124, dev)
+        sinks = wl.sinks(cfg, layer, device=dev)
+        cache = sa.KVCache(cfg.B, cfg.T, cfg.n_kv, cfg.d, device=dev)
+        out, lse = sa.attn_prefill(cache, q, k, v, sinks, window, cfg.sm_scale, rope_fused=False, return_lse=True)
+        ws = torch.empty(sa.sinkattn.lib().sa_attn_backward_workspace_size(cfg.B, cfg.T, cfg.n_q),
+                         dtype=torch.uint8, device=dev)
+
+        def once():
+            sa.attn_backward(q, k, v, out, dout, lse, sinks, window, cfg.sm_scale, workspace=ws)
+        for _ in range(3):
+            once()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            once()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        f = 10 * cfg.d * cfg.B * cfg.n_q * pairs(0, cfg.T, window)
+        tf = f / (ms * 1e-3) / 1e12
+        res["full" if window == 0 else "band"] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                                                  "frac_of_bf16_peak": round(tf / peaks["tf"], 4)}
+        del cache
+    return res
+
+
 def long_decode(dev, peaks, steps=8, layers=24, ring=False, fp8=False):
     """131,072-context decode: 24 layers alternating band / full, one row per
     layer per step, KV bytes actually read / time. ring=True keeps the band
@@ -589,12 +678,25 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------
 
 PROFILE_CASES = ("gptoss_prefill_full", "gptoss_prefill_band", "lite_prefill_full", "long_decode_full",
-                 "long_decode_fp8")
+                 "long_decode_fp8", "gptoss_qkv_proj", "gptoss_out_proj")
 
 
 def profile_case(name, dev, steps, warmup):
     import sink_augmented_gqa_b200 as sa
-    if name.startswith("gptoss") or name.startswith("lite"):
+    if name.endswith("_proj"):
+        which = "qkv" if "qkv" in name else "out"
+        a, w, b, extra = projection_inputs(dev, which)
+        N, K = w.shape
+        if which == "qkv":
+            wf = sa.rmsnorm_fold_weight(w, extra)
+
+            def once():
+                sa.qkv_proj(a, wf, b, 1e-5)
+        else:
+            def once():
+                sa.out_proj(a, w, b, extra)
+        units = 2 * a.shape[0] * N * K
+    elif name.startswith("gptoss") or name.startswith("lite"):
         cfg = wl.CONFIGS["gptoss_prefill" if name.startswith("gptoss") else "lite"]
         window = cfg.window if name.endswith("band") else 0
         y = cfg.yarn
@@ -703,6 +805,8 @@ def main():
     extras = {}
     if not args.no_extras and rank == 0:
         extras["gptoss_prefill_T8192"] = gptoss_prefill(dev, peaks)
+        extras["gptoss_projections"] = projections(dev, peaks)
+        extras["lite_backward_T4096"] = lite_backward(dev, peaks)
         extras["long_context_decode_131072"] = long_decode(dev, peaks)
         extras["long_context_decode_131072_ring"] = long_decode(dev, peaks, ring=True)
         extras["long_context_decode_131072_fp8"] = long_decode(dev, peaks, fp8=True)
