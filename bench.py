@@ -678,12 +678,24 @@ def run_reference(args, rank, world):
 # ---------------------------------------------------------------------------
 
 PROFILE_CASES = ("gptoss_prefill_full", "gptoss_prefill_band", "lite_prefill_full", "long_decode_full",
-                 "long_decode_fp8", "gptoss_qkv_proj", "gptoss_out_proj")
+                 "long_decode_fp8", "gptoss_qkv_proj", "gptoss_out_proj", "lite_backward_b2")
 
 
 def profile_case(name, dev, steps, warmup):
     import sink_augmented_gqa_b200 as sa
-    if name.endswith("_proj"):
+    if name == "lite_backward_b2":
+        # the Lite training layer with 2 of its 8 sequences (a capture-sized case)
+        cfg = wl.scaled(wl.CONFIGS["lite"], B=2)
+        q, k, v = wl.qkv(cfg, cfg.T, layer=1, device=dev)
+        dout = wl.randn_bf16((cfg.B, cfg.T, cfg.n_q, cfg.d), cfg.seed, 124, dev)
+        sinks = wl.sinks(cfg, 1, device=dev)
+        cache = sa.KVCache(cfg.B, cfg.T, cfg.n_kv, cfg.d, device=dev)
+        out, lse = sa.attn_prefill(cache, q, k, v, sinks, 0, cfg.sm_scale, rope_fused=False, return_lse=True)
+
+        def once():
+            sa.attn_backward(q, k, v, out, dout, lse, sinks, 0, cfg.sm_scale)
+        units = 10 * cfg.d * cfg.B * cfg.n_q * pairs(0, cfg.T, 0)
+    elif name.endswith("_proj"):
         which = "qkv" if "qkv" in name else "out"
         a, w, b, extra = projection_inputs(dev, which)
         N, K = w.shape

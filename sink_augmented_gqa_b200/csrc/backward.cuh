@@ -71,27 +71,52 @@ struct BwdCfg {
   static constexpr int TILE = 64;                 // rows of every tile (4 warps x 16)
   static constexpr int RS = D * 2 + 16;           // padded smem row (bytes): ldmatrix rows hit distinct banks
   static constexpr uint32_t TILE_BYTES = TILE * RS;
-  static constexpr uint32_t OFF_A = 0;            // dK/dV pass: K; dQ pass: Q
-  static constexpr uint32_t OFF_B = TILE_BYTES;   // V | dO
-  static constexpr uint32_t OFF_C = 2 * TILE_BYTES;   // Q | K
-  static constexpr uint32_t OFF_E = 3 * TILE_BYTES;   // dO | V
-  static constexpr uint32_t OFF_L = 4 * TILE_BYTES;   // [64] lse * log2(e)
-  static constexpr uint32_t OFF_DV = OFF_L + 256;     // [64] D
-  static constexpr uint32_t SMEM_BYTES = OFF_DV + 256;
+  static constexpr uint32_t OFF_A = 0;            // resident tiles -- dK/dV pass: K; dQ pass: Q
+  static constexpr uint32_t OFF_B = TILE_BYTES;   //                   V | dO
+  // streamed tiles, two buffers -- dK/dV pass: Q, dO; dQ pass: K, V
+  static constexpr uint32_t OFF_S = 2 * TILE_BYTES;
+  static constexpr uint32_t STREAM_BYTES = 2 * TILE_BYTES;
+  // [64] lse and [64] D of the resident (dQ) or streamed (dK/dV, two buffers) query rows
+  static constexpr uint32_t OFF_L = OFF_S + 2 * STREAM_BYTES;
+  static constexpr uint32_t SMEM_BYTES = OFF_L + 2 * 512;
 };
 
-// rows [row0, row0 + 64) of a strided [B][T][H][D] bf16 tensor (head h, batch b)
-// into a padded smem tile; rows at or past T are zero.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Rows [row0, row0 + 64) of a strided [B][T][H][D] bf16 tensor (head and
+// batch folded into base) into a padded smem tile by cp.async; rows at or
+// past T are zero-filled (no bytes read).
 template <int D>
-__device__ __forceinline__ void bwd_load_tile(uint8_t* dst, const __nv_bfloat16* base, long long s1, int row0, int T) {
+__device__ __forceinline__ void bwd_fetch_tile(uint32_t dst, const __nv_bfloat16* base, long long s1, int row0,
+                                               int T) {
   using C = BwdCfg<D>;
   constexpr int CH = D / 8;   // 16-byte chunks per row
   for (int idx = threadIdx.x; idx < C::TILE * CH; idx += blockDim.x) {
     const int r = idx / CH, c = idx % CH;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (row0 + r < T) val = *reinterpret_cast<const uint4*>(base + (long long)(row0 + r) * s1 + 8 * c);
-    *reinterpret_cast<uint4*>(dst + r * C::RS + 16 * c) = val;
+    const bool in = row0 + r < T;
+    const __nv_bfloat16* src = in ? base + (long long)(row0 + r) * s1 + 8 * c : base;
+    cp_async16(dst + (uint32_t)(r * C::RS + 16 * c), src, in ? 16u : 0u);
   }
+}
+
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+// lse and D of 64 query rows (contiguous in [B][n_q][T], at any 4-byte
+// alignment) into 2 x 64 floats: one element per thread, rows past T zero.
+__device__ __forceinline__ void bwd_fetch_rows(uint32_t dst, const float* lse, const float* dvec, int i0, int T) {
+  const int t = threadIdx.x;   // 128 threads: lse by 0-63, D by 64-127
+  const int r = t & 63;
+  const bool in = i0 + r < T;
+  const float* src = (t < 64 ? lse : dvec) + (in ? i0 + r : 0);
+  cp_async4(dst + (uint32_t)(4 * t), src, in ? 4u : 0u);
 }
 
 __device__ __forceinline__ bool bwd_admitted(int i, int j, int T, int window) {
@@ -154,7 +179,9 @@ __device__ __forceinline__ void bwd_accumulate(float (&acc)[D / 8][4], const uin
   }
 }
 
-// dK, dV of keys [j0, j0 + 64) of KV head g, sequence b.
+// dK, dV of keys [j0, j0 + 64) of KV head g, sequence b. K and V stay in
+// shared memory; the (head, query tile) pairs stream through two buffers,
+// the next pair loading (cp.async) while the current one is computed.
 template <int D>
 __global__ void __launch_bounds__(128) bwd_dkdv_kernel(const BwdParams p) {
   using C = BwdCfg<D>;
@@ -163,64 +190,74 @@ __global__ void __launch_bounds__(128) bwd_dkdv_kernel(const BwdParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int j0 = blockIdx.x * C::TILE, g = blockIdx.y, b = blockIdx.z;
   const float LOG2E = 1.4426950408889634f;
-  float* sL = reinterpret_cast<float*>(smem + C::OFF_L);
-  float* sD = reinterpret_cast<float*>(smem + C::OFF_DV);
-  bwd_load_tile<D>(smem + C::OFF_A, p.k + b * p.ks0 + (long long)g * p.ks2, p.ks1, j0, p.T);
-  bwd_load_tile<D>(smem + C::OFF_B, p.v + b * p.vs0 + (long long)g * p.vs2, p.vs1, j0, p.T);
+  bwd_fetch_tile<D>(sb + C::OFF_A, p.k + b * p.ks0 + (long long)g * p.ks2, p.ks1, j0, p.T);
+  bwd_fetch_tile<D>(sb + C::OFF_B, p.v + b * p.vs0 + (long long)g * p.vs2, p.vs1, j0, p.T);
+  // query tiles that see some key of this tile: i >= j0, and i < j0 + 63 + W on band layers
+  const int qt_lo = j0 / C::TILE;
+  int i_end = p.T;
+  if (p.window > 0 && j0 + C::TILE - 1 + p.window < i_end) i_end = j0 + C::TILE - 1 + p.window;
+  const int nqt = (i_end + C::TILE - 1) / C::TILE - qt_lo;
+  const int total = p.q_mult * nqt;
+  auto fetch = [&](int idx) {
+    const int buf = idx & 1;
+    const int h = g * p.q_mult + idx / nqt;
+    const int i0 = (qt_lo + idx % nqt) * C::TILE;
+    const uint32_t st = sb + C::OFF_S + buf * C::STREAM_BYTES;
+    bwd_fetch_tile<D>(st, p.q + b * p.qs0 + (long long)h * p.qs2, p.qs1, i0, p.T);
+    bwd_fetch_tile<D>(st + C::TILE_BYTES, p.dout + b * p.ds0 + (long long)h * p.ds2, p.ds1, i0, p.T);
+    const long long rb = ((long long)b * p.n_q + h) * p.T;
+    bwd_fetch_rows(sb + C::OFF_L + buf * 512, p.lse + rb, p.dvec + rb, i0, p.T);
+  };
+  fetch(0);
+  cp_async_commit();
   float dk[D / 8][4], dv[D / 8][4];
 #pragma unroll
   for (int n = 0; n < D / 8; ++n)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dk[n][e] = dv[n][e] = 0.f;
-  // query tiles that see some key of this tile: i >= j0, and i < j0 + 63 + W on band layers
-  const int qt_lo = j0 / C::TILE;
-  int i_end = p.T;
-  if (p.window > 0 && j0 + C::TILE - 1 + p.window < i_end) i_end = j0 + C::TILE - 1 + p.window;
-  const int qt_hi = (i_end + C::TILE - 1) / C::TILE;
   const int g8 = lane >> 2, t4 = lane & 3;
-  for (int m = 0; m < p.q_mult; ++m) {
-    const int h = g * p.q_mult + m;
-    for (int qt = qt_lo; qt < qt_hi; ++qt) {
-      const int i0 = qt * C::TILE;
-      __syncthreads();   // the previous query tile is no longer read
-      bwd_load_tile<D>(smem + C::OFF_C, p.q + b * p.qs0 + (long long)h * p.qs2, p.qs1, i0, p.T);
-      bwd_load_tile<D>(smem + C::OFF_E, p.dout + b * p.ds0 + (long long)h * p.ds2, p.ds1, i0, p.T);
-      if (threadIdx.x < C::TILE) {
-        const int i = i0 + threadIdx.x;
-        const long long li = ((long long)b * p.n_q + h) * p.T + i;
-        sL[threadIdx.x] = i < p.T ? p.lse[li] * LOG2E : INFINITY;
-        sD[threadIdx.x] = i < p.T ? p.dvec[li] : 0.f;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        // S^T (keys x queries) = K Q^T and dP^T = V dO^T for this warp's 16 keys
-        float s[4][4], dp[4][4];
-        bwd_two_products<D>(sb + C::OFF_A, sb + C::OFF_C, sb + C::OFF_B, sb + C::OFF_E, 16 * warp, 32 * half,
-                            s, dp, lane);
-        uint32_t pp[4][2], dsp[4][2];
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-          float pv[4], dsv[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int kr = 16 * warp + g8 + 8 * (e >> 1);
-            const int qc = 32 * half + 8 * nt + 2 * t4 + (e & 1);
-            const bool ok = bwd_admitted(i0 + qc, j0 + kr, p.T, p.window);
-            const float pr = ok ? ex2(s[nt][e] * p.scale_log2 - sL[qc]) : 0.f;
-            pv[e] = pr;
-            dsv[e] = pr * (dp[nt][e] - sD[qc]);
-          }
-          pp[nt][0] = pack_bf16(pv[0], pv[1]);
-          pp[nt][1] = pack_bf16(pv[2], pv[3]);
-          dsp[nt][0] = pack_bf16(dsv[0], dsv[1]);
-          dsp[nt][1] = pack_bf16(dsv[2], dsv[3]);
-        }
-        // dV += P^T dO, dK += dS^T Q over these 32 queries
-        bwd_accumulate<D>(dv, pp, sb + C::OFF_E, 32 * half, lane);
-        bwd_accumulate<D>(dk, dsp, sb + C::OFF_C, 32 * half, lane);
-      }
+  for (int idx = 0; idx < total; ++idx) {
+    if (idx + 1 < total) {
+      fetch(idx + 1);   // into the buffer the previous iteration finished with
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
+    __syncthreads();   // this iteration's tiles (and K, V) are in shared memory
+    const int buf = idx & 1;
+    const int i0 = (qt_lo + idx % nqt) * C::TILE;
+    const uint32_t sq = sb + C::OFF_S + buf * C::STREAM_BYTES, sdo = sq + C::TILE_BYTES;
+    const float* sL = reinterpret_cast<const float*>(smem + C::OFF_L + buf * 512);
+    const float* sD = sL + 64;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      // S^T (keys x queries) = K Q^T and dP^T = V dO^T for this warp's 16 keys
+      float s[4][4], dp[4][4];
+      bwd_two_products<D>(sb + C::OFF_A, sq, sb + C::OFF_B, sdo, 16 * warp, 32 * half, s, dp, lane);
+      uint32_t pp[4][2], dsp[4][2];
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        float pv[4], dsv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int kr = 16 * warp + g8 + 8 * (e >> 1);
+          const int qc = 32 * half + 8 * nt + 2 * t4 + (e & 1);
+          const bool ok = bwd_admitted(i0 + qc, j0 + kr, p.T, p.window);
+          const float pr = ok ? ex2(s[nt][e] * p.scale_log2 - sL[qc] * LOG2E) : 0.f;
+          pv[e] = pr;
+          dsv[e] = pr * (dp[nt][e] - sD[qc]);
+        }
+        pp[nt][0] = pack_bf16(pv[0], pv[1]);
+        pp[nt][1] = pack_bf16(pv[2], pv[3]);
+        dsp[nt][0] = pack_bf16(dsv[0], dsv[1]);
+        dsp[nt][1] = pack_bf16(dsv[2], dsv[3]);
+      }
+      // dV += P^T dO, dK += dS^T Q over these 32 queries
+      bwd_accumulate<D>(dv, pp, sdo, 32 * half, lane);
+      bwd_accumulate<D>(dk, dsp, sq, 32 * half, lane);
+    }
+    __syncthreads();   // every warp is done with this buffer before it is refilled
   }
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) {
@@ -235,7 +272,8 @@ __global__ void __launch_bounds__(128) bwd_dkdv_kernel(const BwdParams p) {
   }
 }
 
-// dQ of queries [i0, i0 + 64) of query head h, sequence b.
+// dQ of queries [i0, i0 + 64) of query head h, sequence b. Q and dO stay in
+// shared memory; the admitted K/V tiles stream through two buffers.
 template <int D>
 __global__ void __launch_bounds__(128) bwd_dq_kernel(const BwdParams p) {
   using C = BwdCfg<D>;
@@ -245,39 +283,47 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(const BwdParams p) {
   const int i0 = blockIdx.x * C::TILE, h = blockIdx.y, b = blockIdx.z;
   const int g = h / p.q_mult;
   const float LOG2E = 1.4426950408889634f;
-  float* sL = reinterpret_cast<float*>(smem + C::OFF_L);
-  float* sD = reinterpret_cast<float*>(smem + C::OFF_DV);
-  bwd_load_tile<D>(smem + C::OFF_A, p.q + b * p.qs0 + (long long)h * p.qs2, p.qs1, i0, p.T);
-  bwd_load_tile<D>(smem + C::OFF_B, p.dout + b * p.ds0 + (long long)h * p.ds2, p.ds1, i0, p.T);
-  if (threadIdx.x < C::TILE) {
-    const int i = i0 + threadIdx.x;
-    const long long li = ((long long)b * p.n_q + h) * p.T + i;
-    sL[threadIdx.x] = i < p.T ? p.lse[li] * LOG2E : INFINITY;
-    sD[threadIdx.x] = i < p.T ? p.dvec[li] : 0.f;
-  }
+  bwd_fetch_tile<D>(sb + C::OFF_A, p.q + b * p.qs0 + (long long)h * p.qs2, p.qs1, i0, p.T);
+  bwd_fetch_tile<D>(sb + C::OFF_B, p.dout + b * p.ds0 + (long long)h * p.ds2, p.ds1, i0, p.T);
+  const long long rb = ((long long)b * p.n_q + h) * p.T;
+  bwd_fetch_rows(sb + C::OFF_L, p.lse + rb, p.dvec + rb, i0, p.T);
+  // key tiles these queries see: j <= i, and j > i - W on band layers
+  int j_lo = 0;
+  if (p.window > 0 && i0 - p.window + 1 > 0) j_lo = i0 - p.window + 1;
+  const int kt_lo = j_lo / C::TILE;
+  const int total = (min(p.T, i0 + C::TILE) + C::TILE - 1) / C::TILE - kt_lo;
+  auto fetch = [&](int idx) {
+    const uint32_t st = sb + C::OFF_S + (idx & 1) * C::STREAM_BYTES;
+    const int j0 = (kt_lo + idx) * C::TILE;
+    bwd_fetch_tile<D>(st, p.k + b * p.ks0 + (long long)g * p.ks2, p.ks1, j0, p.T);
+    bwd_fetch_tile<D>(st + C::TILE_BYTES, p.v + b * p.vs0 + (long long)g * p.vs2, p.vs1, j0, p.T);
+  };
+  fetch(0);
+  cp_async_commit();
   float dq[D / 8][4];
 #pragma unroll
   for (int n = 0; n < D / 8; ++n)
 #pragma unroll
     for (int e = 0; e < 4; ++e) dq[n][e] = 0.f;
-  // key tiles these queries see: j <= i, and j > i - W on band layers
-  int j_lo = 0;
-  if (p.window > 0 && i0 - p.window + 1 > 0) j_lo = i0 - p.window + 1;
-  const int kt_lo = j_lo / C::TILE;
-  const int kt_hi = (min(p.T, i0 + C::TILE) + C::TILE - 1) / C::TILE;
+  const float* sL = reinterpret_cast<const float*>(smem + C::OFF_L);
+  const float* sD = sL + 64;
   const int g8 = lane >> 2, t4 = lane & 3;
-  for (int kt = kt_lo; kt < kt_hi; ++kt) {
-    const int j0 = kt * C::TILE;
+  for (int idx = 0; idx < total; ++idx) {
+    if (idx + 1 < total) {
+      fetch(idx + 1);
+      cp_async_commit();
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
     __syncthreads();
-    bwd_load_tile<D>(smem + C::OFF_C, p.k + b * p.ks0 + (long long)g * p.ks2, p.ks1, j0, p.T);
-    bwd_load_tile<D>(smem + C::OFF_E, p.v + b * p.vs0 + (long long)g * p.vs2, p.vs1, j0, p.T);
-    __syncthreads();
+    const int j0 = (kt_lo + idx) * C::TILE;
+    const uint32_t sk = sb + C::OFF_S + (idx & 1) * C::STREAM_BYTES, sv = sk + C::TILE_BYTES;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       // S = Q K^T and dP = dO V^T for this warp's 16 queries and 32 keys
       float s[4][4], dp[4][4];
-      bwd_two_products<D>(sb + C::OFF_A, sb + C::OFF_C, sb + C::OFF_B, sb + C::OFF_E, 16 * warp, 32 * half, s,
-                          dp, lane);
+      bwd_two_products<D>(sb + C::OFF_A, sk, sb + C::OFF_B, sv, 16 * warp, 32 * half, s, dp, lane);
       uint32_t dsp[4][2];
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) {
@@ -287,15 +333,16 @@ __global__ void __launch_bounds__(128) bwd_dq_kernel(const BwdParams p) {
           const int qr = 16 * warp + g8 + 8 * (e >> 1);
           const int kc = 32 * half + 8 * nt + 2 * t4 + (e & 1);
           const bool ok = bwd_admitted(i0 + qr, j0 + kc, p.T, p.window);
-          const float pr = ok ? ex2(s[nt][e] * p.scale_log2 - sL[qr]) : 0.f;
+          const float pr = ok ? ex2(s[nt][e] * p.scale_log2 - sL[qr] * LOG2E) : 0.f;
           dsv[e] = pr * (dp[nt][e] - sD[qr]);
         }
         dsp[nt][0] = pack_bf16(dsv[0], dsv[1]);
         dsp[nt][1] = pack_bf16(dsv[2], dsv[3]);
       }
       // dQ += dS K over these 32 keys
-      bwd_accumulate<D>(dq, dsp, sb + C::OFF_C, 32 * half, lane);
+      bwd_accumulate<D>(dq, dsp, sk, 32 * half, lane);
     }
+    __syncthreads();
   }
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) {
