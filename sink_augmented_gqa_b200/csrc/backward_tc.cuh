@@ -1,0 +1,459 @@
+// Backward pass on tcgen05 tensor cores: the same gradients as backward.cuh,
+// from two kernels shaped like the forward prefill kernel:
+//
+//   MODE 0 (dQ)   rows = 128 queries of one head; streams the admitted key
+//                 tiles: S = Q K^T, dP = dO V^T (smem x smem into TMEM),
+//                 dS = P (dP - D) as bf16 into TMEM, dQ += dS K (TMEM x smem).
+//   MODE 1 (dKdV) rows = 128 keys of one KV head; streams the query tiles
+//                 of every head of the group that see them: S^T = K Q^T,
+//                 dP^T = V dO^T, P^T and dS^T as bf16 into TMEM, then
+//                 dV += P^T dO and dK += dS^T Q.
+//
+// One CTA per 128-row tile (heaviest tiles first), 192 threads:
+//   warp 0      TMA loads: the two resident 128-row tiles once, then per
+//               streamed tile its two BN-row tiles into an NS-deep ring (MODE 1
+//               also stages the tile's lse and D values there).
+//   warp 1      one thread issues the MMAs and owns the TMEM allocation. S and
+//               dP are double-buffered in TMEM, so the tensor core computes the
+//               next tile's S, dP while the current tile's dS is formed.
+//   warps 2-9   P, dS from S, dP: two warps per TMEM lane quarter (warp % 4),
+//               each taking half of a tile's columns, one row per thread; tiles
+//               wholly inside the admitted region skip the mask; then the fp32
+//               output rows (the two warps of a quarter split the columns).
+// P_ij = exp2(s_ij scale_log2 - lse_i log2 e) uses the forward's lse (sink
+// included), so no running max is needed.
+#pragma once
+
+#include "backward.cuh"
+#include "ptx.cuh"
+
+namespace sa {
+
+__host__ __device__ constexpr int btc_align32(int x) { return (x + 31) / 32 * 32; }
+
+template <int D, int MODE>
+struct BtcCfg {
+  static constexpr int BM = 128;                                     // resident rows
+  static constexpr int BN = (MODE == 1 && D == 128) ? 32 : 64;       // streamed rows per tile
+  static constexpr int CB = (D % 64 == 0) ? 64 : 32;                 // column block (elements)
+  static constexpr int SWZ = CB * 2;                                 // bytes per block row
+  static constexpr int NCB = D / CB;
+  static constexpr uint32_t LAYOUT = (SWZ == 128) ? 2u : 4u;
+  static constexpr uint32_t SBO = 8u * SWZ;
+  static constexpr uint32_t MBLOCK = (uint32_t)BM * SWZ;
+  static constexpr uint32_t M_BYTES = (uint32_t)BM * D * 2;
+  static constexpr uint32_t NBLOCK = (uint32_t)BN * SWZ;
+  static constexpr uint32_t N_BYTES = (uint32_t)BN * D * 2;
+  static constexpr int NS = (D == 128) ? 3 : 4;
+  static constexpr uint32_t STAGE_BYTES = 2 * N_BYTES;
+  static constexpr uint32_t OFF_R0 = 0;                              // Q (MODE 0) | K (MODE 1)
+  static constexpr uint32_t OFF_R1 = M_BYTES;                        // dO | V
+  static constexpr uint32_t OFF_ST = 2 * M_BYTES;                    // ring: [K | Q], [V | dO]
+  static constexpr uint32_t OFF_ROWV = OFF_ST + NS * STAGE_BYTES;    // MODE 1: [NS][2][BN] fp32
+  static constexpr uint32_t OFF_BAR = OFF_ROWV + NS * 2 * BN * 4;
+  // at least 120 KB: one CTA per SM, since each allocates all 512 TMEM columns
+  static constexpr uint32_t SMEM_BYTES = (OFF_BAR + 256 + 1024) > 120u * 1024 ? (OFF_BAR + 256 + 1024) : 120u * 1024;
+  // TMEM columns
+  static constexpr int S_COL = 0;                  // S[buf] at S_COL + buf * BN
+  static constexpr int DP_COL = 2 * BN;            // dP[buf]
+  static constexpr int P_COL = 4 * BN;             // MODE 1: P (bf16 pairs, BN / 2 columns)
+  static constexpr int DS_COL = 4 * BN + (MODE == 1 ? BN / 2 : 0);   // dS (bf16 pairs)
+  static constexpr int ACC0 = btc_align32(DS_COL + BN / 2);              // dQ | dV
+  static constexpr int ACC1 = ACC0 + D;                              // MODE 1: dK
+  static constexpr int TMEM_COLS = 512;
+  static_assert((MODE == 0 ? ACC0 + D : ACC1 + D) <= TMEM_COLS, "TMEM plan exceeds 512 columns");
+  static_assert(MBLOCK % 1024 == 0 && NBLOCK % 1024 == 0 && M_BYTES % 1024 == 0, "1 KB aligned tiles");
+  static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
+  static constexpr uint32_t IDESC_O = idesc_bf16(128, D, 0, 1);
+  static constexpr int NSW = 8;                                      // P / dS warps (2..9)
+  static constexpr int HC = BN / 2;                                  // columns per P / dS warp
+  static constexpr int NUM_THREADS = 32 * (2 + NSW);
+};
+
+enum : int {
+  BB_RFULL = 0,      // resident tiles landed
+  BB_FULL = 1,       // [4] ring stage landed
+  BB_EMPTY = 5,      // [4] ring stage free (MMA commit)
+  BB_SFULL = 9,      // [2] S, dP of a buffer computed
+  BB_SFREE = 11,     // [2] count 8 warps: S, dP of a buffer read
+  BB_PFULL = 13,     // count 8 warps: P / dS stored in TMEM
+  BB_PDONE = 14,     // the products reading P / dS completed
+  BB_ACCFULL = 15,   // accumulators final
+  BB_DRAIN = 16,
+  BB_TMEM_SLOT = 17,
+  BB_ABORT_SLOT = 18,
+};
+
+// D = sum over K-steps of A (smem, K-major, 128 rows) B (smem, K-major, BN rows)^T
+template <int D, int MODE>
+__device__ __forceinline__ void btc_issue_s(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc) {
+  using C = BtcCfg<D, MODE>;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t cb = kk * 16 / C::CB, cin = (kk * 16 % C::CB) * 2;
+    mma_ss(d_tmem, adesc + ((cb * C::MBLOCK + cin) >> 4), bdesc + ((cb * C::NBLOCK + cin) >> 4), C::IDESC_S,
+           kk > 0 ? 1u : 0u);
+  }
+}
+// acc (+)= A (TMEM bf16, 128 x BN) B (smem [BN][D], MN-major)
+template <int D, int MODE>
+__device__ __forceinline__ void btc_issue_o(uint32_t acc_tmem, uint32_t a_tmem, uint64_t bdesc, bool accumulate) {
+  using C = BtcCfg<D, MODE>;
+#pragma unroll
+  for (int kk = 0; kk < C::BN / 16; ++kk)
+    mma_ts(acc_tmem, a_tmem + kk * 8, bdesc + ((kk * 16 * C::SWZ) >> 4), C::IDESC_O,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(320, 1)
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tmR0, const __grid_constant__ CUtensorMap tmR1,
+                  const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1,
+                  const BwdParams p) {
+  using C = BtcCfg<D, MODE>;
+  constexpr int BN = C::BN;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * BB_TMEM_SLOT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * BB_ABORT_SLOT);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // heaviest row tiles (last queries / first keys of a causal layer) first
+  const int tile = (MODE == 0) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  const int r0 = tile * C::BM;          // first resident row
+  const int head = blockIdx.y;          // query head (MODE 0) or KV head (MODE 1)
+  const int b = blockIdx.z;
+  // Streamed tiles. MODE 0: key tiles [t_lo, t_hi) of BN keys seen by
+  // queries r0..r0+127. MODE 1: for each head of the group, query tiles
+  // [t_lo, t_hi) of BN queries that see keys r0..r0+127.
+  int t_lo, t_hi;
+  if constexpr (MODE == 0) {
+    const int j_lo = p.window > 0 ? max(r0 - p.window + 1, 0) : 0;
+    t_lo = j_lo / BN;
+    t_hi = (min(p.T, r0 + C::BM) + BN - 1) / BN;
+  } else {
+    t_lo = r0 / BN;
+    int i_end = p.T;
+    if (p.window > 0 && r0 + C::BM - 1 + p.window < i_end) i_end = r0 + C::BM - 1 + p.window;
+    t_hi = (i_end + BN - 1) / BN;
+  }
+  const int per = t_hi > t_lo ? t_hi - t_lo : 0;
+  const int n_tiles = (MODE == 0) ? per : per * p.q_mult;
+  const int g = (MODE == 0) ? head / p.q_mult : head;
+  // streamed tile u -> (head of its Q/dO or lse/D rows, first streamed row)
+  auto stream_of = [&](int u, int& hh, int& s0) {
+    if constexpr (MODE == 0) {
+      hh = head;
+      s0 = (t_lo + u) * BN;
+    } else {
+      hh = g * p.q_mult + u / per;
+      s0 = (t_lo + u % per) * BN;
+    }
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(BB_RFULL), 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(bar(BB_FULL + s), 1);
+      mbar_init(bar(BB_EMPTY + s), 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bar(BB_SFULL + x), 1);
+      mbar_init(bar(BB_SFREE + x), C::NSW);
+    }
+    mbar_init(bar(BB_PFULL), C::NSW);
+    mbar_init(bar(BB_PDONE), 1);
+    mbar_init(bar(BB_ACCFULL), 1);
+    mbar_init(bar(BB_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmR0);
+      tma_prefetch_desc(&tmR1);
+      tma_prefetch_desc(&tmS0);
+      tma_prefetch_desc(&tmS1);
+      mbar_arrive_expect_tx(bar(BB_RFULL), 2 * C::M_BYTES);
+      const int rh = (MODE == 0) ? head : g;   // head of the resident tiles
+#pragma unroll
+      for (int cb = 0; cb < C::NCB; ++cb) {
+        tma_load_4d(sbase + C::OFF_R0 + cb * C::MBLOCK, &tmR0, bar(BB_RFULL), cb * C::CB, r0, rh, b);
+        tma_load_4d(sbase + C::OFF_R1 + cb * C::MBLOCK, &tmR1, bar(BB_RFULL), cb * C::CB, r0, rh, b);
+      }
+    }
+    int issued = 0;
+    bool ok = true;
+    for (int u = 0; u < n_tiles; ++u) {
+      const int s = u % C::NS;
+      if (u >= C::NS) {
+        bool w = true;
+        if (lane == 0) w = mbar_wait(bar(BB_EMPTY + s), (uint32_t)(((u / C::NS) - 1) & 1));
+        w = __shfl_sync(0xffffffffu, w, 0);
+        if (!w) { ok = false; break; }
+      }
+      if (*abort_flag) { ok = false; break; }
+      int hh, s0;
+      stream_of(u, hh, s0);
+      if constexpr (MODE == 1) {
+        // lse (times log2 e) and D of the tile's BN query rows, beside its tiles
+        float* rv = reinterpret_cast<float*>(smem + C::OFF_ROWV) + s * 2 * BN;
+        const long long rb = ((long long)b * p.n_q + hh) * p.T;
+        for (int c = lane; c < BN; c += 32) {
+          const int i = s0 + c;
+          rv[c] = i < p.T ? p.lse[rb + i] * 1.4426950408889634f : INFINITY;
+          rv[BN + c] = i < p.T ? p.dvec[rb + i] : 0.f;
+        }
+        __syncwarp();
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(BB_FULL + s), C::STAGE_BYTES);
+        const int sh = (MODE == 0) ? g : hh;   // head of the streamed tiles
+        const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_BYTES;
+#pragma unroll
+        for (int cb = 0; cb < C::NCB; ++cb) {
+          tma_load_4d(st + cb * C::NBLOCK, &tmS0, bar(BB_FULL + s), cb * C::CB, s0, sh, b);
+          tma_load_4d(st + C::N_BYTES + cb * C::NBLOCK, &tmS1, bar(BB_FULL + s), cb * C::CB, s0, sh, b);
+        }
+      }
+      issued = u + 1;
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      for (int u = (issued > C::NS ? issued - C::NS : 0); u < issued; ++u)
+        mbar_wait_drain(bar(BB_FULL + u % C::NS), (uint32_t)((u / C::NS) & 1));
+    }
+    if (lane == 0) mbar_wait_drain(bar(BB_RFULL), 0);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(bar(BB_RFULL), 0);
+      tc_fence_after();
+      const uint64_t a0 = smem_desc(sbase + C::OFF_R0, 16, C::SBO, C::LAYOUT);   // Q | K, K-major
+      const uint64_t a1 = smem_desc(sbase + C::OFF_R1, 16, C::SBO, C::LAYOUT);   // dO | V
+      auto o_products = [&](int v) {   // the products of tile v that read P / dS
+        const int sv = v % C::NS;
+        const uint32_t st = sbase + C::OFF_ST + sv * C::STAGE_BYTES;
+        if constexpr (MODE == 0) {
+          // dQ += dS K (K of the stage, MN-major)
+          btc_issue_o<D, MODE>(tmem + C::ACC0, tmem + C::DS_COL,
+                               smem_desc(st, C::NBLOCK, C::SBO, C::LAYOUT), v > 0);
+        } else {
+          // dV += P^T dO, dK += dS^T Q
+          btc_issue_o<D, MODE>(tmem + C::ACC0, tmem + C::P_COL,
+                               smem_desc(st + C::N_BYTES, C::NBLOCK, C::SBO, C::LAYOUT), v > 0);
+          btc_issue_o<D, MODE>(tmem + C::ACC1, tmem + C::DS_COL, smem_desc(st, C::NBLOCK, C::SBO, C::LAYOUT),
+                               v > 0);
+        }
+        mma_commit(bar(BB_PDONE));
+        mma_commit(bar(BB_EMPTY + sv));
+      };
+      for (int u = 0; u < n_tiles && ok; ++u) {
+        const int s = u % C::NS, x = u & 1;
+        if (!mbar_wait(bar(BB_FULL + s), (uint32_t)((u / C::NS) & 1))) { ok = false; break; }
+        if (u >= 2 && !mbar_wait(bar(BB_SFREE + x), (uint32_t)(((u >> 1) - 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_BYTES;
+        // S = R0 S0^T, dP = R1 S1^T (both K-major)
+        btc_issue_s<D, MODE>(tmem + C::S_COL + x * BN, a0, smem_desc(st, 16, C::SBO, C::LAYOUT));
+        btc_issue_s<D, MODE>(tmem + C::DP_COL + x * BN, a1, smem_desc(st + C::N_BYTES, 16, C::SBO, C::LAYOUT));
+        mma_commit(bar(BB_SFULL + x));
+        if (u > 0) {
+          if (!mbar_wait(bar(BB_PFULL), (uint32_t)((u - 1) & 1))) { ok = false; break; }
+          tc_fence_after();
+          o_products(u - 1);
+        }
+        if (*abort_flag) { ok = false; break; }
+      }
+      if (ok && n_tiles > 0) {
+        if (mbar_wait(bar(BB_PFULL), (uint32_t)((n_tiles - 1) & 1))) {
+          tc_fence_after();
+          o_products(n_tiles - 1);
+          mma_commit(bar(BB_ACCFULL));
+        } else {
+          ok = false;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        mma_commit(bar(BB_DRAIN));
+        mbar_wait_drain(bar(BB_DRAIN), 0);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dS and the epilogue
+    constexpr int HC = C::HC;
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;                    // which half of the columns
+    const int rr = quarter * 32 + lane;                  // resident row of this thread
+    const int row = r0 + rr;                              // query (MODE 0) or key (MODE 1)
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const float LOG2E = 1.4426950408889634f;
+    const float sl2 = p.scale_log2;
+    float lse2 = 0.f, dval = 0.f;
+    if constexpr (MODE == 0) {
+      if (row < p.T) {
+        const long long li = ((long long)b * p.n_q + head) * p.T + row;
+        lse2 = p.lse[li] * LOG2E;
+        dval = p.dvec[li];
+      }
+    }
+    // every wait below is taken warp-uniformly: the TMEM loads and stores
+    // that follow are warp-collective
+    auto wait_all = [&](uint32_t bb, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bb, parity) ? 1 : 0) != 0;
+    };
+    bool ok = true;
+    for (int u = 0; u < n_tiles && ok; ++u) {
+      const int x = u & 1;
+      if (!wait_all(bar(BB_SFULL + x), (uint32_t)((u >> 1) & 1))) { ok = false; break; }
+      tc_fence_after();
+      int hh, s0;
+      stream_of(u, hh, s0);
+      const int c_base = half * HC;                       // this warp's first column of the tile
+      const float* rv = reinterpret_cast<const float*>(smem + C::OFF_ROWV) + (u % C::NS) * 2 * BN;
+      if constexpr (MODE == 1) {
+        // the producer's lse / D values of this stage: acquire them on the
+        // stage's own barrier (its phase cannot move on before this tile's
+        // products have run, which wait for these warps)
+        if (!wait_all(bar(BB_FULL + u % C::NS), (uint32_t)((u / C::NS) & 1))) { ok = false; break; }
+      }
+      // every (row, column) pair of the tile admitted? (pairs past T are
+      // harmless either way: their operand rows are zero or their output
+      // rows are not stored)
+      bool all_in;
+      if constexpr (MODE == 0) {   // rows = queries r0.., columns = keys s0..
+        all_in = s0 + BN - 1 <= r0 && (p.window <= 0 || s0 > r0 + C::BM - 1 - p.window);
+      } else {                     // rows = keys r0.., columns = queries s0..
+        all_in = r0 + C::BM - 1 <= s0 && (p.window <= 0 || r0 > s0 + BN - 1 - p.window);
+      }
+      uint32_t sv[HC], dv[HC];
+      if constexpr (HC == 32) {
+        tmem_ld32(tmem + lane_base + C::S_COL + x * BN + c_base, *reinterpret_cast<uint32_t(*)[32]>(sv));
+        tmem_ld32(tmem + lane_base + C::DP_COL + x * BN + c_base, *reinterpret_cast<uint32_t(*)[32]>(dv));
+      } else {
+        tmem_ld16(tmem + lane_base + C::S_COL + x * BN + c_base, sv);
+        tmem_ld16(tmem + lane_base + C::DP_COL + x * BN + c_base, dv);
+      }
+      tmem_wait_ld();
+      uint32_t pk[HC / 2], dk[HC / 2];
+#pragma unroll
+      for (int c = 0; c < HC; c += 2) {
+        float l0, l1, d0, d1;
+        if constexpr (MODE == 0) {
+          l0 = l1 = lse2;
+          d0 = d1 = dval;
+        } else {
+          const float2 lv = *reinterpret_cast<const float2*>(rv + c_base + c);
+          const float2 dd = *reinterpret_cast<const float2*>(rv + BN + c_base + c);
+          l0 = lv.x; l1 = lv.y; d0 = dd.x; d1 = dd.y;
+        }
+        float x0, x1;
+        fma2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl2, sl2, -l0, -l1);
+        float p0 = ex2(x0), p1 = ex2(x1);
+        if (!all_in) {
+          const int col = s0 + c_base + c;
+          if (MODE == 0) {
+            if (!bwd_admitted(row, col, p.T, p.window)) p0 = 0.f;
+            if (!bwd_admitted(row, col + 1, p.T, p.window)) p1 = 0.f;
+          } else {
+            if (!bwd_admitted(col, row, p.T, p.window)) p0 = 0.f;
+            if (!bwd_admitted(col + 1, row, p.T, p.window)) p1 = 0.f;
+          }
+        }
+        float t0 = __uint_as_float(dv[c]), t1 = __uint_as_float(dv[c + 1]);
+        add2(t0, t1, -d0, -d1);
+        mul2(t0, t1, p0, p1);
+        pk[c / 2] = pack_bf16(p0, p1);
+        dk[c / 2] = pack_bf16(t0, t1);
+      }
+      // P / dS of the previous tile are read by its products until they complete
+      if (u > 0) {
+        if (!wait_all(bar(BB_PDONE), (uint32_t)((u - 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+      }
+      if constexpr (HC == 32) {
+        tmem_st16(tmem + lane_base + C::DS_COL + c_base / 2, dk);
+        if constexpr (MODE == 1) tmem_st16(tmem + lane_base + C::P_COL + c_base / 2, pk);
+      } else {
+        tmem_st8(tmem + lane_base + C::DS_COL + c_base / 2, dk);
+        if constexpr (MODE == 1) tmem_st8(tmem + lane_base + C::P_COL + c_base / 2, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(BB_SFREE + x));
+        mbar_arrive(bar(BB_PFULL));
+      }
+      if (*abort_flag) { ok = false; break; }
+    }
+    // epilogue: the accumulators (zero when no tile was admitted) -> fp32
+    // rows. MODE 0: the two warps of a quarter take alternate 32-column
+    // chunks of dQ; MODE 1: one takes dV, the other dK. Every lane takes
+    // part in the TMEM loads; rows past T store nothing.
+    const bool have = n_tiles > 0;
+    if (ok && have) {
+      if (!wait_all(bar(BB_ACCFULL), 0)) ok = false;
+      tc_fence_after();
+    }
+    if (ok) {
+      float* dst;
+      float mul;
+      int acc;
+      if constexpr (MODE == 0) {
+        dst = p.dq + (((long long)b * p.T + row) * p.n_q + head) * D;
+        mul = p.scale;
+        acc = C::ACC0;
+      } else {
+        dst = (half == 0 ? p.dv : p.dk) + (((long long)b * p.T + row) * p.n_kv + head) * D;
+        mul = half == 0 ? 1.0f : p.scale;
+        acc = half == 0 ? C::ACC0 : C::ACC1;
+      }
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        if (MODE == 0 && ((c0 / 32) & 1) != half) continue;
+        uint32_t a32[32];
+        if (have) {
+          tmem_ld32(tmem + lane_base + acc + c0, a32);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) a32[c] = 0u;
+        }
+        if (row < p.T) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *reinterpret_cast<float4*>(dst + c0 + c) =
+                make_float4(__uint_as_float(a32[c]) * mul, __uint_as_float(a32[c + 1]) * mul,
+                            __uint_as_float(a32[c + 2]) * mul, __uint_as_float(a32[c + 3]) * mul);
+        }
+      }
+    }
+    if (!ok) *abort_flag = 1;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace sa

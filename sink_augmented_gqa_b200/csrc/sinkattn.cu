@@ -12,6 +12,7 @@
 
 #include "../../include/sinkattn.h"
 #include "backward.cuh"
+#include "backward_tc.cuh"
 #include "decode.cuh"
 #include "fp8.cuh"
 #include "gemm.cuh"
@@ -148,12 +149,12 @@ bool make_matrix_map(CUtensorMap* map, const void* base, long long cols, long lo
 // box {CB, 128, 1, 1} -- one 128-row query tile of one head per CB-wide
 // column block; rows past T read as zeros.
 bool make_rows_map(CUtensorMap* map, const void* base, int d, int T, int H, int B,
-                   const int64_t st[3], int cb) {
+                   const int64_t st[3], int cb, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr || T < 1) return false;
   const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)T, (cuuint64_t)H, (cuuint64_t)B};
   const cuuint64_t strides[3] = {(cuuint64_t)st[1] * 2, (cuuint64_t)st[2] * 2, (cuuint64_t)st[0] * 2};
-  const cuuint32_t box[4] = {(cuuint32_t)cb, 128, 1, 1};
+  const cuuint32_t box[4] = {(cuuint32_t)cb, (cuuint32_t)box_rows, 1, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -526,7 +527,6 @@ sa_status launch_gemm(const void* a, int64_t lda, const void* w, int64_t ldw, co
 // Backward pass (csrc/backward.cuh): row pass, key-tile pass, query-tile pass.
 template <int D>
 sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t stream) {
-  using Cfg = sa::BwdCfg<D>;
   sa::BwdParams p;
   p.q = static_cast<const __nv_bfloat16*>(a->q);
   p.k = static_cast<const __nv_bfloat16*>(a->k);
@@ -556,15 +556,29 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
   if (p.dsinks && cudaMemsetAsync(p.dsinks, 0, sizeof(float) * a->n_q, stream) != cudaSuccess) return SA_ERR_CUDA;
   const long long rows = (long long)a->B * a->T * a->n_q;
   sa::bwd_rows_kernel<D><<<grid_for(rows * 32), 256, 0, stream>>>(p);
+  using C0 = sa::BtcCfg<D, 0>;
+  using C1 = sa::BtcCfg<D, 1>;
+  // dQ pass: resident Q, dO (128 rows); streamed K, V (BN rows).
+  // dK/dV pass: resident K, V; streamed Q, dO.
+  CUtensorMap q0, o0, k0, v0, k1, v1, q1, o1;
+  if (!make_rows_map(&q0, a->q, D, a->T, a->n_q, a->B, a->q_strides, C0::CB, 128) ||
+      !make_rows_map(&o0, a->d_out, D, a->T, a->n_q, a->B, a->d_out_strides, C0::CB, 128) ||
+      !make_rows_map(&k0, a->k, D, a->T, a->n_kv, a->B, a->k_strides, C0::CB, C0::BN) ||
+      !make_rows_map(&v0, a->v, D, a->T, a->n_kv, a->B, a->v_strides, C0::CB, C0::BN) ||
+      !make_rows_map(&k1, a->k, D, a->T, a->n_kv, a->B, a->k_strides, C1::CB, 128) ||
+      !make_rows_map(&v1, a->v, D, a->T, a->n_kv, a->B, a->v_strides, C1::CB, 128) ||
+      !make_rows_map(&q1, a->q, D, a->T, a->n_q, a->B, a->q_strides, C1::CB, C1::BN) ||
+      !make_rows_map(&o1, a->d_out, D, a->T, a->n_q, a->B, a->d_out_strides, C1::CB, C1::BN))
+    return SA_ERR_CUDA;
   static bool configured = false;
   if (!configured) {
-    set_smem(sa::bwd_dkdv_kernel<D>, Cfg::SMEM_BYTES);
-    set_smem(sa::bwd_dq_kernel<D>, Cfg::SMEM_BYTES);
+    set_smem(sa::bwd_tc_kernel<D, 0>, C0::SMEM_BYTES);
+    set_smem(sa::bwd_tc_kernel<D, 1>, C1::SMEM_BYTES);
     configured = true;
   }
-  const int tiles = (a->T + Cfg::TILE - 1) / Cfg::TILE;
-  sa::bwd_dkdv_kernel<D><<<dim3(tiles, a->n_kv, a->B), 128, Cfg::SMEM_BYTES, stream>>>(p);
-  sa::bwd_dq_kernel<D><<<dim3(tiles, a->n_q, a->B), 128, Cfg::SMEM_BYTES, stream>>>(p);
+  const int tiles = (a->T + 127) / 128;
+  sa::bwd_tc_kernel<D, 1><<<dim3(tiles, a->n_kv, a->B), C1::NUM_THREADS, C1::SMEM_BYTES, stream>>>(k1, v1, q1, o1, p);
+  sa::bwd_tc_kernel<D, 0><<<dim3(tiles, a->n_q, a->B), C0::NUM_THREADS, C0::SMEM_BYTES, stream>>>(q0, o0, k0, v0, p);
   return last_launch_status();
 }
 
