@@ -28,7 +28,9 @@ struct BwdParams {
   long long qs0, qs1, qs2, ks0, ks1, ks2, vs0, vs1, vs2, os0, os1, os2, ds0, ds1, ds2;
   const float* lse;      // [B][n_q][T], natural log
   const float* sinks;    // [n_q] or null
-  float* dvec;           // [B][n_q][T] workspace: D_i
+  float* dvec;           // [B][n_q][Tp] workspace: D_i (0 for rows past T)
+  float* lse2;           // [B][n_q][Tp] workspace: lse_i * log2(e) (+inf for rows past T)
+  int Tp;                // T rounded up to a multiple of 64 (whole streamed tiles per row)
   float* dq;             // [B][T][n_q][d]
   float* dk;             // [B][T][n_kv][d]
   float* dv;             // [B][T][n_kv][d]
@@ -38,17 +40,26 @@ struct BwdParams {
   float scale_log2;      // sm_scale * log2(e)
 };
 
-// D_i = <dO_i, o_i> per (b, i, h), one warp per row; each row also adds
-// -exp(sink_h - lse_i) D_i to dsinks[h].
+// D_i = <dO_i, o_i> and lse_i log2(e) per (b, i, h) into the padded
+// workspace rows, one warp per row; each row also adds -exp(sink_h - lse_i) D_i
+// to dsinks[h]. Rows T..Tp-1 get the values of an empty row (D 0, lse +inf).
 template <int D>
 __global__ void bwd_rows_kernel(const BwdParams p) {
   const int lane = threadIdx.x & 31;
-  const long long rows = (long long)p.B * p.T * p.n_q;
+  const long long rows = (long long)p.B * p.Tp * p.n_q;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   for (long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
     const int h = (int)(r % p.n_q);
-    const int i = (int)((r / p.n_q) % p.T);
-    const int b = (int)(r / ((long long)p.n_q * p.T));
+    const int i = (int)((r / p.n_q) % p.Tp);
+    const int b = (int)(r / ((long long)p.n_q * p.Tp));
+    const long long wi = ((long long)b * p.n_q + h) * p.Tp + i;
+    if (i >= p.T) {
+      if (lane == 0) {
+        p.dvec[wi] = 0.f;
+        p.lse2[wi] = INFINITY;
+      }
+      continue;
+    }
     const __nv_bfloat16* orow = p.o + b * p.os0 + i * p.os1 + h * p.os2;
     const __nv_bfloat16* drow = p.dout + b * p.ds0 + i * p.ds1 + h * p.ds2;
     float acc = 0.f;
@@ -58,7 +69,8 @@ __global__ void bwd_rows_kernel(const BwdParams p) {
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (lane == 0) {
       const long long li = ((long long)b * p.n_q + h) * p.T + i;
-      p.dvec[li] = acc;
+      p.dvec[wi] = acc;
+      p.lse2[wi] = p.lse[li] * 1.4426950408889634f;
       if (p.sinks && p.dsinks) atomicAdd(p.dsinks + h, -expf(p.sinks[h] - p.lse[li]) * acc);
     }
   }

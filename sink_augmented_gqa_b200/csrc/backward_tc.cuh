@@ -14,8 +14,12 @@
 //               streamed tile its two BN-row tiles into an NS-deep ring (MODE 1
 //               also stages the tile's lse and D values there).
 //   warp 1      one thread issues the MMAs and owns the TMEM allocation. S and
-//               dP are double-buffered in TMEM, so the tensor core computes the
-//               next tile's S, dP while the current tile's dS is formed.
+//               dP are double-buffered in TMEM, and P, dS are written over the
+//               S, dP columns they came from, so a buffer serves one tile from
+//               its S product to its last read (the issuer waits for the
+//               products of tile u - 2 before tile u reuses it): the tensor
+//               core computes the next tile's S, dP while this tile's P, dS are
+//               formed, and nothing waits for the previous tile's products.
 //   warps 2-9   P, dS from S, dP: two warps per TMEM lane quarter (warp % 4),
 //               each taking half of a tile's columns, one row per thread; tiles
 //               wholly inside the admitted region skip the mask; then the fp32
@@ -34,7 +38,7 @@ __host__ __device__ constexpr int btc_align32(int x) { return (x + 31) / 32 * 32
 template <int D, int MODE>
 struct BtcCfg {
   static constexpr int BM = 128;                                     // resident rows
-  static constexpr int BN = (MODE == 1 && D == 128) ? 32 : 64;       // streamed rows per tile
+  static constexpr int BN = 64;                                      // streamed rows per tile
   static constexpr int CB = (D % 64 == 0) ? 64 : 32;                 // column block (elements)
   static constexpr int SWZ = CB * 2;                                 // bytes per block row
   static constexpr int NCB = D / CB;
@@ -54,11 +58,9 @@ struct BtcCfg {
   // at least 120 KB: one CTA per SM, since each allocates all 512 TMEM columns
   static constexpr uint32_t SMEM_BYTES = (OFF_BAR + 256 + 1024) > 120u * 1024 ? (OFF_BAR + 256 + 1024) : 120u * 1024;
   // TMEM columns
-  static constexpr int S_COL = 0;                  // S[buf] at S_COL + buf * BN
-  static constexpr int DP_COL = 2 * BN;            // dP[buf]
-  static constexpr int P_COL = 4 * BN;             // MODE 1: P (bf16 pairs, BN / 2 columns)
-  static constexpr int DS_COL = 4 * BN + (MODE == 1 ? BN / 2 : 0);   // dS (bf16 pairs)
-  static constexpr int ACC0 = btc_align32(DS_COL + BN / 2);              // dQ | dV
+  static constexpr int S_COL = 0;                  // S[buf] at S_COL + buf * BN, then P (bf16 pairs)
+  static constexpr int DP_COL = 2 * BN;            // dP[buf], then dS (bf16 pairs)
+  static constexpr int ACC0 = 4 * BN;              // dQ | dV
   static constexpr int ACC1 = ACC0 + D;                              // MODE 1: dK
   static constexpr int TMEM_COLS = 512;
   static_assert((MODE == 0 ? ACC0 + D : ACC1 + D) <= TMEM_COLS, "TMEM plan exceeds 512 columns");
@@ -75,7 +77,6 @@ enum : int {
   BB_FULL = 1,       // [4] ring stage landed
   BB_EMPTY = 5,      // [4] ring stage free (MMA commit)
   BB_SFULL = 9,      // [2] S, dP of a buffer computed
-  BB_SFREE = 11,     // [2] count 8 warps: S, dP of a buffer read
   BB_PFULL = 13,     // count 8 warps: P / dS stored in TMEM
   BB_PDONE = 14,     // the products reading P / dS completed
   BB_ACCFULL = 15,   // accumulators final
@@ -95,14 +96,19 @@ __device__ __forceinline__ void btc_issue_s(uint32_t d_tmem, uint64_t adesc, uin
            kk > 0 ? 1u : 0u);
   }
 }
-// acc (+)= A (TMEM bf16, 128 x BN) B (smem [BN][D], MN-major)
+// acc (+)= A (TMEM bf16, 128 x BN) B (smem [BN][D], MN-major). A's elements
+// [HC h, HC h + HC) sit, as bf16 pairs, at columns [HC h, HC h + HC / 2) of
+// its buffer (each P / dS warp writes over the start of the columns it read).
 template <int D, int MODE>
 __device__ __forceinline__ void btc_issue_o(uint32_t acc_tmem, uint32_t a_tmem, uint64_t bdesc, bool accumulate) {
   using C = BtcCfg<D, MODE>;
 #pragma unroll
-  for (int kk = 0; kk < C::BN / 16; ++kk)
-    mma_ts(acc_tmem, a_tmem + kk * 8, bdesc + ((kk * 16 * C::SWZ) >> 4), C::IDESC_O,
+  for (int kk = 0; kk < C::BN / 16; ++kk) {
+    const int e = kk * 16;                                        // first element of the K-step
+    const uint32_t col = (uint32_t)(C::HC * (e / C::HC) + (e % C::HC) / 2);
+    mma_ts(acc_tmem, a_tmem + col, bdesc + ((kk * 16 * C::SWZ) >> 4), C::IDESC_O,
            (accumulate || kk > 0) ? 1u : 0u);
+  }
 }
 
 template <int D, int MODE>
@@ -161,10 +167,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(bar(BB_FULL + s), 1);
       mbar_init(bar(BB_EMPTY + s), 1);
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(bar(BB_SFULL + x), 1);
-      mbar_init(bar(BB_SFREE + x), C::NSW);
-    }
+    for (int x = 0; x < 2; ++x) mbar_init(bar(BB_SFULL + x), 1);
     mbar_init(bar(BB_PFULL), C::NSW);
     mbar_init(bar(BB_PDONE), 1);
     mbar_init(bar(BB_ACCFULL), 1);
@@ -209,19 +212,16 @@ __global__ void __launch_bounds__(320, 1)
       if (*abort_flag) { ok = false; break; }
       int hh, s0;
       stream_of(u, hh, s0);
-      if constexpr (MODE == 1) {
-        // lse (times log2 e) and D of the tile's BN query rows, beside its tiles
-        float* rv = reinterpret_cast<float*>(smem + C::OFF_ROWV) + s * 2 * BN;
-        const long long rb = ((long long)b * p.n_q + hh) * p.T;
-        for (int c = lane; c < BN; c += 32) {
-          const int i = s0 + c;
-          rv[c] = i < p.T ? p.lse[rb + i] * 1.4426950408889634f : INFINITY;
-          rv[BN + c] = i < p.T ? p.dvec[rb + i] : 0.f;
-        }
-        __syncwarp();
-      }
       if (lane == 0) {
-        mbar_arrive_expect_tx(bar(BB_FULL + s), C::STAGE_BYTES);
+        mbar_arrive_expect_tx(bar(BB_FULL + s), C::STAGE_BYTES + (MODE == 1 ? 2 * BN * 4 : 0));
+        if constexpr (MODE == 1) {
+          // lse * log2(e) and D of the tile's BN query rows, beside its tiles
+          // (padded workspace rows: 16-byte aligned, valid past T)
+          const long long wb = ((long long)b * p.n_q + hh) * p.Tp + s0;
+          const uint32_t rv = sbase + C::OFF_ROWV + s * 2 * BN * 4;
+          bulk_load(rv, p.lse2 + wb, BN * 4, bar(BB_FULL + s));
+          bulk_load(rv + BN * 4, p.dvec + wb, BN * 4, bar(BB_FULL + s));
+        }
         const int sh = (MODE == 0) ? g : hh;   // head of the streamed tiles
         const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_BYTES;
 #pragma unroll
@@ -247,17 +247,16 @@ __global__ void __launch_bounds__(320, 1)
       const uint64_t a1 = smem_desc(sbase + C::OFF_R1, 16, C::SBO, C::LAYOUT);   // dO | V
       auto o_products = [&](int v) {   // the products of tile v that read P / dS
         const int sv = v % C::NS;
+        const uint32_t pcol = tmem + C::S_COL + (v & 1) * BN, dscol = tmem + C::DP_COL + (v & 1) * BN;
         const uint32_t st = sbase + C::OFF_ST + sv * C::STAGE_BYTES;
         if constexpr (MODE == 0) {
           // dQ += dS K (K of the stage, MN-major)
-          btc_issue_o<D, MODE>(tmem + C::ACC0, tmem + C::DS_COL,
-                               smem_desc(st, C::NBLOCK, C::SBO, C::LAYOUT), v > 0);
+          btc_issue_o<D, MODE>(tmem + C::ACC0, dscol, smem_desc(st, C::NBLOCK, C::SBO, C::LAYOUT), v > 0);
         } else {
           // dV += P^T dO, dK += dS^T Q
-          btc_issue_o<D, MODE>(tmem + C::ACC0, tmem + C::P_COL,
-                               smem_desc(st + C::N_BYTES, C::NBLOCK, C::SBO, C::LAYOUT), v > 0);
-          btc_issue_o<D, MODE>(tmem + C::ACC1, tmem + C::DS_COL, smem_desc(st, C::NBLOCK, C::SBO, C::LAYOUT),
+          btc_issue_o<D, MODE>(tmem + C::ACC0, pcol, smem_desc(st + C::N_BYTES, C::NBLOCK, C::SBO, C::LAYOUT),
                                v > 0);
+          btc_issue_o<D, MODE>(tmem + C::ACC1, dscol, smem_desc(st, C::NBLOCK, C::SBO, C::LAYOUT), v > 0);
         }
         mma_commit(bar(BB_PDONE));
         mma_commit(bar(BB_EMPTY + sv));
@@ -265,7 +264,8 @@ __global__ void __launch_bounds__(320, 1)
       for (int u = 0; u < n_tiles && ok; ++u) {
         const int s = u % C::NS, x = u & 1;
         if (!mbar_wait(bar(BB_FULL + s), (uint32_t)((u / C::NS) & 1))) { ok = false; break; }
-        if (u >= 2 && !mbar_wait(bar(BB_SFREE + x), (uint32_t)(((u >> 1) - 1) & 1))) { ok = false; break; }
+        // buffer x last served tile u - 2: its products have read P / dS
+        if (u >= 2 && !mbar_wait(bar(BB_PDONE), (uint32_t)((u - 2) & 1))) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_BYTES;
         // S = R0 S0^T, dP = R1 S1^T (both K-major)
@@ -302,14 +302,13 @@ __global__ void __launch_bounds__(320, 1)
     const int rr = quarter * 32 + lane;                  // resident row of this thread
     const int row = r0 + rr;                              // query (MODE 0) or key (MODE 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const float LOG2E = 1.4426950408889634f;
     const float sl2 = p.scale_log2;
     float lse2 = 0.f, dval = 0.f;
     if constexpr (MODE == 0) {
-      if (row < p.T) {
-        const long long li = ((long long)b * p.n_q + head) * p.T + row;
-        lse2 = p.lse[li] * LOG2E;
-        dval = p.dvec[li];
+      const long long wi = ((long long)b * p.n_q + head) * p.Tp + row;
+      if (row < p.Tp) {
+        lse2 = p.lse2[wi];
+        dval = p.dvec[wi];
       }
     }
     // every wait below is taken warp-uniformly: the TMEM loads and stores
@@ -351,6 +350,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       tmem_wait_ld();
       uint32_t pk[HC / 2], dk[HC / 2];
+      float4 lv4 = make_float4(0.f, 0.f, 0.f, 0.f), dv4 = lv4;
 #pragma unroll
       for (int c = 0; c < HC; c += 2) {
         float l0, l1, d0, d1;
@@ -358,13 +358,25 @@ __global__ void __launch_bounds__(320, 1)
           l0 = l1 = lse2;
           d0 = d1 = dval;
         } else {
-          const float2 lv = *reinterpret_cast<const float2*>(rv + c_base + c);
-          const float2 dd = *reinterpret_cast<const float2*>(rv + BN + c_base + c);
-          l0 = lv.x; l1 = lv.y; d0 = dd.x; d1 = dd.y;
+          if ((c & 3) == 0) {   // the tile's per-column lse / D, four at a time
+            lv4 = *reinterpret_cast<const float4*>(rv + c_base + c);
+            dv4 = *reinterpret_cast<const float4*>(rv + BN + c_base + c);
+          }
+          l0 = (c & 3) ? lv4.z : lv4.x;
+          l1 = (c & 3) ? lv4.w : lv4.y;
+          d0 = (c & 3) ? dv4.z : dv4.x;
+          d1 = (c & 3) ? dv4.w : dv4.y;
         }
-        float x0, x1;
-        fma2(x0, x1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl2, sl2, -l0, -l1);
-        float p0 = ex2(x0), p1 = ex2(x1);
+        float p0, p1;
+        fma2(p0, p1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl2, sl2, -l0, -l1);
+        // one pair in four on the FMA pipe (the degree-3 exp2 of the
+        // forward), the rest on the MUFU unit
+        if (((c / 2) & 3) == 0) {
+          exp2_fma2(p0, p1);
+        } else {
+          p0 = ex2(p0);
+          p1 = ex2(p1);
+        }
         if (!all_in) {
           const int col = s0 + c_base + c;
           if (MODE == 0) {
@@ -378,28 +390,18 @@ __global__ void __launch_bounds__(320, 1)
         float t0 = __uint_as_float(dv[c]), t1 = __uint_as_float(dv[c + 1]);
         add2(t0, t1, -d0, -d1);
         mul2(t0, t1, p0, p1);
-        pk[c / 2] = pack_bf16(p0, p1);
+        if constexpr (MODE == 1) pk[c / 2] = pack_bf16(p0, p1);
         dk[c / 2] = pack_bf16(t0, t1);
       }
-      // P / dS of the previous tile are read by its products until they complete
-      if (u > 0) {
-        if (!wait_all(bar(BB_PDONE), (uint32_t)((u - 1) & 1))) { ok = false; break; }
-        tc_fence_after();
-      }
-      if constexpr (HC == 32) {
-        tmem_st16(tmem + lane_base + C::DS_COL + c_base / 2, dk);
-        if constexpr (MODE == 1) tmem_st16(tmem + lane_base + C::P_COL + c_base / 2, pk);
-      } else {
-        tmem_st8(tmem + lane_base + C::DS_COL + c_base / 2, dk);
-        if constexpr (MODE == 1) tmem_st8(tmem + lane_base + C::P_COL + c_base / 2, pk);
-      }
+      // P / dS over the start of the S / dP columns this warp read (the
+      // other warp of the quarter reads and writes only its own columns)
+      static_assert(HC == 32, "one 32-column chunk per P / dS warp");
+      tmem_st16(tmem + lane_base + C::DP_COL + x * BN + c_base, dk);
+      if constexpr (MODE == 1) tmem_st16(tmem + lane_base + C::S_COL + x * BN + c_base, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar(BB_SFREE + x));
-        mbar_arrive(bar(BB_PFULL));
-      }
+      if (lane == 0) mbar_arrive(bar(BB_PFULL));
       if (*abort_flag) { ok = false; break; }
     }
     // epilogue: the accumulators (zero when no tile was admitted) -> fp32

@@ -540,7 +540,11 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
   p.ds0 = a->d_out_strides[0]; p.ds1 = a->d_out_strides[1]; p.ds2 = a->d_out_strides[2];
   p.lse = a->lse;
   p.sinks = a->sinks;
+  // rows padded to a multiple of 64 (every streamed tile's BN <= 64 values lie
+  // inside its row; 16-byte aligned)
+  p.Tp = (a->T + 63) / 64 * 64;
   p.dvec = dvec;
+  p.lse2 = dvec + (size_t)a->B * a->n_q * p.Tp;
   p.dq = a->dq;
   p.dk = a->dk;
   p.dv = a->dv;
@@ -554,7 +558,7 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
   p.scale = a->sm_scale;
   p.scale_log2 = a->sm_scale * 1.4426950408889634f;
   if (p.dsinks && cudaMemsetAsync(p.dsinks, 0, sizeof(float) * a->n_q, stream) != cudaSuccess) return SA_ERR_CUDA;
-  const long long rows = (long long)a->B * a->T * a->n_q;
+  const long long rows = (long long)a->B * p.Tp * a->n_q;
   sa::bwd_rows_kernel<D><<<grid_for(rows * 32), 256, 0, stream>>>(p);
   using C0 = sa::BtcCfg<D, 0>;
   using C1 = sa::BtcCfg<D, 1>;
@@ -841,7 +845,8 @@ sa_status sa_out_proj(const void* o, int64_t ldo, const void* w, int64_t ldw, co
 
 size_t sa_attn_backward_workspace_size(int32_t B, int32_t T, int32_t n_q) {
   if (B < 1 || T < 1 || n_q < 1) return 0;
-  return ((size_t)B * n_q * T * 4 + 255) / 256 * 256;
+  const size_t Tp = ((size_t)T + 63) / 64 * 64;   // D and lse * log2(e), rows padded to 64 entries
+  return (2 * (size_t)B * n_q * Tp * 4 + 255) / 256 * 256;
 }
 
 sa_status sa_attn_backward(const sa_attn_bwd_args* a, void* workspace, size_t workspace_bytes,
