@@ -11,20 +11,24 @@
 // normalised activations are never materialised) and s_m = 1 for the out
 // projection, whose epilogue adds the residual (x <- x + out(o), in place).
 //
-// One CTA per SM walks 128 x 256 output tiles (tile t, t + grid, ...):
+// One CTA per SM walks 256 x 256 output tiles (tile t, t + grid, ...):
 //
-//   warp 0      TMA producer: per 64-wide K step, the A tile (128 x 64) and
-//               the W tile (256 x 64), 128-byte swizzled, into a 4-deep ring.
+//   warp 0      TMA producer: per 64-wide K step, the A tile (256 x 64) and
+//               the W tile (256 x 64), 128-byte swizzled, into a 3-deep ring.
 //   warp 1      one thread issues tcgen05.mma (kind::f16, M 128, N 256, K 16
-//               per instruction, fp32 accumulation in TMEM); the tile's
-//               accumulator alternates between two 256-column TMEM buffers so
-//               the epilogue of one tile overlaps the main loop of the next.
+//               per instruction, fp32 accumulation in TMEM): two products per
+//               K step, rows 0-127 and 128-255 of A against the same W tile
+//               (131 flops per operand byte instead of 87 with one), into the
+//               two 256-column halves of TMEM.
 //   warps 2, 3  (RMSNorm only) sum the squares of each A row from the same
 //               shared-memory tiles the tensor core reads, and publish s_m.
-//   warps 4-7   epilogue, one output row per thread (TMEM lane = row): per
-//               32-column chunk, tcgen05.ld, scale, bias, residual, bf16,
-//               staged in shared memory (64-byte swizzle) and written by a
-//               TMA tile store (which clips the ragged edges of M and N).
+//   warps 4-11  epilogue, one output row per thread (warp 4 + 4 h + q reads
+//               TMEM lanes 32 q.. of half h): per 32-column chunk,
+//               tcgen05.ld, scale, bias, residual, bf16, staged in shared
+//               memory (64-byte swizzle) and written by a TMA tile store
+//               (which clips the ragged edges of M and N). The accumulator is
+//               single-buffered: the next tile's products wait for this
+//               drain (a few per cent of a tile's main loop).
 #pragma once
 
 #include "ptx.cuh"
@@ -41,32 +45,41 @@ struct GemmParams {
   int tiles_m, tiles_n;
 };
 
+// BN_: output columns per tile (256); the two accumulator halves sit at TMEM
+// columns 0 and 256.
+template <int BN_>
 struct GemmCfg {
-  static constexpr int BM = 128, BN = 256, BK = 64;
-  static constexpr int NS = 4;                               // ring depth
-  static constexpr uint32_t A_BYTES = BM * BK * 2;           // 16 KB
+  static constexpr int BM = 256, BN = BN_, BK = 64;
+  static constexpr int NS = 3;                               // ring depth
+  static constexpr uint32_t A_BYTES = BM * BK * 2;           // 32 KB
+  static constexpr uint32_t A_HALF = 128 * BK * 2;           // rows 128.. of the A tile
   static constexpr uint32_t B_BYTES = BN * BK * 2;           // 32 KB
   static constexpr uint32_t OFF_A = 0;
   static constexpr uint32_t OFF_B = NS * A_BYTES;
-  static constexpr uint32_t OFF_ST = OFF_B + NS * B_BYTES;   // [4 warps][2] 32 rows x 64 B
+  static constexpr int EPI_WARPS = 8;
+  static constexpr uint32_t OFF_ST = OFF_B + NS * B_BYTES;   // [8 warps][2] 32 rows x 64 B
   static constexpr uint32_t ST_BYTES = 32 * 64;
-  static constexpr uint32_t OFF_RMS = OFF_ST + 8 * ST_BYTES;  // [2][128] fp32 row scales
-  static constexpr uint32_t OFF_BAR = OFF_RMS + 2 * 128 * 4;
+  static constexpr uint32_t OFF_RMS = OFF_ST + EPI_WARPS * 2 * ST_BYTES;   // [256] fp32 row scales
+  static constexpr uint32_t OFF_BAR = OFF_RMS + BM * 4;
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;   // + alignment slack
+  static_assert(SMEM_BYTES <= 232448, "dynamic shared memory per block");
   static constexpr int TMEM_COLS = 512;
-  static constexpr uint32_t IDESC = idesc_bf16(128, 256, 0, 0);
+  static constexpr uint32_t IDESC = idesc_bf16(128, BN, 0, 0);
   static constexpr uint32_t SBO = 1024;                      // 8 rows x 128 B
-  static constexpr int NUM_THREADS = 256;
-  static_assert(OFF_B % 1024 == 0 && OFF_ST % 1024 == 0, "swizzled buffers need 1 KB alignment");
+  static constexpr uint32_t HALF_COL = 256;                  // TMEM column of accumulator half 1
+  static constexpr int NUM_THREADS = 32 * (4 + EPI_WARPS);
+  static_assert(BN % 32 == 0 && BN <= 256, "whole 32-column epilogue chunks");
+  static_assert(OFF_B % 1024 == 0 && OFF_ST % 1024 == 0 && A_HALF % 1024 == 0 && B_BYTES % 1024 == 0,
+                "swizzled buffers need 1 KB alignment");
 };
 
 enum : int {
   GB_FULL = 0,        // [NS] producer -> MMA, RMS warps: A and W tiles landed
   GB_EMPTY = 4,       // [NS] MMA (commit) + RMS warps -> producer
-  GB_ACC_FULL = 8,    // [2] MMA -> epilogue: the tile's accumulator is complete
-  GB_ACC_EMPTY = 10,  // [2] epilogue warps -> MMA: accumulator read
-  GB_RMS_FULL = 12,   // [2] RMS warps -> epilogue: row scales of the tile
-  GB_RMS_EMPTY = 14,  // [2] epilogue warps -> RMS warps
+  GB_ACC_FULL = 8,    // MMA -> epilogue: the tile's accumulator is complete
+  GB_ACC_EMPTY = 10,  // count 8: epilogue warps -> MMA: accumulator read
+  GB_RMS_FULL = 12,   // count 2: RMS warps -> epilogue: row scales of the tile
+  GB_RMS_EMPTY = 14,  // count 8: epilogue warps -> RMS warps
   GB_DRAIN = 16,      // MMA issuer, on abort
   GB_TMEM_SLOT = 17,
   GB_ABORT_SLOT = 18,
@@ -76,10 +89,11 @@ __device__ __forceinline__ void bulk_wait_read_1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
-__global__ void __launch_bounds__(256, 1)
+template <int BN_>
+__global__ void __launch_bounds__(384, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const GemmParams p) {
-  using C = GemmCfg;
+  using C = GemmCfg<BN_>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -98,12 +112,10 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(bar(GB_FULL + s), 1);
       mbar_init(bar(GB_EMPTY + s), p.rms ? 3 : 1);   // MMA commit (+ one arrival per RMS warp)
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bar(GB_ACC_FULL + b), 1);
-      mbar_init(bar(GB_ACC_EMPTY + b), 4);
-      mbar_init(bar(GB_RMS_FULL + b), 2);
-      mbar_init(bar(GB_RMS_EMPTY + b), 4);
-    }
+    mbar_init(bar(GB_ACC_FULL), 1);
+    mbar_init(bar(GB_ACC_EMPTY), C::EPI_WARPS);
+    mbar_init(bar(GB_RMS_FULL), 2);
+    mbar_init(bar(GB_RMS_EMPTY), C::EPI_WARPS);
     mbar_init(bar(GB_DRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -163,10 +175,9 @@ __global__ void __launch_bounds__(256, 1)
       int it = 0, tl = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
-        const int buf = tl & 1;
-        if (tl >= 2 && !mbar_wait(bar(GB_ACC_EMPTY + buf), (uint32_t)(((tl >> 1) - 1) & 1))) { ok = false; break; }
+        // the accumulator (both halves) has been drained by the previous tile's epilogue
+        if (tl >= 1 && !mbar_wait(bar(GB_ACC_EMPTY), (uint32_t)((tl - 1) & 1))) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(buf * C::BN);
         for (int kb = 0; kb < n_kb; ++kb, ++it) {
           const int s = it % C::NS;
           if (!mbar_wait(bar(GB_FULL + s), (uint32_t)((it / C::NS) & 1))) { ok = false; break; }
@@ -174,12 +185,15 @@ __global__ void __launch_bounds__(256, 1)
           const uint64_t ad = ad0 + ((uint32_t)(s * C::A_BYTES) >> 4);
           const uint64_t bd = bd0 + ((uint32_t)(s * C::B_BYTES) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk)   // 32 bytes further along the swizzled rows
-            mma_ss(d, ad + 2 * kk, bd + 2 * kk, C::IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < C::BK / 16; ++kk) {   // 32 bytes further along the swizzled rows
+            mma_ss(tmem, ad + 2 * kk, bd + 2 * kk, C::IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_ss(tmem + C::HALF_COL, ad + (C::A_HALF >> 4) + 2 * kk, bd + 2 * kk, C::IDESC,
+                   (kb > 0 || kk > 0) ? 1u : 0u);
+          }
           mma_commit(bar(GB_EMPTY + s));
         }
         if (!ok) break;
-        mma_commit(bar(GB_ACC_FULL + buf));
+        mma_commit(bar(GB_ACC_FULL));
         if (*abort_flag) { ok = false; break; }
       }
       if (!ok) {
@@ -191,40 +205,40 @@ __global__ void __launch_bounds__(256, 1)
   } else if (warp < 4) {
     // ------------------------------------------------------------ RMSNorm row scales
     if (p.rms) {
-      const int r0 = 32 * (warp - 2) + lane, r1 = r0 + 64;   // rows of the A tile
+      const int rb0 = 32 * (warp - 2) + lane;   // rows rb0 + 64 i of the A tile, i < 4
       const float inv_k = 1.0f / (float)p.K;
       int it = 0, tl = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
-        float s0 = 0.f, s1 = 0.f;
+        float ss[4] = {0.f, 0.f, 0.f, 0.f};
         for (int kb = 0; kb < n_kb; ++kb, ++it) {
           const int s = it % C::NS;
           if (!mbar_wait(bar(GB_FULL + s), (uint32_t)((it / C::NS) & 1))) { ok = false; break; }
           const uint8_t* a = smem + C::OFF_A + s * C::A_BYTES;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {   // 16-byte chunk j of a row sits at chunk j ^ (row % 8)
-            const uint4 u0 = *reinterpret_cast<const uint4*>(a + r0 * 128 + ((j ^ (r0 & 7)) << 4));
-            const uint4 u1 = *reinterpret_cast<const uint4*>(a + r1 * 128 + ((j ^ (r1 & 7)) << 4));
-            const uint32_t w0[4] = {u0.x, u0.y, u0.z, u0.w}, w1[4] = {u1.x, u1.y, u1.z, u1.w};
+          for (int i = 0; i < 4; ++i) {
+            const int r = rb0 + 64 * i;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float a0 = bf16_lo(w0[e]), a1 = bf16_hi(w0[e]);
-              const float b0 = bf16_lo(w1[e]), b1 = bf16_hi(w1[e]);
-              s0 = fmaf(a0, a0, fmaf(a1, a1, s0));
-              s1 = fmaf(b0, b0, fmaf(b1, b1, s1));
+            for (int j = 0; j < 8; ++j) {   // 16-byte chunk j of a row sits at chunk j ^ (row % 8)
+              const uint4 u = *reinterpret_cast<const uint4*>(a + r * 128 + ((j ^ (r & 7)) << 4));
+              const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const float a0 = bf16_lo(w[e]), a1 = bf16_hi(w[e]);
+                ss[i] = fmaf(a0, a0, fmaf(a1, a1, ss[i]));
+              }
             }
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(GB_EMPTY + s));
         }
         if (!ok) break;
-        const int buf = tl & 1;
-        if (tl >= 2 && !mbar_wait(bar(GB_RMS_EMPTY + buf), (uint32_t)(((tl >> 1) - 1) & 1))) { ok = false; break; }
-        float* rb = reinterpret_cast<float*>(smem + C::OFF_RMS) + buf * 128;
-        rb[r0] = 1.0f / sqrtf(s0 * inv_k + p.eps);
-        rb[r1] = 1.0f / sqrtf(s1 * inv_k + p.eps);
+        if (tl >= 1 && !mbar_wait(bar(GB_RMS_EMPTY), (uint32_t)((tl - 1) & 1))) { ok = false; break; }
+        float* rb = reinterpret_cast<float*>(smem + C::OFF_RMS);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) rb[rb0 + 64 * i] = 1.0f / sqrtf(ss[i] * inv_k + p.eps);
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(GB_RMS_FULL + buf));
+        if (lane == 0) mbar_arrive(bar(GB_RMS_FULL));
         if (*abort_flag) { ok = false; break; }
       }
       if (!ok) *abort_flag = 1;
@@ -232,29 +246,29 @@ __global__ void __launch_bounds__(256, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;                  // TMEM lane quarter of this warp
-    const int r = 32 * q + lane;             // row within the tile
+    const int hh = (warp - 4) >> 2;          // accumulator half: rows 128 hh ..
+    const int r = 128 * hh + 32 * q + lane;  // row within the tile
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     int tl = 0, cnt = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
       int m0, n0;
       tile_origin(t, m0, n0);
-      const int buf = tl & 1;
-      if (!mbar_wait(bar(GB_ACC_FULL + buf), (uint32_t)((tl >> 1) & 1))) { ok = false; break; }
+      if (!mbar_wait(bar(GB_ACC_FULL), (uint32_t)(tl & 1))) { ok = false; break; }
       tc_fence_after();
       float sc = 1.f;
       if (p.rms) {
-        if (!mbar_wait(bar(GB_RMS_FULL + buf), (uint32_t)((tl >> 1) & 1))) { ok = false; break; }
-        sc = reinterpret_cast<const float*>(smem + C::OFF_RMS)[buf * 128 + r];
+        if (!mbar_wait(bar(GB_RMS_FULL), (uint32_t)(tl & 1))) { ok = false; break; }
+        sc = reinterpret_cast<const float*>(smem + C::OFF_RMS)[r];
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(GB_RMS_EMPTY + buf));
+        if (lane == 0) mbar_arrive(bar(GB_RMS_EMPTY));
       }
       const int m = m0 + r;
       const bool row_ok = m < p.M;
       const int nch = min(C::BN / 32, (p.N - n0 + 31) / 32);
       for (int c = 0; c < nch; ++c) {
         uint32_t v[32];
-        tmem_ld32(tmem + lane_base + (uint32_t)(buf * C::BN + 32 * c), v);
+        tmem_ld32(tmem + lane_base + (uint32_t)(hh * C::HALF_COL + 32 * c), v);
         tmem_wait_ld();
         const int nb = n0 + 32 * c;
         const bool full = nb + 32 <= p.N;
@@ -295,7 +309,7 @@ __global__ void __launch_bounds__(256, 1)
         // stage the 32 x 32 chunk of this warp (64-byte rows, 64-byte swizzle:
         // 16-byte chunk j of row r at j ^ ((r / 2) % 4)) and store it by TMA
         const int sb = cnt & 1;
-        uint8_t* st = smem + C::OFF_ST + (uint32_t)(q * 2 + sb) * C::ST_BYTES;
+        uint8_t* st = smem + C::OFF_ST + (uint32_t)((warp - 4) * 2 + sb) * C::ST_BYTES;
         if (cnt >= 2) {
           if (lane == 0) bulk_wait_read_1();   // the store that last used this buffer has read it
           __syncwarp();
@@ -312,16 +326,17 @@ __global__ void __launch_bounds__(256, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          if (m0 + 32 * q < p.M)   // rows past M are clipped; a wholly outside chunk is not stored
-            tma_store_4d(&tmC, smem_u32(st), nb, m0 + 32 * q, 0, 0);
+          const int row0 = m0 + 128 * hh + 32 * q;
+          if (row0 < p.M)   // rows past M are clipped; a wholly outside chunk is not stored
+            tma_store_4d(&tmC, smem_u32(st), nb, row0, 0, 0);
           bulk_commit();
         }
         ++cnt;
       }
-      // the accumulator buffer is free for the tile after next
+      // the accumulator is free for the next tile's products
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(GB_ACC_EMPTY + buf));
+      if (lane == 0) mbar_arrive(bar(GB_ACC_EMPTY));
       if (*abort_flag) { ok = false; break; }
     }
     if (lane == 0) bulk_wait_all();   // output stores complete before the CTA exits
