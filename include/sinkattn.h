@@ -344,7 +344,8 @@ sa_status sa_attn_decode_static(sa_kv_cache* cache, const sa_attn_args* args, sa
  * Products run on the tensor cores (bf16 operands, fp32 accumulation); P and
  * dS enter their products as bf16. Errors: SA_ERR_INVALID_ARG (null,
  * misaligned, bad stride, B/T/n_q < 1), SA_ERR_SHAPE (d not in {64, 96,
- * 128}, n_q % n_kv != 0), SA_ERR_WORKSPACE (too small), SA_ERR_CUDA.
+ * 128}, n_q % n_kv != 0, n_q > 8192, ceil(T / 128) (n_q + n_kv) B >= 2^31),
+ * SA_ERR_WORKSPACE (too small), SA_ERR_CUDA.
  */
 typedef struct sa_attn_bwd_args {
   const void* q;     int64_t q_strides[3];

@@ -42,9 +42,16 @@ struct BwdParams {
 
 // D_i = <dO_i, o_i> and lse_i log2(e) per (b, i, h) into the padded
 // workspace rows, one warp per row; each row also adds -exp(sink_h - lse_i) D_i
-// to dsinks[h]. Rows T..Tp-1 get the values of an empty row (D 0, lse +inf).
+// to dsinks[h], through a per-block sum in shared memory (dynamic, n_q
+// floats) so that global memory sees one atomic per block and head. Rows
+// T..Tp-1 get the values of an empty row (D 0, lse +inf).
 template <int D>
 __global__ void bwd_rows_kernel(const BwdParams p) {
+  extern __shared__ float dsink_part[];
+  const bool sink = p.sinks && p.dsinks;
+  if (sink)
+    for (int h = threadIdx.x; h < p.n_q; h += blockDim.x) dsink_part[h] = 0.f;
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const long long rows = (long long)p.B * p.Tp * p.n_q;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -71,8 +78,12 @@ __global__ void bwd_rows_kernel(const BwdParams p) {
       const long long li = ((long long)b * p.n_q + h) * p.T + i;
       p.dvec[wi] = acc;
       p.lse2[wi] = p.lse[li] * 1.4426950408889634f;
-      if (p.sinks && p.dsinks) atomicAdd(p.dsinks + h, -expf(p.sinks[h] - p.lse[li]) * acc);
+      if (sink) atomicAdd(dsink_part + h, -expf(p.sinks[h] - p.lse[li]) * acc);
     }
+  }
+  if (sink) {
+    __syncthreads();
+    for (int h = threadIdx.x; h < p.n_q; h += blockDim.x) atomicAdd(p.dsinks + h, dsink_part[h]);
   }
 }
 

@@ -9,7 +9,8 @@
 //                 dP^T = V dO^T, P^T and dS^T as bf16 into TMEM, then
 //                 dV += P^T dO and dK += dS^T Q.
 //
-// One CTA per 128-row tile (heaviest tiles first), 192 threads:
+// One CTA per 128-row tile (both passes in one launch, heaviest tiles first),
+// 320 threads:
 //   warp 0      TMA loads: the two resident 128-row tiles once, then per
 //               streamed tile its two BN-row tiles into an NS-deep ring (MODE 1
 //               also stages the tile's lse and D values there).
@@ -111,11 +112,13 @@ __device__ __forceinline__ void btc_issue_o(uint32_t acc_tmem, uint32_t a_tmem, 
   }
 }
 
+// One CTA of either pass: resident row tile `tile` of query head (MODE 0) or
+// KV head (MODE 1) `head` of sequence b. tmR0 / tmR1 map the resident tiles'
+// tensors, tmS0 / tmS1 the streamed ones (kernel parameters).
 template <int D, int MODE>
-__global__ void __launch_bounds__(320, 1)
-    bwd_tc_kernel(const __grid_constant__ CUtensorMap tmR0, const __grid_constant__ CUtensorMap tmR1,
-                  const __grid_constant__ CUtensorMap tmS0, const __grid_constant__ CUtensorMap tmS1,
-                  const BwdParams p) {
+__device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtensorMap* tmR1,
+                                           const CUtensorMap* tmS0, const CUtensorMap* tmS1,
+                                           const BwdParams& p, const int tile, const int head, const int b) {
   using C = BtcCfg<D, MODE>;
   constexpr int BN = C::BN;
   extern __shared__ uint8_t smem_raw[];
@@ -128,11 +131,7 @@ __global__ void __launch_bounds__(320, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * BB_ABORT_SLOT);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // heaviest row tiles (last queries / first keys of a causal layer) first
-  const int tile = (MODE == 0) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
   const int r0 = tile * C::BM;          // first resident row
-  const int head = blockIdx.y;          // query head (MODE 0) or KV head (MODE 1)
-  const int b = blockIdx.z;
   // Streamed tiles. MODE 0: key tiles [t_lo, t_hi) of BN keys seen by
   // queries r0..r0+127. MODE 1: for each head of the group, query tiles
   // [t_lo, t_hi) of BN queries that see keys r0..r0+127.
@@ -187,16 +186,16 @@ __global__ void __launch_bounds__(320, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmR0);
-      tma_prefetch_desc(&tmR1);
-      tma_prefetch_desc(&tmS0);
-      tma_prefetch_desc(&tmS1);
+      tma_prefetch_desc(tmR0);
+      tma_prefetch_desc(tmR1);
+      tma_prefetch_desc(tmS0);
+      tma_prefetch_desc(tmS1);
       mbar_arrive_expect_tx(bar(BB_RFULL), 2 * C::M_BYTES);
       const int rh = (MODE == 0) ? head : g;   // head of the resident tiles
 #pragma unroll
       for (int cb = 0; cb < C::NCB; ++cb) {
-        tma_load_4d(sbase + C::OFF_R0 + cb * C::MBLOCK, &tmR0, bar(BB_RFULL), cb * C::CB, r0, rh, b);
-        tma_load_4d(sbase + C::OFF_R1 + cb * C::MBLOCK, &tmR1, bar(BB_RFULL), cb * C::CB, r0, rh, b);
+        tma_load_4d(sbase + C::OFF_R0 + cb * C::MBLOCK, tmR0, bar(BB_RFULL), cb * C::CB, r0, rh, b);
+        tma_load_4d(sbase + C::OFF_R1 + cb * C::MBLOCK, tmR1, bar(BB_RFULL), cb * C::CB, r0, rh, b);
       }
     }
     int issued = 0;
@@ -226,8 +225,8 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_BYTES;
 #pragma unroll
         for (int cb = 0; cb < C::NCB; ++cb) {
-          tma_load_4d(st + cb * C::NBLOCK, &tmS0, bar(BB_FULL + s), cb * C::CB, s0, sh, b);
-          tma_load_4d(st + C::N_BYTES + cb * C::NBLOCK, &tmS1, bar(BB_FULL + s), cb * C::CB, s0, sh, b);
+          tma_load_4d(st + cb * C::NBLOCK, tmS0, bar(BB_FULL + s), cb * C::CB, s0, sh, b);
+          tma_load_4d(st + C::N_BYTES + cb * C::NBLOCK, tmS1, bar(BB_FULL + s), cb * C::CB, s0, sh, b);
         }
       }
       issued = u + 1;
@@ -456,6 +455,28 @@ __global__ void __launch_bounds__(320, 1)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+// Both passes in one launch (they read the same inputs and write disjoint
+// outputs), so the tail of one fills with CTAs of the other. Blocks are
+// ordered by level k = 0, 1, ...: the n_kv B dK/dV CTAs of key tile k, then
+// the n_q B dQ CTAs of query tile tiles - 1 - k; under a causal mask both
+// shrink with k, so the heaviest CTAs start first.
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap k1, const __grid_constant__ CUtensorMap v1,
+                  const __grid_constant__ CUtensorMap q1, const __grid_constant__ CUtensorMap o1,
+                  const __grid_constant__ CUtensorMap q0, const __grid_constant__ CUtensorMap o0,
+                  const __grid_constant__ CUtensorMap k0, const __grid_constant__ CUtensorMap v0,
+                  const BwdParams p) {
+  const int tiles = (p.T + 127) / 128;
+  const int nkv = p.n_kv * p.B, nq = p.n_q * p.B;
+  const int level = (int)blockIdx.x / (nkv + nq);
+  const int r = (int)blockIdx.x % (nkv + nq);
+  if (r < nkv)
+    bwd_tc_cta<D, 1>(&k1, &v1, &q1, &o1, p, level, r % p.n_kv, r / p.n_kv);
+  else
+    bwd_tc_cta<D, 0>(&q0, &o0, &k0, &v0, p, tiles - 1 - level, (r - nkv) % p.n_q, (r - nkv) / p.n_q);
 }
 
 }  // namespace sa

@@ -377,6 +377,18 @@ __device__ __forceinline__ void decode_subtile_f8(uint32_t kst, uint32_t vst, ui
   }
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the kernel before it in the stream is still
+// running; griddep_wait() returns once that kernel has completed and its
+// memory operations are visible (at once when the launch had no such
+// predecessor), so nothing before it may read memory another kernel writes.
+// griddep_launch_dependents() lets the next such kernel be scheduled before
+// this one has finished.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // tmK/tmV: the cache's K/V (bf16 elements, or FP8 code bytes); tmKS/tmVS
 // (FP8 only): the row scales, dims {rows, n_kv, B, 1}, box {R, 1, 1, 1}.
 template <int D, bool F8>
@@ -409,6 +421,9 @@ __global__ void __launch_bounds__(288, 2)
   const int n_stages = r_end > r_begin ? (int)((r_end - r_begin + C::R - 1) / C::R) : 0;
   const bool last_split = split == p.S - 1;
 
+  // The next layer's launch may take this CTA's slot as soon as it frees up;
+  // it does its own set-up there and then waits for this grid to complete.
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(full_bar(s), 1);
@@ -419,6 +434,9 @@ __global__ void __launch_bounds__(288, 2)
     fence_barrier_init();
   }
   __syncthreads();
+  // Everything below reads or writes global memory (q, the cache, the split
+  // workspace, the output), which the kernel before this one may still be using.
+  griddep_wait();
 
   if (warp == C::NCW) {
     // ------------------------------------------------------------ producer

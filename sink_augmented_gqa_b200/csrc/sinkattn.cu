@@ -415,9 +415,21 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
     set_smem(sa::decode_kernel<D, F8>, Cfg::SMEM_BYTES);
     configured = true;
   }
-  dim3 grid(c->n_kv, p.S, a->B);
-  sa::decode_kernel<D, F8><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmK, tmV, tmKS, tmVS, p);
-  return last_launch_status();
+  // Programmatic stream serialization: back-to-back decode launches (one per
+  // layer) overlap one kernel's drain with the next one's launch and set-up;
+  // the kernel waits for its predecessor before touching global memory.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(c->n_kv, p.S, a->B);
+  lc.blockDim = dim3(Cfg::NUM_THREADS);
+  lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  lc.stream = stream;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&lc, sa::decode_kernel<D, F8>, tmK, tmV, tmKS, tmVS, p);
+  return (last_launch_status() == SA_OK && e == cudaSuccess) ? SA_OK : SA_ERR_CUDA;
 }
 
 sa_status launch_append(sa_kv_cache* c, const void* k, const int64_t ks[3], const void* v,
@@ -566,9 +578,12 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
   p.window = a->window;
   p.scale = a->sm_scale;
   p.scale_log2 = a->sm_scale * 1.4426950408889634f;
+  // one CTA per 128-row tile, per head of either pass, per sequence (a 1-D grid)
+  const long long ctas = (long long)((a->T + 127) / 128) * (a->n_kv + a->n_q) * a->B;
+  if (ctas > 0x7fffffffLL || a->n_q > 8192) return SA_ERR_SHAPE;   // (the row pass sums n_q floats in smem)
   if (p.dsinks && cudaMemsetAsync(p.dsinks, 0, sizeof(float) * a->n_q, stream) != cudaSuccess) return SA_ERR_CUDA;
   const long long rows = (long long)a->B * p.Tp * a->n_q;
-  sa::bwd_rows_kernel<D><<<grid_for(rows * 32), 256, 0, stream>>>(p);
+  sa::bwd_rows_kernel<D><<<grid_for(rows * 32), 256, (size_t)a->n_q * sizeof(float), stream>>>(p);
   using C0 = sa::BtcCfg<D, 0>;
   using C1 = sa::BtcCfg<D, 1>;
   // dQ pass: resident Q, dO (128 rows); streamed K, V (BN rows).
@@ -583,15 +598,14 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
       !make_rows_map(&q1, a->q, D, a->T, a->n_q, a->B, a->q_strides, C1::CB, C1::BN) ||
       !make_rows_map(&o1, a->d_out, D, a->T, a->n_q, a->B, a->d_out_strides, C1::CB, C1::BN))
     return SA_ERR_CUDA;
+  static_assert(C0::NUM_THREADS == C1::NUM_THREADS, "both passes share one launch");
+  constexpr uint32_t smem = C0::SMEM_BYTES > C1::SMEM_BYTES ? C0::SMEM_BYTES : C1::SMEM_BYTES;
   static bool configured = false;
   if (!configured) {
-    set_smem(sa::bwd_tc_kernel<D, 0>, C0::SMEM_BYTES);
-    set_smem(sa::bwd_tc_kernel<D, 1>, C1::SMEM_BYTES);
+    set_smem(sa::bwd_tc_kernel<D>, smem);
     configured = true;
   }
-  const int tiles = (a->T + 127) / 128;
-  sa::bwd_tc_kernel<D, 1><<<dim3(tiles, a->n_kv, a->B), C1::NUM_THREADS, C1::SMEM_BYTES, stream>>>(k1, v1, q1, o1, p);
-  sa::bwd_tc_kernel<D, 0><<<dim3(tiles, a->n_q, a->B), C0::NUM_THREADS, C0::SMEM_BYTES, stream>>>(q0, o0, k0, v0, p);
+  sa::bwd_tc_kernel<D><<<(unsigned)ctas, C0::NUM_THREADS, smem, stream>>>(k1, v1, q1, o1, q0, o0, k0, v0, p);
   return last_launch_status();
 }
 
