@@ -41,7 +41,7 @@ struct BwdParams {
 };
 
 // D_i = <dO_i, o_i> and lse_i log2(e) per (b, i, h) into the padded
-// workspace rows, one warp per row; each row also adds -exp(sink_h - lse_i) D_i
+// workspace rows, one warp per four rows; each row also adds -exp(sink_h - lse_i) D_i
 // to dsinks[h], through a per-block sum in shared memory (dynamic, n_q
 // floats) so that global memory sees one atomic per block and head. Rows
 // T..Tp-1 get the values of an empty row (D 0, lse +inf).
@@ -55,30 +55,50 @@ __global__ void bwd_rows_kernel(const BwdParams p) {
   const int lane = threadIdx.x & 31;
   const long long rows = (long long)p.B * p.Tp * p.n_q;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-  for (long long r = blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5); r < rows; r += warps) {
-    const int h = (int)(r % p.n_q);
-    const int i = (int)((r / p.n_q) % p.Tp);
-    const int b = (int)(r / ((long long)p.n_q * p.Tp));
-    const long long wi = ((long long)b * p.n_q + h) * p.Tp + i;
-    if (i >= p.T) {
-      if (lane == 0) {
-        p.dvec[wi] = 0.f;
-        p.lse2[wi] = INFINITY;
+  // NR rows per warp and pass, their loads issued before any reduction (rows
+  // h, h + 1, ... of one (b, i) are adjacent in o and dO)
+  constexpr int NR = 4;
+  for (long long r0 = (blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5)) * NR; r0 < rows;
+       r0 += warps * NR) {
+    float acc[NR];
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+      const long long r = r0 + j;
+      const int h = (int)(r % p.n_q);
+      const int i = (int)((r / p.n_q) % p.Tp);
+      const int b = (int)(r / ((long long)p.n_q * p.Tp));
+      acc[j] = 0.f;
+      if (r < rows && i < p.T) {
+        const __nv_bfloat16* orow = p.o + b * p.os0 + i * p.os1 + h * p.os2;
+        const __nv_bfloat16* drow = p.dout + b * p.ds0 + i * p.ds1 + h * p.ds2;
+#pragma unroll
+        for (int c = lane; c < D; c += 32) acc[j] = fmaf(__bfloat162float(orow[c]), __bfloat162float(drow[c]), acc[j]);
       }
-      continue;
     }
-    const __nv_bfloat16* orow = p.o + b * p.os0 + i * p.os1 + h * p.os2;
-    const __nv_bfloat16* drow = p.dout + b * p.ds0 + i * p.ds1 + h * p.ds2;
-    float acc = 0.f;
 #pragma unroll
-    for (int c = lane; c < D; c += 32) acc = fmaf(__bfloat162float(orow[c]), __bfloat162float(drow[c]), acc);
+    for (int j = 0; j < NR; ++j)
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (lane == 0) {
-      const long long li = ((long long)b * p.n_q + h) * p.T + i;
-      p.dvec[wi] = acc;
-      p.lse2[wi] = p.lse[li] * 1.4426950408889634f;
-      if (sink) atomicAdd(dsink_part + h, -expf(p.sinks[h] - p.lse[li]) * acc);
+      for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+    if (lane < NR) {
+      float a = acc[0];
+#pragma unroll
+      for (int j = 1; j < NR; ++j) a = lane == j ? acc[j] : a;
+      const long long r = r0 + lane;
+      if (r < rows) {
+        const int h = (int)(r % p.n_q);
+        const int i = (int)((r / p.n_q) % p.Tp);
+        const int b = (int)(r / ((long long)p.n_q * p.Tp));
+        const long long wi = ((long long)b * p.n_q + h) * p.Tp + i;
+        if (i >= p.T) {
+          p.dvec[wi] = 0.f;
+          p.lse2[wi] = INFINITY;
+        } else {
+          const long long li = ((long long)b * p.n_q + h) * p.T + i;
+          p.dvec[wi] = a;
+          p.lse2[wi] = p.lse[li] * 1.4426950408889634f;
+          if (sink) atomicAdd(dsink_part + h, -expf(p.sinks[h] - p.lse[li]) * a);
+        }
+      }
     }
   }
   if (sink) {

@@ -10,21 +10,24 @@
 //                 dV += P^T dO and dK += dS^T Q.
 //
 // One CTA per 128-row tile (both passes in one launch, heaviest tiles first),
-// 320 threads:
+// 576 threads:
 //   warp 0      TMA loads: the two resident 128-row tiles once, then per
 //               streamed tile its two BN-row tiles into an NS-deep ring (MODE 1
 //               also stages the tile's lse and D values there).
 //   warp 1      one thread issues the MMAs and owns the TMEM allocation. S and
-//               dP are double-buffered in TMEM, and P, dS are written over the
-//               S, dP columns they came from, so a buffer serves one tile from
-//               its S product to its last read (the issuer waits for the
-//               products of tile u - 2 before tile u reuses it): the tensor
-//               core computes the next tile's S, dP while this tile's P, dS are
-//               formed, and nothing waits for the previous tile's products.
-//   warps 2-9   P, dS from S, dP: two warps per TMEM lane quarter (warp % 4),
-//               each taking half of a tile's columns, one row per thread; tiles
-//               wholly inside the admitted region skip the mask; then the fp32
-//               output rows (the two warps of a quarter split the columns).
+//               dP are double-buffered in TMEM: the tensor core computes the
+//               next tile's S, dP while this tile's P, dS are formed. P and dS
+//               (bf16) get a single buffer of their own where TMEM has room
+//               (every case but dK/dV at d = 128): an S / dP buffer is then
+//               free as soon as its values are read, and the P / dS warps
+//               wait for the previous tile's products only before storing.
+//               Otherwise P, dS are written over the S, dP columns they came
+//               from, and the issuer waits for tile u - 2's products before
+//               tile u reuses that buffer.
+//   warps 2-17  P, dS from S, dP: four warps per TMEM lane quarter (warp % 4),
+//               each taking a quarter of a tile's columns, one row per thread;
+//               tiles wholly inside the admitted region skip the mask; then the
+//               fp32 output rows (the warps of a quarter split the columns).
 // P_ij = exp2(s_ij scale_log2 - lse_i log2 e) uses the forward's lse (sink
 // included), so no running max is needed.
 #pragma once
@@ -58,19 +61,29 @@ struct BtcCfg {
   static constexpr uint32_t OFF_BAR = OFF_ROWV + NS * 2 * BN * 4;
   // at least 120 KB: one CTA per SM, since each allocates all 512 TMEM columns
   static constexpr uint32_t SMEM_BYTES = (OFF_BAR + 256 + 1024) > 120u * 1024 ? (OFF_BAR + 256 + 1024) : 120u * 1024;
-  // TMEM columns
-  static constexpr int S_COL = 0;                  // S[buf] at S_COL + buf * BN, then P (bf16 pairs)
-  static constexpr int DP_COL = 2 * BN;            // dP[buf], then dS (bf16 pairs)
-  static constexpr int ACC0 = 4 * BN;              // dQ | dV
+  // TMEM columns. S[buf] at S_COL + buf * BN, dP[buf] at DP_COL + buf * BN.
+  // SEP: P and dS (bf16 pairs, BN / 2 columns each) have columns of their own
+  // after the S / dP buffers, so an S / dP buffer is free again once its
+  // values are read; otherwise (dK and dV of d = 128 leave no room) P and dS
+  // are written over the start of the S / dP columns they came from.
+  static constexpr int S_COL = 0;
+  static constexpr int DP_COL = 2 * BN;
+  static constexpr bool SEP = 5 * BN + (MODE == 0 ? D : 2 * D) <= 512;
+  static constexpr int P_COL = SEP ? 4 * BN : S_COL;                  // MODE 1
+  static constexpr int DS_COL = SEP ? 4 * BN + BN / 2 : DP_COL;
+  static constexpr int ACC0 = SEP ? 5 * BN : 4 * BN;                  // dQ | dV
   static constexpr int ACC1 = ACC0 + D;                              // MODE 1: dK
   static constexpr int TMEM_COLS = 512;
   static_assert((MODE == 0 ? ACC0 + D : ACC1 + D) <= TMEM_COLS, "TMEM plan exceeds 512 columns");
   static_assert(MBLOCK % 1024 == 0 && NBLOCK % 1024 == 0 && M_BYTES % 1024 == 0, "1 KB aligned tiles");
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
   static constexpr uint32_t IDESC_O = idesc_bf16(128, D, 0, 1);
-  static constexpr int NSW = 8;                                      // P / dS warps (2..9)
-  static constexpr int HC = BN / 2;                                  // columns per P / dS warp
+  static constexpr int NSW = 16;                                     // P / dS warps (2..17)
+  static constexpr int NPART = NSW / 4;                              // P / dS warps per TMEM lane quarter
+  static constexpr int HC = BN / NPART;                              // columns per P / dS warp
   static constexpr int NUM_THREADS = 32 * (2 + NSW);
+  static_assert(HC == 16 || HC == 32, "16 or 32 columns per P / dS warp");
+  static_assert(NPART % 2 == 0, "dK and dV epilogues take half the warps of a quarter each");
 };
 
 enum : int {
@@ -97,16 +110,18 @@ __device__ __forceinline__ void btc_issue_s(uint32_t d_tmem, uint64_t adesc, uin
            kk > 0 ? 1u : 0u);
   }
 }
-// acc (+)= A (TMEM bf16, 128 x BN) B (smem [BN][D], MN-major). A's elements
-// [HC h, HC h + HC) sit, as bf16 pairs, at columns [HC h, HC h + HC / 2) of
-// its buffer (each P / dS warp writes over the start of the columns it read).
+// acc (+)= A (TMEM bf16, 128 x BN) B (smem [BN][D], MN-major). SEP: A's
+// elements sit, as bf16 pairs, at columns [0, BN / 2) of their own buffer;
+// otherwise elements [HC h, HC h + HC) sit at columns [HC h, HC h + HC / 2) of
+// the S / dP buffer (each P / dS warp writes over the start of the columns it
+// read).
 template <int D, int MODE>
 __device__ __forceinline__ void btc_issue_o(uint32_t acc_tmem, uint32_t a_tmem, uint64_t bdesc, bool accumulate) {
   using C = BtcCfg<D, MODE>;
 #pragma unroll
   for (int kk = 0; kk < C::BN / 16; ++kk) {
     const int e = kk * 16;                                        // first element of the K-step
-    const uint32_t col = (uint32_t)(C::HC * (e / C::HC) + (e % C::HC) / 2);
+    const uint32_t col = C::SEP ? (uint32_t)(e / 2) : (uint32_t)(C::HC * (e / C::HC) + (e % C::HC) / 2);
     mma_ts(acc_tmem, a_tmem + col, bdesc + ((kk * 16 * C::SWZ) >> 4), C::IDESC_O,
            (accumulate || kk > 0) ? 1u : 0u);
   }
@@ -246,7 +261,8 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
       const uint64_t a1 = smem_desc(sbase + C::OFF_R1, 16, C::SBO, C::LAYOUT);   // dO | V
       auto o_products = [&](int v) {   // the products of tile v that read P / dS
         const int sv = v % C::NS;
-        const uint32_t pcol = tmem + C::S_COL + (v & 1) * BN, dscol = tmem + C::DP_COL + (v & 1) * BN;
+        const uint32_t pcol = tmem + C::P_COL + (C::SEP ? 0 : (v & 1) * BN);
+        const uint32_t dscol = tmem + C::DS_COL + (C::SEP ? 0 : (v & 1) * BN);
         const uint32_t st = sbase + C::OFF_ST + sv * C::STAGE_BYTES;
         if constexpr (MODE == 0) {
           // dQ += dS K (K of the stage, MN-major)
@@ -263,8 +279,10 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
       for (int u = 0; u < n_tiles && ok; ++u) {
         const int s = u % C::NS, x = u & 1;
         if (!mbar_wait(bar(BB_FULL + s), (uint32_t)((u / C::NS) & 1))) { ok = false; break; }
-        // buffer x last served tile u - 2: its products have read P / dS
-        if (u >= 2 && !mbar_wait(bar(BB_PDONE), (uint32_t)((u - 2) & 1))) { ok = false; break; }
+        // buffer x last served tile u - 2. SEP: its S / dP were read before
+        // tile u - 2's P / dS were signalled (waited for below, one tile ago);
+        // otherwise wait until the products reading its P / dS completed.
+        if (!C::SEP && u >= 2 && !mbar_wait(bar(BB_PDONE), (uint32_t)((u - 2) & 1))) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_BYTES;
         // S = R0 S0^T, dP = R1 S1^T (both K-major)
@@ -297,7 +315,7 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
     // ------------------------------------------------------------ dS and the epilogue
     constexpr int HC = C::HC;
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;                    // which half of the columns
+    const int part = (warp - 2) >> 2;                    // which HC columns of the tile
     const int rr = quarter * 32 + lane;                  // resident row of this thread
     const int row = r0 + rr;                              // query (MODE 0) or key (MODE 1)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -322,7 +340,7 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
       tc_fence_after();
       int hh, s0;
       stream_of(u, hh, s0);
-      const int c_base = half * HC;                       // this warp's first column of the tile
+      const int c_base = part * HC;                       // this warp's first column of the tile
       const float* rv = reinterpret_cast<const float*>(smem + C::OFF_ROWV) + (u % C::NS) * 2 * BN;
       if constexpr (MODE == 1) {
         // the producer's lse / D values of this stage: acquire them on the
@@ -392,11 +410,26 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
         if constexpr (MODE == 1) pk[c / 2] = pack_bf16(p0, p1);
         dk[c / 2] = pack_bf16(t0, t1);
       }
-      // P / dS over the start of the S / dP columns this warp read (the
-      // other warp of the quarter reads and writes only its own columns)
-      static_assert(HC == 32, "one 32-column chunk per P / dS warp");
-      tmem_st16(tmem + lane_base + C::DP_COL + x * BN + c_base, dk);
-      if constexpr (MODE == 1) tmem_st16(tmem + lane_base + C::S_COL + x * BN + c_base, pk);
+      uint32_t ps_off;
+      if constexpr (C::SEP) {
+        // the single P / dS buffer: the previous tile's products must have
+        // read it (their completion is at most one phase behind here: the
+        // S / dP this warp just read were committed after them)
+        if (u >= 1 && !wait_all(bar(BB_PDONE), (uint32_t)((u - 1) & 1))) { ok = false; break; }
+        tc_fence_after();
+        ps_off = (uint32_t)(part * (HC / 2));
+      } else {
+        // over the start of the S / dP columns this warp read (the other
+        // warps of the quarter read and write only their own columns)
+        ps_off = (uint32_t)(x * BN + c_base);
+      }
+      if constexpr (HC == 32) {
+        tmem_st16(tmem + lane_base + C::DS_COL + ps_off, dk);
+        if constexpr (MODE == 1) tmem_st16(tmem + lane_base + C::P_COL + ps_off, pk);
+      } else {
+        tmem_st8(tmem + lane_base + C::DS_COL + ps_off, dk);
+        if constexpr (MODE == 1) tmem_st8(tmem + lane_base + C::P_COL + ps_off, pk);
+      }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -404,9 +437,9 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
       if (*abort_flag) { ok = false; break; }
     }
     // epilogue: the accumulators (zero when no tile was admitted) -> fp32
-    // rows. MODE 0: the two warps of a quarter take alternate 32-column
-    // chunks of dQ; MODE 1: one takes dV, the other dK. Every lane takes
-    // part in the TMEM loads; rows past T store nothing.
+    // rows. MODE 0: the NPART warps of a quarter take 32-column chunks of dQ
+    // in turn; MODE 1: half of them take dV, the other half dK, in turn.
+    // Every lane takes part in the TMEM loads; rows past T store nothing.
     const bool have = n_tiles > 0;
     if (ok && have) {
       if (!wait_all(bar(BB_ACCFULL), 0)) ok = false;
@@ -421,13 +454,15 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
         mul = p.scale;
         acc = C::ACC0;
       } else {
-        dst = (half == 0 ? p.dv : p.dk) + (((long long)b * p.T + row) * p.n_kv + head) * D;
-        mul = half == 0 ? 1.0f : p.scale;
-        acc = half == 0 ? C::ACC0 : C::ACC1;
+        const bool is_dv = part < C::NPART / 2;
+        dst = (is_dv ? p.dv : p.dk) + (((long long)b * p.T + row) * p.n_kv + head) * D;
+        mul = is_dv ? 1.0f : p.scale;
+        acc = is_dv ? C::ACC0 : C::ACC1;
       }
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
-        if (MODE == 0 && ((c0 / 32) & 1) != half) continue;
+        if (MODE == 0 && (c0 / 32) % C::NPART != part) continue;
+        if (MODE == 1 && (c0 / 32) % (C::NPART / 2) != part % (C::NPART / 2)) continue;
         uint32_t a32[32];
         if (have) {
           tmem_ld32(tmem + lane_base + acc + c0, a32);
@@ -463,7 +498,7 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
 // the n_q B dQ CTAs of query tile tiles - 1 - k; under a causal mask both
 // shrink with k, so the heaviest CTAs start first.
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(BtcCfg<D, 0>::NUM_THREADS, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap k1, const __grid_constant__ CUtensorMap v1,
                   const __grid_constant__ CUtensorMap q1, const __grid_constant__ CUtensorMap o1,
                   const __grid_constant__ CUtensorMap q0, const __grid_constant__ CUtensorMap o0,
