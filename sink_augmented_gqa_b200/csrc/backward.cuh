@@ -56,48 +56,74 @@ __global__ void bwd_rows_kernel(const BwdParams p) {
   const long long rows = (long long)p.B * p.Tp * p.n_q;
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   // NR rows per warp and pass, their loads issued before any reduction (rows
-  // h, h + 1, ... of one (b, i) are adjacent in o and dO)
+  // h, h + 1, ... of one (b, i) are adjacent in o and dO). Row r is (b, i, h)
+  // with h fastest; one division per pass (32-bit when the rows allow), the
+  // following rows by stepping h.
   constexpr int NR = 4;
+  auto split = [&](long long r, int& b, int& i, int& h) {
+    if (rows <= 0xffffffffLL) {
+      const uint32_t ru = (uint32_t)r, t = ru / (uint32_t)p.n_q;
+      h = (int)(ru - t * (uint32_t)p.n_q);
+      i = (int)(t % (uint32_t)p.Tp);
+      b = (int)(t / (uint32_t)p.Tp);
+    } else {
+      const long long t = r / p.n_q;
+      h = (int)(r - t * p.n_q);
+      i = (int)(t % p.Tp);
+      b = (int)(t / p.Tp);
+    }
+  };
+  auto step = [&](int& b, int& i, int& h) {
+    if (++h == p.n_q) {
+      h = 0;
+      if (++i == p.Tp) {
+        i = 0;
+        ++b;
+      }
+    }
+  };
   for (long long r0 = (blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5)) * NR; r0 < rows;
        r0 += warps * NR) {
+    int b0, i0, h0;
+    split(r0, b0, i0, h0);
     float acc[NR];
+    {
+      int b = b0, i = i0, h = h0;
 #pragma unroll
-    for (int j = 0; j < NR; ++j) {
-      const long long r = r0 + j;
-      const int h = (int)(r % p.n_q);
-      const int i = (int)((r / p.n_q) % p.Tp);
-      const int b = (int)(r / ((long long)p.n_q * p.Tp));
-      acc[j] = 0.f;
-      if (r < rows && i < p.T) {
-        const __nv_bfloat16* orow = p.o + b * p.os0 + i * p.os1 + h * p.os2;
-        const __nv_bfloat16* drow = p.dout + b * p.ds0 + i * p.ds1 + h * p.ds2;
+      for (int j = 0; j < NR; ++j) {
+        acc[j] = 0.f;
+        if (r0 + j < rows && i < p.T) {
+          const __nv_bfloat16* orow = p.o + b * p.os0 + i * p.os1 + h * p.os2;
+          const __nv_bfloat16* drow = p.dout + b * p.ds0 + i * p.ds1 + h * p.ds2;
 #pragma unroll
-        for (int c = lane; c < D; c += 32) acc[j] = fmaf(__bfloat162float(orow[c]), __bfloat162float(drow[c]), acc[j]);
+          for (int c = lane; c < D; c += 32) acc[j] = fmaf(__bfloat162float(orow[c]), __bfloat162float(drow[c]), acc[j]);
+        }
+        step(b, i, h);
       }
     }
 #pragma unroll
     for (int j = 0; j < NR; ++j)
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
-    if (lane < NR) {
+    if (lane < NR && r0 + lane < rows) {
       float a = acc[0];
+      int b = b0, i = i0, h = h0;
 #pragma unroll
-      for (int j = 1; j < NR; ++j) a = lane == j ? acc[j] : a;
-      const long long r = r0 + lane;
-      if (r < rows) {
-        const int h = (int)(r % p.n_q);
-        const int i = (int)((r / p.n_q) % p.Tp);
-        const int b = (int)(r / ((long long)p.n_q * p.Tp));
-        const long long wi = ((long long)b * p.n_q + h) * p.Tp + i;
-        if (i >= p.T) {
-          p.dvec[wi] = 0.f;
-          p.lse2[wi] = INFINITY;
-        } else {
-          const long long li = ((long long)b * p.n_q + h) * p.T + i;
-          p.dvec[wi] = a;
-          p.lse2[wi] = p.lse[li] * 1.4426950408889634f;
-          if (sink) atomicAdd(dsink_part + h, -expf(p.sinks[h] - p.lse[li]) * a);
+      for (int j = 1; j < NR; ++j) {
+        if (lane >= j) {
+          a = acc[j];
+          step(b, i, h);
         }
+      }
+      const long long wi = ((long long)b * p.n_q + h) * p.Tp + i;
+      if (i >= p.T) {
+        p.dvec[wi] = 0.f;
+        p.lse2[wi] = INFINITY;
+      } else {
+        const long long li = ((long long)b * p.n_q + h) * p.T + i;
+        p.dvec[wi] = a;
+        p.lse2[wi] = p.lse[li] * 1.4426950408889634f;
+        if (sink) atomicAdd(dsink_part + h, -expf(p.sinks[h] - p.lse[li]) * a);
       }
     }
   }

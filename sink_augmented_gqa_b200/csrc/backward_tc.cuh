@@ -92,7 +92,8 @@ enum : int {
   BB_EMPTY = 5,      // [4] ring stage free (MMA commit)
   BB_SFULL = 9,      // [2] S, dP of a buffer computed
   BB_PFULL = 13,     // count 8 warps: P / dS stored in TMEM
-  BB_PDONE = 14,     // the products reading P / dS completed
+  // 14: unused (the products that read P / dS signal on the stage's EMPTY
+  // barrier, which the P / dS warps wait on as well: one commit fewer per tile)
   BB_ACCFULL = 15,   // accumulators final
   BB_DRAIN = 16,
   BB_TMEM_SLOT = 17,
@@ -183,7 +184,6 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
     }
     for (int x = 0; x < 2; ++x) mbar_init(bar(BB_SFULL + x), 1);
     mbar_init(bar(BB_PFULL), C::NSW);
-    mbar_init(bar(BB_PDONE), 1);
     mbar_init(bar(BB_ACCFULL), 1);
     mbar_init(bar(BB_DRAIN), 1);
     *abort_flag = 0;
@@ -273,8 +273,7 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
                                v > 0);
           btc_issue_o<D, MODE>(tmem + C::ACC1, dscol, smem_desc(st, C::NBLOCK, C::SBO, C::LAYOUT), v > 0);
         }
-        mma_commit(bar(BB_PDONE));
-        mma_commit(bar(BB_EMPTY + sv));
+        mma_commit(bar(BB_EMPTY + sv));   // also: tile v's P / dS have been read
       };
       for (int u = 0; u < n_tiles && ok; ++u) {
         const int s = u % C::NS, x = u & 1;
@@ -282,7 +281,11 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
         // buffer x last served tile u - 2. SEP: its S / dP were read before
         // tile u - 2's P / dS were signalled (waited for below, one tile ago);
         // otherwise wait until the products reading its P / dS completed.
-        if (!C::SEP && u >= 2 && !mbar_wait(bar(BB_PDONE), (uint32_t)((u - 2) & 1))) { ok = false; break; }
+        if (!C::SEP && u >= 2 &&
+            !mbar_wait(bar(BB_EMPTY + (u - 2) % C::NS), (uint32_t)(((u - 2) / C::NS) & 1))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_BYTES;
         // S = R0 S0^T, dP = R1 S1^T (both K-major)
@@ -413,9 +416,14 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
       uint32_t ps_off;
       if constexpr (C::SEP) {
         // the single P / dS buffer: the previous tile's products must have
-        // read it (their completion is at most one phase behind here: the
-        // S / dP this warp just read were committed after them)
-        if (u >= 1 && !wait_all(bar(BB_PDONE), (uint32_t)((u - 1) & 1))) { ok = false; break; }
+        // read it. They signal its stage's EMPTY barrier; that barrier's
+        // earlier phase (NS tiles back) is complete here, since the S / dP
+        // this warp just read were committed after those products, and its
+        // next phase needs this tile's P / dS first.
+        if (u >= 1 && !wait_all(bar(BB_EMPTY + (u - 1) % C::NS), (uint32_t)(((u - 1) / C::NS) & 1))) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         ps_off = (uint32_t)(part * (HC / 2));
       } else {

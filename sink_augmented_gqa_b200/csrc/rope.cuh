@@ -7,6 +7,28 @@
 
 namespace sa {
 
+// x = ((b T + t) H + h) chunks + ch  ->  (b, t, h, ch), with 32-bit
+// divisions whenever the index range allows (narrow): a 64-bit division is a
+// long software sequence, and three of them per 16 elements made these
+// kernels issue-bound.
+__device__ __forceinline__ void split_row_chunk(long long x, bool narrow, int chunks, int H, int T, int& b,
+                                                int& t, int& h, int& ch) {
+  if (narrow) {
+    const uint32_t u = (uint32_t)x;
+    const uint32_t q1 = u / (uint32_t)chunks, q2 = q1 / (uint32_t)H, q3 = q2 / (uint32_t)T;
+    ch = (int)(u - q1 * (uint32_t)chunks);
+    h = (int)(q1 - q2 * (uint32_t)H);
+    t = (int)(q2 - q3 * (uint32_t)T);
+    b = (int)q3;
+  } else {
+    const long long q1 = x / chunks, q2 = q1 / H, q3 = q2 / T;
+    ch = (int)(x - q1 * chunks);
+    h = (int)(q1 - q2 * H);
+    t = (int)(q2 - q3 * T);
+    b = (int)q3;
+  }
+}
+
 // cos/sin[t][i] = conc * cos/sin(t * inv_freq[i]) per the YaRN + NTK-by-parts
 // recipe of the MoE-Xtend README, "ROPE + SCALING": geometric base
 // frequencies, extrapolation / interpolation blend through a linear ramp
@@ -62,14 +84,11 @@ __global__ void rope_inplace_kernel(__nv_bfloat16* __restrict__ x, long long s0,
                                     const float* __restrict__ sin_t) {
   const int half = d / 2, chunks = half / 8;
   const long long n = (long long)B * T * H * chunks;
+  const bool narrow = n <= 0xffffffffLL;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
        idx += (long long)gridDim.x * blockDim.x) {
-    const int ch = (int)(idx % chunks);
-    long long r = idx / chunks;
-    const int h = (int)(r % H);
-    r /= H;
-    const int t = (int)(r % T);
-    const int b = (int)(r / T);
+    int b, t, h, ch;
+    split_row_chunk(idx, narrow, chunks, H, T, b, t, h, ch);
     __nv_bfloat16* row = x + b * s0 + t * s1 + h * s2;
     uint4 a = *reinterpret_cast<const uint4*>(row + ch * 8);
     uint4 c = *reinterpret_cast<const uint4*>(row + half + ch * 8);
@@ -91,14 +110,11 @@ __global__ void kv_append_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat16* 
                                  const float* __restrict__ sin_t, int ring) {
   const int half = d / 2, chunks = half / 8;
   const long long n = (long long)B * T * n_kv * chunks;
+  const bool narrow = n <= 0xffffffffLL;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
        idx += (long long)gridDim.x * blockDim.x) {
-    const int ch = (int)(idx % chunks);
-    long long r = idx / chunks;
-    const int g = (int)(r % n_kv);
-    r /= n_kv;
-    const int t = (int)(r % T);
-    const int b = (int)(r / T);
+    int b, t, g, ch;
+    split_row_chunk(idx, narrow, chunks, n_kv, T, b, t, g, ch);
     const __nv_bfloat16* krow = k + b * ks0 + t * ks1 + g * ks2;
     const __nv_bfloat16* vrow = v + b * vs0 + t * vs1 + g * vs2;
     uint4 a = *reinterpret_cast<const uint4*>(krow + ch * 8);
@@ -132,15 +148,12 @@ __global__ void prefill_stage_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat
   const int half = d / 2, chunks = half / 8;
   const long long n_kv_units = (long long)B * T * n_kv * chunks;
   const long long n = n_kv_units + (stage_q ? (long long)B * T * n_q * chunks : 0);
+  const bool narrow = n <= 0xffffffffLL;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
        idx += (long long)gridDim.x * blockDim.x) {
     if (idx < n_kv_units) {
-      const int ch = (int)(idx % chunks);
-      long long r = idx / chunks;
-      const int g = (int)(r % n_kv);
-      r /= n_kv;
-      const int t = (int)(r % T);
-      const int b = (int)(r / T);
+      int b, t, g, ch;
+      split_row_chunk(idx, narrow, chunks, n_kv, T, b, t, g, ch);
       const __nv_bfloat16* krow = k + b * ks0 + t * ks1 + g * ks2;
       const __nv_bfloat16* vrow = v + b * vs0 + t * vs1 + g * vs2;
       uint4 a = *reinterpret_cast<const uint4*>(krow + ch * 8);
@@ -155,12 +168,8 @@ __global__ void prefill_stage_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat
           *reinterpret_cast<const uint4*>(vrow + half + ch * 8);
     } else {
       const long long iq = idx - n_kv_units;
-      const int ch = (int)(iq % chunks);
-      long long r = iq / chunks;
-      const int h = (int)(r % n_q);
-      r /= n_q;
-      const int t = (int)(r % T);
-      const int b = (int)(r / T);
+      int b, t, h, ch;
+      split_row_chunk(iq, narrow, chunks, n_q, T, b, t, h, ch);
       const __nv_bfloat16* qrow = q + b * qs0 + t * qs1 + h * qs2;
       __nv_bfloat16* orow = qo + b * os0 + t * os1 + h * os2;
       uint4 a = *reinterpret_cast<const uint4*>(qrow + ch * 8);
