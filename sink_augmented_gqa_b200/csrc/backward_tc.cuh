@@ -84,6 +84,9 @@ struct BtcCfg {
   static constexpr int NUM_THREADS = 32 * (2 + NSW);
   static_assert(HC == 16 || HC == 32, "16 or 32 columns per P / dS warp");
   static_assert(NPART % 2 == 0, "dK and dV epilogues take half the warps of a quarter each");
+  // the epilogue's 32 x 33 fp32 staging slot per P / dS warp overlays the
+  // resident tiles and the ring (below the row values)
+  static_assert((uint32_t)NSW * 32 * 33 * 4 <= OFF_ROWV, "epilogue staging overlays tiles and ring");
 };
 
 enum : int {
@@ -454,37 +457,48 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
       tc_fence_after();
     }
     if (ok) {
-      float* dst;
+      float* out;
+      long long rstride;   // elements between consecutive rows of the output
       float mul;
       int acc;
       if constexpr (MODE == 0) {
-        dst = p.dq + (((long long)b * p.T + row) * p.n_q + head) * D;
+        out = p.dq + ((long long)b * p.T * p.n_q + head) * D;
+        rstride = (long long)p.n_q * D;
         mul = p.scale;
         acc = C::ACC0;
       } else {
         const bool is_dv = part < C::NPART / 2;
-        dst = (is_dv ? p.dv : p.dk) + (((long long)b * p.T + row) * p.n_kv + head) * D;
+        out = (is_dv ? p.dv : p.dk) + ((long long)b * p.T * p.n_kv + head) * D;
+        rstride = (long long)p.n_kv * D;
         mul = is_dv ? 1.0f : p.scale;
         acc = is_dv ? C::ACC0 : C::ACC1;
       }
+      // Each 32 x 32 chunk (this warp's 32 rows) is transposed through shared
+      // memory so that every store instruction writes one row's 128 bytes:
+      // a thread-per-row store would scatter 16-byte pieces over 32 rows.
+      // The staging slots overlay the resident tiles and the ring, which
+      // every product has finished reading once ACCFULL has completed (with
+      // no tile there is no such wait: zeros are stored directly).
+      float* stg = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 33);
+      const int qrow0 = r0 + quarter * 32;   // first row of this warp's quarter
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
         if (MODE == 0 && (c0 / 32) % C::NPART != part) continue;
         if (MODE == 1 && (c0 / 32) % (C::NPART / 2) != part % (C::NPART / 2)) continue;
-        uint32_t a32[32];
         if (have) {
+          uint32_t a32[32];
           tmem_ld32(tmem + lane_base + acc + c0, a32);
           tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) stg[lane * 33 + c] = __uint_as_float(a32[c]) * mul;
+          __syncwarp();
+#pragma unroll 4
+          for (int r = 0; r < 32; ++r)
+            if (qrow0 + r < p.T) out[(long long)(qrow0 + r) * rstride + c0 + lane] = stg[r * 33 + lane];
+          __syncwarp();
         } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) a32[c] = 0u;
-        }
-        if (row < p.T) {
-#pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            *reinterpret_cast<float4*>(dst + c0 + c) =
-                make_float4(__uint_as_float(a32[c]) * mul, __uint_as_float(a32[c + 1]) * mul,
-                            __uint_as_float(a32[c + 2]) * mul, __uint_as_float(a32[c + 3]) * mul);
+          for (int r = 0; r < 32; ++r)
+            if (qrow0 + r < p.T) out[(long long)(qrow0 + r) * rstride + c0 + lane] = 0.f;
         }
       }
     }
