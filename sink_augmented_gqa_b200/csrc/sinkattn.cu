@@ -578,9 +578,6 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
   p.window = a->window;
   p.scale = a->sm_scale;
   p.scale_log2 = a->sm_scale * 1.4426950408889634f;
-  // one CTA per 128-row tile, per head of either pass, per sequence (a 1-D grid)
-  const long long ctas = (long long)((a->T + 127) / 128) * (a->n_kv + a->n_q) * a->B;
-  if (ctas > 0x7fffffffLL || a->n_q > 8192) return SA_ERR_SHAPE;   // (the row pass sums n_q floats in smem)
   if (p.dsinks && cudaMemsetAsync(p.dsinks, 0, sizeof(float) * a->n_q, stream) != cudaSuccess) return SA_ERR_CUDA;
   const long long rows = (long long)a->B * p.Tp * a->n_q;
   sa::bwd_rows_kernel<D><<<grid_for(rows * 32), 256, (size_t)a->n_q * sizeof(float), stream>>>(p);
@@ -605,7 +602,9 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
     set_smem(sa::bwd_tc_kernel<D>, smem);
     configured = true;
   }
-  sa::bwd_tc_kernel<D><<<(unsigned)ctas, C0::NUM_THREADS, smem, stream>>>(k1, v1, q1, o1, q0, o0, k0, v0, p);
+  // one CTA per 128-row tile, per head of either pass, per sequence (< 2^31: checked by the caller)
+  const unsigned ctas = (unsigned)((a->T + 127) / 128) * (unsigned)(a->n_kv + a->n_q) * (unsigned)a->B;
+  sa::bwd_tc_kernel<D><<<ctas, C0::NUM_THREADS, smem, stream>>>(k1, v1, q1, o1, q0, o0, k0, v0, p);
   return last_launch_status();
 }
 
@@ -877,6 +876,10 @@ sa_status sa_attn_backward(const sa_attn_bwd_args* a, void* workspace, size_t wo
   if (a == nullptr || a->B < 1 || a->T < 1 || a->n_q < 1 || a->n_kv < 1) return SA_ERR_INVALID_ARG;
   if (!head_dim_ok(a->d)) return SA_ERR_SHAPE;
   if (a->n_q % a->n_kv != 0) return SA_ERR_SHAPE;
+  // the row pass sums n_q floats in shared memory; the products launch one CTA
+  // per 128-row tile, per head of either pass, per sequence (a 1-D grid)
+  const long long ctas = (long long)((a->T + 127) / 128) * (a->n_kv + a->n_q) * a->B;
+  if (a->n_q > 8192 || ctas > 0x7fffffffLL) return SA_ERR_SHAPE;
   const void* ins[5] = {a->q, a->k, a->v, a->out, a->d_out};
   const int64_t* st[5] = {a->q_strides, a->k_strides, a->v_strides, a->out_strides, a->d_out_strides};
   for (int i = 0; i < 5; ++i)

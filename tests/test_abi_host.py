@@ -188,3 +188,37 @@ def test_fp8_cache_host_rules(L):
     b, _ = _fake_cache()
     b.kv_dtype = 7
     assert L.sa_kv_snapshot(ctypes.byref(b), ctypes.byref(S._Snapshot())) == 1
+
+
+def _bwd_args(**kw):
+    p = 0x40000   # 16-byte aligned; never dereferenced: every case below fails validation
+    a = S._BwdArgs()
+    for name in ("q", "k", "v", "out", "d_out"):
+        setattr(a, name, p)
+        setattr(a, name + "_strides", S._I64x3(4096, 256, 64))
+    a.lse = a.dq = a.dk = a.dv = a.dsinks = p
+    a.sinks = None
+    a.B, a.T, a.n_q, a.n_kv, a.d, a.window, a.sm_scale = 1, 16, 4, 2, 64, 0, 0.125
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_backward_argument_errors_return_before_launch(L):
+    codes = {v: k for k, v in S.STATUS.items()}
+    ws = ctypes.c_void_p(0x80000)
+    need = L.sa_attn_backward_workspace_size(1, 16, 4)
+    assert need >= 2 * 64 * 4 * 4                                   # D and lse rows padded to 64
+    assert L.sa_attn_backward_workspace_size(0, 16, 4) == 0
+
+    def call(a, nbytes=need):
+        return L.sa_attn_backward(ctypes.byref(a), ws, nbytes, None)
+    assert call(_bwd_args(B=0)) == codes["SA_ERR_INVALID_ARG"]
+    assert call(_bwd_args(d=80)) == codes["SA_ERR_SHAPE"]
+    assert call(_bwd_args(n_kv=3)) == codes["SA_ERR_SHAPE"]           # 4 % 3
+    assert call(_bwd_args(n_q=8200, n_kv=8200)) == codes["SA_ERR_SHAPE"]  # row pass sums n_q floats in smem
+    assert call(_bwd_args(sm_scale=0.0)) == codes["SA_ERR_INVALID_ARG"]
+    a = _bwd_args()
+    a.q_strides = S._I64x3(4096, 256, 60)                             # misaligned head stride
+    assert call(a) == codes["SA_ERR_INVALID_ARG"]
+    assert call(_bwd_args(), nbytes=need - 256) == codes["SA_ERR_WORKSPACE"]
