@@ -197,7 +197,7 @@ def test_attention_layer_composition(cuda_device):
     xr = x.to(DEV).clone()
     sa.out_proj(o.view(T, n_q * d), wo.to(DEV), bo.to(DEV), xr)
     torch.cuda.synchronize()
-    # oracle, fed the library's own bf16 intermediates so each stage is judged alone
+    # oracle, fed the library's own bf16 intermediates so each stage is checked on its own
     ref_qkv = olin.qkv_proj(to64(x), to64(gamma), 1e-5, to64(wqkv), to64(bqkv))
     s_abs = np.abs(olin.rmsnorm(to64(x), to64(gamma), 1e-5)) @ np.abs(to64(wqkv)).T
     _check(qkv, ref_qkv, s_abs, 2.0 ** -9 + 2.0 ** -12, "layer: qkv")
