@@ -245,6 +245,20 @@ void set_smem(K kernel, uint32_t bytes) {
   cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+// The shared-memory opt-in once per kernel and device (the attribute holds
+// per device): `done` has one bit per device ordinal below 64; devices above
+// that set it on every call, which is harmless. Safe to call from several
+// host threads (setting the attribute twice is harmless too).
+template <typename K>
+void set_smem_once(K kernel, uint32_t bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return;
+  set_smem(kernel, bytes);
+  if (bit != 0) done.fetch_or(bit, std::memory_order_release);
+}
+
 template <int D>
 sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream_t stream) {
   using Cfg = PrefillCfg<D>;
@@ -294,11 +308,8 @@ sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream
   // launches may be in flight at once on one device.
   static std::atomic<unsigned> sched_seq{0};
   p.sched_slot = (int)(sched_seq.fetch_add(1, std::memory_order_relaxed) % sa::kPrefillSchedSlots);
-  static bool configured = false;
-  if (!configured) {
-    set_smem(sa::prefill_kernel<D>, Cfg::SMEM_BYTES);
-    configured = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  set_smem_once(sa::prefill_kernel<D>, Cfg::SMEM_BYTES, smem_set);
   // persistent: one CTA per SM (or per item when there are fewer)
   const long long n_items = (long long)p.n_pairs * a->n_q * a->B;
   const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
@@ -410,11 +421,8 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   p.ws_o = reinterpret_cast<float*>(w + cnt);
   p.ws_m = reinterpret_cast<float*>(w + cnt + rows * D * 4);
   p.ws_l = reinterpret_cast<float*>(w + cnt + rows * D * 4 + rows * 4);
-  static bool configured = false;
-  if (!configured) {
-    set_smem(sa::decode_kernel<D, F8>, Cfg::SMEM_BYTES);
-    configured = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  set_smem_once(sa::decode_kernel<D, F8>, Cfg::SMEM_BYTES, smem_set);
   // Programmatic stream serialization: back-to-back decode launches (one per
   // layer) overlap one kernel's drain with the next one's launch and set-up;
   // the kernel waits for its predecessor before touching global memory.
@@ -528,11 +536,8 @@ sa_status launch_gemm_bn(const void* a, int64_t lda, const void* w, int64_t ldw,
   p.tiles_n = (N + C::BN - 1) / C::BN;
   const long long tiles = (long long)p.tiles_m * p.tiles_n;
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  static bool configured = false;
-  if (!configured) {
-    set_smem(sa::gemm_kernel<BN>, C::SMEM_BYTES);
-    configured = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  set_smem_once(sa::gemm_kernel<BN>, C::SMEM_BYTES, smem_set);
   sa::gemm_kernel<BN><<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tmA, tmB, tmC, p);
   return last_launch_status();
 }
@@ -598,11 +603,8 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
     return SA_ERR_CUDA;
   static_assert(C0::NUM_THREADS == C1::NUM_THREADS, "both passes share one launch");
   constexpr uint32_t smem = C0::SMEM_BYTES > C1::SMEM_BYTES ? C0::SMEM_BYTES : C1::SMEM_BYTES;
-  static bool configured = false;
-  if (!configured) {
-    set_smem(sa::bwd_tc_kernel<D>, smem);
-    configured = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  set_smem_once(sa::bwd_tc_kernel<D>, smem, smem_set);
   // one CTA per 128-row tile, per head of either pass, per sequence (< 2^31: checked by the caller)
   const unsigned ctas = (unsigned)((a->T + 127) / 128) * (unsigned)(a->n_kv + a->n_q) * (unsigned)a->B;
   sa::bwd_tc_kernel<D><<<ctas, C0::NUM_THREADS, smem, stream>>>(k1, v1, q1, o1, q0, o0, k0, v0, p);
