@@ -1,19 +1,26 @@
 """Benchmark of the sink-augmented GQA hot path on B200.
 
-One step = the whole hot path over one batch of the GPT-OSS-Lite attention
-workload (B=8, T=4096, 8 query / 4 KV heads of width 96, YaRN to 131072 from
-4096): build the YaRN tables, then for one layer pair -- even layer with the
-128-key band, odd layer full causal -- snapshot the cache, prefill 4096 rows
-(RoPE, append, attention with the sink column), decode one row (the
-prefill -> decode handoff), and restore the snapshot.
+Workload (the largest configuration, the prefill-to-decode handoff): 16
+sequences share a cache already filled to offset 65,536 (random bf16 rows
+standing for a rotated prefix), n_q = 64, n_kv = 8, d = 64, sm_scale = 1/8,
+YaRN theta = 150000, s = 32 from 4096. One step = the whole hot path over one
+batch: build the YaRN tables; for a layer pair -- even layer with the 128-key
+band, odd layer full causal -- restore the snapshot at offset 65,536 and
+prefill a 512-row chunk per sequence (RoPE, append, attention with the sink
+column); then 32 decode steps, each appending one row per sequence and layer.
 
-value = algorithmic TFLOP/s of the step: F = 4 * d * B * n_q * (admitted
-(query, key) pairs), masked or skipped pairs never counted.
+value = algorithmic TFLOP/s of the step's chunk prefill (both layers, the
+K/V staging launch included): F = 4 * d * B * n_q * (admitted (query, key)
+pairs), masked or skipped pairs never counted, divided by the prefill phase's
+device time (CUDA events on the launch stream inside the timed steps). The
+other half of the metric, decode KV GB/s (cache bytes the decode steps read
+/ their device time), is reported beside it with its own roofline block.
 
-Also reported on the same line: the roofline of the dominant call (full-layer
-prefill), the gpt-oss prefill (T=8192, 64/8/64, full layer) and the
-131,072-context decode (24 layers, KV GB/s) as secondary measurements, the
-end-to-end number through host buffers, and the oracle timed on host cores.
+Also on the same line: the roofline of the dominant kernel (full-layer chunk
+prefill attention) and of the full-layer decode kernel, the end-to-end
+numbers through host buffers, secondary measurements (gpt-oss and Lite
+prefill, the 131,072-context decode, projections, backward), and the oracle
+timed on host cores.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 (N > 1: launched by torch.distributed.run, one rank per GPU, weak scaling).
@@ -37,7 +44,7 @@ sys.path.insert(0, ROOT)
 from sink_augmented_gqa_b200 import workloads as wl  # noqa: E402
 
 METRIC = "sink-GQA prefill TFLOP/s and decode KV GB/s at 1 B200, % of roofline"
-WORKLOAD = "lite"
+WORKLOAD = "handoff"
 L2_BYTES = 126 * 2 ** 20
 
 
@@ -150,76 +157,185 @@ class Clocks:
 # The GPU arm
 # ---------------------------------------------------------------------------
 
-class LiteStep:
-    """One step of the hot path on the GPT-OSS-Lite workload (device-resident)."""
+def kv_row_bytes(cfg):
+    """K and V bytes of one position of every KV head of one sequence (bf16)."""
+    return cfg.n_kv * cfg.d * 2 * 2
+
+
+def decode_rows(p, window):
+    """Cache rows a decode row at position p reads (its own row included)."""
+    return min(p + 1, window) if window else p + 1
+
+
+def prefill_bytes(cfg, off, T, window):
+    """Algorithmic HBM bytes of one prefill call: q read, out written, the
+    call's k / v rows read and appended to the cache, and the cache rows
+    below `off` that some query admits read once."""
+    B, d = cfg.B, cfg.d
+    qo = 2 * B * T * cfg.n_q * d * 2
+    new = 2 * B * T * kv_row_bytes(cfg)
+    lo = max(0, off - window + 1) if window else 0
+    prefix = B * (off - lo) * kv_row_bytes(cfg)
+    return qo + new + prefix
+
+
+def roofline_frac(tflops, nbytes, seconds, peaks):
+    """Achieved fraction of min(tensor peak, HBM bandwidth x arithmetic
+    intensity): a kernel of low intensity is held to the bandwidth roofline."""
+    ai = tflops * 1e12 * seconds / nbytes                       # flop per byte
+    bound = min(peaks["tf"], peaks["hbm"] * 1e9 * ai / 1e12)   # TFLOP/s
+    return {"AI_flop_per_byte": round(ai, 1), "roofline_TFLOP/s": round(bound, 1),
+            "bound": "tensor" if bound >= peaks["tf"] else "hbm",
+            "frac_of_roofline": round(tflops / bound, 4)}
+
+
+class HandoffStep:
+    """One step of the hot path on the handoff workload (device-resident)."""
 
     def __init__(self, dev, cfg):
         import sink_augmented_gqa_b200 as sa
         self.sa, self.cfg, self.dev = sa, cfg, dev
-        self.max_pos = cfg.T + 1
-        self.cap = cfg.T + 1
+        self.off, self.T, self.n_dec = cfg.offset, cfg.T, cfg.decode_steps
+        self.cap = self.max_pos = cfg.offset + cfg.T + cfg.decode_steps
         y = cfg.yarn
         self.yarn = (y["theta"], y["scaling"], y["orig_ctx"], y["alpha"], y["beta"])
         self.cos = torch.empty((self.max_pos, cfg.d // 2), dtype=torch.float32, device=dev)
         self.sin = torch.empty_like(self.cos)
         self.layers = []
         for layer in range(2):
-            q, k, v = wl.qkv(cfg, cfg.T + 1, layer=layer, device=dev)
+            cache = sa.KVCache(cfg.B, self.cap, cfg.n_kv, cfg.d, device=dev)
+            kp, vp = wl.prefilled_cache_rows(cfg, layer=layer, device=dev)
+            cache.append(kp, vp)      # the already-rotated prefix, rows [0, offset)
+            del kp, vp
+            q, k, v = wl.qkv(cfg, cfg.T, layer=layer, device=dev)
+            dq, dk, dv = wl.qkv(cfg, cfg.decode_steps, layer=layer, step=1, device=dev)
             self.layers.append(dict(
                 window=cfg.layer_window(layer), sinks=wl.sinks(cfg, layer, device=dev),
-                q=q, k=k, v=v, cache=sa.KVCache(cfg.B, self.cap, cfg.n_kv, cfg.d, device=dev),
+                q=q, k=k, v=v, dq=dq, dk=dk, dv=dv, cache=cache, snap=cache.snapshot(),
                 out=torch.empty((cfg.B, cfg.T, cfg.n_q, cfg.d), dtype=torch.bfloat16, device=dev),
-                dec=torch.empty((cfg.B, 1, cfg.n_q, cfg.d), dtype=torch.bfloat16, device=dev),
+                dec=torch.empty((cfg.B, cfg.decode_steps, cfg.n_q, cfg.d), dtype=torch.bfloat16, device=dev),
                 ws=sa.decode_workspace(cfg.B, cfg.n_q, cfg.n_kv, cfg.d, device=dev)))
-        for L in self.layers:
-            L["snap"] = L["cache"].snapshot()
-        T = cfg.T
-        self.flops = sum(flops(cfg, 0, T, L["window"]) + flops(cfg, T, 1, L["window"]) for L in self.layers)
-        self.launches = 1 + 3 * len(self.layers)
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        off, T = self.off, self.T
+        self.prefill_flops = sum(flops(cfg, off, T, L["window"]) for L in self.layers)
+        self.decode_flops = sum(flops(cfg, off + T + st, 1, L["window"])
+                                for L in self.layers for st in range(self.n_dec))
+        self.decode_bytes = sum(cfg.B * decode_rows(off + T + st, L["window"]) * kv_row_bytes(cfg)
+                                for L in self.layers for st in range(self.n_dec))
+        full = [L for L in self.layers if L["window"] == 0][0]
+        self.full_chunk_flops = flops(cfg, off, T, 0)
+        self.full_decode_bytes = [cfg.B * decode_rows(off + T + st, 0) * kv_row_bytes(cfg)
+                                  for st in range(self.n_dec)]
+        self.full = full
+        # launches per step: the tables, then per layer the prefill (staging +
+        # attention) and one decode kernel per step
+        self.launches = 1 + len(self.layers) * (2 + self.n_dec)
 
     def tables(self):
         from sink_augmented_gqa_b200 import sinkattn as S
-        import ctypes
         S._check(S.lib().sa_yarn_rope_tables(S._ptr(self.cos), S._ptr(self.sin), self.max_pos, self.cfg.d,
                                              *[float(x) for x in self.yarn[:2]], int(self.yarn[2]),
                                              float(self.yarn[3]), float(self.yarn[4]), S._stream(self.cos)),
                  "sa_yarn_rope_tables")
 
-    def run(self, ev_full=None, q_in=None, outs=None):
-        sa, cfg, T = self.sa, self.cfg, self.cfg.T
-        self.tables()
-        for li, L in enumerate(self.layers):
-            c = L["cache"]
-            c.restore(L["snap"])
-            q, k, v = (L["q"], L["k"], L["v"]) if q_in is None else q_in[li]
-            out, dec = (L["out"], L["dec"]) if outs is None else outs[li]
-            if ev_full is not None and L["window"] == 0:
-                sa.set_prefill_events(*ev_full)   # around the attention kernel alone
-            sa.attn_prefill(c, q[:, :T], k[:, :T], v[:, :T], L["sinks"], L["window"], cfg.sm_scale,
-                            self.cos, self.sin, out=out)
-            if ev_full is not None and L["window"] == 0:
-                sa.set_prefill_events()
-            sa.attn_decode(c, q[:, T:], k[:, T:], v[:, T:], L["sinks"], L["window"], cfg.sm_scale,
-                           self.cos, self.sin, workspace=L["ws"], out=dec)
+    def prefill_phase_layer(self, li, ins=None, out=None, ev_full=None):
+        """Restore layer li's snapshot (offset 65,536) and prefill its chunk
+        (the tables are built by the first layer's call)."""
+        sa, cfg, L = self.sa, self.cfg, self.layers[li]
+        if li == 0:
+            self.tables()
+        L["cache"].restore(L["snap"])
+        q, k, v = (L["q"], L["k"], L["v"]) if ins is None else ins[:3]
+        out = L["out"] if out is None else out
+        if ev_full is not None and L["window"] == 0:
+            sa.set_prefill_events(*ev_full)   # around the attention kernel alone
+        sa.attn_prefill(L["cache"], q, k, v, L["sinks"], L["window"], cfg.sm_scale, self.cos, self.sin,
+                        out=out)
+        if ev_full is not None and L["window"] == 0:
+            sa.set_prefill_events()
+
+    def prefill_phase(self, ev_full=None):
+        for li in range(len(self.layers)):
+            self.prefill_phase_layer(li, ev_full=ev_full)
+
+    def decode_phase(self, ins=None, outs=None, ev_dec=None, first=0, count=None):
+        sa, cfg = self.sa, self.cfg
+        count = self.n_dec if count is None else count
+        for st in range(first, first + count):
+            for li, L in enumerate(self.layers):
+                dq, dk, dv = (L["dq"], L["dk"], L["dv"]) if ins is None else ins[li][3:]
+                dec = L["dec"] if outs is None else outs[li][1]
+                j = st if ins is None else st - first
+                timed = ev_dec is not None and L["window"] == 0
+                if timed:
+                    ev_dec[st][0].record()
+                sa.attn_decode(L["cache"], dq[:, j:j + 1], dk[:, j:j + 1], dv[:, j:j + 1], L["sinks"],
+                               L["window"], cfg.sm_scale, self.cos, self.sin, workspace=L["ws"],
+                               out=dec[:, j:j + 1])
+                if timed:
+                    ev_dec[st][1].record()
+
+    def run(self, phase_ev=None):
+        if phase_ev is not None:
+            phase_ev[0].record()
+        self.prefill_phase()
+        if phase_ev is not None:
+            phase_ev[1].record()
+        self.decode_phase()
+        if phase_ev is not None:
+            phase_ev[2].record()
 
 
-def _time_loop(fn, steps, warmup, dist=None):
+def _event():
+    return torch.cuda.Event(enable_timing=True)
+
+
+def time_steps(step, steps, warmup, dist=None):
+    """Whole-step time over `steps` steps (barrier + synchronize on both
+    sides, max over ranks), and each step's prefill / decode phase times from
+    events recorded on the launch stream between the phases."""
     for _ in range(warmup):
-        fn()
+        step.run()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    evs = [(_event(), _event(), _event()) for _ in range(steps)]
+    e0, e1 = _event(), _event()
     e0.record()
-    for _ in range(steps):
-        fn()
+    for i in range(steps):
+        step.run(evs[i])
     e1.record()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    return max_over_ranks(ms, dist, "cuda")
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, "cuda")
+    pre = max_over_ranks(sum(a.elapsed_time(b) for a, b, _ in evs), dist, "cuda")
+    dec = max_over_ranks(sum(b.elapsed_time(c) for _, b, c in evs), dist, "cuda")
+    return ms, pre, dec
+
+
+def kernel_times(step, steps):
+    """Average device time of the two dominant kernels over `steps` further
+    steps: the full layer's chunk-prefill attention kernel (events the library
+    records around that launch on its stream) and the full layer's decode
+    kernel (events around each decode call on the same stream)."""
+    pre_ev = [(_event(), _event()) for _ in range(steps)]
+    for a, b in pre_ev:   # create the events before handing their handles over
+        a.record()
+        b.record()
+    torch.cuda.synchronize()
+    dec_ms = []
+    for i in range(steps):
+        dec_ev = [(_event(), _event()) for _ in range(step.n_dec)]
+        step.prefill_phase(ev_full=pre_ev[i])
+        step.decode_phase(ev_dec=dec_ev)
+        torch.cuda.synchronize()
+        dec_ms.append([a.elapsed_time(b) for a, b in dec_ev])
+    pre_ms = statistics.mean(a.elapsed_time(b) for a, b in pre_ev)
+    per_launch = [statistics.mean(col) for col in zip(*dec_ms)]
+    return pre_ms, per_launch
 
 
 def max_over_ranks(x, dist, device):
@@ -237,29 +353,15 @@ def job_throughput(world, units_per_rank_step, ms_per_step):
     return world * units_per_rank_step / (ms_per_step * 1e-3)
 
 
-def full_prefill_roofline(step, steps, peaks):
-    """Average duration of the full-layer attention kernel over `steps` steps
-    (CUDA events the library records on its stream around that launch)."""
-    pairs_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(steps)]
-    for a, b in pairs_ev:   # create the events before handing their handles over
-        a.record()
-        b.record()
-    torch.cuda.synchronize()
-    for i in range(steps):
-        step.run(ev_full=pairs_ev[i])
-    torch.cuda.synchronize()
-    ms = statistics.mean(a.elapsed_time(b) for a, b in pairs_ev)
-    cfg = step.cfg
-    f = flops(cfg, 0, cfg.T, 0)
-    achieved = f / (ms * 1e-3) / 1e12
-    return ms, achieved
-
-
-def gptoss_prefill(dev, peaks, reps=10):
-    """Full-layer gpt-oss prefill (B=1, T=8192, 64/8/64 from fused qkv)."""
+def prefill_layers(dev, peaks, name, reps=10):
+    """Prefill of one layer pair of a configuration with no cached prefix
+    (gpt-oss: B=1, T=8192, 64/8/64 from fused qkv; Lite: B=8, T=4096,
+    8/4/96): the whole call (staging + attention) between events, and the
+    attention kernel alone (the events the library records around it). Full
+    causal layers are held to the tensor peak, band layers to
+    min(peak, HBM x arithmetic intensity)."""
     import sink_augmented_gqa_b200 as sa
-    cfg = wl.CONFIGS["gptoss_prefill"]
+    cfg = wl.CONFIGS[name]
     y = cfg.yarn
     cos, sin = sa.yarn_rope_tables(cfg.T, cfg.d, y["theta"], y["scaling"], y["orig_ctx"], y["alpha"],
                                    y["beta"], device=dev)
@@ -272,24 +374,39 @@ def gptoss_prefill(dev, peaks, reps=10):
         snap = cache.snapshot()
         out = torch.empty((cfg.B, cfg.T, cfg.n_q, cfg.d), dtype=torch.bfloat16, device=dev)
 
-        def once():
+        def once(ev=None):
             cache.restore(snap)
+            if ev is not None:
+                sa.set_prefill_events(*ev)
             sa.attn_prefill(cache, q, k, v, sinks, window, cfg.sm_scale, cos, sin, out=out)
+            if ev is not None:
+                sa.set_prefill_events()
         for _ in range(3):
             once()
         torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
-        for a, b in evs:
+        evs = [(_event(), _event()) for _ in range(reps)]
+        kev = [(_event(), _event()) for _ in range(reps)]
+        for a, b in kev:
             a.record()
-            once()
+            b.record()
+        torch.cuda.synchronize()
+        for (a, b), ke in zip(evs, kev):
+            a.record()
+            once(ke)
             b.record()
         torch.cuda.synchronize()
         ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+        kms = statistics.median(a.elapsed_time(b) for a, b in kev)
         f = flops(cfg, 0, cfg.T, window)
-        tf = f / (ms * 1e-3) / 1e12
-        key = "full" if window == 0 else "band"
-        res[key] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
-                    "frac_of_bf16_peak": round(tf / peaks["tf"], 4)}
+        nbytes = prefill_bytes(cfg, 0, cfg.T, window)
+        tf, ktf = f / (ms * 1e-3) / 1e12, f / (kms * 1e-3) / 1e12
+        res["full" if window == 0 else "band"] = {
+            "call_ms": round(ms, 4), "call_TFLOP/s": round(tf, 1),
+            "call": roofline_frac(tf, nbytes, ms * 1e-3, peaks),
+            "kernel_ms": round(kms, 4), "kernel_TFLOP/s": round(ktf, 1),
+            "kernel": roofline_frac(ktf, nbytes, kms * 1e-3, peaks),
+            "algorithmic_bytes": nbytes}
+        del cache
     return res
 
 
@@ -376,8 +493,13 @@ def lite_backward(dev, peaks, reps=10):
         ms = e0.elapsed_time(e1) / reps
         f = 10 * cfg.d * cfg.B * cfg.n_q * pairs(0, cfg.T, window)
         tf = f / (ms * 1e-3) / 1e12
+        # q, o, dO, k, v read in bf16 (lse in fp32); dq, dk, dv written in fp32
+        nq, nkv = cfg.B * cfg.T * cfg.n_q * cfg.d, cfg.B * cfg.T * cfg.n_kv * cfg.d
+        nbytes = (3 * nq + 2 * nkv) * 2 + (nq + 2 * nkv) * 4 + cfg.B * cfg.n_q * cfg.T * 4
         res["full" if window == 0 else "band"] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
-                                                  "frac_of_bf16_peak": round(tf / peaks["tf"], 4)}
+                                                  "frac_of_bf16_peak": round(tf / peaks["tf"], 4),
+                                                  "algorithmic_bytes": nbytes,
+                                                  **roofline_frac(tf, nbytes, ms * 1e-3, peaks)}
         del cache
     return res
 
@@ -529,67 +651,81 @@ def long_decode(dev, peaks, steps=8, layers=24, ring=False, fp8=False):
                              + (", e4m3 codes + fp32 row scales [B][n_kv][cap]" if fp8 else ", bf16"))}
 
 
-def e2e_lite(step, steps, warmup):
-    """Same step through host buffers: every step copies its q/k/v from pinned
-    host memory to the device and reads both layers' outputs back to pinned
-    host memory. Steps are pipelined over three streams (host-to-device copies,
-    compute, device-to-host copies) with two buffer sets, so one step's copies
-    overlap its neighbours' work, as a serving loop would run; the timed
-    region spans the first step's first copy to the last step's last copy."""
+def e2e_handoff(step, steps, warmup):
+    """The same step through host buffers, through the library's public API:
+    every step copies its inputs from pinned host memory and its outputs back
+    to pinned host memory.
+    * Prefill phase: the chunk's q/k/v of both layers go up on a copy stream
+      (layer 1's copy overlaps layer 0's prefill), each layer's output comes
+      back on a second copy stream as soon as it is computed; the phase ends
+      when the last output has landed on the host.
+    * Decode phase: per decode step, the new rows' q/k/v of both layers go up,
+      both layers decode, and their outputs come back, in order on one stream
+      (each step's input would depend on the previous step's output).
+    Phase times come from events on the launch stream. Returns (prefill ms,
+    decode ms) per step, and the host-to-device and device-to-host bytes per
+    step."""
     cfg = step.cfg
-    host_in, dev_in, dev_out, host_out = [], [], [], []
-    h2d = d2h = 0
+    host, dev_in, dev_out, host_out = [], [], [], []
     for L in step.layers:
-        hq, hk, hv = (L[n].cpu().pin_memory() for n in ("q", "k", "v"))
-        host_in.append((hq, hk, hv))
-        h2d += sum(t.numel() * t.element_size() for t in (hq, hk, hv))
-    for _ in range(2):
-        dev_in.append([tuple(torch.empty_like(L[n]) for n in ("q", "k", "v")) for L in step.layers])
-        dev_out.append([(torch.empty_like(L["out"]), torch.empty_like(L["dec"])) for L in step.layers])
-        host_out.append([(torch.empty(L["out"].shape, dtype=torch.bfloat16).pin_memory(),
-                          torch.empty(L["dec"].shape, dtype=torch.bfloat16).pin_memory()) for L in step.layers])
-    d2h = sum(a.numel() * 2 + b.numel() * 2 for a, b in host_out[0])
-    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    ev = lambda: torch.cuda.Event(enable_timing=False)
-    computed = [ev(), ev()]   # set s: its inputs are consumed
-    landed = [ev(), ev()]     # set s: its inputs are on the device
-    read = [ev(), ev()]       # set s: its outputs are on the host
-    used = [False, False]
+        host.append([L[n].cpu().pin_memory() for n in ("q", "k", "v", "dq", "dk", "dv")])
+        dev_in.append([torch.empty_like(L[n]) for n in ("q", "k", "v")]
+                      + [torch.empty_like(L[n][:, :1]) for n in ("dq", "dk", "dv")])
+        dev_out.append((torch.empty_like(L["out"]), torch.empty_like(L["dec"][:, :1])))
+        host_out.append((torch.empty(L["out"].shape, dtype=torch.bfloat16).pin_memory(),
+                         torch.empty(L["dec"].shape, dtype=torch.bfloat16).pin_memory()))
+    h2d = sum(t.numel() * t.element_size() for hs in host for t in hs)
+    d2h = sum(a.numel() * 2 + b.numel() * 2 for a, b in host_out)
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    nl = len(step.layers)
+    landed = [torch.cuda.Event() for _ in range(nl)]
+    computed = [torch.cuda.Event() for _ in range(nl)]
+    read = [torch.cuda.Event() for _ in range(nl)]
+    last_read = torch.cuda.Event()
 
-    def run(n, first=None, last=None):
-        for i in range(n):
-            st = i % 2
+    def one(ev=None):
+        if ev is not None:
+            ev[0].record(comp)
+        s_in.wait_stream(comp)     # the previous step has finished with the input buffers
+        for li in range(nl):
             with torch.cuda.stream(s_in):
-                if used[st]:
-                    s_in.wait_event(computed[st])
-                if i == 0 and first is not None:
-                    first.record(s_in)
-                for (hq, hk, hv), (dq, dk, dv) in zip(host_in, dev_in[st]):
-                    dq.copy_(hq, non_blocking=True)
-                    dk.copy_(hk, non_blocking=True)
-                    dv.copy_(hv, non_blocking=True)
-                landed[st].record(s_in)
-            with torch.cuda.stream(s_comp):
-                s_comp.wait_event(landed[st])
-                if used[st]:
-                    s_comp.wait_event(read[st])
-                step.run(q_in=dev_in[st], outs=dev_out[st])
-                computed[st].record(s_comp)
+                for hsrc, dst in zip(host[li][:3], dev_in[li][:3]):
+                    dst.copy_(hsrc, non_blocking=True)
+                landed[li].record(s_in)
+        for li in range(nl):
+            comp.wait_event(landed[li])
+            comp.wait_event(read[li])
+            step.prefill_phase_layer(li, dev_in[li], dev_out[li][0])
+            computed[li].record(comp)
             with torch.cuda.stream(s_out):
-                s_out.wait_event(computed[st])
-                for (ho, hd), (do, dd) in zip(host_out[st], dev_out[st]):
-                    ho.copy_(do, non_blocking=True)
-                    hd.copy_(dd, non_blocking=True)
-                read[st].record(s_out)
-                if i == n - 1 and last is not None:
-                    last.record(s_out)
-            used[st] = True
-        torch.cuda.synchronize()
+                s_out.wait_event(computed[li])
+                host_out[li][0].copy_(dev_out[li][0], non_blocking=True)
+                read[li].record(s_out)
+        last_read.record(s_out)
+        comp.wait_event(last_read)
+        if ev is not None:
+            ev[1].record(comp)
+        for st in range(step.n_dec):
+            for li in range(nl):
+                for hsrc, dst in zip(host[li][3:], dev_in[li][3:]):
+                    dst.copy_(hsrc[:, st:st + 1], non_blocking=True)
+            step.decode_phase(ins=[d for d in dev_in], outs=dev_out, first=st, count=1)
+            for li in range(nl):
+                host_out[li][1][:, st:st + 1].copy_(dev_out[li][1], non_blocking=True)
+        if ev is not None:
+            ev[2].record(comp)
 
-    run(warmup)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    run(steps, e0, e1)
-    return e0.elapsed_time(e1) / steps, h2d, d2h
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    evs = [(_event(), _event(), _event()) for _ in range(steps)]
+    for i in range(steps):
+        one(evs[i])
+    torch.cuda.synchronize()
+    pre = sum(a.elapsed_time(b) for a, b, _ in evs) / steps
+    dec = sum(b.elapsed_time(c) for _, b, c in evs) / steps
+    return pre, dec, h2d, d2h
 
 
 # ---------------------------------------------------------------------------
@@ -598,68 +734,92 @@ def e2e_lite(step, steps, warmup):
 
 def oracle_sample(budget_s=12.0, min_units=1):
     """Times the fp64 oracle on a bounded sample of the bench step: whole
-    (sequence, query head) units, each the step's work for that unit -- both
-    layers (band and full causal), prefill of T rows and the decode row, i.e.
-    T + 1 rows per layer (the decode row attends exactly like a prefill row
-    at position T) -- until the time budget is spent. Returns (TFLOP/s,
-    cores, description)."""
+    (sequence, query head) units of the handoff workload, each the step's work
+    for that unit on both layers (band and full causal) -- the 512-row chunk
+    against the 65,536-row prefix, then the 32 decode rows one call at a time
+    -- until the time budget is spent. The prefix values come from the same
+    seeded recipe (one sequence's worth per unit; they need not match the
+    GPU run's bits to time the arithmetic). Returns (prefill TFLOP/s, decode
+    KV GB/s, cores, description)."""
     from oracle import attention as oatt
+    from oracle import kvcache as okv
     from oracle import rope as orope
     from oracle import yarn as oyarn
     cfg = wl.CONFIGS[WORKLOAD]
     y = cfg.yarn
-    n = cfg.T + 1
-    cos, sin = oyarn.stored_tables(n, cfg.d, y["theta"], y["scaling"], y["orig_ctx"], y["alpha"], y["beta"])
+    off, T, n_dec = cfg.offset, cfg.T, cfg.decode_steps
+    cap = off + T + n_dec
+    cos, sin = oyarn.stored_tables(cap, cfg.d, y["theta"], y["scaling"], y["orig_ctx"], y["alpha"], y["beta"])
+    one = wl.scaled(cfg, B=1)
     layers = []
     for layer in range(2):
-        q, k, v = wl.qkv(cfg, n, layer=layer)
+        kp, vp = wl.prefilled_cache_rows(one, layer=layer)
+        q, k, v = wl.qkv(one, T + n_dec, layer=layer)
         layers.append(dict(window=cfg.layer_window(layer), sinks=wl.sinks(cfg, layer).double().numpy(),
-                           q=q.to(torch.float64).numpy(), k=k.to(torch.float64).numpy(),
+                           kp=kp, vp=vp, q=q.to(torch.float64).numpy(), k=k.to(torch.float64).numpy(),
                            v=v.to(torch.float64).numpy()))
-    done = 0
-    t0 = time.perf_counter()
+    pre_f = dec_b = 0
+    pre_t = dec_t = 0.0
     units = 0
+    t0 = time.perf_counter()
     while True:
-        b, h = divmod(units, cfg.n_q)
-        b %= cfg.B
+        h = units % cfg.n_q
         g = h // cfg.q_mult
         for L in layers:
-            qr = orope.rotate_bsh(L["q"][b:b + 1, :, h:h + 1], 0, cos, sin)
-            kr = orope.rotate_bsh(L["k"][b:b + 1, :, g:g + 1], 0, cos, sin)
-            oatt.sink_attention(qr, kr, L["v"][b:b + 1, :, g:g + 1], L["sinks"][h:h + 1], 0, L["window"],
-                                cfg.sm_scale)
-            done += 4 * cfg.d * pairs(0, n, L["window"])
+            w = L["window"]
+            c = okv.KVCache(1, cap, 1, cfg.d)
+            c.append(L["kp"][:, :, g:g + 1].to(torch.float64).numpy(), L["vp"][:, :, g:g + 1].to(torch.float64).numpy())
+            ta = time.perf_counter()
+            oatt.attend_step(c, L["q"][:, :T, h:h + 1], L["k"][:, :T, g:g + 1], L["v"][:, :T, g:g + 1],
+                             L["sinks"][h:h + 1], w, cfg.sm_scale, cos, sin)
+            tb = time.perf_counter()
+            for st in range(n_dec):
+                r = T + st
+                oatt.attend_step(c, L["q"][:, r:r + 1, h:h + 1], L["k"][:, r:r + 1, g:g + 1],
+                                 L["v"][:, r:r + 1, g:g + 1], L["sinks"][h:h + 1], w, cfg.sm_scale, cos, sin)
+                dec_b += decode_rows(off + r, w) * cfg.d * 2 * 2
+            tc = time.perf_counter()
+            pre_t += tb - ta
+            dec_t += tc - tb
+            pre_f += 4 * cfg.d * pairs(off, T, w)
         units += 1
         if units >= min_units and time.perf_counter() - t0 >= budget_s:
             break
     dt = time.perf_counter() - t0
     threads = int(os.environ.get("OMP_NUM_THREADS", "0")) or os.cpu_count()
     desc = (f"fp64 numpy oracle on {units} of the step's {cfg.B * cfg.n_q} (sequence, head) units: both layers "
-            f"(W={cfg.window} band, full causal), {cfg.T} prefill rows + the decode row each, RoPE included, "
-            f"{dt:.1f} s")
-    return done / dt / 1e12, threads, desc
+            f"(W={cfg.window} band, full causal), the {T}-row chunk against the {off}-row prefix "
+            f"({pre_t:.1f} s) and the {n_dec} decode rows one call at a time ({dec_t:.1f} s), RoPE included; "
+            f"{dt:.1f} s in all")
+    return pre_f / pre_t / 1e12, dec_b / dec_t / 1e9, threads, desc
 
 
 def step_config(cfg, world, parallelism):
     """The bench step's workload, the same for both arms."""
-    return {"workload": "GPT-OSS-Lite attention: B=8, T=4096 prefill + 1 decode row, "
-                        "n_q=8, n_kv=4, d=96, W=128 band layer + full causal layer, "
-                        "YaRN theta=150000 s=32 from 4096",
-            "global_batch": cfg.B * world, "seq_len": cfg.T, "parallelism": parallelism,
-            "l2": "inputs larger than L2 (step working set ~300 MB > 126 MB)"}
+    return {"workload": "prefill-to-decode handoff (the largest configuration): B=16 sequences sharing cache "
+                        "offset 65536, chunked prefill of 512 new rows each, then 32 decode steps; n_q=64, "
+                        "n_kv=8, d=64, sm_scale=1/8; layer pair W=128 band + full causal; YaRN theta=150000 s=32 "
+                        "from 4096",
+            "global_batch": cfg.B * world, "seq_len": cfg.offset + cfg.T + cfg.decode_steps,
+            "parallelism": parallelism,
+            "value_basis": "chunk-prefill phase (both layers, staging launch included), CUDA events on the "
+                           "launch stream inside every timed step",
+            "l2": "inputs larger than L2 (each layer's cache is 2.17 GB > 126 MB)"}
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    per = []
+    per, per_dec = [], []
     desc = ""
+    cores = os.cpu_count()
     for _ in range(args.warmup):
         oracle_sample(budget_s=0.5)
     t_all = time.perf_counter()
     for _ in range(args.steps):
-        tf, cores, desc = oracle_sample(budget_s=max(2.0, 20.0 / max(1, args.steps)))
+        tf, gbs, cores, desc = oracle_sample(budget_s=max(2.0, 20.0 / max(1, args.steps)))
         per.append(tf)
+        per_dec.append(gbs)
     value = statistics.mean(per)
     cfg = wl.CONFIGS[WORKLOAD]
     line = {"metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
@@ -667,6 +827,7 @@ def run_reference(args, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
             "config": step_config(cfg, 1, "none (host oracle)"),
+            "decode": {"value": statistics.mean(per_dec), "unit": "KV GB/s"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                              "sample": desc},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -677,13 +838,38 @@ def run_reference(args, rank, world):
 # Single-call loops for profilers (ncu): no timing, no output but a summary
 # ---------------------------------------------------------------------------
 
-PROFILE_CASES = ("gptoss_prefill_full", "gptoss_prefill_band", "lite_prefill_full", "long_decode_full",
+PROFILE_CASES = ("handoff_prefill_full", "handoff_prefill_full_b2", "handoff_prefill_band",
+                 "gptoss_prefill_full", "gptoss_prefill_band", "lite_prefill_full", "long_decode_full",
                  "long_decode_fp8", "gptoss_qkv_proj", "gptoss_out_proj", "lite_backward_b2")
 
 
 def profile_case(name, dev, steps, warmup):
     import sink_augmented_gqa_b200 as sa
-    if name == "lite_backward_b2":
+    if name.startswith("handoff"):
+        # the chunk prefill at offset 65,536 (b2: 2 of the 16 sequences, a
+        # capture-sized case with the same items: 64 heads x 2 row-tile pairs each)
+        cfg = wl.CONFIGS["handoff"]
+        if name.endswith("_b2"):
+            cfg = wl.scaled(cfg, B=2)
+        window = cfg.window if "band" in name else 0
+        y = cfg.yarn
+        cap = cfg.offset + cfg.T
+        cos, sin = sa.yarn_rope_tables(cap, cfg.d, y["theta"], y["scaling"], y["orig_ctx"], y["alpha"],
+                                       y["beta"], device=dev)
+        cache = sa.KVCache(cfg.B, cap, cfg.n_kv, cfg.d, device=dev)
+        kp, vp = wl.prefilled_cache_rows(cfg, layer=1, device=dev)
+        cache.append(kp, vp)
+        del kp, vp
+        snap = cache.snapshot()
+        q, k, v = wl.qkv(cfg, cfg.T, layer=1, device=dev)
+        sinks = wl.sinks(cfg, 1, device=dev)
+        out = torch.empty((cfg.B, cfg.T, cfg.n_q, cfg.d), dtype=torch.bfloat16, device=dev)
+
+        def once():
+            cache.restore(snap)
+            sa.attn_prefill(cache, q, k, v, sinks, window, cfg.sm_scale, cos, sin, out=out)
+        units = flops(cfg, cfg.offset, cfg.T, window)
+    elif name == "lite_backward_b2":
         # the Lite training layer with 2 of its 8 sequences (a capture-sized case)
         cfg = wl.scaled(wl.CONFIGS["lite"], B=2)
         q, k, v = wl.qkv(cfg, cfg.T, layer=1, device=dev)
@@ -802,21 +988,38 @@ def main():
 
     peaks = _peaks()
     cfg = wl.CONFIGS[WORKLOAD]
-    step = LiteStep(dev, cfg)
+    step = HandoffStep(dev, cfg)
     with Clocks(local) as clk:
-        ms = _time_loop(step.run, args.steps, args.warmup, dist)
-        full_ms, full_tf = full_prefill_roofline(step, max(3, min(args.steps, 10)), peaks)
+        ms, pre_ms, dec_ms = time_steps(step, args.steps, args.warmup, dist)
+        kpre_ms, kdec_ms = kernel_times(step, max(3, min(args.steps, 5)))
     clocks = clk.summary()
-    ms_step = ms / args.steps
-    value = job_throughput(world, step.flops, ms_step) / 1e12
+    K = args.steps
+    ms_step = ms / K
+    value = job_throughput(world, step.prefill_flops, pre_ms / K) / 1e12
+    dec_gbs = job_throughput(world, step.decode_bytes, dec_ms / K) / 1e9
+    step_tf = job_throughput(world, step.prefill_flops + step.decode_flops, ms_step) / 1e12
 
-    e2e_ms, h2d, d2h = e2e_lite(step, max(3, args.steps // 2), 3)
-    e2e_ms = max_over_ranks(e2e_ms, dist, "cuda")
-    e2e_val = job_throughput(world, step.flops, e2e_ms) / 1e12
+    e2e_pre, e2e_dec, h2d, d2h = e2e_handoff(step, max(3, K // 4), 2)
+    e2e_pre = max_over_ranks(e2e_pre, dist, "cuda")
+    e2e_dec = max_over_ranks(e2e_dec, dist, "cuda")
+    e2e_val = job_throughput(world, step.prefill_flops, e2e_pre) / 1e12
+    e2e_dec_gbs = job_throughput(world, step.decode_bytes, e2e_dec) / 1e9
+
+    # the two dominant kernels: full-layer chunk prefill (tensor) and full-layer decode (HBM)
+    k_tf = step.full_chunk_flops / (kpre_ms * 1e-3) / 1e12
+    dec_bytes = statistics.mean(step.full_decode_bytes)
+    k_dec_ms = statistics.mean(kdec_ms)
+    k_gbs = statistics.mean(b / (t * 1e-3) / 1e9 for b, t in zip(step.full_decode_bytes, kdec_ms))
+    band_cfg_bytes = prefill_bytes(cfg, cfg.offset, cfg.T, cfg.window)
+    step_flops = (step.prefill_flops, step.decode_flops, step.decode_bytes)
+    launches = step.launches * K
+    del step
+    torch.cuda.empty_cache()
 
     extras = {}
     if not args.no_extras and rank == 0:
-        extras["gptoss_prefill_T8192"] = gptoss_prefill(dev, peaks)
+        extras["gptoss_prefill_T8192"] = prefill_layers(dev, peaks, "gptoss_prefill")
+        extras["lite_prefill_T4096"] = prefill_layers(dev, peaks, "lite")
         extras["gptoss_projections"] = projections(dev, peaks)
         extras["lite_backward_T4096"] = lite_backward(dev, peaks)
         extras["long_context_decode_131072"] = long_decode(dev, peaks)
@@ -826,27 +1029,45 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
-        tf, cores, desc = oracle_sample()
-        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc}
+        tf, gbs, cores, desc = oracle_sample()
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": desc,
+               "decode_KV_GB/s": gbs}
 
     if dist is not None:
         dist.barrier()
     if rank == 0:
-        traffic = profiled_traffic("prefill_lite_full.md", ("prefill.cuh", "ptx.cuh"))
+        traffic = profiled_traffic("prefill_handoff_full.md", ("prefill.cuh", "ptx.cuh"))
+        dec_traffic = profiled_traffic("decode_handoff_full.md", ("decode.cuh", "fp8.cuh", "ptx.cuh"))
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) bf16 q/k/v, N(0,0.25) fp32 sinks)",
+            "data": "synthetic (seeded N(0,1) bf16 q/k/v and cache prefix, N(0,1) fp32 sinks)",
             "config": step_config(cfg, world, f"dp{world}"),
-            "roofline": {"bound": "tensor", "kernel": "prefill_kernel (full-causal layer attention; the staging launch before it is not included)",
-                         "achieved": round(full_tf, 2), "peak": peaks["tf"], "unit": "TFLOP/s",
-                         "frac": round(full_tf / peaks["tf"], 4), "traffic": traffic,
-                         "peak_source": f"{peaks['src']} dense bf16 (burst)", "ms": round(full_ms, 4)},
+            "phases": {"prefill": {"ms_per_step": round(pre_ms / K, 4), "TFLOP/s": round(value, 3),
+                                   "flops_per_step": step_flops[0]},
+                       "decode": {"ms_per_step": round(dec_ms / K, 4), "KV_GB/s": round(dec_gbs, 1),
+                                  "frac_of_hbm": round(dec_gbs / world / peaks["hbm"], 4),
+                                  "kv_bytes_per_step": step_flops[2], "flops_per_step": step_flops[1]},
+                       "step_TFLOP/s": round(step_tf, 3)},
+            "roofline": {"bound": "tensor",
+                         "kernel": "prefill_kernel<64>, full-causal layer, 512-row chunk at offset 65536, B=16",
+                         "achieved": round(k_tf, 2), "peak": peaks["tf"], "unit": "TFLOP/s",
+                         "frac": round(k_tf / peaks["tf"], 4), "traffic": traffic,
+                         "peak_source": f"{peaks['src']} dense bf16 (burst)",
+                         "frac_of_sustained": round(k_tf / peaks["tf_sus"], 4), "ms": round(kpre_ms, 4)},
+            "roofline_decode": {"bound": "hbm",
+                                "kernel": "decode_kernel<64,0>, full-causal layer, 16 x ~66,050 cached rows",
+                                "achieved": round(k_gbs, 1), "peak": peaks["hbm"], "unit": "GB/s",
+                                "frac": round(k_gbs / peaks["hbm"], 4), "traffic": dec_traffic,
+                                "algorithmic_bytes_per_launch": int(dec_bytes),
+                                "peak_source": f"{peaks['src']} HBM copy", "ms": round(k_dec_ms, 4)},
+            "band_layer_prefill_algorithmic_bytes": band_cfg_bytes,
             "clocks": clocks,
             "e2e": {"value": round(e2e_val, 3), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)},
-            "gpu_launches": step.launches * args.steps,
+                    "d2h_bytes_per_step": d2h, "prefill_ms_per_step": round(e2e_pre, 4),
+                    "decode_ms_per_step": round(e2e_dec, 4), "decode_KV_GB/s": round(e2e_dec_gbs, 1)},
+            "gpu_launches": launches,
             "cpu_baseline": cpu,
             "secondary": extras,
         }

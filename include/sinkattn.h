@@ -266,9 +266,14 @@ sa_status sa_kv_restore(sa_kv_cache* cache, const sa_snapshot* snap);
  * rows, so `out` may be `q` itself but must not overlap k, v, the cache, the
  * sinks, the tables or lse otherwise. Two launches on `stream` (staging,
  * attention). The attention kernel schedules its work items from a device
- * counter; the library keeps 64 such counters per device and hands them out
- * round robin, so at most 64 prefill calls may be in flight on one device at
- * a time (across all streams). SA_ERR_UNSUPPORTED on an FP8 cache.
+ * counter. The library keeps 128 such counters per device and never lets two
+ * calls in flight share one: calls made outside stream capture take the
+ * first 64 round robin, and before one reuses a counter its stream waits for
+ * the event the library recorded after that counter's previous call (on
+ * whatever stream it ran). Calls captured into a CUDA graph take the other
+ * 64 round robin without events; graph replays that run at the same time as
+ * one another must hold at most 64 prefill calls between them.
+ * SA_ERR_UNSUPPORTED on an FP8 cache.
  */
 sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* args, sa_stream_t stream);
 
@@ -425,6 +430,15 @@ sa_status sa_get_device_status(int32_t* code);
  * the timeout path only.
  */
 sa_status sa_set_wait_limit(int64_t cycles);
+
+/*
+ * Which of the 128 schedule counters (sa_attn_prefill above) the index-th
+ * prefill call on a device takes: index counts the calls made outside
+ * stream capture (captured == 0) or inside it (captured != 0) separately.
+ * Pure host arithmetic, no device work (no counterpart in the method;
+ * exposes the allocation rule to tests).
+ */
+int32_t sa_prefill_sched_slot(uint64_t index, int32_t captured);
 
 /*
  * Timing hook for the attention kernel of sa_attn_prefill (no counterpart in

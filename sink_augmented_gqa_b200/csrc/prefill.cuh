@@ -66,9 +66,10 @@ struct PrefillParams {
 };
 
 // Work counters of the dynamic item schedule, one pair per launch slot (the
-// host hands out slots round robin): [0] items handed out beyond the first
-// gridDim.x, [1] CTAs finished. The last CTA to finish resets both.
-constexpr int kPrefillSchedSlots = 64;
+// host hands a slot to one launch in flight at a time): [0] items handed out
+// beyond the first gridDim.x, [1] CTAs finished. The last CTA to finish
+// resets both.
+constexpr int kPrefillSchedSlots = 128;
 __device__ int g_prefill_sched[kPrefillSchedSlots][2];
 
 __host__ __device__ constexpr int align32(int x) { return (x + 31) / 32 * 32; }

@@ -241,22 +241,87 @@ sa_status check_attn(const sa_kv_cache* c, const sa_attn_args* a) {
 }
 
 template <typename K>
-void set_smem(K kernel, uint32_t bytes) {
-  cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+cudaError_t set_smem(K kernel, uint32_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
 // The shared-memory opt-in once per kernel and device (the attribute holds
-// per device): `done` has one bit per device ordinal below 64; devices above
-// that set it on every call, which is harmless. Safe to call from several
-// host threads (setting the attribute twice is harmless too).
+// per device): `done` has one bit per device ordinal below 64, set only once
+// the opt-in succeeded (a failed one is retried by the next launch, and its
+// error returned); devices above 64 opt in on every call, which is harmless.
+// Safe to call from several host threads (setting the attribute twice is
+// harmless too).
 template <typename K>
-void set_smem_once(K kernel, uint32_t bytes, std::atomic<uint64_t>& done) {
+sa_status set_smem_once(K kernel, uint32_t bytes, std::atomic<uint64_t>& done) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
   const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
-  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return;
-  set_smem(kernel, bytes);
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return SA_OK;
+  if (set_smem(kernel, bytes) != cudaSuccess) {
+    cudaGetLastError();   // the failed opt-in is reported here, not by a later launch check
+    return SA_ERR_CUDA;
+  }
   if (bit != 0) done.fetch_or(bit, std::memory_order_release);
+  return SA_OK;
+}
+
+constexpr int kMaxDevices = 64;
+
+// Counter slots of the prefill kernel's dynamic schedule (g_prefill_sched:
+// one counter pair per slot, reset by the last CTA of the launch that used
+// it). Two launches in flight at once must never share a slot.
+//  * Launches made outside stream capture take slots [0, kEagerSchedSlots)
+//    round robin. Before one reuses a slot its stream waits for the event
+//    recorded after the slot's previous launch, so the two are ordered
+//    whatever streams they run on (normally that launch finished long ago
+//    and the wait costs nothing).
+//  * Launches captured into a CUDA graph cannot wait on work outside the
+//    capture; they take slots [kEagerSchedSlots, kPrefillSchedSlots) round
+//    robin, so a graph never shares a slot with an eager launch. Graph
+//    replays that overlap one another must not hold more than
+//    kGraphSchedSlots prefill launches between them.
+constexpr int kEagerSchedSlots = sa::kPrefillSchedSlots / 2;
+constexpr int kGraphSchedSlots = sa::kPrefillSchedSlots - kEagerSchedSlots;
+
+int sched_slot_of(uint64_t index, bool captured) {
+  return captured ? kEagerSchedSlots + (int)(index % kGraphSchedSlots) : (int)(index % kEagerSchedSlots);
+}
+
+struct SchedState {
+  std::mutex mu;
+  uint64_t eager_next = 0, graph_next = 0;
+  cudaEvent_t done[kEagerSchedSlots] = {};
+};
+SchedState g_sched[kMaxDevices];
+
+// Runs launch(slot) with a schedule slot acquired as above; the slot counts
+// as used only if the launch succeeded.
+template <typename F>
+sa_status with_sched_slot(cudaStream_t s, F&& launch) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SA_ERR_INVALID_ARG;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) return SA_ERR_CUDA;
+  SchedState& st = g_sched[dev];
+  std::lock_guard<std::mutex> lock(st.mu);
+  if (cs != cudaStreamCaptureStatusNone) {
+    const sa_status r = launch(sched_slot_of(st.graph_next, true));
+    if (r == SA_OK) ++st.graph_next;
+    return r;
+  }
+  const int slot = sched_slot_of(st.eager_next, false);
+  cudaEvent_t& ev = st.done[slot];
+  if (ev == nullptr) {
+    if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return SA_ERR_CUDA;
+  } else if (cudaStreamWaitEvent(s, ev, 0) != cudaSuccess) {
+    return SA_ERR_CUDA;
+  }
+  const sa_status r = launch(slot);
+  if (r != SA_OK) return r;
+  if (cudaEventRecord(ev, s) != cudaSuccess) return SA_ERR_CUDA;
+  ++st.eager_next;
+  return SA_OK;
 }
 
 template <int D>
@@ -303,18 +368,19 @@ sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream
   p.rope = a->rope_fused ? 1 : 0;
   p.n_pairs = (a->T + 255) / 256;
   p.ring_cap = c->ring > 0 ? c->cap : 0;
-  // Launches take the dynamic-schedule counter pairs round robin; a pair is
-  // reset by the last CTA of its launch, so up to kPrefillSchedSlots
-  // launches may be in flight at once on one device.
-  static std::atomic<unsigned> sched_seq{0};
-  p.sched_slot = (int)(sched_seq.fetch_add(1, std::memory_order_relaxed) % sa::kPrefillSchedSlots);
   static std::atomic<uint64_t> smem_set{0};
-  set_smem_once(sa::prefill_kernel<D>, Cfg::SMEM_BYTES, smem_set);
+  {
+    const sa_status sm = set_smem_once(sa::prefill_kernel<D>, Cfg::SMEM_BYTES, smem_set);
+    if (sm != SA_OK) return sm;
+  }
   // persistent: one CTA per SM (or per item when there are fewer)
   const long long n_items = (long long)p.n_pairs * a->n_q * a->B;
   const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
-  sa::prefill_kernel<D><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmO, p);
-  return last_launch_status();
+  return with_sched_slot(stream, [&](int slot) {
+    p.sched_slot = slot;
+    sa::prefill_kernel<D><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmO, p);
+    return last_launch_status();
+  });
 }
 
 struct DecodeSplit {
@@ -345,6 +411,35 @@ size_t decode_ws_bytes(int B, int n_kv, int q_mult, int d, int S) {
   return cnt + rows * 4 * 2 + rows * d * 4;
 }
 
+// Cache rows per ring stage of decode_kernel<d, f8> (its Cfg::R).
+long long decode_stage_rows(int d, bool f8) {
+  switch (d) {
+    case 64: return f8 ? sa::DecodeCfgT<64, true>::R : sa::DecodeCfgT<64, false>::R;
+    case 96: return f8 ? sa::DecodeCfgT<96, true>::R : sa::DecodeCfgT<96, false>::R;
+    default: return f8 ? sa::DecodeCfgT<128, true>::R : sa::DecodeCfgT<128, false>::R;
+  }
+}
+
+// The rows one decode call reads and how they are split over CTAs: the
+// launch and the allocation-free entry point's size check both take it from
+// here. lo_mask: first admitted key; lo: first row streamed (ring and FP8
+// stages start on multiples of the stage height, so no TMA box wraps a ring
+// and the scale boxes start on their stage's first row).
+struct DecodePlan {
+  long long lo_mask, lo;
+  DecodeSplit split;
+};
+
+DecodePlan plan_decode(const sa_kv_cache* c, const sa_attn_args* a) {
+  const bool f8 = c->kv_dtype == SA_KV_FP8_E4M3;
+  const long long R = decode_stage_rows(c->d, f8);
+  DecodePlan pl;
+  pl.lo_mask = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
+  pl.lo = (c->ring > 0 || f8) ? pl.lo_mask / R * R : pl.lo_mask;
+  pl.split = decode_split(a->B, c->n_kv, a->offset - pl.lo, R);
+  return pl;
+}
+
 template <int D, bool F8>
 sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, size_t ws_bytes,
                         cudaStream_t stream) {
@@ -352,14 +447,12 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   const int q_mult = a->n_q / c->n_kv;
   DecodeParams p;
   p.off = a->offset;
-  p.lo_mask = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
-  // a ring's stages start at multiples of the stage height so that none wraps
   p.ring_cap = c->ring > 0 ? c->cap : 0;
-  // FP8 stages start aligned too: the scales' TMA boxes begin at the stage's
-  // first row, their innermost coordinate
-  p.lo = (p.ring_cap > 0 || F8) ? p.lo_mask / Cfg::R * Cfg::R : p.lo_mask;
+  const DecodePlan pl = plan_decode(c, a);
+  p.lo_mask = pl.lo_mask;
+  p.lo = pl.lo;
   const long long n_cache = p.off - p.lo;
-  const DecodeSplit sp = decode_split(a->B, c->n_kv, n_cache, Cfg::R);
+  const DecodeSplit sp = pl.split;
   p.S = sp.S;
   p.chunk = sp.chunk;
   if (p.S > 1) {
@@ -422,7 +515,10 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   p.ws_m = reinterpret_cast<float*>(w + cnt + rows * D * 4);
   p.ws_l = reinterpret_cast<float*>(w + cnt + rows * D * 4 + rows * 4);
   static std::atomic<uint64_t> smem_set{0};
-  set_smem_once(sa::decode_kernel<D, F8>, Cfg::SMEM_BYTES, smem_set);
+  {
+    const sa_status sm = set_smem_once(sa::decode_kernel<D, F8>, Cfg::SMEM_BYTES, smem_set);
+    if (sm != SA_OK) return sm;
+  }
   // Programmatic stream serialization: back-to-back decode launches (one per
   // layer) overlap one kernel's drain with the next one's launch and set-up;
   // the kernel waits for its predecessor before touching global memory.
@@ -486,7 +582,6 @@ sa_status launch_stage(sa_kv_cache* c, const sa_attn_args* a, cudaStream_t strea
 // address looked up once per device (host code may not use the symbol itself
 // as an address).
 static __device__ __align__(256) uint8_t g_decode_scratch[SA_DECODE_STATIC_SCRATCH_BYTES];
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
@@ -537,7 +632,10 @@ sa_status launch_gemm_bn(const void* a, int64_t lda, const void* w, int64_t ldw,
   const long long tiles = (long long)p.tiles_m * p.tiles_n;
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
   static std::atomic<uint64_t> smem_set{0};
-  set_smem_once(sa::gemm_kernel<BN>, C::SMEM_BYTES, smem_set);
+  {
+    const sa_status sm = set_smem_once(sa::gemm_kernel<BN>, C::SMEM_BYTES, smem_set);
+    if (sm != SA_OK) return sm;
+  }
   sa::gemm_kernel<BN><<<grid, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tmA, tmB, tmC, p);
   return last_launch_status();
 }
@@ -604,7 +702,10 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
   static_assert(C0::NUM_THREADS == C1::NUM_THREADS, "both passes share one launch");
   constexpr uint32_t smem = C0::SMEM_BYTES > C1::SMEM_BYTES ? C0::SMEM_BYTES : C1::SMEM_BYTES;
   static std::atomic<uint64_t> smem_set{0};
-  set_smem_once(sa::bwd_tc_kernel<D>, smem, smem_set);
+  {
+    const sa_status sm = set_smem_once(sa::bwd_tc_kernel<D>, smem, smem_set);
+    if (sm != SA_OK) return sm;
+  }
   // one CTA per 128-row tile, per head of either pass, per sequence (< 2^31: checked by the caller)
   const unsigned ctas = (unsigned)((a->T + 127) / 128) * (unsigned)(a->n_kv + a->n_q) * (unsigned)a->B;
   sa::bwd_tc_kernel<D><<<ctas, C0::NUM_THREADS, smem, stream>>>(k1, v1, q1, o1, q0, o0, k0, v0, p);
@@ -814,14 +915,7 @@ sa_status sa_attn_decode_static(sa_kv_cache* cache, const sa_attn_args* a, sa_st
   if (a->T != 1) return SA_ERR_INVALID_ARG;
   const int q_mult = a->n_q / cache->n_kv;
   if (q_mult > 8) return SA_ERR_SHAPE;
-  long long lo = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
-  // the split of launch_decode: ring and FP8 stages start on multiples of the stage height
-  const bool f8 = cache->kv_dtype == SA_KV_FP8_E4M3;
-  const long long stage = f8 ? (cache->d == 128 ? sa::DecodeF8Cfg<128>::R : sa::DecodeF8Cfg<64>::R) : 128;
-  static_assert(sa::DecodeF8Cfg<64>::R == sa::DecodeF8Cfg<96>::R, "one FP8 stage height for d = 64, 96");
-  static_assert(sa::DecodeCfg<64>::R == 128 && sa::DecodeCfg<128>::R == 128, "bf16 stage height");
-  if (cache->ring > 0 || f8) lo = lo / stage * stage;
-  const DecodeSplit sp = decode_split(a->B, cache->n_kv, a->offset - lo, stage);
+  const DecodeSplit sp = plan_decode(cache, a).split;   // the split the launch will use
   if (sp.S > 1 && decode_ws_bytes(a->B, cache->n_kv, q_mult, cache->d, sp.S) > SA_DECODE_STATIC_SCRATCH_BYTES)
     return SA_ERR_WORKSPACE;
   void* scratch = nullptr;
@@ -919,6 +1013,10 @@ sa_status sa_set_prefill_events(void* before, void* after) {
   g_prefill_ev_before = static_cast<cudaEvent_t>(before);
   g_prefill_ev_after = static_cast<cudaEvent_t>(after);
   return SA_OK;
+}
+
+int32_t sa_prefill_sched_slot(uint64_t index, int32_t captured) {
+  return sched_slot_of(index, captured != 0);
 }
 
 sa_status sa_set_wait_limit(int64_t cycles) {

@@ -91,7 +91,7 @@ EXPORTS = (
     "sa_attn_decode_workspace_size", "sa_get_device_status", "sa_set_wait_limit",
     "sa_attn_decode_static", "sa_set_prefill_events", "sa_kv_cache_init_ring",
     "sa_kv_cache_init_fp8", "sa_rmsnorm_fold_weight", "sa_qkv_proj", "sa_out_proj",
-    "sa_attn_backward", "sa_attn_backward_workspace_size",
+    "sa_attn_backward", "sa_attn_backward_workspace_size", "sa_prefill_sched_slot",
 )
 
 _lib = None
@@ -133,6 +133,7 @@ def lib():
         L.sa_attn_backward.argtypes = [P(_BwdArgs), vp, ctypes.c_size_t, vp]
         L.sa_attn_backward_workspace_size.restype = ctypes.c_size_t
         L.sa_attn_backward_workspace_size.argtypes = [i32, i32, i32]
+        L.sa_prefill_sched_slot.argtypes = [ctypes.c_uint64, i32]
         for name in EXPORTS:
             if name not in ("sa_status_string", "sa_attn_decode_workspace_size",
                             "sa_attn_backward_workspace_size"):

@@ -1,10 +1,17 @@
 """Shared test helpers: tolerance checks and oracle runs on seeded inputs.
 
-Tolerance (the stated bar for bf16 outputs with fp32 accumulation): compared
-with the oracle's exact output rounded to bf16 (the stored precision), every
-element is within max-abs 1e-2 -- or exactly one bf16 step away, which is a
-rounding-boundary flip that max-abs cannot exclude once |out| >= 2, where one
-bf16 step is already 0.0156 -- and the mean absolute error is <= 1e-3.
+Tolerance (the stated bar for bf16 outputs with fp32 accumulation): each GPU
+element is compared with the oracle's exact fp64 value, unrounded. It passes
+when its error is <= 1e-2 (max-abs), and the mean absolute error over all
+compared elements must be <= 1e-3 (mean-abs).
+
+One exemption, counted and reported apart: where |ref| >= 4 the two bf16
+neighbours of the exact value are 2^-5 apart, so even the correctly rounded
+result can miss it by up to 2^-6 = 0.0156 > 1e-2 and the max-abs bar cannot
+be met by any bf16 output. There the bound is half a bf16 step of |ref| plus
+1e-3 (the correctly rounded value plus an fp32 computation error far below
+1e-3). Below |ref| = 4 half a step is at most 2^-7 = 0.0078 and the plain
+1e-2 applies.
 """
 
 import numpy as np
@@ -18,23 +25,36 @@ from oracle import yarn as oyarn
 
 MAX_ABS = 1e-2
 MEAN_ABS = 1e-3
+# Elements that passed only under the |ref| >= 4 exemption: (what, count, compared).
+EXEMPT_LOG = []
 
 
 def to64(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
+def bf16_bound(ref):
+    """Per-element max-abs bound against the exact value ref (see the module
+    docstring): 1e-2, or half a bf16 step of ref plus 1e-3 where that is larger
+    (only |ref| >= 4)."""
+    return np.maximum(MAX_ABS, 0.5 * obf16.bf16_ulp(ref) + 1e-3)
+
+
 def check_bf16_output(gpu, ref, what=""):
-    """gpu: torch bf16 tensor; ref: fp64 numpy array of the same shape."""
+    """gpu: torch bf16 tensor; ref: fp64 numpy array of the same shape (the
+    oracle's exact result, not rounded). Returns (max err, mean err)."""
     g = to64(gpu)
-    r = obf16.round_bf16(ref)
+    r = np.asarray(ref, dtype=np.float64)
     assert g.shape == r.shape, (g.shape, r.shape)
     assert np.all(np.isfinite(g)), f"{what}: non-finite output"
     err = np.abs(g - r)
-    ok = (err <= MAX_ABS) | (err <= obf16.bf16_ulp(r) * 1.0000001)
+    ok = err <= bf16_bound(r)
     bad = np.argwhere(~ok)
     assert bad.size == 0, (f"{what}: {len(bad)} elements beyond tolerance; first {bad[:5].tolist()} "
                            f"gpu={g[tuple(bad[0])]} ref={r[tuple(bad[0])]}")
+    exempt = int(np.count_nonzero(err > MAX_ABS))
+    if exempt:
+        EXEMPT_LOG.append((what, exempt, int(err.size)))
     mean = float(err.mean()) if err.size else 0.0
     assert mean <= MEAN_ABS, f"{what}: mean abs err {mean}"
     return float(err.max()) if err.size else 0.0, mean

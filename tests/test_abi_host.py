@@ -222,3 +222,17 @@ def test_backward_argument_errors_return_before_launch(L):
     a.q_strides = S._I64x3(4096, 256, 60)                             # misaligned head stride
     assert call(a) == codes["SA_ERR_INVALID_ARG"]
     assert call(_bwd_args(), nbytes=need - 256) == codes["SA_ERR_WORKSPACE"]
+
+
+def test_prefill_schedule_slots_wrap(L):
+    """The prefill's schedule counters: eager calls cycle through 64 slots and
+    wrap (the 65th reuses the 1st, after waiting for it on the device);
+    captured calls cycle through 64 others, so a graph never shares one with
+    an eager call."""
+    eager = [L.sa_prefill_sched_slot(i, 0) for i in range(200)]
+    graph = [L.sa_prefill_sched_slot(i, 1) for i in range(200)]
+    assert eager[:64] == list(range(64)) and graph[:64] == list(range(64, 128))
+    assert all(eager[i] == eager[i % 64] for i in range(200))
+    assert all(graph[i] == graph[i % 64] for i in range(200))
+    assert not set(eager) & set(graph)
+    assert L.sa_prefill_sched_slot(2 ** 64 - 1, 0) == (2 ** 64 - 1) % 64

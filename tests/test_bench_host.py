@@ -41,3 +41,35 @@ def test_job_throughput_sums_ranks():
     # whole-job value: units of all ranks over the slowest rank's time
     assert bench.job_throughput(4, 1e12, 1.0) == pytest.approx(4e15)
     assert np.isclose(bench.job_throughput(1, 5e11, 0.5), 1e15)
+
+
+def test_handoff_work_and_bytes():
+    cfg = wl.CONFIGS["handoff"]
+    # the full layer's chunk: 16 sequences x 64 heads x 512 rows at offset 65,536
+    f = bench.flops(cfg, cfg.offset, cfg.T, 0)
+    assert f == 4 * 64 * 16 * 64 * (512 * 65536 + 512 * 513 // 2)
+    assert f == pytest.approx(8.83e12, rel=2e-3)
+    # decode rows read: the whole prefix on full layers, W rows on band layers
+    assert bench.decode_rows(cfg.offset + cfg.T, 0) == cfg.offset + cfg.T + 1
+    assert bench.decode_rows(cfg.offset + cfg.T, 128) == 128
+    assert bench.decode_rows(5, 128) == 6
+    # one decode step of the full layer reads ~2.16 GB of K and V
+    assert cfg.B * bench.decode_rows(cfg.offset + cfg.T, 0) * bench.kv_row_bytes(cfg) == pytest.approx(
+        2.165e9, rel=1e-3)
+    # prefill bytes: q and out, the new k/v rows read and appended, and the
+    # admitted prefix rows (W - 1 per sequence on the band layer)
+    qo = 2 * 16 * 512 * 64 * 64 * 2
+    new = 2 * 16 * 512 * 8 * 64 * 4
+    assert bench.prefill_bytes(cfg, cfg.offset, cfg.T, 128) == qo + new + 16 * 127 * 8 * 64 * 4
+    assert bench.prefill_bytes(cfg, 0, 100, 0) == 2 * 16 * 100 * 64 * 64 * 2 + 2 * 16 * 100 * 8 * 64 * 4
+
+
+def test_roofline_fraction_takes_the_lower_roof():
+    peaks = dict(tf=1000.0, hbm=5000.0)
+    # 1 TFLOP over 1 GB in 2 ms: AI = 1000 flop/B, 500 TFLOP/s against the tensor roof
+    r = bench.roofline_frac(500.0, 1e9, 2e-3, peaks)
+    assert r["bound"] == "tensor" and r["frac_of_roofline"] == pytest.approx(0.5)
+    # 10 GFLOP over 1 GB in 0.4 ms: AI = 10, roof 50 TFLOP/s (HBM), achieved 25
+    r = bench.roofline_frac(25.0, 1e9, 0.4e-3, peaks)
+    assert r["bound"] == "hbm" and r["roofline_TFLOP/s"] == pytest.approx(50.0)
+    assert r["frac_of_roofline"] == pytest.approx(0.5)

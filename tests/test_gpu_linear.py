@@ -47,9 +47,13 @@ def _padded(t, ld):
 
 
 def _check(gpu, ref, s_abs, rel, what):
+    """Against the exact (unrounded) value: the fp32 result lies within
+    e = rel * s_abs of it, and its rounding to bf16 adds at most half a bf16
+    step at |ref| + e."""
     g = to64(gpu)
-    r = obf16.round_bf16(ref)
-    tol = obf16.bf16_ulp(r) * 1.0000001 + rel * s_abs
+    r = np.asarray(ref, dtype=np.float64)
+    e = rel * s_abs
+    tol = 0.5 * obf16.bf16_ulp(np.abs(r) + e) * 1.0000001 + e
     err = np.abs(g - r)
     bad = np.argwhere(~(err <= tol))
     assert np.all(np.isfinite(g)), f"{what}: non-finite output"
