@@ -261,11 +261,13 @@ sa_status sa_kv_restore(sa_kv_cache* cache, const sa_snapshot* snap);
  * note, "How it works"). cache->offset += T on success. T == 0 is a no-op.
  * The attention runs on tcgen05 tensor cores with fp32 accumulation; the
  * softmax weights enter the PV product as bf16.
- * When rope_fused, the rotated queries are first staged in args->out (same
- * [B][T][n_q][d] view) and each output tile overwrites its own staged query
- * rows, so `out` may be `q` itself but must not overlap k, v, the cache, the
- * sinks, the tables or lse otherwise. Two launches on `stream` (staging,
- * attention). The attention kernel schedules its work items from a device
+ * When rope_fused, one launch rotates the K rows as it appends them and
+ * stages the rotated queries in args->out (same [B][T][n_q][d] view); the
+ * attention kernel then loads its query tiles from there and overwrites each
+ * staged tile with its own output rows, so `out` may be `q` itself but must
+ * not overlap k, v, the cache, the sinks, the tables or lse otherwise. Two
+ * launches on `stream` (staging, attention). The
+ * attention kernel schedules its work items from a device
  * counter. The library keeps 128 such counters per device and never lets two
  * calls in flight share one: calls made outside stream capture take the
  * first 64 round robin, and before one reuses a counter its stream waits for

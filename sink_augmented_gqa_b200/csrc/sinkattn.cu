@@ -43,10 +43,21 @@ bool head_dim_ok(int d) { return d == 64 || d == 96 || d == 128; }
 // (128 decode rows; 128, 96, 64 prefill keys), so no tile wraps around.
 constexpr int kRingQuantum = 384;
 
+// SM count of the current device, looked up once per device (it is read on
+// every launch).
 int num_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 256 ? 256 : (n < 1 ? 1 : n);
+  static std::atomic<int> cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64) {
+    const int c = cached[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 148;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  n = n > 256 ? 256 : (n < 1 ? 1 : n);
+  if (dev >= 0 && dev < 64) cached[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
 int grid_for(long long n) {
@@ -562,10 +573,10 @@ sa_status launch_append(sa_kv_cache* c, const void* k, const int64_t ks[3], cons
 cudaEvent_t g_prefill_ev_before = nullptr;
 cudaEvent_t g_prefill_ev_after = nullptr;
 
-// Prefill staging: append K/V (rotating k) and, when RoPE is fused, write the
-// rotated queries into `out` for the attention kernel to load by TMA.
-sa_status launch_stage(sa_kv_cache* c, const sa_attn_args* a, cudaStream_t stream) {
-  const int stage_q = a->rope_fused ? 1 : 0;
+// Prefill staging, one launch: append K/V (rotating k when RoPE is fused)
+// and, with stage_q, write the rotated queries into `out` for the attention
+// kernel to load by TMA.
+sa_status launch_stage(sa_kv_cache* c, const sa_attn_args* a, bool stage_q, cudaStream_t stream) {
   const long long n = (long long)c->B * a->T * (c->n_kv + (stage_q ? a->n_q : 0)) * (c->d / 16);
   sa::prefill_stage_kernel<<<grid_for(n), 256, 0, stream>>>(
       static_cast<__nv_bfloat16*>(c->k), static_cast<__nv_bfloat16*>(c->v), c->cap,
@@ -574,7 +585,7 @@ sa_status launch_stage(sa_kv_cache* c, const sa_attn_args* a, cudaStream_t strea
       c->B, a->T, c->n_kv, c->d, c->offset, a->rope_fused ? 1 : 0, a->cos, a->sin,
       static_cast<const __nv_bfloat16*>(a->q), a->q_strides[0], a->q_strides[1], a->q_strides[2],
       a->n_q, static_cast<__nv_bfloat16*>(a->out), a->out_strides[0], a->out_strides[1],
-      a->out_strides[2], stage_q, c->ring > 0 ? 1 : 0);
+      a->out_strides[2], stage_q ? 1 : 0, c->ring > 0 ? 1 : 0);
   return last_launch_status();
 }
 
@@ -866,7 +877,9 @@ sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* a, sa_stream_t
   if (cache->kv_dtype != SA_KV_BF16) return SA_ERR_UNSUPPORTED;
   if (a->T == 0) return SA_OK;
   cudaStream_t s = (cudaStream_t)stream;
-  st = launch_stage(cache, a, s);
+  // one launch: the call's K rows rotated (when RoPE is fused) and appended
+  // with V, and the rotated queries staged in `out`
+  st = launch_stage(cache, a, a->rope_fused, s);
   if (st != SA_OK) return st;
   cudaEvent_t ev0 = g_prefill_ev_before, ev1 = g_prefill_ev_after;
   if (ev0 != nullptr && cudaEventRecord(ev0, s) != cudaSuccess) return SA_ERR_CUDA;

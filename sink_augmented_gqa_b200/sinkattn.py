@@ -12,6 +12,8 @@ Names mirror the C ABI in ``include/sinkattn.h`` without the ``sa_`` prefix:
 
 import ctypes
 import os
+import struct
+import threading
 
 import torch
 
@@ -69,6 +71,7 @@ class _Snapshot(ctypes.Structure):
 _I64x3 = ctypes.c_int64 * 3
 
 
+
 class _AttnArgs(ctypes.Structure):
     _fields_ = [
         ("q", ctypes.c_void_p), ("q_strides", _I64x3),
@@ -82,6 +85,14 @@ class _AttnArgs(ctypes.Structure):
         ("out", ctypes.c_void_p), ("out_strides", _I64x3),
         ("lse", ctypes.c_void_p),
     ]
+
+# sa_attn_args packed in one step (C layout, native alignment): the per-call
+# marshalling of a decode step is on the host's critical path when layers are
+# launched one by one, and building the ctypes structure field by field costs
+# several times more than the packing.
+_ATTN_FMT = "@P3qP3qP3qPiiiqifiPPiP3qP"
+assert struct.calcsize(_ATTN_FMT) == ctypes.sizeof(_AttnArgs)
+_tls = threading.local()
 
 
 # Every symbol include/sinkattn.h declares.
@@ -150,6 +161,11 @@ def _check(code, where):
 def _stream(t=None):
     dev = t.device if t is not None else torch.device("cuda")
     return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _raw_stream(t):
+    """The current stream of t's device as a raw handle (no Stream object)."""
+    return torch._C._cuda_getCurrentRawStream(t.device.index)
 
 
 def _ptr(t):
@@ -278,26 +294,32 @@ class KVCache:
         _check(lib().sa_kv_restore(ctypes.byref(self.raw), ctypes.byref(snap.raw)), "sa_kv_restore")
 
 
+def _view4(name, t):
+    """Strides [B, T, H] of a bf16 CUDA [B, T, H, d] view with contiguous d."""
+    if t.dtype != torch.bfloat16 or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA bf16 tensor")
+    st = t.stride()
+    if len(st) != 4 or st[3] != 1:
+        raise ValueError("expected a [B, T, H, d] tensor with a contiguous last dimension")
+    return st
+
+
 def _args(cache, q, k, v, sinks, window, sm_scale, cos, sin, rope_fused, out, lse):
-    for n, t in (("q", q), ("k", k), ("v", v), ("out", out)):
-        _require_bf16_cuda(n, t)
+    """sa_attn_args for one call, packed into this thread's reusable struct
+    (the library reads it only during the call)."""
+    qs, ks, vs, os_ = _view4("q", q), _view4("k", k), _view4("v", v), _view4("out", out)
     if sinks is not None and (sinks.dtype != torch.float32 or not sinks.is_contiguous()):
         raise TypeError("sinks must be a contiguous fp32 CUDA tensor")
-    a = _AttnArgs()
-    a.q, a.q_strides = q.data_ptr(), _strides(q)
-    a.k, a.k_strides = k.data_ptr(), _strides(k)
-    a.v, a.v_strides = v.data_ptr(), _strides(v)
-    a.sinks = 0 if sinks is None else sinks.data_ptr()
-    a.B, a.T, a.n_q = q.shape[0], q.shape[1], q.shape[2]
-    a.offset = cache.offset
-    a.window = int(window)
-    a.sm_scale = float(sm_scale)
-    a.rope_fused = 1 if rope_fused else 0
-    a.cos = 0 if cos is None else cos.data_ptr()
-    a.sin = 0 if sin is None else sin.data_ptr()
-    a.max_pos = 0 if cos is None else cos.shape[0]
-    a.out, a.out_strides = out.data_ptr(), _strides(out)
-    a.lse = 0 if lse is None else lse.data_ptr()
+    a = getattr(_tls, "args", None)
+    if a is None:
+        a = _tls.args = _AttnArgs()
+    struct.pack_into(_ATTN_FMT, a, 0,
+                     q.data_ptr(), qs[0], qs[1], qs[2], k.data_ptr(), ks[0], ks[1], ks[2],
+                     v.data_ptr(), vs[0], vs[1], vs[2], 0 if sinks is None else sinks.data_ptr(),
+                     q.shape[0], q.shape[1], q.shape[2], cache.raw.offset, int(window), float(sm_scale),
+                     1 if rope_fused else 0, 0 if cos is None else cos.data_ptr(),
+                     0 if sin is None else sin.data_ptr(), 0 if cos is None else cos.shape[0],
+                     out.data_ptr(), os_[0], os_[1], os_[2], 0 if lse is None else lse.data_ptr())
     return a
 
 
@@ -311,7 +333,7 @@ def attn_prefill(cache, q, k, v, sinks, window, sm_scale, cos=None, sin=None, ro
     if return_lse and lse is None:
         lse = torch.empty((B, n_q, T), dtype=torch.float32, device=q.device)
     a = _args(cache, q, k, v, sinks, window, sm_scale, cos, sin, rope_fused, out, lse)
-    _check(lib().sa_attn_prefill(ctypes.byref(cache.raw), ctypes.byref(a), _stream(q)), "sa_attn_prefill")
+    _check(lib().sa_attn_prefill(ctypes.byref(cache.raw), ctypes.byref(a), _raw_stream(q)), "sa_attn_prefill")
     return (out, lse) if return_lse else out
 
 
@@ -335,8 +357,8 @@ def attn_decode(cache, q, k, v, sinks, window, sm_scale, cos=None, sin=None, rop
     if return_lse and lse is None:
         lse = torch.empty((B, n_q, T), dtype=torch.float32, device=q.device)
     a = _args(cache, q, k, v, sinks, window, sm_scale, cos, sin, rope_fused, out, lse)
-    _check(lib().sa_attn_decode(ctypes.byref(cache.raw), ctypes.byref(a), _ptr(workspace),
-                                workspace.numel() * workspace.element_size(), _stream(q)),
+    _check(lib().sa_attn_decode(ctypes.byref(cache.raw), ctypes.byref(a), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), _raw_stream(q)),
            "sa_attn_decode")
     return (out, lse) if return_lse else out
 
@@ -426,7 +448,7 @@ def attn_decode_static(cache, q, k, v, sinks, window, sm_scale, cos=None, sin=No
     if return_lse and lse is None:
         lse = torch.empty((B, n_q, T), dtype=torch.float32, device=q.device)
     a = _args(cache, q, k, v, sinks, window, sm_scale, cos, sin, rope_fused, out, lse)
-    _check(lib().sa_attn_decode_static(ctypes.byref(cache.raw), ctypes.byref(a), _stream(q)),
+    _check(lib().sa_attn_decode_static(ctypes.byref(cache.raw), ctypes.byref(a), _raw_stream(q)),
            "sa_attn_decode_static")
     return (out, lse) if return_lse else out
 

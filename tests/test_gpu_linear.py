@@ -25,7 +25,7 @@ from oracle import linear as olin
 from oracle import rope as orope
 from sink_augmented_gqa_b200 import workloads as wl
 
-from helpers import check_bf16_output, oracle_tables, to64
+from helpers import check_bf16_output, oracle_attend, oracle_tables, to64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -207,7 +207,7 @@ def test_attention_layer_composition(cuda_device):
     _check(qkv, ref_qkv, s_abs, 2.0 ** -9 + 2.0 ** -12, "layer: qkv")
     qq, kk, vv = olin.split_qkv(to64(qkv), n_q, n_kv, d)
     oc = okv.KVCache(1, T, n_kv, d)
-    ref_o, _ = oatt.attend_step(oc, qq[None], kk[None], vv[None], to64(sinks), 0, cfg.sm_scale, rc, rs)
+    ref_o, _ = oracle_attend(oc, qq[None], kk[None], vv[None], to64(sinks), 0, cfg.sm_scale, rc, rs)
     check_bf16_output(o, ref_o, "layer: attention")
     ref_x = olin.out_proj(to64(o.view(T, n_q * d)), to64(wo), to64(bo), to64(x))
     s_abs_o = np.abs(to64(o.view(T, n_q * d))) @ np.abs(to64(wo)).T

@@ -25,7 +25,7 @@ from oracle import bf16 as obf16
 from oracle import rope as orope
 from sink_augmented_gqa_b200 import workloads as wl
 
-from helpers import check_bf16_output, check_lse, oracle_tables, to64
+from helpers import OracleOut, check_bf16_output, check_lse, oracle_tables, stack_out, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -62,9 +62,10 @@ class _OracleUnit:
     def row(self, q_raw, pos, sink, window, sm_scale, rc, rs):
         """Output and lse of one query row (raw [d]) at position pos."""
         qr = orope.rotate_bsh(q_raw[None, None, None], pos, rc, rs)
-        out, lse = oatt.sink_attention(qr, self.K[None, :pos + 1, None], self.V[None, :pos + 1, None],
-                                       np.array([sink]), pos, window, sm_scale)
-        return out[0, 0, 0], lse[0, 0, 0]
+        K, V = self.K[None, :pos + 1, None], self.V[None, :pos + 1, None]
+        out, lse = oatt.sink_attention(qr, K, V, np.array([sink]), pos, window, sm_scale)
+        vabs, _ = oatt.sink_attention(qr, K, np.abs(V), np.array([sink]), pos, window, sm_scale)
+        return OracleOut(out[0, 0, 0], vabs[0, 0, 0]), lse[0, 0, 0]
 
 
 @pytest.mark.parametrize("layer", [0, 1], ids=["band", "full"])
@@ -102,7 +103,7 @@ def test_long_decode_all_64_steps(cuda_device, layer):
             got.append(out[0, 0, h])
             want.append(ro)
             check_lse(lse[0, h, 0], np.array(rl), f"long decode step {st} h{h}")
-        check_bf16_output(torch.stack(got), np.stack(want), f"long decode step {st}")
+        check_bf16_output(torch.stack(got), stack_out(want), f"long decode step {st}")
     assert cache.offset == off + steps
     n_cnt = cfg.B * cfg.n_kv   # the split tickets end every call at zero
     assert torch.count_nonzero(ws[: 4 * n_cnt]) == 0
@@ -140,7 +141,7 @@ def test_handoff_chunk_then_all_32_steps(cuda_device, layer):
                 ro, _ = u.row(to64(q[b, i, h]), off + i, sk[h], window, cfg.sm_scale, rc, rs)
                 got.append(out[b, i, h])
                 want.append(ro)
-    check_bf16_output(torch.stack(got), np.stack(want), "handoff chunk sampled rows")
+    check_bf16_output(torch.stack(got), stack_out(want), "handoff chunk sampled rows")
     del q, k, v, out
     ws = sa.decode_workspace(cfg.B, cfg.n_q, cfg.n_kv, cfg.d, device=DEV)
     for st in range(steps):
@@ -159,5 +160,5 @@ def test_handoff_chunk_then_all_32_steps(cuda_device, layer):
                 got.append(dec[b, 0, h])
                 want.append(ro)
                 check_lse(lse[b, h, 0], np.array(rl), f"handoff step {st} b{b} h{h}")
-        check_bf16_output(torch.stack(got), np.stack(want), f"handoff decode step {st}")
+        check_bf16_output(torch.stack(got), stack_out(want), f"handoff decode step {st}")
     assert cache.offset == off + T + steps

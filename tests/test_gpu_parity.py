@@ -18,7 +18,7 @@ from oracle import rope as orope
 from sink_augmented_gqa_b200 import workloads as wl
 
 from helpers import (check_bf16_output, check_lse, oracle_cache, oracle_rows, oracle_step,
-                      oracle_tables, to64)
+                      oracle_tables, stack_out, to64)
 
 pytestmark = pytest.mark.gpu
 
@@ -487,7 +487,7 @@ def _sampled_prefill(cfg, layer, n_rows=6, n_heads=3, seed=0):
         for (i, h), (ro, _) in res.items():
             got.append(out[b, i, h])
             want.append(ro)
-    check_bf16_output(torch.stack(got), np.stack(want), f"{cfg.name} sampled rows")
+    check_bf16_output(torch.stack(got), stack_out(want), f"{cfg.name} sampled rows")
 
 
 @pytest.mark.parametrize("layer", [0, 1], ids=["band", "full"])
@@ -527,7 +527,7 @@ def test_full_size_long_decode(cuda_device, layer):
         got.append(out[0, 0, h])
         want.append(ro)
         check_lse(lse[0, h, 0], np.array(rl), f"long decode h{h}")
-    check_bf16_output(torch.stack(got), np.stack(want), "long decode sampled heads")
+    check_bf16_output(torch.stack(got), stack_out(want), "long decode sampled heads")
     torch.cuda.synchronize()
     assert cache.offset == off + 1
 
@@ -563,4 +563,4 @@ def test_full_size_handoff_sampled(cuda_device):
                 got.append(dec[b, 0, h])
                 want.append(r[(cfg.T, 0)][0])
         del cache, kp, vp
-    check_bf16_output(torch.stack(got), np.stack(want), "handoff sampled rows")
+    check_bf16_output(torch.stack(got), stack_out(want), "handoff sampled rows")
