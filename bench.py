@@ -794,6 +794,62 @@ def oracle_sample(budget_s=12.0, min_units=1):
     return pre_f / pre_t / 1e12, dec_b / dec_t / 1e9, threads, desc
 
 
+def oracle_configs(budget_s=4.0):
+    """The fp64 oracle on a bounded sample of every configuration, on the host
+    cores: whole (sequence, query head) units of a call -- the prefill of the
+    configuration's prompt rows (both layer types), or one decode row against
+    the pre-filled cache -- until the budget is spent. Returns one entry per
+    configuration and layer type: TFLOP/s (prefill) or KV GB/s (decode) and
+    the sample."""
+    from oracle import attention as oatt
+    from oracle import kvcache as okv
+    from oracle import yarn as oyarn
+    res = {}
+    for name in ("tiny", "lite", "gptoss_prefill", "long_decode", "handoff"):
+        cfg = wl.CONFIGS[name]
+        y = cfg.yarn
+        one = wl.scaled(cfg, B=1)
+        T = cfg.T if cfg.T else 1
+        off = cfg.offset
+        cos, sin = oyarn.stored_tables(off + T, cfg.d, y["theta"], y["scaling"], y["orig_ctx"], y["alpha"],
+                                       y["beta"])
+        kp = vp = None
+        if off:
+            kp, vp = wl.prefilled_cache_rows(one, layer=1)
+        for layer in (1, 0):
+            w = cfg.layer_window(layer)
+            q, k, v = wl.qkv(one, T, layer=layer)
+            q, k, v = (x.to(torch.float64).numpy() for x in (q, k, v))
+            sinks = wl.sinks(cfg, layer).double().numpy()
+            units, work = 0, 0
+            t0 = time.perf_counter()
+            while True:
+                h = units % cfg.n_q
+                g = h // cfg.q_mult
+                c = okv.KVCache(1, off + T, 1, cfg.d)
+                if off:
+                    c.append(kp[:, :, g:g + 1].to(torch.float64).numpy(), vp[:, :, g:g + 1].to(torch.float64).numpy())
+                oatt.attend_step(c, q[:, :, h:h + 1], k[:, :, g:g + 1], v[:, :, g:g + 1], sinks[h:h + 1], w,
+                                 cfg.sm_scale, cos, sin)
+                units += 1
+                if cfg.T:
+                    work += 4 * cfg.d * pairs(off, T, w)
+                else:
+                    work += decode_rows(off, w) * cfg.d * 2 * 2
+                if time.perf_counter() - t0 >= budget_s:
+                    break
+            dt = time.perf_counter() - t0
+            key = f"{name}/{'full' if w == 0 else 'band'}"
+            if cfg.T:
+                res[key] = {"TFLOP/s": work / dt / 1e12, "units": units,
+                            "sample": f"{units} (sequence, head) units of the {T}-row prefill"
+                                      + (f" at offset {off}" if off else "") + f", {dt:.1f} s"}
+            else:
+                res[key] = {"KV_GB/s": work / dt / 1e9, "units": units,
+                            "sample": f"{units} (sequence, head) decode rows against {off} cached rows, {dt:.1f} s"}
+    return res
+
+
 def step_config(cfg, world, parallelism):
     """The bench step's workload, the same for both arms."""
     return {"workload": "prefill-to-decode handoff (the largest configuration): B=16 sequences sharing cache "
@@ -957,6 +1013,8 @@ def main():
     ap.add_argument("--impl", default="libsinkattn", choices=["libsinkattn", "reference"])
     ap.add_argument("--no-extras", action="store_true", help="skip the secondary measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--oracle-table", action="store_true",
+                    help="only time the oracle on a sample of every configuration (host cores) and print it")
     ap.add_argument("--profile-case", choices=PROFILE_CASES, default=None,
                     help="only run this call warmup+steps times (for profilers); prints no bench line")
     args = ap.parse_args()
@@ -968,6 +1026,11 @@ def main():
     dist = None
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.oracle_table:
+        if rank == 0:
+            cores = int(os.environ.get("OMP_NUM_THREADS", "0")) or os.cpu_count()
+            print(json.dumps({"oracle_table": oracle_configs(), "cores": cores}), flush=True)
         return
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)

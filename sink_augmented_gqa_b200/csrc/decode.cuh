@@ -377,18 +377,6 @@ __device__ __forceinline__ void decode_subtile_f8(uint32_t kst, uint32_t vst, ui
   }
 }
 
-// Programmatic dependent launch: a kernel launched with programmatic stream
-// serialization may start while the kernel before it in the stream is still
-// running; griddep_wait() returns once that kernel has completed and its
-// memory operations are visible (at once when the launch had no such
-// predecessor), so nothing before it may read memory another kernel writes.
-// griddep_launch_dependents() lets the next such kernel be scheduled before
-// this one has finished.
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // tmK/tmV: the cache's K/V (bf16 elements, or FP8 code bytes); tmKS/tmVS
 // (FP8 only): the row scales, dims {rows, n_kv, B, 1}, box {R, 1, 1, 1}.
 template <int D, bool F8>

@@ -340,6 +340,10 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Launched behind the staging kernel with programmatic stream
+  // serialization: the set-up above overlaps its tail; nothing below may read
+  // memory before it has completed (the staged queries, the appended rows).
+  griddep_wait();
 
   if (warp < 4) {
     // Warpgroup 0: producer (warp 0), MMA issuers (warps 1, 2). It gives

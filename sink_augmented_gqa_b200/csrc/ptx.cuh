@@ -455,6 +455,18 @@ __device__ __forceinline__ void rope_pair2(uint32_t& w1, uint32_t& w2, float c0,
   }
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the kernel before it in the stream is still
+// running; griddep_wait() returns once that kernel has completed and its
+// memory operations are visible (at once when the launch had no such
+// predecessor), so nothing before it may read memory another kernel writes.
+// griddep_launch_dependents() lets the next such kernel be scheduled before
+// this one has finished.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Byte offset of element (row, col) in a tile stored as column blocks of
 // `CB` bf16 elements, each block [rows][CB] with the hardware swizzle
 // (bits [4, 4+b) of the address XOR bits [7, 7+b); b = 3 for 128-byte rows,

@@ -135,7 +135,10 @@ __global__ void kv_append_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat16* 
 // Prefill staging, one launch: the kv_append_kernel work for the call's K/V
 // rows, then (stage_q) each query row rotated at its position off + t into
 // qo [B][T][n_q][d] (strides os*), from which the attention kernel reads its
-// query tiles. One thread per (row, 8-pair chunk); K/V units first.
+// query tiles. One thread per (row, 8-pair chunk); K/V units first. The
+// attention kernel, launched behind this one with programmatic stream
+// serialization, may be scheduled as soon as every block of this launch has
+// started.
 __global__ void prefill_stage_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat16* __restrict__ cv,
                                      int cap, const __nv_bfloat16* __restrict__ k, long long ks0,
                                      long long ks1, long long ks2, const __nv_bfloat16* __restrict__ v,
@@ -145,6 +148,7 @@ __global__ void prefill_stage_kernel(__nv_bfloat16* __restrict__ ck, __nv_bfloat
                                      const __nv_bfloat16* q, long long qs0, long long qs1,
                                      long long qs2, int n_q, __nv_bfloat16* qo, long long os0,
                                      long long os1, long long os2, int stage_q, int ring) {
+  griddep_launch_dependents();
   const int half = d / 2, chunks = half / 8;
   const long long n_kv_units = (long long)B * T * n_kv * chunks;
   const long long n = n_kv_units + (stage_q ? (long long)B * T * n_q * chunks : 0);

@@ -336,7 +336,7 @@ sa_status with_sched_slot(cudaStream_t s, F&& launch) {
 }
 
 template <int D>
-sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream_t stream) {
+sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, int slot, cudaStream_t stream) {
   using Cfg = PrefillCfg<D>;
   CUtensorMap tmQ, tmK, tmV;
   // a ring exposes all of its rows (positions outside the band are masked)
@@ -387,11 +387,22 @@ sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, cudaStream
   // persistent: one CTA per SM (or per item when there are fewer)
   const long long n_items = (long long)p.n_pairs * a->n_q * a->B;
   const int grid = (int)(n_items < num_sms() ? n_items : num_sms());
-  return with_sched_slot(stream, [&](int slot) {
-    p.sched_slot = slot;
-    sa::prefill_kernel<D><<<grid, Cfg::NUM_THREADS, Cfg::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, tmO, p);
-    return last_launch_status();
-  });
+  p.sched_slot = slot;
+  // Programmatic stream serialization: the kernel's set-up overlaps the tail
+  // of the staging launch before it; it waits for that launch to complete
+  // before its first global access.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(Cfg::NUM_THREADS);
+  lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  lc.stream = stream;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&lc, sa::prefill_kernel<D>, tmQ, tmK, tmV, tmO, p);
+  return (last_launch_status() == SA_OK && e == cudaSuccess) ? SA_OK : SA_ERR_CUDA;
 }
 
 struct DecodeSplit {
@@ -877,21 +888,27 @@ sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* a, sa_stream_t
   if (cache->kv_dtype != SA_KV_BF16) return SA_ERR_UNSUPPORTED;
   if (a->T == 0) return SA_OK;
   cudaStream_t s = (cudaStream_t)stream;
-  // one launch: the call's K rows rotated (when RoPE is fused) and appended
-  // with V, and the rotated queries staged in `out`
-  st = launch_stage(cache, a, a->rope_fused, s);
-  if (st != SA_OK) return st;
-  cudaEvent_t ev0 = g_prefill_ev_before, ev1 = g_prefill_ev_after;
-  if (ev0 != nullptr && cudaEventRecord(ev0, s) != cudaSuccess) return SA_ERR_CUDA;
-  switch (cache->d) {
-    case 64: st = launch_prefill<64>(cache, a, s); break;
-    case 96: st = launch_prefill<96>(cache, a, s); break;
-    case 128: st = launch_prefill<128>(cache, a, s); break;
-    default: return SA_ERR_SHAPE;
-  }
-  if (ev1 != nullptr && cudaEventRecord(ev1, s) != cudaSuccess) return SA_ERR_CUDA;
-  // The append is enqueued either way; the offset follows it.
-  note_append(cache, cache->offset, a->T);
+  bool staged = false;
+  // The schedule slot (and the wait for its previous user) is taken before
+  // the staging launch, so nothing stands between the two kernels.
+  st = with_sched_slot(s, [&](int slot) -> sa_status {
+    // one launch: the call's K rows rotated (when RoPE is fused) and appended
+    // with V, and the rotated queries staged in `out`
+    sa_status r = launch_stage(cache, a, a->rope_fused, s);
+    if (r != SA_OK) return r;
+    staged = true;
+    cudaEvent_t ev0 = g_prefill_ev_before, ev1 = g_prefill_ev_after;
+    if (ev0 != nullptr && cudaEventRecord(ev0, s) != cudaSuccess) return SA_ERR_CUDA;
+    switch (cache->d) {
+      case 64: r = launch_prefill<64>(cache, a, slot, s); break;
+      case 96: r = launch_prefill<96>(cache, a, slot, s); break;
+      default: r = launch_prefill<128>(cache, a, slot, s); break;
+    }
+    if (ev1 != nullptr && cudaEventRecord(ev1, s) != cudaSuccess) return SA_ERR_CUDA;
+    return r;
+  });
+  // Once the append is enqueued the offset follows it.
+  if (staged) note_append(cache, cache->offset, a->T);
   return st;
 }
 
