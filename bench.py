@@ -894,13 +894,41 @@ def run_reference(args, rank, world):
 # Single-call loops for profilers (ncu): no timing, no output but a summary
 # ---------------------------------------------------------------------------
 
-PROFILE_CASES = ("handoff_prefill_full", "handoff_prefill_full_b4", "handoff_prefill_band",
+PROFILE_CASES = ("handoff_prefill_full", "handoff_prefill_full_b4", "handoff_prefill_band", "handoff_decode_full_b4",
                  "gptoss_prefill_full", "gptoss_prefill_band", "lite_prefill_full", "long_decode_full",
                  "long_decode_fp8", "gptoss_qkv_proj", "gptoss_out_proj", "lite_backward_b2")
 
 
 def profile_case(name, dev, steps, warmup):
     import sink_augmented_gqa_b200 as sa
+    if name == "handoff_decode_full_b4":
+        # a decode step of the handoff's full layer after the chunk (position
+        # 66,048: 66,049 rows read per sequence), for 4 of the 16 sequences
+        cfg = wl.scaled(wl.CONFIGS["handoff"], B=4)
+        off = cfg.offset + cfg.T
+        y = cfg.yarn
+        cos, sin = sa.yarn_rope_tables(off + 1, cfg.d, y["theta"], y["scaling"], y["orig_ctx"], y["alpha"],
+                                       y["beta"], device=dev)
+        cache = sa.KVCache(cfg.B, off + 1, cfg.n_kv, cfg.d, device=dev)
+        kp, vp = wl.prefilled_cache_rows(cfg, layer=1, device=dev, rows=off)
+        cache.append(kp, vp)
+        del kp, vp
+        snap = cache.snapshot()
+        q, k, v = wl.qkv(cfg, 1, layer=1, step=1, device=dev)
+        sinks = wl.sinks(cfg, 1, device=dev)
+        ws = sa.decode_workspace(cfg.B, cfg.n_q, cfg.n_kv, cfg.d, device=dev)
+        out = torch.empty((cfg.B, 1, cfg.n_q, cfg.d), dtype=torch.bfloat16, device=dev)
+
+        def once():
+            cache.restore(snap)
+            sa.attn_decode(cache, q, k, v, sinks, 0, cfg.sm_scale, cos, sin, workspace=ws, out=out)
+        units = cfg.B * (off + 1) * kv_row_bytes(cfg)
+        for _ in range(warmup + steps):
+            once()
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_case": name, "launches": warmup + steps,
+                          "algorithmic_units_per_launch": units, "unit": "bytes"}))
+        return
     if name.startswith("handoff"):
         # the chunk prefill at offset 65,536 (b4: 4 of the 16 sequences, a
         # capture-sized case with the same items -- 64 heads x 2 row-tile
