@@ -564,3 +564,36 @@ def test_full_size_handoff_sampled(cuda_device):
                 want.append(r[(cfg.T, 0)][0])
         del cache, kp, vp
     check_bf16_output(torch.stack(got), stack_out(want), "handoff sampled rows")
+
+
+def test_many_prefills_in_flight_on_several_streams(cuda_device):
+    # More prefill calls in flight than the library has schedule counters for
+    # eager launches (64): four streams, 24 calls each, issued without
+    # synchronising, so counters are reused while other streams' calls may
+    # still run. Every output must equal the one the same call gives alone.
+    cfg = wl.scaled(wl.CONFIGS["tiny"], B=1, n_q=8, n_kv=2, d=64)
+    T, n_streams, per_stream = 384, 4, 24
+    cos, sin = _tables(cfg, T)
+    sinks = wl.sinks(cfg).to(DEV)
+    inputs = [tuple(t.to(DEV) for t in wl.qkv(cfg, T, step=i)) for i in range(n_streams)]
+    ref = []
+    for i in range(n_streams):
+        c = sa.KVCache(cfg.B, T, cfg.n_kv, cfg.d, device=DEV)
+        ref.append(sa.attn_prefill(c, *inputs[i], sinks, 0, cfg.sm_scale, cos, sin))
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in range(n_streams)]
+    caches = [sa.KVCache(cfg.B, T, cfg.n_kv, cfg.d, device=DEV) for _ in range(n_streams)]
+    snaps = [c.snapshot() for c in caches]
+    outs = [[torch.empty_like(ref[i]) for _ in range(per_stream)] for i in range(n_streams)]
+    for s in streams:
+        s.wait_stream(torch.cuda.current_stream())
+    for j in range(per_stream):
+        for i, s in enumerate(streams):
+            with torch.cuda.stream(s):
+                caches[i].restore(snaps[i])
+                sa.attn_prefill(caches[i], *inputs[i], sinks, 0, cfg.sm_scale, cos, sin, out=outs[i][j])
+    torch.cuda.synchronize()
+    assert sa.device_status() == "SA_OK"
+    for i in range(n_streams):
+        for j in range(per_stream):
+            assert torch.equal(outs[i][j], ref[i]), (i, j)
