@@ -289,6 +289,11 @@ sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* args, sa_strea
  * row quantised; queries enter the QK product as f16 after an exact
  * per-head power-of-two scaling, and the scaled softmax weights enter the PV
  * product as f16.
+ * The rows are shared out among the CTAs of each (sequence, KV head) at run
+ * time (the CTAs that stream faster take more), so the fp32 partial sums are
+ * grouped differently from call to call: two identical calls can differ in
+ * the last bit of an output, each within the same rounding of the exact
+ * value.
  * workspace: device memory of at least sa_attn_decode_workspace_size()
  *   bytes, caller-owned, ZERO-FILLED before its first use; the kernel leaves
  *   it zeroed again on completion. Calls that share a workspace must not

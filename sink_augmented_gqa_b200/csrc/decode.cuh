@@ -1,8 +1,12 @@
 // One-token sink-augmented GQA decode, split across SMs.
 //
 // The work is reading the KV cache once: for each (sequence b, KV head g)
-// the rows [lo, off) are cut into S contiguous splits, one CTA each
-// (grid n_kv x S x B). Inside a CTA one producer warp streams 128-row K and V
+// the rows [lo, off) are cut into stages of R rows, streamed by S CTAs
+// (grid n_kv x S x B): each CTA first takes a contiguous run of stages of its
+// own (about half of its share, prefetched into L2 before the kernel ahead
+// of it has finished), then asks a per-(b, g) counter for one more stage at
+// a time until none is left, so CTAs that happen to stream faster do more
+// and all of them finish together. Inside a CTA one producer warp streams 128-row K and V
 // tiles of head g from the cache with TMA (128-byte swizzled smem, rows past
 // `off` read as zeros) through a ring, and eight consumer warps each take
 // 16 rows of every tile. A consumer computes S^T = K Q^T for the q_mult <= 8
@@ -16,9 +20,10 @@
 // a cache row written in the same launch.
 //
 // Partials (m, l, O) of the eight warps are merged in smem; with S > 1 each
-// CTA writes its partial to the workspace and the last CTA of (b, g) to
-// finish (atomic ticket, no spinning) merges all S of them and folds in the
-// sink: M = max(max_s m_s, sink), l = sum_s e^{m_s-M} l_s + e^{sink-M},
+// CTA writes its partial to the workspace as one record and the last CTA of
+// (b, g) to finish (atomic ticket, no spinning) brings all S records into its
+// idle K/V ring with one bulk copy and merges them with the sink:
+// M = max(max_s m_s, sink), l = sum_s e^{m_s-M} l_s + e^{sink-M},
 // out = sum_s e^{m_s-M} O_s / l.
 //
 // FP8 caches (decode_kernel<D, true>) store e4m3 codes plus one fp32 scale
@@ -62,16 +67,19 @@ struct DecodeParams {
   long long lo;     // first cache position of split 0's first stage
   long long lo_mask;  // first cache position attended (keys before it masked)
   int ring_cap;     // 0: row = position; > 0: ring cache, row = position mod ring_cap
-  long long chunk;  // cache rows per split (multiple of 128)
+  long long n_blocks;  // stages of R rows from lo to off (each (b, g) streams all of them)
+  int static_stages;   // split s first takes stages [s F, s F + F); stages from S F on are
+                       // handed out one at a time by ws_grab[b][g] to whichever CTA asks first
   float* cks;       // FP8 caches: row scales [B][n_kv][cap] of K and of V
   float* cvs;
   int S;
+  int pf_stages;    // stages each CTA prefetches into L2 before waiting for its predecessor
   float scale_log2;
   int rope;
-  float* ws_o;  // [B][n_kv][S][q_mult][D] (16-byte aligned rows)
-  float* ws_m;  // [B][n_kv][S][q_mult]
-  float* ws_l;  // [B][n_kv][S][q_mult]
-  int* ws_cnt;  // [B][n_kv]
+  float* ws_rec;   // [B][n_kv][S] records of rec_floats: O [q_mult][D], m [q_mult], l [q_mult]
+  int rec_floats;  // q_mult * D + (2 q_mult rounded up to a multiple of 4): 16-byte records
+  int* ws_cnt;     // [B][n_kv] split tickets
+  int* ws_grab;    // [B][n_kv] next dynamic stage (both end every call at zero)
 };
 
 template <int D>
@@ -96,8 +104,14 @@ struct DecodeCfg {
   static constexpr uint32_t OFF_RED = OFF_K;
   static constexpr uint32_t RED_WARP = (16 + 8 * D) * 4;
   static_assert(NCW * RED_WARP <= 2 * NS * STAGE_BYTES, "warp partials must fit in the ring");
+  static constexpr uint32_t RING_BYTES = 2 * NS * STAGE_BYTES;   // K and V stages
   static constexpr uint32_t OFF_BAR = OFF_XV + XTILE;
-  static constexpr uint32_t SMEM_BYTES = OFF_BAR + 8 * (2 * NS) + 16 + 1024;
+  // after the 2 NS ring barriers: the merge barrier, two flags, the sinks
+  static constexpr uint32_t OFF_MBAR = OFF_BAR + 8 * (2 * NS);
+  static constexpr uint32_t OFF_FLAG = OFF_MBAR + 8;
+  static constexpr uint32_t OFF_SINK = OFF_FLAG + 16;
+  static constexpr uint32_t OFF_SROW = OFF_SINK + 32;   // [NS] first cache position of each stage
+  static constexpr uint32_t SMEM_BYTES = OFF_SROW + 8 * NS + 1024;
   static constexpr int BLKCOLS = CB;                    // tensor-map columns per column block
   static constexpr uint32_t STAGE_TX = 2 * STAGE_BYTES;  // bytes one stage's TMA loads bring
   static constexpr int RW = 16;                         // rows per consumer warp per stage
@@ -140,8 +154,13 @@ struct DecodeF8Cfg {
   static constexpr uint32_t RED_WARP = (16 + 8 * D) * 4;
   static_assert(NCW * RED_WARP <= 2 * NS * STAGE_BYTES, "warp partials must fit in the ring");
   static_assert(OFF_XK % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+  static constexpr uint32_t RING_BYTES = 2 * NS * STAGE_BYTES;   // K and V codes
   static constexpr uint32_t OFF_BAR = OFF_XS + 128;
-  static constexpr uint32_t SMEM_BYTES = OFF_BAR + 8 * (2 * NS) + 16 + 1024;
+  static constexpr uint32_t OFF_MBAR = OFF_BAR + 8 * (2 * NS);
+  static constexpr uint32_t OFF_FLAG = OFF_MBAR + 8;
+  static constexpr uint32_t OFF_SINK = OFF_FLAG + 16;
+  static constexpr uint32_t OFF_SROW = OFF_SINK + 32;   // [NS] first cache position of each stage
+  static constexpr uint32_t SMEM_BYTES = OFF_SROW + 8 * NS + 1024;
 };
 
 template <int D, bool F8>
@@ -377,6 +396,56 @@ __device__ __forceinline__ void decode_subtile_f8(uint32_t kst, uint32_t vst, ui
   }
 }
 
+// The query words (bf16 pairs) one lane of a consumer warp holds as MMA
+// B-fragment registers: word j covers dims base(j) + lane_off + {0, 1}, with
+// lane_off = 2 (lane % 4) for a bf16 cache and 4 (lane % 4) for FP8. Every
+// dim below D/2 and its RoPE partner (+ D/2) sit in the same lane, in words
+// j and partner(j).
+template <int D, bool F8>
+struct QWords {
+  static constexpr int NW = D / 8;
+  __host__ __device__ static constexpr int base(int j) {
+    return F8 ? 32 * (j >> 2) + 16 * (j & 1) + 2 * ((j >> 1) & 1) : 16 * (j >> 1) + 8 * (j & 1);
+  }
+  __host__ __device__ static constexpr int partner(int j) {
+    if (base(j) >= D / 2) return -1;
+    for (int k = 0; k < NW; ++k)
+      if (base(k) == base(j) + D / 2) return k;
+    return -2;
+  }
+  __host__ __device__ static constexpr bool closed() {
+    for (int j = 0; j < NW; ++j)
+      if (partner(j) == -2) return false;
+    return true;
+  }
+  static_assert(closed(), "every lower-half query dim has its RoPE partner in the same lane");
+};
+
+// Loads one lane's query words and rotates them at the table row given by
+// ctab/stab (correctly rounded bf16, rope_pair2). All loads are issued before
+// the first is used.
+template <int D, bool F8>
+__device__ __forceinline__ void load_q_words(const __nv_bfloat16* qrow, int lane_off, const float* ctab,
+                                             const float* stab, int rope, uint32_t (&w)[D / 8]) {
+  using QW = QWords<D, F8>;
+#pragma unroll
+  for (int j = 0; j < QW::NW; ++j) w[j] = *reinterpret_cast<const uint32_t*>(qrow + QW::base(j) + lane_off);
+  if (rope) {
+    float2 cs[QW::NW], sn[QW::NW];
+#pragma unroll
+    for (int j = 0; j < QW::NW; ++j) {
+      if (QW::partner(j) >= 0) {
+        cs[j] = *reinterpret_cast<const float2*>(ctab + QW::base(j) + lane_off);
+        sn[j] = *reinterpret_cast<const float2*>(stab + QW::base(j) + lane_off);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < QW::NW; ++j) {
+      if (QW::partner(j) >= 0) rope_pair2(w[j], w[QW::partner(j)], cs[j].x, cs[j].y, sn[j].x, sn[j].y);
+    }
+  }
+}
+
 // tmK/tmV: the cache's K/V (bf16 elements, or FP8 code bytes); tmKS/tmVS
 // (FP8 only): the row scales, dims {rows, n_kv, B, 1}, box {R, 1, 1, 1}.
 template <int D, bool F8>
@@ -392,8 +461,12 @@ __global__ void __launch_bounds__(288, 2)
   const uint32_t bar0 = sbase + C::OFF_BAR;
   auto full_bar = [&](int s) -> uint32_t { return bar0 + 8u * (uint32_t)s; };
   auto empty_bar = [&](int s) -> uint32_t { return bar0 + 8u * (uint32_t)(C::NS + s); };
-  volatile int* flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * 2 * C::NS);
+  const uint32_t merge_bar = sbase + C::OFF_MBAR;
+  volatile int* flag = reinterpret_cast<volatile int*>(smem + C::OFF_FLAG);
   // flag[0]: abort, flag[1]: "this CTA merges the splits"
+  float* sink_sm = reinterpret_cast<float*>(smem + C::OFF_SINK);   // [q_mult] sinks, log2 units
+  // position of each ring slot's first row, or -1: the producer has no more stages
+  volatile long long* srow = reinterpret_cast<volatile long long*>(smem + C::OFF_SROW);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -403,10 +476,12 @@ __global__ void __launch_bounds__(288, 2)
   const int QM = p.q_mult;
   constexpr int HALF = D / 2;
 
-  const long long r_begin = p.lo + (long long)split * p.chunk;
-  long long r_end = r_begin + p.chunk;
-  if (r_end > p.off) r_end = p.off;
-  const int n_stages = r_end > r_begin ? (int)((r_end - r_begin + C::R - 1) / C::R) : 0;
+  // Stages (R rows from position lo + sidx R) of this (b, g): the split's
+  // static ones first, then dynamic ones while any are left, so CTAs that
+  // stream faster take more and all of them finish at about the same time.
+  const int F = p.static_stages;
+  const long long s_begin = (long long)split * F;
+  const bool dyn = (long long)p.S * F < p.n_blocks;
   const bool last_split = split == p.S - 1;
 
   // The next layer's launch may take this CTA's slot as soon as it frees up;
@@ -417,9 +492,60 @@ __global__ void __launch_bounds__(288, 2)
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), C::NCW);
     }
+    mbar_init(merge_bar, 1);
     flag[0] = 0;
     flag[1] = 0;
     fence_barrier_init();
+  }
+  // The first stages of this split go into L2 while the kernel before this
+  // one is still draining (its tail, or a short band layer). A prefetch
+  // brings nothing into the SM, so it is safe even if that kernel writes
+  // some of these rows: L2 is where its writes land.
+  if (warp == C::NCW && lane == 0 && p.n_blocks > 0) {
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    if constexpr (F8) {
+      tma_prefetch_desc(&tmKS);
+      tma_prefetch_desc(&tmVS);
+    }
+    const int pf = F < p.pf_stages ? F : p.pf_stages;
+    for (int it = 0; it < pf; ++it) {
+#pragma unroll
+      for (int bx = 0; bx < C::NBOX; ++bx) {
+        const long long pos = p.lo + (s_begin + it) * C::R + 128 * bx;
+        const int row = (int)(p.ring_cap > 0 ? pos % p.ring_cap : pos);
+#pragma unroll
+        for (int cb = 0; cb < C::NCB; ++cb) {
+          tma_prefetch_l2_4d(&tmK, cb * C::BLKCOLS, row, g, b);
+          tma_prefetch_l2_4d(&tmV, cb * C::BLKCOLS, row, g, b);
+        }
+        if constexpr (F8) {
+          tma_prefetch_l2_4d(&tmKS, row, g, b, 0);
+          tma_prefetch_l2_4d(&tmVS, row, g, b, 0);
+        }
+      }
+    }
+  }
+  // The small inputs the consumers read first (the group's query rows, the
+  // RoPE table rows at `off`, the sinks, the new K/V row) go into L2 too:
+  // lane i of warp 0 takes the i-th 128-byte line of that list.
+  if (warp == 0) {
+    constexpr int LPR = (D * 2 + 127) / 128;   // lines per bf16 row
+    const int QM_ = p.q_mult;
+    const char* a = nullptr;
+    int i = lane;
+    if (i < QM_ * LPR) {
+      a = reinterpret_cast<const char*>(p.q + b * p.qs0 + (long long)(g * QM_ + i / LPR) * p.qs2) + 128 * (i % LPR);
+    } else if ((i -= QM_ * LPR) < 2 * LPR) {
+      if (p.rope) a = reinterpret_cast<const char*>((i < LPR ? p.cos_t : p.sin_t) + p.off * (D / 2)) + 128 * (i % LPR);
+    } else if ((i -= 2 * LPR) < 2 * LPR) {
+      if (split == p.S - 1)
+        a = reinterpret_cast<const char*>(i < LPR ? p.k + b * p.ks0 + (long long)g * p.ks2
+                                                  : p.v + b * p.vs0 + (long long)g * p.vs2) + 128 * (i % LPR);
+    } else if (i == 2 * LPR) {
+      if (p.sinks) a = reinterpret_cast<const char*>(p.sinks + g * QM_);
+    }
+    if (a) prefetch_l2(a);
   }
   __syncthreads();
   // Everything below reads or writes global memory (q, the cache, the split
@@ -428,22 +554,29 @@ __global__ void __launch_bounds__(288, 2)
 
   if (warp == C::NCW) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n_stages > 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      if constexpr (F8) {
-        tma_prefetch_desc(&tmKS);
-        tma_prefetch_desc(&tmVS);
-      }
-      int issued = 0;
-      for (int it = 0; it < n_stages; ++it) {
+    if (lane == 0) {
+      int* grab = p.ws_grab + (b * p.n_kv + g);
+      int pending = dyn ? atomicAdd(grab, 1) : 0;   // the first dynamic stage, asked for early
+      int it = 0;
+      for (int k = 0; !flag[0]; ++k) {
+        long long sidx;
+        if (k < F) {
+          sidx = s_begin + k;
+        } else {
+          if (!dyn) break;
+          sidx = (long long)p.S * F + pending;
+          if (sidx >= p.n_blocks) break;
+          pending = atomicAdd(grab, 1);   // the next one, in flight while this stage loads
+        }
         const int s = it % C::NS;
         if (!mbar_wait(empty_bar(s), (uint32_t)(((it / C::NS) & 1) ^ 1))) { flag[0] = 1; break; }
+        const long long pos0 = p.lo + sidx * C::R;
+        srow[s] = pos0;
         mbar_arrive_expect_tx(full_bar(s), C::STAGE_TX);
 #pragma unroll
         for (int bx = 0; bx < C::NBOX; ++bx) {
           // boxes of 128 rows: none wraps a ring (ring stages start on multiples of 128)
-          const long long pos = r_begin + (long long)it * C::R + 128 * bx;
+          const long long pos = pos0 + 128 * bx;
           const int row = (int)(p.ring_cap > 0 ? pos % p.ring_cap : pos);
           const uint32_t boff = (uint32_t)bx * 128u * (C::BLOCK_BYTES / C::R);
 #pragma unroll
@@ -460,98 +593,126 @@ __global__ void __launch_bounds__(288, 2)
             tma_load_4d(sbase + C::OFF_VS + s * C::R * 4 + bx * 512, &tmVS, full_bar(s), row, g, b, 0);
           }
         }
-        issued = it + 1;
-        if (flag[0]) break;
+        ++it;
+      }
+      // the end of this CTA's stream: a slot marked -1, completed by a plain arrive
+      if (!flag[0]) {
+        const int s = it % C::NS;
+        if (mbar_wait(empty_bar(s), (uint32_t)(((it / C::NS) & 1) ^ 1))) {
+          srow[s] = -1;
+          mbar_arrive(full_bar(s));
+        } else {
+          flag[0] = 1;
+        }
       }
       if (flag[0]) {
-        for (int it = (issued > C::NS ? issued - C::NS : 0); it < issued; ++it)
-          mbar_wait_drain(full_bar(it % C::NS), (uint32_t)((it / C::NS) & 1));
+        for (int j = (it > C::NS ? it - C::NS : 0); j < it; ++j)
+          mbar_wait_drain(full_bar(j % C::NS), (uint32_t)((j / C::NS) & 1));
       }
     }
     return;  // the producer takes no part in the merge (named barriers below count 32*NCW)
   }
 
   // ---------------------------------------------------------------- consumers
-  // Q fragments (B operand, col-major [d][head]): head n = lane/4 of the group,
-  // dims kk*16 + 2*(lane%4) + {0,1} and +8, rotated at position off.
-  uint32_t qf[D / 16][2];
-  float hs[2] = {0.f, 0.f};   // FP8: score scale of heads 2(lane%4), 2(lane%4)+1
-  if constexpr (F8) {
-    // FP8 layout: fragment (grp, st) holds dims 32 grp + 4(lane%4) + 2 st + {0,1}
-    // (register 0) and the same + 16 (register 1), matching the code bytes
-    // ldmatrix hands each lane. Head n is scaled by 2^-e_n so that its
-    // largest |q| lies in [2^14, 2^15): every bf16 q is then exact in f16
-    // down to 2^-29 of that maximum.
-    const int n = lane >> 2;
-    const bool hv = n < QM;
-    const __nv_bfloat16* qrow = p.q + b * p.qs0 + (long long)(g * QM + (hv ? n : 0)) * p.qs2;
-    const float* cs = p.cos_t + p.off * HALF;
-    const float* sn = p.sin_t + p.off * HALF;
-    float qv[D / 16][2][2];
-    float amax = 0.f;
+  // Every global load a consumer warp needs before its first tile goes out
+  // at once, so their latencies overlap: the sinks (into smem), the query
+  // words and, in warp 0 of the last split, the new K/V row with its RoPE
+  // table entries.
+  // (the sink goes to smem only after the query words have arrived, so its
+  // load does not hold up theirs)
+  const float sink_in = (threadIdx.x < QM && p.sinks) ? p.sinks[g * QM + threadIdx.x] : -INFINITY;
+  const bool new_row = last_split && warp == 0;
+  const long long new_slot = p.ring_cap > 0 ? p.off % p.ring_cap : p.off;
+  const long long new_crow = ((long long)b * p.n_kv + g) * p.cap + new_slot;
+  const __nv_bfloat16* krow = p.k + b * p.ks0 + (long long)g * p.ks2;
+  const __nv_bfloat16* vrow = p.v + b * p.vs0 + (long long)g * p.vs2;
+  const float* ctab = p.cos_t + p.off * HALF;
+  const float* stab = p.sin_t + p.off * HALF;
+  // bf16 cache: unit u < HALF/2 of a lane is K word pair (2u, 2u + HALF),
+  // unit u >= HALF/2 the same pair of V. FP8 cache: the lane's words 2 lane
+  // + 64 i (the quantiser's layout) and, for K, their RoPE partners.
+  constexpr int NRU = F8 ? 2 : (HALF + 31) / 32;
+  uint32_t nr_a[NRU], nr_b[NRU], nr_v[NRU];
+  float2 nr_c[NRU], nr_s[NRU];
+  if (new_row) {
 #pragma unroll
-    for (int f = 0; f < D / 16; ++f) {
-#pragma unroll
-      for (int hlf = 0; hlf < 2; ++hlf) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = 32 * (f >> 1) + 16 * hlf + 4 * (lane & 3) + 2 * (f & 1) + e;
-          float x = __bfloat162float(qrow[c]);
+    for (int i = 0; i < NRU; ++i) {
+      nr_a[i] = nr_b[i] = nr_v[i] = 0u;
+      nr_c[i] = nr_s[i] = make_float2(0.f, 0.f);
+      if constexpr (F8) {
+        const int c = 2 * lane + 64 * i;
+        if (c < D) {
+          const int i0 = c < HALF ? c : c - HALF;
+          nr_a[i] = *reinterpret_cast<const uint32_t*>(krow + i0);
+          nr_b[i] = *reinterpret_cast<const uint32_t*>(krow + i0 + HALF);
+          nr_v[i] = *reinterpret_cast<const uint32_t*>(vrow + c);
           if (p.rope) {
-            const int i = c < HALF ? c : c - HALF;
-            uint32_t y1, y2;
-            rope_pair(__bfloat162float(qrow[i]), __bfloat162float(qrow[i + HALF]), cs[i], sn[i], y1, y2);
-            x = __uint_as_float((c < HALF ? y1 : y2) << 16);
+            nr_c[i] = *reinterpret_cast<const float2*>(ctab + i0);
+            nr_s[i] = *reinterpret_cast<const float2*>(stab + i0);
           }
-          x = hv ? x : 0.f;
-          qv[f][hlf][e] = x;
-          amax = fmaxf(amax, fabsf(x));
         }
-      }
-    }
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    int eq = 0;
-    if (amax > 0.f) {
-      eq = (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127 - 14;
-      eq = eq < -110 ? -110 : (eq > 110 ? 110 : eq);
-    }
-    const float down = __uint_as_float((uint32_t)(127 - eq) << 23);
-#pragma unroll
-    for (int f = 0; f < D / 16; ++f)
-#pragma unroll
-      for (int hlf = 0; hlf < 2; ++hlf) qf[f][hlf] = pack_f16(qv[f][hlf][0] * down, qv[f][hlf][1] * down);
-    const float hs_mine = p.scale_log2 * __uint_as_float((uint32_t)(127 + eq) << 23);
-    hs[0] = __shfl_sync(0xffffffffu, hs_mine, 8 * (lane & 3));
-    hs[1] = __shfl_sync(0xffffffffu, hs_mine, 8 * (lane & 3) + 4);
-  } else {
-    const int n = lane >> 2;
-    const bool hv = n < QM;
-    const __nv_bfloat16* qrow = p.q + b * p.qs0 + (long long)(g * QM + (hv ? n : 0)) * p.qs2;
-    const float* cs = p.cos_t + p.off * HALF;
-    const float* sn = p.sin_t + p.off * HALF;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-#pragma unroll
-      for (int hlf = 0; hlf < 2; ++hlf) {
-        float y[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = kk * 16 + 8 * hlf + 2 * (lane & 3) + e;
-          float x = __bfloat162float(qrow[c]);
-          if (p.rope) {
-            const int i = c < HALF ? c : c - HALF;
-            const float x1 = __bfloat162float(qrow[i]), x2 = __bfloat162float(qrow[i + HALF]);
-            uint32_t y1, y2;
-            rope_pair(x1, x2, cs[i], sn[i], y1, y2);
-            x = __uint_as_float((c < HALF ? y1 : y2) << 16);
+      } else {
+        const int u = lane + 32 * i;
+        if (u < HALF) {
+          const bool is_v = u >= HALF / 2;
+          const int c = 2 * (is_v ? u - HALF / 2 : u);
+          const __nv_bfloat16* row = is_v ? vrow : krow;
+          nr_a[i] = *reinterpret_cast<const uint32_t*>(row + c);
+          nr_b[i] = *reinterpret_cast<const uint32_t*>(row + c + HALF);
+          if (!is_v && p.rope) {
+            nr_c[i] = *reinterpret_cast<const float2*>(ctab + c);
+            nr_s[i] = *reinterpret_cast<const float2*>(stab + c);
           }
-          y[e] = hv ? x : 0.f;
         }
-        qf[kk][hlf] = pack_bf16(y[0], y[1]);
       }
     }
   }
+
+  // Q fragments (B operand, col-major [d][head]): head n = lane/4 of the
+  // group, rotated at position off; the lane's words are listed by QWords.
+  uint32_t qf[D / 16][2];
+  float hs[2] = {0.f, 0.f};   // FP8: score scale of heads 2(lane%4), 2(lane%4)+1
+  {
+    const int n = lane >> 2;
+    const bool hv = n < QM;
+    const __nv_bfloat16* qrow = p.q + b * p.qs0 + (long long)(g * QM + (hv ? n : 0)) * p.qs2;
+    uint32_t w[D / 8];
+    load_q_words<D, F8>(qrow, F8 ? 4 * (lane & 3) : 2 * (lane & 3), ctab, stab, p.rope, w);
+    if constexpr (F8) {
+      // FP8 layout: fragment (grp, st) holds dims 32 grp + 4(lane%4) + 2 st + {0,1}
+      // (register 0) and the same + 16 (register 1), matching the code bytes
+      // ldmatrix hands each lane. Head n is scaled by 2^-e_n so that its
+      // largest |q| lies in [2^14, 2^15): every bf16 q is then exact in f16
+      // down to 2^-29 of that maximum.
+      float qv[D / 16][2][2];
+      float amax = 0.f;
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j) {
+        qv[j >> 1][j & 1][0] = hv ? bf16_lo(w[j]) : 0.f;
+        qv[j >> 1][j & 1][1] = hv ? bf16_hi(w[j]) : 0.f;
+        amax = fmaxf(amax, fmaxf(fabsf(qv[j >> 1][j & 1][0]), fabsf(qv[j >> 1][j & 1][1])));
+      }
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      int eq = 0;
+      if (amax > 0.f) {
+        eq = (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127 - 14;
+        eq = eq < -110 ? -110 : (eq > 110 ? 110 : eq);
+      }
+      const float down = __uint_as_float((uint32_t)(127 - eq) << 23);
+#pragma unroll
+      for (int f = 0; f < D / 16; ++f)
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) qf[f][hlf] = pack_f16(qv[f][hlf][0] * down, qv[f][hlf][1] * down);
+      const float hs_mine = p.scale_log2 * __uint_as_float((uint32_t)(127 + eq) << 23);
+      hs[0] = __shfl_sync(0xffffffffu, hs_mine, 8 * (lane & 3));
+      hs[1] = __shfl_sync(0xffffffffu, hs_mine, 8 * (lane & 3) + 4);
+    } else {
+#pragma unroll
+      for (int j = 0; j < D / 8; ++j) qf[j >> 1][j & 1] = hv ? w[j] : 0u;
+    }
+  }
+  if (threadIdx.x < QM) sink_sm[threadIdx.x] = sink_in * 1.4426950408889634f;
   int ev[2] = {-127, -127};   // FP8: powers of two of the two head columns' accumulators
   // FP8: this lane's shared-memory offsets within a stage (the same for every stage)
   uint32_t f8ko[C::RW / 16], f8vo[C::RW / 16][4];
@@ -562,51 +723,41 @@ __global__ void __launch_bounds__(288, 2)
 #pragma unroll
   for (int md = 0; md < D / 16; ++md) o[md][0] = o[md][1] = o[md][2] = o[md][3] = 0.f;
 
-  // The new row: rotate k, write K/V row `off` of the cache, stage it in smem.
-  // An FP8 cache stores (and this call attends) the row quantised.
-  if constexpr (F8) {
-    if (last_split && warp == 0) {
-      uint8_t* xk = smem + C::OFF_XK;
-      uint8_t* xv = smem + C::OFF_XV;
+  // The new row: rotate k, write K/V row `off` of the cache, stage it in smem
+  // as row 0 of a zeroed 16-row tile. An FP8 cache stores (and this call
+  // attends) the row quantised.
+  if (new_row) {
+    uint8_t* xk = smem + C::OFF_XK;
+    uint8_t* xv = smem + C::OFF_XV;
+    for (int idx = lane; idx < (int)(C::XTILE / 16); idx += 32) {
+      reinterpret_cast<uint4*>(xk)[idx] = make_uint4(0, 0, 0, 0);
+      reinterpret_cast<uint4*>(xv)[idx] = make_uint4(0, 0, 0, 0);
+    }
+    if constexpr (F8) {
       float* xs = reinterpret_cast<float*>(smem + C::OFF_XS);
-      const __nv_bfloat16* krow = p.k + b * p.ks0 + (long long)g * p.ks2;
-      const __nv_bfloat16* vrow = p.v + b * p.vs0 + (long long)g * p.vs2;
-      const long long slot = p.ring_cap > 0 ? p.off % p.ring_cap : p.off;
-      const long long crow = ((long long)b * p.n_kv + g) * p.cap + slot;
-      for (int idx = lane; idx < (int)(C::XTILE / 16); idx += 32) {
-        reinterpret_cast<uint4*>(xk)[idx] = make_uint4(0, 0, 0, 0);
-        reinterpret_cast<uint4*>(xv)[idx] = make_uint4(0, 0, 0, 0);
-      }
       xs[lane] = 0.f;
       __syncwarp();
       float xkv[2][2], xvv[2][2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int c = 2 * lane + 64 * i + e;
-          float kx = 0.f, vx = 0.f;
-          if (c < D) {
-            kx = __bfloat162float(krow[c]);
-            if (p.rope) {
-              const int i0 = c < HALF ? c : c - HALF;
-              uint32_t y1, y2;
-              rope_pair(__bfloat162float(krow[i0]), __bfloat162float(krow[i0 + HALF]),
-                        p.cos_t[p.off * HALF + i0], p.sin_t[p.off * HALF + i0], y1, y2);
-              kx = __uint_as_float((c < HALF ? y1 : y2) << 16);
-            }
-            vx = __bfloat162float(vrow[c]);
-          }
-          xkv[i][e] = kx;
-          xvv[i][e] = vx;
+        const int c = 2 * lane + 64 * i;
+        uint32_t kw = c < HALF ? nr_a[i] : nr_b[i];
+        if (c < D && p.rope) {
+          uint32_t w1 = nr_a[i], w2 = nr_b[i];
+          rope_pair2(w1, w2, nr_c[i].x, nr_c[i].y, nr_s[i].x, nr_s[i].y);
+          kw = c < HALF ? w1 : w2;
         }
+        xkv[i][0] = bf16_lo(kw);
+        xkv[i][1] = bf16_hi(kw);
+        xvv[i][0] = bf16_lo(nr_v[i]);
+        xvv[i][1] = bf16_hi(nr_v[i]);
       }
       uint16_t kc[2], vc[2];
-      const float sk = quantize_row_warp<2>(xkv, D, reinterpret_cast<uint8_t*>(p.ck) + crow * D, lane, kc);
-      const float sv = quantize_row_warp<2>(xvv, D, reinterpret_cast<uint8_t*>(p.cv) + crow * D, lane, vc);
+      const float sk = quantize_row_warp<2>(xkv, D, reinterpret_cast<uint8_t*>(p.ck) + new_crow * D, lane, kc);
+      const float sv = quantize_row_warp<2>(xvv, D, reinterpret_cast<uint8_t*>(p.cv) + new_crow * D, lane, vc);
       if (lane == 0) {
-        p.cks[crow] = sk;
-        p.cvs[crow] = sv;
+        p.cks[new_crow] = sk;
+        p.cvs[new_crow] = sv;
         xs[0] = sk;
         xs[16] = sv;
       }
@@ -618,49 +769,37 @@ __global__ void __launch_bounds__(288, 2)
           *reinterpret_cast<uint16_t*>(xv + swz8<C::ROWB>(0, c, C::XBLOCK)) = vc[i];
         }
       }
+    } else {
       __syncwarp();
-    }
-  } else if (last_split && warp == 0) {
-    uint8_t* xk = smem + C::OFF_XK;
-    uint8_t* xv = smem + C::OFF_XV;
-    const __nv_bfloat16* krow = p.k + b * p.ks0 + (long long)g * p.ks2;
-    const __nv_bfloat16* vrow = p.v + b * p.vs0 + (long long)g * p.vs2;
-    const long long slot = p.ring_cap > 0 ? p.off % p.ring_cap : p.off;
-    __nv_bfloat16* ckrow = p.ck + (((long long)b * p.n_kv + g) * p.cap + slot) * D;
-    __nv_bfloat16* cvrow = p.cv + (((long long)b * p.n_kv + g) * p.cap + slot) * D;
-    // zero rows 1..15 (and row 0, overwritten below)
-    for (int idx = lane; idx < (int)(C::XTILE / 16); idx += 32) {
-      reinterpret_cast<uint4*>(xk)[idx] = make_uint4(0, 0, 0, 0);
-      reinterpret_cast<uint4*>(xv)[idx] = make_uint4(0, 0, 0, 0);
-    }
-    __syncwarp();
-    for (int c = lane; c < HALF; c += 32) {
-      __nv_bfloat16 b1 = krow[c], b2 = krow[c + HALF];
-      if (p.rope) {
-        uint32_t y1, y2;
-        rope_pair(__bfloat162float(b1), __bfloat162float(b2), p.cos_t[p.off * HALF + c],
-                  p.sin_t[p.off * HALF + c], y1, y2);
-        b1 = __ushort_as_bfloat16((unsigned short)y1);
-        b2 = __ushort_as_bfloat16((unsigned short)y2);
+      __nv_bfloat16* ckrow = p.ck + new_crow * D;
+      __nv_bfloat16* cvrow = p.cv + new_crow * D;
+#pragma unroll
+      for (int i = 0; i < NRU; ++i) {
+        const int u = lane + 32 * i;
+        if (u < HALF) {
+          const bool is_v = u >= HALF / 2;
+          const int c = 2 * (is_v ? u - HALF / 2 : u);
+          uint32_t w1 = nr_a[i], w2 = nr_b[i];
+          if (!is_v && p.rope) rope_pair2(w1, w2, nr_c[i].x, nr_c[i].y, nr_s[i].x, nr_s[i].y);
+          __nv_bfloat16* crow = is_v ? cvrow : ckrow;
+          uint8_t* tile = is_v ? xv : xk;
+          *reinterpret_cast<uint32_t*>(crow + c) = w1;
+          *reinterpret_cast<uint32_t*>(crow + c + HALF) = w2;
+          *reinterpret_cast<uint32_t*>(tile + swz_off<C::CB>(0, c, C::XBLOCK)) = w1;
+          *reinterpret_cast<uint32_t*>(tile + swz_off<C::CB>(0, c + HALF, C::XBLOCK)) = w2;
+        }
       }
-      ckrow[c] = b1;
-      ckrow[c + HALF] = b2;
-      *reinterpret_cast<__nv_bfloat16*>(xk + swz_off<C::CB>(0, c, C::XBLOCK)) = b1;
-      *reinterpret_cast<__nv_bfloat16*>(xk + swz_off<C::CB>(0, c + HALF, C::XBLOCK)) = b2;
-      const __nv_bfloat16 v1 = vrow[c], v2 = vrow[c + HALF];
-      cvrow[c] = v1;
-      cvrow[c + HALF] = v2;
-      *reinterpret_cast<__nv_bfloat16*>(xv + swz_off<C::CB>(0, c, C::XBLOCK)) = v1;
-      *reinterpret_cast<__nv_bfloat16*>(xv + swz_off<C::CB>(0, c + HALF, C::XBLOCK)) = v2;
     }
     __syncwarp();
   }
 
-  for (int it = 0; it < n_stages; ++it) {
+  for (int it = 0;; ++it) {
     const int s = it % C::NS;
     if (!mbar_wait(full_bar(s), (uint32_t)((it / C::NS) & 1))) { flag[0] = 1; break; }
-    const long long row0 = r_begin + (long long)it * C::R + C::RW * warp;
-    const long long nv = r_end - row0;
+    const long long pos0 = srow[s];
+    if (pos0 < 0) break;   // the producer's end mark
+    const long long row0 = pos0 + C::RW * warp;
+    const long long nv = p.off - row0;
     const long long nf = p.lo_mask - row0;
     if (nv > 0 && nf < C::RW && !flag[0]) {
       if constexpr (F8) {
@@ -738,153 +877,155 @@ __global__ void __launch_bounds__(288, 2)
   }
   named_bar_sync(1, 32 * C::NCW);
 
-  const float LOG2E = 1.4426950408889634f, LN2 = 0.6931471805599453f;
+  const float LN2 = 0.6931471805599453f;
   const int tid = threadIdx.x;  // 0 .. 32*NCW-1
   constexpr int NT = 32 * C::NCW;
-  const long long slot = ((long long)b * p.n_kv + g) * p.S + split;
-  for (int idx = tid; idx < QM * D; idx += NT) {
+  const int RF = p.rec_floats;
+  float* rec = p.ws_rec + (((long long)b * p.n_kv + g) * p.S + split) * RF;
+  // two adjacent outputs (head n, dims d, d+1) per thread and pass
+  for (int idx = 2 * tid; idx < QM * D; idx += 2 * NT) {
     const int n = idx / D, d = idx % D;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < C::NCW; ++w) M = fmaxf(M, red[w * (C::RED_WARP / 4) + n]);
     const float Mu = (M == -INFINITY) ? 0.f : M;
-    float L = 0.f, O = 0.f;
+    float L = 0.f, O0 = 0.f, O1 = 0.f;
 #pragma unroll
     for (int w = 0; w < C::NCW; ++w) {
       const float* rw = red + w * (C::RED_WARP / 4);
       const float f = ex2(rw[n] - Mu);
       L += rw[8 + n] * f;
-      O += rw[16 + n * D + d] * f;
+      const float2 ov = *reinterpret_cast<const float2*>(rw + 16 + n * D + d);
+      O0 += ov.x * f;
+      O1 += ov.y * f;
     }
     const int h = g * QM + n;
     if (p.S == 1) {
-      const float sink2 = p.sinks ? p.sinks[h] * LOG2E : -INFINITY;
+      const float sink2 = sink_sm[n];
       const float M2 = fmaxf(M, sink2);
       const float fo = ex2(M - M2);
       const float tot = L * fo + ex2(sink2 - M2);
-      p.out[b * p.os0 + (long long)h * p.os2 + d] = __float2bfloat16_rn(O * fo / tot);
+      *reinterpret_cast<uint32_t*>(p.out + b * p.os0 + (long long)h * p.os2 + d) =
+          pack_bf16(O0 * fo / tot, O1 * fo / tot);
       if (d == 0 && p.lse) p.lse[(long long)b * p.n_q + h] = (M2 + __log2f(tot)) * LN2;
     } else {
-      p.ws_o[(slot * QM + n) * D + d] = O;
+      *reinterpret_cast<float2*>(rec + n * D + d) = make_float2(O0, O1);
       if (d == 0) {
-        p.ws_m[slot * QM + n] = M;
-        p.ws_l[slot * QM + n] = L;
+        rec[QM * D + n] = M;
+        rec[QM * D + QM + n] = L;
       }
     }
   }
   if (p.S == 1) return;
 
-  __threadfence();
+  // The ticket: the barrier orders every thread's record stores before
+  // thread 0's release; its acquire makes the other CTAs' records visible to
+  // the merging CTA (whose thread 0 alone reads them, by bulk copy).
   named_bar_sync(1, NT);
   if (tid == 0) {
-    const int ticket = atomicAdd(p.ws_cnt + (b * p.n_kv + g), 1);
+    const int ticket = atom_add_acq_rel_gpu(p.ws_cnt + (b * p.n_kv + g), 1);
     flag[1] = (ticket == p.S - 1) ? 1 : 0;
   }
   named_bar_sync(1, NT);
   if (!flag[1]) return;
-  __threadfence();
 
-  // Merge the S partials of (b, g). The K/V ring is idle now; reuse it for
-  // the per-split weights. Every global read below is batched (independent
-  // loads in flight) because this tail runs on one CTA per (b, g) while the
-  // rest of the GPU has finished.
-  const long long slot0 = ((long long)b * p.n_kv + g) * p.S;
+  // Merge the S records of (b, g). The K/V ring is idle now: one bulk copy
+  // per round brings as many records as it holds (normally all S) into it,
+  // so the tail pays one memory round trip instead of one per batch of
+  // loads. A group of G adjacent lanes owns four outputs (head n, dims
+  // d .. d+3); its lanes take every G-th record and combine by shuffles.
+  // The running maximum starts at the sink (log2 units):
+  // M = max(sink, m_s), l = e^{sink-M} + sum_s e^{m_s-M} l_s.
   const int S = p.S;
-  float* wsm = reinterpret_cast<float*>(smem);                 // [S][QM] m_s, then e^{m_s - M}
-  float* lsm = wsm + (size_t)S * QM;                            // [S][QM] l_s
-  float* Msm = lsm + (size_t)S * QM;                            // [QM] M (log2 units)
-  float* Lsm = Msm + 8;                                         // [QM] total l
-  {
-    const float* gm = p.ws_m + slot0 * QM;
-    const float* gl = p.ws_l + slot0 * QM;
-    const int nml = S * QM;
-    int idx = tid;
-    for (; idx + 3 * NT < nml; idx += 4 * NT) {
-      float a[4], c[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        a[j] = __ldcg(gm + idx + j * NT);
-        c[j] = __ldcg(gl + idx + j * NT);
+  const uint32_t rec_bytes = (uint32_t)RF * 4u;
+  const int per_round = (int)(C::RING_BYTES / rec_bytes);
+  const float* recs = reinterpret_cast<const float*>(smem);
+  const char* gsrc = reinterpret_cast<const char*>(p.ws_rec + ((long long)b * p.n_kv + g) * S * RF);
+  const int nf4 = QM * D / 4;
+  const int G = 2 * nf4 <= NT ? 2 : 1;   // lanes per output group
+  const int f4 = tid / G, part = tid % G;
+  const bool owner = f4 < nf4;
+  const int n = owner ? (4 * f4) / D : 0;
+  const int d = owner ? (4 * f4) % D : 0;
+  const int om = QM * D + n, ol = QM * D + QM + n, oo = n * D + d;
+  float M = sink_sm[n];
+  float L = (M == -INFINITY) ? 0.f : 1.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0, r = 0; s0 < S; s0 += per_round, ++r) {
+    const int cnt = S - s0 < per_round ? S - s0 : per_round;
+    if (tid == 0) {
+      // the records were written by generic stores (other CTAs', acquired
+      // through the ticket) and the ring was last written the same way
+      fence_proxy_async_global();
+      fence_proxy_async_smem();
+      const uint32_t bytes = (uint32_t)cnt * rec_bytes;
+      mbar_arrive_expect_tx(merge_bar, bytes);
+      for (uint32_t o = 0; o < bytes; o += 32768u)
+        bulk_load(sbase + o, gsrc + (size_t)s0 * rec_bytes + o, bytes - o < 32768u ? bytes - o : 32768u,
+                  merge_bar);
+    }
+    // a wait that runs out is recorded in the status word; the copy is then
+    // drained before the ring is read or this CTA exits
+    if (!mbar_wait(merge_bar, (uint32_t)(r & 1))) mbar_wait_drain(merge_bar, (uint32_t)(r & 1));
+    float Mr = M;
+    float4 ar = make_float4(0.f, 0.f, 0.f, 0.f);
+    float Lr = 0.f;
+    if (owner) {
+      float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+      int s2 = part;
+      for (; s2 + 3 * G < cnt; s2 += 4 * G) {
+        m0 = fmaxf(m0, recs[s2 * RF + om]);
+        m1 = fmaxf(m1, recs[(s2 + G) * RF + om]);
+        m2 = fmaxf(m2, recs[(s2 + 2 * G) * RF + om]);
+        m3 = fmaxf(m3, recs[(s2 + 3 * G) * RF + om]);
       }
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        wsm[idx + j * NT] = a[j];
-        lsm[idx + j * NT] = c[j];
+      for (; s2 < cnt; s2 += G) m0 = fmaxf(m0, recs[s2 * RF + om]);
+      Mr = fmaxf(fmaxf(Mr, fmaxf(m0, m1)), fmaxf(m2, m3));
+    }
+    if (G == 2) Mr = fmaxf(Mr, __shfl_xor_sync(0xffffffffu, Mr, 1));
+    const float Mu = (Mr == -INFINITY) ? 0.f : Mr;
+    if (owner) {
+#pragma unroll 4
+      for (int s2 = part; s2 < cnt; s2 += G) {
+        const float* rr = recs + s2 * RF;
+        const float w = ex2(rr[om] - Mu);
+        Lr = fmaf(w, rr[ol], Lr);
+        const float4 v = *reinterpret_cast<const float4*>(rr + oo);
+        ar.x = fmaf(w, v.x, ar.x);
+        ar.y = fmaf(w, v.y, ar.y);
+        ar.z = fmaf(w, v.z, ar.z);
+        ar.w = fmaf(w, v.w, ar.w);
       }
     }
-    for (; idx < nml; idx += NT) {
-      wsm[idx] = __ldcg(gm + idx);
-      lsm[idx] = __ldcg(gl + idx);
+    if (G == 2) {
+      Lr += __shfl_xor_sync(0xffffffffu, Lr, 1);
+      ar.x += __shfl_xor_sync(0xffffffffu, ar.x, 1);
+      ar.y += __shfl_xor_sync(0xffffffffu, ar.y, 1);
+      ar.z += __shfl_xor_sync(0xffffffffu, ar.z, 1);
+      ar.w += __shfl_xor_sync(0xffffffffu, ar.w, 1);
     }
+    const float f = ex2(M - Mu);
+    L = fmaf(L, f, Lr);
+    acc.x = fmaf(acc.x, f, ar.x);
+    acc.y = fmaf(acc.y, f, ar.y);
+    acc.z = fmaf(acc.z, f, ar.z);
+    acc.w = fmaf(acc.w, f, ar.w);
+    M = Mr;
+    named_bar_sync(1, NT);   // the ring is read before the next round's copy overwrites it
   }
-  named_bar_sync(1, NT);
-  {
-    // warp w reduces head n = w (QM <= 8 <= NCW): lanes stride over the splits
-    const int w = tid >> 5;
-    for (int n = w; n < QM; n += C::NCW) {
-      const int h = g * QM + n;
-      const float sink2 = p.sinks ? p.sinks[h] * LOG2E : -INFINITY;
-      float M = sink2;
-      for (int s2 = lane; s2 < S; s2 += 32) M = fmaxf(M, wsm[s2 * QM + n]);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-      float L = 0.f;
-      for (int s2 = lane; s2 < S; s2 += 32) {
-        const float ms = wsm[s2 * QM + n];
-        const float f = (ms == -INFINITY) ? 0.f : ex2(ms - M);
-        wsm[s2 * QM + n] = f;
-        L += lsm[s2 * QM + n] * f;
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-      if (lane == 0) {
-        L += ex2(sink2 - M);
-        Msm[n] = M;
-        Lsm[n] = L;
-      }
-    }
+  if (owner && part == 0) {
+    const int h = g * QM + n;
+    const float inv = 1.0f / L;
+    uint2 packed;
+    packed.x = pack_bf16(acc.x * inv, acc.y * inv);
+    packed.y = pack_bf16(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(p.out + b * p.os0 + (long long)h * p.os2 + d) = packed;
+    if (d == 0 && p.lse) p.lse[(long long)b * p.n_q + h] = (M + __log2f(L)) * LN2;
   }
-  named_bar_sync(1, NT);
-  {
-    // O = sum_s w_s O_s, four consecutive d per thread, eight splits in flight.
-    const int nf4 = QM * D / 4;
-    const float4* src0 = reinterpret_cast<const float4*>(p.ws_o + slot0 * QM * D);
-    for (int idx = tid; idx < nf4; idx += NT) {
-      const int n = (idx * 4) / D, d = (idx * 4) % D;
-      const float4* src = src0 + idx;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      int s2 = 0;
-      for (; s2 + 8 <= S; s2 += 8) {
-        float4 v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) v[j] = __ldcg(src + (size_t)(s2 + j) * nf4);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float w = wsm[(s2 + j) * QM + n];
-          acc.x = fmaf(v[j].x, w, acc.x);
-          acc.y = fmaf(v[j].y, w, acc.y);
-          acc.z = fmaf(v[j].z, w, acc.z);
-          acc.w = fmaf(v[j].w, w, acc.w);
-        }
-      }
-      for (; s2 < S; ++s2) {
-        const float4 v = __ldcg(src + (size_t)s2 * nf4);
-        const float w = wsm[s2 * QM + n];
-        acc.x = fmaf(v.x, w, acc.x);
-        acc.y = fmaf(v.y, w, acc.y);
-        acc.z = fmaf(v.z, w, acc.z);
-        acc.w = fmaf(v.w, w, acc.w);
-      }
-      const int h = g * QM + n;
-      const float inv = 1.0f / Lsm[n];
-      uint2 packed;
-      packed.x = pack_bf16(acc.x * inv, acc.y * inv);
-      packed.y = pack_bf16(acc.z * inv, acc.w * inv);
-      *reinterpret_cast<uint2*>(p.out + b * p.os0 + (long long)h * p.os2 + d) = packed;
-      if (d == 0 && p.lse) p.lse[(long long)b * p.n_q + h] = (Msm[n] + __log2f(Lsm[n])) * LN2;
-    }
+  if (tid == 0) {
+    p.ws_cnt[b * p.n_kv + g] = 0;
+    p.ws_grab[b * p.n_kv + g] = 0;
   }
-  if (tid == 0) p.ws_cnt[b * p.n_kv + g] = 0;
 }
 
 }  // namespace sa

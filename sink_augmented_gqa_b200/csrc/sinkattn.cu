@@ -405,32 +405,29 @@ sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, int slot, 
   return (last_launch_status() == SA_OK && e == cudaSuccess) ? SA_OK : SA_ERR_CUDA;
 }
 
-struct DecodeSplit {
-  int S;
-  long long chunk;
-};
-
-// stage: cache rows per ring stage of the decode kernel (its Cfg::R); every
-// split but the last covers whole stages.
-DecodeSplit decode_split(int B, int n_kv, long long n_cache, long long stage) {
-  DecodeSplit r{1, stage};
-  if (n_cache <= 0) return r;
-  const long long target = 2LL * num_sms();
-  long long S = (target + (long long)B * n_kv - 1) / ((long long)B * n_kv);
-  if (S < 1) S = 1;
-  long long chunk = (n_cache + S - 1) / S;
-  chunk = ((chunk + stage - 1) / stage) * stage;
-  r.chunk = chunk;
-  r.S = (int)((n_cache + chunk - 1) / chunk);
-  return r;
+// CTAs per (b, g) for n_cache cached rows in stages of `stage` rows: at
+// most one wave of CTAs (two per SM) -- the decode kernel balances the
+// stages among the CTAs of each (b, g) by itself, and a partial second wave
+// would only stream its CTAs' static stages at the end -- and no more CTAs
+// than stages.
+int decode_splits(int B, int n_kv, long long n_cache, long long stage) {
+  if (n_cache <= 0) return 1;
+  long long S = 2LL * num_sms() / ((long long)B * n_kv);
+  const long long nb = (n_cache + stage - 1) / stage;
+  if (S > nb) S = nb;
+  return S < 1 ? 1 : (int)S;
 }
 
-// Workspace layout: counters [B*n_kv] int32 (256-byte padded), then
-// O [B*n_kv*S*q_mult*d], m [B*n_kv*S*q_mult], l [same] fp32.
+// Workspace layout: split tickets [B*n_kv] then dynamic-stage counters
+// [B*n_kv], int32 (256-byte padded), then one fp32 record per (b, g, split):
+// O [q_mult][d], m [q_mult], l [q_mult], padded to a multiple of 16 bytes
+// (the merge brings records in by bulk copy).
+int decode_rec_floats(int q_mult, int d) { return q_mult * d + (2 * q_mult + 3) / 4 * 4; }
+
+size_t decode_cnt_bytes(int B, int n_kv) { return (((size_t)B * n_kv * 8) + 255) / 256 * 256; }
+
 size_t decode_ws_bytes(int B, int n_kv, int q_mult, int d, int S) {
-  const size_t cnt = (((size_t)B * n_kv * 4) + 255) / 256 * 256;
-  const size_t rows = (size_t)B * n_kv * S * q_mult;
-  return cnt + rows * 4 * 2 + rows * d * 4;
+  return decode_cnt_bytes(B, n_kv) + (size_t)B * n_kv * S * decode_rec_floats(q_mult, d) * 4;
 }
 
 // Cache rows per ring stage of decode_kernel<d, f8> (its Cfg::R).
@@ -449,7 +446,7 @@ long long decode_stage_rows(int d, bool f8) {
 // and the scale boxes start on their stage's first row).
 struct DecodePlan {
   long long lo_mask, lo;
-  DecodeSplit split;
+  int S;   // CTAs per (b, g)
 };
 
 DecodePlan plan_decode(const sa_kv_cache* c, const sa_attn_args* a) {
@@ -458,9 +455,13 @@ DecodePlan plan_decode(const sa_kv_cache* c, const sa_attn_args* a) {
   DecodePlan pl;
   pl.lo_mask = a->window > 0 ? (a->offset + 1 - a->window > 0 ? a->offset + 1 - a->window : 0) : 0;
   pl.lo = (c->ring > 0 || f8) ? pl.lo_mask / R * R : pl.lo_mask;
-  pl.split = decode_split(a->B, c->n_kv, a->offset - pl.lo, R);
+  pl.S = decode_splits(a->B, c->n_kv, a->offset - pl.lo, R);
   return pl;
 }
+
+// Cache bytes each decode CTA prefetches into L2 before it waits for the
+// kernel ahead of it on the stream (rounded up to whole stages).
+constexpr long long kDecodePrefetchBytes = 128 * 1024;
 
 template <int D, bool F8>
 sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, size_t ws_bytes,
@@ -474,9 +475,12 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   p.lo_mask = pl.lo_mask;
   p.lo = pl.lo;
   const long long n_cache = p.off - p.lo;
-  const DecodeSplit sp = pl.split;
-  p.S = sp.S;
-  p.chunk = sp.chunk;
+  p.S = pl.S;
+  p.n_blocks = n_cache > 0 ? (n_cache + Cfg::R - 1) / Cfg::R : 0;
+  // a lone CTA streams everything in order; with several, half of each
+  // one's share is static and the rest dynamic
+  p.static_stages = p.S == 1 ? (int)p.n_blocks : (int)(p.n_blocks / (2 * p.S));
+  p.pf_stages = (int)((kDecodePrefetchBytes + Cfg::STAGE_TX - 1) / Cfg::STAGE_TX);
   if (p.S > 1) {
     if (ws == nullptr || !aligned16(ws) || ws_bytes < decode_ws_bytes(a->B, c->n_kv, q_mult, D, p.S))
       return SA_ERR_WORKSPACE;
@@ -530,12 +534,10 @@ sa_status launch_decode(const sa_kv_cache* c, const sa_attn_args* a, void* ws, s
   p.scale_log2 = a->sm_scale * 1.4426950408889634f;
   p.rope = a->rope_fused ? 1 : 0;
   uint8_t* w = static_cast<uint8_t*>(ws);
-  const size_t cnt = (((size_t)a->B * c->n_kv * 4) + 255) / 256 * 256;
-  const size_t rows = (size_t)a->B * c->n_kv * p.S * q_mult;
   p.ws_cnt = reinterpret_cast<int*>(w);
-  p.ws_o = reinterpret_cast<float*>(w + cnt);
-  p.ws_m = reinterpret_cast<float*>(w + cnt + rows * D * 4);
-  p.ws_l = reinterpret_cast<float*>(w + cnt + rows * D * 4 + rows * 4);
+  p.ws_grab = p.ws_cnt + (size_t)a->B * c->n_kv;
+  p.ws_rec = reinterpret_cast<float*>(w + decode_cnt_bytes(a->B, c->n_kv));
+  p.rec_floats = decode_rec_floats(q_mult, D);
   static std::atomic<uint64_t> smem_set{0};
   {
     const sa_status sm = set_smem_once(sa::decode_kernel<D, F8>, Cfg::SMEM_BYTES, smem_set);
@@ -945,8 +947,8 @@ sa_status sa_attn_decode_static(sa_kv_cache* cache, const sa_attn_args* a, sa_st
   if (a->T != 1) return SA_ERR_INVALID_ARG;
   const int q_mult = a->n_q / cache->n_kv;
   if (q_mult > 8) return SA_ERR_SHAPE;
-  const DecodeSplit sp = plan_decode(cache, a).split;   // the split the launch will use
-  if (sp.S > 1 && decode_ws_bytes(a->B, cache->n_kv, q_mult, cache->d, sp.S) > SA_DECODE_STATIC_SCRATCH_BYTES)
+  const int S = plan_decode(cache, a).S;   // the split the launch will use
+  if (S > 1 && decode_ws_bytes(a->B, cache->n_kv, q_mult, cache->d, S) > SA_DECODE_STATIC_SCRATCH_BYTES)
     return SA_ERR_WORKSPACE;
   void* scratch = nullptr;
   st = static_scratch(&scratch);
@@ -959,8 +961,7 @@ size_t sa_attn_decode_workspace_size(int32_t B, int32_t n_q, int32_t n_kv, int32
   const int q_mult = n_q / n_kv;
   // B*n_kv*S <= 2*256 + B*n_kv for any device of at most 256 SMs.
   const long long units = 512 + (long long)B * n_kv;
-  const size_t cnt = (((size_t)B * n_kv * 4) + 255) / 256 * 256;
-  return cnt + (size_t)units * q_mult * (2 + d) * 4;
+  return decode_cnt_bytes(B, n_kv) + (size_t)units * decode_rec_floats(q_mult, d) * 4;
 }
 
 sa_status sa_rmsnorm_fold_weight(const void* w, int64_t ldw, const float* gamma, void* w_folded,

@@ -105,8 +105,8 @@ def test_long_decode_all_64_steps(cuda_device, layer):
             check_lse(lse[0, h, 0], np.array(rl), f"long decode step {st} h{h}")
         check_bf16_output(torch.stack(got), stack_out(want), f"long decode step {st}")
     assert cache.offset == off + steps
-    n_cnt = cfg.B * cfg.n_kv   # the split tickets end every call at zero
-    assert torch.count_nonzero(ws[: 4 * n_cnt]) == 0
+    n_cnt = cfg.B * cfg.n_kv   # the split tickets and stage counters end every call at zero
+    assert torch.count_nonzero(ws[: 8 * n_cnt]) == 0
 
 
 @pytest.mark.parametrize("layer", [0, 1], ids=["band", "full"])

@@ -223,8 +223,8 @@ def _decode_steps(cfg, cache, ocache, n_steps, window, cos, sin, rc, rs, sinks, 
                                    cfg.sm_scale, rc, rs)
         check_bf16_output(out, ref, f"decode step {st}")
         check_lse(lse, ref_lse, f"decode step {st}")
-    n_cnt = cfg.B * cfg.n_kv   # the ticket counters lead the workspace and end each call at zero
-    assert torch.count_nonzero(ws[: 4 * n_cnt]) == 0
+    n_cnt = cfg.B * cfg.n_kv   # the tickets and stage counters lead the workspace, zero after each call
+    assert torch.count_nonzero(ws[: 8 * n_cnt]) == 0
     return cache
 
 

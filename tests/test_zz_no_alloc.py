@@ -63,8 +63,9 @@ def test_static_scratch_decode_matches_workspace_decode(cuda_device, window):
 
 
 def test_static_scratch_refuses_oversized_shapes(cuda_device):
-    # 16 sequences x 8 KV heads x 3 splits x 8 query heads x (128 + 2) fp32
-    # needs 1.6 MB of scratch, more than the 1 MiB the library holds.
+    # 16 sequences x 8 KV heads x 3 splits, one record of 8 query heads x
+    # (128 outputs + m + l) fp32 each: 1.6 MB of scratch, more than the 1 MiB
+    # the library holds.
     cfg = wl.scaled(wl.CONFIGS["handoff"], B=16, n_q=64, n_kv=8, d=128, offset=1000, T=0)
     cap = cfg.offset + 2
     cos, sin = _tables(cfg, cap)
