@@ -275,6 +275,12 @@ sa_status sa_kv_restore(sa_kv_cache* cache, const sa_snapshot* snap);
  * whatever stream it ran). Calls captured into a CUDA graph take the other
  * 64 round robin without events; graph replays that run at the same time as
  * one another must hold at most 64 prefill calls between them.
+ * Band layers of d = 64 whose window is narrow enough for the query heads of
+ * a KV group to share one key window of at most 160 columns (128/q_mult +
+ * window + 14 <= 160: W up to 130, 114, 82 or 18 for q_mult 8, 4, 2 or 1)
+ * take a second kernel instead: the staging launch only
+ * appends K/V, the kernel reads q directly and rotates it itself, no
+ * schedule counter is used, and `out` may again be `q` itself.
  * SA_ERR_UNSUPPORTED on an FP8 cache.
  */
 sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* args, sa_stream_t stream);

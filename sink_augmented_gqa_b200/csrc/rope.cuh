@@ -60,20 +60,22 @@ __global__ void yarn_tables_kernel(float* __restrict__ cos_out, float* __restric
   }
 }
 
-// Rotate 8 consecutive pairs (x1[c..c+7], x2[c..c+7]) with fp32 tables
-// (each result the correctly rounded bf16 of the exact rotation; see rope_pair).
-__device__ __forceinline__ void rotate8(uint4& a, uint4& b, const float* __restrict__ cs,
-                                       const float* __restrict__ sn) {
+// Rotate 8 consecutive pairs (x1[c..c+7], x2[c..c+7]) with the table entries
+// cos (c0, c1) and sin (s0, s1) already in registers (each result the
+// correctly rounded bf16 of the exact rotation; see rope_pair).
+__device__ __forceinline__ void rotate8_regs(uint4& a, uint4& b, float4 c0, float4 c1, float4 s0, float4 s1) {
   uint32_t* pa = reinterpret_cast<uint32_t*>(&a);
   uint32_t* pb = reinterpret_cast<uint32_t*>(&b);
-  const float4 c0 = *reinterpret_cast<const float4*>(cs);
-  const float4 c1 = *reinterpret_cast<const float4*>(cs + 4);
-  const float4 s0 = *reinterpret_cast<const float4*>(sn);
-  const float4 s1 = *reinterpret_cast<const float4*>(sn + 4);
   const float cc[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
   const float ss[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
   for (int w = 0; w < 4; ++w) rope_pair2(pa[w], pb[w], cc[2 * w], cc[2 * w + 1], ss[2 * w], ss[2 * w + 1]);
+}
+// The same with the table entries read from cs[0..7], sn[0..7].
+__device__ __forceinline__ void rotate8(uint4& a, uint4& b, const float* __restrict__ cs,
+                                       const float* __restrict__ sn) {
+  rotate8_regs(a, b, *reinterpret_cast<const float4*>(cs), *reinterpret_cast<const float4*>(cs + 4),
+               *reinterpret_cast<const float4*>(sn), *reinterpret_cast<const float4*>(sn + 4));
 }
 
 // In-place RoPE of a strided [B][T][H][d] bf16 tensor at positions off + t.

@@ -12,6 +12,7 @@
 
 #include "../../include/sinkattn.h"
 #include "backward.cuh"
+#include "band.cuh"
 #include "backward_tc.cuh"
 #include "decode.cuh"
 #include "fp8.cuh"
@@ -170,6 +171,25 @@ bool make_rows_map(CUtensorMap* map, const void* base, int d, int T, int H, int 
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          cb == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Tensor map over a strided [B][T][H][d] bf16 activation whose box is
+// box_heads consecutive heads of box_rows consecutive rows (d = 64: one
+// 128-byte swizzled row per (row, head)): dims {d, H, T, B}, box
+// {d, box_heads, box_rows, 1}; rows past T read as zeros and are dropped on
+// store.
+bool make_heads_map(CUtensorMap* map, const void* base, int d, int T, int H, int B, const int64_t st[3],
+                    int box_heads, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || T < 1 || d != 64) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)st[2] * 2, (cuuint64_t)st[1] * 2, (cuuint64_t)st[0] * 2};
+  const cuuint32_t box[4] = {(cuuint32_t)d, (cuuint32_t)box_heads, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -402,6 +422,75 @@ sa_status launch_prefill(const sa_kv_cache* c, const sa_attn_args* a, int slot, 
   lc.attrs = attr;
   lc.numAttrs = 1;
   const cudaError_t e = cudaLaunchKernelEx(&lc, sa::prefill_kernel<D>, tmQ, tmK, tmV, tmO, p);
+  return (last_launch_status() == SA_OK && e == cudaSuccess) ? SA_OK : SA_ERR_CUDA;
+}
+
+// Band layers whose key window fits the packed-head kernel: d = 64, a
+// window, q_mult dividing 128, and R + W - 1 keys (plus the 16-alignment of
+// the window start) within its 160 columns (W up to 130, 114, 82 or 18 for
+// q_mult 8, 4, 2 or 1). Returns the window width N (a multiple of 32) or 0.
+int band_columns(const sa_kv_cache* c, const sa_attn_args* a) {
+  if (c->d != 64 || a->window <= 0 || c->kv_dtype != SA_KV_BF16) return 0;
+  const int qm = a->n_q / c->n_kv;
+  if (qm < 1 || 128 % qm != 0) return 0;
+  const long long need = 128 / qm + (long long)a->window + 14;
+  const int N = (int)((need + 31) / 32 * 32);
+  return N <= sa::BandCfg<64>::NMAX ? N : 0;
+}
+
+sa_status launch_band(const sa_kv_cache* c, const sa_attn_args* a, int N, cudaStream_t stream) {
+  using Cfg = sa::BandCfg<64>;
+  const int qm = a->n_q / c->n_kv;
+  const int R = 128 / qm;
+  CUtensorMap tmQ, tmK, tmV, tmKw, tmVw, tmO;
+  const long long rows = c->ring > 0 ? (long long)c->cap : a->offset + a->T;
+  // K/V boxes: a whole N-row window, or 16 rows (windows that wrap a ring)
+  if (!make_heads_map(&tmQ, a->q, 64, a->T, a->n_q, a->B, a->q_strides, qm, R) ||
+      !make_heads_map(&tmO, a->out, 64, a->T, a->n_q, a->B, a->out_strides, qm, R) ||
+      !make_cache_map(&tmK, c->k, 64, c->n_kv, rows, c->cap, c->B, 16, 64) ||
+      !make_cache_map(&tmV, c->v, 64, c->n_kv, rows, c->cap, c->B, 16, 64) ||
+      !make_cache_map(&tmKw, c->k, 64, c->n_kv, rows, c->cap, c->B, N, 64) ||
+      !make_cache_map(&tmVw, c->v, 64, c->n_kv, rows, c->cap, c->B, N, 64))
+    return SA_ERR_CUDA;
+  sa::BandParams p;
+  p.lse = a->lse;
+  p.sinks = a->sinks;
+  p.cos_t = a->cos;
+  p.sin_t = a->sin;
+  p.B = a->B;
+  p.T = a->T;
+  p.n_q = a->n_q;
+  p.n_kv = c->n_kv;
+  p.q_mult = qm;
+  p.off = a->offset;
+  p.window = a->window;
+  p.scale_log2 = a->sm_scale * 1.4426950408889634f;
+  p.rope = a->rope_fused ? 1 : 0;
+  p.ring_cap = c->ring > 0 ? c->cap : 0;
+  p.R = R;
+  p.N = N;
+  p.n_blk = (a->T + R - 1) / R;
+  const long long units = (long long)a->B * c->n_kv * p.n_blk;
+  if (units > INT32_MAX) return SA_ERR_SHAPE;
+  p.n_units = (int)units;
+  static std::atomic<uint64_t> smem_set{0};
+  {
+    const sa_status sm = set_smem_once(sa::band_kernel<64>, Cfg::SMEM_BYTES, smem_set);
+    if (sm != SA_OK) return sm;
+  }
+  // persistent: one CTA per SM (or per unit when there are fewer)
+  const int grid = (int)(units < num_sms() ? units : num_sms());
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(Cfg::NUM_THREADS);
+  lc.dynamicSmemBytes = Cfg::SMEM_BYTES;
+  lc.stream = stream;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&lc, sa::band_kernel<64>, tmQ, tmK, tmV, tmKw, tmVw, tmO, p);
   return (last_launch_status() == SA_OK && e == cudaSuccess) ? SA_OK : SA_ERR_CUDA;
 }
 
@@ -891,6 +980,21 @@ sa_status sa_attn_prefill(sa_kv_cache* cache, const sa_attn_args* a, sa_stream_t
   if (a->T == 0) return SA_OK;
   cudaStream_t s = (cudaStream_t)stream;
   bool staged = false;
+  const int band_n = band_columns(cache, a);
+  if (band_n > 0) {
+    // band layer with packed heads: the staging launch appends K/V only (the
+    // kernel rotates its own queries) and the kernel needs no schedule slot
+    st = launch_stage(cache, a, false, s);
+    if (st == SA_OK) {
+      staged = true;
+      cudaEvent_t ev0 = g_prefill_ev_before, ev1 = g_prefill_ev_after;
+      if (ev0 != nullptr && cudaEventRecord(ev0, s) != cudaSuccess) st = SA_ERR_CUDA;
+      if (st == SA_OK) st = launch_band(cache, a, band_n, s);
+      if (st == SA_OK && ev1 != nullptr && cudaEventRecord(ev1, s) != cudaSuccess) st = SA_ERR_CUDA;
+    }
+    if (staged) note_append(cache, cache->offset, a->T);
+    return st;
+  }
   // The schedule slot (and the wait for its previous user) is taken before
   // the staging launch, so nothing stands between the two kernels.
   st = with_sched_slot(s, [&](int slot) -> sa_status {

@@ -28,7 +28,8 @@ def _tables(cfg, max_pos):
                                y["beta"], device=DEV)
 
 
-def test_zero_wait_limit_reports_timeout_and_context_survives(cuda_device):
+@pytest.mark.parametrize("window", [0, 16], ids=["full", "band"])
+def test_zero_wait_limit_reports_timeout_and_context_survives(cuda_device, window):
     cfg = wl.scaled(wl.CONFIGS["tiny"], B=2)
     off = 3000
     cap = off + 300
@@ -41,9 +42,9 @@ def test_zero_wait_limit_reports_timeout_and_context_survives(cuda_device):
         kp, vp = wl.prefilled_cache_rows(cfg, rows=off, device=DEV)
         cache.append(kp, vp)
         q, k, v = wl.qkv(cfg, 256, device=DEV)
-        sa.attn_prefill(cache, q, k, v, sinks, 0, cfg.sm_scale, cos, sin)
+        sa.attn_prefill(cache, q, k, v, sinks, window, cfg.sm_scale, cos, sin)
         qd, kd, vd = wl.qkv(cfg, 1, step=1, device=DEV)
-        sa.attn_decode(cache, qd, kd, vd, sinks, 0, cfg.sm_scale, cos, sin)
+        sa.attn_decode(cache, qd, kd, vd, sinks, window, cfg.sm_scale, cos, sin)
         torch.cuda.synchronize()
         status = sa.device_status()
     finally:

@@ -169,6 +169,24 @@ def test_prefill_matches_oracle(cuda_device, name, over, off, T, layer):
     assert cache.offset == ocache.offset == n
 
 
+@pytest.mark.parametrize("q_mult,off,T", [(8, 0, 700), (8, 77, 300), (8, 1000, 33), (8, 0, 1), (4, 13, 500),
+                                         (4, 200, 129), (1, 5, 260)],
+                         ids=["qm8", "qm8_unaligned", "qm8_short", "qm8_one_row", "qm4", "qm4_offset", "mha_w2"])
+def test_band_packed_heads_matches_oracle(cuda_device, q_mult, off, T):
+    # Band layers of d = 64 whose key window fits the packed-head kernel (the
+    # query heads of a KV group share the MMA rows): W = 128 with q_mult 8
+    # (16 positions per unit), W = 96 with q_mult 4 (32), W = 2 with q_mult 1
+    # (128). Unaligned offsets, ragged last units, a single row, a prefix
+    # shorter than the window.
+    window = {8: 128, 4: 96, 1: 2}[q_mult]
+    cfg = wl.scaled(wl.CONFIGS["tiny"], B=2, n_q=2 * q_mult, n_kv=2, d=64)
+    out, lse, ref, ref_lse, cache, ocache = _run_prefill_case(cfg, off, T, window)
+    check_bf16_output(out, ref, f"band q_mult={q_mult} off={off} T={T}")
+    check_lse(lse, ref_lse, f"band q_mult={q_mult} off={off} T={T}")
+    n = off + T
+    assert np.array_equal(to64(cache.v_rows(0, n)), ocache.V[:, :n])
+
+
 @pytest.mark.parametrize("window", [0, 16, 1000])
 def test_prefill_no_sink_and_prerotated(cuda_device, window):
     cfg = wl.scaled(wl.CONFIGS["tiny"], B=2, n_q=8, n_kv=4)
@@ -430,13 +448,14 @@ def test_handoff_prefill_equals_prefix_plus_decode(cuda_device, layer):
         assert cache.offset == cfg.offset + cfg.T
 
 
-@pytest.mark.parametrize("layer", [0, 1], ids=["band", "full"])
+@pytest.mark.parametrize("layer,n_q", [(0, 2), (0, 8), (1, 2)], ids=["band", "band_packed", "full"])
 @pytest.mark.parametrize("off,T", [(0, 300), (65536 - 3, 40)])
-def test_mask_position_probe_bit_exact(cuda_device, layer, off, T):
+def test_mask_position_probe_bit_exact(cuda_device, layer, n_q, off, T):
     # q = 0 and sink = 0: every admitted score is 0, so weights are 1/(n+1).
     # With v_j = e_{j mod d}, round(out_c * (n+1)) counts admitted keys
     # j = c mod d (band layers); lse = ln(n+1) recovers n (full layers).
-    B, n_q, n_kv, d = 1, 2, 1, 64
+    # n_q = 8 on one KV head takes the packed-head band kernel.
+    B, n_kv, d = 1, 1, 64
     window = 128 if layer == 0 else 0
     cap = off + T
     cache = sa.KVCache(B, cap, n_kv, d, device=DEV)
