@@ -205,11 +205,14 @@ __device__ __forceinline__ void band_softmax(const BandParams& p, uint8_t* smem,
     // admitted columns: keys max(qp - W + 1, 0) .. qp
     const int cmin = max(qp - p.window + 1, 0) - kb;
     const int cmax = qp - kb;
-    auto mask16 = [&](uint32_t (&v)[16], int c0) {
+    // masks chunk j's scores in registers and, for pass 2, in TMEM
+    auto mask16 = [&](uint32_t (&v)[16], int j) {
+      const int c0 = 16 * j;
       if (__any_sync(0xffffffffu, c0 < cmin || c0 + 15 > cmax)) {
 #pragma unroll
         for (int c = 0; c < 16; ++c)
           if (c0 + c < cmin || c0 + c > cmax) v[c] = __float_as_uint(-INFINITY);
+        tmem_st16(s_tm + c0, v);
       }
     };
     // pass 1: this half's row maximum, two chunks per TMEM round trip
@@ -222,7 +225,7 @@ __device__ __forceinline__ void band_softmax(const BandParams& p, uint8_t* smem,
         tmem_ld16(s_tm + 16 * (j0 + jj), v0);
         if (two) tmem_ld16(s_tm + 16 * (j0 + jj + 1), v1);
         tmem_wait_ld();
-        mask16(v0, 16 * (j0 + jj));
+        mask16(v0, j0 + jj);
         float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 16; c += 4) {
@@ -230,7 +233,7 @@ __device__ __forceinline__ void band_softmax(const BandParams& p, uint8_t* smem,
           m1 = max3f(m1, __uint_as_float(v0[c + 2]), __uint_as_float(v0[c + 3]));
         }
         if (two) {
-          mask16(v1, 16 * (j0 + jj + 1));
+          mask16(v1, j0 + jj + 1);
 #pragma unroll
           for (int c = 0; c < 16; c += 4) {
             m0 = max3f(m0, __uint_as_float(v1[c]), __uint_as_float(v1[c + 1]));
@@ -256,8 +259,7 @@ __device__ __forceinline__ void band_softmax(const BandParams& p, uint8_t* smem,
     // pass 2: exp2, the partial sum, P. P of chunk j (8 bf16-pair columns)
     // goes over the first half of S chunk j's own columns, already read.
     float l0 = 0.f, l1 = 0.f, l2 = 0.f, l3 = 0.f;
-    auto exp_chunk = [&](uint32_t (&v)[16], int j) {
-      mask16(v, 16 * j);
+    auto exp_chunk = [&](uint32_t (&v)[16], int j) {   // scores masked in pass 1
       uint32_t pk[8];
 #pragma unroll
       for (int c = 0; c < 8; c += 2) {

@@ -465,12 +465,14 @@ __device__ __forceinline__ void rope_pair_f64(float x1, float x2, float c, float
 // bf16 numbers; the midpoint inside v's bf16 interval is v's bit pattern with
 // the low 16 bits set to 0x8000 (same sign and binade, so v - mid is exact),
 // and every other midpoint is at least |v| 2^-10 away. With both distances
-// above e, v and the exact value round to the same bf16.
+// above e, v and the exact value round to the same bf16. The three tests
+// are folded into one compare: min(|v - mid|, |v| 2^-10) > max(e, 2^-110)
+// implies both distances exceed e and |v| > 2^-100.
 __device__ __forceinline__ bool rope_fast_ok(float v, float t) {
   const float av = fabsf(v);
   const float e = (av + fabsf(t)) * 0x1p-23f;
   const float mid = __uint_as_float((__float_as_uint(v) & 0xFFFF0000u) | 0x8000u);
-  return (fabsf(v - mid) > e) & (av * 0x1p-10f > e) & (av >= 0x1p-100f);
+  return fminf(fabsf(v - mid), av * 0x1p-10f) > fmaxf(e, 0x1p-110f);
 }
 
 __device__ __forceinline__ void rope_pair(float x1, float x2, float c, float s, uint32_t& y1,
