@@ -651,68 +651,121 @@ def long_decode(dev, peaks, steps=8, layers=24, ring=False, fp8=False):
                              + (", e4m3 codes + fp32 row scales [B][n_kv][cap]" if fp8 else ", bf16"))}
 
 
-def e2e_handoff(step, steps, warmup):
+def e2e_handoff(step, steps, warmup, groups=4):
     """The same step through host buffers, through the library's public API:
     every step copies its inputs from pinned host memory and its outputs back
     to pinned host memory.
-    * Prefill phase: the chunk's q/k/v of both layers go up on a copy stream
-      (layer 1's copy overlaps layer 0's prefill), each layer's output comes
-      back on a second copy stream as soon as it is computed; the phase ends
-      when the last output has landed on the host.
-    * Decode phase: per decode step, the new rows' q/k/v of both layers go up,
-      both layers decode, and their outputs come back, in order on one stream
-      (each step's input would depend on the previous step's output).
+    * Prefill phase: the 16 sequences go through in `groups` groups (the
+      sequences of a batch are independent): a group's q/k/v of both layers
+      go up on a copy stream, the group's two prefill calls run on caches that
+      view the group's rows of each layer's cache, and its outputs come back
+      on a second copy stream, so the copies of one group overlap the
+      attention of another. The phase ends when the last output has landed
+      on the host.
+    * Decode phase: each layer's whole-batch cache is brought to the chunk's
+      end (its prefix snapshot restored, the chunk rows the group calls wrote
+      appended in place); then per decode step one copy brings the new rows'
+      q/k/v of both layers up (packed in one pinned buffer), both layers
+      decode on the whole batch, and one copy takes both outputs back, in
+      order on one stream (each step's input would depend on the previous
+      step's output).
     Phase times come from events on the launch stream. Returns (prefill ms,
     decode ms) per step, and the host-to-device and device-to-host bytes per
     step."""
-    cfg = step.cfg
-    host, dev_in, dev_out, host_out = [], [], [], []
+    sa, cfg = step.sa, step.cfg
+    B, nl = cfg.B, len(step.layers)
+    gsz = B // groups
+    spans = [(gi * gsz, (gi + 1) * gsz) for gi in range(groups)]
+    # per layer: pinned chunk inputs, device copies, device and pinned outputs
+    host_in, dev_in, dev_out, host_out = [], [], [], []
     for L in step.layers:
-        host.append([L[n].cpu().pin_memory() for n in ("q", "k", "v", "dq", "dk", "dv")])
-        dev_in.append([torch.empty_like(L[n]) for n in ("q", "k", "v")]
-                      + [torch.empty_like(L[n][:, :1]) for n in ("dq", "dk", "dv")])
-        dev_out.append((torch.empty_like(L["out"]), torch.empty_like(L["dec"][:, :1])))
-        host_out.append((torch.empty(L["out"].shape, dtype=torch.bfloat16).pin_memory(),
-                         torch.empty(L["dec"].shape, dtype=torch.bfloat16).pin_memory()))
-    h2d = sum(t.numel() * t.element_size() for hs in host for t in hs)
-    d2h = sum(a.numel() * 2 + b.numel() * 2 for a, b in host_out)
+        host_in.append([L[n].cpu().pin_memory() for n in ("q", "k", "v")])
+        dev_in.append([torch.empty_like(L[n]) for n in ("q", "k", "v")])
+        dev_out.append(torch.empty_like(L["out"]))
+        host_out.append(torch.empty(L["out"].shape, dtype=torch.bfloat16).pin_memory())
+    # caches over each group's sequences, sharing the layers' cache memory,
+    # at the prefix offset
+    sub, sub_snap = [], []
+    for L in step.layers:
+        row, row_snap = [], []
+        for g0, g1 in spans:
+            c = sa.KVCache(g1 - g0, step.cap, cfg.n_kv, cfg.d, device=step.dev, k=L["cache"].k[g0:g1],
+                           v=L["cache"].v[g0:g1])
+            c.append(c.k_rows(0, step.off), c.v_rows(0, step.off))   # in place: rows [0, offset) as they are
+            row.append(c)
+            row_snap.append(c.snapshot())
+        sub.append(row)
+        sub_snap.append(row_snap)
+    # decode: both layers' new rows of every step packed in one pinned buffer
+    n_q, n_kv, d = cfg.n_q, cfg.n_kv, cfg.d
+    per_layer = B * (n_q + 2 * n_kv) * d
+    dec_host = torch.empty((step.n_dec, nl * per_layer), dtype=torch.bfloat16).pin_memory()
+    for li, L in enumerate(step.layers):
+        for st in range(step.n_dec):
+            parts = [L[n][:, st].reshape(-1).cpu() for n in ("dq", "dk", "dv")]
+            dec_host[st, li * per_layer:(li + 1) * per_layer] = torch.cat(parts)
+    dec_dev = torch.empty(nl * per_layer, dtype=torch.bfloat16, device=step.dev)
+    dec_views = []
+    for li in range(nl):
+        base = li * per_layer
+        q = dec_dev[base:base + B * n_q * d].view(B, 1, n_q, d)
+        k = dec_dev[base + B * n_q * d:base + B * (n_q + n_kv) * d].view(B, 1, n_kv, d)
+        v = dec_dev[base + B * (n_q + n_kv) * d:base + per_layer].view(B, 1, n_kv, d)
+        dec_views.append((q, k, v))
+    dec_out_dev = torch.empty((nl, B, 1, n_q, d), dtype=torch.bfloat16, device=step.dev)
+    dec_out_host = torch.empty((step.n_dec, nl, B, 1, n_q, d), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for hs in host_in for t in hs) + dec_host.numel() * 2
+    d2h = sum(t.numel() * 2 for t in host_out) + dec_out_host.numel() * 2
     comp = torch.cuda.current_stream()
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
-    nl = len(step.layers)
-    landed = [torch.cuda.Event() for _ in range(nl)]
-    computed = [torch.cuda.Event() for _ in range(nl)]
-    read = [torch.cuda.Event() for _ in range(nl)]
+    landed = [torch.cuda.Event() for _ in range(groups)]
+    computed = [torch.cuda.Event() for _ in range(groups)]
+    read = [torch.cuda.Event() for _ in range(groups)]
     last_read = torch.cuda.Event()
 
     def one(ev=None):
         if ev is not None:
             ev[0].record(comp)
         s_in.wait_stream(comp)     # the previous step has finished with the input buffers
-        for li in range(nl):
-            with torch.cuda.stream(s_in):
-                for hsrc, dst in zip(host[li][:3], dev_in[li][:3]):
-                    dst.copy_(hsrc, non_blocking=True)
-                landed[li].record(s_in)
-        for li in range(nl):
-            comp.wait_event(landed[li])
-            comp.wait_event(read[li])
-            step.prefill_phase_layer(li, dev_in[li], dev_out[li][0])
-            computed[li].record(comp)
+        with torch.cuda.stream(s_in):
+            for gi, (g0, g1) in enumerate(spans):
+                for li in range(nl):
+                    for hsrc, dst in zip(host_in[li], dev_in[li]):
+                        dst[g0:g1].copy_(hsrc[g0:g1], non_blocking=True)
+                landed[gi].record(s_in)
+        step.tables()
+        for gi, (g0, g1) in enumerate(spans):
+            comp.wait_event(landed[gi])
+            comp.wait_event(read[gi])   # the previous step's outputs of this group have been read
+            for li, L in enumerate(step.layers):
+                c = sub[li][gi]
+                c.restore(sub_snap[li][gi])
+                q, k, v = (t[g0:g1] for t in dev_in[li])
+                sa.attn_prefill(c, q, k, v, L["sinks"], L["window"], cfg.sm_scale, step.cos, step.sin,
+                                out=dev_out[li][g0:g1])
+            computed[gi].record(comp)
             with torch.cuda.stream(s_out):
-                s_out.wait_event(computed[li])
-                host_out[li][0].copy_(dev_out[li][0], non_blocking=True)
-                read[li].record(s_out)
+                s_out.wait_event(computed[gi])
+                for li in range(nl):
+                    host_out[li][g0:g1].copy_(dev_out[li][g0:g1], non_blocking=True)
+                read[gi].record(s_out)
         last_read.record(s_out)
         comp.wait_event(last_read)
         if ev is not None:
             ev[1].record(comp)
+        for L in step.layers:
+            # the whole batch's cache to offset + T over the chunk the group
+            # calls wrote: restore the prefix and append those rows in place
+            c = L["cache"]
+            c.restore(L["snap"])
+            c.append(c.k_rows(step.off, step.off + step.T), c.v_rows(step.off, step.off + step.T))
         for st in range(step.n_dec):
-            for li in range(nl):
-                for hsrc, dst in zip(host[li][3:], dev_in[li][3:]):
-                    dst.copy_(hsrc[:, st:st + 1], non_blocking=True)
-            step.decode_phase(ins=[d for d in dev_in], outs=dev_out, first=st, count=1)
-            for li in range(nl):
-                host_out[li][1][:, st:st + 1].copy_(dev_out[li][1], non_blocking=True)
+            dec_dev.copy_(dec_host[st], non_blocking=True)
+            for li, L in enumerate(step.layers):
+                q, k, v = dec_views[li]
+                sa.attn_decode(L["cache"], q, k, v, L["sinks"], L["window"], cfg.sm_scale, step.cos, step.sin,
+                               workspace=L["ws"], out=dec_out_dev[li])
+            dec_out_host[st].copy_(dec_out_dev, non_blocking=True)
         if ev is not None:
             ev[2].record(comp)
 
