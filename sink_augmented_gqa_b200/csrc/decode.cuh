@@ -214,10 +214,13 @@ __device__ __forceinline__ void decode_subtile(uint32_t kbase, uint32_t vbase, u
     pr[e] = ex2(s[e] - m_use);
     pr[2 + e] = ex2(s[2 + e] - m_use);
     l[e] = l[e] * alpha + pr[e] + pr[2 + e];
+    // the accumulators move only when some head's maximum grew (alpha < 1)
+    if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-    for (int md = 0; md < D / 16; ++md) {
-      o[md][e] *= alpha;
-      o[md][2 + e] *= alpha;
+      for (int md = 0; md < D / 16; ++md) {
+        o[md][e] *= alpha;
+        o[md][2 + e] *= alpha;
+      }
     }
     m[e] = m_new;
   }
@@ -359,10 +362,13 @@ __device__ __forceinline__ void decode_subtile_f8(uint32_t kst, uint32_t vst, ui
       pw[u][2 + e] *= inv;
     }
     const float ao = alpha[e] * fo;
+    // the accumulators move only when a maximum or a power of two changed
+    if (__any_sync(0xffffffffu, ao != 1.f)) {
 #pragma unroll
-    for (int md = 0; md < D / 16; ++md) {
-      o[md][e] *= ao;
-      o[md][2 + e] *= ao;
+      for (int md = 0; md < D / 16; ++md) {
+        o[md][e] *= ao;
+        o[md][2 + e] *= ao;
+      }
     }
   }
   // ---- O^T += V^T P'^T: lane (r, cq) reads one 32-bit word (code bytes
