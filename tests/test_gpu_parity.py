@@ -298,14 +298,17 @@ def test_prefill_and_decode_window_edges_mha(cuda_device, window):
 
 
 @pytest.mark.parametrize("over", [dict(B=2, n_q=8, n_kv=2, d=64),
+                                  dict(B=2, n_q=16, n_kv=2, d=64),
                                   dict(B=2, n_q=8, n_kv=4, d=96, sm_scale=1 / math.sqrt(96)),
                                   dict(B=1, n_q=4, n_kv=1, d=128, sm_scale=1 / math.sqrt(128))],
-                         ids=["d64", "d96", "d128"])
+                         ids=["d64", "d64_packed_heads", "d96", "d128"])
 def test_ring_cache_matches_oracle(cuda_device, over):
     # A band layer on a 384-row ring: prefill, decode, a second prefill chunk
     # that wraps the ring, decode again, then snapshot / restore. Every output
     # against the oracle on a plain (unbounded) cache; the ring's live rows
-    # against the oracle's rows of the same positions.
+    # against the oracle's rows of the same positions. With q_mult 8 the
+    # prefill takes the packed-head band kernel, whose key windows that wrap
+    # the ring are loaded as 16-row boxes.
     cfg = wl.scaled(wl.CONFIGS["tiny"], **over)
     W, cap = 128, 384
     n_total = 200 + 3 + 250 + 6
