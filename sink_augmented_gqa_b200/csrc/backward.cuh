@@ -9,10 +9,10 @@
 //   dv_j = sum P_ij dO_i  (dk, dv summed over the heads of the KV group);
 //   dsink_h = -sum_{b,i} exp(sink_h - lse_i) D_i  (the sink carries no value).
 //
-// Three launches: the row pass below (D and the sink gradient), then the
-// key-tile pass (dK, dV) and the query-tile pass (dQ) of backward_tc.cuh on
-// the tcgen05 tensor cores (bf16 operands, fp32 accumulation in TMEM; P and
-// dS enter their products as bf16); outputs are fp32.
+// Two launches: the row pass below (D, the sink gradient, and dq cleared),
+// then the products of backward_tc.cuh on the tcgen05 tensor cores (bf16
+// operands, fp32 accumulation in TMEM; P and dS enter their products as
+// bf16), which accumulate dq with reductions; outputs are fp32.
 #pragma once
 
 #include "ptx.cuh"
@@ -30,7 +30,7 @@ struct BwdParams {
   const float* sinks;    // [n_q] or null
   float* dvec;           // [B][n_q][Tp] workspace: D_i (0 for rows past T)
   float* lse2;           // [B][n_q][Tp] workspace: lse_i * log2(e) (+inf for rows past T)
-  int Tp;                // T rounded up to a multiple of 64 (whole streamed tiles per row)
+  int Tp;                // T rounded up to a multiple of 384 (whole streamed tiles of 64, 96 or 128 rows)
   float* dq;             // [B][T][n_q][d]
   float* dk;             // [B][T][n_kv][d]
   float* dv;             // [B][T][n_kv][d]
@@ -41,7 +41,8 @@ struct BwdParams {
 };
 
 // D_i = <dO_i, o_i> and lse_i log2(e) per (b, i, h) into the padded
-// workspace rows, one warp per four rows; each row also adds -exp(sink_h - lse_i) D_i
+// workspace rows, one warp per four rows, which also clears the row's dq
+// (the products add into it); each row also adds -exp(sink_h - lse_i) D_i
 // to dsinks[h], through a per-block sum in shared memory (dynamic, n_q
 // floats) so that global memory sees one atomic per block and head. Rows
 // T..Tp-1 get the values of an empty row (D 0, lse +inf).
@@ -97,6 +98,9 @@ __global__ void bwd_rows_kernel(const BwdParams p) {
           const __nv_bfloat16* drow = p.dout + b * p.ds0 + i * p.ds1 + h * p.ds2;
 #pragma unroll
           for (int c = lane; c < D; c += 32) acc[j] = fmaf(__bfloat162float(orow[c]), __bfloat162float(drow[c]), acc[j]);
+          float* qrow = p.dq + (((long long)b * p.T + i) * p.n_q + h) * D;
+#pragma unroll
+          for (int c = lane; c < D; c += 32) qrow[c] = 0.f;
         }
         step(b, i, h);
       }

@@ -1,35 +1,42 @@
-// Backward pass on tcgen05 tensor cores: the same gradients as backward.cuh,
-// from two kernels shaped like the forward prefill kernel:
+// Backward pass on tcgen05 tensor cores: every gradient of backward.cuh
+// (dQ, dK, dV) from one launch whose CTAs each keep 128 keys of one KV head
+// resident and stream the query tiles of every head of the group that see
+// them:
 //
-//   MODE 0 (dQ)   rows = 128 queries of one head; streams the admitted key
-//                 tiles: S = Q K^T, dP = dO V^T (smem x smem into TMEM),
-//                 dS = P (dP - D) as bf16 into TMEM, dQ += dS K (TMEM x smem).
-//   MODE 1 (dKdV) rows = 128 keys of one KV head; streams the query tiles
-//                 of every head of the group that see them: S^T = K Q^T,
-//                 dP^T = V dO^T, P^T and dS^T as bf16 into TMEM, then
-//                 dV += P^T dO and dK += dS^T Q.
+//   S^T  = K Q^T,  dP^T = V dO^T          smem x smem into TMEM (keys = TMEM lanes)
+//   P^T  = exp2(S^T scale log2 e - lse log2 e),  dS^T = P^T (dP^T - D)
+//          formed by 16 warps, one key row per thread, and written as bf16
+//          to shared memory in the layouts the next products read
+//   dV  += P^T dO,  dK += dS^T Q          accumulated in TMEM over the CTA's tiles
+//   dQ^T = K^T dS^T                        per tile, into TMEM; the same warps
+//          add it to the fp32 dq rows in global memory (one 128-byte row
+//          segment per reduction instruction)
 //
-// One CTA per 128-row tile (both passes in one launch, heaviest tiles first),
-// 576 threads:
-//   warp 0      TMA loads: the two resident 128-row tiles once, then per
-//               streamed tile its two BN-row tiles into an NS-deep ring (MODE 1
-//               also stages the tile's lse and D values there).
-//   warp 1      one thread issues the MMAs and owns the TMEM allocation. S and
-//               dP are double-buffered in TMEM: the tensor core computes the
-//               next tile's S, dP while this tile's P, dS are formed. P and dS
-//               (bf16) get a single buffer of their own where TMEM has room
-//               (every case but dK/dV at d = 128): an S / dP buffer is then
-//               free as soon as its values are read, and the P / dS warps
-//               wait for the previous tile's products only before storing.
-//               Otherwise P, dS are written over the S, dP columns they came
-//               from, and the issuer waits for tile u - 2's products before
-//               tile u reuses that buffer.
-//   warps 2-17  P, dS from S, dP: four warps per TMEM lane quarter (warp % 4),
-//               each taking a quarter of a tile's columns, one row per thread;
-//               tiles wholly inside the admitted region skip the mask; then the
-//               fp32 output rows (the warps of a quarter split the columns).
-// P_ij = exp2(s_ij scale_log2 - lse_i log2 e) uses the forward's lse (sink
-// included), so no running max is needed.
+// Five products per (key, query) pair: S and dP are formed once for all
+// three gradients. BN, the query rows of a streamed tile, is what TMEM holds
+// next to the accumulators: S^T, dP^T and dQ^T (BN columns each), dV, dK (D
+// each): 3 BN + 2 D <= 512 gives BN = 128 at d = 64, 96 at d = 96, 64 at
+// d = 128. dQ^T's products have M = 128 rows of d; at d < 128 the rows past d
+// read the start of the V tile (stored right after K) and are never read
+// back.
+//
+// 576 threads per CTA, one CTA per SM (each holds all 512 TMEM columns):
+//   warp 0      TMA: K and V once; per streamed tile its Q and dO tiles and
+//               the tile's lse log2 e and D values (bulk copies) into an
+//               NS-deep ring.
+//   warp 1      one thread issues the MMAs and owns the TMEM allocation. It
+//               issues tile u's S^T, dP^T as soon as the warps have read tile
+//               u - 1's, then tile u - 1's dV, dK and dQ^T products once its
+//               P^T, dS^T are in shared memory: the tensor cores form the
+//               next scores while the warps work on the current tile.
+//   warps 2-17  P^T, dS^T from S^T, dP^T (four warps per TMEM lane quarter,
+//               each a quarter of the tile's columns); then, once the previous
+//               tile's products are done, that tile's dQ^T into dq, and this
+//               tile's P^T, dS^T into shared memory; at the end dV, dK (fp32
+//               rows).
+// dq must be zero before the launch (the row pass clears it). The order in
+// which the key tiles' contributions reach a dq element varies, so dq can
+// differ in the last bits between calls; dk and dv do not.
 #pragma once
 
 #include "backward.cuh"
@@ -37,158 +44,140 @@
 
 namespace sa {
 
-__host__ __device__ constexpr int btc_align32(int x) { return (x + 31) / 32 * 32; }
-
-template <int D, int MODE>
-struct BtcCfg {
-  static constexpr int BM = 128;                                     // resident rows
-  static constexpr int BN = 64;                                      // streamed rows per tile
-  static constexpr int CB = (D % 64 == 0) ? 64 : 32;                 // column block (elements)
+template <int D>
+struct BkvCfg {
+  static constexpr int BM = 128;                                     // resident keys
+  static constexpr int BN = (D == 64) ? 128 : (D == 96 ? 96 : 64);   // streamed queries per tile
+  static constexpr int CB = (D % 64 == 0) ? 64 : 32;                 // d column block (elements)
   static constexpr int SWZ = CB * 2;                                 // bytes per block row
   static constexpr int NCB = D / CB;
   static constexpr uint32_t LAYOUT = (SWZ == 128) ? 2u : 4u;
   static constexpr uint32_t SBO = 8u * SWZ;
-  static constexpr uint32_t MBLOCK = (uint32_t)BM * SWZ;
+  static constexpr uint32_t MBLOCK = (uint32_t)BM * SWZ;             // one d block of K or V
   static constexpr uint32_t M_BYTES = (uint32_t)BM * D * 2;
-  static constexpr uint32_t NBLOCK = (uint32_t)BN * SWZ;
+  static constexpr uint32_t NBLOCK = (uint32_t)BN * SWZ;             // one d block of Q or dO
   static constexpr uint32_t N_BYTES = (uint32_t)BN * D * 2;
-  static constexpr int NS = (D == 128) ? 3 : 4;
-  static constexpr uint32_t STAGE_BYTES = 2 * N_BYTES;
-  static constexpr uint32_t OFF_R0 = 0;                              // Q (MODE 0) | K (MODE 1)
-  static constexpr uint32_t OFF_R1 = M_BYTES;                        // dO | V
-  static constexpr uint32_t OFF_ST = 2 * M_BYTES;                    // ring: [K | Q], [V | dO]
-  static constexpr uint32_t OFF_ROWV = OFF_ST + NS * STAGE_BYTES;    // MODE 1: [NS][2][BN] fp32
+  // P^T and dS^T: [BM keys][BN queries] in column blocks of CQ queries
+  static constexpr int CQ = (BN % 64 == 0) ? 64 : 32;
+  static constexpr int SWQ = CQ * 2;
+  static constexpr uint32_t LAYOUT_Q = (SWQ == 128) ? 2u : 4u;
+  static constexpr uint32_t SBO_Q = 8u * SWQ;
+  static constexpr uint32_t QBLOCK = (uint32_t)BM * SWQ;
+  static constexpr uint32_t PS_BYTES = (uint32_t)BM * BN * 2;
+  static constexpr int NS = 3;
+  static constexpr uint32_t STAGE_BYTES = 2 * N_BYTES;               // [Q | dO]
+  static constexpr uint32_t OFF_K = 0;
+  static constexpr uint32_t OFF_V = M_BYTES;                         // right after K (see dQ^T)
+  static constexpr uint32_t OFF_ST = 2 * M_BYTES;
+  static constexpr uint32_t OFF_P = OFF_ST + NS * STAGE_BYTES;
+  static constexpr uint32_t OFF_DS = OFF_P + PS_BYTES;
+  static constexpr uint32_t OFF_ROWV = OFF_DS + PS_BYTES;            // [NS][2][BN] fp32: lse log2 e, D
   static constexpr uint32_t OFF_BAR = OFF_ROWV + NS * 2 * BN * 4;
-  // at least 120 KB: one CTA per SM, since each allocates all 512 TMEM columns
-  static constexpr uint32_t SMEM_BYTES = (OFF_BAR + 256 + 1024) > 120u * 1024 ? (OFF_BAR + 256 + 1024) : 120u * 1024;
-  // TMEM columns. S[buf] at S_COL + buf * BN, dP[buf] at DP_COL + buf * BN.
-  // SEP: P and dS (bf16 pairs, BN / 2 columns each) have columns of their own
-  // after the S / dP buffers, so an S / dP buffer is free again once its
-  // values are read; otherwise (dK and dV of d = 128 leave no room) P and dS
-  // are written over the start of the S / dP columns they came from.
+  static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
+  // TMEM columns
   static constexpr int S_COL = 0;
-  static constexpr int DP_COL = 2 * BN;
-  static constexpr bool SEP = 5 * BN + (MODE == 0 ? D : 2 * D) <= 512;
-  static constexpr int P_COL = SEP ? 4 * BN : S_COL;                  // MODE 1
-  static constexpr int DS_COL = SEP ? 4 * BN + BN / 2 : DP_COL;
-  static constexpr int ACC0 = SEP ? 5 * BN : 4 * BN;                  // dQ | dV
-  static constexpr int ACC1 = ACC0 + D;                              // MODE 1: dK
+  static constexpr int DP_COL = BN;
+  static constexpr int DV_COL = 2 * BN;
+  static constexpr int DK_COL = 2 * BN + D;
+  static constexpr int DQ_COL = 2 * BN + 2 * D;
   static constexpr int TMEM_COLS = 512;
-  static_assert((MODE == 0 ? ACC0 + D : ACC1 + D) <= TMEM_COLS, "TMEM plan exceeds 512 columns");
-  static_assert(MBLOCK % 1024 == 0 && NBLOCK % 1024 == 0 && M_BYTES % 1024 == 0, "1 KB aligned tiles");
-  static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
-  static constexpr uint32_t IDESC_O = idesc_bf16(128, D, 0, 1);
+  static_assert(DQ_COL + BN <= TMEM_COLS, "TMEM plan exceeds 512 columns");
+  static_assert(MBLOCK % 1024 == 0 && NBLOCK % 1024 == 0 && QBLOCK % 1024 == 0 && M_BYTES % 1024 == 0 &&
+                    N_BYTES % 1024 == 0 && PS_BYTES % 1024 == 0,
+                "1 KB aligned tiles");
+  // dQ^T reads 128 / CB d blocks from OFF_K: K's own, then the start of V
+  static_assert(OFF_V == OFF_K + NCB * MBLOCK && (128 / CB) * MBLOCK <= 2 * M_BYTES, "K^T rows past d read V");
+  static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);     // K-major A and B
+  static constexpr uint32_t IDESC_O = idesc_bf16(128, D, 0, 1);      // K-major A, MN-major B
+  static constexpr uint32_t IDESC_Q = idesc_bf16(128, BN, 1, 1);     // MN-major A and B
   static constexpr int NSW = 16;                                     // P / dS warps (2..17)
-  static constexpr int NPART = NSW / 4;                              // P / dS warps per TMEM lane quarter
-  static constexpr int HC = BN / NPART;                              // columns per P / dS warp
+  static constexpr int HC = BN / 4;                                  // columns per P / dS warp
+  static constexpr int DQ_QUARTERS = (D + 31) / 32;                  // lane quarters with d rows of dQ^T
   static constexpr int NUM_THREADS = 32 * (2 + NSW);
-  static_assert(HC == 16 || HC == 32, "16 or 32 columns per P / dS warp");
-  static_assert(NPART % 2 == 0, "dK and dV epilogues take half the warps of a quarter each");
+  static_assert(HC % 8 == 0 && HC >= 16 && HC <= 32, "whole 16-byte chunks per P / dS warp");
+  static_assert(SMEM_BYTES <= 227u * 1024, "shared memory");
   // the epilogue's 32 x 33 fp32 staging slot per P / dS warp overlays the
-  // resident tiles and the ring (below the row values)
-  static_assert((uint32_t)NSW * 32 * 33 * 4 <= OFF_ROWV, "epilogue staging overlays tiles and ring");
+  // resident tiles, the ring and P / dS (below the row values)
+  static_assert((uint32_t)NSW * 32 * 33 * 4 <= OFF_ROWV, "epilogue staging overlays the tiles");
 };
 
 enum : int {
-  BB_RFULL = 0,      // resident tiles landed
-  BB_FULL = 1,       // [4] ring stage landed
-  BB_EMPTY = 5,      // [4] ring stage free (MMA commit)
-  BB_SFULL = 9,      // [2] S, dP of a buffer computed
-  BB_PFULL = 13,     // count 8 warps: P / dS stored in TMEM
-  // 14: unused (the products that read P / dS signal on the stage's EMPTY
-  // barrier, which the P / dS warps wait on as well: one commit fewer per tile)
-  BB_ACCFULL = 15,   // accumulators final
-  BB_DRAIN = 16,
-  BB_TMEM_SLOT = 17,
-  BB_ABORT_SLOT = 18,
+  BK_RFULL = 0,      // K, V landed
+  BK_FULL = 1,       // [3] ring stage landed
+  BK_EMPTY = 4,      // [3] ring stage free (MMA commit)
+  BK_SFULL = 7,      // S^T, dP^T of the current tile computed
+  BK_SREAD = 8,      // count 16 warps: S^T, dP^T read into registers
+  BK_PFULL = 9,      // count 16 warps: P^T, dS^T in shared memory (and the previous dQ^T read)
+  BK_PEMPTY = 10,    // a tile's dV, dK, dQ^T products done (P^T, dS^T free; dQ^T ready)
+  BK_DRAIN = 11,
+  BK_TMEM_SLOT = 12,
+  BK_ABORT_SLOT = 13,
 };
 
-// D = sum over K-steps of A (smem, K-major, 128 rows) B (smem, K-major, BN rows)^T
-template <int D, int MODE>
-__device__ __forceinline__ void btc_issue_s(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc) {
-  using C = BtcCfg<D, MODE>;
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t cb = kk * 16 / C::CB, cin = (kk * 16 % C::CB) * 2;
-    mma_ss(d_tmem, adesc + ((cb * C::MBLOCK + cin) >> 4), bdesc + ((cb * C::NBLOCK + cin) >> 4), C::IDESC_S,
-           kk > 0 ? 1u : 0u);
-  }
+__device__ __forceinline__ void bkv_tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                 "=r"(r[7])
+               : "r"(taddr));
 }
-// acc (+)= A (TMEM bf16, 128 x BN) B (smem [BN][D], MN-major). SEP: A's
-// elements sit, as bf16 pairs, at columns [0, BN / 2) of their own buffer;
-// otherwise elements [HC h, HC h + HC) sit at columns [HC h, HC h + HC / 2) of
-// the S / dP buffer (each P / dS warp writes over the start of the columns it
-// read).
-template <int D, int MODE>
-__device__ __forceinline__ void btc_issue_o(uint32_t acc_tmem, uint32_t a_tmem, uint64_t bdesc, bool accumulate) {
-  using C = BtcCfg<D, MODE>;
-#pragma unroll
-  for (int kk = 0; kk < C::BN / 16; ++kk) {
-    const int e = kk * 16;                                        // first element of the K-step
-    const uint32_t col = C::SEP ? (uint32_t)(e / 2) : (uint32_t)(C::HC * (e / C::HC) + (e % C::HC) / 2);
-    mma_ts(acc_tmem, a_tmem + col, bdesc + ((kk * 16 * C::SWZ) >> 4), C::IDESC_O,
-           (accumulate || kk > 0) ? 1u : 0u);
-  }
+// N consecutive 32-bit TMEM columns of this warp's 32 lanes (N = 16, 24, 32)
+template <int N>
+__device__ __forceinline__ void bkv_tmem_ld(uint32_t taddr, uint32_t* r) {
+  tmem_ld16(taddr, r);
+  if constexpr (N == 32) tmem_ld16(taddr + 16, r + 16);
+  if constexpr (N == 24) bkv_tmem_ld8(taddr + 16, r + 16);
 }
 
-// One CTA of either pass: resident row tile `tile` of query head (MODE 0) or
-// KV head (MODE 1) `head` of sequence b. tmR0 / tmR1 map the resident tiles'
-// tensors, tmS0 / tmS1 the streamed ones (kernel parameters).
-template <int D, int MODE>
-__device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtensorMap* tmR1,
-                                           const CUtensorMap* tmS0, const CUtensorMap* tmS1,
-                                           const BwdParams& p, const int tile, const int head, const int b) {
-  using C = BtcCfg<D, MODE>;
+// One CTA: keys r0 = 128 tile .. r0 + 127 of KV head g of sequence b.
+template <int D>
+__global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                  const BwdParams p) {
+  using C = BkvCfg<D>;
   constexpr int BN = C::BN;
+  constexpr int HC = C::HC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   const uint32_t bar0 = sbase + C::OFF_BAR;
   auto bar = [&](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * BB_TMEM_SLOT);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * BB_ABORT_SLOT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_BAR + 8 * BK_TMEM_SLOT);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_BAR + 8 * BK_ABORT_SLOT);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int r0 = tile * C::BM;          // first resident row
-  // Streamed tiles. MODE 0: key tiles [t_lo, t_hi) of BN keys seen by
-  // queries r0..r0+127. MODE 1: for each head of the group, query tiles
-  // [t_lo, t_hi) of BN queries that see keys r0..r0+127.
-  int t_lo, t_hi;
-  if constexpr (MODE == 0) {
-    const int j_lo = p.window > 0 ? max(r0 - p.window + 1, 0) : 0;
-    t_lo = j_lo / BN;
-    t_hi = (min(p.T, r0 + C::BM) + BN - 1) / BN;
-  } else {
-    t_lo = r0 / BN;
-    int i_end = p.T;
-    if (p.window > 0 && r0 + C::BM - 1 + p.window < i_end) i_end = r0 + C::BM - 1 + p.window;
-    t_hi = (i_end + BN - 1) / BN;
-  }
+  // Blocks in order of key tile (tile 0, the one the most queries see, first)
+  const int per_level = p.n_kv * p.B;
+  const int tile = (int)blockIdx.x / per_level;
+  const int g = ((int)blockIdx.x % per_level) % p.n_kv;
+  const int b = ((int)blockIdx.x % per_level) / p.n_kv;
+  const int r0 = tile * C::BM;
+  // Query tiles [t_lo, t_hi) of BN rows that see keys r0..r0+127 (key j is
+  // seen by queries j <= i < j + window), for each head of the group
+  const int t_lo = r0 / BN;
+  int i_end = p.T;
+  if (p.window > 0 && r0 + C::BM - 1 + p.window < i_end) i_end = r0 + C::BM - 1 + p.window;
+  const int t_hi = (i_end + BN - 1) / BN;
   const int per = t_hi > t_lo ? t_hi - t_lo : 0;
-  const int n_tiles = (MODE == 0) ? per : per * p.q_mult;
-  const int g = (MODE == 0) ? head / p.q_mult : head;
-  // streamed tile u -> (head of its Q/dO or lse/D rows, first streamed row)
-  auto stream_of = [&](int u, int& hh, int& s0) {
-    if constexpr (MODE == 0) {
-      hh = head;
-      s0 = (t_lo + u) * BN;
-    } else {
-      hh = g * p.q_mult + u / per;
-      s0 = (t_lo + u % per) * BN;
-    }
+  const int n_tiles = per * p.q_mult;
+  auto stream_of = [&](int u, int& hh, int& q0) {
+    const int x = u / per;
+    hh = g * p.q_mult + x;
+    q0 = (t_lo + u - x * per) * BN;
   };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(BB_RFULL), 1);
+    mbar_init(bar(BK_RFULL), 1);
     for (int s = 0; s < C::NS; ++s) {
-      mbar_init(bar(BB_FULL + s), 1);
-      mbar_init(bar(BB_EMPTY + s), 1);
+      mbar_init(bar(BK_FULL + s), 1);
+      mbar_init(bar(BK_EMPTY + s), 1);
     }
-    for (int x = 0; x < 2; ++x) mbar_init(bar(BB_SFULL + x), 1);
-    mbar_init(bar(BB_PFULL), C::NSW);
-    mbar_init(bar(BB_ACCFULL), 1);
-    mbar_init(bar(BB_DRAIN), 1);
+    mbar_init(bar(BK_SFULL), 1);
+    mbar_init(bar(BK_SREAD), C::NSW);
+    mbar_init(bar(BK_PFULL), C::NSW);
+    mbar_init(bar(BK_PEMPTY), 1);
+    mbar_init(bar(BK_DRAIN), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -204,192 +193,193 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      tma_prefetch_desc(tmR0);
-      tma_prefetch_desc(tmR1);
-      tma_prefetch_desc(tmS0);
-      tma_prefetch_desc(tmS1);
-      mbar_arrive_expect_tx(bar(BB_RFULL), 2 * C::M_BYTES);
-      const int rh = (MODE == 0) ? head : g;   // head of the resident tiles
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmO);
+      mbar_arrive_expect_tx(bar(BK_RFULL), 2 * C::M_BYTES);
 #pragma unroll
       for (int cb = 0; cb < C::NCB; ++cb) {
-        tma_load_4d(sbase + C::OFF_R0 + cb * C::MBLOCK, tmR0, bar(BB_RFULL), cb * C::CB, r0, rh, b);
-        tma_load_4d(sbase + C::OFF_R1 + cb * C::MBLOCK, tmR1, bar(BB_RFULL), cb * C::CB, r0, rh, b);
+        tma_load_4d(sbase + C::OFF_K + cb * C::MBLOCK, &tmK, bar(BK_RFULL), cb * C::CB, r0, g, b);
+        tma_load_4d(sbase + C::OFF_V + cb * C::MBLOCK, &tmV, bar(BK_RFULL), cb * C::CB, r0, g, b);
       }
-    }
-    int issued = 0;
-    bool ok = true;
-    for (int u = 0; u < n_tiles; ++u) {
-      const int s = u % C::NS;
-      if (u >= C::NS) {
-        bool w = true;
-        if (lane == 0) w = mbar_wait(bar(BB_EMPTY + s), (uint32_t)(((u / C::NS) - 1) & 1));
-        w = __shfl_sync(0xffffffffu, w, 0);
-        if (!w) { ok = false; break; }
-      }
-      if (*abort_flag) { ok = false; break; }
-      int hh, s0;
-      stream_of(u, hh, s0);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar(BB_FULL + s), C::STAGE_BYTES + (MODE == 1 ? 2 * BN * 4 : 0));
-        if constexpr (MODE == 1) {
-          // lse * log2(e) and D of the tile's BN query rows, beside its tiles
-          // (padded workspace rows: 16-byte aligned, valid past T)
-          const long long wb = ((long long)b * p.n_q + hh) * p.Tp + s0;
-          const uint32_t rv = sbase + C::OFF_ROWV + s * 2 * BN * 4;
-          bulk_load(rv, p.lse2 + wb, BN * 4, bar(BB_FULL + s));
-          bulk_load(rv + BN * 4, p.dvec + wb, BN * 4, bar(BB_FULL + s));
-        }
-        const int sh = (MODE == 0) ? g : hh;   // head of the streamed tiles
-        const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_BYTES;
-#pragma unroll
-        for (int cb = 0; cb < C::NCB; ++cb) {
-          tma_load_4d(st + cb * C::NBLOCK, tmS0, bar(BB_FULL + s), cb * C::CB, s0, sh, b);
-          tma_load_4d(st + C::N_BYTES + cb * C::NBLOCK, tmS1, bar(BB_FULL + s), cb * C::CB, s0, sh, b);
-        }
-      }
-      issued = u + 1;
-    }
-    if (!ok && lane == 0) {
-      *abort_flag = 1;
-      for (int u = (issued > C::NS ? issued - C::NS : 0); u < issued; ++u)
-        mbar_wait_drain(bar(BB_FULL + u % C::NS), (uint32_t)((u / C::NS) & 1));
-    }
-    if (lane == 0) mbar_wait_drain(bar(BB_RFULL), 0);
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(bar(BB_RFULL), 0);
-      tc_fence_after();
-      const uint64_t a0 = smem_desc(sbase + C::OFF_R0, 16, C::SBO, C::LAYOUT);   // Q | K, K-major
-      const uint64_t a1 = smem_desc(sbase + C::OFF_R1, 16, C::SBO, C::LAYOUT);   // dO | V
-      auto o_products = [&](int v) {   // the products of tile v that read P / dS
-        const int sv = v % C::NS;
-        const uint32_t pcol = tmem + C::P_COL + (C::SEP ? 0 : (v & 1) * BN);
-        const uint32_t dscol = tmem + C::DS_COL + (C::SEP ? 0 : (v & 1) * BN);
-        const uint32_t st = sbase + C::OFF_ST + sv * C::STAGE_BYTES;
-        if constexpr (MODE == 0) {
-          // dQ += dS K (K of the stage, MN-major)
-          btc_issue_o<D, MODE>(tmem + C::ACC0, dscol, smem_desc(st, C::NBLOCK, C::SBO, C::LAYOUT), v > 0);
-        } else {
-          // dV += P^T dO, dK += dS^T Q
-          btc_issue_o<D, MODE>(tmem + C::ACC0, pcol, smem_desc(st + C::N_BYTES, C::NBLOCK, C::SBO, C::LAYOUT),
-                               v > 0);
-          btc_issue_o<D, MODE>(tmem + C::ACC1, dscol, smem_desc(st, C::NBLOCK, C::SBO, C::LAYOUT), v > 0);
-        }
-        mma_commit(bar(BB_EMPTY + sv));   // also: tile v's P / dS have been read
-      };
-      for (int u = 0; u < n_tiles && ok; ++u) {
-        const int s = u % C::NS, x = u & 1;
-        if (!mbar_wait(bar(BB_FULL + s), (uint32_t)((u / C::NS) & 1))) { ok = false; break; }
-        // buffer x last served tile u - 2. SEP: its S / dP were read before
-        // tile u - 2's P / dS were signalled (waited for below, one tile ago);
-        // otherwise wait until the products reading its P / dS completed.
-        if (!C::SEP && u >= 2 &&
-            !mbar_wait(bar(BB_EMPTY + (u - 2) % C::NS), (uint32_t)(((u - 2) / C::NS) & 1))) {
+      int issued = 0;
+      bool ok = true;
+      for (int u = 0; u < n_tiles; ++u) {
+        const int s = u % C::NS;
+        if (u >= C::NS && !mbar_wait(bar(BK_EMPTY + s), (uint32_t)(((u / C::NS) - 1) & 1))) {
           ok = false;
           break;
         }
+        if (*abort_flag) {
+          ok = false;
+          break;
+        }
+        int hh, q0;
+        stream_of(u, hh, q0);
+        mbar_arrive_expect_tx(bar(BK_FULL + s), C::STAGE_BYTES + 2 * BN * 4);
+        // lse log2 e and D of the tile's BN query rows (padded workspace
+        // rows: whole tiles, 16-byte aligned)
+        const long long wb = ((long long)b * p.n_q + hh) * p.Tp + q0;
+        const uint32_t rv = sbase + C::OFF_ROWV + s * 2 * BN * 4;
+        bulk_load(rv, p.lse2 + wb, BN * 4, bar(BK_FULL + s));
+        bulk_load(rv + BN * 4, p.dvec + wb, BN * 4, bar(BK_FULL + s));
+        const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_BYTES;
+#pragma unroll
+        for (int cb = 0; cb < C::NCB; ++cb) {
+          tma_load_4d(st + cb * C::NBLOCK, &tmQ, bar(BK_FULL + s), cb * C::CB, q0, hh, b);
+          tma_load_4d(st + C::N_BYTES + cb * C::NBLOCK, &tmO, bar(BK_FULL + s), cb * C::CB, q0, hh, b);
+        }
+        issued = u + 1;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        for (int u = (issued > C::NS ? issued - C::NS : 0); u < issued; ++u)
+          mbar_wait_drain(bar(BK_FULL + u % C::NS), (uint32_t)((u / C::NS) & 1));
+      }
+      mbar_wait_drain(bar(BK_RFULL), 0);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(bar(BK_RFULL), 0);
+      tc_fence_after();
+      const uint64_t a_k = smem_desc(sbase + C::OFF_K, 16, C::SBO, C::LAYOUT);        // K, K-major
+      const uint64_t a_v = smem_desc(sbase + C::OFF_V, 16, C::SBO, C::LAYOUT);        // V, K-major
+      const uint64_t a_kt = smem_desc(sbase + C::OFF_K, C::MBLOCK, C::SBO, C::LAYOUT); // K^T, MN-major
+      const uint64_t a_p = smem_desc(sbase + C::OFF_P, 16, C::SBO_Q, C::LAYOUT_Q);   // P^T, K-major
+      const uint64_t a_ds = smem_desc(sbase + C::OFF_DS, 16, C::SBO_Q, C::LAYOUT_Q); // dS^T, K-major
+      const uint64_t b_ds = smem_desc(sbase + C::OFF_DS, C::QBLOCK, C::SBO_Q, C::LAYOUT_Q);  // dS^T, MN-major
+      // tile v's dV += P^T dO, dK += dS^T Q (K = BN queries) and dQ^T = K^T dS^T (K = 128 keys)
+      auto products = [&](int v) {
+        const int sv = v % C::NS;
+        const uint32_t st = sbase + C::OFF_ST + sv * C::STAGE_BYTES;
+        const uint64_t b_q = smem_desc(st, C::NBLOCK, C::SBO, C::LAYOUT);              // Q, MN-major
+        const uint64_t b_o = smem_desc(st + C::N_BYTES, C::NBLOCK, C::SBO, C::LAYOUT); // dO, MN-major
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint32_t aoff = ((uint32_t)(kk * 16 / C::CQ) * C::QBLOCK + (uint32_t)(kk * 16 % C::CQ) * 2) >> 4;
+          const uint32_t boff = ((uint32_t)kk * 16 * C::SWZ) >> 4;
+          const uint32_t acc = (v > 0 || kk > 0) ? 1u : 0u;
+          mma_ss(tmem + C::DV_COL, a_p + aoff, b_o + boff, C::IDESC_O, acc);
+          mma_ss(tmem + C::DK_COL, a_ds + aoff, b_q + boff, C::IDESC_O, acc);
+        }
+#pragma unroll
+        for (int kk = 0; kk < C::BM / 16; ++kk)
+          mma_ss(tmem + C::DQ_COL, a_kt + (((uint32_t)kk * 16 * C::SWZ) >> 4),
+                 b_ds + (((uint32_t)kk * 16 * C::SWQ) >> 4), C::IDESC_Q, kk > 0 ? 1u : 0u);
+        mma_commit(bar(BK_PEMPTY));
+        mma_commit(bar(BK_EMPTY + sv));
+      };
+      for (int u = 0; u < n_tiles && ok; ++u) {
+        const int s = u % C::NS;
+        if (!mbar_wait(bar(BK_FULL + s), (uint32_t)((u / C::NS) & 1))) { ok = false; break; }
+        // the warps have read the previous tile's S^T, dP^T
+        if (u >= 1 && !mbar_wait(bar(BK_SREAD), (uint32_t)((u - 1) & 1))) { ok = false; break; }
         tc_fence_after();
         const uint32_t st = sbase + C::OFF_ST + s * C::STAGE_BYTES;
-        // S = R0 S0^T, dP = R1 S1^T (both K-major)
-        btc_issue_s<D, MODE>(tmem + C::S_COL + x * BN, a0, smem_desc(st, 16, C::SBO, C::LAYOUT));
-        btc_issue_s<D, MODE>(tmem + C::DP_COL + x * BN, a1, smem_desc(st + C::N_BYTES, 16, C::SBO, C::LAYOUT));
-        mma_commit(bar(BB_SFULL + x));
-        if (u > 0) {
-          if (!mbar_wait(bar(BB_PFULL), (uint32_t)((u - 1) & 1))) { ok = false; break; }
+        const uint64_t b_q = smem_desc(st, 16, C::SBO, C::LAYOUT);                // Q, K-major
+        const uint64_t b_o = smem_desc(st + C::N_BYTES, 16, C::SBO, C::LAYOUT);   // dO, K-major
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t cb = kk * 16 / C::CB, cin = (kk * 16 % C::CB) * 2;
+          mma_ss(tmem + C::S_COL, a_k + ((cb * C::MBLOCK + cin) >> 4), b_q + ((cb * C::NBLOCK + cin) >> 4),
+                 C::IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + C::DP_COL, a_v + ((cb * C::MBLOCK + cin) >> 4), b_o + ((cb * C::NBLOCK + cin) >> 4),
+                 C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar(BK_SFULL));
+        if (u >= 1) {
+          if (!mbar_wait(bar(BK_PFULL), (uint32_t)((u - 1) & 1))) { ok = false; break; }
           tc_fence_after();
-          o_products(u - 1);
+          products(u - 1);
         }
         if (*abort_flag) { ok = false; break; }
       }
       if (ok && n_tiles > 0) {
-        if (mbar_wait(bar(BB_PFULL), (uint32_t)((n_tiles - 1) & 1))) {
+        if (mbar_wait(bar(BK_PFULL), (uint32_t)((n_tiles - 1) & 1))) {
           tc_fence_after();
-          o_products(n_tiles - 1);
-          mma_commit(bar(BB_ACCFULL));
+          products(n_tiles - 1);
         } else {
           ok = false;
         }
       }
       if (!ok) {
         *abort_flag = 1;
-        mma_commit(bar(BB_DRAIN));
-        mbar_wait_drain(bar(BB_DRAIN), 0);
+        mma_commit(bar(BK_DRAIN));
+        mbar_wait_drain(bar(BK_DRAIN), 0);
       }
     }
   } else {
-    // ------------------------------------------------------------ dS and the epilogue
-    constexpr int HC = C::HC;
+    // ------------------------------------------------------------ P^T, dS^T, dQ and the epilogue
     const int quarter = warp & 3;
-    const int part = (warp - 2) >> 2;                    // which HC columns of the tile
-    const int rr = quarter * 32 + lane;                  // resident row of this thread
-    const int row = r0 + rr;                              // query (MODE 0) or key (MODE 1)
+    const int part = (warp - 2) >> 2;                    // which HC columns of a tile
+    const int rr = quarter * 32 + lane;                  // resident key row of this thread
+    const int key = r0 + rr;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int c_base = part * HC;
     const float sl2 = p.scale_log2;
-    float lse2 = 0.f, dval = 0.f;
-    if constexpr (MODE == 0) {
-      const long long wi = ((long long)b * p.n_q + head) * p.Tp + row;
-      if (row < p.Tp) {
-        lse2 = p.lse2[wi];
-        dval = p.dvec[wi];
-      }
-    }
-    // every wait below is taken warp-uniformly: the TMEM loads and stores
-    // that follow are warp-collective
+    // every wait below is taken warp-uniformly: the TMEM loads that follow
+    // are warp-collective
     auto wait_all = [&](uint32_t bb, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bb, parity) ? 1 : 0) != 0;
     };
-    bool ok = true;
-    for (int u = 0; u < n_tiles && ok; ++u) {
-      const int x = u & 1;
-      if (!wait_all(bar(BB_SFULL + x), (uint32_t)((u >> 1) & 1))) { ok = false; break; }
-      tc_fence_after();
-      int hh, s0;
-      stream_of(u, hh, s0);
-      const int c_base = part * HC;                       // this warp's first column of the tile
-      const float* rv = reinterpret_cast<const float*>(smem + C::OFF_ROWV) + (u % C::NS) * 2 * BN;
-      if constexpr (MODE == 1) {
-        // the producer's lse / D values of this stage: acquire them on the
-        // stage's own barrier (its phase cannot move on before this tile's
-        // products have run, which wait for these warps)
-        if (!wait_all(bar(BB_FULL + u % C::NS), (uint32_t)((u / C::NS) & 1))) { ok = false; break; }
+    // dQ^T of a finished tile (query rows q0.. of head hh) into dq: lane =
+    // d row, so each reduction instruction covers one query's 32 consecutive
+    // d values
+    auto drain_dq = [&](int hh, int q0) {
+      if (quarter < C::DQ_QUARTERS) {
+        const int dcol = quarter * 32 + lane;
+        const long long rs = (long long)p.n_q * D;
+        float* base = p.dq + ((long long)b * p.T * p.n_q + hh) * D + dcol;
+#pragma unroll
+        for (int c0 = 0; c0 < HC; c0 += 8) {   // eight columns per TMEM load (few live registers)
+          uint32_t qv[8];
+          bkv_tmem_ld8(tmem + lane_base + C::DQ_COL + c_base + c0, qv);
+          tmem_wait_ld();
+          if (dcol < D) {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const int qi = q0 + c_base + c0 + c;
+              if (qi < p.T) atomicAdd(base + (long long)qi * rs, __uint_as_float(qv[c]) * p.scale);
+            }
+          }
+        }
       }
-      // every (row, column) pair of the tile admitted? (pairs past T are
+    };
+    bool ok = true;
+    int prev_hh = 0, prev_q0 = 0;
+    for (int u = 0; u < n_tiles && ok; ++u) {
+      if (!wait_all(bar(BK_SFULL), (uint32_t)(u & 1))) { ok = false; break; }
+      tc_fence_after();
+      int hh, q0;
+      stream_of(u, hh, q0);
+      uint32_t sv[HC], dv[HC];
+      bkv_tmem_ld<HC>(tmem + lane_base + C::S_COL + c_base, sv);
+      bkv_tmem_ld<HC>(tmem + lane_base + C::DP_COL + c_base, dv);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BK_SREAD));
+      // the stage's lse / D values: acquired on the stage's own barrier (its
+      // phase cannot move on before this tile's products, which wait for
+      // these warps)
+      if (!wait_all(bar(BK_FULL + u % C::NS), (uint32_t)((u / C::NS) & 1))) { ok = false; break; }
+      const float* rv = reinterpret_cast<const float*>(smem + C::OFF_ROWV) + (u % C::NS) * 2 * BN;
+      // every (key, query) pair of the tile admitted? (pairs past T are
       // harmless either way: their operand rows are zero or their output
       // rows are not stored)
-      bool all_in;
-      if constexpr (MODE == 0) {   // rows = queries r0.., columns = keys s0..
-        all_in = s0 + BN - 1 <= r0 && (p.window <= 0 || s0 > r0 + C::BM - 1 - p.window);
-      } else {                     // rows = keys r0.., columns = queries s0..
-        all_in = r0 + C::BM - 1 <= s0 && (p.window <= 0 || r0 > s0 + BN - 1 - p.window);
-      }
-      uint32_t sv[HC], dv[HC];
-      if constexpr (HC == 32) {
-        tmem_ld32(tmem + lane_base + C::S_COL + x * BN + c_base, *reinterpret_cast<uint32_t(*)[32]>(sv));
-        tmem_ld32(tmem + lane_base + C::DP_COL + x * BN + c_base, *reinterpret_cast<uint32_t(*)[32]>(dv));
-      } else {
-        tmem_ld16(tmem + lane_base + C::S_COL + x * BN + c_base, sv);
-        tmem_ld16(tmem + lane_base + C::DP_COL + x * BN + c_base, dv);
-      }
-      tmem_wait_ld();
+      const bool all_in = r0 + C::BM - 1 <= q0 && (p.window <= 0 || r0 > q0 + BN - 1 - p.window);
       uint32_t pk[HC / 2], dk[HC / 2];
       float4 lv4 = make_float4(0.f, 0.f, 0.f, 0.f), dv4 = lv4;
 #pragma unroll
       for (int c = 0; c < HC; c += 2) {
-        float l0, l1, d0, d1;
-        if constexpr (MODE == 0) {
-          l0 = l1 = lse2;
-          d0 = d1 = dval;
-        } else {
-          if ((c & 3) == 0) {   // the tile's per-column lse / D, four at a time
-            lv4 = *reinterpret_cast<const float4*>(rv + c_base + c);
-            dv4 = *reinterpret_cast<const float4*>(rv + BN + c_base + c);
-          }
-          l0 = (c & 3) ? lv4.z : lv4.x;
-          l1 = (c & 3) ? lv4.w : lv4.y;
-          d0 = (c & 3) ? dv4.z : dv4.x;
-          d1 = (c & 3) ? dv4.w : dv4.y;
+        if ((c & 3) == 0) {   // the tile's per-column lse / D, four at a time
+          lv4 = *reinterpret_cast<const float4*>(rv + c_base + c);
+          dv4 = *reinterpret_cast<const float4*>(rv + BN + c_base + c);
         }
+        const float l0 = (c & 3) ? lv4.z : lv4.x, l1 = (c & 3) ? lv4.w : lv4.y;
+        const float d0 = (c & 3) ? dv4.z : dv4.x, d1 = (c & 3) ? dv4.w : dv4.y;
         float p0, p1;
         fma2(p0, p1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl2, sl2, -l0, -l1);
         // one pair in four on the FMA pipe (the degree-3 exp2 of the
@@ -401,90 +391,70 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
           p1 = ex2(p1);
         }
         if (!all_in) {
-          const int col = s0 + c_base + c;
-          if (MODE == 0) {
-            if (!bwd_admitted(row, col, p.T, p.window)) p0 = 0.f;
-            if (!bwd_admitted(row, col + 1, p.T, p.window)) p1 = 0.f;
-          } else {
-            if (!bwd_admitted(col, row, p.T, p.window)) p0 = 0.f;
-            if (!bwd_admitted(col + 1, row, p.T, p.window)) p1 = 0.f;
-          }
+          const int qi = q0 + c_base + c;
+          if (!bwd_admitted(qi, key, p.T, p.window)) p0 = 0.f;
+          if (!bwd_admitted(qi + 1, key, p.T, p.window)) p1 = 0.f;
         }
         float t0 = __uint_as_float(dv[c]), t1 = __uint_as_float(dv[c + 1]);
         add2(t0, t1, -d0, -d1);
         mul2(t0, t1, p0, p1);
-        if constexpr (MODE == 1) pk[c / 2] = pack_bf16(p0, p1);
+        pk[c / 2] = pack_bf16(p0, p1);
         dk[c / 2] = pack_bf16(t0, t1);
       }
-      uint32_t ps_off;
-      if constexpr (C::SEP) {
-        // the single P / dS buffer: the previous tile's products must have
-        // read it. They signal its stage's EMPTY barrier; that barrier's
-        // earlier phase (NS tiles back) is complete here, since the S / dP
-        // this warp just read were committed after those products, and its
-        // next phase needs this tile's P / dS first.
-        if (u >= 1 && !wait_all(bar(BB_EMPTY + (u - 1) % C::NS), (uint32_t)(((u - 1) / C::NS) & 1))) {
-          ok = false;
-          break;
-        }
+      if (u >= 1) {
+        // the previous tile's products are done: its P^T, dS^T buffers are
+        // free and its dQ^T is final
+        if (!wait_all(bar(BK_PEMPTY), (uint32_t)((u - 1) & 1))) { ok = false; break; }
         tc_fence_after();
-        ps_off = (uint32_t)(part * (HC / 2));
-      } else {
-        // over the start of the S / dP columns this warp read (the other
-        // warps of the quarter read and write only their own columns)
-        ps_off = (uint32_t)(x * BN + c_base);
+        drain_dq(prev_hh, prev_q0);
       }
-      if constexpr (HC == 32) {
-        tmem_st16(tmem + lane_base + C::DS_COL + ps_off, dk);
-        if constexpr (MODE == 1) tmem_st16(tmem + lane_base + C::P_COL + ps_off, pk);
-      } else {
-        tmem_st8(tmem + lane_base + C::DS_COL + ps_off, dk);
-        if constexpr (MODE == 1) tmem_st8(tmem + lane_base + C::P_COL + ps_off, pk);
+      // P^T, dS^T rows (this thread's key row, columns c_base..) in 16-byte
+      // chunks of the swizzled layout the products read
+#pragma unroll
+      for (int j = 0; j < HC / 8; ++j) {
+        const uint32_t off = swz_off<C::CQ>(rr, c_base + 8 * j, C::QBLOCK);
+        *reinterpret_cast<uint4*>(smem + C::OFF_P + off) =
+            make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        *reinterpret_cast<uint4*>(smem + C::OFF_DS + off) =
+            make_uint4(dk[4 * j], dk[4 * j + 1], dk[4 * j + 2], dk[4 * j + 3]);
       }
-      tmem_wait_st();
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BB_PFULL));
+      if (lane == 0) mbar_arrive(bar(BK_PFULL));
+      prev_hh = hh;
+      prev_q0 = q0;
       if (*abort_flag) { ok = false; break; }
     }
-    // epilogue: the accumulators (zero when no tile was admitted) -> fp32
-    // rows. MODE 0: the NPART warps of a quarter take 32-column chunks of dQ
-    // in turn; MODE 1: half of them take dV, the other half dK, in turn.
-    // Every lane takes part in the TMEM loads; rows past T store nothing.
+    // the last tile's products (the accumulators are then final too)
     const bool have = n_tiles > 0;
     if (ok && have) {
-      if (!wait_all(bar(BB_ACCFULL), 0)) ok = false;
-      tc_fence_after();
-    }
-    if (ok) {
-      float* out;
-      long long rstride;   // elements between consecutive rows of the output
-      float mul;
-      int acc;
-      if constexpr (MODE == 0) {
-        out = p.dq + ((long long)b * p.T * p.n_q + head) * D;
-        rstride = (long long)p.n_q * D;
-        mul = p.scale;
-        acc = C::ACC0;
+      if (wait_all(bar(BK_PEMPTY), (uint32_t)((n_tiles - 1) & 1))) {
+        tc_fence_after();
+        drain_dq(prev_hh, prev_q0);
       } else {
-        const bool is_dv = part < C::NPART / 2;
-        out = (is_dv ? p.dv : p.dk) + ((long long)b * p.T * p.n_kv + head) * D;
-        rstride = (long long)p.n_kv * D;
-        mul = is_dv ? 1.0f : p.scale;
-        acc = is_dv ? C::ACC0 : C::ACC1;
+        ok = false;
       }
+    }
+    // epilogue: dV (the first two warps of each quarter) and dK (the other
+    // two) -> fp32 rows, 32-column chunks in turn. Every lane takes part in
+    // the TMEM loads; rows past T store nothing.
+    if (ok) {
+      const bool is_dv = part < 2;
+      float* out = (is_dv ? p.dv : p.dk) + ((long long)b * p.T * p.n_kv + g) * D;
+      const long long rstride = (long long)p.n_kv * D;
+      const float mul = is_dv ? 1.0f : p.scale;
+      const int acc = is_dv ? C::DV_COL : C::DK_COL;
       // Each 32 x 32 chunk (this warp's 32 rows) is transposed through shared
-      // memory so that every store instruction writes one row's 128 bytes:
-      // a thread-per-row store would scatter 16-byte pieces over 32 rows.
-      // The staging slots overlay the resident tiles and the ring, which
-      // every product has finished reading once ACCFULL has completed (with
-      // no tile there is no such wait: zeros are stored directly).
+      // memory so that every store instruction writes one row's 128 bytes.
+      // The staging slots overlay the tiles, which every product has
+      // finished reading once the last PEMPTY phase has completed (with no
+      // tile there is no such wait: zeros are stored directly).
       float* stg = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 33);
-      const int qrow0 = r0 + quarter * 32;   // first row of this warp's quarter
+      const int krow0 = r0 + quarter * 32;   // first key row of this warp's quarter
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
-        if (MODE == 0 && (c0 / 32) % C::NPART != part) continue;
-        if (MODE == 1 && (c0 / 32) % (C::NPART / 2) != part % (C::NPART / 2)) continue;
+        if ((c0 / 32) % 2 != part % 2) continue;
         if (have) {
           uint32_t a32[32];
           tmem_ld32(tmem + lane_base + acc + c0, a32);
@@ -494,11 +464,11 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
           __syncwarp();
 #pragma unroll 4
           for (int r = 0; r < 32; ++r)
-            if (qrow0 + r < p.T) out[(long long)(qrow0 + r) * rstride + c0 + lane] = stg[r * 33 + lane];
+            if (krow0 + r < p.T) out[(long long)(krow0 + r) * rstride + c0 + lane] = stg[r * 33 + lane];
           __syncwarp();
         } else {
           for (int r = 0; r < 32; ++r)
-            if (qrow0 + r < p.T) out[(long long)(qrow0 + r) * rstride + c0 + lane] = 0.f;
+            if (krow0 + r < p.T) out[(long long)(krow0 + r) * rstride + c0 + lane] = 0.f;
         }
       }
     }
@@ -512,28 +482,6 @@ __device__ __forceinline__ void bwd_tc_cta(const CUtensorMap* tmR0, const CUtens
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
-}
-
-// Both passes in one launch (they read the same inputs and write disjoint
-// outputs), so the tail of one fills with CTAs of the other. Blocks are
-// ordered by level k = 0, 1, ...: the n_kv B dK/dV CTAs of key tile k, then
-// the n_q B dQ CTAs of query tile tiles - 1 - k; under a causal mask both
-// shrink with k, so the heaviest CTAs start first.
-template <int D>
-__global__ void __launch_bounds__(BtcCfg<D, 0>::NUM_THREADS, 1)
-    bwd_tc_kernel(const __grid_constant__ CUtensorMap k1, const __grid_constant__ CUtensorMap v1,
-                  const __grid_constant__ CUtensorMap q1, const __grid_constant__ CUtensorMap o1,
-                  const __grid_constant__ CUtensorMap q0, const __grid_constant__ CUtensorMap o0,
-                  const __grid_constant__ CUtensorMap k0, const __grid_constant__ CUtensorMap v0,
-                  const BwdParams p) {
-  const int tiles = (p.T + 127) / 128;
-  const int nkv = p.n_kv * p.B, nq = p.n_q * p.B;
-  const int level = (int)blockIdx.x / (nkv + nq);
-  const int r = (int)blockIdx.x % (nkv + nq);
-  if (r < nkv)
-    bwd_tc_cta<D, 1>(&k1, &v1, &q1, &o1, p, level, r % p.n_kv, r / p.n_kv);
-  else
-    bwd_tc_cta<D, 0>(&q0, &o0, &k0, &v0, p, tiles - 1 - level, (r - nkv) % p.n_q, (r - nkv) / p.n_q);
 }
 
 }  // namespace sa

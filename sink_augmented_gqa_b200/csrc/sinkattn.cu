@@ -39,6 +39,9 @@ bool strides_ok(const int64_t s[3]) {
 }
 
 bool head_dim_ok(int d) { return d == 64 || d == 96 || d == 128; }
+// Backward workspace rows per (sequence, head): T rounded up to a multiple of
+// 384, so that every streamed query tile (64, 96 or 128 rows) lies inside.
+int bwd_rows_padded(int T) { return (T + 383) / 384 * 384; }
 
 // Ring capacity granule: a multiple of every key-tile height the kernels use
 // (128 decode rows; 128, 96, 64 prefill keys), so no tile wraps around.
@@ -762,7 +765,8 @@ sa_status launch_gemm(const void* a, int64_t lda, const void* w, int64_t ldw, co
   return launch_gemm_bn<256>(a, lda, w, ldw, bias, residual, ldr, y, ldy, M, N, K, rms, eps, stream);
 }
 
-// Backward pass (csrc/backward.cuh): row pass, key-tile pass, query-tile pass.
+// Backward pass (csrc/backward.cuh): the row pass, then one launch of the
+// products (csrc/backward_tc.cuh).
 template <int D>
 sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t stream) {
   sa::BwdParams p;
@@ -778,9 +782,9 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
   p.ds0 = a->d_out_strides[0]; p.ds1 = a->d_out_strides[1]; p.ds2 = a->d_out_strides[2];
   p.lse = a->lse;
   p.sinks = a->sinks;
-  // rows padded to a multiple of 64 (every streamed tile's BN <= 64 values lie
-  // inside its row; 16-byte aligned)
-  p.Tp = (a->T + 63) / 64 * 64;
+  // rows padded to a multiple of 384 (every streamed tile's 64, 96 or 128
+  // values lie inside its row; 16-byte aligned)
+  p.Tp = bwd_rows_padded(a->T);
   p.dvec = dvec;
   p.lse2 = dvec + (size_t)a->B * a->n_q * p.Tp;
   p.dq = a->dq;
@@ -798,30 +802,22 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
   if (p.dsinks && cudaMemsetAsync(p.dsinks, 0, sizeof(float) * a->n_q, stream) != cudaSuccess) return SA_ERR_CUDA;
   const long long rows = (long long)a->B * p.Tp * a->n_q;
   sa::bwd_rows_kernel<D><<<grid_for(rows * 32), 256, (size_t)a->n_q * sizeof(float), stream>>>(p);
-  using C0 = sa::BtcCfg<D, 0>;
-  using C1 = sa::BtcCfg<D, 1>;
-  // dQ pass: resident Q, dO (128 rows); streamed K, V (BN rows).
-  // dK/dV pass: resident K, V; streamed Q, dO.
-  CUtensorMap q0, o0, k0, v0, k1, v1, q1, o1;
-  if (!make_rows_map(&q0, a->q, D, a->T, a->n_q, a->B, a->q_strides, C0::CB, 128) ||
-      !make_rows_map(&o0, a->d_out, D, a->T, a->n_q, a->B, a->d_out_strides, C0::CB, 128) ||
-      !make_rows_map(&k0, a->k, D, a->T, a->n_kv, a->B, a->k_strides, C0::CB, C0::BN) ||
-      !make_rows_map(&v0, a->v, D, a->T, a->n_kv, a->B, a->v_strides, C0::CB, C0::BN) ||
-      !make_rows_map(&k1, a->k, D, a->T, a->n_kv, a->B, a->k_strides, C1::CB, 128) ||
-      !make_rows_map(&v1, a->v, D, a->T, a->n_kv, a->B, a->v_strides, C1::CB, 128) ||
-      !make_rows_map(&q1, a->q, D, a->T, a->n_q, a->B, a->q_strides, C1::CB, C1::BN) ||
-      !make_rows_map(&o1, a->d_out, D, a->T, a->n_q, a->B, a->d_out_strides, C1::CB, C1::BN))
+  using C = sa::BkvCfg<D>;
+  // resident K, V (128 rows); streamed Q, dO (BN rows)
+  CUtensorMap tk, tv, tq, to;
+  if (!make_rows_map(&tk, a->k, D, a->T, a->n_kv, a->B, a->k_strides, C::CB, C::BM) ||
+      !make_rows_map(&tv, a->v, D, a->T, a->n_kv, a->B, a->v_strides, C::CB, C::BM) ||
+      !make_rows_map(&tq, a->q, D, a->T, a->n_q, a->B, a->q_strides, C::CB, C::BN) ||
+      !make_rows_map(&to, a->d_out, D, a->T, a->n_q, a->B, a->d_out_strides, C::CB, C::BN))
     return SA_ERR_CUDA;
-  static_assert(C0::NUM_THREADS == C1::NUM_THREADS, "both passes share one launch");
-  constexpr uint32_t smem = C0::SMEM_BYTES > C1::SMEM_BYTES ? C0::SMEM_BYTES : C1::SMEM_BYTES;
   static std::atomic<uint64_t> smem_set{0};
   {
-    const sa_status sm = set_smem_once(sa::bwd_tc_kernel<D>, smem, smem_set);
+    const sa_status sm = set_smem_once(sa::bwd_tc_kernel<D>, C::SMEM_BYTES, smem_set);
     if (sm != SA_OK) return sm;
   }
-  // one CTA per 128-row tile, per head of either pass, per sequence (< 2^31: checked by the caller)
-  const unsigned ctas = (unsigned)((a->T + 127) / 128) * (unsigned)(a->n_kv + a->n_q) * (unsigned)a->B;
-  sa::bwd_tc_kernel<D><<<ctas, C0::NUM_THREADS, smem, stream>>>(k1, v1, q1, o1, q0, o0, k0, v0, p);
+  // one CTA per 128-key tile, per KV head, per sequence (< 2^31: checked by the caller)
+  const unsigned ctas = (unsigned)((a->T + 127) / 128) * (unsigned)a->n_kv * (unsigned)a->B;
+  sa::bwd_tc_kernel<D><<<ctas, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tk, tv, tq, to, p);
   return last_launch_status();
 }
 
@@ -1099,7 +1095,7 @@ sa_status sa_out_proj(const void* o, int64_t ldo, const void* w, int64_t ldw, co
 
 size_t sa_attn_backward_workspace_size(int32_t B, int32_t T, int32_t n_q) {
   if (B < 1 || T < 1 || n_q < 1) return 0;
-  const size_t Tp = ((size_t)T + 63) / 64 * 64;   // D and lse * log2(e), rows padded to 64 entries
+  const size_t Tp = (size_t)bwd_rows_padded(T);   // D and lse * log2(e), rows padded to 384 entries
   return (2 * (size_t)B * n_q * Tp * 4 + 255) / 256 * 256;
 }
 
@@ -1109,8 +1105,8 @@ sa_status sa_attn_backward(const sa_attn_bwd_args* a, void* workspace, size_t wo
   if (!head_dim_ok(a->d)) return SA_ERR_SHAPE;
   if (a->n_q % a->n_kv != 0) return SA_ERR_SHAPE;
   // the row pass sums n_q floats in shared memory; the products launch one CTA
-  // per 128-row tile, per head of either pass, per sequence (a 1-D grid)
-  const long long ctas = (long long)((a->T + 127) / 128) * (a->n_kv + a->n_q) * a->B;
+  // per 128-key tile, per KV head, per sequence (a 1-D grid)
+  const long long ctas = (long long)((a->T + 127) / 128) * a->n_kv * a->B;
   if (a->n_q > 8192 || ctas > 0x7fffffffLL) return SA_ERR_SHAPE;
   const void* ins[5] = {a->q, a->k, a->v, a->out, a->d_out};
   const int64_t* st[5] = {a->q_strides, a->k_strides, a->v_strides, a->out_strides, a->d_out_strides};
