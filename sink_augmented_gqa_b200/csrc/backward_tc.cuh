@@ -9,8 +9,9 @@
 //          to shared memory in the layouts the next products read
 //   dV  += P^T dO,  dK += dS^T Q          accumulated in TMEM over the CTA's tiles
 //   dQ^T = K^T dS^T                        per tile, into TMEM; the same warps
-//          add it to the fp32 dq rows in global memory (one 128-byte row
-//          segment per reduction instruction)
+//          stage it as [query][d] fp32 rows in the ring slot its tile's Q and
+//          dO have just left (the same byte count), and the TMA thread adds
+//          the rows to dq with a tensor reduce-add before refilling the slot
 //
 // Five products per (key, query) pair: S and dP are formed once for all
 // three gradients. BN, the query rows of a streamed tile, is what TMEM holds
@@ -23,7 +24,8 @@
 // 576 threads per CTA, one CTA per SM (each holds all 512 TMEM columns):
 //   warp 0      TMA: K and V once; per streamed tile its Q and dO tiles and
 //               the tile's lse log2 e and D values (bulk copies) into an
-//               NS-deep ring.
+//               NS-deep ring; each slot is refilled once the dQ^T rows staged
+//               in it have been read by their reduce-add.
 //   warp 1      one thread issues the MMAs and owns the TMEM allocation. It
 //               issues tile u's S^T, dP^T as soon as the warps have read tile
 //               u - 1's, then tile u - 1's dV, dK and dQ^T products once its
@@ -31,9 +33,13 @@
 //               next scores while the warps work on the current tile.
 //   warps 2-17  P^T, dS^T from S^T, dP^T (four warps per TMEM lane quarter,
 //               each a quarter of the tile's columns); then, once the previous
-//               tile's products are done, that tile's dQ^T into dq, and this
-//               tile's P^T, dS^T into shared memory; at the end dV, dK (fp32
-//               rows).
+//               tile's products are done, that tile's dQ^T into the staging
+//               rows (the warps of the lane quarters that hold d rows), and
+//               this tile's P^T, dS^T into shared memory; at the end dV, dK
+//               (fp32 rows).
+// Adding dq's partial sums is what bounds this kernel: each 128-key tile adds
+// a BN x d fp32 block per query tile, and the reduce-adds move about 8-9
+// bytes per SM cycle (the ring slot they read is refilled only afterwards).
 // dq must be zero before the launch (the row pass clears it). The order in
 // which the key tiles' contributions reach a dq element varies, so dq can
 // differ in the last bits between calls; dk and dv do not.
@@ -73,6 +79,8 @@ struct BkvCfg {
   static constexpr uint32_t OFF_DS = OFF_P + PS_BYTES;
   static constexpr uint32_t OFF_ROWV = OFF_DS + PS_BYTES;            // [NS][2][BN] fp32: lse log2 e, D
   static constexpr uint32_t OFF_BAR = OFF_ROWV + NS * 2 * BN * 4;
+  // a ring slot holds a tile's [Q | dO] bf16, then its dQ^T as [BN][D] fp32
+  static_assert(STAGE_BYTES == (uint32_t)BN * D * 4, "dQ staging fills one ring slot");
   static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
   // TMEM columns
   static constexpr int S_COL = 0;
@@ -93,18 +101,22 @@ struct BkvCfg {
   static constexpr int NSW = 16;                                     // P / dS warps (2..17)
   static constexpr int HC = BN / 4;                                  // columns per P / dS warp
   static constexpr int DQ_QUARTERS = (D + 31) / 32;                  // lane quarters with d rows of dQ^T
+  static constexpr int NDRAIN = 4 * DQ_QUARTERS;                     // warps that stage dQ^T
   static constexpr int NUM_THREADS = 32 * (2 + NSW);
   static_assert(HC % 8 == 0 && HC >= 16 && HC <= 32, "whole 16-byte chunks per P / dS warp");
   static_assert(SMEM_BYTES <= 227u * 1024, "shared memory");
-  // the epilogue's 32 x 33 fp32 staging slot per P / dS warp overlays the
-  // resident tiles, the ring and P / dS (below the row values)
-  static_assert((uint32_t)NSW * 32 * 33 * 4 <= OFF_ROWV, "epilogue staging overlays the tiles");
+  // the epilogue's 32 x 33 fp32 staging slot per P / dS warp overlays K, V
+  // and then P^T, dS^T (not the ring: the last tiles' reduce-adds may still
+  // be reading their dQ^T rows there)
+  static constexpr uint32_t EPI_SLOT = 32 * 33 * 4;
+  static constexpr int EPI_KV_SLOTS = (int)(2 * M_BYTES / EPI_SLOT);
+  static_assert((uint32_t)(NSW - EPI_KV_SLOTS) * EPI_SLOT <= 2 * PS_BYTES, "epilogue staging overlays K, V, P, dS");
 };
 
 enum : int {
   BK_RFULL = 0,      // K, V landed
-  BK_FULL = 1,       // [3] ring stage landed
-  BK_EMPTY = 4,      // [3] ring stage free (MMA commit)
+  BK_FULL = 1,       // [3] ring slot landed
+  BK_STG_FULL = 4,   // [3] count NDRAIN warps: the slot's dQ^T rows staged (its products are done)
   BK_SFULL = 7,      // S^T, dP^T of the current tile computed
   BK_SREAD = 8,      // count 16 warps: S^T, dP^T read into registers
   BK_PFULL = 9,      // count 16 warps: P^T, dS^T in shared memory (and the previous dQ^T read)
@@ -120,6 +132,16 @@ __device__ __forceinline__ void bkv_tmem_ld8(uint32_t taddr, uint32_t* r) {
                  "=r"(r[7])
                : "r"(taddr));
 }
+// TMA reduce-add shared -> global (elements past the tensor map's bounds are
+// dropped), tracked by this thread's bulk group.
+__device__ __forceinline__ void bkv_tma_reduce_add_4d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2,
+                                                      int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(src)
+      : "memory");
+}
 // N consecutive 32-bit TMEM columns of this warp's 32 lanes (N = 16, 24, 32)
 template <int N>
 __device__ __forceinline__ void bkv_tmem_ld(uint32_t taddr, uint32_t* r) {
@@ -133,7 +155,7 @@ template <int D>
 __global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BkvCfg<D>;
   constexpr int BN = C::BN;
   constexpr int HC = C::HC;
@@ -171,7 +193,7 @@ __global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
     mbar_init(bar(BK_RFULL), 1);
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar(BK_FULL + s), 1);
-      mbar_init(bar(BK_EMPTY + s), 1);
+      mbar_init(bar(BK_STG_FULL + s), C::NDRAIN);
     }
     mbar_init(bar(BK_SFULL), 1);
     mbar_init(bar(BK_SREAD), C::NSW);
@@ -203,13 +225,28 @@ __global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
         tma_load_4d(sbase + C::OFF_K + cb * C::MBLOCK, &tmK, bar(BK_RFULL), cb * C::CB, r0, g, b);
         tma_load_4d(sbase + C::OFF_V + cb * C::MBLOCK, &tmV, bar(BK_RFULL), cb * C::CB, r0, g, b);
       }
+      // tile v's dQ^T rows, staged in its slot once its products were done,
+      // added to dq
+      auto reduce_tile = [&](int v) -> bool {
+        const int sv = v % C::NS;
+        if (!mbar_wait(bar(BK_STG_FULL + sv), (uint32_t)((v / C::NS) & 1))) return false;
+        int hh, q0;
+        stream_of(v, hh, q0);
+        bkv_tma_reduce_add_4d(&tmDQ, sbase + C::OFF_ST + sv * C::STAGE_BYTES, 0, hh, q0, b);
+        bulk_commit();
+        return true;
+      };
       int issued = 0;
       bool ok = true;
       for (int u = 0; u < n_tiles; ++u) {
         const int s = u % C::NS;
-        if (u >= C::NS && !mbar_wait(bar(BK_EMPTY + s), (uint32_t)(((u / C::NS) - 1) & 1))) {
-          ok = false;
-          break;
+        if (u >= C::NS) {
+          // the slot's previous tile: reduce its dQ^T rows, wait until they are read
+          if (!reduce_tile(u - C::NS)) {
+            ok = false;
+            break;
+          }
+          bulk_wait_read_all();
         }
         if (*abort_flag) {
           ok = false;
@@ -232,6 +269,9 @@ __global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
         }
         issued = u + 1;
       }
+      for (int v = (n_tiles > C::NS ? n_tiles - C::NS : 0); ok && v < n_tiles; ++v) ok = reduce_tile(v);
+      // every reduce has read its rows and written dq before the CTA ends
+      bulk_wait_all();
       if (!ok) {
         *abort_flag = 1;
         for (int u = (issued > C::NS ? issued - C::NS : 0); u < issued; ++u)
@@ -269,7 +309,6 @@ __global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
           mma_ss(tmem + C::DQ_COL, a_kt + (((uint32_t)kk * 16 * C::SWZ) >> 4),
                  b_ds + (((uint32_t)kk * 16 * C::SWQ) >> 4), C::IDESC_Q, kk > 0 ? 1u : 0u);
         mma_commit(bar(BK_PEMPTY));
-        mma_commit(bar(BK_EMPTY + sv));
       };
       for (int u = 0; u < n_tiles && ok; ++u) {
         const int s = u % C::NS;
@@ -324,31 +363,28 @@ __global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
     auto wait_all = [&](uint32_t bb, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bb, parity) ? 1 : 0) != 0;
     };
-    // dQ^T of a finished tile (query rows q0.. of head hh) into dq: lane =
-    // d row, so each reduction instruction covers one query's 32 consecutive
-    // d values
-    auto drain_dq = [&](int hh, int q0) {
-      if (quarter < C::DQ_QUARTERS) {
-        const int dcol = quarter * 32 + lane;
-        const long long rs = (long long)p.n_q * D;
-        float* base = p.dq + ((long long)b * p.T * p.n_q + hh) * D + dcol;
+    // dQ^T of finished tile v -> [query][d] fp32 rows in its ring slot
+    // (lane = d row: each store covers 32 consecutive words), reduced into dq
+    // by the TMA thread
+    auto drain_dq = [&](int v) {
+      if (quarter >= C::DQ_QUARTERS) return;
+      float* stg = reinterpret_cast<float*>(smem + C::OFF_ST + (v % C::NS) * C::STAGE_BYTES);
+      const int dcol = quarter * 32 + lane;
 #pragma unroll
-        for (int c0 = 0; c0 < HC; c0 += 8) {   // eight columns per TMEM load (few live registers)
-          uint32_t qv[8];
-          bkv_tmem_ld8(tmem + lane_base + C::DQ_COL + c_base + c0, qv);
-          tmem_wait_ld();
-          if (dcol < D) {
+      for (int c0 = 0; c0 < HC; c0 += 8) {   // eight columns per TMEM load (few live registers)
+        uint32_t qv[8];
+        bkv_tmem_ld8(tmem + lane_base + C::DQ_COL + c_base + c0, qv);
+        tmem_wait_ld();
+        if (dcol < D) {
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              const int qi = q0 + c_base + c0 + c;
-              if (qi < p.T) atomicAdd(base + (long long)qi * rs, __uint_as_float(qv[c]) * p.scale);
-            }
-          }
+          for (int c = 0; c < 8; ++c) stg[(c_base + c0 + c) * D + dcol] = __uint_as_float(qv[c]) * p.scale;
         }
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BK_STG_FULL + v % C::NS));
     };
     bool ok = true;
-    int prev_hh = 0, prev_q0 = 0;
     for (int u = 0; u < n_tiles && ok; ++u) {
       if (!wait_all(bar(BK_SFULL), (uint32_t)(u & 1))) { ok = false; break; }
       tc_fence_after();
@@ -406,7 +442,7 @@ __global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
         // free and its dQ^T is final
         if (!wait_all(bar(BK_PEMPTY), (uint32_t)((u - 1) & 1))) { ok = false; break; }
         tc_fence_after();
-        drain_dq(prev_hh, prev_q0);
+        drain_dq(u - 1);
       }
       // P^T, dS^T rows (this thread's key row, columns c_base..) in 16-byte
       // chunks of the swizzled layout the products read
@@ -422,8 +458,6 @@ __global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BK_PFULL));
-      prev_hh = hh;
-      prev_q0 = q0;
       if (*abort_flag) { ok = false; break; }
     }
     // the last tile's products (the accumulators are then final too)
@@ -431,7 +465,7 @@ __global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
     if (ok && have) {
       if (wait_all(bar(BK_PEMPTY), (uint32_t)((n_tiles - 1) & 1))) {
         tc_fence_after();
-        drain_dq(prev_hh, prev_q0);
+        drain_dq(n_tiles - 1);
       } else {
         ok = false;
       }
@@ -447,10 +481,12 @@ __global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
       const int acc = is_dv ? C::DV_COL : C::DK_COL;
       // Each 32 x 32 chunk (this warp's 32 rows) is transposed through shared
       // memory so that every store instruction writes one row's 128 bytes.
-      // The staging slots overlay the tiles, which every product has
-      // finished reading once the last PEMPTY phase has completed (with no
-      // tile there is no such wait: zeros are stored directly).
-      float* stg = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 33);
+      // The staging slots overlay K, V and P^T, dS^T, which every product
+      // has finished reading once the last PEMPTY phase has completed (with
+      // no tile there is no such wait: zeros are stored directly).
+      const int es = warp - 2;
+      float* stg = reinterpret_cast<float*>(
+          smem + (es < C::EPI_KV_SLOTS ? C::OFF_K + es * C::EPI_SLOT : C::OFF_P + (es - C::EPI_KV_SLOTS) * C::EPI_SLOT));
       const int krow0 = r0 + quarter * 32;   // first key row of this warp's quarter
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {

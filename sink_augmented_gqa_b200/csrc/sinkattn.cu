@@ -178,6 +178,22 @@ bool make_rows_map(CUtensorMap* map, const void* base, int d, int T, int H, int 
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map over a dense fp32 [B][T][H][d] array (the backward's dq) whose box
+// is box_rows consecutive rows of one head ({d, 1, box_rows, 1} over dims
+// {d, H, T, B}): the TMA reduce-add target; rows past T are dropped.
+bool make_f32_rows_map(CUtensorMap* map, float* base, int d, int T, int H, int B, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr || T < 1) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)d * 4, (cuuint64_t)H * d * 4, (cuuint64_t)T * H * d * 4};
+  const cuuint32_t box[4] = {(cuuint32_t)d, 1, (cuuint32_t)box_rows, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // Tensor map over a strided [B][T][H][d] bf16 activation whose box is
 // box_heads consecutive heads of box_rows consecutive rows (d = 64: one
 // 128-byte swizzled row per (row, head)): dims {d, H, T, B}, box
@@ -804,11 +820,12 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
   sa::bwd_rows_kernel<D><<<grid_for(rows * 32), 256, (size_t)a->n_q * sizeof(float), stream>>>(p);
   using C = sa::BkvCfg<D>;
   // resident K, V (128 rows); streamed Q, dO (BN rows)
-  CUtensorMap tk, tv, tq, to;
+  CUtensorMap tk, tv, tq, to, tdq;
   if (!make_rows_map(&tk, a->k, D, a->T, a->n_kv, a->B, a->k_strides, C::CB, C::BM) ||
       !make_rows_map(&tv, a->v, D, a->T, a->n_kv, a->B, a->v_strides, C::CB, C::BM) ||
       !make_rows_map(&tq, a->q, D, a->T, a->n_q, a->B, a->q_strides, C::CB, C::BN) ||
-      !make_rows_map(&to, a->d_out, D, a->T, a->n_q, a->B, a->d_out_strides, C::CB, C::BN))
+      !make_rows_map(&to, a->d_out, D, a->T, a->n_q, a->B, a->d_out_strides, C::CB, C::BN) ||
+      !make_f32_rows_map(&tdq, a->dq, D, a->T, a->n_q, a->B, C::BN))
     return SA_ERR_CUDA;
   static std::atomic<uint64_t> smem_set{0};
   {
@@ -817,7 +834,7 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
   }
   // one CTA per 128-key tile, per KV head, per sequence (< 2^31: checked by the caller)
   const unsigned ctas = (unsigned)((a->T + 127) / 128) * (unsigned)a->n_kv * (unsigned)a->B;
-  sa::bwd_tc_kernel<D><<<ctas, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tk, tv, tq, to, p);
+  sa::bwd_tc_kernel<D><<<ctas, C::NUM_THREADS, C::SMEM_BYTES, stream>>>(tk, tv, tq, to, tdq, p);
   return last_launch_status();
 }
 
