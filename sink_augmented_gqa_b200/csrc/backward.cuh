@@ -41,11 +41,13 @@ struct BwdParams {
 };
 
 // D_i = <dO_i, o_i> and lse_i log2(e) per (b, i, h) into the padded
-// workspace rows, one warp per four rows, which also clears the row's dq
-// (the products add into it); each row also adds -exp(sink_h - lse_i) D_i
-// to dsinks[h], through a per-block sum in shared memory (dynamic, n_q
-// floats) so that global memory sees one atomic per block and head. Rows
-// T..Tp-1 get the values of an empty row (D 0, lse +inf).
+// workspace rows; the row's dq is cleared on the way (the products add into
+// it). Half a warp per row, 16-byte pieces (d / 8 lanes read o and dO, all 16
+// clear dq), four rows per half-warp and pass with every load issued before
+// any reduction. Each row also adds -exp(sink_h - lse_i) D_i to dsinks[h],
+// through a per-block sum in shared memory (dynamic, n_q floats) so that
+// global memory sees one atomic per block and head. Rows T..Tp-1 get the
+// values of an empty row (D 0, lse +inf).
 template <int D>
 __global__ void bwd_rows_kernel(const BwdParams p) {
   extern __shared__ float dsink_part[];
@@ -53,13 +55,14 @@ __global__ void bwd_rows_kernel(const BwdParams p) {
   if (sink)
     for (int h = threadIdx.x; h < p.n_q; h += blockDim.x) dsink_part[h] = 0.f;
   __syncthreads();
-  const int lane = threadIdx.x & 31;
+  constexpr int CH = D / 8;   // 16-byte pieces of a bf16 row (8, 12 or 16)
+  static_assert(CH <= 16, "a row fits half a warp");
+  const int sub = threadIdx.x & 15;
   const long long rows = (long long)p.B * p.Tp * p.n_q;
-  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-  // NR rows per warp and pass, their loads issued before any reduction (rows
-  // h, h + 1, ... of one (b, i) are adjacent in o and dO). Row r is (b, i, h)
-  // with h fastest; one division per pass (32-bit when the rows allow), the
-  // following rows by stepping h.
+  const long long groups = (long long)gridDim.x * (blockDim.x >> 4);
+  // Row r is (b, i, h) with h fastest (rows h, h + 1, ... of one (b, i) are
+  // adjacent in o and dO); one division per pass (32-bit when the rows
+  // allow), the following rows by stepping h.
   constexpr int NR = 4;
   auto split = [&](long long r, int& b, int& i, int& h) {
     if (rows <= 0xffffffffLL) {
@@ -83,38 +86,49 @@ __global__ void bwd_rows_kernel(const BwdParams p) {
       }
     }
   };
-  for (long long r0 = (blockIdx.x * (long long)(blockDim.x >> 5) + (threadIdx.x >> 5)) * NR; r0 < rows;
-       r0 += warps * NR) {
+  for (long long r0 = (blockIdx.x * (long long)(blockDim.x >> 4) + (threadIdx.x >> 4)) * NR; r0 < rows;
+       r0 += groups * NR) {
     int b0, i0, h0;
     split(r0, b0, i0, h0);
-    float acc[NR];
+    uint4 ov[NR], dv[NR];
     {
       int b = b0, i = i0, h = h0;
 #pragma unroll
       for (int j = 0; j < NR; ++j) {
-        acc[j] = 0.f;
+        ov[j] = dv[j] = make_uint4(0u, 0u, 0u, 0u);
         if (r0 + j < rows && i < p.T) {
-          const __nv_bfloat16* orow = p.o + b * p.os0 + i * p.os1 + h * p.os2;
-          const __nv_bfloat16* drow = p.dout + b * p.ds0 + i * p.ds1 + h * p.ds2;
+          if (sub < CH) {
+            ov[j] = *reinterpret_cast<const uint4*>(p.o + b * p.os0 + i * p.os1 + h * p.os2 + sub * 8);
+            dv[j] = *reinterpret_cast<const uint4*>(p.dout + b * p.ds0 + i * p.ds1 + h * p.ds2 + sub * 8);
+          }
+          float4* qrow = reinterpret_cast<float4*>(p.dq + (((long long)b * p.T + i) * p.n_q + h) * D);
 #pragma unroll
-          for (int c = lane; c < D; c += 32) acc[j] = fmaf(__bfloat162float(orow[c]), __bfloat162float(drow[c]), acc[j]);
-          float* qrow = p.dq + (((long long)b * p.T + i) * p.n_q + h) * D;
-#pragma unroll
-          for (int c = lane; c < D; c += 32) qrow[c] = 0.f;
+          for (int c = sub; c < D / 4; c += 16) qrow[c] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         step(b, i, h);
       }
     }
+    float acc[NR];
 #pragma unroll
-    for (int j = 0; j < NR; ++j)
+    for (int j = 0; j < NR; ++j) {
+      const uint32_t* o2 = reinterpret_cast<const uint32_t*>(&ov[j]);
+      const uint32_t* d2 = reinterpret_cast<const uint32_t*>(&dv[j]);
+      float a = 0.f;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
-    if (lane < NR && r0 + lane < rows) {
+      for (int e = 0; e < 4; ++e) {
+        a = fmaf(bf16_lo(o2[e]), bf16_lo(d2[e]), a);
+        a = fmaf(bf16_hi(o2[e]), bf16_hi(d2[e]), a);
+      }
+#pragma unroll
+      for (int off = 8; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
+      acc[j] = a;
+    }
+    if (sub < NR && r0 + sub < rows) {
       float a = acc[0];
       int b = b0, i = i0, h = h0;
 #pragma unroll
       for (int j = 1; j < NR; ++j) {
-        if (lane >= j) {
+        if (sub >= j) {
           a = acc[j];
           step(b, i, h);
         }

@@ -817,7 +817,7 @@ sa_status launch_backward(const sa_attn_bwd_args* a, float* dvec, cudaStream_t s
   p.scale_log2 = a->sm_scale * 1.4426950408889634f;
   if (p.dsinks && cudaMemsetAsync(p.dsinks, 0, sizeof(float) * a->n_q, stream) != cudaSuccess) return SA_ERR_CUDA;
   const long long rows = (long long)a->B * p.Tp * a->n_q;
-  sa::bwd_rows_kernel<D><<<grid_for(rows * 32), 256, (size_t)a->n_q * sizeof(float), stream>>>(p);
+  sa::bwd_rows_kernel<D><<<grid_for(rows * 4), 256, (size_t)a->n_q * sizeof(float), stream>>>(p);
   using C = sa::BkvCfg<D>;
   // resident K, V (128 rows); streamed Q, dO (BN rows)
   CUtensorMap tk, tv, tq, to, tdq;
