@@ -464,8 +464,8 @@ def lite_backward(dev, peaks, reps=10):
     """Backward pass of a Lite training layer (B = 8, T = 4096, 8/4 heads,
     d = 96), full causal and band, after the library's own forward. Work is
     counted as the algorithmic 5 products of the backward (S, dP, dV, dK,
-    dQ: 10 d flops per admitted pair and head); the kernels recompute S and
-    dP for dQ, which is not counted."""
+    dQ: 10 d flops per admitted pair and head), which is what the kernel
+    runs (plus, at d = 96, the padded rows of dQ^T's products)."""
     import sink_augmented_gqa_b200 as sa
     cfg = wl.CONFIGS["lite"]
     res = {}
