@@ -360,9 +360,10 @@ sa_status sa_attn_decode_static(sa_kv_cache* cache, const sa_attn_args* args, sa
  * workspace: device memory of sa_attn_backward_workspace_size() bytes
  *   (16-byte aligned, contents irrelevant).
  * Products run on the tensor cores (bf16 operands, fp32 accumulation); P and
- * dS enter their products as bf16. dq is summed over 128-key tiles by
- * reduce-adds whose order varies, so it can differ in the last bits between
- * calls; dk, dv and dsinks do not. Errors: SA_ERR_INVALID_ARG (null,
+ * dS enter their products as bf16. dq (summed over 128-key tiles by
+ * reduce-adds) and dsinks (summed over blocks by atomics) add in a varying
+ * order, so they can differ in the last bits between calls; dk and dv do
+ * not. Errors: SA_ERR_INVALID_ARG (null,
  * misaligned, bad stride, B/T/n_q < 1), SA_ERR_SHAPE (d not in {64, 96,
  * 128}, n_q % n_kv != 0, n_q > 8192, ceil(T / 128) n_kv B >= 2^31),
  * SA_ERR_WORKSPACE (too small), SA_ERR_CUDA.

@@ -139,6 +139,54 @@ def test_backward_full_size_one_group(cuda_device):
     assert torch.isfinite(ds).all()
 
 
+@pytest.mark.parametrize("shape", [(1, 2048, 16, 2, 64, 0), (1, 2048, 16, 2, 64, 128), (1, 1100, 8, 2, 128, 0),
+                                   (2, 1000, 8, 4, 96, 0)],
+                         ids=["d64_full", "d64_band", "d128_ragged", "d96_ragged"])
+def test_backward_long_sequences_one_group(cuda_device, shape):
+    # Longer sequences than the edge cases above, through each query-tile
+    # width of the kernel (128 rows at d = 64, 96 at d = 96, 64 at d = 128),
+    # with T not a multiple of it: every gradient of sequence 0 and KV group 0
+    # against the oracle (dsinks summed over the whole batch: finite).
+    B, T, n_q, n_kv, d, window = shape
+    cfg = wl.scaled(wl.CONFIGS["tiny"], B=B, n_q=n_q, n_kv=n_kv, d=d, sm_scale=1 / math.sqrt(d), seed=600 + T + d)
+    q, k, v = wl.qkv(cfg, T, device=DEV)
+    dout = wl.randn_bf16((B, T, n_q, d), cfg.seed, 125, DEV)
+    sinks = wl.sinks(cfg, device=DEV)
+    cache = sa.KVCache(B, T, n_kv, d, device=DEV)
+    out, lse = sa.attn_prefill(cache, q, k, v, sinks, window, cfg.sm_scale, rope_fused=False, return_lse=True)
+    dq, dk, dv, ds = sa.attn_backward(q, k, v, out, dout, lse, sinks, window, cfg.sm_scale)
+    torch.cuda.synchronize()
+    qm = n_q // n_kv
+    sl = (slice(0, 1), slice(None), slice(0, qm))
+    args = (to64(q[sl]), to64(k[0:1, :, 0:1]), to64(v[0:1, :, 0:1]), to64(sinks[:qm]), window, cfg.sm_scale,
+            to64(dout[sl]))
+    rq, rk, rv, _ = obwd.attention_backward(*args)
+    mq, mk, mv, _ = _magnitudes(*args)
+    _check("dq", dq[sl], rq, mq)
+    _check("dk", dk[0:1, :, 0:1], rk, mk)
+    _check("dv", dv[0:1, :, 0:1], rv, mv)
+    assert torch.isfinite(ds).all()
+
+
+def test_backward_repeat_calls_agree(cuda_device):
+    # dq is summed over key tiles by reduce-adds and dsinks over blocks by
+    # atomics, both in a varying order: two calls agree to rounding there,
+    # and bit for bit on dk and dv.
+    B, T, n_q, n_kv, d = 2, 777, 8, 2, 96
+    cfg = wl.scaled(wl.CONFIGS["tiny"], B=B, n_q=n_q, n_kv=n_kv, d=d, sm_scale=1 / math.sqrt(d), seed=700)
+    q, k, v = wl.qkv(cfg, T, device=DEV)
+    dout = wl.randn_bf16((B, T, n_q, d), cfg.seed, 126, DEV)
+    sinks = wl.sinks(cfg, device=DEV)
+    cache = sa.KVCache(B, T, n_kv, d, device=DEV)
+    out, lse = sa.attn_prefill(cache, q, k, v, sinks, 0, cfg.sm_scale, rope_fused=False, return_lse=True)
+    a = sa.attn_backward(q, k, v, out, dout, lse, sinks, 0, cfg.sm_scale)
+    b = sa.attn_backward(q, k, v, out, dout, lse, sinks, 0, cfg.sm_scale)
+    torch.cuda.synchronize()
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
+    for x, y in (a[0], b[0]), (a[3], b[3]):
+        assert (x - y).abs().amax().item() <= 1e-5 * x.abs().amax().item()
+
+
 def test_backward_argument_errors(cuda_device):
     x = torch.zeros((1, 8, 4, 64), dtype=torch.bfloat16, device=DEV)
     lse = torch.zeros((1, 4, 8), dtype=torch.float32, device=DEV)
