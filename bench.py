@@ -651,7 +651,7 @@ def long_decode(dev, peaks, steps=8, layers=24, ring=False, fp8=False):
                              + (", e4m3 codes + fp32 row scales [B][n_kv][cap]" if fp8 else ", bf16"))}
 
 
-def e2e_handoff(step, steps, warmup, groups=4):
+def e2e_handoff(step, steps, warmup, groups=8):
     """The same step through host buffers, through the library's public API:
     every step copies its inputs from pinned host memory and its outputs back
     to pinned host memory.
@@ -660,8 +660,10 @@ def e2e_handoff(step, steps, warmup, groups=4):
       go up on a copy stream, the group's two prefill calls run on caches that
       view the group's rows of each layer's cache, and its outputs come back
       on a second copy stream, so the copies of one group overlap the
-      attention of another. The phase ends when the last output has landed
-      on the host.
+      attention of another. Groups alternate between two compute streams, so
+      one group's attention launch fills the last, partly idle wave of the
+      previous one. The phase ends when the last output has landed on the
+      host.
     * Decode phase: each layer's whole-batch cache is brought to the chunk's
       end (its prefix snapshot restored, the chunk rows the group calls wrote
       appended in place); then per decode step one copy brings the new rows'
@@ -717,6 +719,7 @@ def e2e_handoff(step, steps, warmup, groups=4):
     h2d = sum(t.numel() * t.element_size() for hs in host_in for t in hs) + dec_host.numel() * 2
     d2h = sum(t.numel() * 2 for t in host_out) + dec_out_host.numel() * 2
     comp = torch.cuda.current_stream()
+    comps = (comp, torch.cuda.Stream())
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     landed = [torch.cuda.Event() for _ in range(groups)]
     computed = [torch.cuda.Event() for _ in range(groups)]
@@ -734,16 +737,19 @@ def e2e_handoff(step, steps, warmup, groups=4):
                         dst[g0:g1].copy_(hsrc[g0:g1], non_blocking=True)
                 landed[gi].record(s_in)
         step.tables()
+        comps[1].wait_stream(comp)     # the tables, and the previous step's decode
         for gi, (g0, g1) in enumerate(spans):
-            comp.wait_event(landed[gi])
-            comp.wait_event(read[gi])   # the previous step's outputs of this group have been read
-            for li, L in enumerate(step.layers):
-                c = sub[li][gi]
-                c.restore(sub_snap[li][gi])
-                q, k, v = (t[g0:g1] for t in dev_in[li])
-                sa.attn_prefill(c, q, k, v, L["sinks"], L["window"], cfg.sm_scale, step.cos, step.sin,
-                                out=dev_out[li][g0:g1])
-            computed[gi].record(comp)
+            cs = comps[gi % 2]
+            cs.wait_event(landed[gi])
+            cs.wait_event(read[gi])   # the previous step's outputs of this group have been read
+            with torch.cuda.stream(cs):
+                for li, L in enumerate(step.layers):
+                    c = sub[li][gi]
+                    c.restore(sub_snap[li][gi])
+                    q, k, v = (t[g0:g1] for t in dev_in[li])
+                    sa.attn_prefill(c, q, k, v, L["sinks"], L["window"], cfg.sm_scale, step.cos, step.sin,
+                                    out=dev_out[li][g0:g1])
+            computed[gi].record(cs)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(computed[gi])
                 for li in range(nl):
