@@ -418,9 +418,11 @@ __global__ void __launch_bounds__(BkvCfg<D>::NUM_THREADS, 1)
         const float d0 = (c & 3) ? dv4.z : dv4.x, d1 = (c & 3) ? dv4.w : dv4.y;
         float p0, p1;
         fma2(p0, p1, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]), sl2, sl2, -l0, -l1);
-        // one pair in four on the FMA pipe (the degree-3 exp2 of the
-        // forward), the rest on the MUFU unit
-        if (((c / 2) & 3) == 0) {
+        // every other pair on the FMA pipe (the degree-3 exp2 of the
+        // forward, relative error < 1.5e-4), the rest on the MUFU unit
+        // (measured: all on MUFU 0.974 ms, one in four on the FMA pipe 0.965,
+        // one in two 0.953 on the Lite full-causal layer)
+        if (((c / 2) & 1) == 0) {
           exp2_fma2(p0, p1);
         } else {
           p0 = ex2(p0);
