@@ -62,3 +62,37 @@ def test_zero_wait_limit_reports_timeout_and_context_survives(cuda_device, windo
     ref, _ = oracle_step(ocache, q, k, v, sinks.cpu(), 16, cfg.sm_scale, rc, rs)
     check_bf16_output(out, ref, "after timeout")
     assert sa.device_status() == "SA_OK"
+
+
+def test_zero_wait_limit_backward_reports_timeout_and_context_survives(cuda_device):
+    # The backward's producer, MMA issuer and P / dS warps give up on their
+    # bounded waits, drain what they started (loads, products, reduce-adds)
+    # and return; afterwards the same context computes the same gradients as
+    # before (dk, dv bit for bit; dq, summed by reduce-adds in a varying
+    # order, to rounding).
+    import math
+    cfg = wl.scaled(wl.CONFIGS["tiny"], B=2, n_q=8, n_kv=2, d=96, sm_scale=1 / math.sqrt(96), seed=900)
+    T = 300
+    q, k, v = wl.qkv(cfg, T, device=DEV)
+    dout = wl.randn_bf16((cfg.B, T, cfg.n_q, cfg.d), cfg.seed, 127, DEV)
+    sinks = wl.sinks(cfg, device=DEV)
+    cache = sa.KVCache(cfg.B, T, cfg.n_kv, cfg.d, device=DEV)
+    out, lse = sa.attn_prefill(cache, q, k, v, sinks, 0, cfg.sm_scale, rope_fused=False, return_lse=True)
+    before = sa.attn_backward(q, k, v, out, dout, lse, sinks, 0, cfg.sm_scale)
+    torch.cuda.synchronize()
+    assert sa.device_status() == "SA_OK"
+    sa.set_wait_limit(0)
+    try:
+        sa.attn_backward(q, k, v, out, dout, lse, sinks, 0, cfg.sm_scale)
+        torch.cuda.synchronize()
+        status = sa.device_status()
+    finally:
+        sa.set_wait_limit(DEFAULT_LIMIT)
+    assert status == "SA_ERR_TIMEOUT"
+    assert sa.device_status() == "SA_OK"
+    after = sa.attn_backward(q, k, v, out, dout, lse, sinks, 0, cfg.sm_scale)
+    torch.cuda.synchronize()
+    assert sa.device_status() == "SA_OK"
+    assert torch.equal(before[1], after[1]) and torch.equal(before[2], after[2])
+    for x, y in (before[0], after[0]), (before[3], after[3]):
+        assert (x - y).abs().amax().item() <= 1e-5 * x.abs().amax().item()
