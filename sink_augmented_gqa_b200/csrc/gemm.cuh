@@ -75,10 +75,10 @@ struct GemmCfg {
 
 enum : int {
   GB_FULL = 0,        // [NS] producer -> MMA, RMS warps: A and W tiles landed
-  GB_EMPTY = 4,       // [NS] MMA (commit) + RMS warps -> producer
+  GB_EMPTY = 4,       // [NS] MMA (commit) + the 64 RMS lanes -> producer
   GB_ACC_FULL = 8,    // MMA -> epilogue: the tile's accumulator is complete
   GB_ACC_EMPTY = 10,  // count 8: epilogue warps -> MMA: accumulator read
-  GB_RMS_FULL = 12,   // count 2: RMS warps -> epilogue: row scales of the tile
+  GB_RMS_FULL = 12,   // count 64: RMS lanes -> epilogue: row scales of the tile
   GB_RMS_EMPTY = 14,  // count 8: epilogue warps -> RMS warps
   GB_DRAIN = 16,      // MMA issuer, on abort
   GB_TMEM_SLOT = 17,
@@ -110,11 +110,11 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
       mbar_init(bar(GB_FULL + s), 1);
-      mbar_init(bar(GB_EMPTY + s), p.rms ? 3 : 1);   // MMA commit (+ one arrival per RMS warp)
+      mbar_init(bar(GB_EMPTY + s), p.rms ? 65 : 1);   // MMA commit (+ one arrival per RMS lane)
     }
     mbar_init(bar(GB_ACC_FULL), 1);
     mbar_init(bar(GB_ACC_EMPTY), C::EPI_WARPS);
-    mbar_init(bar(GB_RMS_FULL), 2);
+    mbar_init(bar(GB_RMS_FULL), 64);
     mbar_init(bar(GB_RMS_EMPTY), C::EPI_WARPS);
     mbar_init(bar(GB_DRAIN), 1);
     *abort_flag = 0;
@@ -204,6 +204,9 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp < 4) {
     // ------------------------------------------------------------ RMSNorm row scales
+    // Every lane waits and arrives on its own (the barriers count 64 RMS
+    // arrivals): there is no warp-collective step, so a wait that runs out in
+    // one lane cannot leave the others waiting for it.
     if (p.rms) {
       const int rb0 = 32 * (warp - 2) + lane;   // rows rb0 + 64 i of the A tile, i < 4
       const float inv_k = 1.0f / (float)p.K;
@@ -229,16 +232,14 @@ __global__ void __launch_bounds__(384, 1)
               }
             }
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bar(GB_EMPTY + s));
+          mbar_arrive(bar(GB_EMPTY + s));
         }
         if (!ok) break;
         if (tl >= 1 && !mbar_wait(bar(GB_RMS_EMPTY), (uint32_t)((tl - 1) & 1))) { ok = false; break; }
         float* rb = reinterpret_cast<float*>(smem + C::OFF_RMS);
 #pragma unroll
         for (int i = 0; i < 4; ++i) rb[rb0 + 64 * i] = 1.0f / sqrtf(ss[i] * inv_k + p.eps);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(GB_RMS_FULL));
+        mbar_arrive(bar(GB_RMS_FULL));
         if (*abort_flag) { ok = false; break; }
       }
       if (!ok) *abort_flag = 1;
@@ -249,16 +250,21 @@ __global__ void __launch_bounds__(384, 1)
     const int hh = (warp - 4) >> 2;          // accumulator half: rows 128 hh ..
     const int r = 128 * hh + 32 * q + lane;  // row within the tile
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    // warp-uniform waits: the TMEM loads and __syncwarp that follow are
+    // warp-collective
+    auto wait_all = [&](uint32_t bb, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bb, parity) ? 1 : 0) != 0;
+    };
     int tl = 0, cnt = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
       int m0, n0;
       tile_origin(t, m0, n0);
-      if (!mbar_wait(bar(GB_ACC_FULL), (uint32_t)(tl & 1))) { ok = false; break; }
+      if (!wait_all(bar(GB_ACC_FULL), (uint32_t)(tl & 1))) { ok = false; break; }
       tc_fence_after();
       float sc = 1.f;
       if (p.rms) {
-        if (!mbar_wait(bar(GB_RMS_FULL), (uint32_t)(tl & 1))) { ok = false; break; }
+        if (!wait_all(bar(GB_RMS_FULL), (uint32_t)(tl & 1))) { ok = false; break; }
         sc = reinterpret_cast<const float*>(smem + C::OFF_RMS)[r];
         __syncwarp();
         if (lane == 0) mbar_arrive(bar(GB_RMS_EMPTY));

@@ -96,3 +96,41 @@ def test_zero_wait_limit_backward_reports_timeout_and_context_survives(cuda_devi
     assert torch.equal(before[1], after[1]) and torch.equal(before[2], after[2])
     for x, y in (before[0], after[0]), (before[3], after[3]):
         assert (x - y).abs().amax().item() <= 1e-5 * x.abs().amax().item()
+
+
+def test_zero_wait_limit_projections_report_timeout_and_context_survives(cuda_device):
+    # The projection GEMM (producer, MMA issuer, RMSNorm warps, epilogue) gives
+    # up on its bounded waits and returns; afterwards the same context
+    # computes bit-identical projections to the ones before the timeout.
+    g = torch.Generator().manual_seed(11)
+    M, N, K = 600, 1280, 1024
+    x = (torch.randn((M, K), generator=g) * 1.0).to(torch.bfloat16).to(DEV)
+    w = (torch.randn((N, K), generator=g) / 32).to(torch.bfloat16).to(DEV)
+    gamma = (torch.rand(K, generator=g) + 0.5).to(DEV)
+    b = (torch.randn((N,), generator=g) * 0.1).to(torch.bfloat16).to(DEV)
+    wf = sa.rmsnorm_fold_weight(w, gamma)
+    o = (torch.randn((M, K), generator=g)).to(torch.bfloat16).to(DEV)
+    w2 = (torch.randn((N, K), generator=g) / 32).to(torch.bfloat16).to(DEV)
+    res = (torch.randn((M, N), generator=g)).to(torch.bfloat16).to(DEV)
+
+    def run():
+        y = sa.qkv_proj(x, wf, b, 1e-5)
+        xr = res.clone()
+        sa.out_proj(o, w2, b, xr)
+        return y, xr
+    y0, r0 = run()
+    torch.cuda.synchronize()
+    assert sa.device_status() == "SA_OK"
+    sa.set_wait_limit(0)
+    try:
+        run()
+        torch.cuda.synchronize()
+        status = sa.device_status()
+    finally:
+        sa.set_wait_limit(DEFAULT_LIMIT)
+    assert status == "SA_ERR_TIMEOUT"
+    assert sa.device_status() == "SA_OK"
+    y1, r1 = run()
+    torch.cuda.synchronize()
+    assert sa.device_status() == "SA_OK"
+    assert torch.equal(y0, y1) and torch.equal(r0, r1)
