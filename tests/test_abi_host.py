@@ -236,3 +236,13 @@ def test_prefill_schedule_slots_wrap(L):
     assert all(graph[i] == graph[i % 64] for i in range(200))
     assert not set(eager) & set(graph)
     assert L.sa_prefill_sched_slot(2 ** 64 - 1, 0) == (2 ** 64 - 1) % 64
+
+
+def test_backward_workspace_rows_pad_to_whole_query_tiles(L):
+    # D and lse * log2(e) rows per (sequence, query head), padded to a
+    # multiple of 384 entries (whole query tiles of 64, 96 and 128 rows),
+    # fp32, the total rounded up to 256 bytes
+    for B, T, n_q in [(1, 1, 1), (1, 383, 4), (1, 384, 4), (1, 385, 4), (3, 4096, 8), (2, 8192, 64)]:
+        Tp = (T + 383) // 384 * 384
+        want = (2 * B * n_q * Tp * 4 + 255) // 256 * 256
+        assert L.sa_attn_backward_workspace_size(B, T, n_q) == want, (B, T, n_q)
